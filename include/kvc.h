@@ -1,0 +1,218 @@
+/*
+ * kvc.h — C ABI of the B200 KV-cache codec library (libkvc.so).
+ *
+ * The codec compresses an exported LLM KV cache laid out [L][2][H][T][D]
+ * (layer, K = 0 / V = 1, KV head, token, channel; one [T][D] block is a
+ * "slice", slice index (l * 2 + kv) * H + h), as in the Codec-Gauge page,
+ * "Problem Statement and Overview" (K_l, V_l in R^{B x H_l x T x d_l}, B = 1).
+ *
+ * Two front-ends feed one entropy back-end and one container:
+ *   lossless   — channel-major reorder of each chunk of floor(values_per_chunk
+ *                / D) tokens, byte-plane split, and per plane the smallest of a
+ *                constant, an rANS-coded or a raw record (AT-1 Memory page,
+ *                "KV & tensor mode"; QATQ page, "qatq encode" and "How it works").
+ *   transform  — sink and recent tokens kept raw, the middle RoPE-undone on
+ *                keys, projected on a given per-(layer, K/V, head) orthonormal
+ *                basis, and quantised per component at an allocated bit width
+ *                with a scale and zero point per 64-token block (KVTC page, "How
+ *                the Pipeline Works", "Why RoPE Has to Be Reversed First", "Bit
+ *                Budget Is Not Fair"; Codec-Gauge page, "Compression Conditions").
+ *   back-end   — chunked, 128-lane interleaved rANS with per-stream frequency
+ *                tables (KVTC page, "rANS Makes the Last Mile Smaller").
+ *   container  — 64-byte header, chunk-offset index with a CRC-32 per record,
+ *                and a header CRC-32 over header and index; corrupt or truncated
+ *                input is refused (QATQ page, "QATC v2 checksum validated").
+ *
+ * Conventions
+ *   - Device pointers (d_*) are CUDA device memory owned by the caller, 16-byte
+ *     aligned; host pointers (h_*) are ordinary host memory owned by the caller.
+ *     The plan owns its own device copies of bases, widths and tables.
+ *   - Calls that take a cudaStream_t are asynchronous on that stream; they
+ *     launch kernels only (no allocation, no host synchronisation).
+ *   - Two error channels: the return value reports what the host can see
+ *     (bad arguments, too small buffers, launch failures); data-dependent
+ *     results (bytes written, corrupt/truncated input, plan mismatch) are
+ *     written by the device into *d_res once the stream reaches that point.
+ *   - On a decode error the output contents are unspecified; read d_res first.
+ *   - A plan is bound to the CUDA device that was current when it was made.
+ */
+#ifndef KVC_H
+#define KVC_H
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KVC_ABI_VERSION 1u
+
+/* status codes (return values and kvc_result.status) */
+enum {
+  KVC_OK = 0,
+  KVC_ERR_INVALID = 1,       /* bad argument or plan description */
+  KVC_ERR_CAPACITY = 2,      /* destination or workspace too small */
+  KVC_ERR_CORRUPT = 3,       /* checksum, structure or rANS end-state failure */
+  KVC_ERR_TRUNCATED = 4,     /* container shorter than its header says */
+  KVC_ERR_PLAN_MISMATCH = 5, /* container made with another shape or plan */
+  KVC_ERR_TIMEOUT = 6,       /* a bounded device wait gave up */
+  KVC_ERR_CUDA = 7,          /* CUDA runtime error on the host side */
+  KVC_ERR_UNSUPPORTED = 8    /* valid request this build does not handle */
+};
+
+enum { KVC_DTYPE_BF16 = 1, KVC_DTYPE_FP16 = 2 };
+enum { KVC_PATH_LOSSLESS = 0, KVC_PATH_TRANSFORM = 1 };
+
+/* Written by the device at the end of an encode or decode: status, and the
+ * container bytes (encode) or decoded bytes (decode); 16 bytes. */
+typedef struct {
+  int32_t status;
+  uint32_t reserved;
+  uint64_t bytes;
+} kvc_result;
+
+typedef struct kvc_plan_s kvc_plan_t;
+
+/* Plan description (host memory; copied by kvc_plan_create).
+ *   abi_version       KVC_ABI_VERSION
+ *   dtype             KVC_DTYPE_BF16 or KVC_DTYPE_FP16 (transform: bf16 only)
+ *   n_layers, n_heads, n_tokens, head_dim   cache shape L, H, T, D
+ *   values_per_chunk  lossless chunk bound (65536): chunks hold
+ *                     floor(values_per_chunk / D) tokens, at most 65536 values
+ *   n_sink, n_recent  transform: leading / trailing tokens kept raw
+ *   block_tokens      transform: tokens per scale/zero-point block (64)
+ *   chunk_tokens      transform: middle tokens per record (multiple of
+ *                     block_tokens, at most 512)
+ *   max_bits          transform: bit-width cap per component (<= 8)
+ *   rope_theta        transform: rotary base; pairs (i, i + D/2), angle
+ *                     t * theta^(-2i/D)
+ *   avg_bits          transform: average code bits per middle value; the budget
+ *                     floor(avg_bits * U + 0.5) over U = L*2*H*D components is
+ *                     spent greedily, one bit at a time, on the component with
+ *                     the largest eigenvalue * 4^-bits (ties: lowest index)
+ *   bases             transform: host [L*2*H][D][D] fp32, element [k*D + j] is
+ *                     channel k of component j; columns orthonormal
+ *   eigvals           transform: host [L*2*H][D] component variances (used when
+ *                     widths is NULL; negative values count as 0)
+ *   widths            transform: optional host [L*2*H][D] bit widths that
+ *                     replace the greedy allocation
+ * For a lossless-only plan set bases, eigvals and widths to NULL. */
+typedef struct {
+  uint32_t abi_version;
+  uint32_t dtype;
+  uint32_t n_layers, n_heads, n_tokens, head_dim;
+  uint32_t values_per_chunk;
+  uint32_t n_sink, n_recent, block_tokens, chunk_tokens, max_bits;
+  double rope_theta;
+  double avg_bits;
+  const float* bases;
+  const double* eigvals;
+  const uint8_t* widths;
+} kvc_plan_desc;
+
+/* Validate the description, allocate bit widths, build the fp32 cos/sin table
+ * (fp64-computed) and upload the plan to the current device. Checks each basis
+ * for orthonormality (max |Q^T Q - I| <= 1e-3). Returns KVC_OK and *out, or an
+ * error (nothing allocated). Blocking; call outside stream capture. */
+int kvc_plan_create(const kvc_plan_desc* desc, kvc_plan_t** out);
+/* Free the plan (device memory included). NULL is ignored. */
+void kvc_plan_destroy(kvc_plan_t* plan);
+/* Copy the plan's bit widths ([L*2*H][D]) to h_out (n bytes). */
+int kvc_plan_widths(const kvc_plan_t* plan, uint8_t* h_out, size_t n);
+/* CRC-32 identifying the transform plan; 0 for a lossless-only plan. */
+uint32_t kvc_plan_crc(const kvc_plan_t* plan);
+
+/* Upper bound of the container size for n_slices slices of the given path
+ * (exact for incompressible input: the codec never exceeds it). 0 on error. */
+size_t kvc_max_encoded_bytes(const kvc_plan_t* plan, int path, uint32_t n_slices);
+/* Device workspace an encode or decode of n_slices slices needs. */
+size_t kvc_workspace_bytes(const kvc_plan_t* plan, int path, int decode, uint32_t n_slices);
+
+/* Encode slices [first_slice, first_slice + n_slices) of the cache.
+ *   d_src     device [n_slices][T][D] 16-bit values (the selected slices only)
+ *   d_dst     device output, dst_cap bytes (>= kvc_max_encoded_bytes)
+ *   d_ws      device workspace, ws_bytes (>= kvc_workspace_bytes(..., 0, n_slices))
+ *   d_res     device kvc_result: status and container bytes
+ * Returns KVC_OK when launched; KVC_ERR_INVALID / KVC_ERR_CAPACITY / KVC_ERR_CUDA
+ * otherwise (then nothing was launched or the stream is in error). */
+int kvc_encode_lossless(const kvc_plan_t* plan, uint32_t first_slice, uint32_t n_slices,
+                        const void* d_src, void* d_dst, size_t dst_cap, void* d_ws,
+                        size_t ws_bytes, kvc_result* d_res, cudaStream_t stream);
+
+/* Decode a lossless container.
+ *   d_src/src_bytes  device container and its exact length in bytes
+ *   d_dst/dst_cap    device output [n_slices][T][D] 16-bit values
+ *   d_ws/ws_bytes    device workspace (>= kvc_workspace_bytes(..., 1, 0))
+ *   d_res            device kvc_result: status (OK, CORRUPT, TRUNCATED,
+ *                    PLAN_MISMATCH, CAPACITY) and decoded bytes
+ * The header, the index and every record's CRC-32 are checked; a record that
+ * fails leaves its output unspecified and sets the status of the lowest
+ * failing record. */
+int kvc_decode_lossless(const kvc_plan_t* plan, const void* d_src, size_t src_bytes, void* d_dst,
+                        size_t dst_cap, void* d_ws, size_t ws_bytes, kvc_result* d_res,
+                        cudaStream_t stream);
+
+/* Transform coding of slices [first_slice, first_slice + n_slices); arguments
+ * as kvc_encode_lossless. Needs a plan with bases; D = 128, bf16. */
+int kvc_encode_transform(const kvc_plan_t* plan, uint32_t first_slice, uint32_t n_slices,
+                         const void* d_src, void* d_dst, size_t dst_cap, void* d_ws,
+                         size_t ws_bytes, kvc_result* d_res, cudaStream_t stream);
+/* Decode a transform container; arguments as kvc_decode_lossless. */
+int kvc_decode_transform(const kvc_plan_t* plan, const void* d_src, size_t src_bytes, void* d_dst,
+                         size_t dst_cap, void* d_ws, size_t ws_bytes, kvc_result* d_res,
+                         cudaStream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* kvc_status_string(int status);
+
+/* Calibration (host, multithreaded): the uncentered second-moment eigenbasis of
+ * each slice (Codec-Gauge page, "Compression Conditions": PCA/KLT at layer,
+ * K/V and head granularity; KVTC page, "The Tradeoff Is Real": calibration).
+ *   h_calib   host [L*2*H][n_calib][D] bf16 calibration tokens at positions
+ *             0..n_calib-1; keys are de-rotated first
+ *   h_bases   host out [L*2*H][D][D] fp32, columns sorted by eigenvalue
+ *             descending, each column's largest-magnitude entry positive
+ *   h_eigvals host out [L*2*H][D]
+ * Shape and rope_theta come from desc (bases/eigvals/widths ignored). */
+int kvc_calibrate_pca(const kvc_plan_desc* desc, const uint16_t* h_calib, uint32_t n_calib,
+                      float* h_bases, double* h_eigvals, int n_threads);
+
+/* Greedy bit allocation on its own (host): the widths kvc_plan_create would
+ * assign. h_eigvals [n_units] (negative values count as 0), h_widths out
+ * [n_units]; the budget is floor(avg_bits * n_units + 0.5) bits, each unit at
+ * most max_bits (KVTC page, "Bit Budget Is Not Fair"). */
+int kvc_allocate_bits(const double* h_eigvals, uint64_t n_units, double avg_bits, uint32_t max_bits,
+                      uint8_t* h_widths);
+
+/* Kernel timing. Between kvc_profile_begin and kvc_profile_end every kernel the
+ * library launches is bracketed by CUDA events on its own stream.
+ * kvc_profile_end waits for those events, fills out[0 .. *n_kernels) with one
+ * entry per kernel name (launch count, summed device time in ms) and stops
+ * recording. Host-side bookkeeping only; not for use under stream capture. */
+typedef struct {
+  char name[40];
+  uint32_t launches;
+  double total_ms;
+} kvc_kernel_time;
+int kvc_profile_begin(void);
+int kvc_profile_end(kvc_kernel_time* out, int max_kernels, int* n_kernels);
+
+/* Stage entry points (check the CRC and rANS stages on their own).
+ * kvc_stage_crc32: CRC-32 of n bytes at d_src into *d_out (one block).
+ * kvc_stage_stream_encode: one stream record of n (<= 65536) byte symbols at
+ *   d_sym into d_out (capacity 16 + n rounded up to 16), using d_scratch
+ *   (2n bytes); d_res gets the record bytes.
+ * kvc_stage_stream_decode: decode the record at d_rec (rec_bytes) holding n
+ *   symbols into d_sym; d_res gets the status and record bytes. */
+int kvc_stage_crc32(const void* d_src, size_t n, uint32_t* d_out, cudaStream_t stream);
+int kvc_stage_stream_encode(const uint8_t* d_sym, uint32_t n, uint8_t* d_out, void* d_scratch,
+                            kvc_result* d_res, cudaStream_t stream);
+int kvc_stage_stream_decode(const uint8_t* d_rec, uint32_t rec_bytes, uint32_t n, uint8_t* d_sym,
+                            kvc_result* d_res, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KVC_H */

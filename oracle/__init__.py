@@ -76,6 +76,7 @@ def _load():
         "kvco_encode_transform": ([P(Desc), u32, u32, vp, vp, sz], sz),
         "kvco_decode_transform": ([P(Desc), vp, sz, vp, sz, P(u64)], i32),
         "kvco_transform_slice_codes": ([P(Desc), u32, vp, vp, vp, vp], i32),
+        "kvco_record_codes": ([P(Desc), u32, vp, u32, u32, vp, vp], i32),
         "kvco_container_codes": ([P(Desc), vp, sz, u32, vp, vp, P(u32)], i32),
         "kvco_pca": ([vp, u32, u32, u32, i32, dbl, vp, vp], i32),
         "kvco_jacobi_eigen": ([vp, u32, vp, vp], i32),
@@ -280,6 +281,16 @@ def transform_slice_codes(plan: Plan, slice_index: int, src_slice: np.ndarray):
     if st != OK:
         raise ValueError("oracle transform_slice_codes refused its arguments")
     return codes, qpre, zs[: _n_mid(plan)]
+
+
+def record_codes(plan: Plan, slice_index: int, rec: bytes, tcc: int):
+    d = plan.desc
+    r = np.frombuffer(bytes(rec), dtype=np.uint8) if len(rec) else np.zeros(1, np.uint8)
+    codes = np.zeros((tcc, d.head_dim), dtype=np.uint8)
+    zs = np.zeros((d.head_dim, d.chunk_tokens // d.block_tokens, 2), dtype=np.float32)
+    st = _load().kvco_record_codes(ctypes.byref(d), slice_index, _ptr(r), len(rec), tcc,
+                                   _ptr(codes), _ptr(zs))
+    return st, codes, zs
 
 
 def container_codes(plan: Plan, buf, n_slices: int):

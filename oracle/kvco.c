@@ -708,9 +708,12 @@ int kvco_allocate(const double* lambda, uint64_t n_units, double avg_bits, uint3
   for (uint64_t u = 0; u < n_units; u++)
     if (lambda[u] != lambda[u]) return KVCO_INVALID;
   heap_item* h = (heap_item*)malloc(sizeof(heap_item) * n_units);
+  /* a variance below zero (eigenvalue round-off) carries no distortion */
+  double* lam = (double*)malloc(sizeof(double) * n_units);
   for (uint64_t u = 0; u < n_units; u++) {
+    lam[u] = lambda[u] > 0.0 ? lambda[u] : 0.0;
     widths[u] = 0;
-    h[u].gain = lambda[u];
+    h[u].gain = lam[u];
     h[u].idx = u;
   }
   size_t n = n_units;
@@ -719,7 +722,7 @@ int kvco_allocate(const double* lambda, uint64_t n_units, double avg_bits, uint3
     uint64_t u = h[0].idx;
     widths[u]++;
     if (widths[u] < max_bits) {
-      h[0].gain = ldexp(lambda[u], -2 * (int)widths[u]);
+      h[0].gain = ldexp(lam[u], -2 * (int)widths[u]);
     } else {
       h[0] = h[n - 1];
       n--;
@@ -727,6 +730,7 @@ int kvco_allocate(const double* lambda, uint64_t n_units, double avg_bits, uint3
     heap_down(h, n, 0);
   }
   free(h);
+  free(lam);
   return KVCO_OK;
 }
 
@@ -1144,6 +1148,23 @@ int kvco_transform_slice_codes(const kvco_desc* d, uint32_t slice, const uint16_
   }
   free(cs); free(y); free(cc); free(qq);
   return KVCO_OK;
+}
+
+/* Test helper: codes [tcc][D] token-major and side info [D][ct / B][2] of one
+ * middle-chunk record of slice sidx (global index) holding tcc tokens. */
+int kvco_record_codes(const kvco_desc* d, uint32_t sidx, const uint8_t* rec, uint32_t len,
+                      uint32_t tcc, uint8_t* codes, float* zs) {
+  if (!transform_ok(d) || sidx >= n_slices_total(d) || tcc == 0 || tcc > d->chunk_tokens)
+    return KVCO_INVALID;
+  uint32_t D = d->head_dim, ct = d->chunk_tokens;
+  uint8_t* cc = (uint8_t*)malloc((size_t)ct * D);
+  uint8_t* syms = (uint8_t*)malloc((size_t)ct * D);
+  int st = mid_chunk_parse(d, sidx, rec, len, tcc, cc, zs, syms);
+  for (uint32_t t = 0; t < tcc && !st; t++)
+    for (uint32_t j = 0; j < D; j++) codes[(size_t)t * D + j] = cc[(size_t)j * ct + t];
+  free(cc);
+  free(syms);
+  return st;
 }
 
 /* Test helper: codes [n_slices][T][D] and side info [n_slices][n_mid][D][ct/B][2]

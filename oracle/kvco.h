@@ -85,6 +85,8 @@ int kvco_decode_transform(const kvco_desc* d, const uint8_t* src, size_t n, uint
                           size_t cap, uint64_t* written);
 int kvco_transform_slice_codes(const kvco_desc* d, uint32_t slice, const uint16_t* src_slice,
                                uint8_t* codes, float* qpre, float* zs);
+int kvco_record_codes(const kvco_desc* d, uint32_t sidx, const uint8_t* rec, uint32_t len,
+                      uint32_t tcc, uint8_t* codes, float* zs);
 int kvco_container_codes(const kvco_desc* d, const uint8_t* src, size_t n, uint32_t rec,
                          uint8_t* codes, float* zs, uint32_t* n_tokens);
 

@@ -1,3 +1,4 @@
+import importlib.util
 import os
 import sys
 
@@ -6,6 +7,18 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
+
+
+def _build_library():
+    """Compile libkvc.so in-tree if it is missing or stale (nvcc cross-compiles)."""
+    path = os.path.join(ROOT, "transform_codec_b200", "build.py")
+    spec = importlib.util.spec_from_file_location("_kvc_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.build()
+
+
+_build_library()
 
 
 def pytest_configure(config):

@@ -1,0 +1,144 @@
+"""Lossless path on the GPU against the oracle: the GPU container must be the
+oracle's container byte for byte, the GPU decoder must restore the oracle's
+containers exactly, and damaged or truncated containers must be refused with
+the oracle's status."""
+import dataclasses
+
+import numpy as np
+import pytest
+
+import kvgen
+import oracle
+import transform_codec_b200 as kvc
+from kvc_gpu import decode, encode
+
+pytestmark = pytest.mark.gpu
+
+
+def _w(name, **kw):
+    return dataclasses.replace(kvgen.WORKLOADS[name], **kw)
+
+
+CASES = [
+    _w("lossless-1x8x512x128-bf16"),
+    _w("lossless-1x8x512x128-bf16", n_tokens=700),
+    _w("lossless-12x12x1024x64-fp16", n_layers=1, n_heads=3, n_tokens=1500),
+    _w("lossless-1x8x512x128-bf16", n_tokens=3, head_dim=10, values_per_chunk=16),
+    _w("lossless-1x8x512x128-bf16", n_tokens=1000, head_dim=24, values_per_chunk=4096),
+    _w("lossless-8x8x1536x128-bf16", n_layers=1, n_heads=2),
+    _w("lossless-12x12x1024x64-fp16", n_layers=2, n_heads=2),
+]
+
+
+def _plans(w):
+    s = kvc.Shape.from_workload(w)
+    return kvc.Plan(s), oracle.Plan.from_workload(w)
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: f"{w.n_layers}x{w.n_heads}x{w.n_tokens}x{w.head_dim}")
+def test_lossless_parity(w):
+    plan, oplan = _plans(w)
+    x = kvgen.slices(w)
+    want = oracle.encode_lossless(oplan, x)
+    st, got = encode(plan, kvc.LOSSLESS, x)
+    assert st == kvc.OK
+    assert len(got) == len(want)
+    assert got == want
+    st, y = decode(plan, kvc.LOSSLESS, want, w.n_slices)
+    assert st == kvc.OK and np.array_equal(y, x)
+
+
+def test_lossless_subrange_and_empty():
+    w = _w("lossless-1x8x512x128-bf16")
+    plan, oplan = _plans(w)
+    x = kvgen.slices(w, first=5, n=3)
+    st, got = encode(plan, kvc.LOSSLESS, x, first_slice=5)
+    assert st == kvc.OK and got == oracle.encode_lossless(oplan, x, first_slice=5)
+    st, y = decode(plan, kvc.LOSSLESS, got, 3)
+    assert st == kvc.OK and np.array_equal(y, x)
+    e = np.zeros((0, w.n_tokens, w.head_dim), np.uint16)
+    st, got = encode(plan, kvc.LOSSLESS, e)
+    assert st == kvc.OK and got == oracle.encode_lossless(oplan, e)
+    st, y = decode(plan, kvc.LOSSLESS, got, 1)
+    assert st == kvc.OK and y.shape[0] == 0
+
+
+def test_random_control_block_takes_raw():
+    raw = kvgen.random_bytes(4 << 20)
+    w = _w("lossless-12x12x1024x64-fp16", n_layers=1, n_heads=1, n_tokens=16384)
+    plan, oplan = _plans(w)
+    x = raw.view(np.uint16).reshape(2, 16384, 64)
+    st, got = encode(plan, kvc.LOSSLESS, x)
+    assert st == kvc.OK
+    assert len(got) == raw.size + 64 + 48 * 32
+    assert got == oracle.encode_lossless(oplan, x)
+    st, y = decode(plan, kvc.LOSSLESS, got, 2)
+    assert st == kvc.OK and np.array_equal(y, x)
+
+
+def test_special_bit_patterns():
+    rng = np.random.default_rng(3)
+    pats = np.array([0x7FC0, 0xFFC0, 0x7F80, 0xFF80, 0x0000, 0x8000, 0x0001, 0x807F, 0x7F81],
+                    np.uint16)
+    x = rng.choice(pats, size=(2, 512, 128)).astype(np.uint16)
+    x[1] = 0x3F80
+    w = _w("lossless-1x8x512x128-bf16", n_heads=1)
+    plan, oplan = _plans(w)
+    st, got = encode(plan, kvc.LOSSLESS, x)
+    assert st == kvc.OK and got == oracle.encode_lossless(oplan, x)
+    st, y = decode(plan, kvc.LOSSLESS, got, 2)
+    assert st == kvc.OK and np.array_equal(y, x)
+
+
+def test_full_size_migration_block():
+    """50,331,648 bytes (8 layers x 8 heads x 1536 x 128, K+V), bit exact."""
+    w = kvgen.WORKLOADS["lossless-8x8x1536x128-bf16"]
+    plan, oplan = _plans(w)
+    x = kvgen.slices(w)
+    assert x.nbytes == 50_331_648
+    st, got = encode(plan, kvc.LOSSLESS, x)
+    assert st == kvc.OK and got == oracle.encode_lossless(oplan, x)
+    st, y = decode(plan, kvc.LOSSLESS, got, w.n_slices)
+    assert st == kvc.OK and np.array_equal(y, x)
+
+
+def test_full_size_frame_of_32k_cache():
+    """One 64 MiB frame (one layer's K: 8 heads x 32768 x 128) of the 64-layer cache."""
+    w = kvgen.WORKLOADS["lossless-64x8x32768x128-bf16"]
+    plan, oplan = _plans(w)
+    x = kvgen.slices(w, first=80, n=8)
+    st, got = encode(plan, kvc.LOSSLESS, x, first_slice=80)
+    assert st == kvc.OK and got == oracle.encode_lossless(oplan, x, first_slice=80)
+    st, y = decode(plan, kvc.LOSSLESS, got, 8)
+    assert st == kvc.OK and np.array_equal(y, x)
+
+
+def test_damage_is_refused_with_oracle_status():
+    w = _w("lossless-1x8x512x128-bf16", n_heads=2)
+    plan, oplan = _plans(w)
+    x = kvgen.slices(w)
+    c = bytearray(oracle.encode_lossless(oplan, x))
+    rng = np.random.default_rng(5)
+    n_idx = 64 + 16 * 4
+    positions = list(range(0, n_idx)) + list(rng.integers(n_idx, len(c), 120))
+    for pos in positions:
+        orig = c[pos]
+        c[pos] = orig ^ int(rng.integers(1, 256))
+        want, _ = oracle.decode_lossless(oplan, bytes(c))
+        got, _ = decode(plan, kvc.LOSSLESS, bytes(c), w.n_slices)
+        assert want != oracle.OK and got == want, (pos, got, want)
+        c[pos] = orig
+    for n in [0, 1, 63, 64, 100, n_idx, len(c) // 2, len(c) - 16, len(c) - 1]:
+        got, _ = decode(plan, kvc.LOSSLESS, bytes(c[:n]), w.n_slices)
+        assert got == kvc.ERR_TRUNCATED, n
+    got, _ = decode(plan, kvc.LOSSLESS, bytes(c) + bytes(16), w.n_slices)
+    assert got == kvc.ERR_CORRUPT
+
+
+def test_plan_mismatch_and_capacity():
+    w = _w("lossless-1x8x512x128-bf16", n_heads=1)
+    plan, oplan = _plans(w)
+    c = oracle.encode_lossless(oplan, kvgen.slices(w))
+    other = kvc.Plan(kvc.Shape(kvc.BF16, 1, 1, 513, 128))
+    assert decode(other, kvc.LOSSLESS, c, 2)[0] == kvc.ERR_PLAN_MISMATCH
+    assert decode(plan, kvc.LOSSLESS, c, 1)[0] == kvc.ERR_CAPACITY

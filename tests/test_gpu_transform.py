@@ -1,0 +1,198 @@
+"""Transform-coding path on the GPU against the oracle, judged by the codec's
+parity rule: at least 99.999% of quantised codes identical, any mismatch only
++-1 where the oracle's pre-rounding quotient lies within 1e-4 of a rounding
+boundary, raw regions bit exact, and reconstruction within relative RMS 1e-3 of
+the oracle's (KVTC page, "How the Pipeline Works"; Codec-Gauge page,
+"Compression Conditions")."""
+import dataclasses
+import struct
+
+import numpy as np
+import pytest
+
+import kvgen
+import oracle
+import transform_codec_b200 as kvc
+from kvc_gpu import decode, encode, rel_rms
+
+pytestmark = pytest.mark.gpu
+
+CODE_MATCH = 0.99999
+BOUNDARY = 1e-4
+REL_RMS = 1e-3
+
+
+def _w(**kw):
+    base = dataclasses.replace(kvgen.WORKLOADS["transform-32x8x8192x128-bf16"], n_layers=1,
+                               n_heads=2)
+    return dataclasses.replace(base, **kw)
+
+
+def _oracle_pca(w, slices):
+    cal = kvgen.calibration(w)
+    out = {}
+    for s in slices:
+        out[s] = oracle.pca(cal[s], (s // w.n_heads) % 2 == 0, w.theta)
+    return out, cal
+
+
+def _small_inputs(w):
+    pcs, _ = _oracle_pca(w, range(w.n_slices))
+    bases = np.stack([pcs[s][0] for s in range(w.n_slices)])
+    lam = np.stack([pcs[s][1] for s in range(w.n_slices)])
+    widths = oracle.allocate(lam, w.avg_bits, w.max_bits).reshape(lam.shape)
+    return bases, lam, widths
+
+
+def _plans(w, bases, widths):
+    plan = kvc.Plan(kvc.Shape.from_workload(w), bases=bases, widths=widths)
+    oplan = oracle.Plan.from_workload(w, bases=bases, widths=widths)
+    return plan, oplan
+
+
+def _check_codes(codes, ocodes, qpre, widths_slice, mid):
+    """Parity rule on one slice's middle tokens; returns (compared, mismatches)."""
+    coded = widths_slice > 0
+    a = codes[mid][:, coded].astype(np.int32)
+    b = ocodes[mid][:, coded].astype(np.int32)
+    q = qpre[mid][:, coded].astype(np.float64)
+    diff = a != b
+    if diff.any():
+        assert np.all(np.abs(a[diff] - b[diff]) == 1)
+        dist = np.abs(q[diff] - (np.floor(q[diff]) + 0.5))
+        assert np.all(dist <= BOUNDARY), dist.max()
+    return a.size, int(diff.sum())
+
+
+def _regions(w):
+    s_end = min(w.n_sink, w.n_tokens)
+    r_start = max(s_end, w.n_tokens - w.n_recent if w.n_tokens > w.n_recent else 0)
+    return s_end, r_start
+
+
+@pytest.mark.parametrize("T", [1024, 640, 644, 100])
+def test_transform_parity(T):
+    w = _w(n_tokens=T)
+    bases, lam, widths = _small_inputs(w)
+    plan, oplan = _plans(w, bases, widths)
+    assert np.array_equal(plan.widths(), widths)
+    assert plan.crc == oracle.plan_crc(oplan)
+    x = kvgen.slices(w)
+    st, got = encode(plan, kvc.TRANSFORM, x)
+    assert st == kvc.OK
+    want = oracle.encode_transform(oplan, x)
+    assert len(got) <= plan.max_encoded_bytes(kvc.TRANSFORM, w.n_slices)
+    st, codes, _ = oracle.container_codes(oplan, got, w.n_slices)
+    assert st == oracle.OK
+    s_end, r_start = _regions(w)
+    mid = slice(s_end, r_start)
+    total = bad = 0
+    for s in range(w.n_slices):
+        oc, qp, _ = oracle.transform_slice_codes(oplan, s, x[s])
+        n, m = _check_codes(codes[s], oc, qp, widths[s], mid)
+        total += n
+        bad += m
+    assert bad <= (1 - CODE_MATCH) * max(total, 1)
+    st_g, y_g = decode(plan, kvc.TRANSFORM, got, w.n_slices)
+    st_o, y_o = oracle.decode_transform(oplan, want)
+    assert st_g == kvc.OK and st_o == oracle.OK
+    assert np.array_equal(y_g[:, :s_end], x[:, :s_end])
+    assert np.array_equal(y_g[:, r_start:], x[:, r_start:])
+    assert rel_rms(y_o, y_g) <= REL_RMS
+    st_go, y_go = decode(plan, kvc.TRANSFORM, want, w.n_slices)  # GPU decoder, oracle bytes
+    assert st_go == kvc.OK and rel_rms(y_o, y_go) <= REL_RMS
+
+
+def test_transform_identity_basis_all_eight_bits():
+    w = _w(n_tokens=900)
+    D, S = w.head_dim, w.n_slices
+    bases = np.broadcast_to(np.eye(D, dtype=np.float32), (S, D, D)).copy()
+    widths = np.full((S, D), 8, np.uint8)
+    plan, oplan = _plans(w, bases, widths)
+    x = kvgen.slices(w)
+    st, got = encode(plan, kvc.TRANSFORM, x)
+    assert st == kvc.OK
+    st, codes, _ = oracle.container_codes(oplan, got, S)
+    assert st == oracle.OK
+    s_end, r_start = _regions(w)
+    total = bad = 0
+    for s in range(S):
+        oc, qp, _ = oracle.transform_slice_codes(oplan, s, x[s])
+        n, m = _check_codes(codes[s], oc, qp, widths[s], slice(s_end, r_start))
+        total += n
+        bad += m
+    assert bad <= (1 - CODE_MATCH) * total
+    st, y = decode(plan, kvc.TRANSFORM, got, S)
+    st_o, y_o = oracle.decode_transform(oplan, oracle.encode_transform(oplan, x))
+    assert st == kvc.OK and rel_rms(y_o, y) <= REL_RMS
+    assert rel_rms(x, y) < 5e-3
+
+
+def test_transform_damage_and_plan_mismatch():
+    w = _w(n_tokens=700)
+    bases, lam, widths = _small_inputs(w)
+    plan, oplan = _plans(w, bases, widths)
+    c = bytearray(oracle.encode_transform(oplan, kvgen.slices(w)))
+    rng = np.random.default_rng(8)
+    for pos in list(range(0, 64 + 16 * 8, 2)) + list(rng.integers(128, len(c), 80)):
+        orig = c[pos]
+        c[pos] = orig ^ int(rng.integers(1, 256))
+        want, _ = oracle.decode_transform(oplan, bytes(c))
+        got, _ = decode(plan, kvc.TRANSFORM, bytes(c), w.n_slices)
+        assert want != oracle.OK and got == want, (pos, got, want)
+        c[pos] = orig
+    for n in [0, 50, 64, 200, len(c) - 16]:
+        assert decode(plan, kvc.TRANSFORM, bytes(c[:n]), w.n_slices)[0] == kvc.ERR_TRUNCATED
+    w2 = widths.copy()
+    w2[0, 0] = 1 if w2[0, 0] != 1 else 2
+    other = kvc.Plan(kvc.Shape.from_workload(w), bases=bases, widths=w2)
+    assert decode(other, kvc.TRANSFORM, bytes(c), w.n_slices)[0] == kvc.ERR_PLAN_MISMATCH
+
+
+def _records(container: bytes):
+    n = struct.unpack_from("<I", container, 36)[0]
+    out = []
+    for i in range(n):
+        off, ln, _ = struct.unpack_from("<QII", container, 64 + 16 * i)
+        out.append(container[off:off + ln])
+    return out
+
+
+def test_transform_full_size_sampled():
+    """Llama-8B-shaped cache (32 x 8 x 8192 x 128, 1.07 GB): the GPU encodes and
+    decodes all 512 slices; sampled slices are checked against the oracle."""
+    w = kvgen.WORKLOADS["transform-32x8x8192x128-bf16"]
+    shape = kvc.Shape.from_workload(w)
+    sampled = [0, 9, 262, 511]
+    pcs, cal = _oracle_pca(w, sampled)
+    bases, lam = kvc.calibrate_pca(shape, cal)
+    for s in sampled:
+        bases[s], lam[s] = pcs[s]
+    widths = oracle.allocate(lam, w.avg_bits, w.max_bits).reshape(lam.shape)
+    plan, oplan = _plans(w, bases, widths)
+    x = kvgen.slices(w)
+    st, got = encode(plan, kvc.TRANSFORM, x)
+    assert st == kvc.OK
+    recs = _records(got)
+    s_end, r_start = _regions(w)
+    rps = 1 + (r_start - s_end + w.chunk_tokens - 1) // w.chunk_tokens
+    assert len(recs) == w.n_slices * rps
+    st_g, y_g = decode(plan, kvc.TRANSFORM, got, w.n_slices)
+    assert st_g == kvc.OK
+    for s in sampled:
+        oc, qp, _ = oracle.transform_slice_codes(oplan, s, x[s])
+        raw = np.concatenate([x[s, :s_end], x[s, r_start:]]).tobytes()
+        assert recs[s * rps] == raw + bytes((-len(raw)) % 16)
+        codes = np.zeros_like(oc)
+        for c in range(rps - 1):
+            t0 = s_end + c * w.chunk_tokens
+            tcc = min(w.chunk_tokens, r_start - t0)
+            st, cc, _ = oracle.record_codes(oplan, s, recs[s * rps + 1 + c], tcc)
+            assert st == oracle.OK
+            codes[t0:t0 + tcc] = cc
+        n, m = _check_codes(codes, oc, qp, widths[s], slice(s_end, r_start))
+        assert m <= (1 - CODE_MATCH) * n
+        one = oracle.encode_transform(oplan, x[s:s + 1], first_slice=s)
+        st_o, y_o = oracle.decode_transform(oplan, one, n_slices_cap=1)
+        assert st_o == oracle.OK
+        assert rel_rms(y_o[0], y_g[s]) <= REL_RMS

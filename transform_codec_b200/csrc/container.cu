@@ -1,0 +1,366 @@
+// Container kernels (sm_100a): header + chunk index writer with the aggregate
+// header CRC, record placement, and the decoder's header/index validation
+// (QATQ page, "How it works": bounded chunks with ordered lengths and an
+// aggregate checksum; "QATC v2 checksum validated": corrupt or truncated
+// payloads are refused before restore). Also the stage kernels used to check
+// the CRC and rANS stages on their own.
+#include "kvc_device.cuh"
+#include "kvc_internal.h"
+
+namespace kvc {
+
+struct Result {
+  int32_t status;
+  uint32_t pad;
+  uint64_t bytes;
+};
+
+namespace {
+
+constexpr uint32_t kBig = 1024;  // threads of the single-block container kernels
+
+__device__ inline uint64_t block_exclusive_scan64(uint64_t v, uint64_t* tmp, uint64_t* total) {
+  const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
+  uint64_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint64_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= uint32_t(o)) x += y;
+  }
+  __syncthreads();
+  if (lane == 31) tmp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t nw = blockDim.x >> 5;
+    uint64_t w = lane < nw ? tmp[lane] : 0ull;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      uint64_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= uint32_t(o)) w += y;
+    }
+    if (lane < nw) tmp[lane] = w;
+  }
+  __syncthreads();
+  uint64_t base = warp ? tmp[warp - 1] : 0ull;
+  *total = tmp[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return base + x - v;
+}
+
+__global__ void __launch_bounds__(kBig)
+k_finalize(HeaderFields h, EncodeLayout ws, uint8_t* dst, uint64_t dst_cap, Result* res) {
+  __shared__ uint32_t crc_t[1024];
+  __shared__ uint32_t red[32];
+  __shared__ uint64_t tmp64[32];
+  const uint32_t tid = threadIdx.x, nthr = blockDim.x;
+  const uint32_t nr = h.n_records;
+  crc_tables_init(crc_t);
+  const uint32_t per = (nr + nthr - 1) / nthr;
+  const uint32_t beg = min(nr, tid * per), end = min(nr, beg + per);
+  uint64_t mine = 0;
+  for (uint32_t i = beg; i < end; ++i) mine += ws.rec_len[i];
+  uint64_t sum_all;
+  uint64_t pre = block_exclusive_scan64(mine, tmp64, &sum_all);
+  const uint64_t first = uint64_t(kHeaderBytes) + uint64_t(kIndexEntry) * nr;
+  const uint64_t total = first + sum_all;
+  if (total > dst_cap) {
+    if (tid == 0) {
+      ws.state->status = kErrCapacity;
+      ws.state->total_bytes = total;
+      res->status = kErrCapacity;
+      res->bytes = total;
+    }
+    return;
+  }
+  uint64_t off = first + pre;
+  for (uint32_t i = beg; i < end; ++i) {
+    ws.rec_off[i] = off;
+    uint32_t len = ws.rec_len[i];
+    uint4 ent = make_uint4(uint32_t(off), uint32_t(off >> 32), len, ws.rec_crc[i]);
+    *reinterpret_cast<uint4*>(dst + kHeaderBytes + uint64_t(kIndexEntry) * i) = ent;
+    off += len;
+  }
+  if (tid == 0) {
+    uint32_t* w = reinterpret_cast<uint32_t*>(dst);
+    w[0] = 0x3143564bu;  // "KVC1"
+    w[1] = 1u | (h.path << 16) | (h.dtype << 24);
+    w[2] = h.L; w[3] = h.H; w[4] = h.T; w[5] = h.D;
+    w[6] = h.first_slice; w[7] = h.n_slices; w[8] = h.chunk_tokens; w[9] = nr;
+    w[10] = uint32_t(total); w[11] = uint32_t(total >> 32);
+    w[12] = h.plan_crc;
+    w[13] = h.n_sink | (h.n_recent << 16);
+    w[14] = h.block_tokens;
+  }
+  __syncthreads();
+  const uint8_t* cdst = dst;
+  uint32_t hcrc = crc32_block_bytes(
+      [cdst](uint64_t i) -> uint32_t { return i < 60 ? cdst[i] : cdst[kHeaderBytes + (i - 60)]; },
+      60ull + uint64_t(kIndexEntry) * nr, crc_t, red);
+  if (tid == 0) {
+    reinterpret_cast<uint32_t*>(dst)[15] = hcrc;
+    ws.state->status = kOk;
+    ws.state->n_records = nr;
+    ws.state->total_bytes = total;
+    res->status = kOk;
+    res->bytes = total;
+  }
+}
+
+__global__ void k_copy_records(EncodeLayout ws, uint32_t nr, uint8_t* dst) {
+  if (ws.state->status != kOk) return;
+  for (uint32_t r = blockIdx.x; r < nr; r += gridDim.x) {
+    const uint4* s = reinterpret_cast<const uint4*>(ws.slots + uint64_t(r) * ws.slot_bytes);
+    uint4* d = reinterpret_cast<uint4*>(dst + ws.rec_off[r]);
+    const uint32_t q = ws.rec_len[r] / 16u;
+    for (uint32_t i = threadIdx.x; i < q; i += blockDim.x) d[i] = s[i];
+  }
+}
+
+__global__ void __launch_bounds__(kBig)
+k_check_container(const uint8_t* src, uint64_t src_bytes, ContainerExpect e, DecodeState* ds,
+                  Result* res) {
+  __shared__ uint32_t crc_t[1024];
+  __shared__ uint32_t red[32];
+  __shared__ int st_s;
+  __shared__ uint32_t nr_s, first_s, ns_s;
+  const uint32_t tid = threadIdx.x, nthr = blockDim.x;
+  crc_tables_init(crc_t);
+  if (tid == 0) {
+    int st = kOk;
+    uint32_t nr = 0;
+    if (src_bytes < kHeaderBytes) st = kErrTruncated;
+    else if (ld_u32(src) != 0x3143564bu || ld_u16(src + 4) != 1u) st = kErrCorrupt;
+    else {
+      uint64_t total = ld_u64(src + 40);
+      if (src_bytes < total) st = kErrTruncated;
+      else if (src_bytes > total) st = kErrCorrupt;
+      else {
+        nr = ld_u32(src + 36);
+        if (uint64_t(kHeaderBytes) + uint64_t(kIndexEntry) * nr > total) st = kErrCorrupt;
+      }
+    }
+    st_s = st;
+    nr_s = nr;
+  }
+  __syncthreads();
+  uint64_t total = 0;
+  if (st_s == kOk) {
+    const uint32_t nr = nr_s;
+    total = ld_u64(src + 40);
+    uint32_t hcrc = crc32_block_bytes(
+        [src](uint64_t i) -> uint32_t { return i < 60 ? src[i] : src[kHeaderBytes + (i - 60)]; },
+        60ull + uint64_t(kIndexEntry) * nr, crc_t, red);
+    if (tid == 0) {
+      int st = kOk;
+      uint32_t first = ld_u32(src + 24), ns = ld_u32(src + 28);
+      if (hcrc != ld_u32(src + 60)) st = kErrCorrupt;
+      else if (src[6] != e.path || src[7] != e.dtype || ld_u32(src + 8) != e.L ||
+               ld_u32(src + 12) != e.H || ld_u32(src + 16) != e.T || ld_u32(src + 20) != e.D ||
+               ld_u32(src + 32) != e.chunk_tokens)
+        st = kErrPlanMismatch;
+      else if (ld_u16(src + 58) != 0) st = kErrCorrupt;
+      else if (e.path == 0) {
+        if (ld_u32(src + 48) || ld_u16(src + 52) || ld_u16(src + 54) || ld_u16(src + 56))
+          st = kErrCorrupt;
+      } else if (ld_u16(src + 52) != e.n_sink || ld_u16(src + 54) != e.n_recent ||
+                 ld_u16(src + 56) != e.block_tokens || ld_u32(src + 48) != e.plan_crc) {
+        st = kErrPlanMismatch;
+      }
+      if (st == kOk && uint64_t(first) + ns > uint64_t(e.L) * 2u * e.H) st = kErrPlanMismatch;
+      if (st == kOk && uint64_t(ns) * e.recs_per_slice != nr) st = kErrCorrupt;
+      st_s = st;
+      first_s = first;
+      ns_s = ns;
+    }
+    __syncthreads();
+    if (st_s == kOk) {
+      const uint64_t start = uint64_t(kHeaderBytes) + uint64_t(kIndexEntry) * nr;
+      int bad = 0;
+      for (uint32_t i = tid; i < nr; i += nthr) {
+        const uint8_t* en = src + kHeaderBytes + uint64_t(kIndexEntry) * i;
+        uint64_t o = ld_u64(en);
+        uint32_t len = ld_u32(en + 8);
+        if (len & 15u) bad = 1;
+        if (i == 0 && o != start) bad = 1;
+        if (i + 1 < nr && ld_u64(en + kIndexEntry) != o + len) bad = 1;
+        if (i + 1 == nr && o + len != total) bad = 1;
+      }
+      if (nr == 0 && start != total) bad = 1;
+      bad = __syncthreads_or(bad);
+      if (tid == 0) {
+        int st = bad ? kErrCorrupt : kOk;
+        if (st == kOk && uint64_t(ns_s) * e.T * e.D * 2u > e.dst_cap) st = kErrCapacity;
+        st_s = st;
+      }
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int st = st_s;
+    ds->status = st;
+    ds->first_slice = st == kOk ? first_s : 0;
+    ds->n_slices = st == kOk ? ns_s : 0;
+    ds->n_records = st == kOk ? nr_s : 0;
+    ds->err_key = ~0ull;
+    ds->out_bytes = st == kOk ? uint64_t(ns_s) * e.T * e.D * 2u : 0;
+    res->status = st;
+    res->bytes = 0;
+  }
+}
+
+__global__ void k_decode_finish(const DecodeState* ds, Result* res) {
+  int st = ds->status;
+  if (st == kOk && ds->err_key != ~0ull) st = int(ds->err_key & 0xffu);
+  res->status = st;
+  res->bytes = st == kOk ? ds->out_bytes : 0;
+}
+
+// ------------------------------------------------------------------ stage kernels
+__global__ void __launch_bounds__(kBig) k_stage_crc32(const uint8_t* src, uint64_t n, uint32_t* out) {
+  __shared__ uint32_t crc_t[1024];
+  __shared__ uint32_t red[32];
+  crc_tables_init(crc_t);
+  uint32_t c = crc32_block_bytes([src](uint64_t i) -> uint32_t { return src[i]; }, n, crc_t, red);
+  if (threadIdx.x == 0) *out = c;
+}
+
+struct __align__(16) StageSmem {
+  uint32_t hist[256], freq[256], rem[256], fc[256], rcp[256], cum[260];
+  uint32_t lut[kProbScale];
+  uint32_t states[kMaxLanes];
+  uint32_t tmp[32];
+  uint32_t W[4], wbeg[4], sub_len[4];
+  uint32_t k, mode, bytes;
+  StreamInfo si;
+};
+
+__global__ void __launch_bounds__(256)
+k_stage_stream_encode(const uint8_t* sym, uint32_t n, uint8_t* out, uint16_t* scratch, Result* res) {
+  __shared__ StageSmem S;
+  const uint32_t tid = threadIdx.x;
+  for (uint32_t i = tid; i < 256; i += blockDim.x) S.hist[i] = 0;
+  __syncthreads();
+  for (uint32_t i = tid; i < n; i += blockDim.x) atomicAdd(&S.hist[sym[i]], 1u);
+  __syncthreads();
+  uint32_t k = block_normalize(S.hist, n, S.freq, S.rem, S.tmp);
+  block_enc_tables(S.freq, S.fc, S.rcp, S.tmp);
+  const uint32_t N = rans_lanes(n), G = rans_groups(N);
+  const uint32_t warp = tid >> 5, lane = tid & 31u;
+  if (k >= 2 && warp < G) {
+    uint32_t b0, len0, b1 = n, len1;
+    lane_range(n, N, warp * kGroupLanes, b0, len0);
+    if (warp + 1 < G) lane_range(n, N, (warp + 1) * kGroupLanes, b1, len1);
+    uint32_t x;
+    uint32_t Wg = rans_encode_group([sym](uint32_t i) -> uint32_t { return sym[i]; }, n, N, warp,
+                                    S.fc, S.rcp, scratch + b0, b1 - b0, &x);
+    if (warp * kGroupLanes + lane < N) S.states[warp * kGroupLanes + lane] = x;
+    if (lane == 0) { S.W[warp] = Wg; S.wbeg[warp] = b1 - Wg; }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t raw_b = 16u + pad16(n);
+    if (k == 1) { S.mode = kModeConst; S.bytes = 16; }
+    else if (k >= 2) {
+      uint32_t rb = rans_layout(n, k, S.W, S.sub_len);
+      if (rb < raw_b) { S.mode = kModeRans; S.bytes = rb; }
+      else { S.mode = kModeRaw; S.bytes = raw_b; }
+    } else { S.mode = kModeRaw; S.bytes = raw_b; }
+    S.k = k;
+  }
+  __syncthreads();
+  block_write_stream(out, S.mode, n, S.bytes, n ? uint32_t(sym[0]) : 0u, S.k, S.freq, S.states,
+                     scratch, S.wbeg, S.W, S.sub_len,
+                     [sym](uint32_t i) -> uint32_t { return sym[i]; }, S.tmp);
+  if (tid == 0) { res->status = kOk; res->bytes = S.bytes; }
+}
+
+__global__ void __launch_bounds__(256)
+k_stage_stream_decode(const uint8_t* rec, uint32_t rec_bytes, uint32_t n, uint8_t* sym, Result* res) {
+  __shared__ StageSmem S;
+  const uint32_t tid = threadIdx.x;
+  int st = block_parse_stream(rec, rec_bytes, n, &S.si, S.freq, S.tmp);
+  bool ok = st == kOk;
+  if (ok) {
+    if (S.si.mode == kModeRaw) {
+      for (uint32_t i = tid; i < n; i += blockDim.x) sym[i] = rec[16 + i];
+    } else if (S.si.mode == kModeConst) {
+      for (uint32_t i = tid; i < n; i += blockDim.x) sym[i] = uint8_t(S.si.sym);
+    } else {
+      block_dec_lut(S.freq, S.cum, S.lut, S.tmp);
+      const uint32_t N = rans_lanes(n), G = rans_groups(N), warp = tid >> 5;
+      bool okw = true;
+      if (warp < G)
+        okw = rans_decode_group(rec + S.si.sub_off[warp], S.si.sub_len[warp], n, N, warp, S.lut,
+                                [sym](uint32_t i, uint32_t s) { sym[i] = uint8_t(s); });
+      ok = __syncthreads_and(okw);
+    }
+  }
+  if (tid == 0) {
+    res->status = ok ? kOk : kErrCorrupt;
+    res->bytes = ok ? S.si.bytes : 0;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_finalize(const HeaderFields& h, const EncodeLayout& ws, uint8_t* dst,
+                            uint64_t dst_cap, void* res, cudaStream_t st) {
+  {
+    ProfRange pr_("finalize", st);
+    k_finalize<<<1, kBig, 0, st>>>(h, ws, dst, dst_cap, static_cast<Result*>(res));
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || h.n_records == 0) return e;
+  uint32_t grid = min(h.n_records, 148u * 8u);
+  {
+    ProfRange pr_("copy_records", st);
+    k_copy_records<<<grid, 256, 0, st>>>(ws, h.n_records, dst);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_check_container(const uint8_t* src, uint64_t src_bytes,
+                                   const ContainerExpect& e, DecodeState* ds, void* res,
+                                   cudaStream_t st) {
+  {
+    ProfRange pr_("check_container", st);
+    k_check_container<<<1, kBig, 0, st>>>(src, src_bytes, e, ds, static_cast<Result*>(res));
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_finish(DecodeState* ds, void* res, cudaStream_t st) {
+  {
+    ProfRange pr_("decode_finish", st);
+    k_decode_finish<<<1, 1, 0, st>>>(ds, static_cast<Result*>(res));
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stage_crc32(const uint8_t* src, uint64_t n, uint32_t* out, cudaStream_t st) {
+  {
+    ProfRange pr_("stage_crc32", st);
+    k_stage_crc32<<<1, kBig, 0, st>>>(src, n, out);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stage_stream_encode(const uint8_t* sym, uint32_t n, uint8_t* out,
+                                       uint16_t* scratch, void* res, cudaStream_t st) {
+  {
+    ProfRange pr_("stage_stream_encode", st);
+    k_stage_stream_encode<<<1, 256, 0, st>>>(sym, n, out, scratch, static_cast<Result*>(res));
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_stage_stream_decode(const uint8_t* rec, uint32_t rec_bytes, uint32_t n,
+                                       uint8_t* sym, void* res, cudaStream_t st) {
+  {
+    ProfRange pr_("stage_stream_decode", st);
+    k_stage_stream_decode<<<1, 256, 0, st>>>(rec, rec_bytes, n, sym, static_cast<Result*>(res));
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace kvc

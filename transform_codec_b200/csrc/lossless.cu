@@ -1,0 +1,285 @@
+// Lossless front-end kernels (sm_100a): per chunk of tc tokens x D channels,
+// channel-major byte planes (p = 0 low byte, p = 1 high byte), each plane one
+// stream record that keeps the smallest of CONST / RANS / RAW (AT-1 Memory
+// page, "KV & tensor mode": channel-major reorder, byte planes, keep whichever
+// is smaller; QATQ page, "qatq encode": bounded chunks, known row width).
+#include "kvc_device.cuh"
+#include "kvc_internal.h"
+
+namespace kvc {
+namespace {
+
+constexpr uint32_t kThreads = 256;  // 8 warps: plane p = warp / 4, group = warp % 4
+
+struct __align__(16) EncSmem {
+  uint32_t crc_t[1024];
+  uint32_t hist[2][256];
+  uint32_t freq[2][256];
+  uint32_t rem[256];
+  uint32_t fc[2][256];
+  uint32_t rcp[2][256];
+  uint32_t states[2][kMaxLanes];
+  uint32_t tmp[32], red[32];
+  uint32_t k[2], mode[2], bytes[2], csym[2];
+  uint32_t W[2][4], wbeg[2][4], sub_len[2][4];
+};
+
+struct __align__(16) DecSmem {
+  uint32_t crc_t[1024];
+  uint32_t freq[2][256];
+  uint32_t cum[2][260];
+  uint32_t lut[2][kProbScale];
+  uint32_t tmp[32], red[32];
+  StreamInfo si[2];
+  uint32_t crc_ok;
+};
+
+// i -> (d, t) for channel-major index i = d * tcc + t
+struct ChanMajor {
+  uint32_t tcc, magic;
+  __device__ ChanMajor(uint32_t tcc_) : tcc(tcc_), magic(0xffffffffu / tcc_) {}
+  __device__ inline void split(uint32_t i, uint32_t& d, uint32_t& t) const {
+    d = __umulhi(i, magic);
+    t = i - d * tcc;
+    if (t >= tcc) { ++d; t -= tcc; }
+  }
+};
+
+__global__ void __launch_bounds__(kThreads)
+k_lossless_encode(LosslessShape sh, const uint16_t* __restrict__ src, EncodeLayout ws) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  EncSmem& S = *reinterpret_cast<EncSmem*>(smem_raw);
+  uint16_t* vals = reinterpret_cast<uint16_t*>(smem_raw + sizeof(EncSmem));
+  const uint32_t tid = threadIdx.x, nthr = blockDim.x;
+  const uint32_t r = blockIdx.x;
+  const uint32_t slice = r / sh.cps, c = r % sh.cps;
+  const uint32_t t0 = c * sh.tc, tcc = min(sh.tc, sh.T - t0), D = sh.D, n = tcc * D;
+  const uint32_t n_max = sh.tc * D;
+  const uint16_t* g = src + (uint64_t(slice) * sh.T + t0) * D;
+
+  crc_tables_init(S.crc_t);
+  for (uint32_t i = tid; i < 512; i += nthr) (&S.hist[0][0])[i] = 0;
+  if ((reinterpret_cast<uintptr_t>(g) & 15u) == 0 && (n & 7u) == 0) {
+    const uint4* g4 = reinterpret_cast<const uint4*>(g);
+    uint4* v4 = reinterpret_cast<uint4*>(vals);
+    for (uint32_t q = tid; q < n / 8u; q += nthr) v4[q] = __ldg(g4 + q);
+  } else {
+    for (uint32_t i = tid; i < n; i += nthr) vals[i] = g[i];
+  }
+  __syncthreads();
+  for (uint32_t i = tid; i < n; i += nthr) {
+    uint32_t v = vals[i];
+    atomicAdd(&S.hist[0][v & 0xffu], 1u);
+    atomicAdd(&S.hist[1][v >> 8], 1u);
+  }
+  __syncthreads();
+  for (uint32_t p = 0; p < 2; ++p) {
+    uint32_t k = block_normalize(S.hist[p], n, S.freq[p], S.rem, S.tmp);
+    if (tid == 0) S.k[p] = k;
+    block_enc_tables(S.freq[p], S.fc[p], S.rcp[p], S.tmp);
+  }
+
+  const ChanMajor cm(tcc);
+  const uint32_t N = rans_lanes(n), G = rans_groups(N);
+  uint8_t* slot = ws.slots + uint64_t(r) * ws.slot_bytes;
+  const uint32_t rec_area = 2u * (16u + pad16(n_max));
+  uint16_t* scratch[2] = {reinterpret_cast<uint16_t*>(slot + rec_area),
+                          reinterpret_cast<uint16_t*>(slot + rec_area + 2u * n_max + 64u)};
+  {
+    const uint32_t warp = tid >> 5, lane = tid & 31u;
+    const uint32_t p = warp >> 2, gg = warp & 3u;
+    if (S.k[p] >= 2 && gg < G) {
+      uint32_t b0, len0, b1 = n, len1;
+      lane_range(n, N, gg * kGroupLanes, b0, len0);
+      if (gg + 1 < G) lane_range(n, N, (gg + 1) * kGroupLanes, b1, len1);
+      auto sym = [&](uint32_t i) -> uint32_t {
+        uint32_t d, t;
+        cm.split(i, d, t);
+        uint32_t v = vals[t * D + d];
+        return p ? (v >> 8) : (v & 0xffu);
+      };
+      uint32_t x;
+      uint32_t Wg = rans_encode_group(sym, n, N, gg, S.fc[p], S.rcp[p], scratch[p] + b0, b1 - b0, &x);
+      uint32_t l = gg * kGroupLanes + lane;
+      if (l < N) S.states[p][l] = x;
+      if (lane == 0) {
+        S.W[p][gg] = Wg;
+        S.wbeg[p][gg] = b0 + (b1 - b0) - Wg;
+      }
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    for (uint32_t p = 0; p < 2; ++p) {
+      uint32_t k = S.k[p], raw_b = 16u + pad16(n);
+      uint32_t v0 = vals[0];
+      S.csym[p] = p ? (v0 >> 8) : (v0 & 0xffu);
+      if (k == 1) { S.mode[p] = kModeConst; S.bytes[p] = 16; }
+      else if (k >= 2) {
+        uint32_t rb = rans_layout(n, k, S.W[p], S.sub_len[p]);
+        if (rb < raw_b) { S.mode[p] = kModeRans; S.bytes[p] = rb; }
+        else { S.mode[p] = kModeRaw; S.bytes[p] = raw_b; }
+      } else { S.mode[p] = kModeRaw; S.bytes[p] = raw_b; }
+    }
+  }
+  __syncthreads();
+  uint8_t* rec = slot;
+  uint32_t off = 0;
+  for (uint32_t p = 0; p < 2; ++p) {
+    auto raw = [&](uint32_t i) -> uint32_t {
+      uint32_t d, t;
+      cm.split(i, d, t);
+      uint32_t v = vals[t * D + d];
+      return p ? (v >> 8) : (v & 0xffu);
+    };
+    block_write_stream(rec + off, S.mode[p], n, S.bytes[p], S.csym[p], S.k[p], S.freq[p],
+                       S.states[p], scratch[p], S.wbeg[p], S.W[p], S.sub_len[p], raw, S.tmp);
+    off += S.bytes[p];
+  }
+  __syncthreads();
+  uint32_t crc = crc32_block_aligned(rec, off, S.crc_t, S.red);
+  if (tid == 0) {
+    ws.rec_len[r] = off;
+    ws.rec_crc[r] = crc;
+  }
+}
+
+__global__ void __launch_bounds__(kThreads)
+k_lossless_decode(LosslessShape sh, const uint8_t* __restrict__ src, uint16_t* __restrict__ dst,
+                  DecodeState* ds) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  DecSmem& S = *reinterpret_cast<DecSmem*>(smem_raw);
+  const uint32_t tid = threadIdx.x, nthr = blockDim.x;
+  const uint32_t D = sh.D, n_max = sh.tc * D;
+  uint8_t* planes[2] = {smem_raw + sizeof(DecSmem), smem_raw + sizeof(DecSmem) + pad16(n_max)};
+  if (ds->status != kOk) return;
+  const uint32_t nrec = ds->n_records;
+  crc_tables_init(S.crc_t);
+  for (uint32_t r = blockIdx.x; r < nrec; r += gridDim.x) {
+    __syncthreads();
+    const uint8_t* e = src + kHeaderBytes + uint64_t(kIndexEntry) * r;
+    const uint64_t off = ld_u64(e);
+    const uint32_t len = ld_u32(e + 8), want = ld_u32(e + 12);
+    const uint8_t* rec = src + off;
+    const uint32_t slice = r / sh.cps, c = r % sh.cps;
+    const uint32_t t0 = c * sh.tc, tcc = min(sh.tc, sh.T - t0), n = tcc * D;
+    uint32_t got = crc32_block_aligned(rec, len, S.crc_t, S.red);
+    if (tid == 0) S.crc_ok = (got == want);
+    __syncthreads();
+    int st = S.crc_ok ? kOk : kErrCorrupt;
+    if (st == kOk) st = block_parse_stream(rec, len, n, &S.si[0], S.freq[0], S.tmp);
+    uint32_t b0 = 0;
+    if (st == kOk) {
+      b0 = S.si[0].bytes;
+      st = block_parse_stream(rec + b0, len - b0, n, &S.si[1], S.freq[1], S.tmp);
+      if (st == kOk && b0 + S.si[1].bytes != len) st = kErrCorrupt;
+    }
+    if (st != kOk) {
+      if (tid == 0) atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(st));
+      continue;
+    }
+    const uint8_t* recp[2] = {rec, rec + b0};
+    for (uint32_t p = 0; p < 2; ++p) {
+      const uint32_t mode = S.si[p].mode;
+      if (mode == kModeRans) {
+        block_dec_lut(S.freq[p], S.cum[p], S.lut[p], S.tmp);
+      } else if (mode == kModeRaw) {
+        const uint4* s4 = reinterpret_cast<const uint4*>(recp[p] + 16);
+        uint4* d4 = reinterpret_cast<uint4*>(planes[p]);
+        for (uint32_t q = tid; q < n / 16u; q += nthr) d4[q] = s4[q];
+        for (uint32_t i = (n & ~15u) + tid; i < n; i += nthr) planes[p][i] = recp[p][16 + i];
+      } else {
+        const uint8_t v = uint8_t(S.si[p].sym);
+        for (uint32_t i = tid; i < n; i += nthr) planes[p][i] = v;
+      }
+    }
+    __syncthreads();
+    bool ok = true;
+    {
+      const uint32_t warp = tid >> 5, p = warp >> 2, gg = warp & 3u;
+      const uint32_t N = rans_lanes(n), G = rans_groups(N);
+      if (S.si[p].mode == kModeRans && gg < G) {
+        uint8_t* pl = planes[p];
+        ok = rans_decode_group(recp[p] + S.si[p].sub_off[gg], S.si[p].sub_len[gg], n, N, gg,
+                               S.lut[p], [&](uint32_t i, uint32_t s) { pl[i] = uint8_t(s); });
+      }
+    }
+    if (!__syncthreads_and(ok)) {
+      if (tid == 0)
+        atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(kErrCorrupt));
+      continue;
+    }
+    uint16_t* out = dst + (uint64_t(slice) * sh.T + t0) * D;
+    if ((D & 7u) == 0 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0) {
+      const uint32_t per_row = D / 8u;
+      for (uint32_t q = tid; q < tcc * per_row; q += nthr) {
+        uint32_t t = q / per_row, d0 = (q - t * per_row) * 8u;
+        uint32_t w[4];
+        for (uint32_t e2 = 0; e2 < 4; ++e2) {
+          uint32_t i0 = (d0 + 2 * e2) * tcc + t, i1 = i0 + tcc;
+          uint32_t v0 = planes[0][i0] | (uint32_t(planes[1][i0]) << 8);
+          uint32_t v1 = planes[0][i1] | (uint32_t(planes[1][i1]) << 8);
+          w[e2] = v0 | (v1 << 16);
+        }
+        reinterpret_cast<uint4*>(out)[q] = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    } else {
+      for (uint32_t q = tid; q < n; q += nthr) {
+        uint32_t t = q / D, d = q - t * D;
+        uint32_t i = d * tcc + t;
+        out[q] = uint16_t(planes[0][i] | (uint32_t(planes[1][i]) << 8));
+      }
+    }
+  }
+}
+
+int g_num_sms = 0;
+int num_sms() {
+  if (!g_num_sms) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&g_num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (g_num_sms <= 0) g_num_sms = 148;
+  }
+  return g_num_sms;
+}
+
+}  // namespace
+
+uint64_t lossless_slot_bytes(const LosslessShape& s) {
+  const uint64_t n_max = uint64_t(s.tc) * s.D;
+  uint64_t b = 2u * (16u + pad16_64(n_max)) + 2u * (2u * n_max + 64u);
+  return (b + 255u) & ~uint64_t(255);
+}
+
+cudaError_t launch_lossless_encode(const LosslessShape& s, const uint16_t* src, uint32_t n_slices,
+                                   const EncodeLayout& ws, cudaStream_t st) {
+  const uint32_t nrec = n_slices * s.cps;
+  if (nrec == 0) return cudaSuccess;
+  size_t smem = sizeof(EncSmem) + pad16(s.tc * s.D * 2u);
+  cudaError_t e = cudaFuncSetAttribute(k_lossless_encode, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem));
+  if (e != cudaSuccess) return e;
+  {
+    ProfRange pr_("lossless_encode", st);
+    k_lossless_encode<<<nrec, kThreads, smem, st>>>(s, src, ws);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_lossless_decode(const LosslessShape& s, const uint8_t* src, uint16_t* dst,
+                                   DecodeState* ds, uint32_t max_records, cudaStream_t st) {
+  if (max_records == 0) return cudaSuccess;
+  size_t smem = sizeof(DecSmem) + 2u * pad16(s.tc * s.D);
+  cudaError_t e = cudaFuncSetAttribute(k_lossless_decode, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem));
+  if (e != cudaSuccess) return e;
+  uint32_t grid = min(max_records, uint32_t(num_sms()));
+  {
+    ProfRange pr_("lossless_decode", st);
+    k_lossless_decode<<<grid, kThreads, smem, st>>>(s, src, dst, ds);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace kvc
