@@ -364,7 +364,7 @@ int decode_common(const kvc_plan_t* plan, int path, const void* d_src, size_t sr
   if (!d_src || !d_ws || !d_res || (dst_cap && !d_dst)) return KVC_ERR_INVALID;
   if (!aligned16(d_src) || !aligned16(d_dst) || !aligned16(d_ws) || !aligned16(d_res))
     return KVC_ERR_INVALID;
-  if (ws_bytes < sizeof(DecodeState)) return KVC_ERR_CAPACITY;
+  if (ws_bytes < kvc_workspace_bytes(plan, path, 1, 0)) return KVC_ERR_CAPACITY;
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev != plan->device) return KVC_ERR_INVALID;
@@ -420,7 +420,8 @@ extern "C" size_t kvc_max_encoded_bytes(const kvc_plan_t* plan, int path, uint32
 
 extern "C" size_t kvc_workspace_bytes(const kvc_plan_t* plan, int path, int decode, uint32_t n_slices) {
   if (!path_ok(plan, path)) return 0;
-  if (decode) return size_t(pad256u(sizeof(DecodeState)));
+  if (decode)
+    return size_t(kDecodeStateBytes + pad256u(4ull * plan->S * records_per_slice(plan, path)));
   return size_t(encode_ws_bytes(plan, path, n_slices));
 }
 

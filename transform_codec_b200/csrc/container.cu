@@ -202,6 +202,7 @@ k_check_container(const uint8_t* src, uint64_t src_bytes, ContainerExpect e, Dec
     ds->n_slices = st == kOk ? ns_s : 0;
     ds->n_records = st == kOk ? nr_s : 0;
     ds->err_key = ~0ull;
+    ds->n_deferred = 0;
     ds->out_bytes = st == kOk ? uint64_t(ns_s) * e.T * e.D * 2u : 0;
     res->status = st;
     res->bytes = 0;

@@ -194,7 +194,9 @@ __device__ inline uint32_t crc32_block_aligned(const uint8_t* p, uint32_t len, c
 }
 
 // CRC-32 of a virtual message of len bytes whose byte i is fetch(i), any
-// length; result valid in thread 0.
+// length; result valid in thread 0. The initial value 0xFFFFFFFF is applied by
+// complementing the first four bytes (the register absorbs exactly the next 32
+// message bits), or for shorter messages by adding 0xFFFFFFFF * x^(8 len).
 template <class Fetch>
 __device__ inline uint32_t crc32_block_bytes(Fetch fetch, uint64_t len, const uint32_t* t,
                                              uint32_t* red) {
@@ -212,13 +214,16 @@ __device__ inline uint32_t crc32_block_bytes(Fetch fetch, uint64_t len, const ui
       int64_t off = run0 + k;
       if (off < 0) continue;
       uint32_t b = fetch(uint64_t(off));
-      if (off < 4) b ^= 0xffu;
+      if (off < 4 && len >= 4) b ^= 0xffu;
       c = crc_byte(t, c, b);
     }
     acc ^= c;
   }
   uint32_t total = crc_block_join(acc, red);
-  return len ? (total ^ 0xffffffffu) : 0u;
+  if (len == 0) return 0u;
+  // under four bytes the initial register is shifted through the message instead
+  if (len < 4) total ^= gf2_mul(0xffffffffu, gf2_xpow8(len));
+  return total ^ 0xffffffffu;
 }
 
 // ---------------------------------------------------------------- block helpers

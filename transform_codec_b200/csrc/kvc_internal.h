@@ -33,7 +33,14 @@ struct DecodeState {
   uint32_t first_slice, n_slices, n_records;
   unsigned long long err_key;  // min over failing records of (record << 8) | status
   uint64_t out_bytes;
+  uint32_t n_deferred;         // records the fast decoder left to the general one
+  uint32_t reserved;
 };
+// the deferred-record list follows the state in the decode workspace
+constexpr uint32_t kDecodeStateBytes = 256;
+inline __host__ __device__ uint32_t* deferred_list(DecodeState* ds) {
+  return reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(ds) + kDecodeStateBytes);
+}
 
 // Encoder workspace header (device), followed by per-record arrays and slots.
 struct EncodeState {

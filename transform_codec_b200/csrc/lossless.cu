@@ -144,6 +144,8 @@ k_lossless_encode(LosslessShape sh, const uint16_t* __restrict__ src, EncodeLayo
   }
 }
 
+// General decoder: any chunk shape and any plane modes; stages both planes in
+// shared memory (one CTA per SM). Runs the records the fast decoder deferred.
 __global__ void __launch_bounds__(kThreads)
 k_lossless_decode(LosslessShape sh, const uint8_t* __restrict__ src, uint16_t* __restrict__ dst,
                   DecodeState* ds) {
@@ -153,10 +155,13 @@ k_lossless_decode(LosslessShape sh, const uint8_t* __restrict__ src, uint16_t* _
   const uint32_t D = sh.D, n_max = sh.tc * D;
   uint8_t* planes[2] = {smem_raw + sizeof(DecSmem), smem_raw + sizeof(DecSmem) + pad16(n_max)};
   if (ds->status != kOk) return;
-  const uint32_t nrec = ds->n_records;
+  const uint32_t n_todo = ds->n_deferred;
+  if (blockIdx.x >= n_todo) return;
+  const uint32_t* todo = deferred_list(ds);
   crc_tables_init(S.crc_t);
-  for (uint32_t r = blockIdx.x; r < nrec; r += gridDim.x) {
+  for (uint32_t i = blockIdx.x; i < n_todo; i += gridDim.x) {
     __syncthreads();
+    const uint32_t r = todo[i];
     const uint8_t* e = src + kHeaderBytes + uint64_t(kIndexEntry) * r;
     const uint64_t off = ld_u64(e);
     const uint32_t len = ld_u32(e + 8), want = ld_u32(e + 12);
@@ -233,6 +238,175 @@ k_lossless_decode(LosslessShape sh, const uint8_t* __restrict__ src, uint16_t* _
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Fast decoder for full chunks (D * tc = 65536 values, tc a multiple of 512):
+// then every stream has 128 lanes of 512 symbols and lane l's symbol tau sits at
+// channel-major index l * 512 + tau in both planes, i.e. channel l / lpc, token
+// (l % lpc) * 512 + tau with lpc = tc / 512. Thread l owns lane l of both planes
+// (warp w = rANS group w), decodes token-synchronously, merges the other
+// plane's raw bytes from registers and writes 32-token tiles of token-major
+// rows through shared memory. Records with two rANS planes or other shapes are
+// deferred to the general decoder.
+constexpr uint32_t kFastThreads = 128;
+
+struct __align__(16) FastSmem {
+  uint32_t crc_t[1024];
+  uint32_t lut[kProbScale];
+  uint16_t tile[32 * 128];
+  uint32_t freq[2][256];
+  uint32_t cum[260];
+  uint32_t tmp[32], red[32];
+  StreamInfo si[2];
+  uint32_t crc_ok;
+};
+
+struct LaneRans {
+  uint32_t x, pos, W;
+  const uint16_t* w16;
+  bool bad;
+  __device__ inline uint32_t step(const uint32_t* lut, uint32_t lt) {
+    const uint32_t e = lut[x & (kProbScale - 1u)];
+    x = ((e >> 8) & 0xfffu) * (x >> kProbBits) + (e >> 20);
+    const bool need = x < kRansLow;
+    const uint32_t mask = __ballot_sync(0xffffffffu, need);
+    if (need) {
+      const uint32_t idx = pos + __popc(mask & lt);
+      if (idx < W) x = (x << 16) | w16[idx];
+      else bad = true;
+    }
+    pos += __popc(mask);
+    return e & 0xffu;
+  }
+};
+
+template <uint32_t M0, uint32_t M1>
+__device__ inline bool fast_tiles(FastSmem& S, const uint8_t* const recp[2], uint16_t* out,
+                                  uint32_t D, uint32_t lpc_log2) {
+  const uint32_t l = threadIdx.x, lane = l & 31u, g = l >> 5;
+  const uint32_t lt = lanemask_lt();
+  const uint32_t lpc = 1u << lpc_log2;
+  const uint32_t tbase = (l & (lpc - 1u)) * 32u * D + (l >> lpc_log2);
+  LaneRans rs{kRansLow, 0, 0, nullptr, false};
+  const uint8_t* raw0 = recp[0] + 16 + l * 512u;
+  const uint8_t* raw1 = recp[1] + 16 + l * 512u;
+  const uint32_t c0 = S.si[0].sym, c1 = S.si[1].sym;
+  constexpr uint32_t RP = (M0 == kModeRans) ? 0u : 1u;  // the rANS plane, if any
+  if (M0 == kModeRans || M1 == kModeRans) {
+    const StreamInfo& si = S.si[RP];
+    const uint8_t* sub = recp[RP] + si.sub_off[g];
+    const uint32_t sl = si.sub_len[g];
+    if (sl < 128u || (sl & 1u)) rs.bad = true;
+    else {
+      rs.x = reinterpret_cast<const uint32_t*>(sub)[lane];
+      rs.W = (sl - 128u) >> 1;
+      rs.w16 = reinterpret_cast<const uint16_t*>(sub + 128);
+    }
+  }
+  const bool live = __all_sync(0xffffffffu, !rs.bad);
+  for (uint32_t k = 0; k < 16; ++k) {
+    uint32_t r0[8], r1[8];
+    if (M0 == kModeRaw) {
+      const uint4 a = *reinterpret_cast<const uint4*>(raw0 + 32u * k);
+      const uint4 b = *reinterpret_cast<const uint4*>(raw0 + 32u * k + 16u);
+      r0[0] = a.x; r0[1] = a.y; r0[2] = a.z; r0[3] = a.w;
+      r0[4] = b.x; r0[5] = b.y; r0[6] = b.z; r0[7] = b.w;
+    }
+    if (M1 == kModeRaw) {
+      const uint4 a = *reinterpret_cast<const uint4*>(raw1 + 32u * k);
+      const uint4 b = *reinterpret_cast<const uint4*>(raw1 + 32u * k + 16u);
+      r1[0] = a.x; r1[1] = a.y; r1[2] = a.z; r1[3] = a.w;
+      r1[4] = b.x; r1[5] = b.y; r1[6] = b.z; r1[7] = b.w;
+    }
+#pragma unroll
+    for (uint32_t j = 0; j < 32; ++j) {
+      uint32_t lo, hi;
+      if (M0 == kModeRaw) lo = (r0[j >> 2] >> (8u * (j & 3u))) & 0xffu;
+      else if (M0 == kModeConst) lo = c0;
+      else lo = live ? rs.step(S.lut, lt) : 0u;
+      if (M1 == kModeRaw) hi = (r1[j >> 2] >> (8u * (j & 3u))) & 0xffu;
+      else if (M1 == kModeConst) hi = c1;
+      else hi = live ? rs.step(S.lut, lt) : 0u;
+      S.tile[tbase + j * D] = uint16_t(lo | (hi << 8));
+    }
+    __syncthreads();
+    // tile = lpc blocks of 32 token rows x D channels, each contiguous in the output
+    const uint32_t per_block = 4u * D;  // uint4 per block
+    for (uint32_t q = l; q < 512u; q += kFastThreads) {
+      const uint32_t s = q / per_block, w = q - s * per_block;
+      uint4* o = reinterpret_cast<uint4*>(out + (uint64_t(s) * 512u + 32u * k) * D);
+      o[w] = reinterpret_cast<const uint4*>(S.tile)[q];
+    }
+    __syncthreads();
+  }
+  bool ok = !rs.bad;
+  if (M0 == kModeRans || M1 == kModeRans) ok = ok && live && rs.pos == rs.W && rs.x == kRansLow;
+  return ok;
+}
+
+__global__ void __launch_bounds__(kFastThreads)
+k_lossless_decode_fast(LosslessShape sh, const uint8_t* __restrict__ src, uint16_t* __restrict__ dst,
+                       DecodeState* ds) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  FastSmem& S = *reinterpret_cast<FastSmem*>(smem_raw);
+  const uint32_t tid = threadIdx.x;
+  if (ds->status != kOk) return;
+  const uint32_t nrec = ds->n_records;
+  const uint32_t D = sh.D;
+  const bool shape_ok = (D * sh.tc == kMaxChunkValues) && (sh.tc % 512u == 0);
+  const uint32_t lpc_log2 = shape_ok ? uint32_t(ilog2_u32(sh.tc / 512u)) : 0u;
+  crc_tables_init(S.crc_t);
+  for (uint32_t r = blockIdx.x; r < nrec; r += gridDim.x) {
+    __syncthreads();
+    const uint32_t slice = r / sh.cps, c = r % sh.cps;
+    const uint32_t t0 = c * sh.tc, tcc = min(sh.tc, sh.T - t0);
+    bool defer = !shape_ok || tcc != sh.tc;
+    const uint8_t* e = src + kHeaderBytes + uint64_t(kIndexEntry) * r;
+    const uint64_t off = ld_u64(e);
+    const uint32_t len = ld_u32(e + 8), want = ld_u32(e + 12);
+    const uint8_t* rec = src + off;
+    int st = kOk;
+    if (!defer) {
+      uint32_t got = crc32_block_aligned(rec, len, S.crc_t, S.red);
+      if (tid == 0) S.crc_ok = (got == want);
+      __syncthreads();
+      st = S.crc_ok ? kOk : kErrCorrupt;
+      const uint32_t n = kMaxChunkValues;
+      if (st == kOk) st = block_parse_stream(rec, len, n, &S.si[0], S.freq[0], S.tmp);
+      if (st == kOk) {
+        const uint32_t b0 = S.si[0].bytes;
+        st = block_parse_stream(rec + b0, len - b0, n, &S.si[1], S.freq[1], S.tmp);
+        if (st == kOk && b0 + S.si[1].bytes != len) st = kErrCorrupt;
+      }
+      if (st == kOk && S.si[0].mode == kModeRans && S.si[1].mode == kModeRans) defer = true;
+    }
+    if (defer) {
+      if (tid == 0) deferred_list(ds)[atomicAdd(&ds->n_deferred, 1u)] = r;
+      continue;
+    }
+    if (st != kOk) {
+      if (tid == 0) atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(st));
+      continue;
+    }
+    const uint32_t m0 = S.si[0].mode, m1 = S.si[1].mode;
+    if (m0 == kModeRans) block_dec_lut(S.freq[0], S.cum, S.lut, S.tmp);
+    else if (m1 == kModeRans) block_dec_lut(S.freq[1], S.cum, S.lut, S.tmp);
+    const uint8_t* recp[2] = {rec, rec + S.si[0].bytes};
+    uint16_t* out = dst + (uint64_t(slice) * sh.T + t0) * D;
+    bool ok;
+    if (m0 == kModeRaw && m1 == kModeRans) ok = fast_tiles<kModeRaw, kModeRans>(S, recp, out, D, lpc_log2);
+    else if (m0 == kModeRaw && m1 == kModeRaw) ok = fast_tiles<kModeRaw, kModeRaw>(S, recp, out, D, lpc_log2);
+    else if (m0 == kModeRaw && m1 == kModeConst) ok = fast_tiles<kModeRaw, kModeConst>(S, recp, out, D, lpc_log2);
+    else if (m0 == kModeRans && m1 == kModeRaw) ok = fast_tiles<kModeRans, kModeRaw>(S, recp, out, D, lpc_log2);
+    else if (m0 == kModeRans && m1 == kModeConst) ok = fast_tiles<kModeRans, kModeConst>(S, recp, out, D, lpc_log2);
+    else if (m0 == kModeConst && m1 == kModeRans) ok = fast_tiles<kModeConst, kModeRans>(S, recp, out, D, lpc_log2);
+    else if (m0 == kModeConst && m1 == kModeRaw) ok = fast_tiles<kModeConst, kModeRaw>(S, recp, out, D, lpc_log2);
+    else ok = fast_tiles<kModeConst, kModeConst>(S, recp, out, D, lpc_log2);
+    if (!__syncthreads_and(ok) && tid == 0)
+      atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(kErrCorrupt));
+  }
+}
+
 int g_num_sms = 0;
 int num_sms() {
   if (!g_num_sms) {
@@ -270,13 +444,29 @@ cudaError_t launch_lossless_encode(const LosslessShape& s, const uint16_t* src, 
 cudaError_t launch_lossless_decode(const LosslessShape& s, const uint8_t* src, uint16_t* dst,
                                    DecodeState* ds, uint32_t max_records, cudaStream_t st) {
   if (max_records == 0) return cudaSuccess;
-  size_t smem = sizeof(DecSmem) + 2u * pad16(s.tc * s.D);
-  cudaError_t e = cudaFuncSetAttribute(k_lossless_decode, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(smem));
+  static int fast_blocks_per_sm = 0;
+  const size_t fsmem = sizeof(FastSmem);
+  cudaError_t e = cudaFuncSetAttribute(k_lossless_decode_fast,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(fsmem));
   if (e != cudaSuccess) return e;
-  uint32_t grid = min(max_records, uint32_t(num_sms()));
+  if (!fast_blocks_per_sm) {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fast_blocks_per_sm, k_lossless_decode_fast,
+                                                      kFastThreads, fsmem);
+    if (e != cudaSuccess || fast_blocks_per_sm < 1) fast_blocks_per_sm = 1;
+  }
   {
     ProfRange pr_("lossless_decode", st);
+    uint32_t grid = min(max_records, uint32_t(num_sms() * fast_blocks_per_sm));
+    k_lossless_decode_fast<<<grid, kFastThreads, fsmem, st>>>(s, src, dst, ds);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem = sizeof(DecSmem) + 2u * pad16(s.tc * s.D);
+  e = cudaFuncSetAttribute(k_lossless_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  {
+    ProfRange pr_("lossless_decode_general", st);
+    uint32_t grid = min(max_records, uint32_t(num_sms()));
     k_lossless_decode<<<grid, kThreads, smem, st>>>(s, src, dst, ds);
   }
   return cudaGetLastError();
