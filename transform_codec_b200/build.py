@@ -12,7 +12,7 @@ BUILD = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libkvc.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
 SOURCES = ["api.cpp", "container.cu", "lossless.cu", "transform.cu"]
-HEADERS = ["kvc_device.cuh", "kvc_internal.h"]
+HEADERS = ["kvc_device.cuh", "kvc_internal.h", "tcgen05.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

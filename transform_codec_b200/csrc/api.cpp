@@ -74,6 +74,7 @@ struct kvc_plan_s {
   float* d_bases = nullptr;
   uint8_t* d_widths = nullptr;
   float* d_rope = nullptr;
+  uint8_t* d_qsplit = nullptr;
 };
 
 namespace {
@@ -175,11 +176,54 @@ bool bases_orthonormal(const float* bases, uint32_t S, uint32_t D, double tol) {
   return ok;
 }
 
+uint16_t bf16_rne(float f) {
+  uint32_t x;
+  std::memcpy(&x, &f, 4);
+  if ((x & 0x7fffffffu) > 0x7f800000u) return uint16_t((x >> 16) | 0x40u);
+  uint32_t upper = x >> 16, lower = x & 0xffffu;
+  if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) ++upper;
+  return uint16_t(upper);
+}
+
+// Byte offset of element (row, kbyte) in a K-major operand of `rows` rows stored
+// in 128-byte-swizzled atoms (the tensor cores' layout: 16-byte chunk c of row r
+// sits at chunk c ^ (r mod 8)), K split into 128-byte blocks rows*128 bytes apart.
+uint32_t sw128_offset_host(uint32_t row, uint32_t kbyte, uint32_t rows) {
+  const uint32_t kb = kbyte >> 7, in = kbyte & 127u;
+  const uint32_t chunk = (in >> 4) ^ (row & 7u);
+  return kb * rows * 128u + row * 128u + (chunk << 4) + (in & 15u);
+}
+
+// Per slice, Q as two bf16 pieces (hi = rne(Q), lo = rne(Q - hi)) laid out as the
+// B operand of D[token][k] = sum_j y[token][j] * Q[k][j]: row k, K index j.
+void split_bases(const float* bases, uint32_t S, std::vector<uint8_t>& out) {
+  const uint32_t D = 128;
+  out.assign(size_t(S) * kQSplitBytes, 0);
+  for (uint32_t s = 0; s < S; ++s) {
+    uint8_t* hi = out.data() + size_t(s) * kQSplitBytes;
+    uint8_t* lo = hi + kQSplitBytes / 2;
+    const float* Q = bases + size_t(s) * D * D;
+    for (uint32_t k = 0; k < D; ++k)
+      for (uint32_t j = 0; j < D; ++j) {
+        const float q = Q[size_t(k) * D + j];
+        const uint16_t h = bf16_rne(q);
+        uint32_t hb = uint32_t(h) << 16;
+        float hf;
+        std::memcpy(&hf, &hb, 4);
+        const uint16_t l = bf16_rne(q - hf);
+        const uint32_t off = sw128_offset_host(k, 2 * j, D);
+        std::memcpy(hi + off, &h, 2);
+        std::memcpy(lo + off, &l, 2);
+      }
+  }
+}
+
 void free_plan(kvc_plan_s* p) {
   if (!p) return;
   if (p->d_bases) cudaFree(p->d_bases);
   if (p->d_widths) cudaFree(p->d_widths);
   if (p->d_rope) cudaFree(p->d_rope);
+  if (p->d_qsplit) cudaFree(p->d_qsplit);
   delete p;
 }
 
@@ -248,6 +292,8 @@ extern "C" int kvc_plan_create(const kvc_plan_desc* desc, kvc_plan_t** out) {
     p->plan_crc = compute_plan_crc(d, p->widths, p->S);
     std::vector<float> cs;
     rope_table(d.n_tokens, d.head_dim, d.rope_theta, cs);
+    std::vector<uint8_t> qs;
+    split_bases(d.bases, p->S, qs);
     const size_t nb = size_t(p->S) * d.head_dim * d.head_dim * sizeof(float);
     bool ok = cudaMalloc(&p->d_bases, nb) == cudaSuccess &&
               cudaMalloc(&p->d_widths, p->widths.size()) == cudaSuccess &&
@@ -256,7 +302,9 @@ extern "C" int kvc_plan_create(const kvc_plan_desc* desc, kvc_plan_t** out) {
               cudaMemcpy(p->d_widths, p->widths.data(), p->widths.size(), cudaMemcpyHostToDevice) ==
                   cudaSuccess &&
               cudaMemcpy(p->d_rope, cs.data(), cs.size() * sizeof(float), cudaMemcpyHostToDevice) ==
-                  cudaSuccess;
+                  cudaSuccess &&
+              cudaMalloc(&p->d_qsplit, qs.size()) == cudaSuccess &&
+              cudaMemcpy(p->d_qsplit, qs.data(), qs.size(), cudaMemcpyHostToDevice) == cudaSuccess;
     if (!ok) {
       free_plan(p);
       return KVC_ERR_CUDA;
@@ -349,7 +397,7 @@ int encode_common(const kvc_plan_t* plan, int path, uint32_t first_slice, uint32
     h.n_sink = plan->d.n_sink;
     h.n_recent = plan->d.n_recent;
     h.block_tokens = plan->d.block_tokens;
-    TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope};
+    TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope, plan->d_qsplit};
     e = launch_transform_encode(plan->ts, pd, src, first_slice, n_slices, L, stream);
   }
   if (e != cudaSuccess) return KVC_ERR_CUDA;
@@ -394,7 +442,7 @@ int decode_common(const kvc_plan_t* plan, int path, const void* d_src, size_t sr
   if (path == KVC_PATH_LOSSLESS) {
     e = launch_lossless_decode(plan->ls, src, dst, ds, max_rec, stream);
   } else {
-    TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope};
+    TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope, plan->d_qsplit};
     e = launch_transform_decode(plan->ts, pd, src, dst, ds, max_rec, stream);
   }
   if (e != cudaSuccess) return KVC_ERR_CUDA;

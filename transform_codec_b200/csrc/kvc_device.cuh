@@ -265,37 +265,56 @@ __device__ inline uint32_t block_sum(uint32_t v, uint32_t* tmp) {
 
 // ---------------------------------------------------------------- frequency tables
 // Largest-remainder normalisation of a 256-bin histogram of n symbols to a
-// total of 4096 (needs blockDim.x >= 256): f_s = 1 + floor(c_s (4096 - k) / n),
+// total of 4096 (any power-of-two block of 64..1024 threads): f_s = 1 + floor(c_s (4096 - k) / n),
 // the 4096 - sum f_s symbols with the largest remainders c_s (4096 - k) mod n
 // (ties: smaller symbol) get one more. freq and rem are 256-word shared arrays.
 // Returns k, the number of present symbols (block-uniform).
 __device__ inline uint32_t block_normalize(const uint32_t* hist, uint32_t n, uint32_t* freq,
                                            uint32_t* rem, uint32_t* tmp) {
-  const uint32_t s = threadIdx.x;
-  const uint32_t c = s < 256 ? hist[s] : 0u;
-  const uint32_t k = __syncthreads_count(c > 0);
-  uint32_t f = 0, r = 0;
-  if (k >= 2 && c) {
-    uint32_t q = c * (kProbScale - k);  // < 2^28
-    f = 1u + q / n;
-    r = q % n;
-  }
-  if (s < 256) rem[s] = r;
-  uint32_t sum = block_sum(f, tmp);  // synchronises
-  if (k >= 2) {
-    uint32_t d = kProbScale - sum;
-    if (c && d) {
-      uint32_t rank = 0;
-      for (uint32_t s2 = 0; s2 < 256; ++s2) {
-        uint32_t r2 = rem[s2];
-        rank += (hist[s2] != 0u) & ((r2 > r) | ((r2 == r) & (s2 < s)));
-      }
-      if (rank < d) ++f;
+  // thread owns symbols [s0, s0 + per); blockDim.x is a power of two <= 1024
+  const uint32_t per = blockDim.x >= 256 ? 1u : 256u / blockDim.x;
+  const uint32_t s0 = threadIdx.x * per;
+  uint32_t present = 0;
+  for (uint32_t i = 0; i < per; ++i) present += (s0 + i < 256 && hist[s0 + i]) ? 1u : 0u;
+  const uint32_t k = block_sum(present, tmp);
+  uint32_t fsum = 0;
+  for (uint32_t i = 0; i < per; ++i) {
+    const uint32_t s = s0 + i;
+    if (s >= 256) break;
+    const uint32_t c = hist[s];
+    uint32_t f = 0, r = 0;
+    if (k >= 2 && c) {
+      const uint32_t q = c * (kProbScale - k);  // < 2^28
+      f = 1u + q / n;
+      r = q % n;
+    } else if (k == 1 && c) {
+      f = kProbScale;
     }
-  } else if (k == 1) {
-    f = c ? kProbScale : 0u;
+    rem[s] = r;
+    freq[s] = f;
+    fsum += f;
   }
-  if (s < 256) freq[s] = f;
+  const uint32_t sum = block_sum(fsum, tmp);  // synchronises: rem and freq complete
+  if (k >= 2) {
+    const uint32_t d = kProbScale - sum;
+    uint32_t add[4] = {0, 0, 0, 0};
+    if (d) {
+      for (uint32_t i = 0; i < per; ++i) {
+        const uint32_t s = s0 + i;
+        if (s >= 256 || !hist[s]) continue;
+        const uint32_t r = rem[s];
+        uint32_t rank = 0;
+        for (uint32_t s2 = 0; s2 < 256; ++s2) {
+          const uint32_t r2 = rem[s2];
+          rank += (hist[s2] != 0u) & ((r2 > r) | ((r2 == r) & (s2 < s)));
+        }
+        add[i] = rank < d ? 1u : 0u;
+      }
+    }
+    __syncthreads();
+    for (uint32_t i = 0; i < per; ++i)
+      if (s0 + i < 256) freq[s0 + i] += add[i];
+  }
   __syncthreads();
   return k;
 }
@@ -303,12 +322,18 @@ __device__ inline uint32_t block_normalize(const uint32_t* hist, uint32_t n, uin
 // From freq[256] (sum 4096): fc[s] = f | cum << 16 and rcp[s] = floor((2^32-1)/f).
 __device__ inline void block_enc_tables(const uint32_t* freq, uint32_t* fc, uint32_t* rcp,
                                         uint32_t* tmp) {
-  const uint32_t s = threadIdx.x;
-  uint32_t f = s < 256 ? freq[s] : 0u;
-  uint32_t cum = block_exclusive_scan(f, tmp, nullptr);
-  if (s < 256) {
+  const uint32_t per = blockDim.x >= 256 ? 1u : 256u / blockDim.x;
+  const uint32_t s0 = threadIdx.x * per;
+  uint32_t mine = 0;
+  for (uint32_t i = 0; i < per; ++i) mine += s0 + i < 256 ? freq[s0 + i] : 0u;
+  uint32_t cum = block_exclusive_scan(mine, tmp, nullptr);
+  for (uint32_t i = 0; i < per; ++i) {
+    const uint32_t s = s0 + i;
+    if (s >= 256) break;
+    const uint32_t f = freq[s];
     fc[s] = f | (cum << 16);
     rcp[s] = f ? 0xffffffffu / f : 0u;
+    cum += f;
   }
   __syncthreads();
 }
@@ -317,11 +342,17 @@ __device__ inline void block_enc_tables(const uint32_t* freq, uint32_t* fc, uint
 // symbols' cumulative starts in cum[257]. freq must be validated (sum 4096).
 __device__ inline void block_dec_lut(const uint32_t* freq, uint32_t* cum, uint32_t* lut,
                                      uint32_t* tmp) {
-  const uint32_t s = threadIdx.x;
-  uint32_t f = s < 256 ? freq[s] : 0u;
-  uint32_t c = block_exclusive_scan(f, tmp, nullptr);
-  if (s < 256) cum[s] = c;
-  if (s == 0) cum[256] = kProbScale;
+  const uint32_t per = blockDim.x >= 256 ? 1u : 256u / blockDim.x;
+  const uint32_t s0 = threadIdx.x * per;
+  uint32_t mine = 0;
+  for (uint32_t i = 0; i < per; ++i) mine += s0 + i < 256 ? freq[s0 + i] : 0u;
+  uint32_t c = block_exclusive_scan(mine, tmp, nullptr);
+  for (uint32_t i = 0; i < per; ++i) {
+    if (s0 + i >= 256) break;
+    cum[s0 + i] = c;
+    c += freq[s0 + i];
+  }
+  if (threadIdx.x == 0) cum[256] = kProbScale;
   __syncthreads();
   for (uint32_t slot = threadIdx.x; slot < kProbScale; slot += blockDim.x) {
     uint32_t lo = 0, hi = 255;  // largest symbol with cum <= slot
@@ -480,17 +511,32 @@ __device__ inline int block_parse_stream(const uint8_t* rec, uint32_t avail, uin
   int st = si->status;
   if (st != kOk || si->mode != kModeRans) return st;
   // RANS table: presence bitmap + k u16 frequencies
-  const uint32_t s = threadIdx.x;
-  uint32_t present = s < 256 ? (rec[16 + (s >> 3)] >> (s & 7u)) & 1u : 0u;
+  const uint32_t per = blockDim.x >= 256 ? 1u : 256u / blockDim.x;
+  const uint32_t s0 = threadIdx.x * per;
+  uint32_t mine = 0;
+  for (uint32_t i = 0; i < per; ++i) {
+    const uint32_t s = s0 + i;
+    if (s < 256) mine += (rec[16 + (s >> 3)] >> (s & 7u)) & 1u;
+  }
   uint32_t total_present;
-  uint32_t idx = block_exclusive_scan(present, tmp, &total_present);
-  uint32_t f = 0;
-  if (present && total_present == si->k) f = ld_u16(rec + 48 + 2u * idx);
-  uint32_t bad = (total_present != si->k) || (present && f == 0);
-  uint32_t fsum = block_sum(f, tmp);
+  uint32_t idx = block_exclusive_scan(mine, tmp, &total_present);
+  uint32_t bad = total_present != si->k;
+  uint32_t fs = 0;
+  for (uint32_t i = 0; i < per; ++i) {
+    const uint32_t s = s0 + i;
+    if (s >= 256) break;
+    const uint32_t present = (rec[16 + (s >> 3)] >> (s & 7u)) & 1u;
+    uint32_t f = 0;
+    if (present && !bad) {
+      f = ld_u16(rec + 48 + 2u * idx);
+      ++idx;
+      if (f == 0) bad = 1;
+    }
+    fs += f;
+    freq[s] = f;
+  }
+  const uint32_t fsum = block_sum(fs, tmp);
   bad = __syncthreads_or(bad) || fsum != kProbScale;
-  if (s < 256) freq[s] = f;
-  __syncthreads();
   return bad ? kErrCorrupt : kOk;
 }
 
@@ -544,13 +590,21 @@ __device__ inline void block_write_stream(uint8_t* rec, uint32_t mode, uint32_t 
   const uint32_t N = rans_lanes(n), G = rans_groups(N);
   const uint32_t lane = tid & 31u, warp = tid >> 5;
   if (tid == 0) *reinterpret_cast<uint4*>(rec) = make_uint4(kModeRans | (G << 16), bytes, n, k);
-  // bitmap: warp w covers symbols 32w .. 32w+31 (blockDim.x >= 256)
-  uint32_t f = tid < 256 ? freq[tid] : 0u;
-  uint32_t bits = __ballot_sync(0xffffffffu, f != 0u);
-  if (warp < 8 && lane == 0) reinterpret_cast<uint32_t*>(rec + 16)[warp] = bits;
-  uint32_t idx = block_exclusive_scan(f != 0u ? 1u : 0u, tmp, nullptr);
+  // bitmap word w (symbols 32w .. 32w+31) from a ballot of warp w % nwarps
+  for (uint32_t w = warp; w < 8; w += nthr >> 5) {
+    const uint32_t bits = __ballot_sync(0xffffffffu, freq[32 * w + lane] != 0u);
+    if (lane == 0) reinterpret_cast<uint32_t*>(rec + 16)[w] = bits;
+  }
+  const uint32_t per = nthr >= 256 ? 1u : 256u / nthr;
+  const uint32_t s0 = tid * per;
+  uint32_t mine = 0;
+  for (uint32_t i = 0; i < per; ++i) mine += (s0 + i < 256 && freq[s0 + i]) ? 1u : 0u;
+  uint32_t idx = block_exclusive_scan(mine, tmp, nullptr);
   const uint32_t ftab_end = 48u + 2u * k, lens_at = pad16(ftab_end);
-  if (f) st_u16(rec + 48 + 2u * idx, f);
+  for (uint32_t i = 0; i < per; ++i) {
+    const uint32_t s = s0 + i;
+    if (s < 256 && freq[s]) st_u16(rec + 48 + 2u * idx++, freq[s]);
+  }
   if (tid < lens_at - ftab_end) rec[ftab_end + tid] = 0;
   const uint32_t lens_end = lens_at + 4u * G, sub0 = pad16(lens_end);
   if (tid < G) reinterpret_cast<uint32_t*>(rec + lens_at)[tid] = sub_len[tid];

@@ -98,7 +98,9 @@ struct TransformPlanDev {
   const float* bases;      // [S][D][D], Q[k*D + j]
   const uint8_t* widths;   // [S][D]
   const float* rope;       // [T][D/2][2] cos, sin
+  const uint8_t* qsplit;   // [S][hi, lo][128 x 256 B] Q as bf16 pieces, B-operand layout
 };
+constexpr uint32_t kQSplitBytes = 2u * 128u * 256u;  // per slice
 uint64_t transform_slot_bytes(const TransformShape& s);
 cudaError_t launch_transform_encode(const TransformShape& s, const TransformPlanDev& p,
                                     const uint16_t* src, uint32_t first_slice, uint32_t n_slices,

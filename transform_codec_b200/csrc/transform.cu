@@ -13,6 +13,7 @@
 // zero point are fp32 with IEEE division; codes use round-half-even.
 #include "kvc_device.cuh"
 #include "kvc_internal.h"
+#include "tcgen05.cuh"
 
 namespace kvc {
 namespace {
@@ -21,6 +22,8 @@ constexpr uint32_t kThreads = 256;
 constexpr uint32_t kD = 128;        // head_dim handled by these kernels
 constexpr uint32_t kTile = 64;      // tokens per tile = quantiser block
 constexpr uint32_t kMaxCt = 512;    // max tokens per middle chunk
+constexpr uint32_t kTcRows = 128;   // tokens per tensor-core tile (MMA M)
+constexpr uint32_t kTcCols = 128;   // tensor-memory columns: one fp32 128 x 128 accumulator
 
 __device__ inline float bf16_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
 __device__ inline uint32_t f32_to_bf16_rne(float f) {
@@ -271,34 +274,59 @@ k_transform_encode_raw(TransformShape sh, const uint16_t* __restrict__ src, Enco
   }
 }
 
-struct __align__(16) DecSmem {
-  float Qt[kD * kD];           // Qt[j][k] = Q[k][j]
-  float yh[kTile * kD];        // y^ then x^, [token][j or k]
-  uint8_t codes[kD * kMaxCt];  // [j][t]
+// Decoder shared memory. Operand tiles come first so each 128-byte-swizzled
+// tile starts on a 1024-byte boundary.
+struct __align__(1024) DecSmem {
+  uint8_t a_hi[kTcRows * 256];   // y^ as bf16 pieces, A operand [token][component]
+  uint8_t a_lo[kTcRows * 256];
+  uint8_t b_hi[kD * 256];        // Q as bf16 pieces, B operand [channel][component]
+  uint8_t b_lo[kD * 256];
+  uint8_t codes[kD * kMaxCt];    // [j][t]
   float zs[kD][kMaxCt / kTile][2];
   uint32_t crc_t[1024];
   uint32_t freq[256], cum[260], lut[kProbScale];
   uint32_t tmp[32], red[32];
   StreamInfo si;
   CompInfo ci;
+  uint64_t bar;
+  uint32_t tmem_base;
   uint32_t crc_ok, cur_slice, bad;
 };
+
+static_assert(sizeof(DecSmem) + 1024 <= 232448, "decoder shared memory exceeds the per-block limit");
 
 __global__ void __launch_bounds__(kThreads)
 k_transform_decode(TransformShape sh, TransformPlanDev pl, const uint8_t* __restrict__ src,
                    uint16_t* __restrict__ dst, DecodeState* ds) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  DecSmem& S = *reinterpret_cast<DecSmem*>(smem_raw);
+  // the swizzled operand tiles need 1024-byte-aligned shared addresses
+  const uint32_t pad = (1024u - (tc::smem_addr(smem_raw) & 1023u)) & 1023u;
+  DecSmem& S = *reinterpret_cast<DecSmem*>(smem_raw + pad);
   const uint32_t tid = threadIdx.x, nthr = blockDim.x;
+  const uint32_t warp = tid >> 5, lane = tid & 31u;
   if (ds->status != kOk) return;
   const uint32_t nrec = ds->n_records, first = ds->first_slice;
   const uint32_t per = (nrec + gridDim.x - 1) / gridDim.x;
   const uint32_t rbeg = blockIdx.x * per, rend = min(nrec, rbeg + per);
+  if (rbeg >= rend) return;
   crc_tables_init(S.crc_t);
-  if (tid == 0) S.cur_slice = 0xffffffffu;
+  if (warp == 0) {
+    tc::tmem_alloc(&S.tmem_base, kTcCols);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) {
+    S.cur_slice = 0xffffffffu;
+    tc::mbar_init(&S.bar, 1);
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = S.tmem_base;
+  uint32_t phase = 0;
+  bool alive = true;
   const uint32_t rps = 1u + sh.n_mid;
-  const uint32_t tg = tid >> 4, kg = tid & 15u;
-  for (uint32_t r = rbeg; r < rend; ++r) {
+  constexpr uint32_t idesc = tc::idesc_bf16_f32(kTcRows, kD);
+  for (uint32_t r = rbeg; r < rend && alive; ++r) {
     __syncthreads();
     const uint8_t* e = src + kHeaderBytes + uint64_t(kIndexEntry) * r;
     const uint64_t off0 = ld_u64(e);
@@ -332,11 +360,9 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, const uint8_t* __rest
     const uint32_t nb = (tcc + kTile - 1) / kTile;
     if (S.cur_slice != sidx) {
       __syncthreads();
-      const float* Q = pl.bases + uint64_t(sidx) * kD * kD;
-      for (uint32_t i = tid; i < kD * kD; i += nthr) {
-        uint32_t k = i / kD, j = i % kD;
-        S.Qt[j * kD + k] = __ldg(Q + i);
-      }
+      const uint4* q4 = reinterpret_cast<const uint4*>(pl.qsplit + uint64_t(sidx) * kQSplitBytes);
+      uint4* b4 = reinterpret_cast<uint4*>(S.b_hi);  // b_hi and b_lo are contiguous
+      for (uint32_t i = tid; i < kQSplitBytes / 16u; i += nthr) b4[i] = __ldg(q4 + i);
       build_comp_info(pl.widths + uint64_t(sidx) * kD, S.ci, S.tmp);
       if (tid == 0) S.cur_slice = sidx;
       __syncthreads();
@@ -362,11 +388,11 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, const uint8_t* __rest
       __syncthreads();
       st = block_parse_stream(rec + off, len - off, n, &S.si, S.freq, S.tmp);
       if (st != kOk) break;
-      auto put = [&](uint32_t i, uint32_t s) {
+      auto put = [&](uint32_t i, uint32_t sy) {
         uint32_t a, t;
         split(i, a, t);
-        if (s > levels) S.bad = 1;
-        S.codes[S.ci.comp[base + a] * kMaxCt + t] = uint8_t(s);
+        if (sy > levels) S.bad = 1;
+        S.codes[S.ci.comp[base + a] * kMaxCt + t] = uint8_t(sy);
       };
       bool ok = true;
       if (S.si.mode == kModeRaw) {
@@ -375,7 +401,7 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, const uint8_t* __rest
         for (uint32_t i = tid; i < n; i += nthr) put(i, S.si.sym);
       } else {
         block_dec_lut(S.freq, S.cum, S.lut, S.tmp);
-        const uint32_t N = rans_lanes(n), G = rans_groups(N), warp = tid >> 5;
+        const uint32_t N = rans_lanes(n), G = rans_groups(N);
         if (warp < G)
           ok = rans_decode_group(rec + off + S.si.sub_off[warp], S.si.sub_len[warp], n, N, warp,
                                  S.lut, put);
@@ -389,56 +415,100 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, const uint8_t* __rest
       if (tid == 0) atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(st));
       continue;
     }
-    __syncthreads();
-    for (uint32_t blk = 0; blk < nb; ++blk) {
-      const uint32_t bl = min(kTile, tcc - blk * kTile);
-      const uint32_t tb = t0 + blk * kTile;
-      for (uint32_t idx = tid; idx < kTile * kD; idx += nthr) {
-        const uint32_t tt = idx / kD, j = idx % kD;
+    // inverse projection on the tensor cores, 128 tokens at a time:
+    // x^[t][k] = sum_j y^[t][j] Q[k][j] with y^ and Q split into bf16 hi + lo
+    // pieces (hi*hi + hi*lo + lo*hi, fp32 accumulation in tensor memory)
+    for (uint32_t t_base = 0; t_base < tcc; t_base += kTcRows) {
+      const uint32_t bl = min(kTcRows, tcc - t_base);
+      __syncthreads();
+      for (uint32_t idx = tid; idx < kTcRows * kD; idx += nthr) {
+        const uint32_t tt = idx >> 7, j = idx & (kD - 1u);
         float v = 0.0f;
-        if (tt < bl && S.ci.width[j])
-          v = __fmaf_rn(float(S.codes[j * kMaxCt + blk * kTile + tt]), S.zs[j][blk][1], S.zs[j][blk][0]);
-        S.yh[idx] = v;
+        if (tt < bl && S.ci.width[j]) {
+          const uint32_t t = t_base + tt, blk = t / kTile;
+          v = __fmaf_rn(float(S.codes[j * kMaxCt + t]), S.zs[j][blk][1], S.zs[j][blk][0]);
+        }
+        const uint32_t h = f32_to_bf16_rne(v);
+        const uint32_t l = f32_to_bf16_rne(__fsub_rn(v, bf16_to_f32(h)));
+        const uint32_t o = tc::sw128_offset(tt, 2u * j, kTcRows);
+        *reinterpret_cast<uint16_t*>(S.a_hi + o) = uint16_t(h);
+        *reinterpret_cast<uint16_t*>(S.a_lo + o) = uint16_t(l);
       }
+      tc::fence_async_smem();
       __syncthreads();
-      double acc[4][8];
+      if (tid == 0) {
+        tc::fence_after_sync();
+        const uint32_t ah = tc::smem_addr(S.a_hi), al = tc::smem_addr(S.a_lo);
+        const uint32_t bh = tc::smem_addr(S.b_hi), bo = tc::smem_addr(S.b_lo);
+        uint32_t acc = 0;
+        for (uint32_t ks = 0; ks < kD / 16u; ++ks) {  // K = 16 components per MMA
+          const uint32_t koff = (ks >> 2) * (kTcRows * 128u) + (ks & 3u) * 32u;
+          const uint32_t kboff = (ks >> 2) * (kD * 128u) + (ks & 3u) * 32u;
+          tc::mma_bf16(tmem, tc::desc_sw128(ah + koff), tc::desc_sw128(bh + kboff), idesc, acc);
+          acc = 1;
+          tc::mma_bf16(tmem, tc::desc_sw128(ah + koff), tc::desc_sw128(bo + kboff), idesc, 1);
+          tc::mma_bf16(tmem, tc::desc_sw128(al + koff), tc::desc_sw128(bh + kboff), idesc, 1);
+        }
+        tc::mma_commit(&S.bar);
+      }
+      const bool done = tc::mbar_wait(&S.bar, phase, 1u << 22);
+      phase ^= 1u;
+      if (!__syncthreads_and(done)) {
+        if (tid == 0) atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(kErrTimeout));
+        tc::mbar_wait(&S.bar, phase ^ 1u, 1u << 22);
+        alive = false;
+        break;
+      }
+      tc::fence_after_sync();
+      // epilogue: warp w reads token rows 32 (w % 4) .., channel quarter (w / 4):
+      // channels [32q, 32q + 32) and their RoPE partners [32q + 64, 32q + 96)
+      {
+        const uint32_t sub = warp & 3u, q = warp >> 2;
+        const uint32_t tt = sub * 32u + lane;
+        const uint32_t c0 = q * 32u;
+        uint32_t va[32], vb[32];
+        const uint32_t ta = tmem + ((sub * 32u) << 16);
+        tc::tmem_ld16(ta + c0, va);
+        tc::tmem_ld16(ta + c0 + 16u, va + 16);
+        tc::tmem_ld16(ta + c0 + 64u, vb);
+        tc::tmem_ld16(ta + c0 + 80u, vb + 16);
+        tc::tmem_wait_ld();
+        if (tt < bl) {
+          const uint32_t t = t0 + t_base + tt;
+          const float2* cs = reinterpret_cast<const float2*>(pl.rope) + uint64_t(t) * (kD / 2) + c0;
+          uint32_t pa[16], pb[16];
 #pragma unroll
-      for (int a = 0; a < 4; ++a)
+          for (uint32_t i = 0; i < 32; i += 2) {
+            float a0 = __uint_as_float(va[i]), b0 = __uint_as_float(vb[i]);
+            float a1 = __uint_as_float(va[i + 1]), b1 = __uint_as_float(vb[i + 1]);
+            if (is_key) {
+              const float2 k0 = cs[i], k1 = cs[i + 1];
+              const float na0 = __fsub_rn(__fmul_rn(a0, k0.x), __fmul_rn(b0, k0.y));
+              const float nb0 = __fadd_rn(__fmul_rn(a0, k0.y), __fmul_rn(b0, k0.x));
+              const float na1 = __fsub_rn(__fmul_rn(a1, k1.x), __fmul_rn(b1, k1.y));
+              const float nb1 = __fadd_rn(__fmul_rn(a1, k1.y), __fmul_rn(b1, k1.x));
+              a0 = na0; b0 = nb0; a1 = na1; b1 = nb1;
+            }
+            pa[i >> 1] = f32_to_bf16_rne(a0) | (f32_to_bf16_rne(a1) << 16);
+            pb[i >> 1] = f32_to_bf16_rne(b0) | (f32_to_bf16_rne(b1) << 16);
+          }
+          uint4* ra = reinterpret_cast<uint4*>(xs + uint64_t(t) * kD + c0);
+          uint4* rb = reinterpret_cast<uint4*>(xs + uint64_t(t) * kD + c0 + 64u);
 #pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] = 0.0;
-      for (uint32_t j = 0; j < kD; ++j) {
-        const float4 q0 = *reinterpret_cast<const float4*>(&S.Qt[j * kD + kg * 8]);
-        const float4 q1 = *reinterpret_cast<const float4*>(&S.Qt[j * kD + kg * 8 + 4]);
-        const double qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-        for (int a = 0; a < 4; ++a) {
-          const double yv = S.yh[(tg * 4 + a) * kD + j];
-#pragma unroll
-          for (int b = 0; b < 8; ++b) acc[a][b] = fma(qv[b], yv, acc[a][b]);
+          for (uint32_t v = 0; v < 4; ++v) {
+            ra[v] = make_uint4(pa[4 * v], pa[4 * v + 1], pa[4 * v + 2], pa[4 * v + 3]);
+            rb[v] = make_uint4(pb[4 * v], pb[4 * v + 1], pb[4 * v + 2], pb[4 * v + 3]);
+          }
         }
       }
-      __syncthreads();
-#pragma unroll
-      for (int a = 0; a < 4; ++a)
-#pragma unroll
-        for (int b = 0; b < 8; ++b) S.yh[(tg * 4 + a) * kD + kg * 8 + b] = __double2float_rn(acc[a][b]);
-      __syncthreads();
-      for (uint32_t idx = tid; idx < bl * (kD / 2); idx += nthr) {
-        const uint32_t tt = idx / (kD / 2), i = idx % (kD / 2);
-        float a = S.yh[tt * kD + i], b = S.yh[tt * kD + i + kD / 2];
-        if (is_key) {
-          const float2 cs = reinterpret_cast<const float2*>(pl.rope)[uint64_t(tb + tt) * (kD / 2) + i];
-          float na = __fsub_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y));
-          float nb2 = __fadd_rn(__fmul_rn(a, cs.y), __fmul_rn(b, cs.x));
-          a = na;
-          b = nb2;
-        }
-        uint16_t* row = xs + uint64_t(tb + tt) * kD;
-        row[i] = uint16_t(f32_to_bf16_rne(a));
-        row[i + kD / 2] = uint16_t(f32_to_bf16_rne(b));
-      }
-      __syncthreads();
+      tc::fence_before_sync();
     }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, kTcCols);
   }
 }
 
@@ -487,7 +557,7 @@ cudaError_t launch_transform_decode(const TransformShape& s, const TransformPlan
                                     const uint8_t* src, uint16_t* dst, DecodeState* ds,
                                     uint32_t max_records, cudaStream_t st) {
   if (max_records == 0) return cudaSuccess;
-  size_t smem = sizeof(DecSmem);
+  size_t smem = sizeof(DecSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_transform_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   uint32_t grid = min(max_records, uint32_t(num_sms()));
