@@ -33,8 +33,8 @@ WORKLOAD_L = "lossless-64x8x32768x128-bf16"
 WORKLOAD_T = "transform-64x8x32768x128-bf16"
 METRIC = "KV codec encode/decode GB/s (raw bytes) vs HBM roofline; compression ratio"
 
-# algorithmic work per launch of each kernel, given the frame's raw bytes R, its
-# container bytes C and middle values V (see the kernel table of the design notes)
+# algorithmic work per step of each kernel, given the step's raw bytes R, its
+# container bytes C and its middle (transform-coded) values V
 KERNEL_WORK = {
     "lossless_encode": ("hbm", lambda R, C, V: R + C),
     "lossless_decode": ("hbm", lambda R, C, V: R + C),
@@ -168,6 +168,17 @@ class Job:
         self.cont_t = torch.empty(self.frames * self.cap_t, dtype=torch.uint8, device="cuda")
         self.out = torch.empty(self.frames * self.frame_vals, dtype=torch.int16, device="cuda")
         self.res = torch.zeros(self.frames * 4, 2, dtype=torch.int64, device="cuda")
+        # batch workspaces: encode groups of up to 16 frames, decode up to 64 frames per launch
+        grp = min(16, self.frames)
+        self.ws_enc_l = torch.empty(kvc.batch_workspace_bytes(self.plan_l, kvc.LOSSLESS, False, grp,
+                                                              self.spf), dtype=torch.uint8, device="cuda")
+        self.ws_enc_t = torch.empty(kvc.batch_workspace_bytes(self.plan_t, kvc.TRANSFORM, False, grp,
+                                                              self.spf), dtype=torch.uint8, device="cuda")
+        self.ws_dec = torch.empty(max(kvc.batch_workspace_bytes(self.plan_l, kvc.LOSSLESS, True,
+                                                                self.frames, self.spf),
+                                      kvc.batch_workspace_bytes(self.plan_t, kvc.TRANSFORM, True,
+                                                                self.frames, self.spf)),
+                                  dtype=torch.uint8, device="cuda")
         self.sizes_l = self.sizes_t = None
         # middle values per frame (transform path)
         s_end = min(w_t.n_sink, self.T)
@@ -179,12 +190,12 @@ class Job:
 
     def encode_all(self, path):
         kvc = self.kvc
-        codec, cont, cap, base = ((self.codec_l, self.cont_l, self.cap_l, 0) if path == kvc.LOSSLESS
-                                  else (self.codec_t, self.cont_t, self.cap_t, self.frames))
-        for f in range(self.frames):
-            codec.container = self._frame(cont, f, cap)
-            codec.encode(self.x[f * self.frame_vals:(f + 1) * self.frame_vals], f * self.spf,
-                         res=self.res[base + f])
+        cont, cap, base, plan, ws = ((self.cont_l, self.cap_l, 0, self.plan_l, self.ws_enc_l)
+                                     if path == kvc.LOSSLESS else
+                                     (self.cont_t, self.cap_t, self.frames, self.plan_t, self.ws_enc_t))
+        frames = [(f * self.spf, self.spf, self.x[f * self.frame_vals:(f + 1) * self.frame_vals],
+                   self._frame(cont, f, cap), self.res[base + f]) for f in range(self.frames)]
+        kvc.encode_batch(plan, path, frames, ws)
 
     def read_sizes(self):
         r = self.res[: 2 * self.frames].cpu().numpy()
@@ -196,14 +207,14 @@ class Job:
 
     def decode_all(self, path):
         kvc = self.kvc
-        codec, cont, cap, sizes, base = (
-            (self.codec_l, self.cont_l, self.cap_l, self.sizes_l, 2 * self.frames)
+        cont, cap, sizes, base, plan = (
+            (self.cont_l, self.cap_l, self.sizes_l, 2 * self.frames, self.plan_l)
             if path == kvc.LOSSLESS else
-            (self.codec_t, self.cont_t, self.cap_t, self.sizes_t, 3 * self.frames))
-        for f in range(self.frames):
-            codec.decode(self._frame(cont, f, cap), sizes[f],
-                         out=self.out[f * self.frame_vals:(f + 1) * self.frame_vals],
-                         res=self.res[base + f])
+            (self.cont_t, self.cap_t, self.sizes_t, 3 * self.frames, self.plan_t))
+        frames = [(self._frame(cont, f, cap), sizes[f],
+                   self.out[f * self.frame_vals:(f + 1) * self.frame_vals], self.res[base + f])
+                  for f in range(self.frames)]
+        kvc.decode_batch(plan, path, frames, self.ws_dec, self.spf)
 
     def step(self, ev):
         kvc = self.kvc
@@ -341,25 +352,26 @@ def run_kvc(args):
     hbm_peak, sm_max, peak_kind = measured_peaks()
     fp64_peak = 148 * 64 * 2 * sm_max * 1e6 / 1e12  # TFLOP/s, 64 fp64 FMA/clk/SM
     launches = sum(n for n, _ in kernels.values())
-    avg_cont = {"lossless_encode": cont_l / job.frames, "lossless_decode": cont_l / job.frames,
-                "transform_encode_mid": cont_t / job.frames, "transform_decode": cont_t / job.frames}
+    step_cont = {"lossless_encode": cont_l, "lossless_decode": cont_l,
+                 "transform_encode_mid": cont_t, "transform_decode": cont_t}
     kern_out = {}
     total_kern_ms = sum(t for _, t in kernels.values()) or 1.0
     for name, (n, t) in kernels.items():
         entry = {"launches": n, "total_ms": round(t, 3), "share": round(t / total_kern_ms, 4)}
         if name in KERNEL_WORK and n:
             bound, fn = KERNEL_WORK[name]
-            per_launch_ms = t / n
-            work = fn(job.frame_bytes, avg_cont[name], job.mid_vals)
+            work = fn(raw, step_cont[name], job.mid_vals * job.frames) * args.steps
+            secs = t * 1e-3
             if bound == "hbm":
-                ach = work / (per_launch_ms * 1e-3) / 1e9
+                ach = work / secs / 1e9
                 entry.update(bound="hbm", achieved=round(ach, 1), peak=hbm_peak, unit="GB/s",
-                             frac=round(ach / hbm_peak, 4), algorithmic_bytes=int(work))
+                             frac=round(ach / hbm_peak, 4),
+                             algorithmic_bytes_per_launch=int(work / n))
             else:
-                ach = work / (per_launch_ms * 1e-3) / 1e12
+                ach = work / secs / 1e12
                 entry.update(bound="alu", achieved=round(ach, 3), peak=round(fp64_peak, 2),
                              unit="TFLOP/s", frac=round(ach / fp64_peak, 4),
-                             algorithmic_flops=int(work))
+                             algorithmic_flops_per_launch=int(work / n))
         kern_out[name] = entry
     dominant = max(kern_out, key=lambda k: kern_out[k]["total_ms"]) if kern_out else None
     roof = None

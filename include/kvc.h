@@ -127,7 +127,10 @@ uint32_t kvc_plan_crc(const kvc_plan_t* plan);
 /* Upper bound of the container size for n_slices slices of the given path
  * (exact for incompressible input: the codec never exceeds it). 0 on error. */
 size_t kvc_max_encoded_bytes(const kvc_plan_t* plan, int path, uint32_t n_slices);
-/* Device workspace an encode or decode of n_slices slices needs. */
+/* Device workspace an encode of n_slices slices needs; for a decode, n_slices
+ * is the most slices a container will hold (0: any container of the plan), and
+ * a container with more slices than the workspace allows reports
+ * KVC_ERR_CAPACITY in its result. */
 size_t kvc_workspace_bytes(const kvc_plan_t* plan, int path, int decode, uint32_t n_slices);
 
 /* Encode slices [first_slice, first_slice + n_slices) of the cache.
@@ -163,6 +166,39 @@ int kvc_encode_transform(const kvc_plan_t* plan, uint32_t first_slice, uint32_t 
 int kvc_decode_transform(const kvc_plan_t* plan, const void* d_src, size_t src_bytes, void* d_dst,
                          size_t dst_cap, void* d_ws, size_t ws_bytes, kvc_result* d_res,
                          cudaStream_t stream);
+
+/* Batches. Each frame is an independent container (for example one 64 MiB
+ * layer-K or layer-V tensor of a long cache); a batch codes many frames with
+ * one launch per kernel for every 64 frames, which keeps all SMs busy when a
+ * single frame has too few chunks to fill the GPU.
+ *   encode: src = device [n_slices][T][D] values of slices
+ *           [first_slice, first_slice + n_slices); dst/dst_cap = container
+ *           buffer (>= kvc_max_encoded_bytes for n_slices)
+ *   decode: src/src_bytes = device container; dst/dst_cap = output values;
+ *           first_slice and n_slices are ignored
+ *   res:    device kvc_result of this frame
+ * Frames in one call must not share dst buffers. */
+typedef struct {
+  uint32_t first_slice;
+  uint32_t n_slices;
+  const void* src;
+  size_t src_bytes;
+  void* dst;
+  size_t dst_cap;
+  kvc_result* res;
+} kvc_frame;
+
+/* Device workspace for a batch call of n_frames frames of at most
+ * max_slices_per_frame slices each. Decoding a container with more slices
+ * than max_slices_per_frame reports KVC_ERR_CAPACITY in its result. */
+size_t kvc_batch_workspace_bytes(const kvc_plan_t* plan, int path, int decode, uint32_t n_frames,
+                                 uint32_t max_slices_per_frame);
+/* Encode or decode n_frames frames (host array h_frames) on one stream. Return
+ * values and per-frame results as for the single-container calls. */
+int kvc_encode_batch(const kvc_plan_t* plan, int path, const kvc_frame* h_frames, uint32_t n_frames,
+                     void* d_ws, size_t ws_bytes, cudaStream_t stream);
+int kvc_decode_batch(const kvc_plan_t* plan, int path, const kvc_frame* h_frames, uint32_t n_frames,
+                     uint32_t max_slices_per_frame, void* d_ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Human-readable name of a status code (static string). */
 const char* kvc_status_string(int status);

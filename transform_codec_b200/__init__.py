@@ -28,6 +28,7 @@ EXPORTS = [
     "kvc_status_string", "kvc_calibrate_pca", "kvc_allocate_bits",
     "kvc_stage_crc32", "kvc_stage_stream_encode", "kvc_stage_stream_decode",
     "kvc_profile_begin", "kvc_profile_end",
+    "kvc_batch_workspace_bytes", "kvc_encode_batch", "kvc_decode_batch",
 ]
 
 
@@ -49,6 +50,13 @@ class PlanDesc(ctypes.Structure):
         ("rope_theta", ctypes.c_double), ("avg_bits", ctypes.c_double),
         ("bases", ctypes.c_void_p), ("eigvals", ctypes.c_void_p), ("widths", ctypes.c_void_p),
     ]
+
+
+class Frame(ctypes.Structure):
+    _fields_ = [("first_slice", ctypes.c_uint32), ("n_slices", ctypes.c_uint32),
+                ("src", ctypes.c_void_p), ("src_bytes", ctypes.c_size_t),
+                ("dst", ctypes.c_void_p), ("dst_cap", ctypes.c_size_t),
+                ("res", ctypes.c_void_p)]
 
 
 class KernelTime(ctypes.Structure):
@@ -75,6 +83,9 @@ def _load():
         "kvc_status_string": ([i32], ctypes.c_char_p),
         "kvc_calibrate_pca": ([ctypes.POINTER(PlanDesc), vp, u32, vp, vp, i32], i32),
         "kvc_allocate_bits": ([vp, ctypes.c_uint64, ctypes.c_double, u32, vp], i32),
+        "kvc_batch_workspace_bytes": ([vp, i32, i32, u32, u32], sz),
+        "kvc_encode_batch": ([vp, i32, ctypes.POINTER(Frame), u32, vp, sz, vp], i32),
+        "kvc_decode_batch": ([vp, i32, ctypes.POINTER(Frame), u32, u32, vp, sz, vp], i32),
         "kvc_profile_begin": ([], i32),
         "kvc_profile_end": ([ctypes.POINTER(KernelTime), i32, ctypes.POINTER(i32)], i32),
         "kvc_stage_crc32": ([vp, sz, vp, vp], i32),
@@ -228,6 +239,38 @@ class Codec:
                 self.ws_dec.numel(), _dptr(r), _stream(stream))
         _check(st, "decode")
         return r
+
+
+def batch_workspace_bytes(plan: Plan, path: int, decode: bool, n_frames: int,
+                          max_slices_per_frame: int) -> int:
+    return _lib.kvc_batch_workspace_bytes(plan.handle, path, int(decode), n_frames,
+                                          max_slices_per_frame)
+
+
+def _frames(items):
+    arr = (Frame * max(len(items), 1))()
+    for i, it in enumerate(items):
+        arr[i] = Frame(*it)
+    return arr
+
+
+def encode_batch(plan: Plan, path: int, frames, ws, stream=None):
+    """frames: sequence of (first_slice, n_slices, src_tensor, dst_tensor, res_tensor)."""
+    items = [(fs, ns, src.data_ptr() if src is not None and src.numel() else None, 0,
+              dst.data_ptr(), dst.numel() * dst.element_size(), res.data_ptr())
+             for fs, ns, src, dst, res in frames]
+    _check(_lib.kvc_encode_batch(plan.handle, path, _frames(items), len(items), _dptr(ws),
+                                 ws.numel() * ws.element_size(), _stream(stream)),
+           "kvc_encode_batch")
+
+
+def decode_batch(plan: Plan, path: int, frames, ws, max_slices_per_frame: int = 0, stream=None):
+    """frames: sequence of (src_tensor, src_bytes, dst_tensor, res_tensor)."""
+    items = [(0, 0, src.data_ptr(), nbytes, dst.data_ptr(), dst.numel() * dst.element_size(),
+              res.data_ptr()) for src, nbytes, dst, res in frames]
+    _check(_lib.kvc_decode_batch(plan.handle, path, _frames(items), len(items),
+                                 max_slices_per_frame, _dptr(ws), ws.numel() * ws.element_size(),
+                                 _stream(stream)), "kvc_decode_batch")
 
 
 def read_result(res) -> tuple[int, int]:

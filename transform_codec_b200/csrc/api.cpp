@@ -1,6 +1,6 @@
 // Host side of the KV codec library: plans, workspace sizing and the C ABI
 // declared in include/kvc.h. Kernels live in the .cu files of this directory.
-#include "../../include/kvc.h"
+#include "kvc.h"
 
 #include <algorithm>
 #include <atomic>
@@ -339,90 +339,132 @@ bool path_ok(const kvc_plan_s* p, int path) {
   return p && (path == KVC_PATH_LOSSLESS || (path == KVC_PATH_TRANSFORM && p->transform));
 }
 
-uint64_t encode_ws_bytes(const kvc_plan_s* p, int path, uint32_t n_slices) {
-  const uint64_t nr = uint64_t(n_slices) * records_per_slice(p, path);
-  return pad256u(sizeof(EncodeState)) + pad256u(nr * 4) * 2 + pad256u(nr * 8) + nr * slot_bytes(p, path);
+// encode workspace for `frames` frames holding `recs` records in total
+uint64_t encode_ws_for(const kvc_plan_s* p, int path, uint64_t recs) {
+  return pad256u(sizeof(EncodeState) * kBatchMax) + pad256u(recs * 4) * 2 + pad256u(recs * 8) +
+         recs * slot_bytes(p, path);
 }
 
-EncodeLayout encode_layout(const kvc_plan_s* p, int path, uint32_t n_slices, void* ws) {
-  const uint64_t nr = uint64_t(n_slices) * records_per_slice(p, path);
+EncodeLayout encode_layout(const kvc_plan_s* p, int path, uint64_t recs, void* ws) {
   uint8_t* b = static_cast<uint8_t*>(ws);
   EncodeLayout L;
   L.state = reinterpret_cast<EncodeState*>(b);
-  b += pad256u(sizeof(EncodeState));
+  b += pad256u(sizeof(EncodeState) * kBatchMax);
   L.rec_len = reinterpret_cast<uint32_t*>(b);
-  b += pad256u(nr * 4);
+  b += pad256u(recs * 4);
   L.rec_crc = reinterpret_cast<uint32_t*>(b);
-  b += pad256u(nr * 4);
+  b += pad256u(recs * 4);
   L.rec_off = reinterpret_cast<uint64_t*>(b);
-  b += pad256u(nr * 8);
+  b += pad256u(recs * 8);
   L.slots = b;
   L.slot_bytes = slot_bytes(p, path);
   return L;
+}
+
+uint64_t decode_ws_for(const kvc_plan_s* p, int path, uint32_t frames, uint32_t max_slices) {
+  const uint64_t f = std::min<uint32_t>(frames, kBatchMax);
+  return kDecodeWsFixed + pad256u(8ull * f * max_slices * records_per_slice(p, path));
 }
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? KVC_OK : KVC_ERR_CUDA; }
 
-int encode_common(const kvc_plan_t* plan, int path, uint32_t first_slice, uint32_t n_slices,
-                  const void* d_src, void* d_dst, size_t dst_cap, void* d_ws, size_t ws_bytes,
-                  kvc_result* d_res, cudaStream_t stream) {
-  if (!path_ok(plan, path)) return plan ? KVC_ERR_UNSUPPORTED : KVC_ERR_INVALID;
-  if (uint64_t(first_slice) + n_slices > plan->S || !d_dst || !d_ws || !d_res) return KVC_ERR_INVALID;
-  if ((n_slices && !d_src) || !aligned16(d_src) || !aligned16(d_dst) || !aligned16(d_ws) ||
-      !aligned16(d_res))
-    return KVC_ERR_INVALID;
-  if (dst_cap < kvc_max_encoded_bytes(plan, path, n_slices)) return KVC_ERR_CAPACITY;
-  if (ws_bytes < encode_ws_bytes(plan, path, n_slices)) return KVC_ERR_CAPACITY;
+int check_plan_device(const kvc_plan_s* p) {
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev != plan->device) return KVC_ERR_INVALID;
-  const EncodeLayout L = encode_layout(plan, path, n_slices, d_ws);
-  const uint16_t* src = static_cast<const uint16_t*>(d_src);
-  cudaError_t e;
-  HeaderFields h{};
-  h.path = uint32_t(path);
-  h.dtype = plan->d.dtype;
-  h.L = plan->d.n_layers; h.H = plan->d.n_heads; h.T = plan->d.n_tokens; h.D = plan->d.head_dim;
-  h.first_slice = first_slice;
-  h.n_slices = n_slices;
-  h.n_records = n_slices * records_per_slice(plan, path);
-  if (path == KVC_PATH_LOSSLESS) {
-    h.chunk_tokens = plan->ls.tc;
-    e = launch_lossless_encode(plan->ls, src, n_slices, L, stream);
-  } else {
-    h.chunk_tokens = plan->ts.ct;
-    h.plan_crc = plan->plan_crc;
-    h.n_sink = plan->d.n_sink;
-    h.n_recent = plan->d.n_recent;
-    h.block_tokens = plan->d.block_tokens;
-    TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope, plan->d_qsplit};
-    e = launch_transform_encode(plan->ts, pd, src, first_slice, n_slices, L, stream);
-  }
-  if (e != cudaSuccess) return KVC_ERR_CUDA;
-  e = launch_finalize(h, L, static_cast<uint8_t*>(d_dst), dst_cap, d_res, stream);
-  return cuda_status(e);
+  return dev == p->device ? KVC_OK : KVC_ERR_INVALID;
 }
 
-int decode_common(const kvc_plan_t* plan, int path, const void* d_src, size_t src_bytes, void* d_dst,
-                  size_t dst_cap, void* d_ws, size_t ws_bytes, kvc_result* d_res,
-                  cudaStream_t stream) {
+HeaderFields header_fields(const kvc_plan_s* p, int path) {
+  HeaderFields h{};
+  h.path = uint32_t(path);
+  h.dtype = p->d.dtype;
+  h.L = p->d.n_layers; h.H = p->d.n_heads; h.T = p->d.n_tokens; h.D = p->d.head_dim;
+  h.recs_per_slice = records_per_slice(p, path);
+  if (path == KVC_PATH_LOSSLESS) {
+    h.chunk_tokens = p->ls.tc;
+  } else {
+    h.chunk_tokens = p->ts.ct;
+    h.plan_crc = p->plan_crc;
+    h.n_sink = p->d.n_sink;
+    h.n_recent = p->d.n_recent;
+    h.block_tokens = p->d.block_tokens;
+  }
+  return h;
+}
+
+int encode_frames(const kvc_plan_s* plan, int path, const kvc_frame* fr, uint32_t n, void* d_ws,
+                  size_t ws_bytes, cudaStream_t stream) {
   if (!path_ok(plan, path)) return plan ? KVC_ERR_UNSUPPORTED : KVC_ERR_INVALID;
-  if (!d_src || !d_ws || !d_res || (dst_cap && !d_dst)) return KVC_ERR_INVALID;
-  if (!aligned16(d_src) || !aligned16(d_dst) || !aligned16(d_ws) || !aligned16(d_res))
-    return KVC_ERR_INVALID;
-  if (ws_bytes < kvc_workspace_bytes(plan, path, 1, 0)) return KVC_ERR_CAPACITY;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev != plan->device) return KVC_ERR_INVALID;
-  DecodeState* ds = static_cast<DecodeState*>(d_ws);
+  if ((n && !fr) || !d_ws || !aligned16(d_ws)) return KVC_ERR_INVALID;
+  int st = check_plan_device(plan);
+  if (st) return st;
+  const uint32_t rps = records_per_slice(plan, path);
+  for (uint32_t i = 0; i < n; ++i) {
+    const kvc_frame& f = fr[i];
+    if (uint64_t(f.first_slice) + f.n_slices > plan->S || !f.dst || !f.res) return KVC_ERR_INVALID;
+    if ((f.n_slices && !f.src) || !aligned16(f.src) || !aligned16(f.dst) || !aligned16(f.res))
+      return KVC_ERR_INVALID;
+    if (f.dst_cap < kvc_max_encoded_bytes(plan, path, f.n_slices)) return KVC_ERR_CAPACITY;
+  }
+  const HeaderFields h = header_fields(plan, path);
+  uint32_t i = 0;
+  while (i < n) {  // groups of frames whose records fit the workspace
+    FrameBatch b{};
+    uint64_t recs = 0;
+    while (i < n && b.n < kBatchMax) {
+      const uint64_t r = uint64_t(fr[i].n_slices) * rps;
+      if (encode_ws_for(plan, path, recs + r) > ws_bytes) break;
+      FrameDesc& d = b.f[b.n];
+      d.src = static_cast<const uint8_t*>(fr[i].src);
+      d.dst = static_cast<uint8_t*>(fr[i].dst);
+      d.res = fr[i].res;
+      d.dst_cap = fr[i].dst_cap;
+      d.first_slice = fr[i].first_slice;
+      d.n_slices = fr[i].n_slices;
+      b.rec_base[b.n] = uint32_t(recs);
+      recs += r;
+      ++b.n;
+      ++i;
+    }
+    if (b.n == 0) return KVC_ERR_CAPACITY;
+    b.rec_base[b.n] = uint32_t(recs);
+    const EncodeLayout L = encode_layout(plan, path, recs, d_ws);
+    cudaError_t e;
+    if (path == KVC_PATH_LOSSLESS) {
+      e = launch_lossless_encode(plan->ls, b, L, stream);
+    } else {
+      TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope, plan->d_qsplit};
+      e = launch_transform_encode(plan->ts, pd, b, L, stream);
+    }
+    if (e != cudaSuccess) return KVC_ERR_CUDA;
+    e = launch_finalize(h, b, L, stream);
+    if (e != cudaSuccess) return KVC_ERR_CUDA;
+  }
+  return KVC_OK;
+}
+
+int decode_frames(const kvc_plan_s* plan, int path, const kvc_frame* fr, uint32_t n,
+                  uint32_t max_slices, void* d_ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!path_ok(plan, path)) return plan ? KVC_ERR_UNSUPPORTED : KVC_ERR_INVALID;
+  if ((n && !fr) || !d_ws || !aligned16(d_ws)) return KVC_ERR_INVALID;
+  if (max_slices == 0 || max_slices > plan->S) max_slices = plan->S;
+  if (ws_bytes < decode_ws_for(plan, path, n, max_slices)) return KVC_ERR_CAPACITY;
+  int st = check_plan_device(plan);
+  if (st) return st;
+  for (uint32_t i = 0; i < n; ++i) {
+    const kvc_frame& f = fr[i];
+    if (!f.src || !f.res || (f.dst_cap && !f.dst) || !aligned16(f.src) || !aligned16(f.dst) ||
+        !aligned16(f.res))
+      return KVC_ERR_INVALID;
+  }
   ContainerExpect ex{};
   ex.path = uint32_t(path);
   ex.dtype = plan->d.dtype;
   ex.L = plan->d.n_layers; ex.H = plan->d.n_heads; ex.T = plan->d.n_tokens; ex.D = plan->d.head_dim;
   ex.recs_per_slice = records_per_slice(plan, path);
-  ex.dst_cap = dst_cap;
+  ex.max_slices = max_slices;
   if (path == KVC_PATH_LOSSLESS) {
     ex.chunk_tokens = plan->ls.tc;
   } else {
@@ -432,21 +474,56 @@ int decode_common(const kvc_plan_t* plan, int path, const void* d_src, size_t sr
     ex.block_tokens = plan->d.block_tokens;
     ex.plan_crc = plan->plan_crc;
   }
-  const uint8_t* src = static_cast<const uint8_t*>(d_src);
-  uint16_t* dst = static_cast<uint16_t*>(d_dst);
-  cudaError_t e = launch_check_container(src, src_bytes, ex, ds, d_res, stream);
-  if (e != cudaSuccess) return KVC_ERR_CUDA;
-  // upper bound of records a valid container for this plan can hold
-  const uint64_t max_rec64 = uint64_t(plan->S) * records_per_slice(plan, path);
-  const uint32_t max_rec = uint32_t(std::min<uint64_t>(max_rec64, 0xffffffffu));
-  if (path == KVC_PATH_LOSSLESS) {
-    e = launch_lossless_decode(plan->ls, src, dst, ds, max_rec, stream);
-  } else {
-    TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope, plan->d_qsplit};
-    e = launch_transform_decode(plan->ts, pd, src, dst, ds, max_rec, stream);
+  uint8_t* ws = static_cast<uint8_t*>(d_ws);
+  for (uint32_t i = 0; i < n; i += kBatchMax) {
+    FrameBatch b{};
+    b.n = std::min<uint32_t>(kBatchMax, n - i);
+    for (uint32_t k = 0; k < b.n; ++k) {
+      FrameDesc& d = b.f[k];
+      d.src = static_cast<const uint8_t*>(fr[i + k].src);
+      d.src_bytes = fr[i + k].src_bytes;
+      d.dst = static_cast<uint8_t*>(fr[i + k].dst);
+      d.dst_cap = fr[i + k].dst_cap;
+      d.res = fr[i + k].res;
+    }
+    cudaError_t e = launch_check_container(b, ex, ws, stream);
+    if (e != cudaSuccess) return KVC_ERR_CUDA;
+    const uint64_t max_rec64 = uint64_t(b.n) * max_slices * ex.recs_per_slice;
+    const uint32_t max_rec = uint32_t(std::min<uint64_t>(max_rec64, 0xffffffffu));
+    if (path == KVC_PATH_LOSSLESS) {
+      e = launch_lossless_decode(plan->ls, b, ws, max_rec, stream);
+    } else {
+      TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope, plan->d_qsplit};
+      e = launch_transform_decode(plan->ts, pd, b, ws, max_rec, stream);
+    }
+    if (e != cudaSuccess) return KVC_ERR_CUDA;
+    e = launch_decode_finish(b, ws, stream);
+    if (e != cudaSuccess) return KVC_ERR_CUDA;
   }
-  if (e != cudaSuccess) return KVC_ERR_CUDA;
-  return cuda_status(launch_decode_finish(ds, d_res, stream));
+  return KVC_OK;
+}
+
+int encode_common(const kvc_plan_t* plan, int path, uint32_t first_slice, uint32_t n_slices,
+                  const void* d_src, void* d_dst, size_t dst_cap, void* d_ws, size_t ws_bytes,
+                  kvc_result* d_res, cudaStream_t stream) {
+  if (!path_ok(plan, path)) return plan ? KVC_ERR_UNSUPPORTED : KVC_ERR_INVALID;
+  if (ws_bytes < encode_ws_for(plan, path, uint64_t(n_slices) * records_per_slice(plan, path)))
+    return KVC_ERR_CAPACITY;
+  kvc_frame f{first_slice, n_slices, d_src, 0, d_dst, dst_cap, d_res};
+  return encode_frames(plan, path, &f, 1, d_ws, ws_bytes, stream);
+}
+
+int decode_common(const kvc_plan_t* plan, int path, const void* d_src, size_t src_bytes, void* d_dst,
+                  size_t dst_cap, void* d_ws, size_t ws_bytes, kvc_result* d_res,
+                  cudaStream_t stream) {
+  if (!path_ok(plan, path)) return plan ? KVC_ERR_UNSUPPORTED : KVC_ERR_INVALID;
+  // the workspace bounds the slices a container may hold in this call
+  const uint64_t per_slice = 8ull * records_per_slice(plan, path);
+  const uint64_t room = ws_bytes > kDecodeWsFixed ? (ws_bytes - kDecodeWsFixed) / per_slice : 0;
+  const uint32_t ms = uint32_t(std::min<uint64_t>(room, plan->S));
+  if (ms == 0) return KVC_ERR_CAPACITY;
+  kvc_frame f{0, 0, d_src, src_bytes, d_dst, dst_cap, d_res};
+  return decode_frames(plan, path, &f, 1, ms, d_ws, ws_bytes, stream);
 }
 
 }  // namespace
@@ -468,9 +545,28 @@ extern "C" size_t kvc_max_encoded_bytes(const kvc_plan_t* plan, int path, uint32
 
 extern "C" size_t kvc_workspace_bytes(const kvc_plan_t* plan, int path, int decode, uint32_t n_slices) {
   if (!path_ok(plan, path)) return 0;
-  if (decode)
-    return size_t(kDecodeStateBytes + pad256u(4ull * plan->S * records_per_slice(plan, path)));
-  return size_t(encode_ws_bytes(plan, path, n_slices));
+  if (decode) return size_t(decode_ws_for(plan, path, 1, n_slices ? n_slices : plan->S));
+  return size_t(encode_ws_for(plan, path, uint64_t(n_slices) * records_per_slice(plan, path)));
+}
+
+extern "C" size_t kvc_batch_workspace_bytes(const kvc_plan_t* plan, int path, int decode,
+                                            uint32_t n_frames, uint32_t max_slices_per_frame) {
+  if (!path_ok(plan, path)) return 0;
+  const uint32_t ms = max_slices_per_frame ? max_slices_per_frame : plan->S;
+  if (decode) return size_t(decode_ws_for(plan, path, n_frames, ms));
+  const uint64_t f = std::min<uint32_t>(std::max<uint32_t>(n_frames, 1u), kBatchMax);
+  return size_t(encode_ws_for(plan, path, f * ms * records_per_slice(plan, path)));
+}
+
+extern "C" int kvc_encode_batch(const kvc_plan_t* plan, int path, const kvc_frame* h_frames,
+                                uint32_t n_frames, void* d_ws, size_t ws_bytes, cudaStream_t stream) {
+  return encode_frames(plan, path, h_frames, n_frames, d_ws, ws_bytes, stream);
+}
+
+extern "C" int kvc_decode_batch(const kvc_plan_t* plan, int path, const kvc_frame* h_frames,
+                                uint32_t n_frames, uint32_t max_slices_per_frame, void* d_ws,
+                                size_t ws_bytes, cudaStream_t stream) {
+  return decode_frames(plan, path, h_frames, n_frames, max_slices_per_frame, d_ws, ws_bytes, stream);
 }
 
 extern "C" int kvc_encode_lossless(const kvc_plan_t* plan, uint32_t first_slice, uint32_t n_slices,

@@ -47,26 +47,33 @@ __device__ inline uint64_t block_exclusive_scan64(uint64_t v, uint64_t* tmp, uin
   return base + x - v;
 }
 
+// One CTA per frame: offsets from the frame's record lengths, the index, the
+// header and its CRC; the frame's result.
 __global__ void __launch_bounds__(kBig)
-k_finalize(HeaderFields h, EncodeLayout ws, uint8_t* dst, uint64_t dst_cap, Result* res) {
+k_finalize(HeaderFields h, FrameBatch b, EncodeLayout ws) {
   __shared__ uint32_t crc_t[1024];
   __shared__ uint32_t red[32];
   __shared__ uint64_t tmp64[32];
   const uint32_t tid = threadIdx.x, nthr = blockDim.x;
-  const uint32_t nr = h.n_records;
+  const uint32_t f = blockIdx.x;
+  const FrameDesc& fd = b.f[f];
+  const uint32_t g0 = b.rec_base[f], nr = b.rec_base[f + 1] - g0;
+  uint8_t* dst = fd.dst;
+  Result* res = static_cast<Result*>(fd.res);
+  EncodeState* es = ws.state + f;
   crc_tables_init(crc_t);
   const uint32_t per = (nr + nthr - 1) / nthr;
   const uint32_t beg = min(nr, tid * per), end = min(nr, beg + per);
   uint64_t mine = 0;
-  for (uint32_t i = beg; i < end; ++i) mine += ws.rec_len[i];
+  for (uint32_t i = beg; i < end; ++i) mine += ws.rec_len[g0 + i];
   uint64_t sum_all;
   uint64_t pre = block_exclusive_scan64(mine, tmp64, &sum_all);
   const uint64_t first = uint64_t(kHeaderBytes) + uint64_t(kIndexEntry) * nr;
   const uint64_t total = first + sum_all;
-  if (total > dst_cap) {
+  if (total > fd.dst_cap) {
     if (tid == 0) {
-      ws.state->status = kErrCapacity;
-      ws.state->total_bytes = total;
+      es->status = kErrCapacity;
+      es->total_bytes = total;
       res->status = kErrCapacity;
       res->bytes = total;
     }
@@ -74,9 +81,9 @@ k_finalize(HeaderFields h, EncodeLayout ws, uint8_t* dst, uint64_t dst_cap, Resu
   }
   uint64_t off = first + pre;
   for (uint32_t i = beg; i < end; ++i) {
-    ws.rec_off[i] = off;
-    uint32_t len = ws.rec_len[i];
-    uint4 ent = make_uint4(uint32_t(off), uint32_t(off >> 32), len, ws.rec_crc[i]);
+    ws.rec_off[g0 + i] = off;
+    uint32_t len = ws.rec_len[g0 + i];
+    uint4 ent = make_uint4(uint32_t(off), uint32_t(off >> 32), len, ws.rec_crc[g0 + i]);
     *reinterpret_cast<uint4*>(dst + kHeaderBytes + uint64_t(kIndexEntry) * i) = ent;
     off += len;
   }
@@ -85,7 +92,7 @@ k_finalize(HeaderFields h, EncodeLayout ws, uint8_t* dst, uint64_t dst_cap, Resu
     w[0] = 0x3143564bu;  // "KVC1"
     w[1] = 1u | (h.path << 16) | (h.dtype << 24);
     w[2] = h.L; w[3] = h.H; w[4] = h.T; w[5] = h.D;
-    w[6] = h.first_slice; w[7] = h.n_slices; w[8] = h.chunk_tokens; w[9] = nr;
+    w[6] = fd.first_slice; w[7] = fd.n_slices; w[8] = h.chunk_tokens; w[9] = nr;
     w[10] = uint32_t(total); w[11] = uint32_t(total >> 32);
     w[12] = h.plan_crc;
     w[13] = h.n_sink | (h.n_recent << 16);
@@ -98,32 +105,39 @@ k_finalize(HeaderFields h, EncodeLayout ws, uint8_t* dst, uint64_t dst_cap, Resu
       60ull + uint64_t(kIndexEntry) * nr, crc_t, red);
   if (tid == 0) {
     reinterpret_cast<uint32_t*>(dst)[15] = hcrc;
-    ws.state->status = kOk;
-    ws.state->n_records = nr;
-    ws.state->total_bytes = total;
+    es->status = kOk;
+    es->n_records = nr;
+    es->total_bytes = total;
     res->status = kOk;
     res->bytes = total;
   }
 }
 
-__global__ void k_copy_records(EncodeLayout ws, uint32_t nr, uint8_t* dst) {
-  if (ws.state->status != kOk) return;
-  for (uint32_t r = blockIdx.x; r < nr; r += gridDim.x) {
-    const uint4* s = reinterpret_cast<const uint4*>(ws.slots + uint64_t(r) * ws.slot_bytes);
-    uint4* d = reinterpret_cast<uint4*>(dst + ws.rec_off[r]);
-    const uint32_t q = ws.rec_len[r] / 16u;
+__global__ void k_copy_records(FrameBatch b, EncodeLayout ws) {
+  const uint32_t total = b.rec_base[b.n];
+  for (uint32_t g = blockIdx.x; g < total; g += gridDim.x) {
+    const uint32_t f = frame_of(b.rec_base, b.n, g);
+    if (ws.state[f].status != kOk) continue;
+    const uint4* s = reinterpret_cast<const uint4*>(ws.slots + uint64_t(g) * ws.slot_bytes);
+    uint4* d = reinterpret_cast<uint4*>(b.f[f].dst + ws.rec_off[g]);
+    const uint32_t q = ws.rec_len[g] / 16u;
     for (uint32_t i = threadIdx.x; i < q; i += blockDim.x) d[i] = s[i];
   }
 }
 
+// One CTA per frame: validate the header and index in the codec's fixed order.
 __global__ void __launch_bounds__(kBig)
-k_check_container(const uint8_t* src, uint64_t src_bytes, ContainerExpect e, DecodeState* ds,
-                  Result* res) {
+k_check_container(FrameBatch b, ContainerExpect e, uint8_t* ws) {
   __shared__ uint32_t crc_t[1024];
   __shared__ uint32_t red[32];
   __shared__ int st_s;
   __shared__ uint32_t nr_s, first_s, ns_s;
   const uint32_t tid = threadIdx.x, nthr = blockDim.x;
+  const uint32_t f = blockIdx.x;
+  const uint8_t* src = b.f[f].src;
+  const uint64_t src_bytes = b.f[f].src_bytes;
+  DecodeState* ds = decode_state(ws, f);
+  Result* res = static_cast<Result*>(b.f[f].res);
   crc_tables_init(crc_t);
   if (tid == 0) {
     int st = kOk;
@@ -141,6 +155,8 @@ k_check_container(const uint8_t* src, uint64_t src_bytes, ContainerExpect e, Dec
     }
     st_s = st;
     nr_s = nr;
+    first_s = 0;
+    ns_s = 0;
   }
   __syncthreads();
   uint64_t total = 0;
@@ -189,7 +205,8 @@ k_check_container(const uint8_t* src, uint64_t src_bytes, ContainerExpect e, Dec
       bad = __syncthreads_or(bad);
       if (tid == 0) {
         int st = bad ? kErrCorrupt : kOk;
-        if (st == kOk && uint64_t(ns_s) * e.T * e.D * 2u > e.dst_cap) st = kErrCapacity;
+        if (st == kOk && (uint64_t(ns_s) * e.T * e.D * 2u > b.f[f].dst_cap || ns_s > e.max_slices))
+          st = kErrCapacity;
         st_s = st;
       }
     }
@@ -202,14 +219,18 @@ k_check_container(const uint8_t* src, uint64_t src_bytes, ContainerExpect e, Dec
     ds->n_slices = st == kOk ? ns_s : 0;
     ds->n_records = st == kOk ? nr_s : 0;
     ds->err_key = ~0ull;
-    ds->n_deferred = 0;
     ds->out_bytes = st == kOk ? uint64_t(ns_s) * e.T * e.D * 2u : 0;
+    if (f == 0) batch_state(ws)->n_deferred = 0;
     res->status = st;
     res->bytes = 0;
   }
 }
 
-__global__ void k_decode_finish(const DecodeState* ds, Result* res) {
+__global__ void k_decode_finish(FrameBatch b, uint8_t* ws) {
+  const uint32_t f = threadIdx.x;
+  if (f >= b.n) return;
+  const DecodeState* ds = decode_state(ws, f);
+  Result* res = static_cast<Result*>(b.f[f].res);
   int st = ds->status;
   if (st == kOk && ds->err_key != ~0ull) st = int(ds->err_key & 0xffu);
   res->status = st;
@@ -304,36 +325,38 @@ k_stage_stream_decode(const uint8_t* rec, uint32_t rec_bytes, uint32_t n, uint8_
 
 }  // namespace
 
-cudaError_t launch_finalize(const HeaderFields& h, const EncodeLayout& ws, uint8_t* dst,
-                            uint64_t dst_cap, void* res, cudaStream_t st) {
+cudaError_t launch_finalize(const HeaderFields& h, const FrameBatch& b, const EncodeLayout& ws,
+                            cudaStream_t st) {
+  if (b.n == 0) return cudaSuccess;
   {
     ProfRange pr_("finalize", st);
-    k_finalize<<<1, kBig, 0, st>>>(h, ws, dst, dst_cap, static_cast<Result*>(res));
+    k_finalize<<<b.n, kBig, 0, st>>>(h, b, ws);
   }
   cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || h.n_records == 0) return e;
-  uint32_t grid = min(h.n_records, 148u * 8u);
+  const uint32_t total = b.rec_base[b.n];
+  if (e != cudaSuccess || total == 0) return e;
   {
     ProfRange pr_("copy_records", st);
-    k_copy_records<<<grid, 256, 0, st>>>(ws, h.n_records, dst);
+    k_copy_records<<<min(total, 148u * 8u), 256, 0, st>>>(b, ws);
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_check_container(const uint8_t* src, uint64_t src_bytes,
-                                   const ContainerExpect& e, DecodeState* ds, void* res,
+cudaError_t launch_check_container(const FrameBatch& b, const ContainerExpect& e, uint8_t* ws,
                                    cudaStream_t st) {
+  if (b.n == 0) return cudaSuccess;
   {
     ProfRange pr_("check_container", st);
-    k_check_container<<<1, kBig, 0, st>>>(src, src_bytes, e, ds, static_cast<Result*>(res));
+    k_check_container<<<b.n, kBig, 0, st>>>(b, e, ws);
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode_finish(DecodeState* ds, void* res, cudaStream_t st) {
+cudaError_t launch_decode_finish(const FrameBatch& b, uint8_t* ws, cudaStream_t st) {
+  if (b.n == 0) return cudaSuccess;
   {
     ProfRange pr_("decode_finish", st);
-    k_decode_finish<<<1, 1, 0, st>>>(ds, static_cast<Result*>(res));
+    k_decode_finish<<<1, kBatchMax, 0, st>>>(b, ws);
   }
   return cudaGetLastError();
 }

@@ -180,7 +180,7 @@ __device__ inline uint32_t crc32_block_aligned(const uint8_t* p, uint32_t len, c
     for (uint32_t k = 0; k < kCrcRun; k += 16) {
       int64_t off = run0 + k;
       if (off < 0) continue;
-      uint4 v = *reinterpret_cast<const uint4*>(p + off);
+      uint4 v = __ldcg(reinterpret_cast<const uint4*>(p + off));
       if (off == 0) v.x = ~v.x;
       c = crc_word(t, c, v.x);
       c = crc_word(t, c, v.y);
@@ -224,6 +224,86 @@ __device__ inline uint32_t crc32_block_bytes(Fetch fetch, uint64_t len, const ui
   // under four bytes the initial register is shifted through the message instead
   if (len < 4) total ^= gf2_mul(0xffffffffu, gf2_xpow8(len));
   return total ^ 0xffffffffu;
+}
+
+// One-round block CRC for records up to kCrcOneRound bytes: thread t owns the
+// run [t R, (t + 1) R) of the record padded in front to 128 R bytes (R = 1040),
+// so every shift in the join is a compile-time constant: x^(8 R 2^l). Joins
+// multiply by those constants with per-nibble tables (8 lookups instead of a
+// 32-step bitwise product). The tables are built once per CTA.
+constexpr uint32_t kCrcRunR = 1040;                       // 65 x 16 bytes
+constexpr uint32_t kCrcOneRound = 128u * kCrcRunR;        // 133120 bytes
+struct CrcJoin {
+  uint32_t nib[8][8][16];  // [level][nibble position][value]: (v << 4 pos) * x^(8 R 2^level)
+};
+struct CrcRunShifts { uint32_t v[8]; };
+constexpr CrcRunShifts make_run_shifts() {
+  CrcRunShifts s{};
+  for (int l = 0; l < 8; ++l) s.v[l] = gf2_xpow8(uint64_t(kCrcRunR) << l);
+  return s;
+}
+__constant__ CrcRunShifts kCrcRunShift = make_run_shifts();
+
+__device__ inline void crc_join_init(CrcJoin* J) {
+  for (uint32_t i = threadIdx.x; i < 8 * 8 * 16; i += blockDim.x) {
+    const uint32_t l = i >> 7, pos = (i >> 4) & 7u, val = i & 15u;
+    J->nib[l][pos][val] = gf2_mul(val << (4 * pos), kCrcRunShift.v[l]);
+  }
+  __syncthreads();
+}
+__device__ inline uint32_t crc_join_mul(const CrcJoin* J, uint32_t level, uint32_t a) {
+  uint32_t r = 0;
+#pragma unroll
+  for (uint32_t pos = 0; pos < 8; ++pos) r ^= J->nib[level][pos][(a >> (4 * pos)) & 15u];
+  return r;
+}
+
+// CRC-32 of len (multiple of 16, <= kCrcOneRound) bytes at p (16-byte aligned)
+// by a block of exactly 128 threads; result valid in thread 0.
+__device__ inline uint32_t crc32_block_128(const uint8_t* p, uint32_t len, const uint32_t* t,
+                                           const CrcJoin* J, uint32_t* red) {
+  const uint32_t pad = kCrcOneRound - len;
+  const int64_t run0 = int64_t(threadIdx.x) * kCrcRunR - int64_t(pad);
+  uint32_t c = 0;
+  if (run0 + int64_t(kCrcRunR) > 0) {
+    // 65 vectors per run, loaded five at a time so five loads are in flight
+    const uint32_t k0 = run0 < 0 ? uint32_t(-run0) / 16u : 0u;  // first real vector
+    for (uint32_t kb = 0; kb < kCrcRunR / 16u; kb += 5) {
+      uint4 v[5];
+#pragma unroll
+      for (uint32_t i = 0; i < 5; ++i) {
+        const uint32_t k = kb + i;
+        v[i] = k >= k0 ? __ldcg(reinterpret_cast<const uint4*>(p + uint32_t(run0 + 16 * int64_t(k))))
+                       : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (uint32_t i = 0; i < 5; ++i) {
+        const uint32_t k = kb + i;
+        if (k < k0) continue;
+        if (run0 + 16 * int64_t(k) == 0) v[i].x = ~v[i].x;
+        c = crc_word(t, c, v[i].x);
+        c = crc_word(t, c, v[i].y);
+        c = crc_word(t, c, v[i].z);
+        c = crc_word(t, c, v[i].w);
+      }
+    }
+  }
+  const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (uint32_t l = 0; l < 5; ++l) {
+    const uint32_t other = __shfl_down_sync(0xffffffffu, c, 1u << l);
+    if ((lane & ((2u << l) - 1u)) == 0) c = crc_join_mul(J, l, c) ^ other;
+  }
+  __syncthreads();
+  if (lane == 0) red[warp] = c;
+  __syncthreads();
+  uint32_t total = 0;
+  if (threadIdx.x == 0) {
+    const uint32_t a = crc_join_mul(J, 5, red[0]) ^ red[1];
+    const uint32_t b = crc_join_mul(J, 5, red[2]) ^ red[3];
+    total = crc_join_mul(J, 6, a) ^ b;
+  }
+  return len ? (total ^ 0xffffffffu) : 0u;
 }
 
 // ---------------------------------------------------------------- block helpers
@@ -338,8 +418,9 @@ __device__ inline void block_enc_tables(const uint32_t* freq, uint32_t* fc, uint
   __syncthreads();
 }
 
-// Decode table: lut[slot] = symbol | f << 8 | (slot - cum) << 20, and the
+// Decode table: lut[slot] = (slot - cum_s) | f_s << 12 | s << 24, and the
 // symbols' cumulative starts in cum[257]. freq must be validated (sum 4096).
+// Each thread fills a contiguous run of slots, walking the symbols forward.
 __device__ inline void block_dec_lut(const uint32_t* freq, uint32_t* cum, uint32_t* lut,
                                      uint32_t* tmp) {
   const uint32_t per = blockDim.x >= 256 ? 1u : 256u / blockDim.x;
@@ -354,14 +435,25 @@ __device__ inline void block_dec_lut(const uint32_t* freq, uint32_t* cum, uint32
   }
   if (threadIdx.x == 0) cum[256] = kProbScale;
   __syncthreads();
-  for (uint32_t slot = threadIdx.x; slot < kProbScale; slot += blockDim.x) {
-    uint32_t lo = 0, hi = 255;  // largest symbol with cum <= slot
-    while (lo < hi) {
-      uint32_t mid = (lo + hi + 1) >> 1;
-      if (cum[mid] <= slot) lo = mid; else hi = mid - 1;
+  // lane j of warp w fills slots base_w + j + 32 i (i = 0 .. per_lane - 1): one
+  // bank per lane, ascending slots per lane so the symbol walk only moves forward
+  const uint32_t nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
+  const uint32_t span = kProbScale / nw, per_lane = span / 32u;
+  const uint32_t first = warp * span + lane;
+  uint32_t lo = 0, hi = 255;  // largest symbol with cum <= first
+  while (lo < hi) {
+    const uint32_t mid = (lo + hi + 1) >> 1;
+    if (cum[mid] <= first) lo = mid; else hi = mid - 1;
+  }
+  uint32_t sym = lo, cs = cum[sym], ce = cum[sym + 1];
+  for (uint32_t i = 0; i < per_lane; ++i) {
+    const uint32_t slot = first + 32u * i;
+    while (slot >= ce) {  // next symbol with a nonzero frequency
+      ++sym;
+      cs = ce;
+      ce = cum[sym + 1];
     }
-    uint32_t fs = cum[lo + 1] - cum[lo];
-    lut[slot] = lo | (fs << 8) | ((slot - cum[lo]) << 20);
+    lut[slot] = (slot - cs) | ((ce - cs) << 12) | (sym << 24);
   }
   __syncthreads();
 }
@@ -434,8 +526,8 @@ __device__ inline bool rans_decode_group(const uint8_t* sub, uint32_t sub_len, u
     const bool act = live && tau < len;
     if (act) {
       uint32_t e = lut[x & (kProbScale - 1u)];
-      x = ((e >> 8) & 0xfffu) * (x >> kProbBits) + (e >> 20);
-      out(start + tau, e & 0xffu);
+      x = ((e >> 12) & 0xfffu) * (x >> kProbBits) + (e & 0xfffu);
+      out(start + tau, e >> 24);
     }
     bool need = act && x < kRansLow;
     uint32_t mask = __ballot_sync(0xffffffffu, need);
@@ -475,10 +567,12 @@ __device__ inline int block_parse_stream(const uint8_t* rec, uint32_t avail, uin
     int st = kOk;
     if (avail < 16) st = kErrCorrupt;
     else {
-      uint32_t mode = rec[0], csym = rec[1], G = rec[2];
-      uint32_t bytes = ld_u32(rec + 4), rn = ld_u32(rec + 8), k = ld_u32(rec + 12);
+      const uint4 hv = __ldg(reinterpret_cast<const uint4*>(rec));  // records are 16-byte aligned
+      uint32_t mode = hv.x & 0xffu, csym = (hv.x >> 8) & 0xffu, G = (hv.x >> 16) & 0xffu;
+      uint32_t bytes = hv.y, rn = hv.z, k = hv.w;
+      const uint32_t b3 = hv.x >> 24;
       si->mode = mode; si->sym = csym; si->groups = G; si->bytes = bytes; si->k = k;
-      if (rec[3] != 0 || rn != n || (bytes & 15u) || bytes < 16 || bytes > avail) st = kErrCorrupt;
+      if (b3 != 0 || rn != n || (bytes & 15u) || bytes < 16 || bytes > avail) st = kErrCorrupt;
       else if (mode == kModeRaw) {
         if (csym || G || k || bytes != 16u + pad16(n)) st = kErrCorrupt;
       } else if (mode == kModeConst) {
@@ -491,8 +585,13 @@ __device__ inline int block_parse_stream(const uint8_t* rec, uint32_t avail, uin
           uint32_t lens_at = p;
           p = pad16(p + 4u * G);
           if (p > bytes) st = kErrCorrupt;
+          uint32_t lens[4] = {0, 0, 0, 0};
+          if (st == kOk) {  // G <= 4 lengths in one aligned 16-byte load
+            const uint4 lv = __ldg(reinterpret_cast<const uint4*>(rec + lens_at));
+            lens[0] = lv.x; lens[1] = lv.y; lens[2] = lv.z; lens[3] = lv.w;
+          }
           for (uint32_t g = 0; g < G && st == kOk; ++g) {
-            uint32_t sl = ld_u32(rec + lens_at + 4u * g);
+            uint32_t sl = lens[g];
             if (sl > bytes || p + pad16(sl) > bytes) { st = kErrCorrupt; break; }
             si->sub_off[g] = p;
             si->sub_len[g] = sl;

@@ -27,26 +27,59 @@ struct ProfRange {
   }
 };
 
-// Decoder workspace (device): header/index verdict and the first failing record.
+// A group of up to kBatchMax frames (independent containers) coded by one
+// launch per kernel; passed to kernels by value.
+constexpr uint32_t kBatchMax = 64;
+struct FrameDesc {
+  const uint8_t* src;   // encode: values; decode: container
+  uint8_t* dst;         // encode: container; decode: values
+  void* res;            // kvc_result
+  uint64_t src_bytes, dst_cap;
+  uint32_t first_slice, n_slices;
+};
+struct FrameBatch {
+  uint32_t n;
+  uint32_t rec_base[kBatchMax + 1];  // encode: first global record of each frame
+  FrameDesc f[kBatchMax];
+};
+
+// Decoder workspace: one DecodeState per frame of the group, then the batch
+// state and the list of records the fast decoders deferred.
 struct DecodeState {
   int status;                  // container-level status (header, index, capacity)
   uint32_t first_slice, n_slices, n_records;
   unsigned long long err_key;  // min over failing records of (record << 8) | status
   uint64_t out_bytes;
-  uint32_t n_deferred;         // records the fast decoder left to the general one
-  uint32_t reserved;
 };
-// the deferred-record list follows the state in the decode workspace
 constexpr uint32_t kDecodeStateBytes = 256;
-inline __host__ __device__ uint32_t* deferred_list(DecodeState* ds) {
-  return reinterpret_cast<uint32_t*>(reinterpret_cast<uint8_t*>(ds) + kDecodeStateBytes);
+struct BatchDecodeState {
+  uint32_t n_deferred;
+};
+inline __host__ __device__ DecodeState* decode_state(uint8_t* ws, uint32_t f) {
+  return reinterpret_cast<DecodeState*>(ws + uint64_t(f) * kDecodeStateBytes);
 }
+inline __host__ __device__ BatchDecodeState* batch_state(uint8_t* ws) {
+  return reinterpret_cast<BatchDecodeState*>(ws + uint64_t(kBatchMax) * kDecodeStateBytes);
+}
+inline __host__ __device__ unsigned long long* deferred_list(uint8_t* ws) {
+  return reinterpret_cast<unsigned long long*>(ws + uint64_t(kBatchMax + 1) * kDecodeStateBytes);
+}
+constexpr uint64_t kDecodeWsFixed = uint64_t(kBatchMax + 1) * kDecodeStateBytes;
 
-// Encoder workspace header (device), followed by per-record arrays and slots.
+// Encoder workspace (device): per frame an EncodeState, per global record its
+// length, CRC and container offset, then one slot per record.
 struct EncodeState {
   int status;
   uint32_t n_records;
   uint64_t total_bytes;
+};
+struct EncodeLayout {
+  EncodeState* state;   // [frames]
+  uint32_t* rec_len;    // [records]
+  uint32_t* rec_crc;
+  uint64_t* rec_off;
+  uint8_t* slots;
+  uint64_t slot_bytes;
 };
 
 // What a valid container header must carry for this plan.
@@ -54,40 +87,42 @@ struct ContainerExpect {
   uint32_t path, dtype, L, H, T, D, chunk_tokens;
   uint32_t n_sink, n_recent, block_tokens, plan_crc;
   uint32_t recs_per_slice;     // records per slice
-  uint64_t dst_cap;            // decode output capacity in bytes
+  uint32_t max_slices;         // slices a container may hold in this call
 };
 
-struct EncodeLayout {          // workspace carve-up for an encode call
-  EncodeState* state;
-  uint32_t* rec_len;
-  uint32_t* rec_crc;
-  uint64_t* rec_off;
-  uint8_t* slots;
-  uint64_t slot_bytes;
-};
-
-// header writer / record copier shared by both paths
+// header fields common to the frames of a batch
 struct HeaderFields {
-  uint32_t path, dtype, L, H, T, D, first_slice, n_slices, chunk_tokens, n_records;
+  uint32_t path, dtype, L, H, T, D, chunk_tokens, recs_per_slice;
   uint32_t plan_crc, n_sink, n_recent, block_tokens;
 };
 
-cudaError_t launch_finalize(const HeaderFields& h, const EncodeLayout& ws, uint8_t* dst,
-                            uint64_t dst_cap, void* res, cudaStream_t st);
-cudaError_t launch_check_container(const uint8_t* src, uint64_t src_bytes,
-                                   const ContainerExpect& e, DecodeState* ds, void* res,
+cudaError_t launch_finalize(const HeaderFields& h, const FrameBatch& b, const EncodeLayout& ws,
+                            cudaStream_t st);
+cudaError_t launch_check_container(const FrameBatch& b, const ContainerExpect& e, uint8_t* ws,
                                    cudaStream_t st);
-cudaError_t launch_decode_finish(DecodeState* ds, void* res, cudaStream_t st);
+cudaError_t launch_decode_finish(const FrameBatch& b, uint8_t* ws, cudaStream_t st);
+
+#ifdef __CUDACC__
+// frame of global record g: largest f with rec_base[f] <= g
+__device__ inline uint32_t frame_of(const uint32_t* base, uint32_t n, uint32_t g) {
+  uint32_t lo = 0, hi = n - 1;
+  while (lo < hi) {
+    const uint32_t mid = (lo + hi + 1) >> 1;
+    if (base[mid] <= g) lo = mid; else hi = mid - 1;
+  }
+  return lo;
+}
+#endif
 
 // lossless
 struct LosslessShape {
   uint32_t T, D, tc, cps;      // tokens, head_dim, chunk tokens, chunks per slice
 };
 uint64_t lossless_slot_bytes(const LosslessShape& s);
-cudaError_t launch_lossless_encode(const LosslessShape& s, const uint16_t* src, uint32_t n_slices,
+cudaError_t launch_lossless_encode(const LosslessShape& s, const FrameBatch& b,
                                    const EncodeLayout& ws, cudaStream_t st);
-cudaError_t launch_lossless_decode(const LosslessShape& s, const uint8_t* src, uint16_t* dst,
-                                   DecodeState* ds, uint32_t max_records, cudaStream_t st);
+cudaError_t launch_lossless_decode(const LosslessShape& s, const FrameBatch& b, uint8_t* ws,
+                                   uint32_t max_records, cudaStream_t st);
 
 // transform coding
 struct TransformShape {
@@ -103,11 +138,10 @@ struct TransformPlanDev {
 constexpr uint32_t kQSplitBytes = 2u * 128u * 256u;  // per slice
 uint64_t transform_slot_bytes(const TransformShape& s);
 cudaError_t launch_transform_encode(const TransformShape& s, const TransformPlanDev& p,
-                                    const uint16_t* src, uint32_t first_slice, uint32_t n_slices,
-                                    const EncodeLayout& ws, cudaStream_t st);
+                                    const FrameBatch& b, const EncodeLayout& ws, cudaStream_t st);
 cudaError_t launch_transform_decode(const TransformShape& s, const TransformPlanDev& p,
-                                    const uint8_t* src, uint16_t* dst, DecodeState* ds,
-                                    uint32_t max_records, cudaStream_t st);
+                                    const FrameBatch& b, uint8_t* ws, uint32_t max_records,
+                                    cudaStream_t st);
 
 // stage entry points
 cudaError_t launch_stage_crc32(const uint8_t* src, uint64_t n, uint32_t* out, cudaStream_t st);

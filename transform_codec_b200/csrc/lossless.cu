@@ -4,6 +4,7 @@
 // page, "KV & tensor mode": channel-major reorder, byte planes, keep whichever
 // is smaller; QATQ page, "qatq encode": bounded chunks, known row width).
 #include "kvc_device.cuh"
+#include "tcgen05.cuh"
 #include "kvc_internal.h"
 
 namespace kvc {
@@ -46,12 +47,15 @@ struct ChanMajor {
 };
 
 __global__ void __launch_bounds__(kThreads)
-k_lossless_encode(LosslessShape sh, const uint16_t* __restrict__ src, EncodeLayout ws) {
+k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   EncSmem& S = *reinterpret_cast<EncSmem*>(smem_raw);
   uint16_t* vals = reinterpret_cast<uint16_t*>(smem_raw + sizeof(EncSmem));
   const uint32_t tid = threadIdx.x, nthr = blockDim.x;
-  const uint32_t r = blockIdx.x;
+  const uint32_t gr = blockIdx.x;  // record of the batch
+  const uint32_t fr = frame_of(b.rec_base, b.n, gr);
+  const uint32_t r = gr - b.rec_base[fr];
+  const uint16_t* src = reinterpret_cast<const uint16_t*>(b.f[fr].src);
   const uint32_t slice = r / sh.cps, c = r % sh.cps;
   const uint32_t t0 = c * sh.tc, tcc = min(sh.tc, sh.T - t0), D = sh.D, n = tcc * D;
   const uint32_t n_max = sh.tc * D;
@@ -81,7 +85,7 @@ k_lossless_encode(LosslessShape sh, const uint16_t* __restrict__ src, EncodeLayo
 
   const ChanMajor cm(tcc);
   const uint32_t N = rans_lanes(n), G = rans_groups(N);
-  uint8_t* slot = ws.slots + uint64_t(r) * ws.slot_bytes;
+  uint8_t* slot = ws.slots + uint64_t(gr) * ws.slot_bytes;
   const uint32_t rec_area = 2u * (16u + pad16(n_max));
   uint16_t* scratch[2] = {reinterpret_cast<uint16_t*>(slot + rec_area),
                           reinterpret_cast<uint16_t*>(slot + rec_area + 2u * n_max + 64u)};
@@ -139,29 +143,30 @@ k_lossless_encode(LosslessShape sh, const uint16_t* __restrict__ src, EncodeLayo
   __syncthreads();
   uint32_t crc = crc32_block_aligned(rec, off, S.crc_t, S.red);
   if (tid == 0) {
-    ws.rec_len[r] = off;
-    ws.rec_crc[r] = crc;
+    ws.rec_len[gr] = off;
+    ws.rec_crc[gr] = crc;
   }
 }
 
 // General decoder: any chunk shape and any plane modes; stages both planes in
 // shared memory (one CTA per SM). Runs the records the fast decoder deferred.
 __global__ void __launch_bounds__(kThreads)
-k_lossless_decode(LosslessShape sh, const uint8_t* __restrict__ src, uint16_t* __restrict__ dst,
-                  DecodeState* ds) {
+k_lossless_decode(LosslessShape sh, FrameBatch b, uint8_t* ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   DecSmem& S = *reinterpret_cast<DecSmem*>(smem_raw);
   const uint32_t tid = threadIdx.x, nthr = blockDim.x;
   const uint32_t D = sh.D, n_max = sh.tc * D;
   uint8_t* planes[2] = {smem_raw + sizeof(DecSmem), smem_raw + sizeof(DecSmem) + pad16(n_max)};
-  if (ds->status != kOk) return;
-  const uint32_t n_todo = ds->n_deferred;
+  const uint32_t n_todo = batch_state(ws)->n_deferred;
   if (blockIdx.x >= n_todo) return;
-  const uint32_t* todo = deferred_list(ds);
+  const unsigned long long* todo = deferred_list(ws);
   crc_tables_init(S.crc_t);
   for (uint32_t i = blockIdx.x; i < n_todo; i += gridDim.x) {
     __syncthreads();
-    const uint32_t r = todo[i];
+    const uint32_t fr = uint32_t(todo[i] >> 32), r = uint32_t(todo[i]);
+    const uint8_t* src = b.f[fr].src;
+    uint16_t* dst = reinterpret_cast<uint16_t*>(b.f[fr].dst);
+    DecodeState* ds = decode_state(ws, fr);
     const uint8_t* e = src + kHeaderBytes + uint64_t(kIndexEntry) * r;
     const uint64_t off = ld_u64(e);
     const uint32_t len = ld_u32(e + 8), want = ld_u32(e + 12);
@@ -258,106 +263,196 @@ struct __align__(16) FastSmem {
   uint32_t cum[260];
   uint32_t tmp[32], red[32];
   StreamInfo si[2];
+  uint16_t ring[kFastThreads / 32][1024];  // per-group window of rANS refill words
+  CrcJoin join;
+  uint32_t base[kBatchMax + 1];
   uint32_t crc_ok;
 };
 
+// One rANS lane of a 32-lane group (warp-synchronous). Refill words come from
+// the group's window in shared memory (word i at ring[i % 1024]); a lane whose
+// index runs past the sub-stream marks the record bad and its state is junk.
 struct LaneRans {
   uint32_t x, pos, W;
-  const uint16_t* w16;
-  bool bad;
-  __device__ inline uint32_t step(const uint32_t* lut, uint32_t lt) {
+  const uint16_t* ring;
+  uint32_t bad;
+  __device__ __forceinline__ uint32_t step(const uint32_t* lut, uint32_t lt) {
     const uint32_t e = lut[x & (kProbScale - 1u)];
-    x = ((e >> 8) & 0xfffu) * (x >> kProbBits) + (e >> 20);
+    x = ((e >> 12) & 0xfffu) * (x >> kProbBits) + (e & 0xfffu);
     const bool need = x < kRansLow;
     const uint32_t mask = __ballot_sync(0xffffffffu, need);
-    if (need) {
-      const uint32_t idx = pos + __popc(mask & lt);
-      if (idx < W) x = (x << 16) | w16[idx];
-      else bad = true;
-    }
+    const uint32_t idx = pos + __popc(mask & lt);
+    const uint32_t w = ring[idx & 1023u];
+    x = need ? ((x << 16) | w) : x;
+    bad |= uint32_t(need && idx >= W);
     pos += __popc(mask);
-    return e & 0xffu;
+    return e >> 24;
   }
 };
 
-template <uint32_t M0, uint32_t M1>
-__device__ inline bool fast_tiles(FastSmem& S, const uint8_t* const recp[2], uint16_t* out,
-                                  uint32_t D, uint32_t lpc_log2) {
+// The refill window of one group: 16-byte units of the sub-stream's words are
+// copied asynchronously into a 1024-word ring. At every stage (8 decode steps,
+// at most 256 words consumed) the group waits for all but the newest copy
+// group, then requests units up to 1024 words past the unit holding `pos`, so
+// a unit is only overwritten once every word in it has been consumed and the
+// words of the coming stage were requested at least one stage earlier. Units
+// past the last word stay inside the record: sub-streams are padded to 16
+// bytes and start 16-byte aligned.
+struct RefillWindow {
+  const uint8_t* units;  // first refill word, 16-byte aligned
+  uint32_t n_units, loaded, ring_saddr;
+  __device__ __forceinline__ void request(uint32_t pos, uint32_t lane) {
+    const uint32_t target = min(n_units, (pos >> 3) + 128u);
+    for (uint32_t u = loaded + lane; u < target; u += 32u)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ring_saddr + ((u & 127u) << 4)),
+                   "l"(units + (uint64_t(u) << 4))
+                   : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    loaded = max(loaded, target);
+  }
+  __device__ __forceinline__ void settle() {  // all but the newest group landed, visible to the warp
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+    __syncwarp();
+  }
+};
+
+// value of step j: byte (j % 4) of raw word r (plane 0) and decoded symbol (plane 1),
+// or the other way round, merged into one 16-bit value
+__device__ __forceinline__ uint32_t merge_raw_lo(uint32_t r, uint32_t j, uint32_t hi) {
+  return __byte_perm(r, hi, (j & 3u) | 0x40u);  // byte0 = r.byte(j%4), byte1 = hi.byte0
+}
+__device__ __forceinline__ uint32_t merge_raw_hi(uint32_t r, uint32_t j, uint32_t lo) {
+  return __byte_perm(lo, r, 0u | ((4u + (j & 3u)) << 4));  // byte0 = lo.byte0, byte1 = r.byte(j%4)
+}
+
+template <uint32_t M0, uint32_t M1, uint32_t D>
+__device__ inline bool fast_tiles(FastSmem& S, const uint8_t* const recp[2], uint16_t* out) {
+  constexpr uint32_t LPC = 128u / D;  // lanes per channel
   const uint32_t l = threadIdx.x, lane = l & 31u, g = l >> 5;
   const uint32_t lt = lanemask_lt();
-  const uint32_t lpc = 1u << lpc_log2;
-  const uint32_t tbase = (l & (lpc - 1u)) * 32u * D + (l >> lpc_log2);
-  LaneRans rs{kRansLow, 0, 0, nullptr, false};
+  const uint32_t tbase = (l % LPC) * 32u * D + (l / LPC);
+  uint16_t* tile = S.tile + tbase;
+  LaneRans rs{kRansLow, 0, 0, S.ring[g], 0};
+  RefillWindow win{nullptr, 0, 0, tc::smem_addr(S.ring[g])};
   const uint8_t* raw0 = recp[0] + 16 + l * 512u;
   const uint8_t* raw1 = recp[1] + 16 + l * 512u;
   const uint32_t c0 = S.si[0].sym, c1 = S.si[1].sym;
+  constexpr bool kRans = (M0 == kModeRans || M1 == kModeRans);
   constexpr uint32_t RP = (M0 == kModeRans) ? 0u : 1u;  // the rANS plane, if any
-  if (M0 == kModeRans || M1 == kModeRans) {
+  if (kRans) {
     const StreamInfo& si = S.si[RP];
     const uint8_t* sub = recp[RP] + si.sub_off[g];
     const uint32_t sl = si.sub_len[g];
-    if (sl < 128u || (sl & 1u)) rs.bad = true;
+    if (sl < 128u || (sl & 1u)) rs.bad = 1;
     else {
       rs.x = reinterpret_cast<const uint32_t*>(sub)[lane];
       rs.W = (sl - 128u) >> 1;
-      rs.w16 = reinterpret_cast<const uint16_t*>(sub + 128);
+      win.units = sub + 128;
+      win.n_units = (rs.W + 7u) >> 3;
     }
   }
-  const bool live = __all_sync(0xffffffffu, !rs.bad);
+  const bool live = __all_sync(0xffffffffu, rs.bad == 0);
+  uint4 n0a = make_uint4(0, 0, 0, 0), n0b = n0a, n1a = n0a, n1b = n0a;  // next tile's raw bytes
+  if (M0 == kModeRaw) { n0a = __ldcs(reinterpret_cast<const uint4*>(raw0)); n0b = __ldcs(reinterpret_cast<const uint4*>(raw0 + 16)); }
+  if (M1 == kModeRaw) { n1a = __ldcs(reinterpret_cast<const uint4*>(raw1)); n1b = __ldcs(reinterpret_cast<const uint4*>(raw1 + 16)); }
+  if (kRans && !live) return false;
+  if (kRans) {
+    win.request(0, lane);
+    asm volatile("cp.async.commit_group;" ::: "memory");  // empty group: the first settle waits for the window
+  }
   for (uint32_t k = 0; k < 16; ++k) {
     uint32_t r0[8], r1[8];
     if (M0 == kModeRaw) {
-      const uint4 a = *reinterpret_cast<const uint4*>(raw0 + 32u * k);
-      const uint4 b = *reinterpret_cast<const uint4*>(raw0 + 32u * k + 16u);
-      r0[0] = a.x; r0[1] = a.y; r0[2] = a.z; r0[3] = a.w;
-      r0[4] = b.x; r0[5] = b.y; r0[6] = b.z; r0[7] = b.w;
+      r0[0] = n0a.x; r0[1] = n0a.y; r0[2] = n0a.z; r0[3] = n0a.w;
+      r0[4] = n0b.x; r0[5] = n0b.y; r0[6] = n0b.z; r0[7] = n0b.w;
+      if (k + 1 < 16) {
+        n0a = __ldcs(reinterpret_cast<const uint4*>(raw0 + 32u * (k + 1)));
+        n0b = __ldcs(reinterpret_cast<const uint4*>(raw0 + 32u * (k + 1) + 16u));
+      }
     }
     if (M1 == kModeRaw) {
-      const uint4 a = *reinterpret_cast<const uint4*>(raw1 + 32u * k);
-      const uint4 b = *reinterpret_cast<const uint4*>(raw1 + 32u * k + 16u);
-      r1[0] = a.x; r1[1] = a.y; r1[2] = a.z; r1[3] = a.w;
-      r1[4] = b.x; r1[5] = b.y; r1[6] = b.z; r1[7] = b.w;
+      r1[0] = n1a.x; r1[1] = n1a.y; r1[2] = n1a.z; r1[3] = n1a.w;
+      r1[4] = n1b.x; r1[5] = n1b.y; r1[6] = n1b.z; r1[7] = n1b.w;
+      if (k + 1 < 16) {
+        n1a = __ldcs(reinterpret_cast<const uint4*>(raw1 + 32u * (k + 1)));
+        n1b = __ldcs(reinterpret_cast<const uint4*>(raw1 + 32u * (k + 1) + 16u));
+      }
     }
 #pragma unroll
     for (uint32_t j = 0; j < 32; ++j) {
-      uint32_t lo, hi;
-      if (M0 == kModeRaw) lo = (r0[j >> 2] >> (8u * (j & 3u))) & 0xffu;
-      else if (M0 == kModeConst) lo = c0;
-      else lo = live ? rs.step(S.lut, lt) : 0u;
-      if (M1 == kModeRaw) hi = (r1[j >> 2] >> (8u * (j & 3u))) & 0xffu;
-      else if (M1 == kModeConst) hi = c1;
-      else hi = live ? rs.step(S.lut, lt) : 0u;
-      S.tile[tbase + j * D] = uint16_t(lo | (hi << 8));
+      if (kRans && (j & 7u) == 0) {
+        win.settle();
+        win.request(rs.pos, lane);
+      }
+      uint32_t v;
+      if (M0 == kModeRaw && M1 == kModeRans) v = merge_raw_lo(r0[j >> 2], j, rs.step(S.lut, lt));
+      else if (M0 == kModeRans && M1 == kModeRaw) v = merge_raw_hi(r1[j >> 2], j, rs.step(S.lut, lt));
+      else if (M0 == kModeRaw && M1 == kModeRaw) v = __byte_perm(r0[j >> 2], r1[j >> 2], (j & 3u) | ((4u + (j & 3u)) << 4));
+      else if (M0 == kModeRaw && M1 == kModeConst) v = merge_raw_lo(r0[j >> 2], j, c1);
+      else if (M0 == kModeConst && M1 == kModeRaw) v = merge_raw_hi(r1[j >> 2], j, c0);
+      else if (M0 == kModeRans && M1 == kModeConst) v = rs.step(S.lut, lt) | (c1 << 8);
+      else if (M0 == kModeConst && M1 == kModeRans) v = c0 | (rs.step(S.lut, lt) << 8);
+      else v = c0 | (c1 << 8);
+      tile[j * D] = uint16_t(v);
     }
     __syncthreads();
-    // tile = lpc blocks of 32 token rows x D channels, each contiguous in the output
-    const uint32_t per_block = 4u * D;  // uint4 per block
-    for (uint32_t q = l; q < 512u; q += kFastThreads) {
-      const uint32_t s = q / per_block, w = q - s * per_block;
-      uint4* o = reinterpret_cast<uint4*>(out + (uint64_t(s) * 512u + 32u * k) * D);
+    // tile = LPC blocks of 32 token rows x D channels, each contiguous in the output
+    constexpr uint32_t per_block = 4u * D;  // uint4 per block
+#pragma unroll
+    for (uint32_t i = 0; i < 4; ++i) {
+      const uint32_t q = l + i * kFastThreads;
+      const uint32_t sblk = q / per_block, w = q % per_block;
+      uint4* o = reinterpret_cast<uint4*>(out + (uint64_t(sblk) * 512u + 32u * k) * D);
       o[w] = reinterpret_cast<const uint4*>(S.tile)[q];
     }
     __syncthreads();
   }
-  bool ok = !rs.bad;
-  if (M0 == kModeRans || M1 == kModeRans) ok = ok && live && rs.pos == rs.W && rs.x == kRansLow;
+  if (kRans) asm volatile("cp.async.wait_group 0;" ::: "memory");  // no copy outlives the record
+  bool ok = rs.bad == 0;
+  if (kRans) ok = ok && rs.pos == rs.W && rs.x == kRansLow;
   return ok;
 }
 
+template <uint32_t D>
+__device__ inline bool fast_dispatch(FastSmem& S, const uint8_t* const recp[2], uint16_t* out,
+                                     uint32_t m0, uint32_t m1) {
+  if (m0 == kModeRaw && m1 == kModeRans) return fast_tiles<kModeRaw, kModeRans, D>(S, recp, out);
+  if (m0 == kModeRaw && m1 == kModeRaw) return fast_tiles<kModeRaw, kModeRaw, D>(S, recp, out);
+  if (m0 == kModeRaw && m1 == kModeConst) return fast_tiles<kModeRaw, kModeConst, D>(S, recp, out);
+  if (m0 == kModeRans && m1 == kModeRaw) return fast_tiles<kModeRans, kModeRaw, D>(S, recp, out);
+  if (m0 == kModeRans && m1 == kModeConst) return fast_tiles<kModeRans, kModeConst, D>(S, recp, out);
+  if (m0 == kModeConst && m1 == kModeRans) return fast_tiles<kModeConst, kModeRans, D>(S, recp, out);
+  if (m0 == kModeConst && m1 == kModeRaw) return fast_tiles<kModeConst, kModeRaw, D>(S, recp, out);
+  return fast_tiles<kModeConst, kModeConst, D>(S, recp, out);
+}
+
 __global__ void __launch_bounds__(kFastThreads)
-k_lossless_decode_fast(LosslessShape sh, const uint8_t* __restrict__ src, uint16_t* __restrict__ dst,
-                       DecodeState* ds) {
+k_lossless_decode_fast(LosslessShape sh, FrameBatch b, uint8_t* ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   FastSmem& S = *reinterpret_cast<FastSmem*>(smem_raw);
   const uint32_t tid = threadIdx.x;
-  if (ds->status != kOk) return;
-  const uint32_t nrec = ds->n_records;
+  if (tid == 0) {  // records of the batch: prefix over frames that passed the header check
+    uint32_t acc = 0;
+    for (uint32_t f = 0; f < b.n; ++f) {
+      S.base[f] = acc;
+      const DecodeState* d = decode_state(ws, f);
+      acc += d->status == kOk ? d->n_records : 0u;
+    }
+    S.base[b.n] = acc;
+  }
+  __syncthreads();
+  const uint32_t nrec = S.base[b.n];
+  if (blockIdx.x >= nrec) return;
   const uint32_t D = sh.D;
-  const bool shape_ok = (D * sh.tc == kMaxChunkValues) && (sh.tc % 512u == 0);
-  const uint32_t lpc_log2 = shape_ok ? uint32_t(ilog2_u32(sh.tc / 512u)) : 0u;
+  const bool shape_ok = (D * sh.tc == kMaxChunkValues) && (D == 128u || D == 64u);
   crc_tables_init(S.crc_t);
-  for (uint32_t r = blockIdx.x; r < nrec; r += gridDim.x) {
+  crc_join_init(&S.join);
+  for (uint32_t g = blockIdx.x; g < nrec; g += gridDim.x) {
     __syncthreads();
+    const uint32_t fr = frame_of(S.base, b.n, g), r = g - S.base[fr];
+    const uint8_t* src = b.f[fr].src;
+    uint16_t* dst = reinterpret_cast<uint16_t*>(b.f[fr].dst);
+    DecodeState* ds = decode_state(ws, fr);
     const uint32_t slice = r / sh.cps, c = r % sh.cps;
     const uint32_t t0 = c * sh.tc, tcc = min(sh.tc, sh.T - t0);
     bool defer = !shape_ok || tcc != sh.tc;
@@ -366,8 +461,11 @@ k_lossless_decode_fast(LosslessShape sh, const uint8_t* __restrict__ src, uint16
     const uint32_t len = ld_u32(e + 8), want = ld_u32(e + 12);
     const uint8_t* rec = src + off;
     int st = kOk;
+    if (!defer && len > kCrcOneRound) {  // cannot be a valid full-chunk record; let the general decoder report it
+      defer = true;
+    }
     if (!defer) {
-      uint32_t got = crc32_block_aligned(rec, len, S.crc_t, S.red);
+      uint32_t got = crc32_block_128(rec, len, S.crc_t, &S.join, S.red);
       if (tid == 0) S.crc_ok = (got == want);
       __syncthreads();
       st = S.crc_ok ? kOk : kErrCorrupt;
@@ -381,7 +479,9 @@ k_lossless_decode_fast(LosslessShape sh, const uint8_t* __restrict__ src, uint16
       if (st == kOk && S.si[0].mode == kModeRans && S.si[1].mode == kModeRans) defer = true;
     }
     if (defer) {
-      if (tid == 0) deferred_list(ds)[atomicAdd(&ds->n_deferred, 1u)] = r;
+      if (tid == 0)
+        deferred_list(ws)[atomicAdd(&batch_state(ws)->n_deferred, 1u)] =
+            (static_cast<unsigned long long>(fr) << 32) | r;
       continue;
     }
     if (st != kOk) {
@@ -393,15 +493,8 @@ k_lossless_decode_fast(LosslessShape sh, const uint8_t* __restrict__ src, uint16
     else if (m1 == kModeRans) block_dec_lut(S.freq[1], S.cum, S.lut, S.tmp);
     const uint8_t* recp[2] = {rec, rec + S.si[0].bytes};
     uint16_t* out = dst + (uint64_t(slice) * sh.T + t0) * D;
-    bool ok;
-    if (m0 == kModeRaw && m1 == kModeRans) ok = fast_tiles<kModeRaw, kModeRans>(S, recp, out, D, lpc_log2);
-    else if (m0 == kModeRaw && m1 == kModeRaw) ok = fast_tiles<kModeRaw, kModeRaw>(S, recp, out, D, lpc_log2);
-    else if (m0 == kModeRaw && m1 == kModeConst) ok = fast_tiles<kModeRaw, kModeConst>(S, recp, out, D, lpc_log2);
-    else if (m0 == kModeRans && m1 == kModeRaw) ok = fast_tiles<kModeRans, kModeRaw>(S, recp, out, D, lpc_log2);
-    else if (m0 == kModeRans && m1 == kModeConst) ok = fast_tiles<kModeRans, kModeConst>(S, recp, out, D, lpc_log2);
-    else if (m0 == kModeConst && m1 == kModeRans) ok = fast_tiles<kModeConst, kModeRans>(S, recp, out, D, lpc_log2);
-    else if (m0 == kModeConst && m1 == kModeRaw) ok = fast_tiles<kModeConst, kModeRaw>(S, recp, out, D, lpc_log2);
-    else ok = fast_tiles<kModeConst, kModeConst>(S, recp, out, D, lpc_log2);
+    const bool ok = D == 128u ? fast_dispatch<128>(S, recp, out, m0, m1)
+                              : fast_dispatch<64>(S, recp, out, m0, m1);
     if (!__syncthreads_and(ok) && tid == 0)
       atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(kErrCorrupt));
   }
@@ -426,9 +519,9 @@ uint64_t lossless_slot_bytes(const LosslessShape& s) {
   return (b + 255u) & ~uint64_t(255);
 }
 
-cudaError_t launch_lossless_encode(const LosslessShape& s, const uint16_t* src, uint32_t n_slices,
+cudaError_t launch_lossless_encode(const LosslessShape& s, const FrameBatch& b,
                                    const EncodeLayout& ws, cudaStream_t st) {
-  const uint32_t nrec = n_slices * s.cps;
+  const uint32_t nrec = b.rec_base[b.n];
   if (nrec == 0) return cudaSuccess;
   size_t smem = sizeof(EncSmem) + pad16(s.tc * s.D * 2u);
   cudaError_t e = cudaFuncSetAttribute(k_lossless_encode, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -436,14 +529,14 @@ cudaError_t launch_lossless_encode(const LosslessShape& s, const uint16_t* src, 
   if (e != cudaSuccess) return e;
   {
     ProfRange pr_("lossless_encode", st);
-    k_lossless_encode<<<nrec, kThreads, smem, st>>>(s, src, ws);
+    k_lossless_encode<<<nrec, kThreads, smem, st>>>(s, b, ws);
   }
   return cudaGetLastError();
 }
 
-cudaError_t launch_lossless_decode(const LosslessShape& s, const uint8_t* src, uint16_t* dst,
-                                   DecodeState* ds, uint32_t max_records, cudaStream_t st) {
-  if (max_records == 0) return cudaSuccess;
+cudaError_t launch_lossless_decode(const LosslessShape& s, const FrameBatch& b, uint8_t* ws,
+                                   uint32_t max_records, cudaStream_t st) {
+  if (max_records == 0 || b.n == 0) return cudaSuccess;
   static int fast_blocks_per_sm = 0;
   const size_t fsmem = sizeof(FastSmem);
   cudaError_t e = cudaFuncSetAttribute(k_lossless_decode_fast,
@@ -457,7 +550,7 @@ cudaError_t launch_lossless_decode(const LosslessShape& s, const uint8_t* src, u
   {
     ProfRange pr_("lossless_decode", st);
     uint32_t grid = min(max_records, uint32_t(num_sms() * fast_blocks_per_sm));
-    k_lossless_decode_fast<<<grid, kFastThreads, fsmem, st>>>(s, src, dst, ds);
+    k_lossless_decode_fast<<<grid, kFastThreads, fsmem, st>>>(s, b, ws);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -467,7 +560,7 @@ cudaError_t launch_lossless_decode(const LosslessShape& s, const uint8_t* src, u
   {
     ProfRange pr_("lossless_decode_general", st);
     uint32_t grid = min(max_records, uint32_t(num_sms()));
-    k_lossless_decode<<<grid, kThreads, smem, st>>>(s, src, dst, ds);
+    k_lossless_decode<<<grid, kThreads, smem, st>>>(s, b, ws);
   }
   return cudaGetLastError();
 }

@@ -97,15 +97,18 @@ struct __align__(16) EncSmem {
 };
 
 __global__ void __launch_bounds__(kThreads)
-k_transform_encode_mid(TransformShape sh, TransformPlanDev pl, const uint16_t* __restrict__ src,
-                       uint32_t first_slice, EncodeLayout ws) {
+k_transform_encode_mid(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLayout ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   EncSmem& S = *reinterpret_cast<EncSmem*>(smem_raw);
   const uint32_t tid = threadIdx.x, nthr = blockDim.x;
-  const uint32_t ls = blockIdx.x / sh.n_mid, c = blockIdx.x % sh.n_mid;
-  const uint32_t sidx = first_slice + ls;
+  const uint32_t rps = 1u + sh.n_mid;
+  const uint32_t gs = blockIdx.x / sh.n_mid, c = blockIdx.x % sh.n_mid;  // slice of the batch
+  const uint32_t r = gs * rps + 1u + c;                                   // record of the batch
+  const uint32_t fr = frame_of(b.rec_base, b.n, r);
+  const uint32_t ls = (r - b.rec_base[fr]) / rps;
+  const uint16_t* src = reinterpret_cast<const uint16_t*>(b.f[fr].src);
+  const uint32_t sidx = b.f[fr].first_slice + ls;
   const bool is_key = ((sidx / sh.H) & 1u) == 0;
-  const uint32_t r = ls * (1u + sh.n_mid) + 1u + c;
   const uint32_t t0 = sh.s_end + c * sh.ct, tcc = min(sh.ct, sh.r_start - t0);
   const uint32_t nb = (tcc + kTile - 1) / kTile;
   const uint16_t* xs = src + uint64_t(ls) * sh.T * kD;
@@ -250,11 +253,15 @@ k_transform_encode_mid(TransformShape sh, TransformPlanDev pl, const uint16_t* _
 
 // Raw record of each slice: sink rows, then recent rows, bf16 bytes, padded.
 __global__ void __launch_bounds__(kThreads)
-k_transform_encode_raw(TransformShape sh, const uint16_t* __restrict__ src, EncodeLayout ws) {
+k_transform_encode_raw(TransformShape sh, FrameBatch b, EncodeLayout ws) {
   __shared__ uint32_t crc_t[1024];
   __shared__ uint32_t red[32];
-  const uint32_t ls = blockIdx.x, tid = threadIdx.x;
-  const uint32_t r = ls * (1u + sh.n_mid);
+  const uint32_t tid = threadIdx.x;
+  const uint32_t rps = 1u + sh.n_mid;
+  const uint32_t r = blockIdx.x * rps;  // record of the batch
+  const uint32_t fr = frame_of(b.rec_base, b.n, r);
+  const uint32_t ls = (r - b.rec_base[fr]) / rps;
+  const uint16_t* src = reinterpret_cast<const uint16_t*>(b.f[fr].src);
   uint8_t* rec = ws.slots + uint64_t(r) * ws.slot_bytes;
   const uint32_t n_rows = sh.s_end + (sh.T - sh.r_start);
   const uint32_t bytes = n_rows * kD * 2u, len = pad16(bytes);
@@ -289,6 +296,7 @@ struct __align__(1024) DecSmem {
   StreamInfo si;
   CompInfo ci;
   uint64_t bar;
+  uint32_t base[kBatchMax + 1];
   uint32_t tmem_base;
   uint32_t crc_ok, cur_slice, bad;
 };
@@ -296,16 +304,24 @@ struct __align__(1024) DecSmem {
 static_assert(sizeof(DecSmem) + 1024 <= 232448, "decoder shared memory exceeds the per-block limit");
 
 __global__ void __launch_bounds__(kThreads)
-k_transform_decode(TransformShape sh, TransformPlanDev pl, const uint8_t* __restrict__ src,
-                   uint16_t* __restrict__ dst, DecodeState* ds) {
+k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t* ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   // the swizzled operand tiles need 1024-byte-aligned shared addresses
   const uint32_t pad = (1024u - (tc::smem_addr(smem_raw) & 1023u)) & 1023u;
   DecSmem& S = *reinterpret_cast<DecSmem*>(smem_raw + pad);
   const uint32_t tid = threadIdx.x, nthr = blockDim.x;
   const uint32_t warp = tid >> 5, lane = tid & 31u;
-  if (ds->status != kOk) return;
-  const uint32_t nrec = ds->n_records, first = ds->first_slice;
+  if (tid == 0) {  // records of the batch: prefix over frames that passed the header check
+    uint32_t acc = 0;
+    for (uint32_t f = 0; f < b.n; ++f) {
+      S.base[f] = acc;
+      const DecodeState* d = decode_state(ws, f);
+      acc += d->status == kOk ? d->n_records : 0u;
+    }
+    S.base[b.n] = acc;
+  }
+  __syncthreads();
+  const uint32_t nrec = S.base[b.n];
   const uint32_t per = (nrec + gridDim.x - 1) / gridDim.x;
   const uint32_t rbeg = blockIdx.x * per, rend = min(nrec, rbeg + per);
   if (rbeg >= rend) return;
@@ -326,8 +342,13 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, const uint8_t* __rest
   bool alive = true;
   const uint32_t rps = 1u + sh.n_mid;
   constexpr uint32_t idesc = tc::idesc_bf16_f32(kTcRows, kD);
-  for (uint32_t r = rbeg; r < rend && alive; ++r) {
+  for (uint32_t g = rbeg; g < rend && alive; ++g) {
     __syncthreads();
+    const uint32_t fr = frame_of(S.base, b.n, g), r = g - S.base[fr];
+    const uint8_t* src = b.f[fr].src;
+    uint16_t* dst = reinterpret_cast<uint16_t*>(b.f[fr].dst);
+    DecodeState* ds = decode_state(ws, fr);
+    const uint32_t first = ds->first_slice;
     const uint8_t* e = src + kHeaderBytes + uint64_t(kIndexEntry) * r;
     const uint64_t off0 = ld_u64(e);
     const uint32_t len = ld_u32(e + 8), want = ld_u32(e + 12);
@@ -534,12 +555,12 @@ uint64_t transform_slot_bytes(const TransformShape& s) {
 }
 
 cudaError_t launch_transform_encode(const TransformShape& s, const TransformPlanDev& p,
-                                    const uint16_t* src, uint32_t first_slice, uint32_t n_slices,
-                                    const EncodeLayout& ws, cudaStream_t st) {
+                                    const FrameBatch& b, const EncodeLayout& ws, cudaStream_t st) {
+  const uint32_t n_slices = b.rec_base[b.n] / (1u + s.n_mid);
   if (n_slices == 0) return cudaSuccess;
   {
     ProfRange pr_("transform_encode_raw", st);
-    k_transform_encode_raw<<<n_slices, kThreads, 0, st>>>(s, src, ws);
+    k_transform_encode_raw<<<n_slices, kThreads, 0, st>>>(s, b, ws);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || s.n_mid == 0) return e;
@@ -548,22 +569,22 @@ cudaError_t launch_transform_encode(const TransformShape& s, const TransformPlan
   if (e != cudaSuccess) return e;
   {
     ProfRange pr_("transform_encode_mid", st);
-    k_transform_encode_mid<<<n_slices * s.n_mid, kThreads, smem, st>>>(s, p, src, first_slice, ws);
+    k_transform_encode_mid<<<n_slices * s.n_mid, kThreads, smem, st>>>(s, p, b, ws);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_transform_decode(const TransformShape& s, const TransformPlanDev& p,
-                                    const uint8_t* src, uint16_t* dst, DecodeState* ds,
-                                    uint32_t max_records, cudaStream_t st) {
-  if (max_records == 0) return cudaSuccess;
+                                    const FrameBatch& b, uint8_t* ws, uint32_t max_records,
+                                    cudaStream_t st) {
+  if (max_records == 0 || b.n == 0) return cudaSuccess;
   size_t smem = sizeof(DecSmem) + 1024;
   cudaError_t e = cudaFuncSetAttribute(k_transform_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   uint32_t grid = min(max_records, uint32_t(num_sms()));
   {
     ProfRange pr_("transform_decode", st);
-    k_transform_decode<<<grid, kThreads, smem, st>>>(s, p, src, dst, ds);
+    k_transform_decode<<<grid, kThreads, smem, st>>>(s, p, b, ws);
   }
   return cudaGetLastError();
 }
