@@ -142,3 +142,59 @@ def test_plan_mismatch_and_capacity():
     other = kvc.Plan(kvc.Shape(kvc.BF16, 1, 1, 513, 128))
     assert decode(other, kvc.LOSSLESS, c, 2)[0] == kvc.ERR_PLAN_MISMATCH
     assert decode(plan, kvc.LOSSLESS, c, 1)[0] == kvc.ERR_CAPACITY
+
+
+RAW, CONST, RANS = 0, 1, 2
+_SKEW = np.array([.5, .2, .1, .08, .05, .04, .02, .01])
+
+
+def _plane(rng, kind, shape):
+    if kind == RAW:
+        return rng.integers(0, 256, shape)
+    if kind == CONST:
+        return np.full(shape, 0x3F)
+    return rng.choice(np.arange(8) * 29, size=shape, p=_SKEW)
+
+
+def _records(c: bytes):
+    """(offset, length) of every record of a container, from its index."""
+    n = int.from_bytes(c[36:40], "little")
+    out = []
+    for i in range(n):
+        e = 64 + 16 * i
+        out.append((int.from_bytes(c[e:e + 8], "little"), int.from_bytes(c[e + 8:e + 12], "little")))
+    return out
+
+
+@pytest.mark.parametrize("D", [128, 64])
+def test_full_chunk_mode_pairs_and_damage(D):
+    """Full chunks (the token-synchronous decoder) with every pair of plane
+    modes but two rANS planes, decoded exactly; damage in either stream's
+    header or payload, or at the record's ends, is refused as the oracle does."""
+    pairs = [(RAW, RANS), (RAW, RAW), (RAW, CONST), (RANS, RAW), (RANS, CONST), (CONST, RANS),
+             (CONST, RAW), (CONST, CONST)]
+    T = 65536 // D
+    rng = np.random.default_rng(11 + D)
+    x = np.stack([(_plane(rng, lo, (T, D)) | (_plane(rng, hi, (T, D)) << 8)).astype(np.uint16)
+                  for lo, hi in pairs])
+    w = _w("lossless-1x8x512x128-bf16", n_heads=4, n_tokens=T, head_dim=D)
+    plan, oplan = _plans(w)
+    c = bytearray(oracle.encode_lossless(oplan, x))
+    recs = _records(c)
+    assert len(recs) == len(pairs)
+    for (off, ln), (lo, hi) in zip(recs, pairs):  # the encoder chose the intended modes
+        b0 = int.from_bytes(c[off + 4:off + 8], "little")
+        assert (c[off], c[off + b0]) == (lo, hi)
+    st, y = decode(plan, kvc.LOSSLESS, bytes(c), len(pairs))
+    assert st == kvc.OK and np.array_equal(y, x)
+    for off, ln in recs:
+        b0 = int.from_bytes(c[off + 4:off + 8], "little")
+        spots = {off, off + 1, off + 12, off + 16, off + b0 // 2, off + b0 - 1, off + b0,
+                 off + b0 + 16, off + (b0 + ln) // 2, off + ln - 1}
+        for pos in sorted(p for p in spots if p < off + ln):
+            orig = c[pos]
+            c[pos] = orig ^ 0x5A
+            want, _ = oracle.decode_lossless(oplan, bytes(c))
+            got, _ = decode(plan, kvc.LOSSLESS, bytes(c), len(pairs))
+            assert want != oracle.OK and got == want, (pos - off, got, want)
+            c[pos] = orig

@@ -226,84 +226,68 @@ __device__ inline uint32_t crc32_block_bytes(Fetch fetch, uint64_t len, const ui
   return total ^ 0xffffffffu;
 }
 
-// One-round block CRC for records up to kCrcOneRound bytes: thread t owns the
-// run [t R, (t + 1) R) of the record padded in front to 128 R bytes (R = 1040),
-// so every shift in the join is a compile-time constant: x^(8 R 2^l). Joins
-// multiply by those constants with per-nibble tables (8 lookups instead of a
-// 32-step bitwise product). The tables are built once per CTA.
-constexpr uint32_t kCrcRunR = 1040;                       // 65 x 16 bytes
-constexpr uint32_t kCrcOneRound = 128u * kCrcRunR;        // 133120 bytes
-struct CrcJoin {
-  uint32_t nib[8][8][16];  // [level][nibble position][value]: (v << 4 pos) * x^(8 R 2^level)
+constexpr uint32_t kCrcRegionMaxUnits = 33;  // runs of at most 33 * 16 bytes: regions <= 67584 bytes
+
+// Powers of x used to join CRC pieces: q[n][l] = x^(8 * 16n * 2^l) joins
+// neighbouring runs of 16n bytes (l-th level of a tree); u[m] = x^(8 * 16m).
+struct CrcPowTables {
+  uint32_t q[34][8];
+  uint32_t u[128];
 };
-struct CrcRunShifts { uint32_t v[8]; };
-constexpr CrcRunShifts make_run_shifts() {
-  CrcRunShifts s{};
-  for (int l = 0; l < 8; ++l) s.v[l] = gf2_xpow8(uint64_t(kCrcRunR) << l);
-  return s;
-}
-__constant__ CrcRunShifts kCrcRunShift = make_run_shifts();
-
-__device__ inline void crc_join_init(CrcJoin* J) {
-  for (uint32_t i = threadIdx.x; i < 8 * 8 * 16; i += blockDim.x) {
-    const uint32_t l = i >> 7, pos = (i >> 4) & 7u, val = i & 15u;
-    J->nib[l][pos][val] = gf2_mul(val << (4 * pos), kCrcRunShift.v[l]);
-  }
-  __syncthreads();
-}
-__device__ inline uint32_t crc_join_mul(const CrcJoin* J, uint32_t level, uint32_t a) {
-  uint32_t r = 0;
-#pragma unroll
-  for (uint32_t pos = 0; pos < 8; ++pos) r ^= J->nib[level][pos][(a >> (4 * pos)) & 15u];
-  return r;
-}
-
-// CRC-32 of len (multiple of 16, <= kCrcOneRound) bytes at p (16-byte aligned)
-// by a block of exactly 128 threads; result valid in thread 0.
-__device__ inline uint32_t crc32_block_128(const uint8_t* p, uint32_t len, const uint32_t* t,
-                                           const CrcJoin* J, uint32_t* red) {
-  const uint32_t pad = kCrcOneRound - len;
-  const int64_t run0 = int64_t(threadIdx.x) * kCrcRunR - int64_t(pad);
-  uint32_t c = 0;
-  if (run0 + int64_t(kCrcRunR) > 0) {
-    // 65 vectors per run, loaded five at a time so five loads are in flight
-    const uint32_t k0 = run0 < 0 ? uint32_t(-run0) / 16u : 0u;  // first real vector
-    for (uint32_t kb = 0; kb < kCrcRunR / 16u; kb += 5) {
-      uint4 v[5];
-#pragma unroll
-      for (uint32_t i = 0; i < 5; ++i) {
-        const uint32_t k = kb + i;
-        v[i] = k >= k0 ? __ldcg(reinterpret_cast<const uint4*>(p + uint32_t(run0 + 16 * int64_t(k))))
-                       : make_uint4(0, 0, 0, 0);
-      }
-#pragma unroll
-      for (uint32_t i = 0; i < 5; ++i) {
-        const uint32_t k = kb + i;
-        if (k < k0) continue;
-        if (run0 + 16 * int64_t(k) == 0) v[i].x = ~v[i].x;
-        c = crc_word(t, c, v[i].x);
-        c = crc_word(t, c, v[i].y);
-        c = crc_word(t, c, v[i].z);
-        c = crc_word(t, c, v[i].w);
-      }
+constexpr CrcPowTables make_crc_pow_tables() {
+  CrcPowTables t{};
+  const uint32_t x16 = gf2_xpow8(16);
+  uint32_t p = 0x80000000u;  // x^0
+  for (int n = 0; n < 34; ++n) {
+    uint32_t c = p;
+    for (int l = 0; l < 8; ++l) {
+      t.q[n][l] = c;
+      c = gf2_mul(c, c);
     }
+    p = gf2_mul(p, x16);
   }
-  const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
+  p = 0x80000000u;
+  for (int m = 0; m < 128; ++m) {
+    t.u[m] = p;
+    p = gf2_mul(p, x16);
+  }
+  return t;
+}
+__constant__ CrcPowTables kCrcPow = make_crc_pow_tables();
+
+// Per-thread powers for joining the registers of 128 consecutive runs of 16q
+// bytes: the register of run t, multiplied by x^(8 * 16q * (127 - t)), is its
+// share of the register of the concatenation, so the join is one multiply per
+// thread and an exclusive-or reduction.
+struct CrcLanePow {
+  uint32_t v[kCrcRegionMaxUnits + 1][128];
+};
+constexpr CrcLanePow make_crc_lane_pow() {
+  CrcLanePow t{};
+  const uint32_t x16 = gf2_xpow8(16);
+  uint32_t step = 0x80000000u;  // x^(8 * 16q)
+  for (uint32_t q = 0; q <= kCrcRegionMaxUnits; ++q) {
+    uint32_t p = 0x80000000u;
+    for (int i = 127; i >= 0; --i) {
+      t.v[q][i] = p;
+      p = gf2_mul(p, step);
+    }
+    step = gf2_mul(step, x16);
+  }
+  return t;
+}
+__device__ const CrcLanePow kCrcLanePow = make_crc_lane_pow();
+
+// Join the registers of 128 consecutive runs of 16q bytes (thread t holds run
+// t, exactly 128 threads); result in thread 0.
+__device__ inline uint32_t crc_join_lanes(uint32_t c, uint32_t q, uint32_t* red) {
+  c = gf2_mul(c, __ldg(&kCrcLanePow.v[q][threadIdx.x]));
 #pragma unroll
-  for (uint32_t l = 0; l < 5; ++l) {
-    const uint32_t other = __shfl_down_sync(0xffffffffu, c, 1u << l);
-    if ((lane & ((2u << l) - 1u)) == 0) c = crc_join_mul(J, l, c) ^ other;
-  }
+  for (uint32_t o = 16; o; o >>= 1) c ^= __shfl_xor_sync(0xffffffffu, c, o);
   __syncthreads();
-  if (lane == 0) red[warp] = c;
+  if ((threadIdx.x & 31u) == 0) red[threadIdx.x >> 5] = c;
   __syncthreads();
-  uint32_t total = 0;
-  if (threadIdx.x == 0) {
-    const uint32_t a = crc_join_mul(J, 5, red[0]) ^ red[1];
-    const uint32_t b = crc_join_mul(J, 5, red[2]) ^ red[3];
-    total = crc_join_mul(J, 6, a) ^ b;
-  }
-  return len ? (total ^ 0xffffffffu) : 0u;
+  return threadIdx.x == 0 ? red[0] ^ red[1] ^ red[2] ^ red[3] : 0u;
 }
 
 // ---------------------------------------------------------------- block helpers
@@ -418,9 +402,11 @@ __device__ inline void block_enc_tables(const uint32_t* freq, uint32_t* fc, uint
   __syncthreads();
 }
 
-// Decode table: lut[slot] = (slot - cum_s) | f_s << 12 | s << 24, and the
+// Decode table: lut[slot] = s | (slot - cum_s) << 8 | f_s << 20, and the
 // symbols' cumulative starts in cum[257]. freq must be validated (sum 4096).
-// Each thread fills a contiguous run of slots, walking the symbols forward.
+// The first slot of every present symbol is marked with s + 1; each warp then
+// resolves its span of slots 32 at a time, a running maximum of the marks
+// giving every slot its symbol.
 __device__ inline void block_dec_lut(const uint32_t* freq, uint32_t* cum, uint32_t* lut,
                                      uint32_t* tmp) {
   const uint32_t per = blockDim.x >= 256 ? 1u : 256u / blockDim.x;
@@ -434,26 +420,38 @@ __device__ inline void block_dec_lut(const uint32_t* freq, uint32_t* cum, uint32
     c += freq[s0 + i];
   }
   if (threadIdx.x == 0) cum[256] = kProbScale;
+  for (uint32_t i = threadIdx.x; i < kProbScale / 4u; i += blockDim.x)
+    reinterpret_cast<uint4*>(lut)[i] = make_uint4(0, 0, 0, 0);
   __syncthreads();
-  // lane j of warp w fills slots base_w + j + 32 i (i = 0 .. per_lane - 1): one
-  // bank per lane, ascending slots per lane so the symbol walk only moves forward
+  for (uint32_t s = threadIdx.x; s < 256; s += blockDim.x)
+    if (freq[s]) lut[cum[s]] = s + 1u;
+  __syncthreads();
   const uint32_t nw = blockDim.x >> 5, warp = threadIdx.x >> 5, lane = threadIdx.x & 31u;
-  const uint32_t span = kProbScale / nw, per_lane = span / 32u;
-  const uint32_t first = warp * span + lane;
-  uint32_t lo = 0, hi = 255;  // largest symbol with cum <= first
-  while (lo < hi) {
-    const uint32_t mid = (lo + hi + 1) >> 1;
-    if (cum[mid] <= first) lo = mid; else hi = mid - 1;
-  }
-  uint32_t sym = lo, cs = cum[sym], ce = cum[sym + 1];
-  for (uint32_t i = 0; i < per_lane; ++i) {
-    const uint32_t slot = first + 32u * i;
-    while (slot >= ce) {  // next symbol with a nonzero frequency
-      ++sym;
-      cs = ce;
-      ce = cum[sym + 1];
+  const uint32_t span = kProbScale / nw, first = warp * span;
+  // mark carried into the span: the last symbol starting before it (its start
+  // is below `first`, and the largest such s has a nonzero frequency)
+  uint32_t carry = 0;
+  if (first) {
+    uint32_t lo = 0, hi = 255;
+    while (lo < hi) {
+      const uint32_t mid = (lo + hi + 1) >> 1;
+      if (cum[mid] < first) lo = mid; else hi = mid - 1;
     }
-    lut[slot] = (slot - cs) | ((ce - cs) << 12) | (sym << 24);
+    carry = lo + 1u;
+  }
+#pragma unroll 4
+  for (uint32_t b = 0; b < span; b += 32u) {
+    const uint32_t slot = first + b + lane;
+    uint32_t m = lut[slot];
+#pragma unroll
+    for (uint32_t o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, m, o);
+      if (lane >= o) m = max(m, y);
+    }
+    m = max(m, carry);
+    carry = __shfl_sync(0xffffffffu, m, 31);
+    const uint32_t sym = m - 1u;
+    lut[slot] = sym | ((slot - cum[sym]) << 8) | (freq[sym] << 20);
   }
   __syncthreads();
 }
@@ -526,8 +524,8 @@ __device__ inline bool rans_decode_group(const uint8_t* sub, uint32_t sub_len, u
     const bool act = live && tau < len;
     if (act) {
       uint32_t e = lut[x & (kProbScale - 1u)];
-      x = ((e >> 12) & 0xfffu) * (x >> kProbBits) + (e & 0xfffu);
-      out(start + tau, e >> 24);
+      x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xfffu);
+      out(start + tau, e & 0xffu);
     }
     bool need = act && x < kRansLow;
     uint32_t mask = __ballot_sync(0xffffffffu, need);

@@ -245,48 +245,51 @@ k_lossless_decode(LosslessShape sh, FrameBatch b, uint8_t* ws) {
 
 
 // ---------------------------------------------------------------------------
-// Fast decoder for full chunks (D * tc = 65536 values, tc a multiple of 512):
-// then every stream has 128 lanes of 512 symbols and lane l's symbol tau sits at
-// channel-major index l * 512 + tau in both planes, i.e. channel l / lpc, token
-// (l % lpc) * 512 + tau with lpc = tc / 512. Thread l owns lane l of both planes
-// (warp w = rANS group w), decodes token-synchronously, merges the other
-// plane's raw bytes from registers and writes 32-token tiles of token-major
-// rows through shared memory. Records with two rANS planes or other shapes are
-// deferred to the general decoder.
+// Fast decoder for full chunks of D = 128 or 64 channels (tc * D = 65536
+// values): every stream then has 128 lanes of 512 symbols and lane l's symbol
+// tau sits at channel-major index l * 512 + tau in both planes, i.e. channel
+// l / lpc, token (l % lpc) * 512 + tau with lpc = 128 / D. Thread l owns lane l
+// of both planes (warp w = rANS group w), decodes token-synchronously, merges
+// the other plane's raw bytes from registers and stores the values straight
+// to the token-major output, two channels per 32-bit store after one exchange
+// between neighbouring channels. Records with two rANS planes or other shapes
+// are deferred to the general decoder.
+//
+// The record's CRC is checked without a second pass over the raw plane: each
+// lane folds its own 512 raw bytes into a CRC register as it consumes them, a
+// short pre-pass covers the other stream record, and the pieces are joined
+// with powers of x (crc(A || B) = crc(A) * x^(8|B|) + crc(B)). The output of a
+// record that fails the check is unspecified, as for every decode error.
 constexpr uint32_t kFastThreads = 128;
+constexpr uint32_t kRawStream = 16u + kMaxChunkValues;  // bytes of a full-chunk RAW stream record
 
 struct __align__(16) FastSmem {
   uint32_t crc_t[1024];
   uint32_t lut[kProbScale];
-  uint16_t tile[32 * 128];
+  uint16_t ring[kFastThreads / 32][1024];  // per-group window of rANS refill words
   uint32_t freq[2][256];
   uint32_t cum[260];
   uint32_t tmp[32], red[32];
   StreamInfo si[2];
-  uint16_t ring[kFastThreads / 32][1024];  // per-group window of rANS refill words
-  CrcJoin join;
   uint32_t base[kBatchMax + 1];
-  uint32_t crc_ok;
 };
 
 // One rANS lane of a 32-lane group (warp-synchronous). Refill words come from
-// the group's window in shared memory (word i at ring[i % 1024]); a lane whose
-// index runs past the sub-stream marks the record bad and its state is junk.
+// the group's window in shared memory (word i at ring[i % 1024]). A lane whose
+// index runs past the sub-stream reads a stale word, but then the group's word
+// count ends above the sub-stream's and the final check rejects the record.
 struct LaneRans {
   uint32_t x, pos, W;
   const uint16_t* ring;
-  uint32_t bad;
   __device__ __forceinline__ uint32_t step(const uint32_t* lut, uint32_t lt) {
     const uint32_t e = lut[x & (kProbScale - 1u)];
-    x = ((e >> 12) & 0xfffu) * (x >> kProbBits) + (e & 0xfffu);
+    x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xfffu);
     const bool need = x < kRansLow;
     const uint32_t mask = __ballot_sync(0xffffffffu, need);
-    const uint32_t idx = pos + __popc(mask & lt);
-    const uint32_t w = ring[idx & 1023u];
+    const uint32_t w = ring[(pos + __popc(mask & lt)) & 1023u];
     x = need ? ((x << 16) | w) : x;
-    bad |= uint32_t(need && idx >= W);
     pos += __popc(mask);
-    return e >> 24;
+    return e;  // symbol in the low byte
   }
 };
 
@@ -316,117 +319,201 @@ struct RefillWindow {
   }
 };
 
-// value of step j: byte (j % 4) of raw word r (plane 0) and decoded symbol (plane 1),
-// or the other way round, merged into one 16-bit value
-__device__ __forceinline__ uint32_t merge_raw_lo(uint32_t r, uint32_t j, uint32_t hi) {
-  return __byte_perm(r, hi, (j & 3u) | 0x40u);  // byte0 = r.byte(j%4), byte1 = hi.byte0
-}
-__device__ __forceinline__ uint32_t merge_raw_hi(uint32_t r, uint32_t j, uint32_t lo) {
-  return __byte_perm(lo, r, 0u | ((4u + (j & 3u)) << 4));  // byte0 = lo.byte0, byte1 = r.byte(j%4)
+// Value of step j (low 16 bits; the high half is don't-care) from the two
+// planes' bytes: a RAW plane gives byte j % 4 of its word r, a rANS plane the
+// low byte of the table entry, a CONST plane its symbol.
+template <uint32_t M0, uint32_t M1>
+__device__ __forceinline__ uint32_t merge_planes(uint32_t j, uint32_t a, uint32_t b) {
+  constexpr bool raw0 = M0 == kModeRaw, raw1 = M1 == kModeRaw;
+  const uint32_t s0 = raw0 ? (j & 3u) : 0u;
+  const uint32_t s1 = raw1 ? 4u + (j & 3u) : 4u;
+  return __byte_perm(a, b, s0 | (s1 << 4));
 }
 
+// CRC register of this thread's run of the pre-pass region (the record bytes
+// the tiles do not see: everything but the RAW payloads). Thread t owns a run
+// of q 16-byte units, q = ceil(len / 2048), right-aligned (leading zero units,
+// which leave a zero register unchanged; comp complements the record's first
+// four bytes, the standard CRC's initial value) or left-aligned (trailing zero
+// units, processed: the result is then multiplied by x^(8 * (2048q - len))).
+// The units are spread over the 16 tiles and loaded one tile ahead.
+struct PreRun {
+  const uint8_t* p;
+  uint32_t len, q, upt;  // upt: units per tile, ceil(q / 16) <= 3
+  int32_t run0;
+  bool left, comp;
+  uint32_t c;
+  uint4 nxt[3];
+  __device__ __forceinline__ void init(const uint8_t* base, uint32_t n, bool left_aligned, bool comp_first) {
+    p = base;
+    len = n;
+    q = (n + 2047u) >> 11;
+    upt = (q + 15u) >> 4;
+    left = left_aligned;
+    comp = comp_first;
+    run0 = int32_t(threadIdx.x * 16u * q) - (left ? 0 : int32_t(128u * 16u * q - n));
+    c = 0;
+    fetch(0);
+  }
+  __device__ __forceinline__ void fetch(uint32_t k) {
+#pragma unroll
+    for (uint32_t i = 0; i < 3; ++i) {
+      const uint32_t u = k * upt + i;
+      const int32_t off = run0 + int32_t(16u * u);
+      const bool in = i < upt && u < q && off >= 0 && uint32_t(off) < len;
+      nxt[i] = in ? __ldcg(reinterpret_cast<const uint4*>(p + off)) : make_uint4(0, 0, 0, 0);
+    }
+  }
+  // fold in tile k's units (loaded by the previous fetch) and load tile k + 1's
+  __device__ __forceinline__ void tile(const uint32_t* t, uint32_t k) {
+    uint4 cur[3] = {nxt[0], nxt[1], nxt[2]};
+    if (k + 1 < 16) fetch(k + 1);
+#pragma unroll
+    for (uint32_t i = 0; i < 3; ++i) {
+      const uint32_t u = k * upt + i;
+      const int32_t off = run0 + int32_t(16u * u);
+      if (i < upt && u < q && (left || off >= 0)) {
+        if (comp && off == 0) cur[i].x = ~cur[i].x;
+        c = crc_word(t, c, cur[i].x);
+        c = crc_word(t, c, cur[i].y);
+        c = crc_word(t, c, cur[i].z);
+        c = crc_word(t, c, cur[i].w);
+      }
+    }
+  }
+};
+
+// Decode the 16 tiles of 32 steps of one record. crc0 / crc1 return the CRC
+// register of this lane's 512 bytes of plane 0 / 1 when that plane is RAW; pre
+// folds in this thread's run of the pre-pass region.
 template <uint32_t M0, uint32_t M1, uint32_t D>
-__device__ inline bool fast_tiles(FastSmem& S, const uint8_t* const recp[2], uint16_t* out) {
+__device__ inline bool fast_tiles(FastSmem& S, const uint8_t* const recp[2], uint16_t* out,
+                                  PreRun& pre, uint32_t& crc0, uint32_t& crc1) {
   constexpr uint32_t LPC = 128u / D;  // lanes per channel
+  constexpr bool kRaw0 = M0 == kModeRaw, kRaw1 = M1 == kModeRaw;
+  constexpr bool kRans = (M0 == kModeRans || M1 == kModeRans);
+  constexpr bool kPre = !(kRaw0 && kRaw1);
+  constexpr uint32_t RP = (M0 == kModeRans) ? 0u : 1u;  // the rANS plane, if any
   const uint32_t l = threadIdx.x, lane = l & 31u, g = l >> 5;
   const uint32_t lt = lanemask_lt();
-  const uint32_t tbase = (l % LPC) * 32u * D + (l / LPC);
-  uint16_t* tile = S.tile + tbase;
-  LaneRans rs{kRansLow, 0, 0, S.ring[g], 0};
+  // Lanes l and l ^ LPC hold neighbouring channels (ch, ch ^ 1) of the same
+  // tokens. Of each pair of steps (j, j + 1) the even channel stores token j
+  // and the odd channel token j + 1, both channels in one 32-bit word.
+  const uint32_t ch = l / LPC, role = ch & 1u;
+  const uint32_t pair_sel = role ? 0x1054u : 0x5410u;
+  uint32_t* o32 = reinterpret_cast<uint32_t*>(out + (uint64_t(l % LPC) * 512u + role) * D + (ch & ~1u));
+  LaneRans rs{kRansLow, 0, 0, S.ring[g]};
   RefillWindow win{nullptr, 0, 0, tc::smem_addr(S.ring[g])};
   const uint8_t* raw0 = recp[0] + 16 + l * 512u;
   const uint8_t* raw1 = recp[1] + 16 + l * 512u;
   const uint32_t c0 = S.si[0].sym, c1 = S.si[1].sym;
-  constexpr bool kRans = (M0 == kModeRans || M1 == kModeRans);
-  constexpr uint32_t RP = (M0 == kModeRans) ? 0u : 1u;  // the rANS plane, if any
+  bool live = true;
   if (kRans) {
     const StreamInfo& si = S.si[RP];
     const uint8_t* sub = recp[RP] + si.sub_off[g];
     const uint32_t sl = si.sub_len[g];
-    if (sl < 128u || (sl & 1u)) rs.bad = 1;
+    if (sl < 128u || (sl & 1u)) live = false;
     else {
       rs.x = reinterpret_cast<const uint32_t*>(sub)[lane];
       rs.W = (sl - 128u) >> 1;
       win.units = sub + 128;
       win.n_units = (rs.W + 7u) >> 3;
     }
-  }
-  const bool live = __all_sync(0xffffffffu, rs.bad == 0);
-  uint4 n0a = make_uint4(0, 0, 0, 0), n0b = n0a, n1a = n0a, n1b = n0a;  // next tile's raw bytes
-  if (M0 == kModeRaw) { n0a = __ldcs(reinterpret_cast<const uint4*>(raw0)); n0b = __ldcs(reinterpret_cast<const uint4*>(raw0 + 16)); }
-  if (M1 == kModeRaw) { n1a = __ldcs(reinterpret_cast<const uint4*>(raw1)); n1b = __ldcs(reinterpret_cast<const uint4*>(raw1 + 16)); }
-  if (kRans && !live) return false;
-  if (kRans) {
+    if (!__all_sync(0xffffffffu, live)) return false;
     win.request(0, lane);
     asm volatile("cp.async.commit_group;" ::: "memory");  // empty group: the first settle waits for the window
   }
+  uint4 n0a = make_uint4(0, 0, 0, 0), n0b = n0a, n1a = n0a, n1b = n0a;  // next tile's raw bytes
+  if (kRaw0) { n0a = __ldcg(reinterpret_cast<const uint4*>(raw0)); n0b = __ldcg(reinterpret_cast<const uint4*>(raw0 + 16)); }
+  if (kRaw1) { n1a = __ldcg(reinterpret_cast<const uint4*>(raw1)); n1b = __ldcg(reinterpret_cast<const uint4*>(raw1 + 16)); }
+  uint32_t k0 = 0, k1 = 0;  // CRC registers of the raw runs
+#pragma unroll 1
   for (uint32_t k = 0; k < 16; ++k) {
     uint32_t r0[8], r1[8];
-    if (M0 == kModeRaw) {
+    if (kRaw0) {
       r0[0] = n0a.x; r0[1] = n0a.y; r0[2] = n0a.z; r0[3] = n0a.w;
       r0[4] = n0b.x; r0[5] = n0b.y; r0[6] = n0b.z; r0[7] = n0b.w;
       if (k + 1 < 16) {
-        n0a = __ldcs(reinterpret_cast<const uint4*>(raw0 + 32u * (k + 1)));
-        n0b = __ldcs(reinterpret_cast<const uint4*>(raw0 + 32u * (k + 1) + 16u));
+        n0a = __ldcg(reinterpret_cast<const uint4*>(raw0 + 32u * (k + 1)));
+        n0b = __ldcg(reinterpret_cast<const uint4*>(raw0 + 32u * (k + 1) + 16u));
       }
     }
-    if (M1 == kModeRaw) {
+    if (kRaw1) {
       r1[0] = n1a.x; r1[1] = n1a.y; r1[2] = n1a.z; r1[3] = n1a.w;
       r1[4] = n1b.x; r1[5] = n1b.y; r1[6] = n1b.z; r1[7] = n1b.w;
       if (k + 1 < 16) {
-        n1a = __ldcs(reinterpret_cast<const uint4*>(raw1 + 32u * (k + 1)));
-        n1b = __ldcs(reinterpret_cast<const uint4*>(raw1 + 32u * (k + 1) + 16u));
+        n1a = __ldcg(reinterpret_cast<const uint4*>(raw1 + 32u * (k + 1)));
+        n1b = __ldcg(reinterpret_cast<const uint4*>(raw1 + 32u * (k + 1) + 16u));
       }
     }
-#pragma unroll
-    for (uint32_t j = 0; j < 32; ++j) {
-      if (kRans && (j & 7u) == 0) {
+    if (kPre) pre.tile(S.crc_t, k);
+    uint32_t* o = o32 + (k * 32u) * (D / 2u);
+    // four stages of 8 steps; each consumes raw words 0 and 1, then the words shift down
+#pragma unroll 1
+    for (uint32_t st = 0; st < 4; ++st) {
+      if (kRans) {
         win.settle();
         win.request(rs.pos, lane);
       }
-      uint32_t v;
-      if (M0 == kModeRaw && M1 == kModeRans) v = merge_raw_lo(r0[j >> 2], j, rs.step(S.lut, lt));
-      else if (M0 == kModeRans && M1 == kModeRaw) v = merge_raw_hi(r1[j >> 2], j, rs.step(S.lut, lt));
-      else if (M0 == kModeRaw && M1 == kModeRaw) v = __byte_perm(r0[j >> 2], r1[j >> 2], (j & 3u) | ((4u + (j & 3u)) << 4));
-      else if (M0 == kModeRaw && M1 == kModeConst) v = merge_raw_lo(r0[j >> 2], j, c1);
-      else if (M0 == kModeConst && M1 == kModeRaw) v = merge_raw_hi(r1[j >> 2], j, c0);
-      else if (M0 == kModeRans && M1 == kModeConst) v = rs.step(S.lut, lt) | (c1 << 8);
-      else if (M0 == kModeConst && M1 == kModeRans) v = c0 | (rs.step(S.lut, lt) << 8);
-      else v = c0 | (c1 << 8);
-      tile[j * D] = uint16_t(v);
-    }
-    __syncthreads();
-    // tile = LPC blocks of 32 token rows x D channels, each contiguous in the output
-    constexpr uint32_t per_block = 4u * D;  // uint4 per block
 #pragma unroll
-    for (uint32_t i = 0; i < 4; ++i) {
-      const uint32_t q = l + i * kFastThreads;
-      const uint32_t sblk = q / per_block, w = q % per_block;
-      uint4* o = reinterpret_cast<uint4*>(out + (uint64_t(sblk) * 512u + 32u * k) * D);
-      o[w] = reinterpret_cast<const uint4*>(S.tile)[q];
+      for (uint32_t j = 0; j < 8; j += 2) {
+        uint32_t v[2];
+#pragma unroll
+        for (uint32_t h = 0; h < 2; ++h) {
+          const uint32_t jj = j + h;
+          const uint32_t e = kRans ? rs.step(S.lut, lt) : 0u;
+          const uint32_t a = kRaw0 ? r0[jj >> 2] : (M0 == kModeRans ? e : c0);
+          const uint32_t b = kRaw1 ? r1[jj >> 2] : (M1 == kModeRans ? e : c1);
+          v[h] = merge_planes<M0, M1>(jj, a, b);
+        }
+        const uint32_t send = role ? v[0] : v[1];
+        const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, LPC);
+        o[j * (D / 2u)] = __byte_perm(role ? v[1] : v[0], recv, pair_sel);
+      }
+      if (kRaw0) {
+        k0 = crc_word(S.crc_t, crc_word(S.crc_t, k0, r0[0]), r0[1]);
+#pragma unroll
+        for (uint32_t i = 0; i < 6; ++i) r0[i] = r0[i + 2];
+      }
+      if (kRaw1) {
+        k1 = crc_word(S.crc_t, crc_word(S.crc_t, k1, r1[0]), r1[1]);
+#pragma unroll
+        for (uint32_t i = 0; i < 6; ++i) r1[i] = r1[i + 2];
+      }
+      o += 8u * (D / 2u);
     }
-    __syncthreads();
   }
+  crc0 = k0;
+  crc1 = k1;
   if (kRans) asm volatile("cp.async.wait_group 0;" ::: "memory");  // no copy outlives the record
-  bool ok = rs.bad == 0;
-  if (kRans) ok = ok && rs.pos == rs.W && rs.x == kRansLow;
-  return ok;
+  return !kRans || (rs.pos == rs.W && rs.x == kRansLow);
 }
 
 template <uint32_t D>
 __device__ inline bool fast_dispatch(FastSmem& S, const uint8_t* const recp[2], uint16_t* out,
-                                     uint32_t m0, uint32_t m1) {
-  if (m0 == kModeRaw && m1 == kModeRans) return fast_tiles<kModeRaw, kModeRans, D>(S, recp, out);
-  if (m0 == kModeRaw && m1 == kModeRaw) return fast_tiles<kModeRaw, kModeRaw, D>(S, recp, out);
-  if (m0 == kModeRaw && m1 == kModeConst) return fast_tiles<kModeRaw, kModeConst, D>(S, recp, out);
-  if (m0 == kModeRans && m1 == kModeRaw) return fast_tiles<kModeRans, kModeRaw, D>(S, recp, out);
-  if (m0 == kModeRans && m1 == kModeConst) return fast_tiles<kModeRans, kModeConst, D>(S, recp, out);
-  if (m0 == kModeConst && m1 == kModeRans) return fast_tiles<kModeConst, kModeRans, D>(S, recp, out);
-  if (m0 == kModeConst && m1 == kModeRaw) return fast_tiles<kModeConst, kModeRaw, D>(S, recp, out);
-  return fast_tiles<kModeConst, kModeConst, D>(S, recp, out);
+                                     uint32_t m0, uint32_t m1, PreRun& pre, uint32_t& crc0, uint32_t& crc1) {
+  if (m0 == kModeRaw && m1 == kModeRans) return fast_tiles<kModeRaw, kModeRans, D>(S, recp, out, pre, crc0, crc1);
+  if (m0 == kModeRaw && m1 == kModeRaw) return fast_tiles<kModeRaw, kModeRaw, D>(S, recp, out, pre, crc0, crc1);
+  if (m0 == kModeRaw && m1 == kModeConst) return fast_tiles<kModeRaw, kModeConst, D>(S, recp, out, pre, crc0, crc1);
+  if (m0 == kModeRans && m1 == kModeRaw) return fast_tiles<kModeRans, kModeRaw, D>(S, recp, out, pre, crc0, crc1);
+  if (m0 == kModeRans && m1 == kModeConst) return fast_tiles<kModeRans, kModeConst, D>(S, recp, out, pre, crc0, crc1);
+  if (m0 == kModeConst && m1 == kModeRans) return fast_tiles<kModeConst, kModeRans, D>(S, recp, out, pre, crc0, crc1);
+  if (m0 == kModeConst && m1 == kModeRaw) return fast_tiles<kModeConst, kModeRaw, D>(S, recp, out, pre, crc0, crc1);
+  return fast_tiles<kModeConst, kModeConst, D>(S, recp, out, pre, crc0, crc1);
 }
 
-__global__ void __launch_bounds__(kFastThreads)
+// CRC register of a 16-byte stream header; comp complements its first four
+// bytes (the record's initial value when the header opens the record)
+__device__ inline uint32_t crc_header16(const uint32_t* t, const uint8_t* h, bool comp) {
+  uint4 v = __ldcg(reinterpret_cast<const uint4*>(h));
+  if (comp) v.x = ~v.x;
+  uint32_t c = crc_word(t, 0u, v.x);
+  c = crc_word(t, c, v.y);
+  c = crc_word(t, c, v.z);
+  return crc_word(t, c, v.w);
+}
+
+__global__ void __launch_bounds__(kFastThreads, 6)
 k_lossless_decode_fast(LosslessShape sh, FrameBatch b, uint8_t* ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   FastSmem& S = *reinterpret_cast<FastSmem*>(smem_raw);
@@ -446,7 +533,6 @@ k_lossless_decode_fast(LosslessShape sh, FrameBatch b, uint8_t* ws) {
   const uint32_t D = sh.D;
   const bool shape_ok = (D * sh.tc == kMaxChunkValues) && (D == 128u || D == 64u);
   crc_tables_init(S.crc_t);
-  crc_join_init(&S.join);
   for (uint32_t g = blockIdx.x; g < nrec; g += gridDim.x) {
     __syncthreads();
     const uint32_t fr = frame_of(S.base, b.n, g), r = g - S.base[fr];
@@ -461,22 +547,24 @@ k_lossless_decode_fast(LosslessShape sh, FrameBatch b, uint8_t* ws) {
     const uint32_t len = ld_u32(e + 8), want = ld_u32(e + 12);
     const uint8_t* rec = src + off;
     int st = kOk;
-    if (!defer && len > kCrcOneRound) {  // cannot be a valid full-chunk record; let the general decoder report it
-      defer = true;
-    }
+    if (!defer && len > 2u * kRawStream) defer = true;  // cannot be a valid full-chunk record
+    uint32_t b0 = 0, b1 = 0;
     if (!defer) {
-      uint32_t got = crc32_block_128(rec, len, S.crc_t, &S.join, S.red);
-      if (tid == 0) S.crc_ok = (got == want);
-      __syncthreads();
-      st = S.crc_ok ? kOk : kErrCorrupt;
       const uint32_t n = kMaxChunkValues;
-      if (st == kOk) st = block_parse_stream(rec, len, n, &S.si[0], S.freq[0], S.tmp);
+      st = block_parse_stream(rec, len, n, &S.si[0], S.freq[0], S.tmp);
       if (st == kOk) {
-        const uint32_t b0 = S.si[0].bytes;
+        b0 = S.si[0].bytes;
         st = block_parse_stream(rec + b0, len - b0, n, &S.si[1], S.freq[1], S.tmp);
-        if (st == kOk && b0 + S.si[1].bytes != len) st = kErrCorrupt;
+        b1 = S.si[1].bytes;
+        if (st == kOk && b0 + b1 != len) st = kErrCorrupt;
       }
-      if (st == kOk && S.si[0].mode == kModeRans && S.si[1].mode == kModeRans) defer = true;
+      if (st == kOk) {
+        const uint32_t m0 = S.si[0].mode, m1 = S.si[1].mode;
+        if (m0 == kModeRans && m1 == kModeRans) defer = true;
+        // the pre-pass region must fit one round of runs
+        const uint32_t pre = m0 != kModeRaw && m1 != kModeRaw ? len : m0 != kModeRaw ? b0 : m1 != kModeRaw ? b1 : 0u;
+        if (pre > 2048u * kCrcRegionMaxUnits) defer = true;
+      }
     }
     if (defer) {
       if (tid == 0)
@@ -489,12 +577,44 @@ k_lossless_decode_fast(LosslessShape sh, FrameBatch b, uint8_t* ws) {
       continue;
     }
     const uint32_t m0 = S.si[0].mode, m1 = S.si[1].mode;
+    const bool raw0 = m0 == kModeRaw, raw1 = m1 == kModeRaw;
+    // CRC pre-pass region: the bytes the tiles do not see. The whole record when
+    // neither plane is RAW, else the other stream record (left-aligned when it
+    // follows the RAW stream, so that no shift by its runtime length is needed)
+    PreRun pre;
+    if (!raw0 && !raw1) pre.init(rec, len, false, true);
+    else if (raw0 && !raw1) pre.init(rec + b0, b1, true, false);
+    else if (!raw0 && raw1) pre.init(rec, b0, false, true);
+    else pre.init(rec, 0, false, false);
     if (m0 == kModeRans) block_dec_lut(S.freq[0], S.cum, S.lut, S.tmp);
     else if (m1 == kModeRans) block_dec_lut(S.freq[1], S.cum, S.lut, S.tmp);
-    const uint8_t* recp[2] = {rec, rec + S.si[0].bytes};
+    const uint8_t* recp[2] = {rec, rec + b0};
     uint16_t* out = dst + (uint64_t(slice) * sh.T + t0) * D;
-    const bool ok = D == 128u ? fast_dispatch<128>(S, recp, out, m0, m1)
-                              : fast_dispatch<64>(S, recp, out, m0, m1);
+    uint32_t cr0 = 0, cr1 = 0;
+    bool ok = D == 128u ? fast_dispatch<128>(S, recp, out, m0, m1, pre, cr0, cr1)
+                        : fast_dispatch<64>(S, recp, out, m0, m1, pre, cr0, cr1);
+    const uint32_t prc = !(raw0 && raw1) ? crc_join_lanes(pre.c, pre.q, S.red) : 0u;
+    const uint32_t p0 = raw0 ? crc_join_lanes(cr0, 32u, S.red) : 0u;  // 512-byte lane runs
+    const uint32_t p1 = raw1 ? crc_join_lanes(cr1, 32u, S.red) : 0u;
+    if (tid == 0) {
+      const uint32_t x64k = kCrcPow.q[32][7], x16 = kCrcPow.u[1];  // x^(8 * 65536), x^(8 * 16)
+      const uint32_t xraw = gf2_mul(x64k, x16);                     // x^(8 * full RAW stream record)
+      const uint32_t fin = want ^ 0xffffffffu;
+      uint32_t lhs = prc, rhs = fin;
+      if (raw0 && !raw1) {
+        // register(H0' P0) * x^(8 * 2048q) + pre == register(record') * x^(8 * pad)
+        const uint32_t q = (b1 + 2047u) >> 11, pad = 2048u * q - b1;
+        const uint32_t hp = gf2_mul(crc_header16(S.crc_t, rec, true), x64k) ^ p0;
+        lhs = gf2_mul(hp, kCrcPow.q[q][7]) ^ prc;
+        rhs = gf2_mul(fin, kCrcPow.u[pad >> 4]);
+      } else if (!raw0 && raw1) {
+        lhs = gf2_mul(prc, xraw) ^ gf2_mul(crc_header16(S.crc_t, rec + b0, false), x64k) ^ p1;
+      } else if (raw0 && raw1) {
+        const uint32_t hp = gf2_mul(crc_header16(S.crc_t, rec, true), x64k) ^ p0;
+        lhs = gf2_mul(hp, xraw) ^ gf2_mul(crc_header16(S.crc_t, rec + b0, false), x64k) ^ p1;
+      }
+      ok = ok && lhs == rhs;
+    }
     if (!__syncthreads_and(ok) && tid == 0)
       atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(kErrCorrupt));
   }
