@@ -248,6 +248,23 @@ int kvc_stage_stream_encode(const uint8_t* d_sym, uint32_t n, uint8_t* d_out, vo
 int kvc_stage_stream_decode(const uint8_t* d_rec, uint32_t rec_bytes, uint32_t n, uint8_t* d_sym,
                             kvc_result* d_res, cudaStream_t stream);
 
+/* kvc_stage_stream_encode_noalloc: kvc_stage_stream_encode without a caller
+ * scratch buffer and without allocating anything. It is for callers that must
+ * not allocate device memory at the point of the call: a serving loop that has
+ * handed all device memory to a preallocated pool, code running inside an
+ * allocator's out-of-memory handler (where allocating again would recurse), or
+ * a latency-critical path that must not wait on an allocation. The scratch is
+ * a fixed 128 KiB array inside the library, one per device, so n is limited to
+ * 65536 symbols; larger n returns KVC_ERR_CAPACITY. The output bytes and
+ * d_res are those of kvc_stage_stream_encode for the same symbols.
+ * The first call on a device looks the array up (set-up on the host); make
+ * that first call before starting any stream capture. Calls that overlap on
+ * the device (on different streams, or from different host threads without
+ * ordering) share the one array and race: order them. The container format
+ * has no counterpart of this call; it only changes where the scratch lives. */
+int kvc_stage_stream_encode_noalloc(const uint8_t* d_sym, uint32_t n, uint8_t* d_out,
+                                    kvc_result* d_res, cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

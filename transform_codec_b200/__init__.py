@@ -27,6 +27,7 @@ EXPORTS = [
     "kvc_encode_lossless", "kvc_decode_lossless", "kvc_encode_transform", "kvc_decode_transform",
     "kvc_status_string", "kvc_calibrate_pca", "kvc_allocate_bits",
     "kvc_stage_crc32", "kvc_stage_stream_encode", "kvc_stage_stream_decode",
+    "kvc_stage_stream_encode_noalloc",
     "kvc_profile_begin", "kvc_profile_end",
     "kvc_batch_workspace_bytes", "kvc_encode_batch", "kvc_decode_batch",
 ]
@@ -91,6 +92,7 @@ def _load():
         "kvc_stage_crc32": ([vp, sz, vp, vp], i32),
         "kvc_stage_stream_encode": ([vp, u32, vp, vp, vp, vp], i32),
         "kvc_stage_stream_decode": ([vp, u32, u32, vp, vp, vp], i32),
+        "kvc_stage_stream_encode_noalloc": ([vp, u32, vp, vp, vp], i32),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -319,6 +321,13 @@ def stage_crc32(src, n: int, out, stream=None):
 def stage_stream_encode(sym, n: int, out, scratch, res, stream=None):
     _check(_lib.kvc_stage_stream_encode(_dptr(sym), n, _dptr(out), _dptr(scratch), _dptr(res),
                                         _stream(stream)), "kvc_stage_stream_encode")
+
+
+def stage_stream_encode_noalloc(sym, n: int, out, res, stream=None):
+    """kvc_stage_stream_encode with the library's own fixed scratch (n <= 65536);
+    allocates nothing. Overlapping calls on one device share that scratch."""
+    _check(_lib.kvc_stage_stream_encode_noalloc(_dptr(sym), n, _dptr(out), _dptr(res),
+                                                _stream(stream)), "kvc_stage_stream_encode_noalloc")
 
 
 def stage_stream_decode(rec, rec_bytes: int, n: int, sym, res, stream=None):

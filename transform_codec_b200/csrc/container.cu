@@ -4,6 +4,9 @@
 // aggregate checksum; "QATC v2 checksum validated": corrupt or truncated
 // payloads are refused before restore). Also the stage kernels used to check
 // the CRC and rANS stages on their own.
+#include <mutex>
+
+#include "kvc.h"
 #include "kvc_device.cuh"
 #include "kvc_internal.h"
 
@@ -388,3 +391,50 @@ cudaError_t launch_stage_stream_decode(const uint8_t* rec, uint32_t rec_bytes, u
 }
 
 }  // namespace kvc
+
+// ------------------------------------------------------------ no-alloc stage encode
+// Word scratch of kvc_stage_stream_encode_noalloc: the rANS encoder emits at
+// most one 16-bit word per symbol, so kMaxChunkValues words (128 KiB) cover the
+// largest stream. The encoder writes every scratch word it later reads, so the
+// array needs no clearing between calls.
+static __device__ __align__(256) uint16_t g_noalloc_scratch[kvc::kMaxChunkValues];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+uint16_t* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device, looked up once
+// per device (the first call on a device does this set-up).
+uint16_t* noalloc_scratch(int* status) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) {
+    *status = KVC_ERR_CUDA;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+      *status = KVC_ERR_CUDA;
+      return nullptr;
+    }
+    g_noalloc_ptr[dev] = static_cast<uint16_t*>(p);
+  }
+  *status = KVC_OK;
+  return g_noalloc_ptr[dev];
+}
+}  // namespace
+
+extern "C" int kvc_stage_stream_encode_noalloc(const uint8_t* d_sym, uint32_t n, uint8_t* d_out,
+                                               kvc_result* d_res, cudaStream_t stream) {
+  if (n > kvc::kMaxChunkValues) return KVC_ERR_CAPACITY;
+  if (n == 0 || !d_sym || !d_out || !d_res || (reinterpret_cast<uintptr_t>(d_out) & 15u))
+    return KVC_ERR_INVALID;
+  int status = KVC_OK;
+  uint16_t* scratch = noalloc_scratch(&status);
+  if (!scratch) return status;
+  return kvc::launch_stage_stream_encode(d_sym, n, d_out, scratch, d_res, stream) == cudaSuccess
+             ? KVC_OK
+             : KVC_ERR_CUDA;
+}
