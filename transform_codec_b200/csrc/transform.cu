@@ -82,24 +82,34 @@ struct Split {  // i -> (component slot, token) for i = slot * tcc + t
   }
 };
 
-struct __align__(16) EncSmem {
-  float Q[kD * kD];            // Q[k][j]
-  float xy[kTile * kD];        // x' then y, [token][k or j]
-  uint8_t codes[kD * kMaxCt];  // [j][t]
-  float zs[kD][kMaxCt / kTile][2];
-  uint32_t crc_t[1024];
-  uint32_t hist[256], freq[256], rem[256], fc[256], rcp[256];
-  uint32_t states[kMaxLanes];
-  uint32_t tmp[32], red[32];
-  uint32_t W[4], wbeg[4], sub_len[4];
-  uint32_t k, mode, bytes, off;
+// ---------------------------------------------------------------------------
+// Transform encode, part 1 (k_transform_project): one CTA per middle record.
+// Per 128-token tile the keys are de-rotated into x[k][t] (fp32), then every
+// thread accumulates an 8-token x 8-component tile of y_c = sum_k Q[k][c] x_k
+// in fp64 with k ascending over the coded components only (Q's coded columns
+// converted to fp64 once per record), and y is rounded to fp32. Each (coded
+// component, 64-token block) pair is then quantised by one thread: zero point
+// and scale go straight to the record's side information in the slot, the
+// codes to a token-major [t][128] byte array in the slot's scratch area.
+constexpr uint32_t kProjTokens = 128;  // tokens per projection tile
+constexpr uint32_t kCodesRow = 128;    // bytes per token row of the code array in the slot
+
+struct __align__(16) ProjSmem {
+  double Qd[kD * kD];               // Q[k][c], coded components c < n_coded, fp64
+  float xy[kD * kProjTokens];       // x[k][t], then y[c][t]
   CompInfo ci;
+  uint32_t cidx[kD];                // coded component c -> channel-space index j
+  uint32_t tmp[32];
 };
 
+__device__ inline uint8_t* slot_codes(uint8_t* slot, uint64_t slot_bytes) {
+  return slot + slot_bytes - (2u * kD * kMaxCt + 64u);
+}
+
 __global__ void __launch_bounds__(kThreads)
-k_transform_encode_mid(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLayout ws) {
+k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLayout ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  EncSmem& S = *reinterpret_cast<EncSmem*>(smem_raw);
+  ProjSmem& S = *reinterpret_cast<ProjSmem*>(smem_raw);
   const uint32_t tid = threadIdx.x, nthr = blockDim.x;
   const uint32_t rps = 1u + sh.n_mid;
   const uint32_t gs = blockIdx.x / sh.n_mid, c = blockIdx.x % sh.n_mid;  // slice of the batch
@@ -112,144 +122,354 @@ k_transform_encode_mid(TransformShape sh, TransformPlanDev pl, FrameBatch b, Enc
   const uint32_t t0 = sh.s_end + c * sh.ct, tcc = min(sh.ct, sh.r_start - t0);
   const uint32_t nb = (tcc + kTile - 1) / kTile;
   const uint16_t* xs = src + uint64_t(ls) * sh.T * kD;
+  uint8_t* rec = ws.slots + uint64_t(r) * ws.slot_bytes;
+  uint8_t* codes = slot_codes(rec, ws.slot_bytes);
+
+  build_comp_info(pl.widths + uint64_t(sidx) * kD, S.ci, S.tmp);
+  if (tid < kD && S.ci.width[tid]) S.cidx[S.ci.coded_idx[tid]] = tid;
+  __syncthreads();
+  const uint32_t nc = S.ci.n_coded;
+  {
+    const float* q = pl.bases + uint64_t(sidx) * kD * kD;
+    for (uint32_t i = tid; i < kD * nc; i += nthr) {
+      const uint32_t k = i / nc, cc = i - k * nc;
+      S.Qd[k * kD + cc] = double(__ldg(q + k * kD + S.cidx[cc]));
+    }
+  }
+  // side-information padding of the record (its values are written below)
+  const uint32_t side = 8u * nc * nb;
+  if (tid < pad16(side) - side) rec[side + tid] = 0;
+  __syncthreads();
+
+  const uint32_t tg = tid >> 4, cg = tid & 15u;  // tokens 8tg .. 8tg+7, components 8cg .. 8cg+7
+  const bool busy = 8u * cg < nc;
+  for (uint32_t tb = 0; tb < tcc; tb += kProjTokens) {
+    const uint32_t bl = min(kProjTokens, tcc - tb);
+    // x[k][t]: thread handles (token, 8-channel group q < 8) and the RoPE partners q + 8
+    for (uint32_t idx = tid; idx < kProjTokens * 8u; idx += nthr) {
+      const uint32_t tt = idx % kProjTokens, q = idx / kProjTokens;  // a warp: 32 consecutive tokens
+      float a[8], bb[8];
+      if (tt < bl) {
+        const uint4* row = reinterpret_cast<const uint4*>(xs + uint64_t(t0 + tb + tt) * kD);
+        const uint4 va = __ldg(row + q), vb = __ldg(row + q + 8u);
+        const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+#pragma unroll
+        for (uint32_t i = 0; i < 4; ++i) {
+          a[2 * i] = bf16_to_f32(wa[i] & 0xffffu);
+          a[2 * i + 1] = bf16_to_f32(wa[i] >> 16);
+          bb[2 * i] = bf16_to_f32(wb[i] & 0xffffu);
+          bb[2 * i + 1] = bf16_to_f32(wb[i] >> 16);
+        }
+        if (is_key) {
+          const float4* cs = reinterpret_cast<const float4*>(pl.rope + (uint64_t(t0 + tb + tt) * (kD / 2) + 8u * q) * 2u);
+#pragma unroll
+          for (uint32_t i = 0; i < 4; ++i) {
+            const float4 v = __ldg(cs + i);  // (cos, sin) of channels 8q + 2i, 8q + 2i + 1
+            const float c0 = v.x, s0 = v.y, c1 = v.z, s1 = v.w;
+            const float na0 = __fadd_rn(__fmul_rn(a[2 * i], c0), __fmul_rn(bb[2 * i], s0));
+            const float nb0 = __fsub_rn(__fmul_rn(bb[2 * i], c0), __fmul_rn(a[2 * i], s0));
+            const float na1 = __fadd_rn(__fmul_rn(a[2 * i + 1], c1), __fmul_rn(bb[2 * i + 1], s1));
+            const float nb1 = __fsub_rn(__fmul_rn(bb[2 * i + 1], c1), __fmul_rn(a[2 * i + 1], s1));
+            a[2 * i] = na0; bb[2 * i] = nb0; a[2 * i + 1] = na1; bb[2 * i + 1] = nb1;
+          }
+        }
+      } else {
+#pragma unroll
+        for (uint32_t i = 0; i < 8; ++i) a[i] = bb[i] = 0.0f;
+      }
+#pragma unroll
+      for (uint32_t i = 0; i < 8; ++i) {
+        S.xy[(8u * q + i) * kProjTokens + tt] = a[i];
+        S.xy[(8u * q + i + 64u) * kProjTokens + tt] = bb[i];
+      }
+    }
+    __syncthreads();
+    double acc[8][8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
+    if (busy) {
+#pragma unroll 2
+      for (uint32_t k = 0; k < kD; ++k) {
+        const float4 x0 = *reinterpret_cast<const float4*>(&S.xy[k * kProjTokens + 8u * tg]);
+        const float4 x1 = *reinterpret_cast<const float4*>(&S.xy[k * kProjTokens + 8u * tg + 4u]);
+        const double xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        const double2* qp = reinterpret_cast<const double2*>(&S.Qd[k * kD + 8u * cg]);
+        const double2 q0 = qp[0], q1 = qp[1], q2 = qp[2], q3 = qp[3];
+        const double qv[8] = {q0.x, q0.y, q1.x, q1.y, q2.x, q2.y, q3.x, q3.y};
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[i][j] = fma(qv[j], xv[i], acc[i][j]);
+      }
+    }
+    __syncthreads();
+    if (busy) {
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const uint32_t cc = 8u * cg + j;
+        if (cc < nc) {
+          float4* yp = reinterpret_cast<float4*>(&S.xy[cc * kProjTokens + 8u * tg]);
+          yp[0] = make_float4(__double2float_rn(acc[0][j]), __double2float_rn(acc[1][j]),
+                              __double2float_rn(acc[2][j]), __double2float_rn(acc[3][j]));
+          yp[1] = make_float4(__double2float_rn(acc[4][j]), __double2float_rn(acc[5][j]),
+                              __double2float_rn(acc[6][j]), __double2float_rn(acc[7][j]));
+        }
+      }
+    }
+    __syncthreads();
+    // quantiser: one thread per (coded component, 64-token block of this tile)
+    const uint32_t nbt = (bl + kTile - 1) / kTile;
+    for (uint32_t p = tid; p < nc * nbt; p += nthr) {
+      const uint32_t cc = p / nbt, h = p - cc * nbt;
+      const uint32_t j = S.cidx[cc], w = S.ci.width[j];
+      const uint32_t lo = h * kTile, n = min(kTile, bl - lo);
+      const float* y = &S.xy[cc * kProjTokens + lo];
+      float mn = y[0], mx = mn;
+      for (uint32_t tt = 1; tt < n; ++tt) {
+        const float v = y[tt];
+        if (v < mn) mn = v;
+        if (v > mx) mx = v;
+      }
+      const uint32_t levels = (1u << w) - 1u;
+      const float s = (mx == mn) ? 0.0f : __fdiv_rn(__fsub_rn(mx, mn), float(levels));
+      uint8_t* cp = codes + uint64_t(tb + lo) * kCodesRow + j;
+      for (uint32_t tt = 0; tt < n; ++tt) cp[tt * kCodesRow] = uint8_t(quantize(y[tt], mn, s, levels));
+      const uint32_t blk = (tb + lo) / kTile;
+      uint32_t* zp = reinterpret_cast<uint32_t*>(rec + 8u * (cc * nb + blk));
+      zp[0] = __float_as_uint(mn);
+      zp[1] = __float_as_uint(s);
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Transform encode, part 2 (k_transform_entropy): one CTA per middle record.
+// The codes come back from the slot into shared rows of 132 bytes (conflict-
+// free both along a row and down a column). Warp w owns the stream of width
+// b = w + 1: it counts the stream's symbols (ballots for alphabets up to 32,
+// shared atomics above), normalises the counts and builds its coding tables.
+// The rANS groups of all streams then run side by side, one warp per (stream,
+// group), and the record is laid out and written stream by stream.
+constexpr uint32_t kCodesStride = 132;  // shared code row: 128 bytes + 4 bytes of padding
+constexpr uint32_t kTabPool = 512;      // sum over widths 1..8 of 2^b, rounded up
+
+struct __align__(16) EntSmem {
+  uint8_t codes[kMaxCt * kCodesStride];  // codes[t * 132 + j]
+  uint32_t freq[8][256];                 // per width stream, zero past its alphabet
+  uint32_t fc[kTabPool], rcp[kTabPool], rem[kTabPool], hist[kTabPool];
+  uint32_t states[8][kMaxLanes];
+  uint32_t W[8][4], wbeg[8][4], sub_len[8][4];
+  uint32_t k[8], mode[8], bytes[8], off[9];
+  uint32_t crc_t[1024];
+  uint32_t tmp[32], red[32];
+  CompInfo ci;
+};
+
+__device__ inline uint32_t tab_base(uint32_t b) { return (1u << b) - 2u; }  // 2 + 4 + ... + 2^(b-1)
+
+// Largest-remainder normalisation of one width stream by one warp (the rule of
+// block_normalize): counts hist[0 .. A), A = 2^b, n symbols; writes freq[0 .. 256)
+// and the coding tables fc / rcp of the first A symbols. Returns k.
+__device__ inline uint32_t warp_normalize(const uint32_t* hist, uint32_t A, uint32_t n, uint32_t* freq,
+                                          uint32_t* rem, uint32_t* fc, uint32_t* rcp) {
+  const uint32_t lane = threadIdx.x & 31u;
+  uint32_t present = 0;
+  for (uint32_t s = lane; s < A; s += 32u) present += hist[s] ? 1u : 0u;
+  const uint32_t k = __reduce_add_sync(0xffffffffu, present);
+  uint32_t fsum = 0;
+  for (uint32_t s = lane; s < 256u; s += 32u) {
+    const uint32_t c = s < A ? hist[s] : 0u;
+    uint32_t f = 0, r = 0;
+    if (k >= 2 && c) {
+      const uint32_t q = c * (kProbScale - k);
+      f = 1u + q / n;
+      r = q % n;
+    } else if (k == 1 && c) {
+      f = kProbScale;
+    }
+    if (s < A) rem[s] = r;
+    freq[s] = f;
+    fsum += f;
+  }
+  const uint32_t sum = __reduce_add_sync(0xffffffffu, fsum);
+  __syncwarp();
+  if (k >= 2 && sum < kProbScale) {
+    const uint32_t d = kProbScale - sum;
+    for (uint32_t s = lane; s < A; s += 32u) {
+      if (!hist[s]) continue;
+      const uint32_t r = rem[s];
+      uint32_t rank = 0;
+      for (uint32_t s2 = 0; s2 < A; ++s2) {
+        const uint32_t r2 = rem[s2];
+        rank += (hist[s2] != 0u) & ((r2 > r) | ((r2 == r) & (s2 < s)));
+      }
+      if (rank < d) freq[s] += 1u;
+    }
+  }
+  __syncwarp();
+  // coding tables: fc[s] = f | cum << 16, rcp[s] = floor((2^32 - 1) / f)
+  uint32_t carry = 0;
+  for (uint32_t s0 = 0; s0 < A; s0 += 32u) {
+    const uint32_t s = s0 + lane;
+    const uint32_t f = s < A ? freq[s] : 0u;
+    uint32_t incl = f;
+#pragma unroll
+    for (uint32_t o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (s < A) {
+      fc[s] = f | ((carry + incl - f) << 16);
+      rcp[s] = f ? 0xffffffffu / f : 0u;
+    }
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  __syncwarp();
+  return k;
+}
+
+__global__ void __launch_bounds__(kThreads)
+k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLayout ws) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  EntSmem& S = *reinterpret_cast<EntSmem*>(smem_raw);
+  const uint32_t tid = threadIdx.x, nthr = blockDim.x;
+  const uint32_t warp = tid >> 5, lane = tid & 31u;
+  const uint32_t rps = 1u + sh.n_mid;
+  const uint32_t gs = blockIdx.x / sh.n_mid, c = blockIdx.x % sh.n_mid;
+  const uint32_t r = gs * rps + 1u + c;
+  const uint32_t fr = frame_of(b.rec_base, b.n, r);
+  const uint32_t ls = (r - b.rec_base[fr]) / rps;
+  const uint32_t sidx = b.f[fr].first_slice + ls;
+  const uint32_t t0 = sh.s_end + c * sh.ct, tcc = min(sh.ct, sh.r_start - t0);
+  const uint32_t nb = (tcc + kTile - 1) / kTile;
+  uint8_t* rec = ws.slots + uint64_t(r) * ws.slot_bytes;
+  const uint8_t* codes_g = slot_codes(rec, ws.slot_bytes);
+  uint16_t* scratch = reinterpret_cast<uint16_t*>(rec + ws.slot_bytes - (2u * kD * kMaxCt + 64u));
 
   crc_tables_init(S.crc_t);
-  {
-    const uint4* q4 = reinterpret_cast<const uint4*>(pl.bases + uint64_t(sidx) * kD * kD);
-    uint4* d4 = reinterpret_cast<uint4*>(S.Q);
-    for (uint32_t i = tid; i < kD * kD / 4; i += nthr) d4[i] = __ldg(q4 + i);
-  }
   build_comp_info(pl.widths + uint64_t(sidx) * kD, S.ci, S.tmp);
-
-  const uint32_t tg = tid >> 4, jg = tid & 15u;  // projection tile: tokens 4tg.., comps 8jg..
-  for (uint32_t blk = 0; blk < nb; ++blk) {
-    const uint32_t bl = min(kTile, tcc - blk * kTile);
-    const uint32_t tb = t0 + blk * kTile;
-    for (uint32_t idx = tid; idx < kTile * (kD / 2); idx += nthr) {
-      const uint32_t tt = idx / (kD / 2), i = idx % (kD / 2);
-      float a = 0.0f, b = 0.0f;
-      if (tt < bl) {
-        const uint16_t* row = xs + uint64_t(tb + tt) * kD;
-        a = bf16_to_f32(row[i]);
-        b = bf16_to_f32(row[i + kD / 2]);
-        if (is_key) {
-          const float2 cs = reinterpret_cast<const float2*>(pl.rope)[uint64_t(tb + tt) * (kD / 2) + i];
-          float na = __fadd_rn(__fmul_rn(a, cs.x), __fmul_rn(b, cs.y));
-          float nb2 = __fsub_rn(__fmul_rn(b, cs.x), __fmul_rn(a, cs.y));
-          a = na;
-          b = nb2;
-        }
-      }
-      S.xy[tt * kD + i] = a;
-      S.xy[tt * kD + i + kD / 2] = b;
-    }
-    __syncthreads();
-    double acc[4][8];
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 8; ++b) acc[a][b] = 0.0;
-    for (uint32_t k = 0; k < kD; ++k) {
-      const float4 q0 = *reinterpret_cast<const float4*>(&S.Q[k * kD + jg * 8]);
-      const float4 q1 = *reinterpret_cast<const float4*>(&S.Q[k * kD + jg * 8 + 4]);
-      const double qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const double xv = S.xy[(tg * 4 + a) * kD + k];
-#pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] = fma(qv[b], xv, acc[a][b]);
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int a = 0; a < 4; ++a)
-#pragma unroll
-      for (int b = 0; b < 8; ++b) S.xy[(tg * 4 + a) * kD + jg * 8 + b] = __double2float_rn(acc[a][b]);
-    __syncthreads();
-    if (tid < kD) {
-      const uint32_t j = tid, w = S.ci.width[j];
-      if (w) {
-        float mn = S.xy[j], mx = mn;
-        for (uint32_t tt = 1; tt < bl; ++tt) {
-          float v = S.xy[tt * kD + j];
-          if (v < mn) mn = v;
-          if (v > mx) mx = v;
-        }
-        const uint32_t levels = (1u << w) - 1u;
-        const float s = (mx == mn) ? 0.0f : __fdiv_rn(__fsub_rn(mx, mn), float(levels));
-        for (uint32_t tt = 0; tt < bl; ++tt)
-          S.codes[j * kMaxCt + blk * kTile + tt] = uint8_t(quantize(S.xy[tt * kD + j], mn, s, levels));
-        S.zs[j][blk][0] = mn;
-        S.zs[j][blk][1] = s;
-      }
-    }
-    __syncthreads();
+  for (uint32_t i = tid; i < tcc * (kCodesRow / 4u); i += nthr) {
+    const uint32_t t = i >> 5, q = i & 31u;
+    *reinterpret_cast<uint32_t*>(&S.codes[t * kCodesStride + 4u * q]) =
+        __ldcg(reinterpret_cast<const uint32_t*>(codes_g + uint64_t(t) * kCodesRow) + q);
   }
+  __syncthreads();  // the codes are in shared memory: the slot's scratch may now take words
 
-  // record: side info, then one stream per present bit width
-  uint8_t* rec = ws.slots + uint64_t(r) * ws.slot_bytes;
-  uint16_t* scratch = reinterpret_cast<uint16_t*>(rec + ws.slot_bytes - (2u * kD * kMaxCt + 64u));
-  const uint32_t side = 8u * S.ci.n_coded * nb;
-  if (tid < kD && S.ci.width[tid]) {
-    uint32_t* p32 = reinterpret_cast<uint32_t*>(rec + 8u * S.ci.coded_idx[tid] * nb);
-    for (uint32_t blk = 0; blk < nb; ++blk) {
-      p32[2 * blk] = __float_as_uint(S.zs[tid][blk][0]);
-      p32[2 * blk + 1] = __float_as_uint(S.zs[tid][blk][1]);
-    }
-  }
-  if (tid < pad16(side) - side) rec[side + tid] = 0;
-  uint32_t off = pad16(side);
   const Split split(tcc);
-  for (uint32_t b = 1; b <= 8; ++b) {
-    const uint32_t m = S.ci.bcount[b];
+  // ---- per-stream counts and tables: warp w takes width b = w + 1
+  {
+    const uint32_t bw = warp + 1u, m = S.ci.bcount[bw];
+    if (m) {
+      const uint32_t A = 1u << bw, n = m * tcc, base = S.ci.bstart[bw];
+      uint32_t* hist = S.hist + tab_base(bw);
+      for (uint32_t s = lane; s < A; s += 32u) hist[s] = 0;
+      __syncwarp();
+      uint32_t cnt = 0;
+      for (uint32_t i0 = 0; i0 < n; i0 += 32u) {
+        const uint32_t i = i0 + lane;
+        uint32_t v = 0xffffffffu;
+        if (i < n) {
+          uint32_t a, t;
+          split(i, a, t);
+          v = S.codes[t * kCodesStride + S.ci.comp[base + a]];
+        }
+        if (A <= 32u) {
+          for (uint32_t s = 0; s < A; ++s) {
+            const uint32_t bal = __ballot_sync(0xffffffffu, v == s);
+            if (lane == s) cnt += __popc(bal);
+          }
+        } else if (i < n) {
+          atomicAdd(&hist[v], 1u);
+        }
+      }
+      if (A <= 32u && lane < A) hist[lane] = cnt;
+      __syncwarp();
+      S.k[warp] = 0;  // written by every lane with the same value below
+      const uint32_t k = warp_normalize(hist, A, n, S.freq[warp], S.rem + tab_base(bw),
+                                        S.fc + tab_base(bw), S.rcp + tab_base(bw));
+      if (lane == 0) S.k[warp] = k;
+    }
+  }
+  __syncthreads();
+  // ---- rANS groups of every stream, one warp per (stream, group)
+  {
+    uint32_t pair = 0;
+    for (uint32_t bw = 1; bw <= 8; ++bw) {
+      const uint32_t m = S.ci.bcount[bw];
+      if (!m || S.k[bw - 1] < 2) continue;
+      const uint32_t n = m * tcc, base = S.ci.bstart[bw];
+      const uint32_t N = rans_lanes(n), G = rans_groups(N);
+      const uint32_t wbase = base * tcc;  // word scratch of this stream: one word per symbol
+      for (uint32_t g = 0; g < G; ++g, ++pair) {
+        if (pair % (nthr >> 5) != warp) continue;
+        uint32_t b0, len0, b1 = n, len1;
+        lane_range(n, N, g * kGroupLanes, b0, len0);
+        if (g + 1 < G) lane_range(n, N, (g + 1) * kGroupLanes, b1, len1);
+        auto sym = [&](uint32_t i) -> uint32_t {
+          uint32_t a, t;
+          split(i, a, t);
+          return S.codes[t * kCodesStride + S.ci.comp[base + a]];
+        };
+        uint32_t x;
+        const uint32_t Wg = rans_encode_group(sym, n, N, g, S.fc + tab_base(bw), S.rcp + tab_base(bw),
+                                              scratch + wbase + b0, b1 - b0, &x);
+        if (g * kGroupLanes + lane < N) S.states[bw - 1][g * kGroupLanes + lane] = x;
+        if (lane == 0) {
+          S.W[bw - 1][g] = Wg;
+          S.wbeg[bw - 1][g] = wbase + b1 - Wg;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // ---- layout: modes and record offsets
+  const uint32_t side = 8u * S.ci.n_coded * nb;
+  if (tid == 0) {
+    uint32_t off = pad16(side);
+    for (uint32_t bw = 1; bw <= 8; ++bw) {
+      S.off[bw - 1] = off;
+      const uint32_t m = S.ci.bcount[bw];
+      if (!m) continue;
+      const uint32_t n = m * tcc, k = S.k[bw - 1], raw_b = 16u + pad16(n);
+      uint32_t mode, bytes;
+      if (k == 1) { mode = kModeConst; bytes = 16; }
+      else {
+        const uint32_t rb = rans_layout(n, k, S.W[bw - 1], S.sub_len[bw - 1]);
+        if (rb < raw_b) { mode = kModeRans; bytes = rb; }
+        else { mode = kModeRaw; bytes = raw_b; }
+      }
+      S.mode[bw - 1] = mode;
+      S.bytes[bw - 1] = bytes;
+      off += bytes;
+    }
+    S.off[8] = off;
+  }
+  __syncthreads();
+  for (uint32_t bw = 1; bw <= 8; ++bw) {
+    const uint32_t m = S.ci.bcount[bw];
     if (!m) continue;
-    const uint32_t n = m * tcc, base = S.ci.bstart[b];
+    const uint32_t n = m * tcc, base = S.ci.bstart[bw];
     auto sym = [&](uint32_t i) -> uint32_t {
       uint32_t a, t;
       split(i, a, t);
-      return S.codes[S.ci.comp[base + a] * kMaxCt + t];
+      return S.codes[t * kCodesStride + S.ci.comp[base + a]];
     };
+    block_write_stream(rec + S.off[bw - 1], S.mode[bw - 1], n, S.bytes[bw - 1], sym(0), S.k[bw - 1],
+                       S.freq[bw - 1], S.states[bw - 1], scratch, S.wbeg[bw - 1], S.W[bw - 1],
+                       S.sub_len[bw - 1], sym, S.tmp);
     __syncthreads();
-    for (uint32_t i = tid; i < 256; i += nthr) S.hist[i] = 0;
-    __syncthreads();
-    for (uint32_t i = tid; i < n; i += nthr) atomicAdd(&S.hist[sym(i)], 1u);
-    __syncthreads();
-    const uint32_t k = block_normalize(S.hist, n, S.freq, S.rem, S.tmp);
-    block_enc_tables(S.freq, S.fc, S.rcp, S.tmp);
-    const uint32_t N = rans_lanes(n), G = rans_groups(N);
-    const uint32_t warp = tid >> 5, lane = tid & 31u;
-    if (k >= 2 && warp < G) {
-      uint32_t b0, len0, b1 = n, len1;
-      lane_range(n, N, warp * kGroupLanes, b0, len0);
-      if (warp + 1 < G) lane_range(n, N, (warp + 1) * kGroupLanes, b1, len1);
-      uint32_t x;
-      uint32_t Wg = rans_encode_group(sym, n, N, warp, S.fc, S.rcp, scratch + b0, b1 - b0, &x);
-      if (warp * kGroupLanes + lane < N) S.states[warp * kGroupLanes + lane] = x;
-      if (lane == 0) { S.W[warp] = Wg; S.wbeg[warp] = b1 - Wg; }
-    }
-    __syncthreads();
-    if (tid == 0) {
-      const uint32_t raw_b = 16u + pad16(n);
-      if (k == 1) { S.mode = kModeConst; S.bytes = 16; }
-      else {
-        uint32_t rb = rans_layout(n, k, S.W, S.sub_len);
-        if (rb < raw_b) { S.mode = kModeRans; S.bytes = rb; }
-        else { S.mode = kModeRaw; S.bytes = raw_b; }
-      }
-      S.k = k;
-    }
-    __syncthreads();
-    block_write_stream(rec + off, S.mode, n, S.bytes, sym(0), S.k, S.freq, S.states, scratch,
-                       S.wbeg, S.W, S.sub_len, sym, S.tmp);
-    off += S.bytes;
   }
-  __syncthreads();
-  uint32_t crc = crc32_block_aligned(rec, off, S.crc_t, S.red);
+  const uint32_t len = S.off[8];
+  const uint32_t crc = crc32_block_aligned(rec, len, S.crc_t, S.red);
   if (tid == 0) {
-    ws.rec_len[r] = off;
+    ws.rec_len[r] = len;
     ws.rec_crc[r] = crc;
   }
 }
+
 
 // Raw record of each slice: sink rows, then recent rows, bf16 bytes, padded.
 __global__ void __launch_bounds__(kThreads)
@@ -302,6 +522,8 @@ struct __align__(1024) DecSmem {
 };
 
 static_assert(sizeof(DecSmem) + 1024 <= 232448, "decoder shared memory exceeds the per-block limit");
+static_assert(sizeof(ProjSmem) <= 232448, "projection shared memory exceeds the per-block limit");
+static_assert(sizeof(EntSmem) <= 232448 / 2, "entropy kernel should fit two blocks per SM");
 
 __global__ void __launch_bounds__(kThreads)
 k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t* ws) {
@@ -564,12 +786,22 @@ cudaError_t launch_transform_encode(const TransformShape& s, const TransformPlan
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || s.n_mid == 0) return e;
-  size_t smem = sizeof(EncSmem);
-  e = cudaFuncSetAttribute(k_transform_encode_mid, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  const uint32_t grid = n_slices * s.n_mid;
+  e = cudaFuncSetAttribute(k_transform_project, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(sizeof(ProjSmem)));
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_transform_entropy, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(sizeof(EntSmem)));
   if (e != cudaSuccess) return e;
   {
-    ProfRange pr_("transform_encode_mid", st);
-    k_transform_encode_mid<<<n_slices * s.n_mid, kThreads, smem, st>>>(s, p, b, ws);
+    ProfRange pr_("transform_project", st);
+    k_transform_project<<<grid, kThreads, sizeof(ProjSmem), st>>>(s, p, b, ws);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  {
+    ProfRange pr_("transform_entropy", st);
+    k_transform_entropy<<<grid, kThreads, sizeof(EntSmem), st>>>(s, p, b, ws);
   }
   return cudaGetLastError();
 }
