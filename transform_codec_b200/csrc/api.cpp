@@ -75,6 +75,7 @@ struct kvc_plan_s {
   uint8_t* d_widths = nullptr;
   float* d_rope = nullptr;
   uint8_t* d_qsplit = nullptr;
+  CompInfo* d_comp = nullptr;
 };
 
 namespace {
@@ -196,6 +197,25 @@ uint32_t sw128_offset_host(uint32_t row, uint32_t kbyte, uint32_t rows) {
 
 // Per slice, Q as two bf16 pieces (hi = rne(Q), lo = rne(Q - hi)) laid out as the
 // B operand of D[token][k] = sum_j y[token][j] * Q[k][j]: row k, K index j.
+// Component order of one slice from its 128 widths (see CompInfo).
+void comp_info(const uint8_t* widths, CompInfo& ci) {
+  ci = CompInfo{};
+  uint32_t coded = 0;
+  for (uint32_t j = 0; j < 128; ++j) {
+    ci.width[j] = widths[j];
+    ci.coded_idx[j] = coded;
+    if (widths[j]) ++coded;
+  }
+  ci.n_coded = coded;
+  uint32_t base = 0;
+  for (uint32_t b = 1; b <= 8; ++b) {
+    ci.bstart[b] = base;
+    for (uint32_t j = 0; j < 128; ++j)
+      if (widths[j] == b) ci.comp[base++] = j;
+    ci.bcount[b] = base - ci.bstart[b];
+  }
+}
+
 void split_bases(const float* bases, uint32_t S, std::vector<uint8_t>& out) {
   const uint32_t D = 128;
   out.assign(size_t(S) * kQSplitBytes, 0);
@@ -224,6 +244,7 @@ void free_plan(kvc_plan_s* p) {
   if (p->d_widths) cudaFree(p->d_widths);
   if (p->d_rope) cudaFree(p->d_rope);
   if (p->d_qsplit) cudaFree(p->d_qsplit);
+  if (p->d_comp) cudaFree(p->d_comp);
   delete p;
 }
 
@@ -294,6 +315,8 @@ extern "C" int kvc_plan_create(const kvc_plan_desc* desc, kvc_plan_t** out) {
     rope_table(d.n_tokens, d.head_dim, d.rope_theta, cs);
     std::vector<uint8_t> qs;
     split_bases(d.bases, p->S, qs);
+    std::vector<CompInfo> ci(p->S);
+    for (uint32_t s = 0; s < p->S; ++s) comp_info(p->widths.data() + size_t(s) * 128u, ci[s]);
     const size_t nb = size_t(p->S) * d.head_dim * d.head_dim * sizeof(float);
     bool ok = cudaMalloc(&p->d_bases, nb) == cudaSuccess &&
               cudaMalloc(&p->d_widths, p->widths.size()) == cudaSuccess &&
@@ -304,7 +327,10 @@ extern "C" int kvc_plan_create(const kvc_plan_desc* desc, kvc_plan_t** out) {
               cudaMemcpy(p->d_rope, cs.data(), cs.size() * sizeof(float), cudaMemcpyHostToDevice) ==
                   cudaSuccess &&
               cudaMalloc(&p->d_qsplit, qs.size()) == cudaSuccess &&
-              cudaMemcpy(p->d_qsplit, qs.data(), qs.size(), cudaMemcpyHostToDevice) == cudaSuccess;
+              cudaMemcpy(p->d_qsplit, qs.data(), qs.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMalloc(&p->d_comp, ci.size() * sizeof(CompInfo)) == cudaSuccess &&
+              cudaMemcpy(p->d_comp, ci.data(), ci.size() * sizeof(CompInfo), cudaMemcpyHostToDevice) ==
+                  cudaSuccess;
     if (!ok) {
       free_plan(p);
       return KVC_ERR_CUDA;
@@ -435,7 +461,7 @@ int encode_frames(const kvc_plan_s* plan, int path, const kvc_frame* fr, uint32_
     if (path == KVC_PATH_LOSSLESS) {
       e = launch_lossless_encode(plan->ls, b, L, stream);
     } else {
-      TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope, plan->d_qsplit};
+      TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope, plan->d_qsplit, plan->d_comp};
       e = launch_transform_encode(plan->ts, pd, b, L, stream);
     }
     if (e != cudaSuccess) return KVC_ERR_CUDA;
@@ -493,7 +519,7 @@ int decode_frames(const kvc_plan_s* plan, int path, const kvc_frame* fr, uint32_
     if (path == KVC_PATH_LOSSLESS) {
       e = launch_lossless_decode(plan->ls, b, ws, max_rec, stream);
     } else {
-      TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope, plan->d_qsplit};
+      TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope, plan->d_qsplit, plan->d_comp};
       e = launch_transform_decode(plan->ts, pd, b, ws, max_rec, stream);
     }
     if (e != cudaSuccess) return KVC_ERR_CUDA;

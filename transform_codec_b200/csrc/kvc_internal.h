@@ -129,11 +129,23 @@ struct TransformShape {
   uint32_t L, H, T, D, ct, block, n_sink, n_recent;
   uint32_t s_end, r_start, n_mid;   // regions and middle chunks per slice
 };
+// Per-slice component order of the transform path (head_dim 128), computed on
+// the host when the plan is made: the coded components (width >= 1) grouped by
+// width b = 1..8, ascending index within a width; coded_idx is the rank of a
+// coded component among all coded components in index order.
+struct alignas(16) CompInfo {
+  uint32_t width[128];
+  uint32_t comp[128];       // components ordered by (width, index), widths >= 1
+  uint32_t coded_idx[128];  // rank among coded components (width >= 1)
+  uint32_t bstart[10], bcount[10];
+  uint32_t n_coded;
+};
 struct TransformPlanDev {
   const float* bases;      // [S][D][D], Q[k*D + j]
   const uint8_t* widths;   // [S][D]
   const float* rope;       // [T][D/2][2] cos, sin
   const uint8_t* qsplit;   // [S][hi, lo][128 x 256 B] Q as bf16 pieces, B-operand layout
+  const CompInfo* comp;    // [S]
 };
 constexpr uint32_t kQSplitBytes = 2u * 128u * 256u;  // per slice
 uint64_t transform_slot_bytes(const TransformShape& s);

@@ -43,32 +43,33 @@ __device__ inline uint32_t quantize(float y, float z, float s, uint32_t levels) 
   return uint32_t(r);
 }
 
-struct __align__(16) CompInfo {
-  uint32_t width[kD];
-  uint32_t comp[kD];        // components ordered by (width, index), widths >= 1
-  uint32_t coded_idx[kD];   // rank among coded components (width >= 1)
-  uint32_t bstart[10], bcount[10];
-  uint32_t n_coded;
-};
+// quantize() with the division replaced where it cannot matter. With r =
+// RN(1/s), qa = RN((y - z) * r) is within 2^-22 * qa of the correctly rounded
+// quotient RN((y - z) / s) (two roundings of relative size 2^-24 against one).
+// Every decision quantize() takes on the quotient (rounding to an integer,
+// the clamps at 0 and at levels) changes only at half-integers, so when qa is
+// farther than qa * 2^-19 from the nearest half-integer both give the same
+// code; the few values inside that window, and every value of a block whose
+// reciprocal is not finite, take the IEEE division. The result always equals
+// quantize().
+__device__ inline uint32_t quantize_r(float y, float z, float s, float r, bool exact, uint32_t levels) {
+  if (s == 0.0f) return 0u;
+  const float a = __fsub_rn(y, z);
+  float q = __fmul_rn(a, r);
+  const float fl = floorf(q);
+  const float d = fabsf(__fsub_rn(__fsub_rn(q, fl), 0.5f));  // distance to floor(q) + 0.5
+  if (exact || d <= __fmul_rn(q, 0x1p-19f)) q = __fdiv_rn(a, s);
+  const float rr = rintf(q);
+  if (!(rr > 0.0f)) return 0u;
+  if (rr >= float(levels)) return levels;
+  return uint32_t(rr);
+}
 
-// widths of slice sidx -> component order per bit width (needs blockDim >= 128)
-__device__ inline void build_comp_info(const uint8_t* widths, CompInfo& ci, uint32_t* tmp) {
-  const uint32_t j = threadIdx.x;
-  const uint32_t w = j < kD ? widths[j] : 0u;
-  if (j < kD) ci.width[j] = w;
-  uint32_t tot;
-  uint32_t ci_idx = block_exclusive_scan(j < kD && w > 0 ? 1u : 0u, tmp, &tot);
-  if (j < kD) ci.coded_idx[j] = ci_idx;
-  if (j == 0) ci.n_coded = tot;
-  uint32_t base = 0;
-  for (uint32_t b = 1; b <= 8; ++b) {
-    uint32_t flag = (j < kD && w == b) ? 1u : 0u;
-    uint32_t cnt;
-    uint32_t ex = block_exclusive_scan(flag, tmp, &cnt);
-    if (flag) ci.comp[base + ex] = j;
-    if (j == 0) { ci.bstart[b] = base; ci.bcount[b] = cnt; }
-    base += cnt;
-  }
+// The plan's per-slice component order, copied into shared memory.
+__device__ inline void load_comp_info(const CompInfo* src, CompInfo& dst) {
+  const uint4* s4 = reinterpret_cast<const uint4*>(src);
+  uint4* d4 = reinterpret_cast<uint4*>(&dst);
+  for (uint32_t i = threadIdx.x; i < sizeof(CompInfo) / 16u; i += blockDim.x) d4[i] = __ldg(s4 + i);
   __syncthreads();
 }
 
@@ -83,23 +84,37 @@ struct Split {  // i -> (component slot, token) for i = slot * tcc + t
 };
 
 // ---------------------------------------------------------------------------
-// Transform encode, part 1 (k_transform_project): one CTA per middle record.
-// Per 128-token tile the keys are de-rotated into x[k][t] (fp32), then every
-// thread accumulates an 8-token x 8-component tile of y_c = sum_k Q[k][c] x_k
-// in fp64 with k ascending over the coded components only (Q's coded columns
-// converted to fp64 once per record), and y is rounded to fp32. Each (coded
-// component, 64-token block) pair is then quantised by one thread: zero point
-// and scale go straight to the record's side information in the slot, the
-// codes to a token-major [t][128] byte array in the slot's scratch area.
-constexpr uint32_t kProjTokens = 128;  // tokens per projection tile
+// Transform encode, part 1 (k_transform_project): one CTA per middle record,
+// 64-token tiles (one quantiser block each). The keys are de-rotated in fp32
+// and x is kept as fp64 in x[k][t]; every thread accumulates a 4-token x
+// 8-component tile of y_c = sum_k Q[k][c] x_k with fused multiply-adds, k
+// ascending, over the coded components (Q's coded columns converted to fp64
+// once per record), and y is rounded to fp32. One thread per coded component
+// then scans the block's tokens in order for the minimum and maximum and sets
+// the scale; all threads then quantise (component, 8-token chunk) items. Zero
+// point and scale go straight to the record's side information in the slot.
+// The codes are staged in padded token rows and
+// copied to a token-major [t][128] byte array in the slot's scratch area, and
+// the symbol counts of every width stream are gathered behind them for the
+// entropy kernel.
+constexpr uint32_t kProjTokens = 64;   // tokens per projection tile = quantiser block
 constexpr uint32_t kCodesRow = 128;    // bytes per token row of the code array in the slot
+constexpr uint32_t kCodesStride = 132; // shared code row: 128 bytes + 4 bytes of padding
+constexpr uint32_t kTabPool = 512;     // sum over widths 1..8 of 2^b, rounded up
+constexpr uint32_t kHistOffset = kCodesRow * kMaxCt;  // counts follow the codes in the slot
+constexpr uint32_t kYStride = kD + 1u;                 // y[t][c] row stride in floats (odd: conflict-free)
+
+__device__ inline uint32_t tab_base(uint32_t b) { return (1u << b) - 2u; }  // 2 + 4 + ... + 2^(b-1)
 
 struct __align__(16) ProjSmem {
-  double Qd[kD * kD];               // Q[k][c], coded components c < n_coded, fp64
-  float xy[kD * kProjTokens];       // x[k][t], then y[c][t]
+  double Qd[kD * kD];                          // Q[k][c], coded components c < n_coded, fp64
+  double x[kD * kProjTokens];                  // x[k][t]; then y[c][t] as fp32 in the same space
+  uint8_t codes[kProjTokens * kCodesStride];   // this tile's codes, codes[t * 132 + j]
+  uint32_t hist[kTabPool];                     // symbol counts of the record per width stream
+  float4 qp[kD];                               // per coded component: zero point, scale, 1/scale, flags
+  uint32_t ccnt[8][kD];                        // counts of symbols 0..7 per coded component
   CompInfo ci;
-  uint32_t cidx[kD];                // coded component c -> channel-space index j
-  uint32_t tmp[32];
+  uint32_t cidx[kD];                           // coded component c -> channel-space index j
 };
 
 __device__ inline uint8_t* slot_codes(uint8_t* slot, uint64_t slot_bytes) {
@@ -111,6 +126,7 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
   extern __shared__ __align__(16) uint8_t smem_raw[];
   ProjSmem& S = *reinterpret_cast<ProjSmem*>(smem_raw);
   const uint32_t tid = threadIdx.x, nthr = blockDim.x;
+  const uint32_t warp = tid >> 5, lane = tid & 31u;
   const uint32_t rps = 1u + sh.n_mid;
   const uint32_t gs = blockIdx.x / sh.n_mid, c = blockIdx.x % sh.n_mid;  // slice of the batch
   const uint32_t r = gs * rps + 1u + c;                                   // record of the batch
@@ -125,15 +141,35 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
   uint8_t* rec = ws.slots + uint64_t(r) * ws.slot_bytes;
   uint8_t* codes = slot_codes(rec, ws.slot_bytes);
 
-  build_comp_info(pl.widths + uint64_t(sidx) * kD, S.ci, S.tmp);
+  load_comp_info(pl.comp + sidx, S.ci);
   if (tid < kD && S.ci.width[tid]) S.cidx[S.ci.coded_idx[tid]] = tid;
+  for (uint32_t i = tid; i < kTabPool; i += nthr) S.hist[i] = 0;
+  for (uint32_t i = tid; i < 8u * kD; i += nthr) (&S.ccnt[0][0])[i] = 0;
   __syncthreads();
   const uint32_t nc = S.ci.n_coded;
   {
     const float* q = pl.bases + uint64_t(sidx) * kD * kD;
-    for (uint32_t i = tid; i < kD * nc; i += nthr) {
-      const uint32_t k = i / nc, cc = i - k * nc;
-      S.Qd[k * kD + cc] = double(__ldg(q + k * kD + S.cidx[cc]));
+    // warp per row k, lanes along the coded columns; a lane's four column
+    // indices are read once and four rows' loads are issued together
+    uint32_t col[4];
+#pragma unroll
+    for (uint32_t u = 0; u < 4; ++u) col[u] = lane + 32u * u < nc ? S.cidx[lane + 32u * u] : 0u;
+    for (uint32_t k0 = warp; k0 < kD; k0 += 4u * (nthr >> 5)) {
+      float v[4][4];
+#pragma unroll
+      for (uint32_t kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (uint32_t u = 0; u < 4; ++u) {
+          const uint32_t k = k0 + kk * (nthr >> 5);
+          v[kk][u] = (k < kD && lane + 32u * u < nc) ? __ldg(q + k * kD + col[u]) : 0.0f;
+        }
+#pragma unroll
+      for (uint32_t kk = 0; kk < 4; ++kk)
+#pragma unroll
+        for (uint32_t u = 0; u < 4; ++u) {
+          const uint32_t k = k0 + kk * (nthr >> 5);
+          if (k < kD && lane + 32u * u < nc) S.Qd[k * kD + lane + 32u * u] = double(v[kk][u]);
+        }
     }
   }
   // side-information padding of the record (its values are written below)
@@ -141,13 +177,15 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
   if (tid < pad16(side) - side) rec[side + tid] = 0;
   __syncthreads();
 
-  const uint32_t tg = tid >> 4, cg = tid & 15u;  // tokens 8tg .. 8tg+7, components 8cg .. 8cg+7
-  const bool busy = 8u * cg < nc;
+  float* y = reinterpret_cast<float*>(S.x);    // y[t][c] (row stride kYStride), after the projection
+  // thread: tokens 4tg .. 4tg+3; components 32jb + 2cg + h for jb < 4, h < 2, so the
+  // 16 threads of a token group read a whole row of Q with 16-byte loads
+  const uint32_t tg = tid >> 4, cg = tid & 15u;
   for (uint32_t tb = 0; tb < tcc; tb += kProjTokens) {
     const uint32_t bl = min(kProjTokens, tcc - tb);
     // x[k][t]: thread handles (token, 8-channel group q < 8) and the RoPE partners q + 8
     for (uint32_t idx = tid; idx < kProjTokens * 8u; idx += nthr) {
-      const uint32_t tt = idx % kProjTokens, q = idx / kProjTokens;  // a warp: 32 consecutive tokens
+      const uint32_t tt = idx % kProjTokens, q = idx / kProjTokens;
       float a[8], bb[8];
       if (tt < bl) {
         const uint4* row = reinterpret_cast<const uint4*>(xs + uint64_t(t0 + tb + tt) * kD);
@@ -179,70 +217,126 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
       }
 #pragma unroll
       for (uint32_t i = 0; i < 8; ++i) {
-        S.xy[(8u * q + i) * kProjTokens + tt] = a[i];
-        S.xy[(8u * q + i + 64u) * kProjTokens + tt] = bb[i];
+        S.x[(8u * q + i) * kProjTokens + tt] = double(a[i]);
+        S.x[(8u * q + i + 64u) * kProjTokens + tt] = double(bb[i]);
       }
     }
     __syncthreads();
-    double acc[8][8];
+    double acc[4][8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
-    if (busy) {
 #pragma unroll 2
-      for (uint32_t k = 0; k < kD; ++k) {
-        const float4 x0 = *reinterpret_cast<const float4*>(&S.xy[k * kProjTokens + 8u * tg]);
-        const float4 x1 = *reinterpret_cast<const float4*>(&S.xy[k * kProjTokens + 8u * tg + 4u]);
-        const double xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-        const double2* qp = reinterpret_cast<const double2*>(&S.Qd[k * kD + 8u * cg]);
-        const double2 q0 = qp[0], q1 = qp[1], q2 = qp[2], q3 = qp[3];
-        const double qv[8] = {q0.x, q0.y, q1.x, q1.y, q2.x, q2.y, q3.x, q3.y};
+    for (uint32_t k = 0; k < kD; ++k) {
+      const double2* xp = reinterpret_cast<const double2*>(&S.x[k * kProjTokens + 4u * tg]);
+      const double2 x0 = xp[0], x1 = xp[1];
+      const double xv[4] = {x0.x, x0.y, x1.x, x1.y};
+      const double* qrow = &S.Qd[k * kD + 2u * cg];
+      double qv[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+      for (int jb = 0; jb < 4; ++jb) {
+        const double2 q2 = *reinterpret_cast<const double2*>(qrow + 32 * jb);
+        qv[2 * jb] = q2.x;
+        qv[2 * jb + 1] = q2.y;
+      }
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[i][j] = fma(qv[j], xv[i], acc[i][j]);
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fma(qv[j], xv[i], acc[i][j]);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t cc = 32u * (j >> 1) + 2u * cg + (j & 1);
+      if (cc < nc) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) y[(4u * tg + i) * kYStride + cc] = __double2float_rn(acc[i][j]);
       }
     }
     __syncthreads();
-    if (busy) {
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const uint32_t cc = 8u * cg + j;
-        if (cc < nc) {
-          float4* yp = reinterpret_cast<float4*>(&S.xy[cc * kProjTokens + 8u * tg]);
-          yp[0] = make_float4(__double2float_rn(acc[0][j]), __double2float_rn(acc[1][j]),
-                              __double2float_rn(acc[2][j]), __double2float_rn(acc[3][j]));
-          yp[1] = make_float4(__double2float_rn(acc[4][j]), __double2float_rn(acc[5][j]),
-                              __double2float_rn(acc[6][j]), __double2float_rn(acc[7][j]));
-        }
-      }
-    }
-    __syncthreads();
-    // quantiser: one thread per (coded component, 64-token block of this tile)
-    const uint32_t nbt = (bl + kTile - 1) / kTile;
-    for (uint32_t p = tid; p < nc * nbt; p += nthr) {
-      const uint32_t cc = p / nbt, h = p - cc * nbt;
-      const uint32_t j = S.cidx[cc], w = S.ci.width[j];
-      const uint32_t lo = h * kTile, n = min(kTile, bl - lo);
-      const float* y = &S.xy[cc * kProjTokens + lo];
-      float mn = y[0], mx = mn;
-      for (uint32_t tt = 1; tt < n; ++tt) {
-        const float v = y[tt];
+    // quantiser, part 1: one thread per coded component scans the block's
+    // tokens in order for the minimum and maximum (as a sequential scan finds
+    // them) and sets the scale
+    const uint32_t blk = tb / kTile;
+    if (tid < nc) {
+      const uint32_t cc = tid, j = S.cidx[cc], w = S.ci.width[j];
+      const float* yc = y + cc;
+      float mn = yc[0], mx = mn;
+#pragma unroll 8
+      for (uint32_t tt = 1; tt < bl; ++tt) {
+        const float v = yc[tt * kYStride];
         if (v < mn) mn = v;
         if (v > mx) mx = v;
       }
       const uint32_t levels = (1u << w) - 1u;
       const float s = (mx == mn) ? 0.0f : __fdiv_rn(__fsub_rn(mx, mn), float(levels));
-      uint8_t* cp = codes + uint64_t(tb + lo) * kCodesRow + j;
-      for (uint32_t tt = 0; tt < n; ++tt) cp[tt * kCodesRow] = uint8_t(quantize(y[tt], mn, s, levels));
-      const uint32_t blk = (tb + lo) / kTile;
+      const float rs = s == 0.0f ? 0.0f : __frcp_rn(s);
+      S.qp[cc] = make_float4(mn, s, rs, __uint_as_float(levels | (rs < 0x1p126f ? 0u : 0x100u)));
       uint32_t* zp = reinterpret_cast<uint32_t*>(rec + 8u * (cc * nb + blk));
       zp[0] = __float_as_uint(mn);
       zp[1] = __float_as_uint(s);
     }
     __syncthreads();
+    // part 2: every thread takes (component, 8-token chunk) items, consecutive
+    // threads consecutive components
+    const uint32_t nch = (bl + 7u) >> 3;
+    for (uint32_t it = tid; it < nc * nch; it += nthr) {
+      const uint32_t ch = it / nc, cc = it - ch * nc;
+      const uint32_t j = S.cidx[cc], w = S.ci.width[j];
+      const float4 qp = S.qp[cc];
+      const uint32_t levels = __float_as_uint(qp.w) & 0xffu;
+      const bool exact = (__float_as_uint(qp.w) & 0x100u) != 0u;
+      const uint32_t t8 = 8u * ch;
+      float v[8];
+      uint32_t qv[8];
+#pragma unroll
+      for (uint32_t i = 0; i < 8; ++i) v[i] = t8 + i < bl ? y[(t8 + i) * kYStride + cc] : qp.x;
+#pragma unroll
+      for (uint32_t i = 0; i < 8; ++i) qv[i] = quantize_r(v[i], qp.x, qp.y, qp.z, exact, levels);
+      uint32_t cnt_lo = 0, cnt_hi = 0;  // counts of symbols 0..3 and 4..7, a byte each
+      uint32_t* hist = S.hist + tab_base(w);
+#pragma unroll
+      for (uint32_t i = 0; i < 8; ++i) {
+        if (t8 + i < bl) {
+          const uint32_t q = qv[i];
+          S.codes[(t8 + i) * kCodesStride + j] = uint8_t(q);
+          if (q < 8u) {
+            const uint32_t inc = 1u << (8u * (q & 3u));
+            if (q < 4u) cnt_lo += inc; else cnt_hi += inc;
+          } else {
+            atomicAdd(&hist[q], 1u);
+          }
+        }
+      }
+#pragma unroll
+      for (uint32_t q = 0; q < 8; ++q) {
+        const uint32_t n = ((q < 4u ? cnt_lo : cnt_hi) >> (8u * (q & 3u))) & 0xffu;
+        if (n) atomicAdd(&S.ccnt[q][cc], n);  // consecutive lanes, consecutive components
+      }
+    }
+    __syncthreads();
+    // the tile's code rows to the slot (uncoded channels carry whatever was staged)
+    for (uint32_t i = tid; i < bl * (kCodesRow / 4u); i += nthr) {
+      const uint32_t t = i >> 5, q = i & 31u;
+      reinterpret_cast<uint32_t*>(codes + uint64_t(tb + t) * kCodesRow)[q] =
+          *reinterpret_cast<const uint32_t*>(&S.codes[t * kCodesStride + 4u * q]);
+    }
+    __syncthreads();
   }
+  // counts of symbols 0..7 summed over the components of each width
+  if (tid < 64u) {
+    const uint32_t bw = (tid >> 3) + 1u, q = tid & 7u;
+    if (q < (1u << bw)) {
+      uint32_t sum = 0;
+      for (uint32_t cc = 0; cc < nc; ++cc)
+        if (S.ci.width[S.cidx[cc]] == bw) sum += S.ccnt[q][cc];
+      S.hist[tab_base(bw) + q] += sum;
+    }
+  }
+  __syncthreads();
+  for (uint32_t i = tid; i < kTabPool; i += nthr)
+    reinterpret_cast<uint32_t*>(codes + kHistOffset)[i] = S.hist[i];
 }
 
 // ---------------------------------------------------------------------------
@@ -253,8 +347,6 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
 // shared atomics above), normalises the counts and builds its coding tables.
 // The rANS groups of all streams then run side by side, one warp per (stream,
 // group), and the record is laid out and written stream by stream.
-constexpr uint32_t kCodesStride = 132;  // shared code row: 128 bytes + 4 bytes of padding
-constexpr uint32_t kTabPool = 512;      // sum over widths 1..8 of 2^b, rounded up
 
 struct __align__(16) EntSmem {
   uint8_t codes[kMaxCt * kCodesStride];  // codes[t * 132 + j]
@@ -267,8 +359,6 @@ struct __align__(16) EntSmem {
   uint32_t tmp[32], red[32];
   CompInfo ci;
 };
-
-__device__ inline uint32_t tab_base(uint32_t b) { return (1u << b) - 2u; }  // 2 + 4 + ... + 2^(b-1)
 
 // Largest-remainder normalisation of one width stream by one warp (the rule of
 // block_normalize): counts hist[0 .. A), A = 2^b, n symbols; writes freq[0 .. 256)
@@ -331,6 +421,58 @@ __device__ inline uint32_t warp_normalize(const uint32_t* hist, uint32_t A, uint
   return k;
 }
 
+// rANS encode of group g of one width stream (all 32 lanes call): symbol i =
+// a * tcc + t is codes[t * 132 + comp[a]], a < m. The steps are those of
+// rans_encode_group (reverse order, ascending-lane word placement), but each
+// lane's next symbol and its table entries are fetched one step ahead, so
+// only the state update stays on the loop's dependency chain.
+__device__ inline uint32_t encode_codes_group(const uint8_t* codes, const uint32_t* comp, uint32_t m,
+                                              uint32_t tcc, uint32_t n, uint32_t N, uint32_t g,
+                                              const uint32_t* fc, const uint32_t* rcp, uint16_t* words,
+                                              uint32_t cap, uint32_t* x_out) {
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t l = g * kGroupLanes + lane;
+  const bool live = l < N;
+  uint32_t start = 0, len = 0, start0, maxlen;
+  if (live) lane_range(n, N, l, start, len);
+  lane_range(n, N, g * kGroupLanes, start0, maxlen);
+  const uint32_t lt = lanemask_lt();
+  // (a, t) of symbol start + tau, tau counting down from maxlen - 1
+  uint32_t i0 = start + maxlen - 1u;
+  uint32_t a = i0 / tcc, t = i0 - a * tcc;
+  uint32_t j = a < m ? comp[a] : 0u;
+  uint32_t s = (live && maxlen - 1u < len) ? codes[t * kCodesStride + j] : 0u;
+  uint32_t e = fc[s], rc = rcp[s];
+  uint32_t x = kRansLow, pos = cap;
+  for (uint32_t tau = maxlen; tau-- > 0;) {
+    const bool act = live && tau < len;
+    // the next step's symbol and tables, independent of the state
+    uint32_t na = a, nt = t;
+    if (nt == 0u) { na = a - 1u; nt = tcc - 1u; } else { nt = t - 1u; }
+    const uint32_t nj = (na != a && na < m) ? comp[na] : j;
+    const bool nact = live && tau > 0u && tau - 1u < len;
+    const uint32_t ns = nact ? codes[nt * kCodesStride + nj] : 0u;
+    const uint32_t ne = fc[ns], nrc = rcp[ns];
+    const uint32_t f = e & 0xffffu, cum = e >> 16;
+    const bool emit = act && x >= (f << 20);
+    const uint32_t mask = __ballot_sync(0xffffffffu, emit);
+    pos -= __popc(mask);
+    if (emit) {
+      words[pos + __popc(mask & lt)] = uint16_t(x & 0xffffu);
+      x >>= 16;
+    }
+    if (act) {
+      uint32_t q = __umulhi(x, rc);
+      uint32_t rr = x - q * f;
+      if (rr >= f) { ++q; rr -= f; }
+      x = (q << kProbBits) + rr + cum;
+    }
+    a = na; t = nt; j = nj; e = ne; rc = nrc;
+  }
+  *x_out = x;
+  return cap - pos;
+}
+
 __global__ void __launch_bounds__(kThreads)
 k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLayout ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -350,46 +492,36 @@ k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
   uint16_t* scratch = reinterpret_cast<uint16_t*>(rec + ws.slot_bytes - (2u * kD * kMaxCt + 64u));
 
   crc_tables_init(S.crc_t);
-  build_comp_info(pl.widths + uint64_t(sidx) * kD, S.ci, S.tmp);
-  for (uint32_t i = tid; i < tcc * (kCodesRow / 4u); i += nthr) {
-    const uint32_t t = i >> 5, q = i & 31u;
-    *reinterpret_cast<uint32_t*>(&S.codes[t * kCodesStride + 4u * q]) =
-        __ldcg(reinterpret_cast<const uint32_t*>(codes_g + uint64_t(t) * kCodesRow) + q);
+  load_comp_info(pl.comp + sidx, S.ci);
+  {
+    // code rows: 8 vectors of 16 bytes per token, every thread's loads issued first
+    constexpr uint32_t kPer = kMaxCt * 8u / kThreads;
+    uint4 v[kPer];
+#pragma unroll
+    for (uint32_t u = 0; u < kPer; ++u) {
+      const uint32_t i = tid + u * nthr;
+      v[u] = (i >> 3) < tcc ? __ldcg(reinterpret_cast<const uint4*>(codes_g) + i) : make_uint4(0, 0, 0, 0);
+    }
+    for (uint32_t i = tid; i < kTabPool; i += nthr)
+      S.hist[i] = __ldcg(reinterpret_cast<const uint32_t*>(codes_g + kHistOffset) + i);
+#pragma unroll
+    for (uint32_t u = 0; u < kPer; ++u) {
+      const uint32_t i = tid + u * nthr, t = i >> 3, q = i & 7u;
+      if (t < tcc) {
+        uint32_t* d = reinterpret_cast<uint32_t*>(&S.codes[t * kCodesStride + 16u * q]);
+        d[0] = v[u].x; d[1] = v[u].y; d[2] = v[u].z; d[3] = v[u].w;
+      }
+    }
   }
-  __syncthreads();  // the codes are in shared memory: the slot's scratch may now take words
+  __syncthreads();  // codes and counts are in shared memory: the slot's scratch may now take words
 
   const Split split(tcc);
-  // ---- per-stream counts and tables: warp w takes width b = w + 1
+  // ---- per-stream tables from the counts: warp w takes width b = w + 1
   {
     const uint32_t bw = warp + 1u, m = S.ci.bcount[bw];
     if (m) {
-      const uint32_t A = 1u << bw, n = m * tcc, base = S.ci.bstart[bw];
-      uint32_t* hist = S.hist + tab_base(bw);
-      for (uint32_t s = lane; s < A; s += 32u) hist[s] = 0;
-      __syncwarp();
-      uint32_t cnt = 0;
-      for (uint32_t i0 = 0; i0 < n; i0 += 32u) {
-        const uint32_t i = i0 + lane;
-        uint32_t v = 0xffffffffu;
-        if (i < n) {
-          uint32_t a, t;
-          split(i, a, t);
-          v = S.codes[t * kCodesStride + S.ci.comp[base + a]];
-        }
-        if (A <= 32u) {
-          for (uint32_t s = 0; s < A; ++s) {
-            const uint32_t bal = __ballot_sync(0xffffffffu, v == s);
-            if (lane == s) cnt += __popc(bal);
-          }
-        } else if (i < n) {
-          atomicAdd(&hist[v], 1u);
-        }
-      }
-      if (A <= 32u && lane < A) hist[lane] = cnt;
-      __syncwarp();
-      S.k[warp] = 0;  // written by every lane with the same value below
-      const uint32_t k = warp_normalize(hist, A, n, S.freq[warp], S.rem + tab_base(bw),
-                                        S.fc + tab_base(bw), S.rcp + tab_base(bw));
+      const uint32_t k = warp_normalize(S.hist + tab_base(bw), 1u << bw, m * tcc, S.freq[warp],
+                                        S.rem + tab_base(bw), S.fc + tab_base(bw), S.rcp + tab_base(bw));
       if (lane == 0) S.k[warp] = k;
     }
   }
@@ -408,14 +540,10 @@ k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
         uint32_t b0, len0, b1 = n, len1;
         lane_range(n, N, g * kGroupLanes, b0, len0);
         if (g + 1 < G) lane_range(n, N, (g + 1) * kGroupLanes, b1, len1);
-        auto sym = [&](uint32_t i) -> uint32_t {
-          uint32_t a, t;
-          split(i, a, t);
-          return S.codes[t * kCodesStride + S.ci.comp[base + a]];
-        };
         uint32_t x;
-        const uint32_t Wg = rans_encode_group(sym, n, N, g, S.fc + tab_base(bw), S.rcp + tab_base(bw),
-                                              scratch + wbase + b0, b1 - b0, &x);
+        const uint32_t Wg = encode_codes_group(S.codes, S.ci.comp + base, m, tcc, n, N, g,
+                                               S.fc + tab_base(bw), S.rcp + tab_base(bw),
+                                               scratch + wbase + b0, b1 - b0, &x);
         if (g * kGroupLanes + lane < N) S.states[bw - 1][g * kGroupLanes + lane] = x;
         if (lane == 0) {
           S.W[bw - 1][g] = Wg;
@@ -606,7 +734,7 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
       const uint4* q4 = reinterpret_cast<const uint4*>(pl.qsplit + uint64_t(sidx) * kQSplitBytes);
       uint4* b4 = reinterpret_cast<uint4*>(S.b_hi);  // b_hi and b_lo are contiguous
       for (uint32_t i = tid; i < kQSplitBytes / 16u; i += nthr) b4[i] = __ldg(q4 + i);
-      build_comp_info(pl.widths + uint64_t(sidx) * kD, S.ci, S.tmp);
+      load_comp_info(pl.comp + sidx, S.ci);
       if (tid == 0) S.cur_slice = sidx;
       __syncthreads();
     }
