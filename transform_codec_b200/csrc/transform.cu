@@ -43,26 +43,21 @@ __device__ inline uint32_t quantize(float y, float z, float s, uint32_t levels) 
   return uint32_t(r);
 }
 
-// quantize() with the division replaced where it cannot matter. With r =
-// RN(1/s), qa = RN((y - z) * r) is within 2^-22 * qa of the correctly rounded
-// quotient RN((y - z) / s) (two roundings of relative size 2^-24 against one).
-// Every decision quantize() takes on the quotient (rounding to an integer,
-// the clamps at 0 and at levels) changes only at half-integers, so when qa is
+// quantize() without the division where it cannot matter. With r = RN(1/s),
+// qa = RN((y - z) * r) is within 2^-22 * qa of the correctly rounded quotient
+// RN((y - z) / s) (two roundings of relative size 2^-24 against one). Every
+// decision quantize() takes on the quotient (rounding to an integer, the
+// clamps at 0 and at levels) changes only at half-integers, so when qa is
 // farther than qa * 2^-19 from the nearest half-integer both give the same
-// code; the few values inside that window, and every value of a block whose
-// reciprocal is not finite, take the IEEE division. The result always equals
-// quantize().
-__device__ inline uint32_t quantize_r(float y, float z, float s, float r, bool exact, uint32_t levels) {
-  if (s == 0.0f) return 0u;
-  const float a = __fsub_rn(y, z);
-  float q = __fmul_rn(a, r);
+// code. `need` flags the values inside that window, and every value of a
+// block whose reciprocal is not finite: for those the caller uses quantize().
+// A zero scale has r = 0 and gives code 0, as quantize() does.
+__device__ inline uint32_t quantize_fast(float y, float z, float r, uint32_t levels, bool exact, bool& need) {
+  const float q = __fmul_rn(__fsub_rn(y, z), r);
   const float fl = floorf(q);
   const float d = fabsf(__fsub_rn(__fsub_rn(q, fl), 0.5f));  // distance to floor(q) + 0.5
-  if (exact || d <= __fmul_rn(q, 0x1p-19f)) q = __fdiv_rn(a, s);
-  const float rr = rintf(q);
-  if (!(rr > 0.0f)) return 0u;
-  if (rr >= float(levels)) return levels;
-  return uint32_t(rr);
+  need = exact || d <= __fmul_rn(q, 0x1p-19f);
+  return min(__float2uint_rz(rintf(q)), levels);  // negative values convert to 0
 }
 
 // The plan's per-slice component order, copied into shared memory.
@@ -89,10 +84,10 @@ struct Split {  // i -> (component slot, token) for i = slot * tcc + t
 // and x is kept as fp64 in x[k][t]; every thread accumulates a 4-token x
 // 8-component tile of y_c = sum_k Q[k][c] x_k with fused multiply-adds, k
 // ascending, over the coded components (Q's coded columns converted to fp64
-// once per record), and y is rounded to fp32. One thread per coded component
-// then scans the block's tokens in order for the minimum and maximum and sets
-// the scale; all threads then quantise (component, 8-token chunk) items. Zero
-// point and scale go straight to the record's side information in the slot.
+// once per record), and y is rounded to fp32. Two threads per coded
+// component, one per half-block, find the block's minimum and maximum as a
+// sequential scan does, set the scale and quantise their tokens. Zero point
+// and scale go straight to the record's side information in the slot.
 // The codes are staged in padded token rows and
 // copied to a token-major [t][128] byte array in the slot's scratch area, and
 // the symbol counts of every width stream are gathered behind them for the
@@ -111,7 +106,7 @@ struct __align__(16) ProjSmem {
   double x[kD * kProjTokens];                  // x[k][t]; then y[c][t] as fp32 in the same space
   uint8_t codes[kProjTokens * kCodesStride];   // this tile's codes, codes[t * 132 + j]
   uint32_t hist[kTabPool];                     // symbol counts of the record per width stream
-  float4 qp[kD];                               // per coded component: zero point, scale, 1/scale, flags
+  float2 mm[2][kD];                            // per coded component: the two half-blocks' min and max
   uint32_t ccnt[8][kD];                        // counts of symbols 0..7 per coded component
   CompInfo ci;
   uint32_t cidx[kD];                           // coded component c -> channel-space index j
@@ -119,6 +114,106 @@ struct __align__(16) ProjSmem {
 
 __device__ inline uint8_t* slot_codes(uint8_t* slot, uint64_t slot_bytes) {
   return slot + slot_bytes - (2u * kD * kMaxCt + 64u);
+}
+
+// One thread's share of a tile's inputs: items (token tt, 8-channel group q)
+// for idx = tid + 256u, u < 2: bf16 channels 8q .. 8q+7 and their RoPE partners
+// 8q+64 .. 8q+71 and, for keys, the cos/sin pairs. load() issues the global
+// reads; stage() de-rotates in fp32 and writes x[k][t] as fp64.
+struct XFetch {
+  uint4 va[2], vb[2];
+  float4 cs[2][4];
+  uint32_t bl;
+  __device__ __forceinline__ void load(const uint16_t* xs, const float* rope, bool is_key, uint32_t t0,
+                                       uint32_t tb, uint32_t n) {
+    bl = n;
+#pragma unroll
+    for (uint32_t u = 0; u < 2; ++u) {
+      const uint32_t idx = threadIdx.x + u * kThreads, tt = idx % kProjTokens, q = idx / kProjTokens;
+      if (tt < bl) {
+        const uint4* row = reinterpret_cast<const uint4*>(xs + uint64_t(t0 + tb + tt) * kD);
+        va[u] = __ldg(row + q);
+        vb[u] = __ldg(row + q + 8u);
+        if (is_key) {
+          const float4* c4 = reinterpret_cast<const float4*>(rope + (uint64_t(t0 + tb + tt) * (kD / 2) + 8u * q) * 2u);
+#pragma unroll
+          for (uint32_t i = 0; i < 4; ++i) cs[u][i] = __ldg(c4 + i);  // (cos, sin) of channels 8q+2i, 8q+2i+1
+        }
+      }
+    }
+  }
+  __device__ __forceinline__ void stage(double* x, bool is_key) const {
+#pragma unroll
+    for (uint32_t u = 0; u < 2; ++u) {
+      const uint32_t idx = threadIdx.x + u * kThreads, tt = idx % kProjTokens, q = idx / kProjTokens;
+      float a[8], bb[8];
+      if (tt < bl) {
+        const uint32_t wa[4] = {va[u].x, va[u].y, va[u].z, va[u].w}, wb[4] = {vb[u].x, vb[u].y, vb[u].z, vb[u].w};
+#pragma unroll
+        for (uint32_t i = 0; i < 4; ++i) {
+          a[2 * i] = bf16_to_f32(wa[i] & 0xffffu);
+          a[2 * i + 1] = bf16_to_f32(wa[i] >> 16);
+          bb[2 * i] = bf16_to_f32(wb[i] & 0xffffu);
+          bb[2 * i + 1] = bf16_to_f32(wb[i] >> 16);
+        }
+        if (is_key) {
+#pragma unroll
+          for (uint32_t i = 0; i < 4; ++i) {
+            const float c0 = cs[u][i].x, s0 = cs[u][i].y, c1 = cs[u][i].z, s1 = cs[u][i].w;
+            const float na0 = __fadd_rn(__fmul_rn(a[2 * i], c0), __fmul_rn(bb[2 * i], s0));
+            const float nb0 = __fsub_rn(__fmul_rn(bb[2 * i], c0), __fmul_rn(a[2 * i], s0));
+            const float na1 = __fadd_rn(__fmul_rn(a[2 * i + 1], c1), __fmul_rn(bb[2 * i + 1], s1));
+            const float nb1 = __fsub_rn(__fmul_rn(bb[2 * i + 1], c1), __fmul_rn(a[2 * i + 1], s1));
+            a[2 * i] = na0; bb[2 * i] = nb0; a[2 * i + 1] = na1; bb[2 * i + 1] = nb1;
+          }
+        }
+      } else {
+#pragma unroll
+        for (uint32_t i = 0; i < 8; ++i) a[i] = bb[i] = 0.0f;
+      }
+#pragma unroll
+      for (uint32_t i = 0; i < 8; ++i) {
+        x[(8u * q + i) * kProjTokens + tt] = double(a[i]);
+        x[(8u * q + i + 64u) * kProjTokens + tt] = double(bb[i]);
+      }
+    }
+  }
+};
+
+// y[t][c] = sum_k Q[k][c] x[k][t] for this thread's tokens 4tg .. 4tg+3 and
+// components cg + 16jb (jb < NJB), fused multiply-adds with k ascending; then,
+// after a barrier (y overwrites x), the fp32 results of components c < nc.
+template <uint32_t NJB>
+__device__ __forceinline__ void project_tile(const double* x, const double* Qd, float* y, uint32_t tg,
+                                             uint32_t cg, uint32_t nc) {
+  double acc[4][NJB];
+#pragma unroll
+  for (uint32_t i = 0; i < 4; ++i)
+#pragma unroll
+    for (uint32_t jb = 0; jb < NJB; ++jb) acc[i][jb] = 0.0;
+#pragma unroll 2
+  for (uint32_t k = 0; k < kD; ++k) {
+    const double2* xp = reinterpret_cast<const double2*>(&x[k * kProjTokens + 4u * tg]);
+    const double2 x0 = xp[0], x1 = xp[1];
+    const double xv[4] = {x0.x, x0.y, x1.x, x1.y};
+    const double* qrow = &Qd[k * kD + cg];
+    double qv[NJB];
+#pragma unroll
+    for (uint32_t jb = 0; jb < NJB; ++jb) qv[jb] = qrow[16u * jb];
+#pragma unroll
+    for (uint32_t i = 0; i < 4; ++i)
+#pragma unroll
+      for (uint32_t jb = 0; jb < NJB; ++jb) acc[i][jb] = fma(qv[jb], xv[i], acc[i][jb]);
+  }
+  __syncthreads();
+#pragma unroll
+  for (uint32_t jb = 0; jb < NJB; ++jb) {
+    const uint32_t cc = cg + 16u * jb;
+    if (cc < nc) {
+#pragma unroll
+      for (uint32_t i = 0; i < 4; ++i) y[(4u * tg + i) * kYStride + cc] = __double2float_rn(acc[i][jb]);
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -178,141 +273,103 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
   __syncthreads();
 
   float* y = reinterpret_cast<float*>(S.x);    // y[t][c] (row stride kYStride), after the projection
-  // thread: tokens 4tg .. 4tg+3; components 32jb + 2cg + h for jb < 4, h < 2, so the
-  // 16 threads of a token group read a whole row of Q with 16-byte loads
+  // thread: tokens 4tg .. 4tg+3 and components cg + 16jb, jb < ceil(nc / 16)
   const uint32_t tg = tid >> 4, cg = tid & 15u;
+  const uint32_t njb = (nc + 15u) >> 4;
+  XFetch xf;
+  xf.load(xs, pl.rope, is_key, t0, 0, min(kProjTokens, tcc));
   for (uint32_t tb = 0; tb < tcc; tb += kProjTokens) {
     const uint32_t bl = min(kProjTokens, tcc - tb);
-    // x[k][t]: thread handles (token, 8-channel group q < 8) and the RoPE partners q + 8
-    for (uint32_t idx = tid; idx < kProjTokens * 8u; idx += nthr) {
-      const uint32_t tt = idx % kProjTokens, q = idx / kProjTokens;
-      float a[8], bb[8];
-      if (tt < bl) {
-        const uint4* row = reinterpret_cast<const uint4*>(xs + uint64_t(t0 + tb + tt) * kD);
-        const uint4 va = __ldg(row + q), vb = __ldg(row + q + 8u);
-        const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
-#pragma unroll
-        for (uint32_t i = 0; i < 4; ++i) {
-          a[2 * i] = bf16_to_f32(wa[i] & 0xffffu);
-          a[2 * i + 1] = bf16_to_f32(wa[i] >> 16);
-          bb[2 * i] = bf16_to_f32(wb[i] & 0xffffu);
-          bb[2 * i + 1] = bf16_to_f32(wb[i] >> 16);
-        }
-        if (is_key) {
-          const float4* cs = reinterpret_cast<const float4*>(pl.rope + (uint64_t(t0 + tb + tt) * (kD / 2) + 8u * q) * 2u);
-#pragma unroll
-          for (uint32_t i = 0; i < 4; ++i) {
-            const float4 v = __ldg(cs + i);  // (cos, sin) of channels 8q + 2i, 8q + 2i + 1
-            const float c0 = v.x, s0 = v.y, c1 = v.z, s1 = v.w;
-            const float na0 = __fadd_rn(__fmul_rn(a[2 * i], c0), __fmul_rn(bb[2 * i], s0));
-            const float nb0 = __fsub_rn(__fmul_rn(bb[2 * i], c0), __fmul_rn(a[2 * i], s0));
-            const float na1 = __fadd_rn(__fmul_rn(a[2 * i + 1], c1), __fmul_rn(bb[2 * i + 1], s1));
-            const float nb1 = __fsub_rn(__fmul_rn(bb[2 * i + 1], c1), __fmul_rn(a[2 * i + 1], s1));
-            a[2 * i] = na0; bb[2 * i] = nb0; a[2 * i + 1] = na1; bb[2 * i + 1] = nb1;
-          }
-        }
-      } else {
-#pragma unroll
-        for (uint32_t i = 0; i < 8; ++i) a[i] = bb[i] = 0.0f;
-      }
-#pragma unroll
-      for (uint32_t i = 0; i < 8; ++i) {
-        S.x[(8u * q + i) * kProjTokens + tt] = double(a[i]);
-        S.x[(8u * q + i + 64u) * kProjTokens + tt] = double(bb[i]);
-      }
+    xf.stage(S.x, is_key);
+    __syncthreads();
+    switch (njb) {
+      case 1: project_tile<1>(S.x, S.Qd, y, tg, cg, nc); break;
+      case 2: project_tile<2>(S.x, S.Qd, y, tg, cg, nc); break;
+      case 3: project_tile<3>(S.x, S.Qd, y, tg, cg, nc); break;
+      case 4: project_tile<4>(S.x, S.Qd, y, tg, cg, nc); break;
+      case 5: project_tile<5>(S.x, S.Qd, y, tg, cg, nc); break;
+      case 6: project_tile<6>(S.x, S.Qd, y, tg, cg, nc); break;
+      case 7: project_tile<7>(S.x, S.Qd, y, tg, cg, nc); break;
+      default: project_tile<8>(S.x, S.Qd, y, tg, cg, nc); break;
     }
     __syncthreads();
-    double acc[4][8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 8; ++j) acc[i][j] = 0.0;
-#pragma unroll 2
-    for (uint32_t k = 0; k < kD; ++k) {
-      const double2* xp = reinterpret_cast<const double2*>(&S.x[k * kProjTokens + 4u * tg]);
-      const double2 x0 = xp[0], x1 = xp[1];
-      const double xv[4] = {x0.x, x0.y, x1.x, x1.y};
-      const double* qrow = &S.Qd[k * kD + 2u * cg];
-      double qv[8];
-#pragma unroll
-      for (int jb = 0; jb < 4; ++jb) {
-        const double2 q2 = *reinterpret_cast<const double2*>(qrow + 32 * jb);
-        qv[2 * jb] = q2.x;
-        qv[2 * jb + 1] = q2.y;
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fma(qv[j], xv[i], acc[i][j]);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const uint32_t cc = 32u * (j >> 1) + 2u * cg + (j & 1);
-      if (cc < nc) {
-#pragma unroll
-        for (int i = 0; i < 4; ++i) y[(4u * tg + i) * kYStride + cc] = __double2float_rn(acc[i][j]);
-      }
-    }
-    __syncthreads();
-    // quantiser, part 1: one thread per coded component scans the block's
-    // tokens in order for the minimum and maximum (as a sequential scan finds
-    // them) and sets the scale
+    // quantiser: thread (component cc, half h) owns tokens 32h .. 32h+31 of the
+    // block. The halves' minima and maxima, each a sequential scan, combine with
+    // the first half winning ties, which is the sequential scan of the block.
     const uint32_t blk = tb / kTile;
-    if (tid < nc) {
-      const uint32_t cc = tid, j = S.cidx[cc], w = S.ci.width[j];
-      const float* yc = y + cc;
-      float mn = yc[0], mx = mn;
+    const bool qthr = tid < 2u * nc;
+    const uint32_t h = tid >= nc ? 1u : 0u, cc = tid - h * nc;
+    const uint32_t lo = 32u * h, n = bl > lo ? min(32u, bl - lo) : 0u;
+    if (qthr) {
+      const float* yc = y + lo * kYStride + cc;
+      float mn = __int_as_float(0x7f800000), mx = __int_as_float(0xff800000);
+      if (n) {
+        mn = mx = yc[0];
 #pragma unroll 8
-      for (uint32_t tt = 1; tt < bl; ++tt) {
-        const float v = yc[tt * kYStride];
-        if (v < mn) mn = v;
-        if (v > mx) mx = v;
+        for (uint32_t tt = 1; tt < n; ++tt) {
+          const float v = yc[tt * kYStride];
+          if (v < mn) mn = v;
+          if (v > mx) mx = v;
+        }
       }
+      S.mm[h][cc] = make_float2(mn, mx);
+    }
+    __syncthreads();
+    // the next tile's rows are fetched now and land while this one is quantised
+    if (tb + kProjTokens < tcc) xf.load(xs, pl.rope, is_key, t0, tb + kProjTokens, min(kProjTokens, tcc - tb - kProjTokens));
+    if (qthr) {
+      const float2 m0 = S.mm[0][cc], m1 = S.mm[1][cc];
+      const float mn = m1.x < m0.x ? m1.x : m0.x, mx = m1.y > m0.y ? m1.y : m0.y;
+      const uint32_t j = S.cidx[cc], w = S.ci.width[j];
       const uint32_t levels = (1u << w) - 1u;
       const float s = (mx == mn) ? 0.0f : __fdiv_rn(__fsub_rn(mx, mn), float(levels));
       const float rs = s == 0.0f ? 0.0f : __frcp_rn(s);
-      S.qp[cc] = make_float4(mn, s, rs, __uint_as_float(levels | (rs < 0x1p126f ? 0u : 0x100u)));
-      uint32_t* zp = reinterpret_cast<uint32_t*>(rec + 8u * (cc * nb + blk));
-      zp[0] = __float_as_uint(mn);
-      zp[1] = __float_as_uint(s);
-    }
-    __syncthreads();
-    // part 2: every thread takes (component, 8-token chunk) items, consecutive
-    // threads consecutive components
-    const uint32_t nch = (bl + 7u) >> 3;
-    for (uint32_t it = tid; it < nc * nch; it += nthr) {
-      const uint32_t ch = it / nc, cc = it - ch * nc;
-      const uint32_t j = S.cidx[cc], w = S.ci.width[j];
-      const float4 qp = S.qp[cc];
-      const uint32_t levels = __float_as_uint(qp.w) & 0xffu;
-      const bool exact = (__float_as_uint(qp.w) & 0x100u) != 0u;
-      const uint32_t t8 = 8u * ch;
-      float v[8];
-      uint32_t qv[8];
-#pragma unroll
-      for (uint32_t i = 0; i < 8; ++i) v[i] = t8 + i < bl ? y[(t8 + i) * kYStride + cc] : qp.x;
-#pragma unroll
-      for (uint32_t i = 0; i < 8; ++i) qv[i] = quantize_r(v[i], qp.x, qp.y, qp.z, exact, levels);
+      const bool exact = !(rs < 0x1p126f);
+      if (h == 0) {
+        uint32_t* zp = reinterpret_cast<uint32_t*>(rec + 8u * (cc * nb + blk));
+        zp[0] = __float_as_uint(mn);
+        zp[1] = __float_as_uint(s);
+      }
       uint32_t cnt_lo = 0, cnt_hi = 0;  // counts of symbols 0..3 and 4..7, a byte each
-      uint32_t* hist = S.hist + tab_base(w);
+      for (uint32_t t8 = 0; t8 < n; t8 += 8u) {
+        float v[8];
+        uint32_t qv[8], need = 0;
 #pragma unroll
-      for (uint32_t i = 0; i < 8; ++i) {
-        if (t8 + i < bl) {
-          const uint32_t q = qv[i];
-          S.codes[(t8 + i) * kCodesStride + j] = uint8_t(q);
-          if (q < 8u) {
-            const uint32_t inc = 1u << (8u * (q & 3u));
-            if (q < 4u) cnt_lo += inc; else cnt_hi += inc;
-          } else {
-            atomicAdd(&hist[q], 1u);
+        for (uint32_t i = 0; i < 8; ++i) v[i] = t8 + i < n ? y[(lo + t8 + i) * kYStride + cc] : mn;
+#pragma unroll
+        for (uint32_t i = 0; i < 8; ++i) {
+          bool nd;
+          qv[i] = quantize_fast(v[i], mn, rs, levels, exact, nd);
+          need |= uint32_t(nd) << i;
+        }
+        while (need) {  // quotients near a half-integer: the IEEE division decides
+          const uint32_t i = __ffs(need) - 1u;
+          need &= need - 1u;
+          float vi = v[0];
+#pragma unroll
+          for (uint32_t u = 1; u < 8; ++u) vi = u == i ? v[u] : vi;
+          const uint32_t qi = quantize(vi, mn, s, levels);
+#pragma unroll
+          for (uint32_t u = 0; u < 8; ++u) qv[u] = u == i ? qi : qv[u];
+        }
+#pragma unroll
+        for (uint32_t i = 0; i < 8; ++i) {
+          if (t8 + i < n) {
+            const uint32_t q = qv[i];
+            S.codes[(lo + t8 + i) * kCodesStride + j] = uint8_t(q);
+            if (q < 8u) {
+              const uint32_t inc = 1u << (8u * (q & 3u));
+              if (q < 4u) cnt_lo += inc; else cnt_hi += inc;
+            } else {
+              atomicAdd(&S.hist[tab_base(w) + q], 1u);
+            }
           }
         }
       }
 #pragma unroll
       for (uint32_t q = 0; q < 8; ++q) {
-        const uint32_t n = ((q < 4u ? cnt_lo : cnt_hi) >> (8u * (q & 3u))) & 0xffu;
-        if (n) atomicAdd(&S.ccnt[q][cc], n);  // consecutive lanes, consecutive components
+        const uint32_t c = ((q < 4u ? cnt_lo : cnt_hi) >> (8u * (q & 3u))) & 0xffu;
+        if (c) atomicAdd(&S.ccnt[q][cc], c);
       }
     }
     __syncthreads();
