@@ -686,25 +686,156 @@ k_transform_encode_raw(TransformShape sh, FrameBatch b, EncodeLayout ws) {
   }
 }
 
-// Decoder shared memory. Operand tiles come first so each 128-byte-swizzled
-// tile starts on a 1024-byte boundary.
+// Decoder shared memory. The first 128 KiB hold, in turn, the entropy stage's
+// decode tables and refill rings and then the tensor-core operand tiles
+// (each 128-byte-swizzled tile on a 1024-byte boundary).
+constexpr uint32_t kDecLuts = 6;  // rANS streams decoded side by side per round
 struct __align__(1024) DecSmem {
-  uint8_t a_hi[kTcRows * 256];   // y^ as bf16 pieces, A operand [token][component]
-  uint8_t a_lo[kTcRows * 256];
-  uint8_t b_hi[kD * 256];        // Q as bf16 pieces, B operand [channel][component]
-  uint8_t b_lo[kD * 256];
-  uint8_t codes[kD * kMaxCt];    // [j][t]
+  union {
+    struct {
+      uint8_t a_hi[kTcRows * 256];  // y^ as bf16 pieces, A operand [token][component]
+      uint8_t a_lo[kTcRows * 256];
+      uint8_t b_hi[kD * 256];       // Q as bf16 pieces, B operand [channel][component]
+      uint8_t b_lo[kD * 256];
+    } tc;
+    struct {
+      uint32_t lut[kDecLuts][kProbScale];
+      uint16_t ring[kThreads / 32][1024];  // one refill window per warp
+    } ent;
+  } u;
+  uint8_t codes[kMaxCt * kCodesStride];  // codes[t * 132 + j]
   float zs[kD][kMaxCt / kTile][2];
   uint32_t crc_t[1024];
-  uint32_t freq[256], cum[260], lut[kProbScale];
+  uint32_t freq[8][256];                 // per width stream; then f << 16 | cum for the tables
   uint32_t tmp[32], red[32];
-  StreamInfo si;
+  StreamInfo si[8];
+  uint32_t str_off[8];                   // stream record offsets within the record, by width - 1
   CompInfo ci;
   uint64_t bar;
   uint32_t base[kBatchMax + 1];
   uint32_t tmem_base;
-  uint32_t crc_ok, cur_slice, bad;
+  uint32_t crc_ok, bad, walk_ok;
 };
+
+// Decode table of one rANS stream built by one warp: freq[256] (validated,
+// sum 4096) becomes freq[s] = f_s << 16 | cum_s, and lut[slot] = s | (slot -
+// cum_s) << 8 | f_s << 20 with the marks-and-running-maximum fill of
+// block_dec_lut.
+__device__ inline void warp_dec_lut(uint32_t* freq, uint32_t* lut) {
+  const uint32_t lane = threadIdx.x & 31u;
+  uint32_t f[8], mine = 0;
+#pragma unroll
+  for (uint32_t i = 0; i < 8; ++i) {
+    f[i] = freq[8u * lane + i];
+    mine += f[i];
+  }
+  uint32_t incl = mine;
+#pragma unroll
+  for (uint32_t o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  uint32_t cum = incl - mine;
+  for (uint32_t i = lane; i < kProbScale / 4u; i += 32u) reinterpret_cast<uint4*>(lut)[i] = make_uint4(0, 0, 0, 0);
+  __syncwarp();
+#pragma unroll
+  for (uint32_t i = 0; i < 8; ++i) {
+    const uint32_t s = 8u * lane + i;
+    if (f[i]) lut[cum] = s + 1u;
+    freq[s] = (f[i] << 16) | cum;
+    cum += f[i];
+  }
+  __syncwarp();
+  uint32_t carry = 0;
+#pragma unroll 4
+  for (uint32_t b0 = 0; b0 < kProbScale; b0 += 32u) {
+    const uint32_t slot = b0 + lane;
+    uint32_t m = lut[slot];
+#pragma unroll
+    for (uint32_t o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, m, o);
+      if (lane >= o) m = max(m, y);
+    }
+    m = max(m, carry);
+    carry = __shfl_sync(0xffffffffu, m, 31);
+    const uint32_t sym = m - 1u, e = freq[sym];
+    lut[slot] = sym | ((slot - (e & 0xffffu)) << 8) | ((e >> 16) << 20);
+  }
+  __syncwarp();
+}
+
+// rANS decode of group g of one width stream by one warp: n symbols on N
+// lanes; symbol i = a * tcc + t is written to codes[t * 132 + comp[a]] (m
+// components). The sub-stream (sl bytes at sub, 16-byte aligned) holds the
+// lanes' states, then the refill words. Its 16-byte units, from the one
+// holding the first word on, are copied by cp.async into a 1024-entry ring of
+// 16-bit positions counted from the sub-stream's start (the words begin at
+// position 2 * lanes_g), so no more than the ring's 128 units are requested
+// at once: at every stage of 8 steps (at most 256 words consumed) the warp waits for all but the
+// newest copy group and requests units up to 1024 positions past the unit
+// holding the next word, so no unit is overwritten before it is consumed and
+// the coming stage's words were requested a stage earlier. Returns false (on
+// every lane) when a symbol exceeds levels, a lane reads past its sub-stream
+// or the final states and word count do not match.
+__device__ inline bool decode_codes_group(const uint8_t* sub, uint32_t sl, uint32_t n, uint32_t N, uint32_t g,
+                                          const uint32_t* lut, uint16_t* ring, uint8_t* codes,
+                                          const uint32_t* comp, uint32_t m, uint32_t tcc, uint32_t levels) {
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t lanes_g = min(kGroupLanes, N - g * kGroupLanes);
+  if (sl < 4u * lanes_g || ((sl - 4u * lanes_g) & 1u)) return false;
+  const uint32_t W = (sl - 4u * lanes_g) >> 1, w0 = 2u * lanes_g;
+  const bool live = lane < lanes_g;
+  uint32_t start = 0, len = 0, start0, maxlen;
+  if (live) lane_range(n, N, g * kGroupLanes + lane, start, len);
+  lane_range(n, N, g * kGroupLanes, start0, maxlen);
+  const uint32_t lt = lanemask_lt();
+  uint32_t x = live ? reinterpret_cast<const uint32_t*>(sub)[lane] : kRansLow;
+  uint32_t a = start / tcc, t = start - a * tcc;
+  uint32_t j = (live && len && a < m) ? comp[a] : 0u;
+  uint32_t pos = 0, bad = 0;
+  const uint32_t n_units = (sl + 15u) >> 4, ring_saddr = static_cast<uint32_t>(__cvta_generic_to_shared(ring));
+  uint32_t loaded = w0 >> 3;  // units wholly inside the states are never needed (and would alias live slots)
+  auto request = [&]() {
+    const uint32_t target = min(n_units, ((w0 + pos) >> 3) + 128u);
+    for (uint32_t u = loaded + lane; u < target; u += 32u)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ring_saddr + ((u & 127u) << 4)),
+                   "l"(sub + (uint64_t(u) << 4))
+                   : "memory");
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    loaded = max(loaded, target);
+  };
+  request();
+  asm volatile("cp.async.commit_group;" ::: "memory");  // empty group: the first wait covers the window
+  for (uint32_t tau = 0; tau < maxlen; ++tau) {
+    if ((tau & 7u) == 0) {
+      asm volatile("cp.async.wait_group 1;" ::: "memory");
+      __syncwarp();
+      request();
+    }
+    const bool act = live && tau < len;
+    if (act) {
+      const uint32_t e = lut[x & (kProbScale - 1u)];
+      x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xfffu);
+      const uint32_t sym = e & 0xffu;
+      bad |= uint32_t(sym > levels);
+      codes[t * kCodesStride + j] = uint8_t(sym);
+      if (++t == tcc) {
+        t = 0;
+        ++a;
+        j = a < m ? comp[a] : 0u;
+      }
+    }
+    const bool need = act && x < kRansLow;
+    const uint32_t mask = __ballot_sync(0xffffffffu, need);
+    const uint32_t w = ring[(w0 + pos + __popc(mask & lt)) & 1023u];
+    if (need) x = (x << 16) | w;
+    pos += __popc(mask);
+  }
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+  __syncwarp();
+  const bool ok = !bad && pos == W && x == kRansLow;
+  return __all_sync(0xffffffffu, ok);
+}
 
 static_assert(sizeof(DecSmem) + 1024 <= 232448, "decoder shared memory exceeds the per-block limit");
 static_assert(sizeof(ProjSmem) <= 232448, "projection shared memory exceeds the per-block limit");
@@ -737,10 +868,7 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
     tc::tmem_alloc(&S.tmem_base, kTcCols);
     tc::tmem_relinquish();
   }
-  if (tid == 0) {
-    S.cur_slice = 0xffffffffu;
-    tc::mbar_init(&S.bar, 1);
-  }
+  if (tid == 0) tc::mbar_init(&S.bar, 1);
   tc::fence_before_sync();
   __syncthreads();
   tc::fence_after_sync();
@@ -786,62 +914,98 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
     const uint32_t c = kind - 1;
     const uint32_t t0 = sh.s_end + c * sh.ct, tcc = min(sh.ct, sh.r_start - t0);
     const uint32_t nb = (tcc + kTile - 1) / kTile;
-    if (S.cur_slice != sidx) {
-      __syncthreads();
-      const uint4* q4 = reinterpret_cast<const uint4*>(pl.qsplit + uint64_t(sidx) * kQSplitBytes);
-      uint4* b4 = reinterpret_cast<uint4*>(S.b_hi);  // b_hi and b_lo are contiguous
-      for (uint32_t i = tid; i < kQSplitBytes / 16u; i += nthr) b4[i] = __ldg(q4 + i);
-      load_comp_info(pl.comp + sidx, S.ci);
-      if (tid == 0) S.cur_slice = sidx;
-      __syncthreads();
-    }
+    load_comp_info(pl.comp + sidx, S.ci);
     const uint32_t side = 8u * S.ci.n_coded * nb;
     if (st == kOk && pad16(side) > len) st = kErrCorrupt;
-    if (st == kOk) {
-      if (tid < kD && S.ci.width[tid]) {
-        const uint32_t* p32 = reinterpret_cast<const uint32_t*>(rec + 8u * S.ci.coded_idx[tid] * nb);
-        for (uint32_t blk = 0; blk < nb; ++blk) {
-          S.zs[tid][blk][0] = __uint_as_float(p32[2 * blk]);
-          S.zs[tid][blk][1] = __uint_as_float(p32[2 * blk + 1]);
-        }
+    // stream records: walk the headers for their offsets, then parse each one
+    if (tid == 0) {
+      uint32_t o = pad16(side), ok = st == kOk ? 1u : 0u;
+      for (uint32_t bw = 1; bw <= 8 && ok; ++bw) {
+        if (!S.ci.bcount[bw]) continue;
+        S.str_off[bw - 1] = o;
+        if (o + 16u > len) { ok = 0; break; }
+        const uint32_t bytes = ld_u32(rec + o + 4);
+        if (bytes < 16u || (bytes & 15u) || bytes > len - o) { ok = 0; break; }
+        o += bytes;
       }
-      if (tid == 0) S.bad = 0;
+      S.walk_ok = ok && o == len;
+      S.bad = 0;
     }
-    uint32_t off = pad16(side);
-    const Split split(tcc);
-    for (uint32_t b = 1; b <= 8 && st == kOk; ++b) {
-      const uint32_t m = S.ci.bcount[b];
+    __syncthreads();
+    if (st == kOk && !S.walk_ok) st = kErrCorrupt;
+    for (uint32_t bw = 1; bw <= 8 && st == kOk; ++bw) {
+      const uint32_t m = S.ci.bcount[bw];
       if (!m) continue;
-      const uint32_t n = m * tcc, base = S.ci.bstart[b], levels = (1u << b) - 1u;
-      __syncthreads();
-      st = block_parse_stream(rec + off, len - off, n, &S.si, S.freq, S.tmp);
-      if (st != kOk) break;
-      auto put = [&](uint32_t i, uint32_t sy) {
-        uint32_t a, t;
-        split(i, a, t);
-        if (sy > levels) S.bad = 1;
-        S.codes[S.ci.comp[base + a] * kMaxCt + t] = uint8_t(sy);
-      };
-      bool ok = true;
-      if (S.si.mode == kModeRaw) {
-        for (uint32_t i = tid; i < n; i += nthr) put(i, rec[off + 16 + i]);
-      } else if (S.si.mode == kModeConst) {
-        for (uint32_t i = tid; i < n; i += nthr) put(i, S.si.sym);
-      } else {
-        block_dec_lut(S.freq, S.cum, S.lut, S.tmp);
-        const uint32_t N = rans_lanes(n), G = rans_groups(N);
-        if (warp < G)
-          ok = rans_decode_group(rec + off + S.si.sub_off[warp], S.si.sub_len[warp], n, N, warp,
-                                 S.lut, put);
-      }
-      ok = __syncthreads_and(ok);
-      if (!ok || S.bad) st = kErrCorrupt;
-      off += S.si.bytes;
+      const uint32_t o = S.str_off[bw - 1];
+      st = block_parse_stream(rec + o, len - o, m * tcc, &S.si[bw - 1], S.freq[bw - 1], S.tmp);
     }
-    if (st == kOk && off != len) st = kErrCorrupt;
     if (st != kOk) {
       if (tid == 0) atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(st));
       continue;
+    }
+    if (tid < kD && S.ci.width[tid]) {
+      const uint32_t* p32 = reinterpret_cast<const uint32_t*>(rec + 8u * S.ci.coded_idx[tid] * nb);
+      for (uint32_t blk = 0; blk < nb; ++blk) {
+        S.zs[tid][blk][0] = __uint_as_float(p32[2 * blk]);
+        S.zs[tid][blk][1] = __uint_as_float(p32[2 * blk + 1]);
+      }
+    }
+    // RAW and CONST streams: every thread writes codes
+    {
+      const Split split(tcc);
+      for (uint32_t bw = 1; bw <= 8; ++bw) {
+        const uint32_t m = S.ci.bcount[bw];
+        const uint32_t mode = S.si[bw - 1].mode;
+        if (!m || mode == kModeRans) continue;
+        const uint32_t n = m * tcc, base = S.ci.bstart[bw], levels = (1u << bw) - 1u;
+        const uint8_t* raw = rec + S.str_off[bw - 1] + 16u;
+        const uint32_t csym = S.si[bw - 1].sym;
+        uint32_t bad = 0;
+        for (uint32_t i = tid; i < n; i += nthr) {
+          uint32_t a, t;
+          split(i, a, t);
+          const uint32_t sy = mode == kModeRaw ? uint32_t(raw[i]) : csym;
+          bad |= uint32_t(sy > levels);
+          S.codes[t * kCodesStride + S.ci.comp[base + a]] = uint8_t(sy);
+        }
+        if (bad) S.bad = 1;
+      }
+    }
+    // rANS streams, up to kDecLuts at a time: one warp builds each table, then
+    // one warp per (stream, group) decodes
+    for (uint32_t bw0 = 1; bw0 <= 8;) {
+      uint32_t sel[kDecLuts], ns = 0, bw = bw0;
+      for (; bw <= 8 && ns < kDecLuts; ++bw)
+        if (S.ci.bcount[bw] && S.si[bw - 1].mode == kModeRans) sel[ns++] = bw;
+      bw0 = bw;
+      if (!ns) break;
+      if (warp < ns) warp_dec_lut(S.freq[sel[warp] - 1], S.u.ent.lut[warp]);
+      __syncthreads();
+      uint32_t pair = 0;
+      for (uint32_t q = 0; q < ns; ++q) {
+        const uint32_t sw = sel[q], m = S.ci.bcount[sw], n = m * tcc;
+        const uint32_t N = rans_lanes(n), G = rans_groups(N);
+        const StreamInfo& si = S.si[sw - 1];
+        for (uint32_t gg = 0; gg < G; ++gg, ++pair) {
+          if (pair % (nthr >> 5) != warp) continue;
+          const bool ok = decode_codes_group(rec + S.str_off[sw - 1] + si.sub_off[gg], si.sub_len[gg], n, N, gg,
+                                             S.u.ent.lut[q], S.u.ent.ring[warp], S.codes,
+                                             S.ci.comp + S.ci.bstart[sw], m, tcc, (1u << sw) - 1u);
+          if (!ok && lane == 0) S.bad = 1;
+        }
+      }
+      __syncthreads();
+    }
+    __syncthreads();  // every stream's codes and flags are in
+    if (S.bad) {
+      if (tid == 0) atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(kErrCorrupt));
+      continue;
+    }
+    // the B operand (Q as bf16 pieces) of this slice over the entropy stage's space
+    {
+      const uint4* q4 = reinterpret_cast<const uint4*>(pl.qsplit + uint64_t(sidx) * kQSplitBytes);
+      uint4* b4 = reinterpret_cast<uint4*>(S.u.tc.b_hi);  // b_hi and b_lo are contiguous
+      for (uint32_t i = tid; i < kQSplitBytes / 16u; i += nthr) b4[i] = __ldg(q4 + i);
     }
     // inverse projection on the tensor cores, 128 tokens at a time:
     // x^[t][k] = sum_j y^[t][j] Q[k][j] with y^ and Q split into bf16 hi + lo
@@ -854,20 +1018,20 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
         float v = 0.0f;
         if (tt < bl && S.ci.width[j]) {
           const uint32_t t = t_base + tt, blk = t / kTile;
-          v = __fmaf_rn(float(S.codes[j * kMaxCt + t]), S.zs[j][blk][1], S.zs[j][blk][0]);
+          v = __fmaf_rn(float(S.codes[t * kCodesStride + j]), S.zs[j][blk][1], S.zs[j][blk][0]);
         }
         const uint32_t h = f32_to_bf16_rne(v);
         const uint32_t l = f32_to_bf16_rne(__fsub_rn(v, bf16_to_f32(h)));
         const uint32_t o = tc::sw128_offset(tt, 2u * j, kTcRows);
-        *reinterpret_cast<uint16_t*>(S.a_hi + o) = uint16_t(h);
-        *reinterpret_cast<uint16_t*>(S.a_lo + o) = uint16_t(l);
+        *reinterpret_cast<uint16_t*>(S.u.tc.a_hi + o) = uint16_t(h);
+        *reinterpret_cast<uint16_t*>(S.u.tc.a_lo + o) = uint16_t(l);
       }
       tc::fence_async_smem();
       __syncthreads();
       if (tid == 0) {
         tc::fence_after_sync();
-        const uint32_t ah = tc::smem_addr(S.a_hi), al = tc::smem_addr(S.a_lo);
-        const uint32_t bh = tc::smem_addr(S.b_hi), bo = tc::smem_addr(S.b_lo);
+        const uint32_t ah = tc::smem_addr(S.u.tc.a_hi), al = tc::smem_addr(S.u.tc.a_lo);
+        const uint32_t bh = tc::smem_addr(S.u.tc.b_hi), bo = tc::smem_addr(S.u.tc.b_lo);
         uint32_t acc = 0;
         for (uint32_t ks = 0; ks < kD / 16u; ++ks) {  // K = 16 components per MMA
           const uint32_t koff = (ks >> 2) * (kTcRows * 128u) + (ks & 3u) * 32u;
