@@ -500,6 +500,70 @@ __device__ inline uint32_t rans_encode_group(SymFn sym, uint32_t n, uint32_t N, 
   return cap - pos;
 }
 
+// rANS encode of group g of a stream of n symbols laid out as a strided 2-D
+// byte array (all 32 lanes call): symbol i = col * tcc + t is the byte at
+// col_base(col) + t * stride. The steps and word placement are those of
+// rans_encode_group; each lane walks a byte pointer backwards (recomputing it
+// only when it wraps to the previous column) and fetches its next symbol and
+// that symbol's table entry tab[s] = {f | cum << 16, floor((2^32 - 1) / f)}
+// one step ahead, so the loop's dependency chain is the state update alone.
+template <class ColBase>
+__device__ inline uint32_t rans_encode_strided(ColBase col_base, uint32_t stride, uint32_t tcc, uint32_t n,
+                                               uint32_t N, uint32_t g, const uint2* tab, uint16_t* words,
+                                               uint32_t cap, uint32_t* x_out) {
+  const uint32_t lane = threadIdx.x & 31u;
+  const uint32_t l = g * kGroupLanes + lane;
+  const bool live = l < N;
+  uint32_t start = 0, len = 0, start0, maxlen;
+  if (live) lane_range(n, N, l, start, len);
+  lane_range(n, N, g * kGroupLanes, start0, maxlen);
+  const uint32_t lt = lanemask_lt();
+  uint32_t col = 0, t = 0;
+  const uint8_t* p = nullptr;
+  uint32_t s = 0;
+  if (live) {
+    const uint32_t last = start + len - 1u;
+    col = last / tcc;
+    t = last - col * tcc;
+    p = col_base(col) + uint64_t(t) * stride;
+    s = *p;
+  }
+  uint2 e = tab[s];
+  uint32_t x = kRansLow, pos = cap;
+  for (uint32_t tau = maxlen; tau-- > 0;) {
+    const bool act = live && tau < len;
+    uint32_t ns = s;
+    if (act && tau > 0u) {  // the lane's next symbol (tau - 1 < len)
+      if (t == 0u) {
+        t = tcc - 1u;
+        --col;
+        p = col_base(col) + uint64_t(t) * stride;
+      } else {
+        --t;
+        p -= stride;
+      }
+      ns = *p;
+    }
+    const uint2 ne = tab[ns];
+    const uint32_t f = e.x & 0xffffu, cum = e.x >> 16;
+    const bool emit = act && x >= (f << 20);
+    const uint32_t mask = __ballot_sync(0xffffffffu, emit);
+    pos -= __popc(mask);
+    if (emit) words[pos + __popc(mask & lt)] = uint16_t(x & 0xffffu);
+    const uint32_t xe = emit ? (x >> 16) : x;
+    uint32_t q = __umulhi(xe, e.y);
+    uint32_t r = xe - q * f;
+    const bool over = r >= f;
+    q += over ? 1u : 0u;
+    r -= over ? f : 0u;
+    x = act ? (q << kProbBits) + r + cum : xe;
+    s = ns;
+    e = ne;
+  }
+  *x_out = x;
+  return cap - pos;
+}
+
 // Warp-level rANS decode of group g from its sub-stream (sub_len bytes, states
 // then words; sub is 4-byte aligned). out(i, s) receives symbol i. Returns
 // true when every lane ends at 2^16 and exactly all words were read.

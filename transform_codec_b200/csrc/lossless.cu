@@ -19,6 +19,7 @@ struct __align__(16) EncSmem {
   uint32_t rem[256];
   uint32_t fc[2][256];
   uint32_t rcp[2][256];
+  uint2 tab[2][256];             // {f | cum << 16, 1/f} per plane
   uint32_t states[2][kMaxLanes];
   uint32_t tmp[32], red[32];
   uint32_t k[2], mode[2], bytes[2], csym[2];
@@ -81,7 +82,9 @@ k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
     uint32_t k = block_normalize(S.hist[p], n, S.freq[p], S.rem, S.tmp);
     if (tid == 0) S.k[p] = k;
     block_enc_tables(S.freq[p], S.fc[p], S.rcp[p], S.tmp);
+    for (uint32_t i = tid; i < 256; i += nthr) S.tab[p][i] = make_uint2(S.fc[p][i], S.rcp[p][i]);
   }
+  __syncthreads();
 
   const ChanMajor cm(tcc);
   const uint32_t N = rans_lanes(n), G = rans_groups(N);
@@ -96,14 +99,11 @@ k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
       uint32_t b0, len0, b1 = n, len1;
       lane_range(n, N, gg * kGroupLanes, b0, len0);
       if (gg + 1 < G) lane_range(n, N, (gg + 1) * kGroupLanes, b1, len1);
-      auto sym = [&](uint32_t i) -> uint32_t {
-        uint32_t d, t;
-        cm.split(i, d, t);
-        uint32_t v = vals[t * D + d];
-        return p ? (v >> 8) : (v & 0xffu);
-      };
+      // symbol i of plane p: byte p of the value of channel d = i / tcc, token t = i % tcc
+      const uint8_t* v8 = reinterpret_cast<const uint8_t*>(vals) + p;
       uint32_t x;
-      uint32_t Wg = rans_encode_group(sym, n, N, gg, S.fc[p], S.rcp[p], scratch[p] + b0, b1 - b0, &x);
+      uint32_t Wg = rans_encode_strided([v8](uint32_t d) { return v8 + 2u * d; }, 2u * D, tcc, n, N, gg,
+                                        S.tab[p], scratch[p] + b0, b1 - b0, &x);
       uint32_t l = gg * kGroupLanes + lane;
       if (l < N) S.states[p][l] = x;
       if (lane == 0) {
@@ -136,8 +136,21 @@ k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
       uint32_t v = vals[t * D + d];
       return p ? (v >> 8) : (v & 0xffu);
     };
-    block_write_stream(rec + off, S.mode[p], n, S.bytes[p], S.csym[p], S.k[p], S.freq[p],
-                       S.states[p], scratch[p], S.wbeg[p], S.W[p], S.sub_len[p], raw, S.tmp);
+    if (S.mode[p] == kModeRaw && (tcc & 15u) == 0) {
+      // raw plane: thread writes 16 tokens of one channel, neighbouring threads neighbouring channels
+      if (tid == 0) *reinterpret_cast<uint4*>(rec + off) = make_uint4(kModeRaw, S.bytes[p], n, 0u);
+      const uint8_t* v8 = reinterpret_cast<const uint8_t*>(vals) + p;
+      for (uint32_t idx = tid; idx < n / 16u; idx += nthr) {
+        const uint32_t d = idx % D, t0 = 16u * (idx / D);
+        uint32_t w[4] = {0, 0, 0, 0};
+#pragma unroll
+        for (uint32_t k = 0; k < 16; ++k) w[k >> 2] |= uint32_t(v8[2u * ((t0 + k) * D + d)]) << (8u * (k & 3u));
+        *reinterpret_cast<uint4*>(rec + off + 16u + d * tcc + t0) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    } else {
+      block_write_stream(rec + off, S.mode[p], n, S.bytes[p], S.csym[p], S.k[p], S.freq[p],
+                         S.states[p], scratch[p], S.wbeg[p], S.W[p], S.sub_len[p], raw, S.tmp);
+    }
     off += S.bytes[p];
   }
   __syncthreads();

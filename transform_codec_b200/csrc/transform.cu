@@ -408,7 +408,8 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
 struct __align__(16) EntSmem {
   uint8_t codes[kMaxCt * kCodesStride];  // codes[t * 132 + j]
   uint32_t freq[8][256];                 // per width stream, zero past its alphabet
-  uint32_t fc[kTabPool], rcp[kTabPool], rem[kTabPool], hist[kTabPool];
+  uint2 tab[kTabPool];                   // per symbol of each width stream: {f | cum << 16, 1/f}
+  uint32_t rem[kTabPool], hist[kTabPool];
   uint32_t states[8][kMaxLanes];
   uint32_t W[8][4], wbeg[8][4], sub_len[8][4];
   uint32_t k[8], mode[8], bytes[8], off[9];
@@ -419,9 +420,9 @@ struct __align__(16) EntSmem {
 
 // Largest-remainder normalisation of one width stream by one warp (the rule of
 // block_normalize): counts hist[0 .. A), A = 2^b, n symbols; writes freq[0 .. 256)
-// and the coding tables fc / rcp of the first A symbols. Returns k.
+// and the coding table tab of the first A symbols. Returns k.
 __device__ inline uint32_t warp_normalize(const uint32_t* hist, uint32_t A, uint32_t n, uint32_t* freq,
-                                          uint32_t* rem, uint32_t* fc, uint32_t* rcp) {
+                                          uint32_t* rem, uint2* tab) {
   const uint32_t lane = threadIdx.x & 31u;
   uint32_t present = 0;
   for (uint32_t s = lane; s < A; s += 32u) present += hist[s] ? 1u : 0u;
@@ -468,66 +469,11 @@ __device__ inline uint32_t warp_normalize(const uint32_t* hist, uint32_t A, uint
       const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += y;
     }
-    if (s < A) {
-      fc[s] = f | ((carry + incl - f) << 16);
-      rcp[s] = f ? 0xffffffffu / f : 0u;
-    }
+    if (s < A) tab[s] = make_uint2(f | ((carry + incl - f) << 16), f ? 0xffffffffu / f : 0u);
     carry += __shfl_sync(0xffffffffu, incl, 31);
   }
   __syncwarp();
   return k;
-}
-
-// rANS encode of group g of one width stream (all 32 lanes call): symbol i =
-// a * tcc + t is codes[t * 132 + comp[a]], a < m. The steps are those of
-// rans_encode_group (reverse order, ascending-lane word placement), but each
-// lane's next symbol and its table entries are fetched one step ahead, so
-// only the state update stays on the loop's dependency chain.
-__device__ inline uint32_t encode_codes_group(const uint8_t* codes, const uint32_t* comp, uint32_t m,
-                                              uint32_t tcc, uint32_t n, uint32_t N, uint32_t g,
-                                              const uint32_t* fc, const uint32_t* rcp, uint16_t* words,
-                                              uint32_t cap, uint32_t* x_out) {
-  const uint32_t lane = threadIdx.x & 31u;
-  const uint32_t l = g * kGroupLanes + lane;
-  const bool live = l < N;
-  uint32_t start = 0, len = 0, start0, maxlen;
-  if (live) lane_range(n, N, l, start, len);
-  lane_range(n, N, g * kGroupLanes, start0, maxlen);
-  const uint32_t lt = lanemask_lt();
-  // (a, t) of symbol start + tau, tau counting down from maxlen - 1
-  uint32_t i0 = start + maxlen - 1u;
-  uint32_t a = i0 / tcc, t = i0 - a * tcc;
-  uint32_t j = a < m ? comp[a] : 0u;
-  uint32_t s = (live && maxlen - 1u < len) ? codes[t * kCodesStride + j] : 0u;
-  uint32_t e = fc[s], rc = rcp[s];
-  uint32_t x = kRansLow, pos = cap;
-  for (uint32_t tau = maxlen; tau-- > 0;) {
-    const bool act = live && tau < len;
-    // the next step's symbol and tables, independent of the state
-    uint32_t na = a, nt = t;
-    if (nt == 0u) { na = a - 1u; nt = tcc - 1u; } else { nt = t - 1u; }
-    const uint32_t nj = (na != a && na < m) ? comp[na] : j;
-    const bool nact = live && tau > 0u && tau - 1u < len;
-    const uint32_t ns = nact ? codes[nt * kCodesStride + nj] : 0u;
-    const uint32_t ne = fc[ns], nrc = rcp[ns];
-    const uint32_t f = e & 0xffffu, cum = e >> 16;
-    const bool emit = act && x >= (f << 20);
-    const uint32_t mask = __ballot_sync(0xffffffffu, emit);
-    pos -= __popc(mask);
-    if (emit) {
-      words[pos + __popc(mask & lt)] = uint16_t(x & 0xffffu);
-      x >>= 16;
-    }
-    if (act) {
-      uint32_t q = __umulhi(x, rc);
-      uint32_t rr = x - q * f;
-      if (rr >= f) { ++q; rr -= f; }
-      x = (q << kProbBits) + rr + cum;
-    }
-    a = na; t = nt; j = nj; e = ne; rc = nrc;
-  }
-  *x_out = x;
-  return cap - pos;
 }
 
 __global__ void __launch_bounds__(kThreads)
@@ -578,7 +524,7 @@ k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
     const uint32_t bw = warp + 1u, m = S.ci.bcount[bw];
     if (m) {
       const uint32_t k = warp_normalize(S.hist + tab_base(bw), 1u << bw, m * tcc, S.freq[warp],
-                                        S.rem + tab_base(bw), S.fc + tab_base(bw), S.rcp + tab_base(bw));
+                                        S.rem + tab_base(bw), S.tab + tab_base(bw));
       if (lane == 0) S.k[warp] = k;
     }
   }
@@ -598,9 +544,11 @@ k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
         lane_range(n, N, g * kGroupLanes, b0, len0);
         if (g + 1 < G) lane_range(n, N, (g + 1) * kGroupLanes, b1, len1);
         uint32_t x;
-        const uint32_t Wg = encode_codes_group(S.codes, S.ci.comp + base, m, tcc, n, N, g,
-                                               S.fc + tab_base(bw), S.rcp + tab_base(bw),
-                                               scratch + wbase + b0, b1 - b0, &x);
+        const uint32_t* comp = S.ci.comp + base;
+        const uint8_t* codes = S.codes;
+        const uint32_t Wg = rans_encode_strided([comp, codes](uint32_t col) { return codes + comp[col]; },
+                                                kCodesStride, tcc, n, N, g, S.tab + tab_base(bw),
+                                                scratch + wbase + b0, b1 - b0, &x);
         if (g * kGroupLanes + lane < N) S.states[bw - 1][g * kGroupLanes + lane] = x;
         if (lane == 0) {
           S.W[bw - 1][g] = Wg;
