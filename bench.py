@@ -35,22 +35,30 @@ METRIC = "KV codec encode/decode GB/s (raw bytes) vs HBM roofline; compression r
 
 # algorithmic work per step of each kernel, given the step's raw bytes R, its
 # container bytes C and its middle (transform-coded) values V
+# Algorithmic work per step of each kernel with a roofline: bytes for the
+# lossless kernels (raw + container), and for the transform contraction 2 * 128
+# flops per middle value (one contraction; the projection kernel runs it in
+# fp64 on the CUDA cores, the decoder in bf16 pieces on the tensor cores).
+# R = raw bytes, C = container bytes, V = middle values of the step.
 KERNEL_WORK = {
     "lossless_encode": ("hbm", lambda R, C, V: R + C),
     "lossless_decode": ("hbm", lambda R, C, V: R + C),
-    "transform_encode_mid": ("alu", lambda R, C, V: 2 * 128 * V),
-    "transform_decode": ("alu", lambda R, C, V: 2 * 128 * V),
+    "transform_project": ("alu", lambda R, C, V: 2 * 128 * V),
+    "transform_decode": ("tensor", lambda R, C, V: 2 * 128 * V),
 }
 
 
 def measured_peaks():
+    """(HBM GB/s, sustained bf16 TFLOP/s, max SM MHz, source): the driver's
+    measurements, else the pool's earlier figures."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), float(p.get("sm_max_mhz", 1965.0)), "measured"
+        return (float(p["hbm_gbs"]), float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                float(p.get("sm_max_mhz", 1965.0)), "measured")
     except (OSError, KeyError, ValueError):
-        return 6650.0, 1965.0, "fallback"
+        return 6650.0, 1400.0, 1965.0, "fallback"
 
 
 class ClockSampler:
@@ -349,11 +357,11 @@ def run_kvc(args):
     raw = job.raw_bytes
     cont_l, cont_t = sum(job.sizes_l), sum(job.sizes_t)
     value = world * 4 * raw / (ms_step * 1e-3) / 1e9
-    hbm_peak, sm_max, peak_kind = measured_peaks()
+    hbm_peak, bf16_peak, sm_max, peak_kind = measured_peaks()
     fp64_peak = 148 * 64 * 2 * sm_max * 1e6 / 1e12  # TFLOP/s, 64 fp64 FMA/clk/SM
     launches = sum(n for n, _ in kernels.values())
     step_cont = {"lossless_encode": cont_l, "lossless_decode": cont_l,
-                 "transform_encode_mid": cont_t, "transform_decode": cont_t}
+                 "transform_project": cont_t, "transform_decode": cont_t}
     kern_out = {}
     total_kern_ms = sum(t for _, t in kernels.values()) or 1.0
     for name, (n, t) in kernels.items():
@@ -369,8 +377,9 @@ def run_kvc(args):
                              algorithmic_bytes_per_launch=int(work / n))
             else:
                 ach = work / secs / 1e12
-                entry.update(bound="alu", achieved=round(ach, 3), peak=round(fp64_peak, 2),
-                             unit="TFLOP/s", frac=round(ach / fp64_peak, 4),
+                peak = fp64_peak if bound == "alu" else bf16_peak
+                entry.update(bound=bound, achieved=round(ach, 3), peak=round(peak, 2),
+                             unit="TFLOP/s", frac=round(ach / peak, 4),
                              algorithmic_flops_per_launch=int(work / n))
         kern_out[name] = entry
     dominant = max(kern_out, key=lambda k: kern_out[k]["total_ms"]) if kern_out else None
@@ -379,8 +388,9 @@ def run_kvc(args):
         d = kern_out[dominant]
         roof = {"kernel": dominant, "bound": d["bound"], "achieved": d["achieved"],
                 "peak": d["peak"], "unit": d["unit"], "frac": d["frac"], "traffic": None,
-                "peak_source": peak_kind if d["bound"] == "hbm" else
-                "derived: 148 SMs x 64 fp64 FMA/clk x 2 x max SM clock"}
+                "peak_source": {"hbm": peak_kind + " copy bandwidth",
+                                "tensor": peak_kind + " sustained cuBLAS bf16",
+                                "alu": "derived: 148 SMs x 64 fp64 FMA/clk x 2 x max SM clock"}[d["bound"]]}
     e2e = None
     if not args.no_e2e:
         e_ms, h2d, d2h = run_e2e(job, max(1, min(args.steps, 2)), 1)
