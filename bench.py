@@ -112,7 +112,10 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
-def dist_setup():
+def dist_setup(backend: str = "nccl"):
+    """Rank, world and local rank from the launcher's environment; for more than
+    one rank, the process group (NCCL on the GPUs; gloo runs the same code on
+    the CPU). The only collectives are the timing reductions below."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -121,17 +124,20 @@ def dist_setup():
 
         import torch
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(minutes=10))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(minutes=5))
     return world, rank, local
 
 
 def max_over_ranks(values, world):
+    """Element-wise maximum of each rank's values (device timings), on every rank."""
     if world == 1:
         return list(values)
     import torch
     import torch.distributed as dist
-    t = torch.tensor(list(values), dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor(list(values), dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return t.cpu().tolist()
 
