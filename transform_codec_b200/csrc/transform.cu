@@ -26,12 +26,12 @@ constexpr uint32_t kTcRows = 128;   // tokens per tensor-core tile (MMA M)
 constexpr uint32_t kTcCols = 128;   // tensor-memory columns: one fp32 128 x 128 accumulator
 
 __device__ inline float bf16_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
-__device__ inline uint32_t f32_to_bf16_rne(float f) {
-  uint32_t x = __float_as_uint(f);
-  if ((x & 0x7fffffffu) > 0x7f800000u) return ((x >> 16) | 0x40u) & 0xffffu;
-  uint32_t upper = x >> 16, lower = x & 0xffffu;
-  if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) ++upper;
-  return upper & 0xffffu;
+
+// two fp32 values rounded to bf16 (nearest, ties to even) and packed, lo in bits 0-15
+__device__ inline uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
 __device__ inline uint32_t quantize(float y, float z, float s, uint32_t levels) {
@@ -961,18 +961,35 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
     for (uint32_t t_base = 0; t_base < tcc; t_base += kTcRows) {
       const uint32_t bl = min(kTcRows, tcc - t_base);
       __syncthreads();
-      for (uint32_t idx = tid; idx < kTcRows * kD; idx += nthr) {
-        const uint32_t tt = idx >> 7, j = idx & (kD - 1u);
-        float v = 0.0f;
-        if (tt < bl && S.ci.width[j]) {
+      // item: 8 consecutive components of one token -> one 16-byte chunk of each piece
+      for (uint32_t it = tid; it < kTcRows * (kD / 8u); it += nthr) {
+        const uint32_t tt = it >> 4, j0 = 8u * (it & 15u);
+        float v[8];
+#pragma unroll
+        for (uint32_t i = 0; i < 8; ++i) v[i] = 0.0f;
+        if (tt < bl) {
           const uint32_t t = t_base + tt, blk = t / kTile;
-          v = __fmaf_rn(float(S.codes[t * kCodesStride + j]), S.zs[j][blk][1], S.zs[j][blk][0]);
+          const uint32_t* cw = reinterpret_cast<const uint32_t*>(&S.codes[t * kCodesStride + j0]);
+          const uint32_t c4[2] = {cw[0], cw[1]};
+#pragma unroll
+          for (uint32_t i = 0; i < 8; ++i) {
+            const uint32_t j = j0 + i;
+            if (S.ci.width[j]) {
+              const float2 zs = *reinterpret_cast<const float2*>(S.zs[j][blk]);
+              v[i] = __fmaf_rn(float((c4[i >> 2] >> (8u * (i & 3u))) & 0xffu), zs.y, zs.x);
+            }
+          }
         }
-        const uint32_t h = f32_to_bf16_rne(v);
-        const uint32_t l = f32_to_bf16_rne(__fsub_rn(v, bf16_to_f32(h)));
-        const uint32_t o = tc::sw128_offset(tt, 2u * j, kTcRows);
-        *reinterpret_cast<uint16_t*>(S.u.tc.a_hi + o) = uint16_t(h);
-        *reinterpret_cast<uint16_t*>(S.u.tc.a_lo + o) = uint16_t(l);
+        uint32_t h[4], l[4];
+#pragma unroll
+        for (uint32_t i = 0; i < 4; ++i) {
+          h[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+          l[i] = pack_bf16x2(__fsub_rn(v[2 * i], bf16_to_f32(h[i] & 0xffffu)),
+                             __fsub_rn(v[2 * i + 1], bf16_to_f32(h[i] >> 16)));
+        }
+        const uint32_t o = tc::sw128_offset(tt, 2u * j0, kTcRows);
+        *reinterpret_cast<uint4*>(S.u.tc.a_hi + o) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(S.u.tc.a_lo + o) = make_uint4(l[0], l[1], l[2], l[3]);
       }
       tc::fence_async_smem();
       __syncthreads();
@@ -1022,15 +1039,16 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
             float a0 = __uint_as_float(va[i]), b0 = __uint_as_float(vb[i]);
             float a1 = __uint_as_float(va[i + 1]), b1 = __uint_as_float(vb[i + 1]);
             if (is_key) {
-              const float2 k0 = cs[i], k1 = cs[i + 1];
+              const float4 kk = __ldg(reinterpret_cast<const float4*>(cs) + (i >> 1));  // pairs i, i + 1
+              const float2 k0 = make_float2(kk.x, kk.y), k1 = make_float2(kk.z, kk.w);
               const float na0 = __fsub_rn(__fmul_rn(a0, k0.x), __fmul_rn(b0, k0.y));
               const float nb0 = __fadd_rn(__fmul_rn(a0, k0.y), __fmul_rn(b0, k0.x));
               const float na1 = __fsub_rn(__fmul_rn(a1, k1.x), __fmul_rn(b1, k1.y));
               const float nb1 = __fadd_rn(__fmul_rn(a1, k1.y), __fmul_rn(b1, k1.x));
               a0 = na0; b0 = nb0; a1 = na1; b1 = nb1;
             }
-            pa[i >> 1] = f32_to_bf16_rne(a0) | (f32_to_bf16_rne(a1) << 16);
-            pb[i >> 1] = f32_to_bf16_rne(b0) | (f32_to_bf16_rne(b1) << 16);
+            pa[i >> 1] = pack_bf16x2(a0, a1);
+            pb[i >> 1] = pack_bf16x2(b0, b1);
           }
           uint4* ra = reinterpret_cast<uint4*>(xs + uint64_t(t) * kD + c0);
           uint4* rb = reinterpret_cast<uint4*>(xs + uint64_t(t) * kD + c0 + 64u);
