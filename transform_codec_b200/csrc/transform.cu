@@ -740,11 +740,14 @@ __device__ inline bool decode_codes_group(const uint8_t* sub, uint32_t sl, uint3
   uint32_t x = live ? reinterpret_cast<const uint32_t*>(sub)[lane] : kRansLow;
   uint32_t a = start / tcc, t = start - a * tcc;
   uint32_t j = (live && len && a < m) ? comp[a] : 0u;
-  uint32_t pos = 0, bad = 0;
+  const uint32_t codes_saddr = static_cast<uint32_t>(__cvta_generic_to_shared(codes));
+  uint32_t cp = codes_saddr + t * kCodesStride + j;  // shared address of this lane's next code
+  uint32_t left = tcc - t;                            // steps until the lane moves to the next component
+  uint32_t rp = w0, orv = 0;                          // ring position of the next word; OR of the entries
   const uint32_t n_units = (sl + 15u) >> 4, ring_saddr = static_cast<uint32_t>(__cvta_generic_to_shared(ring));
   uint32_t loaded = w0 >> 3;  // units wholly inside the states are never needed (and would alias live slots)
   auto request = [&]() {
-    const uint32_t target = min(n_units, ((w0 + pos) >> 3) + 128u);
+    const uint32_t target = min(n_units, (rp >> 3) + 128u);
     for (uint32_t u = loaded + lane; u < target; u += 32u)
       asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ring_saddr + ((u & 127u) << 4)),
                    "l"(sub + (uint64_t(u) << 4))
@@ -754,31 +757,33 @@ __device__ inline bool decode_codes_group(const uint8_t* sub, uint32_t sl, uint3
   };
   request();
   asm volatile("cp.async.commit_group;" ::: "memory");  // empty group: the first wait covers the window
-  for (uint32_t tau = 0; tau < maxlen; ++tau) {
-    if ((tau & 7u) == 0) {
-      asm volatile("cp.async.wait_group 1;" ::: "memory");
-      __syncwarp();
-      request();
-    }
-    const bool act = live && tau < len;
-    if (act) {
-      const uint32_t e = lut[x & (kProbScale - 1u)];
-      x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xfffu);
-      const uint32_t sym = e & 0xffu;
-      bad |= uint32_t(sym > levels);
-      codes[t * kCodesStride + j] = uint8_t(sym);
-      if (++t == tcc) {
-        t = 0;
-        ++a;
-        j = a < m ? comp[a] : 0u;
+  for (uint32_t tau0 = 0; tau0 < maxlen; tau0 += 8u) {
+    asm volatile("cp.async.wait_group 1;" ::: "memory");
+    __syncwarp();
+    request();
+#pragma unroll
+    for (uint32_t k = 0; k < 8; ++k) {
+      const bool act = live && tau0 + k < len;
+      if (act) {
+        const uint32_t e = lut[x & (kProbScale - 1u)];
+        x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xfffu);
+        orv |= e;
+        asm volatile("st.shared.u8 [%0], %1;" ::"r"(cp), "r"(e) : "memory");
+        cp += kCodesStride;
+        if (--left == 0u) {
+          ++a;
+          cp = codes_saddr + (a < m ? comp[a] : 0u);
+          left = tcc;
+        }
       }
+      const bool need = act && x < kRansLow;
+      const uint32_t mask = __ballot_sync(0xffffffffu, need);
+      const uint32_t w = ring[(rp + __popc(mask & lt)) & 1023u];
+      if (need) x = (x << 16) | w;
+      rp += __popc(mask);
     }
-    const bool need = act && x < kRansLow;
-    const uint32_t mask = __ballot_sync(0xffffffffu, need);
-    const uint32_t w = ring[(w0 + pos + __popc(mask & lt)) & 1023u];
-    if (need) x = (x << 16) | w;
-    pos += __popc(mask);
   }
+  const uint32_t pos = rp - w0, bad = (orv & 0xffu & ~levels) != 0u;
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncwarp();
   const bool ok = !bad && pos == W && x == kRansLow;
@@ -1007,6 +1012,14 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
           tc::mma_bf16(tmem, tc::desc_sw128(al + koff), tc::desc_sw128(bh + kboff), idesc, 1);
         }
         tc::mma_commit(&S.bar);
+      }
+      if (is_key) {  // this thread's RoPE pairs for the epilogue, fetched while the MMAs run
+        const uint32_t ptt = (warp & 3u) * 32u + lane;
+        if (ptt < bl) {
+          const float* cs = pl.rope + (uint64_t(t0 + t_base + ptt) * (kD / 2) + (warp >> 2) * 32u) * 2u;
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(cs));
+          asm volatile("prefetch.global.L1 [%0];" ::"l"(cs + 32));
+        }
       }
       const bool done = tc::mbar_wait(&S.bar, phase, 1u << 22);
       phase ^= 1u;
