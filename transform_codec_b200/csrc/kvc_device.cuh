@@ -532,18 +532,18 @@ __device__ inline uint32_t rans_encode_strided(ColBase col_base, uint32_t stride
   uint32_t x = kRansLow, pos = cap;
   for (uint32_t tau = maxlen; tau-- > 0;) {
     const bool act = live && tau < len;
-    uint32_t ns = s;
-    if (act && tau > 0u) {  // the lane's next symbol (tau - 1 < len)
-      if (t == 0u) {
-        t = tcc - 1u;
-        --col;
-        p = col_base(col) + uint64_t(t) * stride;
-      } else {
-        --t;
-        p -= stride;
-      }
-      ns = *p;
+    // the lane's next symbol (tau - 1 < len), without a branch: the pointer only
+    // ever points into the lane's own range, so the load is always in bounds
+    const bool adv = act && tau > 0u;
+    const bool wrap = adv && t == 0u;
+    if (wrap) {
+      t = tcc;
+      --col;
+      p = col_base(col) + uint64_t(tcc) * stride;
     }
+    t -= adv ? 1u : 0u;
+    p -= adv ? stride : 0u;
+    const uint32_t ns = live ? uint32_t(*p) : 0u;
     const uint2 ne = tab[ns];
     const uint32_t f = e.x & 0xffffu, cum = e.x >> 16;
     const bool emit = act && x >= (f << 20);
