@@ -60,6 +60,9 @@ def _load():
         "kvco_normalize": ([vp, vp], i32),
         "kvco_stream_bound": ([u32], sz),
         "kvco_stream_encode": ([vp, u32, vp], sz),
+        "kvco_stream_encode_delta": ([vp, u32, vp], sz),
+        "kvco_lane_delta": ([vp, u32, vp], None),
+        "kvco_lane_undelta": ([vp, u32], None),
         "kvco_stream_decode": ([vp, sz, u32, vp, P(sz)], i32),
         "kvco_rans_payload_bytes": ([vp, u32], sz),
         "kvco_lossless_bound": ([P(Desc), u32], sz),
@@ -142,6 +145,30 @@ def stream_encode(sym: np.ndarray) -> bytes:
     out = np.zeros(lib.kvco_stream_bound(s.size), dtype=np.uint8)
     n = lib.kvco_stream_encode(_ptr(s) if s.size else None, s.size, _ptr(out))
     return out[:n].tobytes()
+
+
+def stream_encode_delta(sym: np.ndarray) -> bytes:
+    """Stream record with the lane-delta candidate (the high byte plane's coder)."""
+    s = np.ascontiguousarray(sym, dtype=np.uint8)
+    lib = _load()
+    out = np.zeros(lib.kvco_stream_bound(s.size), dtype=np.uint8)
+    n = lib.kvco_stream_encode_delta(_ptr(s) if s.size else None, s.size, _ptr(out))
+    return out[:n].tobytes()
+
+
+def lane_delta(sym: np.ndarray) -> np.ndarray:
+    s = np.ascontiguousarray(sym, dtype=np.uint8)
+    out = np.zeros_like(s)
+    if s.size:
+        _load().kvco_lane_delta(_ptr(s), s.size, _ptr(out))
+    return out
+
+
+def lane_undelta(sym: np.ndarray) -> np.ndarray:
+    s = np.array(sym, dtype=np.uint8, copy=True)
+    if s.size:
+        _load().kvco_lane_undelta(_ptr(s), s.size)
+    return s
 
 
 def stream_decode(rec, n: int):

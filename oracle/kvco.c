@@ -254,7 +254,8 @@ static int rans_decode_group(const uint8_t* sub, size_t sub_len, uint32_t n, uin
  * smallest: CONST (one distinct symbol), RANS if strictly smaller than RAW,
  * else RAW ([AT1] "KV & tensor mode": keep whichever is smaller, so never worse
  * than the fallback).
- *   header (16 bytes): u8 mode, u8 const symbol, u8 groups, u8 0,
+ *   header (16 bytes): u8 mode, u8 const symbol, u8 groups, u8 flags (bit 0: the
+ *                      RANS symbols are lane deltas, see kvco_lane_delta; 0 otherwise),
  *                      u32 record bytes (multiple of 16, header included),
  *                      u32 n, u32 k (present symbols: RAW 0, CONST 1, RANS k)
  *   RAW:   n bytes, zero padded to 16
@@ -278,7 +279,7 @@ static size_t stream_raw(const uint8_t* sym, uint32_t n, uint8_t* out) {
 
 /* Build the RANS record into out (capacity 2n + 4096); returns its size. */
 static size_t stream_rans(const uint8_t* sym, uint32_t n, const uint16_t freq[256],
-                          uint32_t k, uint8_t* out, size_t* payload) {
+                          uint32_t k, uint32_t flags, uint8_t* out, size_t* payload) {
   uint32_t cum[256];
   cum_from_freq(freq, cum);
   uint32_t N = lanes_for(n);
@@ -308,7 +309,7 @@ static size_t stream_rans(const uint8_t* sym, uint32_t n, const uint16_t freq[25
   out[0] = MODE_RANS;
   out[1] = 0;
   out[2] = (uint8_t)G;
-  out[3] = 0;
+  out[3] = (uint8_t)flags;
   put32(out + 4, (uint32_t)p);
   put32(out + 8, n);
   put32(out + 12, k);
@@ -320,6 +321,63 @@ static int stream_table(const uint8_t* sym, uint32_t n, uint16_t freq[256]) {
   memset(count, 0, sizeof count);
   for (uint32_t i = 0; i < n; i++) count[sym[i]]++;
   return kvco_normalize(count, freq);
+}
+
+/* Lane delta ([QATQ] "How it works": delta-XOR along tokens in channel-major
+ * order). Reading: within each rANS lane's contiguous range of the stream, a
+ * symbol is replaced by its XOR with the previous symbol of the same lane; the
+ * lane's first symbol is kept. Undone lane by lane in order. */
+void kvco_lane_delta(const uint8_t* sym, uint32_t n, uint8_t* out) {
+  if (!n) return;
+  uint32_t N = lanes_for(n);
+  for (uint32_t l = 0; l < N; l++) {
+    uint32_t start, len;
+    lane_range(n, N, l, &start, &len);
+    for (uint32_t i = 0; i < len; i++)
+      out[start + i] = i ? (uint8_t)(sym[start + i] ^ sym[start + i - 1]) : sym[start];
+  }
+}
+
+void kvco_lane_undelta(uint8_t* sym, uint32_t n) {
+  if (!n) return;
+  uint32_t N = lanes_for(n);
+  for (uint32_t l = 0; l < N; l++) {
+    uint32_t start, len;
+    lane_range(n, N, l, &start, &len);
+    for (uint32_t i = 1; i < len; i++) sym[start + i] ^= sym[start + i - 1];
+  }
+}
+
+/* Stream with the lane-delta candidate: the plain choice of
+ * kvco_stream_encode, unless a RANS record of the lane-delta symbols (flag
+ * byte 1) is strictly smaller than both the plain RANS record and RAW. */
+size_t kvco_stream_encode_delta(const uint8_t* sym, uint32_t n, uint8_t* out) {
+  uint16_t freq[256], dfreq[256];
+  int k = stream_table(sym, n, freq);
+  if (k < 2) return kvco_stream_encode(sym, n, out);
+  uint8_t* dsym = (uint8_t*)malloc(n);
+  kvco_lane_delta(sym, n, dsym);
+  int kd = stream_table(dsym, n, dfreq);
+  size_t raw_bytes = 16u + pad16(n);
+  uint8_t* tmp = (uint8_t*)malloc(2u * (size_t)n + 4096u);
+  uint8_t* dtmp = (uint8_t*)malloc(2u * (size_t)n + 4096u);
+  size_t payload;
+  size_t rb = stream_rans(sym, n, freq, (uint32_t)k, 0, tmp, &payload);
+  size_t rd = kd >= 2 ? stream_rans(dsym, n, dfreq, (uint32_t)kd, 1, dtmp, &payload) : (size_t)-1;
+  size_t out_bytes;
+  if (rd < rb && rd < raw_bytes) {
+    memcpy(out, dtmp, rd);
+    out_bytes = rd;
+  } else if (rb < raw_bytes) {
+    memcpy(out, tmp, rb);
+    out_bytes = rb;
+  } else {
+    out_bytes = stream_raw(sym, n, out);
+  }
+  free(tmp);
+  free(dtmp);
+  free(dsym);
+  return out_bytes;
 }
 
 size_t kvco_stream_encode(const uint8_t* sym, uint32_t n, uint8_t* out) {
@@ -338,7 +396,7 @@ size_t kvco_stream_encode(const uint8_t* sym, uint32_t n, uint8_t* out) {
   size_t raw_bytes = 16u + pad16(n);
   uint8_t* tmp = (uint8_t*)malloc(2u * (size_t)n + 4096u);
   size_t payload;
-  size_t rb = stream_rans(sym, n, freq, (uint32_t)k, tmp, &payload);
+  size_t rb = stream_rans(sym, n, freq, (uint32_t)k, 0, tmp, &payload);
   size_t out_bytes;
   if (rb < raw_bytes) {
     memcpy(out, tmp, rb);
@@ -358,17 +416,18 @@ size_t kvco_rans_payload_bytes(const uint8_t* sym, uint32_t n) {
   if (k < 2) return 0;
   uint8_t* tmp = (uint8_t*)malloc(2u * (size_t)n + 4096u);
   size_t payload;
-  stream_rans(sym, n, freq, (uint32_t)k, tmp, &payload);
+  stream_rans(sym, n, freq, (uint32_t)k, 0, tmp, &payload);
   free(tmp);
   return payload;
 }
 
-int kvco_stream_decode(const uint8_t* rec, size_t avail, uint32_t n, uint8_t* sym,
-                       size_t* used) {
+static int stream_decode(const uint8_t* rec, size_t avail, uint32_t n, uint8_t* sym, size_t* used,
+                         int allow_delta) {
   if (avail < 16) return KVCO_CORRUPT;
-  uint32_t mode = rec[0], csym = rec[1], G = rec[2];
+  uint32_t mode = rec[0], csym = rec[1], G = rec[2], flags = rec[3];
   uint32_t bytes = get32(rec + 4), rn = get32(rec + 8), k = get32(rec + 12);
-  if (rec[3] != 0 || rn != n || (bytes & 15u) || bytes < 16 || bytes > avail)
+  if (flags > (allow_delta && mode == MODE_RANS ? 1u : 0u) || rn != n || (bytes & 15u) ||
+      bytes < 16 || bytes > avail)
     return KVCO_CORRUPT;
   *used = bytes;
   if (mode == MODE_RAW) {
@@ -418,7 +477,13 @@ int kvco_stream_decode(const uint8_t* rec, size_t avail, uint32_t n, uint8_t* sy
     p += pad16(sub);
   }
   if (p != bytes) return KVCO_CORRUPT;
+  if (flags) kvco_lane_undelta(sym, n);
   return KVCO_OK;
+}
+
+int kvco_stream_decode(const uint8_t* rec, size_t avail, uint32_t n, uint8_t* sym,
+                       size_t* used) {
+  return stream_decode(rec, avail, n, sym, used, 1);
 }
 
 /* ---------------------------------------------------------------------------
@@ -579,7 +644,7 @@ size_t kvco_encode_lossless(const kvco_desc* d, uint32_t first_slice, uint32_t n
         }
       size_t start = p;
       p += kvco_stream_encode(p0, n, dst + p);
-      p += kvco_stream_encode(p1, n, dst + p);
+      p += kvco_stream_encode_delta(p1, n, dst + p);
       uint8_t* e = dst + HDR_BYTES + (size_t)IDX_ENTRY * r;
       put64(e, start);
       put32(e + 8, (uint32_t)(p - start));
@@ -1031,7 +1096,7 @@ static int mid_chunk_parse(const kvco_desc* d, uint32_t sidx, const uint8_t* rec
     uint32_t m = count_width(w, D, b);
     if (!m) continue;
     size_t used = 0;
-    int st = kvco_stream_decode(rec + p, len - p, m * tcc, syms, &used);
+    int st = stream_decode(rec + p, len - p, m * tcc, syms, &used, 0);  /* no lane delta here */
     if (st) return st;
     p += used;
     uint32_t mm = 0;
