@@ -314,9 +314,14 @@ k_stage_stream_decode(const uint8_t* rec, uint32_t rec_bytes, uint32_t n, uint8_
       block_dec_lut(S.freq, S.cum, S.lut, S.tmp);
       const uint32_t N = rans_lanes(n), G = rans_groups(N), warp = tid >> 5;
       bool okw = true;
+      const uint32_t dm = S.si.delta ? 0xffu : 0u;  // lane deltas: running XOR per lane
+      uint32_t prev = 0;
       if (warp < G)
         okw = rans_decode_group(rec + S.si.sub_off[warp], S.si.sub_len[warp], n, N, warp, S.lut,
-                                [sym](uint32_t i, uint32_t s) { sym[i] = uint8_t(s); });
+                                [&](uint32_t i, uint32_t s) {
+                                  prev = s ^ (prev & dm);
+                                  sym[i] = uint8_t(prev);
+                                });
       ok = __syncthreads_and(okw);
     }
   }

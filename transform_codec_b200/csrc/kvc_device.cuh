@@ -507,7 +507,10 @@ __device__ inline uint32_t rans_encode_group(SymFn sym, uint32_t n, uint32_t N, 
 // only when it wraps to the previous column) and fetches its next symbol and
 // that symbol's table entry tab[s] = {f | cum << 16, floor((2^32 - 1) / f)}
 // one step ahead, so the loop's dependency chain is the state update alone.
-template <class ColBase>
+// With kDelta the coded symbol is the lane delta: the byte XORed with the
+// lane's previous byte (the one at the next smaller index), except for the
+// lane's first symbol.
+template <bool kDelta = false, class ColBase>
 __device__ inline uint32_t rans_encode_strided(ColBase col_base, uint32_t stride, uint32_t tcc, uint32_t n,
                                                uint32_t N, uint32_t g, const uint2* tab, uint16_t* words,
                                                uint32_t cap, uint32_t* x_out) {
@@ -521,12 +524,17 @@ __device__ inline uint32_t rans_encode_strided(ColBase col_base, uint32_t stride
   uint32_t col = 0, t = 0;
   const uint8_t* p = nullptr;
   uint32_t s = 0;
+  // byte before the one at (col, t) in stream order (for the lane delta)
+  auto prev_byte = [&](uint32_t c, uint32_t tt, const uint8_t* q) -> uint32_t {
+    return tt ? uint32_t(q[-int64_t(stride)]) : uint32_t(col_base(c - 1u)[uint64_t(tcc - 1u) * stride]);
+  };
   if (live) {
     const uint32_t last = start + len - 1u;
     col = last / tcc;
     t = last - col * tcc;
     p = col_base(col) + uint64_t(t) * stride;
     s = *p;
+    if (kDelta && len > 1u) s ^= prev_byte(col, t, p);
   }
   uint2 e = tab[s];
   uint32_t x = kRansLow, pos = cap;
@@ -543,7 +551,11 @@ __device__ inline uint32_t rans_encode_strided(ColBase col_base, uint32_t stride
     }
     t -= adv ? 1u : 0u;
     p -= adv ? stride : 0u;
-    const uint32_t ns = live ? uint32_t(*p) : 0u;
+    uint32_t ns = live ? uint32_t(*p) : 0u;
+    if (kDelta) {
+      if (adv && tau > 1u) ns ^= prev_byte(col, t, p);  // the next symbol is not the lane's first
+      ns = adv ? ns : s;  // a lane waiting for its first step keeps its (delta) symbol
+    }
     const uint2 ne = tab[ns];
     const uint32_t f = e.x & 0xffffu, cum = e.x >> 16;
     const bool emit = act && x >= (f << 20);
@@ -610,6 +622,7 @@ __device__ inline bool rans_decode_group(const uint8_t* sub, uint32_t sub_len, u
 // frequencies + pad, G u32 sub-stream lengths + pad, padded sub-streams.
 struct StreamInfo {
   uint32_t mode, sym, groups, bytes, k;
+  uint32_t delta;  // 1: the RANS symbols are lane deltas (header byte 3)
   uint32_t sub_off[4], sub_len[4];
   int status;
 };
@@ -624,7 +637,8 @@ __host__ __device__ inline uint32_t rans_record_bytes(uint32_t k, uint32_t G, co
 // chunk record) for n symbols and, for RANS, load its frequency table into
 // freq[256]. Block-cooperative; si is shared. Returns status (block-uniform).
 __device__ inline int block_parse_stream(const uint8_t* rec, uint32_t avail, uint32_t n,
-                                         StreamInfo* si, uint32_t* freq, uint32_t* tmp) {
+                                         StreamInfo* si, uint32_t* freq, uint32_t* tmp,
+                                         bool allow_delta = true) {
   if (threadIdx.x == 0) {
     int st = kOk;
     if (avail < 16) st = kErrCorrupt;
@@ -633,8 +647,10 @@ __device__ inline int block_parse_stream(const uint8_t* rec, uint32_t avail, uin
       uint32_t mode = hv.x & 0xffu, csym = (hv.x >> 8) & 0xffu, G = (hv.x >> 16) & 0xffu;
       uint32_t bytes = hv.y, rn = hv.z, k = hv.w;
       const uint32_t b3 = hv.x >> 24;
-      si->mode = mode; si->sym = csym; si->groups = G; si->bytes = bytes; si->k = k;
-      if (b3 != 0 || rn != n || (bytes & 15u) || bytes < 16 || bytes > avail) st = kErrCorrupt;
+      si->mode = mode; si->sym = csym; si->groups = G; si->bytes = bytes; si->k = k; si->delta = b3;
+      if (b3 > (allow_delta && mode == kModeRans ? 1u : 0u) || rn != n || (bytes & 15u) || bytes < 16 ||
+          bytes > avail)
+        st = kErrCorrupt;
       else if (mode == kModeRaw) {
         if (csym || G || k || bytes != 16u + pad16(n)) st = kErrCorrupt;
       } else if (mode == kModeConst) {
@@ -725,7 +741,8 @@ __device__ inline void block_write_stream(uint8_t* rec, uint32_t mode, uint32_t 
                                           uint32_t csym, uint32_t k, const uint32_t* freq,
                                           const uint32_t* states, const uint16_t* words,
                                           const uint32_t* wbeg, const uint32_t* W,
-                                          const uint32_t* sub_len, RawFn raw, uint32_t* tmp) {
+                                          const uint32_t* sub_len, RawFn raw, uint32_t* tmp,
+                                          uint32_t delta = 0) {
   const uint32_t tid = threadIdx.x, nthr = blockDim.x;
   if (mode == kModeRaw || mode == kModeConst) {
     if (tid == 0) {
@@ -750,7 +767,7 @@ __device__ inline void block_write_stream(uint8_t* rec, uint32_t mode, uint32_t 
   // RANS
   const uint32_t N = rans_lanes(n), G = rans_groups(N);
   const uint32_t lane = tid & 31u, warp = tid >> 5;
-  if (tid == 0) *reinterpret_cast<uint4*>(rec) = make_uint4(kModeRans | (G << 16), bytes, n, k);
+  if (tid == 0) *reinterpret_cast<uint4*>(rec) = make_uint4(kModeRans | (G << 16) | (delta << 24), bytes, n, k);
   // bitmap word w (symbols 32w .. 32w+31) from a ballot of warp w % nwarps
   for (uint32_t w = warp; w < 8; w += nthr >> 5) {
     const uint32_t bits = __ballot_sync(0xffffffffu, freq[32 * w + lane] != 0u);

@@ -12,18 +12,23 @@ namespace {
 
 constexpr uint32_t kThreads = 256;  // 8 warps: plane p = warp / 4, group = warp % 4
 
+// Encode: one CTA per chunk, 16 warps. Warps 0-11 code the variants v = warp / 4:
+// plane 0 (v = 0), plane 1 (v = 1) and plane 1's lane deltas (v = 2), warp % 4
+// being the rANS group; all 16 share the histograms, the writes and the CRC.
+constexpr uint32_t kEncThreads = 512;
+
 struct __align__(16) EncSmem {
   uint32_t crc_t[1024];
-  uint32_t hist[2][256];
-  uint32_t freq[2][256];
+  uint32_t hist[3][256];
+  uint32_t freq[3][256];
   uint32_t rem[256];
-  uint32_t fc[2][256];
-  uint32_t rcp[2][256];
-  uint2 tab[2][256];             // {f | cum << 16, 1/f} per plane
-  uint32_t states[2][kMaxLanes];
+  uint32_t fc[3][256];
+  uint32_t rcp[3][256];
+  uint2 tab[3][256];             // {f | cum << 16, 1/f} per variant
+  uint32_t states[3][kMaxLanes];
   uint32_t tmp[32], red[32];
-  uint32_t k[2], mode[2], bytes[2], csym[2];
-  uint32_t W[2][4], wbeg[2][4], sub_len[2][4];
+  uint32_t k[3], mode[2], bytes[2], csym[2], var[2];
+  uint32_t W[3][4], wbeg[3][4], sub_len[3][4];
 };
 
 struct __align__(16) DecSmem {
@@ -47,7 +52,14 @@ struct ChanMajor {
   }
 };
 
-__global__ void __launch_bounds__(kThreads)
+// Whether stream index i starts a rANS lane (lanes of a stream of n symbols on N lanes).
+__device__ inline bool lane_start(uint32_t i, uint32_t n, uint32_t N) {
+  const uint32_t base = n / N, extra = n - base * N;
+  const uint32_t big = extra * (base + 1u);
+  return i < big ? (i % (base + 1u)) == 0u : ((i - big) % base) == 0u;
+}
+
+__global__ void __launch_bounds__(kEncThreads)
 k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   EncSmem& S = *reinterpret_cast<EncSmem*>(smem_raw);
@@ -63,7 +75,7 @@ k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
   const uint16_t* g = src + (uint64_t(slice) * sh.T + t0) * D;
 
   crc_tables_init(S.crc_t);
-  for (uint32_t i = tid; i < 512; i += nthr) (&S.hist[0][0])[i] = 0;
+  for (uint32_t i = tid; i < 3u * 256u; i += nthr) (&S.hist[0][0])[i] = 0;
   if ((reinterpret_cast<uintptr_t>(g) & 15u) == 0 && (n & 7u) == 0) {
     const uint4* g4 = reinterpret_cast<const uint4*>(g);
     uint4* v4 = reinterpret_cast<uint4*>(vals);
@@ -72,58 +84,79 @@ k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
     for (uint32_t i = tid; i < n; i += nthr) vals[i] = g[i];
   }
   __syncthreads();
-  for (uint32_t i = tid; i < n; i += nthr) {
-    uint32_t v = vals[i];
-    atomicAdd(&S.hist[0][v & 0xffu], 1u);
-    atomicAdd(&S.hist[1][v >> 8], 1u);
+  const uint32_t N = rans_lanes(n), G = rans_groups(N);
+  {
+    // histograms; stream index of value (t, d) is d * tcc + t, its predecessor in
+    // stream order is (t - 1, d), or (tcc - 1, d - 1) at t = 0
+    for (uint32_t i = tid; i < n; i += nthr) {
+      const uint32_t v = vals[i];
+      atomicAdd(&S.hist[0][v & 0xffu], 1u);
+      atomicAdd(&S.hist[1][v >> 8], 1u);
+      const uint32_t t = i / D, d = i - t * D, si = d * tcc + t;
+      uint32_t dv = v >> 8;
+      if (!lane_start(si, n, N)) {
+        const uint32_t pv = t ? vals[i - D] : vals[(tcc - 1u) * D + d - 1u];
+        dv ^= pv >> 8;
+      }
+      atomicAdd(&S.hist[2][dv], 1u);
+    }
   }
   __syncthreads();
-  for (uint32_t p = 0; p < 2; ++p) {
-    uint32_t k = block_normalize(S.hist[p], n, S.freq[p], S.rem, S.tmp);
-    if (tid == 0) S.k[p] = k;
-    block_enc_tables(S.freq[p], S.fc[p], S.rcp[p], S.tmp);
-    for (uint32_t i = tid; i < 256; i += nthr) S.tab[p][i] = make_uint2(S.fc[p][i], S.rcp[p][i]);
+  for (uint32_t v = 0; v < 3; ++v) {
+    uint32_t k = block_normalize(S.hist[v], n, S.freq[v], S.rem, S.tmp);
+    if (tid == 0) S.k[v] = k;
+    block_enc_tables(S.freq[v], S.fc[v], S.rcp[v], S.tmp);
+    for (uint32_t i = tid; i < 256; i += nthr) S.tab[v][i] = make_uint2(S.fc[v][i], S.rcp[v][i]);
   }
   __syncthreads();
 
   const ChanMajor cm(tcc);
-  const uint32_t N = rans_lanes(n), G = rans_groups(N);
   uint8_t* slot = ws.slots + uint64_t(gr) * ws.slot_bytes;
   const uint32_t rec_area = 2u * (16u + pad16(n_max));
-  uint16_t* scratch[2] = {reinterpret_cast<uint16_t*>(slot + rec_area),
-                          reinterpret_cast<uint16_t*>(slot + rec_area + 2u * n_max + 64u)};
+  uint16_t* scratch0 = reinterpret_cast<uint16_t*>(slot + rec_area);
   {
     const uint32_t warp = tid >> 5, lane = tid & 31u;
-    const uint32_t p = warp >> 2, gg = warp & 3u;
-    if (S.k[p] >= 2 && gg < G) {
+    const uint32_t v = warp >> 2, gg = warp & 3u;
+    if (v < 3 && S.k[v] >= 2 && gg < G) {
       uint32_t b0, len0, b1 = n, len1;
       lane_range(n, N, gg * kGroupLanes, b0, len0);
       if (gg + 1 < G) lane_range(n, N, (gg + 1) * kGroupLanes, b1, len1);
       // symbol i of plane p: byte p of the value of channel d = i / tcc, token t = i % tcc
-      const uint8_t* v8 = reinterpret_cast<const uint8_t*>(vals) + p;
-      uint32_t x;
-      uint32_t Wg = rans_encode_strided([v8](uint32_t d) { return v8 + 2u * d; }, 2u * D, tcc, n, N, gg,
-                                        S.tab[p], scratch[p] + b0, b1 - b0, &x);
+      const uint8_t* v8 = reinterpret_cast<const uint8_t*>(vals) + (v ? 1u : 0u);
+      uint16_t* scratch = scratch0 + uint64_t(v) * (n_max + 32u);
+      uint32_t x, Wg;
+      if (v < 2)
+        Wg = rans_encode_strided([v8](uint32_t d) { return v8 + 2u * d; }, 2u * D, tcc, n, N, gg, S.tab[v],
+                                 scratch + b0, b1 - b0, &x);
+      else
+        Wg = rans_encode_strided<true>([v8](uint32_t d) { return v8 + 2u * d; }, 2u * D, tcc, n, N, gg,
+                                       S.tab[v], scratch + b0, b1 - b0, &x);
       uint32_t l = gg * kGroupLanes + lane;
-      if (l < N) S.states[p][l] = x;
+      if (l < N) S.states[v][l] = x;
       if (lane == 0) {
-        S.W[p][gg] = Wg;
-        S.wbeg[p][gg] = b0 + (b1 - b0) - Wg;
+        S.W[v][gg] = Wg;
+        S.wbeg[v][gg] = b0 + (b1 - b0) - Wg;
       }
     }
   }
   __syncthreads();
   if (tid == 0) {
+    // per plane: CONST for one symbol; else the smallest of RANS (plain), RANS of
+    // the lane deltas (plane 1, only if strictly smaller than both others) and RAW
+    const uint32_t raw_b = 16u + pad16(n);
     for (uint32_t p = 0; p < 2; ++p) {
-      uint32_t k = S.k[p], raw_b = 16u + pad16(n);
-      uint32_t v0 = vals[0];
+      const uint32_t k = S.k[p];
+      const uint32_t v0 = vals[0];
       S.csym[p] = p ? (v0 >> 8) : (v0 & 0xffu);
-      if (k == 1) { S.mode[p] = kModeConst; S.bytes[p] = 16; }
-      else if (k >= 2) {
-        uint32_t rb = rans_layout(n, k, S.W[p], S.sub_len[p]);
-        if (rb < raw_b) { S.mode[p] = kModeRans; S.bytes[p] = rb; }
-        else { S.mode[p] = kModeRaw; S.bytes[p] = raw_b; }
-      } else { S.mode[p] = kModeRaw; S.bytes[p] = raw_b; }
+      S.var[p] = p;
+      if (k == 1) { S.mode[p] = kModeConst; S.bytes[p] = 16; continue; }
+      if (k < 2) { S.mode[p] = kModeRaw; S.bytes[p] = raw_b; continue; }
+      const uint32_t rb = rans_layout(n, k, S.W[p], S.sub_len[p]);
+      uint32_t rd = 0xffffffffu;
+      if (p == 1 && S.k[2] >= 2) rd = rans_layout(n, S.k[2], S.W[2], S.sub_len[2]);
+      if (rd < rb && rd < raw_b) { S.mode[p] = kModeRans; S.bytes[p] = rd; S.var[p] = 2; }
+      else if (rb < raw_b) { S.mode[p] = kModeRans; S.bytes[p] = rb; }
+      else { S.mode[p] = kModeRaw; S.bytes[p] = raw_b; }
     }
   }
   __syncthreads();
@@ -136,20 +169,22 @@ k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
       uint32_t v = vals[t * D + d];
       return p ? (v >> 8) : (v & 0xffu);
     };
+    const uint32_t v = S.var[p];
     if (S.mode[p] == kModeRaw && (tcc & 15u) == 0) {
       // raw plane: thread writes 16 tokens of one channel, neighbouring threads neighbouring channels
       if (tid == 0) *reinterpret_cast<uint4*>(rec + off) = make_uint4(kModeRaw, S.bytes[p], n, 0u);
       const uint8_t* v8 = reinterpret_cast<const uint8_t*>(vals) + p;
       for (uint32_t idx = tid; idx < n / 16u; idx += nthr) {
-        const uint32_t d = idx % D, t0 = 16u * (idx / D);
+        const uint32_t d = idx % D, tq = 16u * (idx / D);
         uint32_t w[4] = {0, 0, 0, 0};
 #pragma unroll
-        for (uint32_t k = 0; k < 16; ++k) w[k >> 2] |= uint32_t(v8[2u * ((t0 + k) * D + d)]) << (8u * (k & 3u));
-        *reinterpret_cast<uint4*>(rec + off + 16u + d * tcc + t0) = make_uint4(w[0], w[1], w[2], w[3]);
+        for (uint32_t k = 0; k < 16; ++k) w[k >> 2] |= uint32_t(v8[2u * ((tq + k) * D + d)]) << (8u * (k & 3u));
+        *reinterpret_cast<uint4*>(rec + off + 16u + d * tcc + tq) = make_uint4(w[0], w[1], w[2], w[3]);
       }
     } else {
-      block_write_stream(rec + off, S.mode[p], n, S.bytes[p], S.csym[p], S.k[p], S.freq[p],
-                         S.states[p], scratch[p], S.wbeg[p], S.W[p], S.sub_len[p], raw, S.tmp);
+      block_write_stream(rec + off, S.mode[p], n, S.bytes[p], S.csym[p], S.k[v], S.freq[v], S.states[v],
+                         scratch0 + uint64_t(v) * (n_max + 32u), S.wbeg[v], S.W[v], S.sub_len[v], raw, S.tmp,
+                         v == 2 ? 1u : 0u);
     }
     off += S.bytes[p];
   }
@@ -223,8 +258,14 @@ k_lossless_decode(LosslessShape sh, FrameBatch b, uint8_t* ws) {
       const uint32_t N = rans_lanes(n), G = rans_groups(N);
       if (S.si[p].mode == kModeRans && gg < G) {
         uint8_t* pl = planes[p];
-        ok = rans_decode_group(recp[p] + S.si[p].sub_off[gg], S.si[p].sub_len[gg], n, N, gg,
-                               S.lut[p], [&](uint32_t i, uint32_t s) { pl[i] = uint8_t(s); });
+        // a lane-delta record: each lane's outputs are the running XOR of its symbols
+        const uint32_t dm = S.si[p].delta ? 0xffu : 0u;
+        uint32_t prev = 0;
+        ok = rans_decode_group(recp[p] + S.si[p].sub_off[gg], S.si[p].sub_len[gg], n, N, gg, S.lut[p],
+                               [&](uint32_t i, uint32_t s) {
+                                 prev = s ^ (prev & dm);
+                                 pl[i] = uint8_t(prev);
+                               });
       }
     }
     if (!__syncthreads_and(ok)) {
@@ -436,6 +477,9 @@ __device__ inline bool fast_tiles(FastSmem& S, const uint8_t* const recp[2], uin
     win.request(0, lane);
     asm volatile("cp.async.commit_group;" ::: "memory");  // empty group: the first settle waits for the window
   }
+  // lane deltas: each decoded symbol is XORed with the lane's previous output
+  const uint32_t dm = (kRans && S.si[RP].delta) ? 0xffu : 0u;
+  uint32_t prev = 0;
   uint4 n0a = make_uint4(0, 0, 0, 0), n0b = n0a, n1a = n0a, n1b = n0a;  // next tile's raw bytes
   if (kRaw0) { n0a = __ldcg(reinterpret_cast<const uint4*>(raw0)); n0b = __ldcg(reinterpret_cast<const uint4*>(raw0 + 16)); }
   if (kRaw1) { n1a = __ldcg(reinterpret_cast<const uint4*>(raw1)); n1b = __ldcg(reinterpret_cast<const uint4*>(raw1 + 16)); }
@@ -474,7 +518,11 @@ __device__ inline bool fast_tiles(FastSmem& S, const uint8_t* const recp[2], uin
 #pragma unroll
         for (uint32_t h = 0; h < 2; ++h) {
           const uint32_t jj = j + h;
-          const uint32_t e = kRans ? rs.step(S.lut, lt) : 0u;
+          uint32_t e = 0u;
+          if (kRans) {
+            e = rs.step(S.lut, lt) ^ (prev & dm);
+            prev = e;
+          }
           const uint32_t a = kRaw0 ? r0[jj >> 2] : (M0 == kModeRans ? e : c0);
           const uint32_t b = kRaw1 ? r1[jj >> 2] : (M1 == kModeRans ? e : c1);
           v[h] = merge_planes<M0, M1>(jj, a, b);
@@ -648,7 +696,7 @@ int num_sms() {
 
 uint64_t lossless_slot_bytes(const LosslessShape& s) {
   const uint64_t n_max = uint64_t(s.tc) * s.D;
-  uint64_t b = 2u * (16u + pad16_64(n_max)) + 2u * (2u * n_max + 64u);
+  uint64_t b = 2u * (16u + pad16_64(n_max)) + 3u * (2u * n_max + 64u);  // records + 3 word scratch areas
   return (b + 255u) & ~uint64_t(255);
 }
 
@@ -662,7 +710,7 @@ cudaError_t launch_lossless_encode(const LosslessShape& s, const FrameBatch& b,
   if (e != cudaSuccess) return e;
   {
     ProfRange pr_("lossless_encode", st);
-    k_lossless_encode<<<nrec, kThreads, smem, st>>>(s, b, ws);
+    k_lossless_encode<<<nrec, kEncThreads, smem, st>>>(s, b, ws);
   }
   return cudaGetLastError();
 }

@@ -890,7 +890,7 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
       const uint32_t m = S.ci.bcount[bw];
       if (!m) continue;
       const uint32_t o = S.str_off[bw - 1];
-      st = block_parse_stream(rec + o, len - o, m * tcc, &S.si[bw - 1], S.freq[bw - 1], S.tmp);
+      st = block_parse_stream(rec + o, len - o, m * tcc, &S.si[bw - 1], S.freq[bw - 1], S.tmp, false);
     }
     if (st != kOk) {
       if (tid == 0) atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(st));
