@@ -402,6 +402,23 @@ __device__ inline void block_enc_tables(const uint32_t* freq, uint32_t* fc, uint
   __syncthreads();
 }
 
+// The same tables packed per symbol: tab[s] = {f | cum << 16, floor((2^32-1)/f)}.
+__device__ inline void block_enc_tab(const uint32_t* freq, uint2* tab, uint32_t* tmp) {
+  const uint32_t per = blockDim.x >= 256 ? 1u : 256u / blockDim.x;
+  const uint32_t s0 = threadIdx.x * per;
+  uint32_t mine = 0;
+  for (uint32_t i = 0; i < per; ++i) mine += s0 + i < 256 ? freq[s0 + i] : 0u;
+  uint32_t cum = block_exclusive_scan(mine, tmp, nullptr);
+  for (uint32_t i = 0; i < per; ++i) {
+    const uint32_t s = s0 + i;
+    if (s >= 256) break;
+    const uint32_t f = freq[s];
+    tab[s] = make_uint2(f | (cum << 16), f ? 0xffffffffu / f : 0u);
+    cum += f;
+  }
+  __syncthreads();
+}
+
 // Decode table: lut[slot] = s | (slot - cum_s) << 8 | f_s << 20, and the
 // symbols' cumulative starts in cum[257]. freq must be validated (sum 4096).
 // The first slot of every present symbol is marked with s + 1; each warp then

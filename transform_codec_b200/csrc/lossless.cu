@@ -60,12 +60,14 @@ __device__ inline bool lane_start(uint32_t i, uint32_t n, uint32_t N) {
 }
 
 __global__ void __launch_bounds__(kEncThreads)
-k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
+k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws, uint32_t tail_only) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   EncSmem& S = *reinterpret_cast<EncSmem*>(smem_raw);
   uint16_t* vals = reinterpret_cast<uint16_t*>(smem_raw + sizeof(EncSmem));
   const uint32_t tid = threadIdx.x, nthr = blockDim.x;
-  const uint32_t gr = blockIdx.x;  // record of the batch
+  // record of the batch: every record, or the last chunk of every slice (frames
+  // hold whole slices, so those are records cps - 1, 2 cps - 1, ...)
+  const uint32_t gr = tail_only ? (blockIdx.x + 1u) * sh.cps - 1u : blockIdx.x;
   const uint32_t fr = frame_of(b.rec_base, b.n, gr);
   const uint32_t r = gr - b.rec_base[fr];
   const uint16_t* src = reinterpret_cast<const uint16_t*>(b.f[fr].src);
@@ -297,6 +299,387 @@ k_lossless_decode(LosslessShape sh, FrameBatch b, uint8_t* ws) {
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Fast encoder for full chunks of D = 128 or 64 channels (tc * D = 65536
+// values, 16-byte aligned input). 128 threads; thread l is rANS lane l of all
+// three variants (lane l: channel l / LPC, tokens (l % LPC) * 512 .. + 512,
+// LPC = 128 / D; warp w = rANS group w). Only tables and a small refill ring
+// live in shared memory, so several chunks share an SM. Phases:
+//  1. histograms of plane 0, plane 1 and plane 1's lane deltas in one pass.
+//     Plane 1 and the deltas are counted by runs of equal high bytes along
+//     tokens: a delta is zero exactly while a run goes on, so the hot bins see
+//     one atomic per run instead of one per value;
+//  2. the three frequency tables;
+//  3. each thread runs its lane's three rANS chains side by side, reading
+//     token rows that cp.async stages into a four-slot ring per warp;
+//  4. the smallest choice per plane, by the general encoder's rule;
+//  5. each thread assembles a contiguous run of the record's 16-byte units
+//     (prefix and states from shared memory, words from the scratch, a RAW
+//     payload transposed through a shared tile) and folds it into its CRC
+//     register; the registers are joined with powers of x.
+constexpr uint32_t kFencThreads = 128;
+constexpr uint32_t kFencStage = 16;                     // rANS steps per ring stage
+constexpr uint32_t kFencSlots = 4;                      // ring slots: 3 stages in flight
+constexpr uint32_t kFencRowBytes = 64;                  // one token row of a warp's 32 lanes
+constexpr uint32_t kFencSlotBytes = kFencStage * kFencRowBytes;
+constexpr uint32_t kGroupWords = kGroupLanes * 512u;    // scratch words of one (variant, group)
+constexpr uint32_t kVarWords = kMaxChunkValues + 32u;   // scratch words of one variant
+constexpr uint32_t kRecArea = 2u * (16u + kMaxChunkValues);
+constexpr uint32_t kXRawPayload = gf2_xpow8(kMaxChunkValues);  // joins a RAW header to its payload
+
+struct __align__(16) FencSmem {
+  uint32_t crc_t[1024];
+  uint32_t freq[3][256];
+  uint2 tab[3][256];
+  uint32_t states[3][kMaxLanes];
+  union {
+    struct {
+      uint32_t hist[3][256];
+      uint32_t rem[256];
+    } h;                                                // phases 1-2
+    uint8_t ring[kFencThreads / 32][kFencSlots][kFencSlotBytes];  // phase 3
+    uint4 tile[256];                                    // phase 5, RAW planes
+  } u;
+  uint4 prefix[2][36];  // RANS record prefix: header, bitmap, frequencies, lengths (<= 576 B)
+  uint32_t tmp[32], red[32];
+  uint32_t k[3], W[3][4], sub_len[2][4], subst[2][5];
+  uint32_t mode[2], bytes[2], var[2], csym[2], pbytes[2], crc[2];
+};
+
+__device__ __forceinline__ uint32_t crc_unit(const uint32_t* t, uint32_t c, uint4 v) {
+  c = crc_word(t, c, v.x);
+  c = crc_word(t, c, v.y);
+  c = crc_word(t, c, v.z);
+  return crc_word(t, c, v.w);
+}
+
+// One rANS encode step of a warp's 32 lanes (all active): renormalise into the
+// group's word area (ascending lanes at ascending addresses), then encode sym.
+__device__ __forceinline__ void fenc_step(const uint2* tab, uint32_t sym, uint32_t& x, uint32_t& pos,
+                                          uint16_t* words, uint32_t lt) {
+  const uint2 e = tab[sym];
+  const uint32_t f = e.x & 0xffffu, cum = e.x >> 16;
+  const bool emit = x >= (f << 20);
+  const uint32_t mask = __ballot_sync(0xffffffffu, emit);
+  pos -= __popc(mask);
+  if (emit) words[pos + __popc(mask & lt)] = uint16_t(x & 0xffffu);
+  const uint32_t xe = emit ? (x >> 16) : x;
+  uint32_t q = __umulhi(xe, e.y);
+  uint32_t r = xe - q * f;
+  const bool over = r >= f;
+  q += over ? 1u : 0u;
+  r -= over ? f : 0u;
+  x = (q << kProbBits) + r + cum;
+}
+
+__device__ __forceinline__ uint32_t lds_u16(const uint8_t* p) {
+  return *reinterpret_cast<const uint16_t*>(p);
+}
+
+template <uint32_t D>
+__global__ void __launch_bounds__(kFencThreads, 6)
+k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
+  constexpr uint32_t TCC = kMaxChunkValues / D, LPC = 128u / D;
+  constexpr uint32_t CB = D / 8u;                       // 16-byte column blocks of a token row
+  constexpr uint32_t SEGLEN = TCC / (kFencThreads / CB);  // tokens per histogram segment (64)
+  constexpr uint32_t n = kMaxChunkValues;
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  FencSmem& S = *reinterpret_cast<FencSmem*>(smem_raw);
+  const uint32_t tid = threadIdx.x, lane = tid & 31u, warp = tid >> 5;
+  const uint32_t gr = blockIdx.x;  // record of the batch
+  const uint32_t fr = frame_of(b.rec_base, b.n, gr), r = gr - b.rec_base[fr];
+  const uint32_t slice = r / sh.cps, t0 = (r % sh.cps) * sh.tc;
+  if (sh.T - t0 < TCC) return;  // ragged last chunk: the general encoder's
+  const uint16_t* g = reinterpret_cast<const uint16_t*>(b.f[fr].src) + (uint64_t(slice) * sh.T + t0) * D;
+  const uint4* g4 = reinterpret_cast<const uint4*>(g);
+
+  crc_tables_init(S.crc_t);
+  for (uint32_t i = tid; i < 3u * 256u; i += kFencThreads) (&S.u.h.hist[0][0])[i] = 0;
+  __syncthreads();
+  {
+    // thread: column block cb (8 channels), tokens [tb, tb + SEGLEN); cur[j] is
+    // the previous token's high byte (0 before a lane's first token, which
+    // makes its delta the byte itself), run[j] the count of equal bytes so far
+    const uint32_t cb = tid % CB, tb = (tid / CB) * SEGLEN;
+    const uint4* col = g4 + cb;
+    uint32_t cur[8], run[8], zeros = 0;
+    if (tb % 512u == 0) {
+#pragma unroll
+      for (uint32_t j = 0; j < 8; ++j) cur[j] = 0;
+    } else {
+      const uint4 w = __ldg(col + uint64_t(tb - 1u) * CB);
+      const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (uint32_t j = 0; j < 8; ++j) cur[j] = (wv[j >> 1] >> (16u * (j & 1u) + 8u)) & 0xffu;
+    }
+#pragma unroll
+    for (uint32_t j = 0; j < 8; ++j) run[j] = 0;
+#pragma unroll 1
+    for (uint32_t t = tb; t < tb + SEGLEN; t += 4) {
+      uint4 rows[4];
+#pragma unroll
+      for (uint32_t i = 0; i < 4; ++i) rows[i] = __ldg(col + uint64_t(t + i) * CB);
+#pragma unroll
+      for (uint32_t i = 0; i < 4; ++i) {
+        const uint32_t wv[4] = {rows[i].x, rows[i].y, rows[i].z, rows[i].w};
+#pragma unroll
+        for (uint32_t j = 0; j < 8; ++j) {
+          const uint32_t v = wv[j >> 1] >> (16u * (j & 1u));
+          atomicAdd(&S.u.h.hist[0][v & 0xffu], 1u);
+          const uint32_t hb = (v >> 8) & 0xffu;
+          if (hb == cur[j]) {
+            ++run[j];
+            ++zeros;
+          } else {
+            if (run[j]) atomicAdd(&S.u.h.hist[1][cur[j]], run[j]);
+            atomicAdd(&S.u.h.hist[2][hb ^ cur[j]], 1u);
+            cur[j] = hb;
+            run[j] = 1;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (uint32_t j = 0; j < 8; ++j)
+      if (run[j]) atomicAdd(&S.u.h.hist[1][cur[j]], run[j]);
+    if (zeros) atomicAdd(&S.u.h.hist[2][0], zeros);
+  }
+  __syncthreads();
+  for (uint32_t v = 0; v < 3; ++v) {
+    const uint32_t k = block_normalize(S.u.h.hist[v], n, S.freq[v], S.u.h.rem, S.tmp);
+    if (tid == 0) S.k[v] = k;
+    if (k >= 2) block_enc_tab(S.freq[v], S.tab[v], S.tmp);
+  }
+  __syncthreads();
+  const bool en0 = S.k[0] >= 2, en1 = S.k[1] >= 2, en2 = en1 && S.k[2] >= 2;
+  uint8_t* slot = ws.slots + uint64_t(gr) * ws.slot_bytes;
+  uint16_t* scratch0 = reinterpret_cast<uint16_t*>(slot + kRecArea);
+  {
+    // ring stage s holds lane steps tau = 16 s .. 16 s + 15; unit u = 4 j + q of
+    // a stage is 16 bytes of token row j: D = 128: channels 32 w + 8 q .. + 7 of
+    // token tau; D = 64: channels 16 w + 8 (q & 1) .. + 7 of token (q >> 1) * 512 + tau
+    uint16_t* sc0 = scratch0 + warp * kGroupWords;
+    uint16_t* sc1 = sc0 + kVarWords;
+    uint16_t* sc2 = sc1 + kVarWords;
+    const uint8_t* ring = &S.u.ring[warp][0][0];
+    const uint32_t ring_saddr = tc::smem_addr(ring);
+    const uint32_t loff = LPC == 1 ? 2u * lane : (lane & 1u) * 32u + (lane >> 1) * 2u;
+    auto issue = [&](uint32_t s) {
+#pragma unroll
+      for (uint32_t i = 0; i < 2; ++i) {
+        const uint32_t u = lane + 32u * i, j = u >> 2, q = u & 3u;
+        const uint32_t row = (LPC == 1 ? 0u : (q >> 1) * 512u) + s * kFencStage + j;
+        const uint32_t c0 = LPC == 1 ? 32u * warp + 8u * q : 16u * warp + 8u * (q & 1u);
+        const uint16_t* src = g + uint64_t(row) * D + c0;
+        const uint32_t dst = ring_saddr + (s % kFencSlots) * kFencSlotBytes + 16u * u;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    const uint32_t lt = lanemask_lt();
+    uint32_t x0 = kRansLow, x1 = kRansLow, x2 = kRansLow;
+    uint32_t p0 = kGroupWords, p1 = kGroupWords, p2 = kGroupWords;
+    constexpr uint32_t kStages = 512u / kFencStage;
+    issue(kStages - 1);
+    issue(kStages - 2);
+    issue(kStages - 3);
+    uint32_t vcur = 0;
+#pragma unroll 1
+    for (int s = int(kStages) - 1; s >= 0; --s) {
+      __syncwarp();  // every lane is done with the slot the next copy overwrites
+      if (s >= 3) issue(uint32_t(s) - 3u);
+      else asm volatile("cp.async.commit_group;" ::: "memory");
+      asm volatile("cp.async.wait_group 2;" ::: "memory");  // stages s and s - 1 landed
+      __syncwarp();
+      const uint8_t* cur = ring + (uint32_t(s) % kFencSlots) * kFencSlotBytes + loff;
+      const uint8_t* prv = ring + ((uint32_t(s) + kFencSlots - 1u) % kFencSlots) * kFencSlotBytes + loff;
+      if (s == int(kStages) - 1) vcur = lds_u16(cur + (kFencStage - 1u) * kFencRowBytes);
+#pragma unroll
+      for (int j = int(kFencStage) - 1; j >= 0; --j) {
+        // the value one step earlier in the lane (0 before the lane's first)
+        const uint32_t vprev = j ? lds_u16(cur + uint32_t(j - 1) * kFencRowBytes)
+                                 : (s ? lds_u16(prv + (kFencStage - 1u) * kFencRowBytes) : 0u);
+        const uint32_t hb = vcur >> 8;
+        if (en0) fenc_step(S.tab[0], vcur & 0xffu, x0, p0, sc0, lt);
+        if (en1) fenc_step(S.tab[1], hb, x1, p1, sc1, lt);
+        if (en2) fenc_step(S.tab[2], hb ^ (vprev >> 8), x2, p2, sc2, lt);
+        vcur = vprev;
+      }
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    S.states[0][tid] = x0;
+    S.states[1][tid] = x1;
+    S.states[2][tid] = x2;
+    if (lane == 0) {
+      S.W[0][warp] = kGroupWords - p0;
+      S.W[1][warp] = kGroupWords - p1;
+      S.W[2][warp] = kGroupWords - p2;
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    // per plane: CONST for one symbol; else the smallest of RANS (plain), RANS of
+    // the lane deltas (plane 1, only if strictly smaller than both others) and RAW
+    const uint32_t raw_b = 16u + n, v0 = g[0];
+    for (uint32_t p = 0; p < 2; ++p) {
+      const uint32_t k = S.k[p];
+      S.csym[p] = p ? (v0 >> 8) : (v0 & 0xffu);
+      S.var[p] = p;
+      if (k == 1) {
+        S.mode[p] = kModeConst;
+        S.bytes[p] = 16;
+        continue;
+      }
+      const uint32_t rb = rans_layout(n, k, S.W[p], S.sub_len[p]);
+      uint32_t rd = 0xffffffffu, dl[4];
+      if (p == 1 && S.k[2] >= 2) rd = rans_layout(n, S.k[2], S.W[2], dl);
+      if (rd < rb && rd < raw_b) {
+        S.mode[p] = kModeRans;
+        S.bytes[p] = rd;
+        S.var[p] = 2;
+        for (uint32_t q = 0; q < 4; ++q) S.sub_len[p][q] = dl[q];
+      } else if (rb < raw_b) {
+        S.mode[p] = kModeRans;
+        S.bytes[p] = rb;
+      } else {
+        S.mode[p] = kModeRaw;
+        S.bytes[p] = raw_b;
+      }
+      if (S.mode[p] == kModeRans) {
+        const uint32_t pb = pad16(48u + 2u * S.k[S.var[p]]) + 16u;
+        S.pbytes[p] = pb;
+        uint32_t o = pb;
+        for (uint32_t q = 0; q < 4; ++q) {
+          S.subst[p][q] = o;
+          o += pad16(S.sub_len[p][q]);
+        }
+        S.subst[p][4] = o;
+      }
+    }
+  }
+  for (uint32_t i = tid; i < 2u * 36u; i += kFencThreads) (&S.prefix[0][0])[i] = make_uint4(0, 0, 0, 0);
+  __syncthreads();
+  // RANS prefixes: header, presence bitmap, frequencies of present symbols, sub-stream lengths
+  for (uint32_t p = 0; p < 2; ++p) {
+    if (S.mode[p] != kModeRans) continue;
+    const uint32_t v = S.var[p], k = S.k[v];
+    uint8_t* pf = reinterpret_cast<uint8_t*>(S.prefix[p]);
+    const uint32_t* fq = S.freq[v];
+    if (tid == 0)
+      *reinterpret_cast<uint4*>(pf) = make_uint4(kModeRans | (4u << 16) | ((v == 2 ? 1u : 0u) << 24), S.bytes[p], n, k);
+    for (uint32_t wd = warp; wd < 8; wd += kFencThreads / 32u) {
+      const uint32_t bits = __ballot_sync(0xffffffffu, fq[32u * wd + lane] != 0u);
+      if (lane == 0) reinterpret_cast<uint32_t*>(pf + 16)[wd] = bits;
+    }
+    const uint32_t s0 = 2u * tid, f0 = fq[s0], f1 = fq[s0 + 1u];
+    uint32_t idx = block_exclusive_scan((f0 ? 1u : 0u) + (f1 ? 1u : 0u), S.tmp, nullptr);
+    uint16_t* fl = reinterpret_cast<uint16_t*>(pf + 48);
+    if (f0) fl[idx++] = uint16_t(f0);
+    if (f1) fl[idx] = uint16_t(f1);
+    if (tid < 4) reinterpret_cast<uint32_t*>(pf + S.pbytes[p] - 16u)[tid] = S.sub_len[p][tid];
+  }
+  __syncthreads();
+  uint8_t* rec = slot;
+  uint32_t off = 0;
+  for (uint32_t p = 0; p < 2; ++p) {
+    const uint32_t mode = S.mode[p], bytes = S.bytes[p];
+    uint8_t* out = rec + off;
+    uint32_t creg = 0;  // CRC register of this plane's stream record (thread 0 after the join)
+    if (mode == kModeConst) {
+      if (tid == 0) {
+        uint4 h = make_uint4(kModeConst | (S.csym[p] << 8), 16u, n, 1u);
+        *reinterpret_cast<uint4*>(out) = h;
+        if (p == 0) h.x = ~h.x;
+        creg = crc_unit(S.crc_t, 0u, h);
+      }
+    } else if (mode == kModeRaw) {
+      // payload unit 1 + 32 t + i: 16 tokens (block i) of thread t's lane range,
+      // i.e. channel t / LPC, tokens (t % LPC) * 512 + 16 i .. + 15; the tile holds
+      // those 16 token rows of every lane (both halves for D = 64)
+      uint32_t hreg = 0;
+      if (tid == 0) {
+        uint4 h = make_uint4(kModeRaw, bytes, n, 0u);
+        *reinterpret_cast<uint4*>(out) = h;
+        if (p == 0) h.x = ~h.x;
+        hreg = crc_unit(S.crc_t, 0u, h);
+      }
+      auto tile_src = [&](uint32_t i, uint32_t m) -> const uint4* {
+        return LPC == 1 ? g4 + (16u * i) * CB + m
+                        : g4 + uint64_t((m >> 7) * 512u + 16u * i) * CB + (m & 127u);
+      };
+      uint4 nx0 = __ldcg(tile_src(0, tid)), nx1 = __ldcg(tile_src(0, tid + 128u));
+      const uint8_t* tb = reinterpret_cast<const uint8_t*>(S.u.tile) + p +
+                          (LPC == 1 ? 2u * tid : (tid & 1u) * 2048u + 2u * (tid >> 1));
+      constexpr uint32_t RS = 2u * D;  // tile row stride
+#pragma unroll 1
+      for (uint32_t i = 0; i < 32; ++i) {
+        __syncthreads();
+        S.u.tile[tid] = nx0;
+        S.u.tile[tid + 128u] = nx1;
+        __syncthreads();
+        if (i + 1 < 32) {
+          nx0 = __ldcg(tile_src(i + 1, tid));
+          nx1 = __ldcg(tile_src(i + 1, tid + 128u));
+        }
+        uint32_t w[4];
+#pragma unroll
+        for (uint32_t e = 0; e < 4; ++e)
+          w[e] = uint32_t(tb[(4u * e) * RS]) | (uint32_t(tb[(4u * e + 1u) * RS]) << 8) |
+                 (uint32_t(tb[(4u * e + 2u) * RS]) << 16) | (uint32_t(tb[(4u * e + 3u) * RS]) << 24);
+        const uint4 val = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(out + 16u * (1u + 32u * tid + i)) = val;
+        creg = crc_unit(S.crc_t, creg, val);
+      }
+      creg = crc_join_lanes(creg, 32u, S.red);
+      if (tid == 0) creg = gf2_mul(hreg, kXRawPayload) ^ creg;
+    } else {
+      // RANS: thread t owns units [t q, t q + q) of the record right-aligned in
+      // 128 q units (leading zero units leave a zero register unchanged)
+      const uint32_t v = S.var[p], U = bytes >> 4, q = (U + 127u) >> 7, z = 128u * q - U;
+      const uint16_t* scv = scratch0 + v * kVarWords;
+      for (uint32_t i = 0; i < q; ++i) {
+        const int32_t u = int32_t(tid * q + i) - int32_t(z);
+        if (u < 0) continue;
+        const uint32_t o = 16u * uint32_t(u);
+        uint4 val;
+        if (o < S.pbytes[p]) {
+          val = S.prefix[p][u];
+        } else {
+          uint32_t gg = 0;
+          while (gg < 3 && o >= S.subst[p][gg + 1]) ++gg;
+          const uint32_t ro = o - S.subst[p][gg];
+          if (ro < 4u * kGroupLanes) {
+            val = *reinterpret_cast<const uint4*>(&S.states[v][kGroupLanes * gg + (ro >> 2)]);
+          } else {
+            const uint32_t wi = (ro - 4u * kGroupLanes) >> 1, Wg = S.W[v][gg];
+            const uint16_t* src = scv + gg * kGroupWords + (kGroupWords - Wg);
+            uint32_t w[4];
+#pragma unroll
+            for (uint32_t e = 0; e < 4; ++e) {
+              const uint32_t i0 = wi + 2u * e;
+              const uint32_t lo = i0 < Wg ? uint32_t(src[i0]) : 0u;
+              const uint32_t hi = i0 + 1u < Wg ? uint32_t(src[i0 + 1u]) : 0u;
+              w[e] = lo | (hi << 16);
+            }
+            val = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+        *reinterpret_cast<uint4*>(out + o) = val;
+        if (p == 0 && u == 0) val.x = ~val.x;
+        creg = crc_unit(S.crc_t, creg, val);
+      }
+      creg = crc_join_lanes(creg, q, S.red);
+    }
+    if (tid == 0) S.crc[p] = creg;
+    off += bytes;
+  }
+  if (tid == 0) {
+    const uint32_t c = gf2_mul(S.crc[0], gf2_xpow8(S.bytes[1])) ^ S.crc[1];
+    ws.rec_len[gr] = off;
+    ws.rec_crc[gr] = c ^ 0xffffffffu;
+  }
+}
 
 // ---------------------------------------------------------------------------
 // Fast decoder for full chunks of D = 128 or 64 channels (tc * D = 65536
@@ -704,13 +1087,31 @@ cudaError_t launch_lossless_encode(const LosslessShape& s, const FrameBatch& b,
                                    const EncodeLayout& ws, cudaStream_t st) {
   const uint32_t nrec = b.rec_base[b.n];
   if (nrec == 0) return cudaSuccess;
+  // full chunks of 65536 values with D = 128 or 64 and 16-byte aligned input go
+  // to the fast encoder; the general one takes the rest (with the fast one, only
+  // the ragged last chunk of each slice)
+  bool fast = s.tc * s.D == kMaxChunkValues && (s.D == 128u || s.D == 64u);
+  for (uint32_t f = 0; f < b.n; ++f)
+    if (reinterpret_cast<uintptr_t>(b.f[f].src) & 15u) fast = false;
+  cudaError_t e;
+  if (fast) {
+    const size_t fsmem = sizeof(FencSmem);
+    auto kern = s.D == 128u ? k_lossless_encode_fast<128> : k_lossless_encode_fast<64>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(fsmem));
+    if (e != cudaSuccess) return e;
+    {
+      ProfRange pr_("lossless_encode", st);
+      kern<<<nrec, kFencThreads, fsmem, st>>>(s, b, ws);
+    }
+    e = cudaGetLastError();
+    if (e != cudaSuccess || s.T % s.tc == 0) return e;
+  }
   size_t smem = sizeof(EncSmem) + pad16(s.tc * s.D * 2u);
-  cudaError_t e = cudaFuncSetAttribute(k_lossless_encode, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(smem));
+  e = cudaFuncSetAttribute(k_lossless_encode, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   {
-    ProfRange pr_("lossless_encode", st);
-    k_lossless_encode<<<nrec, kEncThreads, smem, st>>>(s, b, ws);
+    ProfRange pr_(fast ? "lossless_encode_tail" : "lossless_encode", st);
+    k_lossless_encode<<<fast ? nrec / s.cps : nrec, kEncThreads, smem, st>>>(s, b, ws, fast ? 1u : 0u);
   }
   return cudaGetLastError();
 }
