@@ -359,25 +359,31 @@ __device__ inline uint32_t block_normalize(const uint32_t* hist, uint32_t n, uin
     fsum += f;
   }
   const uint32_t sum = block_sum(fsum, tmp);  // synchronises: rem and freq complete
-  if (k >= 2) {
-    const uint32_t d = kProbScale - sum;
-    uint32_t add[4] = {0, 0, 0, 0};
-    if (d) {
+  const uint32_t d = k >= 2 ? kProbScale - sum : 0u;
+  if (d) {
+    // The d present symbols with the largest keys (r << 8) | (255 - s) (largest
+    // remainder, ties to the smaller symbol; keys are distinct) get one more.
+    // Radix select of the d-th largest key, one bit per round: P holds the key
+    // bits fixed so far, need the rank still sought among keys with prefix P.
+    uint32_t P = 0, need = d;
+    for (int bit = 23; bit >= 0; --bit) {
+      uint32_t cnt = 0;
       for (uint32_t i = 0; i < per; ++i) {
         const uint32_t s = s0 + i;
-        if (s >= 256 || !hist[s]) continue;
-        const uint32_t r = rem[s];
-        uint32_t rank = 0;
-        for (uint32_t s2 = 0; s2 < 256; ++s2) {
-          const uint32_t r2 = rem[s2];
-          rank += (hist[s2] != 0u) & ((r2 > r) | ((r2 == r) & (s2 < s)));
-        }
-        add[i] = rank < d ? 1u : 0u;
+        const bool present = s < 256 && hist[s];
+        const uint32_t key = present ? (rem[s] << 8) | (255u - s) : 0u;
+        cnt += __syncthreads_count(present && (key >> bit) == ((P << 1) | 1u));
+      }
+      if (cnt >= need) P = (P << 1) | 1u;
+      else {
+        need -= cnt;
+        P <<= 1;
       }
     }
-    __syncthreads();
-    for (uint32_t i = 0; i < per; ++i)
-      if (s0 + i < 256) freq[s0 + i] += add[i];
+    for (uint32_t i = 0; i < per; ++i) {
+      const uint32_t s = s0 + i;
+      if (s < 256 && hist[s] && ((rem[s] << 8) | (255u - s)) >= P) freq[s] += 1u;
+    }
   }
   __syncthreads();
   return k;
@@ -402,21 +408,69 @@ __device__ inline void block_enc_tables(const uint32_t* freq, uint32_t* fc, uint
   __syncthreads();
 }
 
-// The same tables packed per symbol: tab[s] = {f | cum << 16, floor((2^32-1)/f)}.
-__device__ inline void block_enc_tab(const uint32_t* freq, uint2* tab, uint32_t* tmp) {
-  const uint32_t per = blockDim.x >= 256 ? 1u : 256u / blockDim.x;
-  const uint32_t s0 = threadIdx.x * per;
-  uint32_t mine = 0;
-  for (uint32_t i = 0; i < per; ++i) mine += s0 + i < 256 ? freq[s0 + i] : 0u;
-  uint32_t cum = block_exclusive_scan(mine, tmp, nullptr);
-  for (uint32_t i = 0; i < per; ++i) {
-    const uint32_t s = s0 + i;
-    if (s >= 256) break;
-    const uint32_t f = freq[s];
-    tab[s] = make_uint2(f | (cum << 16), f ? 0xffffffffu / f : 0u);
-    cum += f;
+// Largest-remainder normalisation by one warp (the rule of block_normalize) of
+// hist[0 .. A), A <= 256, n symbols: writes freq[0 .. 256) and the coding table
+// tab[0 .. A) = {f | cum << 16, floor((2^32-1)/f)}; rem[0 .. A) is scratch.
+// Returns k. The d symbols that get one more are found by a radix select over
+// the keys 1 << 24 | r << 8 | (255 - s) of the present symbols (absent: 0).
+__device__ inline uint32_t warp_normalize(const uint32_t* hist, uint32_t A, uint32_t n, uint32_t* freq,
+                                          uint32_t* rem, uint2* tab) {
+  const uint32_t lane = threadIdx.x & 31u;
+  uint32_t present = 0;
+  for (uint32_t s = lane; s < A; s += 32u) present += hist[s] ? 1u : 0u;
+  const uint32_t k = __reduce_add_sync(0xffffffffu, present);
+  uint32_t fsum = 0;
+  for (uint32_t s = lane; s < 256u; s += 32u) {
+    const uint32_t c = s < A ? hist[s] : 0u;
+    uint32_t f = 0, r = 0;
+    if (k >= 2 && c) {
+      const uint32_t q = c * (kProbScale - k);
+      f = 1u + q / n;
+      r = q % n;
+    } else if (k == 1 && c) {
+      f = kProbScale;
+    }
+    if (s < A) rem[s] = c ? (1u << 24) | (r << 8) | (255u - s) : 0u;
+    freq[s] = f;
+    fsum += f;
   }
-  __syncthreads();
+  const uint32_t sum = __reduce_add_sync(0xffffffffu, fsum);
+  if (k >= 2 && sum < kProbScale) {
+    // P: the key bits fixed so far (bit 24, presence, is 1); need: the rank
+    // still sought among the keys that start with P
+    uint32_t P = 1, need = kProbScale - sum;
+    for (int bit = 23; bit >= 0; --bit) {
+      uint32_t cnt = 0;
+      for (uint32_t s0 = 0; s0 < A; s0 += 32u) {
+        const uint32_t s = s0 + lane;
+        const bool hit = s < A && (rem[s] >> bit) == ((P << 1) | 1u);
+        cnt += __popc(__ballot_sync(0xffffffffu, hit));
+      }
+      if (cnt >= need) P = (P << 1) | 1u;
+      else {
+        need -= cnt;
+        P <<= 1;
+      }
+    }
+    for (uint32_t s = lane; s < A; s += 32u)
+      if (rem[s] >= P) freq[s] += 1u;
+  }
+  __syncwarp();
+  uint32_t carry = 0;
+  for (uint32_t s0 = 0; s0 < A; s0 += 32u) {
+    const uint32_t s = s0 + lane;
+    const uint32_t f = s < A ? freq[s] : 0u;
+    uint32_t incl = f;
+#pragma unroll
+    for (uint32_t o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (s < A) tab[s] = make_uint2(f | ((carry + incl - f) << 16), f ? 0xffffffffu / f : 0u);
+    carry += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  __syncwarp();
+  return k;
 }
 
 // Decode table: lut[slot] = s | (slot - cum_s) << 8 | f_s << 20, and the

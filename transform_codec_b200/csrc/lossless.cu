@@ -310,9 +310,9 @@ k_lossless_decode(LosslessShape sh, FrameBatch b, uint8_t* ws) {
 //     Plane 1 and the deltas are counted by runs of equal high bytes along
 //     tokens: a delta is zero exactly while a run goes on, so the hot bins see
 //     one atomic per run instead of one per value;
-//  2. the three frequency tables;
+//  2. the three frequency tables, one warp each;
 //  3. each thread runs its lane's three rANS chains side by side, reading
-//     token rows that cp.async stages into a four-slot ring per warp;
+//     token rows that cp.async stages into a three-slot ring per warp;
 //  4. the smallest choice per plane, by the general encoder's rule;
 //  5. each thread assembles a contiguous run of the record's 16-byte units
 //     (prefix and states from shared memory, words from the scratch, a RAW
@@ -320,7 +320,7 @@ k_lossless_decode(LosslessShape sh, FrameBatch b, uint8_t* ws) {
 //     register; the registers are joined with powers of x.
 constexpr uint32_t kFencThreads = 128;
 constexpr uint32_t kFencStage = 16;                     // rANS steps per ring stage
-constexpr uint32_t kFencSlots = 4;                      // ring slots: 3 stages in flight
+constexpr uint32_t kFencSlots = 3;                      // ring slots: 2 stages in flight
 constexpr uint32_t kFencRowBytes = 64;                  // one token row of a warp's 32 lanes
 constexpr uint32_t kFencSlotBytes = kFencStage * kFencRowBytes;
 constexpr uint32_t kGroupWords = kGroupLanes * 512u;    // scratch words of one (variant, group)
@@ -329,17 +329,19 @@ constexpr uint32_t kRecArea = 2u * (16u + kMaxChunkValues);
 constexpr uint32_t kXRawPayload = gf2_xpow8(kMaxChunkValues);  // joins a RAW header to its payload
 
 struct __align__(16) FencSmem {
-  uint32_t crc_t[1024];
   uint32_t freq[3][256];
   uint2 tab[3][256];
   uint32_t states[3][kMaxLanes];
   union {
     struct {
       uint32_t hist[3][256];
-      uint32_t rem[256];
+      uint32_t rem[3][256];
     } h;                                                // phases 1-2
     uint8_t ring[kFencThreads / 32][kFencSlots][kFencSlotBytes];  // phase 3
-    uint4 tile[256];                                    // phase 5, RAW planes
+    struct {
+      uint32_t crc_t[1024];
+      uint4 tile[256];                                  // RAW planes
+    } a;                                                // phase 5
   } u;
   uint4 prefix[2][36];  // RANS record prefix: header, bitmap, frequencies, lengths (<= 576 B)
   uint32_t tmp[32], red[32];
@@ -378,7 +380,7 @@ __device__ __forceinline__ uint32_t lds_u16(const uint8_t* p) {
 }
 
 template <uint32_t D>
-__global__ void __launch_bounds__(kFencThreads, 6)
+__global__ void __launch_bounds__(kFencThreads, 8)
 k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
   constexpr uint32_t TCC = kMaxChunkValues / D, LPC = 128u / D;
   constexpr uint32_t CB = D / 8u;                       // 16-byte column blocks of a token row
@@ -394,7 +396,6 @@ k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
   const uint16_t* g = reinterpret_cast<const uint16_t*>(b.f[fr].src) + (uint64_t(slice) * sh.T + t0) * D;
   const uint4* g4 = reinterpret_cast<const uint4*>(g);
 
-  crc_tables_init(S.crc_t);
   for (uint32_t i = tid; i < 3u * 256u; i += kFencThreads) (&S.u.h.hist[0][0])[i] = 0;
   __syncthreads();
   {
@@ -446,10 +447,9 @@ k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
     if (zeros) atomicAdd(&S.u.h.hist[2][0], zeros);
   }
   __syncthreads();
-  for (uint32_t v = 0; v < 3; ++v) {
-    const uint32_t k = block_normalize(S.u.h.hist[v], n, S.freq[v], S.u.h.rem, S.tmp);
-    if (tid == 0) S.k[v] = k;
-    if (k >= 2) block_enc_tab(S.freq[v], S.tab[v], S.tmp);
+  if (warp < 3) {  // warp v: the table of variant v
+    const uint32_t k = warp_normalize(S.u.h.hist[warp], 256u, n, S.freq[warp], S.u.h.rem[warp], S.tab[warp]);
+    if (lane == 0) S.k[warp] = k;
   }
   __syncthreads();
   const bool en0 = S.k[0] >= 2, en1 = S.k[1] >= 2, en2 = en1 && S.k[2] >= 2;
@@ -483,14 +483,13 @@ k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
     constexpr uint32_t kStages = 512u / kFencStage;
     issue(kStages - 1);
     issue(kStages - 2);
-    issue(kStages - 3);
     uint32_t vcur = 0;
 #pragma unroll 1
     for (int s = int(kStages) - 1; s >= 0; --s) {
       __syncwarp();  // every lane is done with the slot the next copy overwrites
-      if (s >= 3) issue(uint32_t(s) - 3u);
+      if (s >= 2) issue(uint32_t(s) - 2u);
       else asm volatile("cp.async.commit_group;" ::: "memory");
-      asm volatile("cp.async.wait_group 2;" ::: "memory");  // stages s and s - 1 landed
+      asm volatile("cp.async.wait_group 1;" ::: "memory");  // stages s and s - 1 landed
       __syncwarp();
       const uint8_t* cur = ring + (uint32_t(s) % kFencSlots) * kFencSlotBytes + loff;
       const uint8_t* prv = ring + ((uint32_t(s) + kFencSlots - 1u) % kFencSlots) * kFencSlotBytes + loff;
@@ -559,7 +558,7 @@ k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
     }
   }
   for (uint32_t i = tid; i < 2u * 36u; i += kFencThreads) (&S.prefix[0][0])[i] = make_uint4(0, 0, 0, 0);
-  __syncthreads();
+  crc_tables_init(S.u.a.crc_t);  // synchronises
   // RANS prefixes: header, presence bitmap, frequencies of present symbols, sub-stream lengths
   for (uint32_t p = 0; p < 2; ++p) {
     if (S.mode[p] != kModeRans) continue;
@@ -591,7 +590,7 @@ k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
         uint4 h = make_uint4(kModeConst | (S.csym[p] << 8), 16u, n, 1u);
         *reinterpret_cast<uint4*>(out) = h;
         if (p == 0) h.x = ~h.x;
-        creg = crc_unit(S.crc_t, 0u, h);
+        creg = crc_unit(S.u.a.crc_t, 0u, h);
       }
     } else if (mode == kModeRaw) {
       // payload unit 1 + 32 t + i: 16 tokens (block i) of thread t's lane range,
@@ -602,21 +601,21 @@ k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
         uint4 h = make_uint4(kModeRaw, bytes, n, 0u);
         *reinterpret_cast<uint4*>(out) = h;
         if (p == 0) h.x = ~h.x;
-        hreg = crc_unit(S.crc_t, 0u, h);
+        hreg = crc_unit(S.u.a.crc_t, 0u, h);
       }
       auto tile_src = [&](uint32_t i, uint32_t m) -> const uint4* {
         return LPC == 1 ? g4 + (16u * i) * CB + m
                         : g4 + uint64_t((m >> 7) * 512u + 16u * i) * CB + (m & 127u);
       };
       uint4 nx0 = __ldcg(tile_src(0, tid)), nx1 = __ldcg(tile_src(0, tid + 128u));
-      const uint8_t* tb = reinterpret_cast<const uint8_t*>(S.u.tile) + p +
+      const uint8_t* tb = reinterpret_cast<const uint8_t*>(S.u.a.tile) + p +
                           (LPC == 1 ? 2u * tid : (tid & 1u) * 2048u + 2u * (tid >> 1));
       constexpr uint32_t RS = 2u * D;  // tile row stride
 #pragma unroll 1
       for (uint32_t i = 0; i < 32; ++i) {
         __syncthreads();
-        S.u.tile[tid] = nx0;
-        S.u.tile[tid + 128u] = nx1;
+        S.u.a.tile[tid] = nx0;
+        S.u.a.tile[tid + 128u] = nx1;
         __syncthreads();
         if (i + 1 < 32) {
           nx0 = __ldcg(tile_src(i + 1, tid));
@@ -629,7 +628,7 @@ k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
                  (uint32_t(tb[(4u * e + 2u) * RS]) << 16) | (uint32_t(tb[(4u * e + 3u) * RS]) << 24);
         const uint4 val = make_uint4(w[0], w[1], w[2], w[3]);
         *reinterpret_cast<uint4*>(out + 16u * (1u + 32u * tid + i)) = val;
-        creg = crc_unit(S.crc_t, creg, val);
+        creg = crc_unit(S.u.a.crc_t, creg, val);
       }
       creg = crc_join_lanes(creg, 32u, S.red);
       if (tid == 0) creg = gf2_mul(hreg, kXRawPayload) ^ creg;
@@ -667,7 +666,7 @@ k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
         }
         *reinterpret_cast<uint4*>(out + o) = val;
         if (p == 0 && u == 0) val.x = ~val.x;
-        creg = crc_unit(S.crc_t, creg, val);
+        creg = crc_unit(S.u.a.crc_t, creg, val);
       }
       creg = crc_join_lanes(creg, q, S.red);
     }

@@ -418,64 +418,6 @@ struct __align__(16) EntSmem {
   CompInfo ci;
 };
 
-// Largest-remainder normalisation of one width stream by one warp (the rule of
-// block_normalize): counts hist[0 .. A), A = 2^b, n symbols; writes freq[0 .. 256)
-// and the coding table tab of the first A symbols. Returns k.
-__device__ inline uint32_t warp_normalize(const uint32_t* hist, uint32_t A, uint32_t n, uint32_t* freq,
-                                          uint32_t* rem, uint2* tab) {
-  const uint32_t lane = threadIdx.x & 31u;
-  uint32_t present = 0;
-  for (uint32_t s = lane; s < A; s += 32u) present += hist[s] ? 1u : 0u;
-  const uint32_t k = __reduce_add_sync(0xffffffffu, present);
-  uint32_t fsum = 0;
-  for (uint32_t s = lane; s < 256u; s += 32u) {
-    const uint32_t c = s < A ? hist[s] : 0u;
-    uint32_t f = 0, r = 0;
-    if (k >= 2 && c) {
-      const uint32_t q = c * (kProbScale - k);
-      f = 1u + q / n;
-      r = q % n;
-    } else if (k == 1 && c) {
-      f = kProbScale;
-    }
-    if (s < A) rem[s] = r;
-    freq[s] = f;
-    fsum += f;
-  }
-  const uint32_t sum = __reduce_add_sync(0xffffffffu, fsum);
-  __syncwarp();
-  if (k >= 2 && sum < kProbScale) {
-    const uint32_t d = kProbScale - sum;
-    for (uint32_t s = lane; s < A; s += 32u) {
-      if (!hist[s]) continue;
-      const uint32_t r = rem[s];
-      uint32_t rank = 0;
-      for (uint32_t s2 = 0; s2 < A; ++s2) {
-        const uint32_t r2 = rem[s2];
-        rank += (hist[s2] != 0u) & ((r2 > r) | ((r2 == r) & (s2 < s)));
-      }
-      if (rank < d) freq[s] += 1u;
-    }
-  }
-  __syncwarp();
-  // coding tables: fc[s] = f | cum << 16, rcp[s] = floor((2^32 - 1) / f)
-  uint32_t carry = 0;
-  for (uint32_t s0 = 0; s0 < A; s0 += 32u) {
-    const uint32_t s = s0 + lane;
-    const uint32_t f = s < A ? freq[s] : 0u;
-    uint32_t incl = f;
-#pragma unroll
-    for (uint32_t o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    if (s < A) tab[s] = make_uint2(f | ((carry + incl - f) << 16), f ? 0xffffffffu / f : 0u);
-    carry += __shfl_sync(0xffffffffu, incl, 31);
-  }
-  __syncwarp();
-  return k;
-}
-
 __global__ void __launch_bounds__(kThreads)
 k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLayout ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
