@@ -389,7 +389,9 @@ EncodeLayout encode_layout(const kvc_plan_s* p, int path, uint64_t recs, void* w
 
 uint64_t decode_ws_for(const kvc_plan_s* p, int path, uint32_t frames, uint32_t max_slices) {
   const uint64_t f = std::min<uint32_t>(frames, kBatchMax);
-  return kDecodeWsFixed + pad256u(8ull * f * max_slices * records_per_slice(p, path));
+  const uint64_t recs = f * max_slices * records_per_slice(p, path);
+  return kDecodeWsFixed + pad256u(8ull * recs) +
+         (path == KVC_PATH_TRANSFORM ? transform_decode_ws_extra(p->ts, recs) : 0u);
 }
 
 bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
@@ -544,9 +546,12 @@ int decode_common(const kvc_plan_t* plan, int path, const void* d_src, size_t sr
                   cudaStream_t stream) {
   if (!path_ok(plan, path)) return plan ? KVC_ERR_UNSUPPORTED : KVC_ERR_INVALID;
   // the workspace bounds the slices a container may hold in this call
-  const uint64_t per_slice = 8ull * records_per_slice(plan, path);
-  const uint64_t room = ws_bytes > kDecodeWsFixed ? (ws_bytes - kDecodeWsFixed) / per_slice : 0;
-  const uint32_t ms = uint32_t(std::min<uint64_t>(room, plan->S));
+  uint32_t ms = plan->S;
+  while (ms > 0 && decode_ws_for(plan, path, 1, ms) > ws_bytes) {
+    const uint64_t per = std::max<uint64_t>(1u, (decode_ws_for(plan, path, 1, ms) - ws_bytes) /
+                                                    (decode_ws_for(plan, path, 1, 1) - kDecodeWsFixed));
+    ms = per >= ms ? 0u : ms - uint32_t(per);
+  }
   if (ms == 0) return KVC_ERR_CAPACITY;
   kvc_frame f{0, 0, d_src, src_bytes, d_dst, dst_cap, d_res};
   return decode_frames(plan, path, &f, 1, ms, d_ws, ws_bytes, stream);

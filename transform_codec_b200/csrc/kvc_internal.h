@@ -151,6 +151,9 @@ constexpr uint32_t kQSplitBytes = 2u * 128u * 256u;  // per slice
 uint64_t transform_slot_bytes(const TransformShape& s);
 cudaError_t launch_transform_encode(const TransformShape& s, const TransformPlanDev& p,
                                     const FrameBatch& b, const EncodeLayout& ws, cudaStream_t st);
+// Transform decode workspace beyond the common part, for `records` records:
+// a status word and a code block of ct rows of 128 bytes per record.
+uint64_t transform_decode_ws_extra(const TransformShape& s, uint64_t records);
 cudaError_t launch_transform_decode(const TransformShape& s, const TransformPlanDev& p,
                                     const FrameBatch& b, uint8_t* ws, uint32_t max_records,
                                     cudaStream_t st);

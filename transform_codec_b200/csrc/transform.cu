@@ -576,42 +576,56 @@ k_transform_encode_raw(TransformShape sh, FrameBatch b, EncodeLayout ws) {
   }
 }
 
-// Decoder shared memory. The first 128 KiB hold, in turn, the entropy stage's
-// decode tables and refill rings and then the tensor-core operand tiles
-// (each 128-byte-swizzled tile on a 1024-byte boundary).
-constexpr uint32_t kDecLuts = 6;  // rANS streams decoded side by side per round
-struct __align__(1024) DecSmem {
-  union {
-    struct {
-      uint8_t a_hi[kTcRows * 256];  // y^ as bf16 pieces, A operand [token][component]
-      uint8_t a_lo[kTcRows * 256];
-      uint8_t b_hi[kD * 256];       // Q as bf16 pieces, B operand [channel][component]
-      uint8_t b_lo[kD * 256];
-    } tc;
-    struct {
-      uint32_t lut[kDecLuts][kProbScale];
-      uint16_t ring[kThreads / 32][1024];  // one refill window per warp
-    } ent;
-  } u;
-  uint8_t codes[kMaxCt * kCodesStride];  // codes[t * 132 + j]
-  float zs[kD][kMaxCt / kTile][2];
+// ---------------------------------------------------------------------------
+// Transform decoder, in two stages.
+//
+// Entropy stage (k_transform_decode_codes): one block of 8 warps per record,
+// three blocks per SM. A raw record is copied to its rows. A middle record is
+// checked (CRC, stream walk, stream headers, side information length) and its
+// codes are decoded into the record's code block in the workspace,
+// codes[t * 128 + j] for token t of the chunk and component j; the record's
+// status word tells the tensor stage whether to use the block. A width
+// stream's decode table is one byte per slot (its symbol) and f << 16 | cum
+// per symbol: 5 KiB instead of a word per slot, so the tables of all eight
+// streams of a record and the warps' refill rings fit a third of an SM.
+//
+// Tensor stage (k_transform_decode): dequantisation, the inverse projection
+// on the tensor cores and the RoPE epilogue of every middle record whose
+// status is OK, reading its code block.
+constexpr uint32_t kCodeRow = kD;  // bytes of a code block's token row
+
+struct CodeBlocks {
+  uint32_t* status;  // per record of the batch: kOk when the code block is complete
+  uint8_t* codes;    // per record of the batch: ct token rows of kCodeRow bytes
+};
+__device__ inline CodeBlocks code_blocks(uint8_t* ws, uint32_t max_records) {
+  uint8_t* p = ws + kDecodeWsFixed + ((8ull * max_records + 255u) & ~255ull);
+  CodeBlocks c;
+  c.status = reinterpret_cast<uint32_t*>(p);
+  c.codes = p + ((4ull * max_records + 255u) & ~255ull);
+  return c;
+}
+
+struct __align__(16) DecEntSmem {
+  uint8_t lut[8][kProbScale];          // per width stream: symbol of each slot
+  uint16_t ring[kThreads / 32][1024];  // one refill window per warp
   uint32_t crc_t[1024];
-  uint32_t freq[8][256];                 // per width stream; then f << 16 | cum for the tables
+  uint32_t freq[8][256];               // per width stream; f << 16 | cum after the table build
   uint32_t tmp[32], red[32];
   StreamInfo si[8];
-  uint32_t str_off[8];                   // stream record offsets within the record, by width - 1
+  uint32_t str_off[8];                 // stream record offsets within the record, by width - 1
   CompInfo ci;
-  uint64_t bar;
   uint32_t base[kBatchMax + 1];
-  uint32_t tmem_base;
   uint32_t crc_ok, bad, walk_ok;
 };
 
-// Decode table of one rANS stream built by one warp: freq[256] (validated,
-// sum 4096) becomes freq[s] = f_s << 16 | cum_s, and lut[slot] = s | (slot -
-// cum_s) << 8 | f_s << 20 with the marks-and-running-maximum fill of
-// block_dec_lut.
-__device__ inline void warp_dec_lut(uint32_t* freq, uint32_t* lut) {
+// Decode table of one rANS stream built by one warp: freq[256] (validated, sum
+// 4096) becomes freq[s] = f_s << 16 | cum_s, and lut[slot] the symbol whose
+// range [cum_s, cum_s + f_s) holds slot: each present symbol's first slot is
+// marked with the symbol, and a running maximum over the slots (unmarked slots
+// are 0, which before the first mark is symbol 0's range) fills the rest,
+// four slots per lane and step.
+__device__ inline void warp_dec_lut8(uint32_t* freq, uint8_t* lut) {
   const uint32_t lane = threadIdx.x & 31u;
   uint32_t f[8], mine = 0;
 #pragma unroll
@@ -626,49 +640,53 @@ __device__ inline void warp_dec_lut(uint32_t* freq, uint32_t* lut) {
     if (lane >= o) incl += y;
   }
   uint32_t cum = incl - mine;
-  for (uint32_t i = lane; i < kProbScale / 4u; i += 32u) reinterpret_cast<uint4*>(lut)[i] = make_uint4(0, 0, 0, 0);
+  uint32_t* lut32 = reinterpret_cast<uint32_t*>(lut);
+  for (uint32_t i = lane; i < kProbScale / 16u; i += 32u) reinterpret_cast<uint4*>(lut)[i] = make_uint4(0, 0, 0, 0);
   __syncwarp();
 #pragma unroll
   for (uint32_t i = 0; i < 8; ++i) {
     const uint32_t s = 8u * lane + i;
-    if (f[i]) lut[cum] = s + 1u;
+    if (f[i]) lut[cum] = uint8_t(s);
     freq[s] = (f[i] << 16) | cum;
     cum += f[i];
   }
   __syncwarp();
   uint32_t carry = 0;
-#pragma unroll 4
-  for (uint32_t b0 = 0; b0 < kProbScale; b0 += 32u) {
-    const uint32_t slot = b0 + lane;
-    uint32_t m = lut[slot];
+#pragma unroll 2
+  for (uint32_t w0 = 0; w0 < kProbScale / 4u; w0 += 32u) {
+    const uint32_t w = lut32[w0 + lane];
+    const uint32_t m0 = w & 0xffu, m1 = max(m0, (w >> 8) & 0xffu);
+    const uint32_t m2 = max(m1, (w >> 16) & 0xffu), m3 = max(m2, w >> 24);
+    uint32_t x = m3;
 #pragma unroll
     for (uint32_t o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, m, o);
-      if (lane >= o) m = max(m, y);
+      const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x = max(x, y);
     }
-    m = max(m, carry);
-    carry = __shfl_sync(0xffffffffu, m, 31);
-    const uint32_t sym = m - 1u, e = freq[sym];
-    lut[slot] = sym | ((slot - (e & 0xffffu)) << 8) | ((e >> 16) << 20);
+    uint32_t before = __shfl_up_sync(0xffffffffu, x, 1);
+    before = max(lane ? before : 0u, carry);
+    lut32[w0 + lane] = max(m0, before) | (max(m1, before) << 8) | (max(m2, before) << 16) | (max(m3, before) << 24);
+    carry = max(carry, __shfl_sync(0xffffffffu, x, 31));
   }
   __syncwarp();
 }
 
 // rANS decode of group g of one width stream by one warp: n symbols on N
-// lanes; symbol i = a * tcc + t is written to codes[t * 132 + comp[a]] (m
-// components). The sub-stream (sl bytes at sub, 16-byte aligned) holds the
-// lanes' states, then the refill words. Its 16-byte units, from the one
-// holding the first word on, are copied by cp.async into a 1024-entry ring of
-// 16-bit positions counted from the sub-stream's start (the words begin at
-// position 2 * lanes_g), so no more than the ring's 128 units are requested
-// at once: at every stage of 8 steps (at most 256 words consumed) the warp waits for all but the
-// newest copy group and requests units up to 1024 positions past the unit
-// holding the next word, so no unit is overwritten before it is consumed and
-// the coming stage's words were requested a stage earlier. Returns false (on
-// every lane) when a symbol exceeds levels, a lane reads past its sub-stream
-// or the final states and word count do not match.
+// lanes; symbol i = a * tcc + t is written to codes[t * 128 + comp[a]] (m
+// components, codes in global memory). The sub-stream (sl bytes at sub,
+// 16-byte aligned) holds the lanes' states, then the refill words. Its 16-byte
+// units, from the one holding the first word on, are copied by cp.async into
+// a 1024-entry ring of 16-bit positions counted from the sub-stream's start
+// (the words begin at position 2 * lanes_g), so no more than the ring's 128
+// units are requested at once: at every stage of 8 steps (at most 256 words
+// consumed) the warp waits for all but the newest copy group and requests
+// units up to 1024 positions past the unit holding the next word, so no unit
+// is overwritten before it is consumed and the coming stage's words were
+// requested a stage earlier. Returns false (on every lane) when a symbol
+// exceeds levels, a lane reads past its sub-stream or the final states and
+// word count do not match.
 __device__ inline bool decode_codes_group(const uint8_t* sub, uint32_t sl, uint32_t n, uint32_t N, uint32_t g,
-                                          const uint32_t* lut, uint16_t* ring, uint8_t* codes,
+                                          const uint8_t* lut, const uint32_t* fc, uint16_t* ring, uint8_t* codes,
                                           const uint32_t* comp, uint32_t m, uint32_t tcc, uint32_t levels) {
   const uint32_t lane = threadIdx.x & 31u;
   const uint32_t lanes_g = min(kGroupLanes, N - g * kGroupLanes);
@@ -682,10 +700,9 @@ __device__ inline bool decode_codes_group(const uint8_t* sub, uint32_t sl, uint3
   uint32_t x = live ? reinterpret_cast<const uint32_t*>(sub)[lane] : kRansLow;
   uint32_t a = start / tcc, t = start - a * tcc;
   uint32_t j = (live && len && a < m) ? comp[a] : 0u;
-  const uint32_t codes_saddr = static_cast<uint32_t>(__cvta_generic_to_shared(codes));
-  uint32_t cp = codes_saddr + t * kCodesStride + j;  // shared address of this lane's next code
-  uint32_t left = tcc - t;                            // steps until the lane moves to the next component
-  uint32_t rp = w0, orv = 0;                          // ring position of the next word; OR of the entries
+  uint8_t* cp = codes + uint64_t(t) * kCodeRow + j;  // this lane's next code
+  uint32_t left = tcc - t;                          // steps until the lane moves to the next component
+  uint32_t rp = w0, orv = 0;                        // ring position of the next word; OR of the symbols
   const uint32_t n_units = (sl + 15u) >> 4, ring_saddr = static_cast<uint32_t>(__cvta_generic_to_shared(ring));
   uint32_t loaded = w0 >> 3;  // units wholly inside the states are never needed (and would alias live slots)
   auto request = [&]() {
@@ -707,14 +724,16 @@ __device__ inline bool decode_codes_group(const uint8_t* sub, uint32_t sl, uint3
     for (uint32_t k = 0; k < 8; ++k) {
       const bool act = live && tau0 + k < len;
       if (act) {
-        const uint32_t e = lut[x & (kProbScale - 1u)];
-        x = (e >> 20) * (x >> kProbBits) + ((e >> 8) & 0xfffu);
-        orv |= e;
-        asm volatile("st.shared.u8 [%0], %1;" ::"r"(cp), "r"(e) : "memory");
-        cp += kCodesStride;
+        const uint32_t slot = x & (kProbScale - 1u);
+        const uint32_t sym = lut[slot];
+        const uint32_t e = fc[sym];
+        x = (e >> 16) * (x >> kProbBits) + slot - (e & 0xffffu);
+        orv |= sym;
+        *cp = uint8_t(sym);
+        cp += kCodeRow;
         if (--left == 0u) {
           ++a;
-          cp = codes_saddr + (a < m ? comp[a] : 0u);
+          cp = codes + (a < m ? comp[a] : 0u);
           left = tcc;
         }
       }
@@ -725,23 +744,20 @@ __device__ inline bool decode_codes_group(const uint8_t* sub, uint32_t sl, uint3
       rp += __popc(mask);
     }
   }
-  const uint32_t pos = rp - w0, bad = (orv & 0xffu & ~levels) != 0u;
+  const uint32_t pos = rp - w0, bad = (orv & ~levels) != 0u;
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncwarp();
   const bool ok = !bad && pos == W && x == kRansLow;
   return __all_sync(0xffffffffu, ok);
 }
 
-static_assert(sizeof(DecSmem) + 1024 <= 232448, "decoder shared memory exceeds the per-block limit");
-static_assert(sizeof(ProjSmem) <= 232448, "projection shared memory exceeds the per-block limit");
-static_assert(sizeof(EntSmem) <= 232448 / 2, "entropy kernel should fit two blocks per SM");
+static_assert(sizeof(DecEntSmem) <= 232448 / 3, "entropy stage should fit three blocks per SM");
 
-__global__ void __launch_bounds__(kThreads)
-k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t* ws) {
+__global__ void __launch_bounds__(kThreads, 3)
+k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t* ws,
+                         uint32_t max_records) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  // the swizzled operand tiles need 1024-byte-aligned shared addresses
-  const uint32_t pad = (1024u - (tc::smem_addr(smem_raw) & 1023u)) & 1023u;
-  DecSmem& S = *reinterpret_cast<DecSmem*>(smem_raw + pad);
+  DecEntSmem& S = *reinterpret_cast<DecEntSmem*>(smem_raw);
   const uint32_t tid = threadIdx.x, nthr = blockDim.x;
   const uint32_t warp = tid >> 5, lane = tid & 31u;
   if (tid == 0) {  // records of the batch: prefix over frames that passed the header check
@@ -755,43 +771,28 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
   }
   __syncthreads();
   const uint32_t nrec = S.base[b.n];
-  const uint32_t per = (nrec + gridDim.x - 1) / gridDim.x;
-  const uint32_t rbeg = blockIdx.x * per, rend = min(nrec, rbeg + per);
-  if (rbeg >= rend) return;
+  if (blockIdx.x >= nrec) return;
+  const CodeBlocks cb = code_blocks(ws, max_records);
   crc_tables_init(S.crc_t);
-  if (warp == 0) {
-    tc::tmem_alloc(&S.tmem_base, kTcCols);
-    tc::tmem_relinquish();
-  }
-  if (tid == 0) tc::mbar_init(&S.bar, 1);
-  tc::fence_before_sync();
-  __syncthreads();
-  tc::fence_after_sync();
-  const uint32_t tmem = S.tmem_base;
-  uint32_t phase = 0;
-  bool alive = true;
   const uint32_t rps = 1u + sh.n_mid;
-  constexpr uint32_t idesc = tc::idesc_bf16_f32(kTcRows, kD);
-  for (uint32_t g = rbeg; g < rend && alive; ++g) {
+  for (uint32_t g = blockIdx.x; g < nrec; g += gridDim.x) {
     __syncthreads();
     const uint32_t fr = frame_of(S.base, b.n, g), r = g - S.base[fr];
     const uint8_t* src = b.f[fr].src;
     uint16_t* dst = reinterpret_cast<uint16_t*>(b.f[fr].dst);
     DecodeState* ds = decode_state(ws, fr);
-    const uint32_t first = ds->first_slice;
     const uint8_t* e = src + kHeaderBytes + uint64_t(kIndexEntry) * r;
     const uint64_t off0 = ld_u64(e);
     const uint32_t len = ld_u32(e + 8), want = ld_u32(e + 12);
     const uint8_t* rec = src + off0;
     const uint32_t ls = r / rps, kind = r % rps;
-    const uint32_t sidx = first + ls;
-    const bool is_key = ((sidx / sh.H) & 1u) == 0;
-    uint16_t* xs = dst + uint64_t(ls) * sh.T * kD;
+    const uint32_t sidx = ds->first_slice + ls;
     uint32_t got = crc32_block_aligned(rec, len, S.crc_t, S.red);
     if (tid == 0) S.crc_ok = (got == want);
     __syncthreads();
     int st = S.crc_ok ? kOk : kErrCorrupt;
     if (kind == 0) {
+      uint16_t* xs = dst + uint64_t(ls) * sh.T * kD;
       const uint32_t n_rows = sh.s_end + (sh.T - sh.r_start);
       if (st == kOk && len != pad16(n_rows * kD * 2u)) st = kErrCorrupt;
       if (st != kOk) {
@@ -835,16 +836,13 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
       st = block_parse_stream(rec + o, len - o, m * tcc, &S.si[bw - 1], S.freq[bw - 1], S.tmp, false);
     }
     if (st != kOk) {
-      if (tid == 0) atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(st));
+      if (tid == 0) {
+        atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(st));
+        cb.status[g] = uint32_t(st);
+      }
       continue;
     }
-    if (tid < kD && S.ci.width[tid]) {
-      const uint32_t* p32 = reinterpret_cast<const uint32_t*>(rec + 8u * S.ci.coded_idx[tid] * nb);
-      for (uint32_t blk = 0; blk < nb; ++blk) {
-        S.zs[tid][blk][0] = __uint_as_float(p32[2 * blk]);
-        S.zs[tid][blk][1] = __uint_as_float(p32[2 * blk + 1]);
-      }
-    }
+    uint8_t* codes = cb.codes + uint64_t(g) * sh.ct * kCodeRow;
     // RAW and CONST streams: every thread writes codes
     {
       const Split split(tcc);
@@ -861,46 +859,127 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
           split(i, a, t);
           const uint32_t sy = mode == kModeRaw ? uint32_t(raw[i]) : csym;
           bad |= uint32_t(sy > levels);
-          S.codes[t * kCodesStride + S.ci.comp[base + a]] = uint8_t(sy);
+          codes[t * kCodeRow + S.ci.comp[base + a]] = uint8_t(sy);
         }
         if (bad) S.bad = 1;
       }
     }
-    // rANS streams, up to kDecLuts at a time: one warp builds each table, then
-    // one warp per (stream, group) decodes
-    for (uint32_t bw0 = 1; bw0 <= 8;) {
-      uint32_t sel[kDecLuts], ns = 0, bw = bw0;
-      for (; bw <= 8 && ns < kDecLuts; ++bw)
-        if (S.ci.bcount[bw] && S.si[bw - 1].mode == kModeRans) sel[ns++] = bw;
-      bw0 = bw;
-      if (!ns) break;
-      if (warp < ns) warp_dec_lut(S.freq[sel[warp] - 1], S.u.ent.lut[warp]);
-      __syncthreads();
+    // rANS streams: warp w builds the table of width w + 1, then one warp per
+    // (stream, group) decodes
+    if (S.ci.bcount[warp + 1] && S.si[warp].mode == kModeRans) warp_dec_lut8(S.freq[warp], S.lut[warp]);
+    __syncthreads();
+    {
       uint32_t pair = 0;
-      for (uint32_t q = 0; q < ns; ++q) {
-        const uint32_t sw = sel[q], m = S.ci.bcount[sw], n = m * tcc;
-        const uint32_t N = rans_lanes(n), G = rans_groups(N);
+      for (uint32_t sw = 1; sw <= 8; ++sw) {
+        const uint32_t m = S.ci.bcount[sw];
+        if (!m || S.si[sw - 1].mode != kModeRans) continue;
+        const uint32_t n = m * tcc, N = rans_lanes(n), G = rans_groups(N);
         const StreamInfo& si = S.si[sw - 1];
         for (uint32_t gg = 0; gg < G; ++gg, ++pair) {
           if (pair % (nthr >> 5) != warp) continue;
           const bool ok = decode_codes_group(rec + S.str_off[sw - 1] + si.sub_off[gg], si.sub_len[gg], n, N, gg,
-                                             S.u.ent.lut[q], S.u.ent.ring[warp], S.codes,
+                                             S.lut[sw - 1], S.freq[sw - 1], S.ring[warp], codes,
                                              S.ci.comp + S.ci.bstart[sw], m, tcc, (1u << sw) - 1u);
           if (!ok && lane == 0) S.bad = 1;
         }
       }
-      __syncthreads();
     }
-    __syncthreads();  // every stream's codes and flags are in
-    if (S.bad) {
-      if (tid == 0) atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(kErrCorrupt));
-      continue;
+    __syncthreads();
+    if (tid == 0) {
+      if (S.bad) atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(kErrCorrupt));
+      cb.status[g] = S.bad ? uint32_t(kErrCorrupt) : uint32_t(kOk);
     }
-    // the B operand (Q as bf16 pieces) of this slice over the entropy stage's space
-    {
+  }
+}
+
+// Tensor stage shared memory: the operand tiles (each 128-byte-swizzled tile
+// on a 1024-byte boundary), the record's scales and zero points.
+struct __align__(1024) DecSmem {
+  struct {
+    uint8_t a_hi[kTcRows * 256];  // y^ as bf16 pieces, A operand [token][component]
+    uint8_t a_lo[kTcRows * 256];
+    uint8_t b_hi[kD * 256];       // Q as bf16 pieces, B operand [channel][component]
+    uint8_t b_lo[kD * 256];
+  } tc;
+  float zs[kD][kMaxCt / kTile][2];
+  CompInfo ci;
+  uint64_t bar;
+  uint32_t base[kBatchMax + 1];
+  uint32_t tmem_base;
+};
+
+static_assert(sizeof(DecSmem) + 1024 <= 232448, "decoder shared memory exceeds the per-block limit");
+static_assert(sizeof(ProjSmem) <= 232448, "projection shared memory exceeds the per-block limit");
+static_assert(sizeof(EntSmem) <= 232448 / 2, "entropy kernel should fit two blocks per SM");
+
+__global__ void __launch_bounds__(kThreads)
+k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t* ws, uint32_t max_records) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  // the swizzled operand tiles need 1024-byte-aligned shared addresses
+  const uint32_t pad = (1024u - (tc::smem_addr(smem_raw) & 1023u)) & 1023u;
+  DecSmem& S = *reinterpret_cast<DecSmem*>(smem_raw + pad);
+  const uint32_t tid = threadIdx.x, nthr = blockDim.x;
+  const uint32_t warp = tid >> 5, lane = tid & 31u;
+  if (tid == 0) {  // records of the batch: prefix over frames that passed the header check
+    uint32_t acc = 0;
+    for (uint32_t f = 0; f < b.n; ++f) {
+      S.base[f] = acc;
+      const DecodeState* d = decode_state(ws, f);
+      acc += d->status == kOk ? d->n_records : 0u;
+    }
+    S.base[b.n] = acc;
+  }
+  __syncthreads();
+  const uint32_t nrec = S.base[b.n];
+  const uint32_t per = (nrec + gridDim.x - 1) / gridDim.x;
+  const uint32_t rbeg = blockIdx.x * per, rend = min(nrec, rbeg + per);
+  if (rbeg >= rend) return;
+  const CodeBlocks cb = code_blocks(ws, max_records);
+  if (warp == 0) {
+    tc::tmem_alloc(&S.tmem_base, kTcCols);
+    tc::tmem_relinquish();
+  }
+  if (tid == 0) tc::mbar_init(&S.bar, 1);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = S.tmem_base;
+  uint32_t phase = 0;
+  bool alive = true;
+  const uint32_t rps = 1u + sh.n_mid;
+  constexpr uint32_t idesc = tc::idesc_bf16_f32(kTcRows, kD);
+  uint32_t cur_sidx = 0xffffffffu;  // slice whose component order and Q pieces are loaded
+  for (uint32_t g = rbeg; g < rend && alive; ++g) {
+    const uint32_t fr = frame_of(S.base, b.n, g), r = g - S.base[fr];
+    const uint32_t ls = r / rps, kind = r % rps;
+    if (kind == 0 || cb.status[g] != uint32_t(kOk)) continue;  // raw record, or one the entropy stage refused
+    __syncthreads();
+    const uint8_t* src = b.f[fr].src;
+    uint16_t* dst = reinterpret_cast<uint16_t*>(b.f[fr].dst);
+    DecodeState* ds = decode_state(ws, fr);
+    const uint8_t* e = src + kHeaderBytes + uint64_t(kIndexEntry) * r;
+    const uint8_t* rec = src + ld_u64(e);
+    const uint32_t sidx = ds->first_slice + ls;
+    const bool is_key = ((sidx / sh.H) & 1u) == 0;
+    uint16_t* xs = dst + uint64_t(ls) * sh.T * kD;
+    const uint32_t c = kind - 1;
+    const uint32_t t0 = sh.s_end + c * sh.ct, tcc = min(sh.ct, sh.r_start - t0);
+    const uint32_t nb = (tcc + kTile - 1) / kTile;
+    const uint8_t* codes = cb.codes + uint64_t(g) * sh.ct * kCodeRow;
+    if (sidx != cur_sidx) {
+      load_comp_info(pl.comp + sidx, S.ci);
+      // the B operand: Q of this slice as bf16 pieces (b_hi and b_lo are contiguous)
       const uint4* q4 = reinterpret_cast<const uint4*>(pl.qsplit + uint64_t(sidx) * kQSplitBytes);
-      uint4* b4 = reinterpret_cast<uint4*>(S.u.tc.b_hi);  // b_hi and b_lo are contiguous
+      uint4* b4 = reinterpret_cast<uint4*>(S.tc.b_hi);
       for (uint32_t i = tid; i < kQSplitBytes / 16u; i += nthr) b4[i] = __ldg(q4 + i);
+      cur_sidx = sidx;
+    }
+    if (tid < kD && S.ci.width[tid]) {
+      const uint32_t* p32 = reinterpret_cast<const uint32_t*>(rec + 8u * S.ci.coded_idx[tid] * nb);
+      for (uint32_t blk = 0; blk < nb; ++blk) {
+        S.zs[tid][blk][0] = __uint_as_float(__ldg(&p32[2 * blk]));
+        S.zs[tid][blk][1] = __uint_as_float(__ldg(&p32[2 * blk + 1]));
+      }
     }
     // inverse projection on the tensor cores, 128 tokens at a time:
     // x^[t][k] = sum_j y^[t][j] Q[k][j] with y^ and Q split into bf16 hi + lo
@@ -916,8 +995,8 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
         for (uint32_t i = 0; i < 8; ++i) v[i] = 0.0f;
         if (tt < bl) {
           const uint32_t t = t_base + tt, blk = t / kTile;
-          const uint32_t* cw = reinterpret_cast<const uint32_t*>(&S.codes[t * kCodesStride + j0]);
-          const uint32_t c4[2] = {cw[0], cw[1]};
+          const uint2 cw = *reinterpret_cast<const uint2*>(codes + t * kCodeRow + j0);
+          const uint32_t c4[2] = {cw.x, cw.y};
 #pragma unroll
           for (uint32_t i = 0; i < 8; ++i) {
             const uint32_t j = j0 + i;
@@ -935,15 +1014,15 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
                              __fsub_rn(v[2 * i + 1], bf16_to_f32(h[i] >> 16)));
         }
         const uint32_t o = tc::sw128_offset(tt, 2u * j0, kTcRows);
-        *reinterpret_cast<uint4*>(S.u.tc.a_hi + o) = make_uint4(h[0], h[1], h[2], h[3]);
-        *reinterpret_cast<uint4*>(S.u.tc.a_lo + o) = make_uint4(l[0], l[1], l[2], l[3]);
+        *reinterpret_cast<uint4*>(S.tc.a_hi + o) = make_uint4(h[0], h[1], h[2], h[3]);
+        *reinterpret_cast<uint4*>(S.tc.a_lo + o) = make_uint4(l[0], l[1], l[2], l[3]);
       }
       tc::fence_async_smem();
       __syncthreads();
       if (tid == 0) {
         tc::fence_after_sync();
-        const uint32_t ah = tc::smem_addr(S.u.tc.a_hi), al = tc::smem_addr(S.u.tc.a_lo);
-        const uint32_t bh = tc::smem_addr(S.u.tc.b_hi), bo = tc::smem_addr(S.u.tc.b_lo);
+        const uint32_t ah = tc::smem_addr(S.tc.a_hi), al = tc::smem_addr(S.tc.a_lo);
+        const uint32_t bh = tc::smem_addr(S.tc.b_hi), bo = tc::smem_addr(S.tc.b_lo);
         uint32_t acc = 0;
         for (uint32_t ks = 0; ks < kD / 16u; ++ks) {  // K = 16 components per MMA
           const uint32_t koff = (ks >> 2) * (kTcRows * 128u) + (ks & 3u) * 32u;
@@ -1080,15 +1159,35 @@ cudaError_t launch_transform_decode(const TransformShape& s, const TransformPlan
                                     const FrameBatch& b, uint8_t* ws, uint32_t max_records,
                                     cudaStream_t st) {
   if (max_records == 0 || b.n == 0) return cudaSuccess;
-  size_t smem = sizeof(DecSmem) + 1024;
-  cudaError_t e = cudaFuncSetAttribute(k_transform_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  static int ent_blocks_per_sm = 0;
+  const size_t esmem = sizeof(DecEntSmem);
+  cudaError_t e = cudaFuncSetAttribute(k_transform_decode_codes, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(esmem));
   if (e != cudaSuccess) return e;
-  uint32_t grid = min(max_records, uint32_t(num_sms()));
+  if (!ent_blocks_per_sm) {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ent_blocks_per_sm, k_transform_decode_codes, kThreads, esmem);
+    if (e != cudaSuccess || ent_blocks_per_sm < 1) ent_blocks_per_sm = 1;
+  }
+  {
+    ProfRange pr_("transform_decode_codes", st);
+    const uint32_t grid = min(max_records, uint32_t(num_sms() * ent_blocks_per_sm));
+    k_transform_decode_codes<<<grid, kThreads, esmem, st>>>(s, p, b, ws, max_records);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  size_t smem = sizeof(DecSmem) + 1024;
+  e = cudaFuncSetAttribute(k_transform_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
   {
     ProfRange pr_("transform_decode", st);
-    k_transform_decode<<<grid, kThreads, smem, st>>>(s, p, b, ws);
+    const uint32_t grid = min(max_records, uint32_t(num_sms()));
+    k_transform_decode<<<grid, kThreads, smem, st>>>(s, p, b, ws, max_records);
   }
   return cudaGetLastError();
+}
+
+uint64_t transform_decode_ws_extra(const TransformShape& s, uint64_t records) {
+  return ((4u * records + 255u) & ~uint64_t(255)) + records * uint64_t(s.ct) * kCodeRow;
 }
 
 }  // namespace kvc
