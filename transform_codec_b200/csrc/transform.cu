@@ -901,7 +901,9 @@ struct __align__(1024) DecSmem {
     uint8_t b_hi[kD * 256];       // Q as bf16 pieces, B operand [channel][component]
     uint8_t b_lo[kD * 256];
   } tc;
-  float zs[kD][kMaxCt / kTile][2];
+  // scale and zero point (s, z) of component j in block blk at zsT[j % 8][blk][j / 8]:
+  // the 16 threads that share a token read 16 consecutive entries
+  float2 zsT[8][kMaxCt / kTile][kD / 8];
   CompInfo ci;
   uint64_t bar;
   uint32_t base[kBatchMax + 1];
@@ -912,7 +914,7 @@ static_assert(sizeof(DecSmem) + 1024 <= 232448, "decoder shared memory exceeds t
 static_assert(sizeof(ProjSmem) <= 232448, "projection shared memory exceeds the per-block limit");
 static_assert(sizeof(EntSmem) <= 232448 / 2, "entropy kernel should fit two blocks per SM");
 
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 1)
 k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t* ws, uint32_t max_records) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   // the swizzled operand tiles need 1024-byte-aligned shared addresses
@@ -974,11 +976,16 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
       for (uint32_t i = tid; i < kQSplitBytes / 16u; i += nthr) b4[i] = __ldg(q4 + i);
       cur_sidx = sidx;
     }
+    // this thread's A-operand components j0 .. j0 + 7 and which of them are coded
+    const uint32_t j0 = 8u * (tid & 15u);
+    uint32_t wmask = 0;
+#pragma unroll
+    for (uint32_t i = 0; i < 8; ++i) wmask |= S.ci.width[j0 + i] ? (1u << i) : 0u;
     if (tid < kD && S.ci.width[tid]) {
       const uint32_t* p32 = reinterpret_cast<const uint32_t*>(rec + 8u * S.ci.coded_idx[tid] * nb);
       for (uint32_t blk = 0; blk < nb; ++blk) {
-        S.zs[tid][blk][0] = __uint_as_float(__ldg(&p32[2 * blk]));
-        S.zs[tid][blk][1] = __uint_as_float(__ldg(&p32[2 * blk + 1]));
+        S.zsT[tid & 7u][blk][tid >> 3] =
+            make_float2(__uint_as_float(__ldg(&p32[2 * blk])), __uint_as_float(__ldg(&p32[2 * blk + 1])));
       }
     }
     // inverse projection on the tensor cores, 128 tokens at a time:
@@ -987,23 +994,37 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
     for (uint32_t t_base = 0; t_base < tcc; t_base += kTcRows) {
       const uint32_t bl = min(kTcRows, tcc - t_base);
       __syncthreads();
-      // item: 8 consecutive components of one token -> one 16-byte chunk of each piece
-      for (uint32_t it = tid; it < kTcRows * (kD / 8u); it += nthr) {
-        const uint32_t tt = it >> 4, j0 = 8u * (it & 15u);
+      // item k of this thread: token tt = tid / 16 + 16 k, components j0 .. j0 + 7
+      // (the same for all its items) -> one 16-byte chunk of each piece. The
+      // codes are loaded first, so their latencies overlap; the scales and zero
+      // points of the tile's two blocks come from shared memory once.
+      constexpr uint32_t kItems = kTcRows * (kD / 8u) / kThreads;
+      static_assert(kItems == 8 && kTcRows == 2 * kTile, "item k lies in the tile's block k / 4");
+      uint2 cw8[kItems];
+#pragma unroll
+      for (uint32_t k = 0; k < kItems; ++k) {
+        const uint32_t tt = (tid >> 4) + 16u * k;
+        cw8[k] = tt < bl ? __ldcg(reinterpret_cast<const uint2*>(codes + (t_base + tt) * kCodeRow + j0))
+                         : make_uint2(0, 0);
+      }
+      float2 zr[2][8];
+#pragma unroll
+      for (uint32_t b2 = 0; b2 < 2; ++b2)
+#pragma unroll
+        for (uint32_t i = 0; i < 8; ++i) zr[b2][i] = S.zsT[i][t_base / kTile + b2][tid & 15u];
+#pragma unroll
+      for (uint32_t k = 0; k < kItems; ++k) {
+        const uint32_t tt = (tid >> 4) + 16u * k;
         float v[8];
 #pragma unroll
         for (uint32_t i = 0; i < 8; ++i) v[i] = 0.0f;
         if (tt < bl) {
-          const uint32_t t = t_base + tt, blk = t / kTile;
-          const uint2 cw = *reinterpret_cast<const uint2*>(codes + t * kCodeRow + j0);
-          const uint32_t c4[2] = {cw.x, cw.y};
+          const uint32_t c4[2] = {cw8[k].x, cw8[k].y};
 #pragma unroll
           for (uint32_t i = 0; i < 8; ++i) {
-            const uint32_t j = j0 + i;
-            if (S.ci.width[j]) {
-              const float2 zs = *reinterpret_cast<const float2*>(S.zs[j][blk]);
-              v[i] = __fmaf_rn(float((c4[i >> 2] >> (8u * (i & 3u))) & 0xffu), zs.y, zs.x);
-            }
+            const float2 zs = zr[k >> 2][i];
+            const float y = __fmaf_rn(float((c4[i >> 2] >> (8u * (i & 3u))) & 0xffu), zs.y, zs.x);
+            v[i] = (wmask >> i) & 1u ? y : 0.0f;
           }
         }
         uint32_t h[4], l[4];
