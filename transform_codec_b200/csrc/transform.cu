@@ -93,10 +93,11 @@ struct Split {  // i -> (component slot, token) for i = slot * tcc + t
 // the symbol counts of every width stream are gathered behind them for the
 // entropy kernel.
 constexpr uint32_t kProjTokens = 64;   // tokens per projection tile = quantiser block
-constexpr uint32_t kCodesRow = 128;    // bytes per token row of the code array in the slot
-constexpr uint32_t kCodesStride = 132; // shared code row: 128 bytes + 4 bytes of padding
+constexpr uint32_t kCodesRow = kMaxCt;  // bytes per component row of the code array in the slot
 constexpr uint32_t kTabPool = 512;     // sum over widths 1..8 of 2^b, rounded up
-constexpr uint32_t kHistOffset = kCodesRow * kMaxCt;  // counts follow the codes in the slot
+constexpr uint32_t kHistOffset = kCodesRow * kD;      // counts follow the codes in the slot
+constexpr uint32_t kCodesArea = kHistOffset + 4u * kTabPool;
+constexpr uint32_t kWordsArea = 2u * kD * kMaxCt + 64u;  // rANS word scratch: a word per symbol
 constexpr uint32_t kYStride = kD + 1u;                 // y[t][c] row stride in floats (odd: conflict-free)
 
 __device__ inline uint32_t tab_base(uint32_t b) { return (1u << b) - 2u; }  // 2 + 4 + ... + 2^(b-1)
@@ -104,7 +105,6 @@ __device__ inline uint32_t tab_base(uint32_t b) { return (1u << b) - 2u; }  // 2
 struct __align__(16) ProjSmem {
   double Qd[kD * kD];                          // Q[k][c], coded components c < n_coded, fp64
   double x[kD * kProjTokens];                  // x[k][t]; then y[c][t] as fp32 in the same space
-  uint8_t codes[kProjTokens * kCodesStride];   // this tile's codes, codes[t * 132 + j]
   uint32_t hist[kTabPool];                     // symbol counts of the record per width stream
   float2 mm[2][kD];                            // per coded component: the two half-blocks' min and max
   uint32_t ccnt[8][kD];                        // counts of symbols 0..7 per coded component
@@ -112,8 +112,12 @@ struct __align__(16) ProjSmem {
   uint32_t cidx[kD];                           // coded component c -> channel-space index j
 };
 
-__device__ inline uint8_t* slot_codes(uint8_t* slot, uint64_t slot_bytes) {
-  return slot + slot_bytes - (2u * kD * kMaxCt + 64u);
+// The tail of a middle record's slot: the rANS word scratch, then the code
+// array (component-major: codes[j * kCodesRow + t] for component j, token t)
+// and the symbol counts per width stream.
+__device__ inline uint8_t* slot_codes(uint8_t* slot, uint64_t slot_bytes) { return slot + slot_bytes - kCodesArea; }
+__device__ inline uint16_t* slot_words(uint8_t* slot, uint64_t slot_bytes) {
+  return reinterpret_cast<uint16_t*>(slot + slot_bytes - kCodesArea - kWordsArea);
 }
 
 // One thread's share of a tile's inputs: items (token tt, 8-channel group q)
@@ -352,11 +356,14 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
 #pragma unroll
           for (uint32_t u = 0; u < 8; ++u) qv[u] = u == i ? qi : qv[u];
         }
+        // the 8 codes (past n: zeros) go to the component's row in one store
+        *reinterpret_cast<uint2*>(codes + uint64_t(j) * kCodesRow + tb + lo + t8) =
+            make_uint2(qv[0] | (qv[1] << 8) | (qv[2] << 16) | (qv[3] << 24),
+                       qv[4] | (qv[5] << 8) | (qv[6] << 16) | (qv[7] << 24));
 #pragma unroll
         for (uint32_t i = 0; i < 8; ++i) {
           if (t8 + i < n) {
             const uint32_t q = qv[i];
-            S.codes[(lo + t8 + i) * kCodesStride + j] = uint8_t(q);
             if (q < 8u) {
               const uint32_t inc = 1u << (8u * (q & 3u));
               if (q < 4u) cnt_lo += inc; else cnt_hi += inc;
@@ -371,13 +378,6 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
         const uint32_t c = ((q < 4u ? cnt_lo : cnt_hi) >> (8u * (q & 3u))) & 0xffu;
         if (c) atomicAdd(&S.ccnt[q][cc], c);
       }
-    }
-    __syncthreads();
-    // the tile's code rows to the slot (uncoded channels carry whatever was staged)
-    for (uint32_t i = tid; i < bl * (kCodesRow / 4u); i += nthr) {
-      const uint32_t t = i >> 5, q = i & 31u;
-      reinterpret_cast<uint32_t*>(codes + uint64_t(tb + t) * kCodesRow)[q] =
-          *reinterpret_cast<const uint32_t*>(&S.codes[t * kCodesStride + 4u * q]);
     }
     __syncthreads();
   }
@@ -397,16 +397,16 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
 }
 
 // ---------------------------------------------------------------------------
-// Transform encode, part 2 (k_transform_entropy): one CTA per middle record.
-// The codes come back from the slot into shared rows of 132 bytes (conflict-
-// free both along a row and down a column). Warp w owns the stream of width
-// b = w + 1: it counts the stream's symbols (ballots for alphabets up to 32,
-// shared atomics above), normalises the counts and builds its coding tables.
+// Transform encode, part 2 (k_transform_entropy): one CTA per middle record,
+// several per SM (no codes in shared memory). Warp w owns the stream of width
+// b = w + 1: it normalises the stream's counts and builds its coding tables.
 // The rANS groups of all streams then run side by side, one warp per (stream,
-// group), and the record is laid out and written stream by stream.
+// group), reading the codes from the slot: in a full chunk every lane is one
+// component, whose 512 codes are one row, read 16 at a time into registers;
+// otherwise symbol by symbol. The record is then laid out and written stream
+// by stream.
 
 struct __align__(16) EntSmem {
-  uint8_t codes[kMaxCt * kCodesStride];  // codes[t * 132 + j]
   uint32_t freq[8][256];                 // per width stream, zero past its alphabet
   uint2 tab[kTabPool];                   // per symbol of each width stream: {f | cum << 16, 1/f}
   uint32_t rem[kTabPool], hist[kTabPool];
@@ -418,7 +418,45 @@ struct __align__(16) EntSmem {
   CompInfo ci;
 };
 
-__global__ void __launch_bounds__(kThreads)
+// rANS encode of one group (warp-synchronous) of a stream in which lane l
+// (live lanes only) codes the 512 symbols row[0 .. 512) of its own row, last
+// symbol first. The row is read as 16-byte vectors, two ahead of use. Words go
+// to words[.. cap), filled downwards; returns their count and the final state.
+__device__ inline uint32_t rans_encode_rows(const uint8_t* row, bool live, const uint2* tab, uint16_t* words,
+                                            uint32_t cap, uint32_t* x_out) {
+  const uint32_t lt = lanemask_lt();
+  const uint4* r4 = reinterpret_cast<const uint4*>(row);
+  const uint4 z4 = make_uint4(0, 0, 0, 0);
+  uint4 cur = live ? __ldcg(r4 + 31) : z4, nxt = live ? __ldcg(r4 + 30) : z4;
+  uint32_t x = kRansLow, pos = cap;
+#pragma unroll 1
+  for (int c = 31; c >= 0; --c) {
+    const uint4 nn = (live && c >= 2) ? __ldcg(r4 + (c - 2)) : z4;
+    const uint32_t w[4] = {cur.x, cur.y, cur.z, cur.w};
+#pragma unroll
+    for (int i = 15; i >= 0; --i) {
+      const uint2 e = tab[(w[i >> 2] >> (8 * (i & 3))) & 0xffu];
+      const uint32_t f = e.x & 0xffffu, cum = e.x >> 16;
+      const bool emit = live && x >= (f << 20);
+      const uint32_t mask = __ballot_sync(0xffffffffu, emit);
+      pos -= __popc(mask);
+      if (emit) words[pos + __popc(mask & lt)] = uint16_t(x & 0xffffu);
+      const uint32_t xe = emit ? (x >> 16) : x;
+      uint32_t q = __umulhi(xe, e.y);
+      uint32_t r = xe - q * f;
+      const bool over = r >= f;
+      q += over ? 1u : 0u;
+      r -= over ? f : 0u;
+      x = live ? (q << kProbBits) + r + cum : x;
+    }
+    cur = nxt;
+    nxt = nn;
+  }
+  *x_out = x;
+  return cap - pos;
+}
+
+__global__ void __launch_bounds__(kThreads, 3)
 k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLayout ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   EntSmem& S = *reinterpret_cast<EntSmem*>(smem_raw);
@@ -434,31 +472,13 @@ k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
   const uint32_t nb = (tcc + kTile - 1) / kTile;
   uint8_t* rec = ws.slots + uint64_t(r) * ws.slot_bytes;
   const uint8_t* codes_g = slot_codes(rec, ws.slot_bytes);
-  uint16_t* scratch = reinterpret_cast<uint16_t*>(rec + ws.slot_bytes - (2u * kD * kMaxCt + 64u));
+  uint16_t* scratch = slot_words(rec, ws.slot_bytes);
 
   crc_tables_init(S.crc_t);
   load_comp_info(pl.comp + sidx, S.ci);
-  {
-    // code rows: 8 vectors of 16 bytes per token, every thread's loads issued first
-    constexpr uint32_t kPer = kMaxCt * 8u / kThreads;
-    uint4 v[kPer];
-#pragma unroll
-    for (uint32_t u = 0; u < kPer; ++u) {
-      const uint32_t i = tid + u * nthr;
-      v[u] = (i >> 3) < tcc ? __ldcg(reinterpret_cast<const uint4*>(codes_g) + i) : make_uint4(0, 0, 0, 0);
-    }
-    for (uint32_t i = tid; i < kTabPool; i += nthr)
-      S.hist[i] = __ldcg(reinterpret_cast<const uint32_t*>(codes_g + kHistOffset) + i);
-#pragma unroll
-    for (uint32_t u = 0; u < kPer; ++u) {
-      const uint32_t i = tid + u * nthr, t = i >> 3, q = i & 7u;
-      if (t < tcc) {
-        uint32_t* d = reinterpret_cast<uint32_t*>(&S.codes[t * kCodesStride + 16u * q]);
-        d[0] = v[u].x; d[1] = v[u].y; d[2] = v[u].z; d[3] = v[u].w;
-      }
-    }
-  }
-  __syncthreads();  // codes and counts are in shared memory: the slot's scratch may now take words
+  for (uint32_t i = tid; i < kTabPool; i += nthr)
+    S.hist[i] = __ldcg(reinterpret_cast<const uint32_t*>(codes_g + kHistOffset) + i);
+  __syncthreads();
 
   const Split split(tcc);
   // ---- per-stream tables from the counts: warp w takes width b = w + 1
@@ -485,12 +505,17 @@ k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
         uint32_t b0, len0, b1 = n, len1;
         lane_range(n, N, g * kGroupLanes, b0, len0);
         if (g + 1 < G) lane_range(n, N, (g + 1) * kGroupLanes, b1, len1);
-        uint32_t x;
+        uint32_t x, Wg;
         const uint32_t* comp = S.ci.comp + base;
-        const uint8_t* codes = S.codes;
-        const uint32_t Wg = rans_encode_strided([comp, codes](uint32_t col) { return codes + comp[col]; },
-                                                kCodesStride, tcc, n, N, g, S.tab + tab_base(bw),
-                                                scratch + wbase + b0, b1 - b0, &x);
+        if (tcc == kMaxCt) {  // lane l: component l, all 512 tokens
+          const uint32_t l = g * kGroupLanes + lane;
+          const bool live = l < N;
+          Wg = rans_encode_rows(codes_g + uint64_t(live ? comp[l] : 0u) * kCodesRow, live, S.tab + tab_base(bw),
+                                scratch + wbase + b0, b1 - b0, &x);
+        } else {
+          Wg = rans_encode_strided([comp, codes_g](uint32_t col) { return codes_g + uint64_t(comp[col]) * kCodesRow; },
+                                   1u, tcc, n, N, g, S.tab + tab_base(bw), scratch + wbase + b0, b1 - b0, &x);
+        }
         if (g * kGroupLanes + lane < N) S.states[bw - 1][g * kGroupLanes + lane] = x;
         if (lane == 0) {
           S.W[bw - 1][g] = Wg;
@@ -530,7 +555,7 @@ k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
     auto sym = [&](uint32_t i) -> uint32_t {
       uint32_t a, t;
       split(i, a, t);
-      return S.codes[t * kCodesStride + S.ci.comp[base + a]];
+      return uint32_t(codes_g[uint64_t(S.ci.comp[base + a]) * kCodesRow + t]);
     };
     block_write_stream(rec + S.off[bw - 1], S.mode[bw - 1], n, S.bytes[bw - 1], sym(0), S.k[bw - 1],
                        S.freq[bw - 1], S.states[bw - 1], scratch, S.wbeg[bw - 1], S.W[bw - 1],
@@ -912,7 +937,7 @@ struct __align__(1024) DecSmem {
 
 static_assert(sizeof(DecSmem) + 1024 <= 232448, "decoder shared memory exceeds the per-block limit");
 static_assert(sizeof(ProjSmem) <= 232448, "projection shared memory exceeds the per-block limit");
-static_assert(sizeof(EntSmem) <= 232448 / 2, "entropy kernel should fit two blocks per SM");
+static_assert(sizeof(EntSmem) <= 232448 / 4, "entropy kernel should fit four blocks per SM");
 
 __global__ void __launch_bounds__(kThreads, 1)
 k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t* ws, uint32_t max_records) {
@@ -1142,7 +1167,7 @@ uint64_t transform_slot_bytes(const TransformShape& s) {
   // largest record: side info + up to 8 streams of the codes, or the raw rows
   uint64_t mid = pad16_64(8ull * kD * (kMaxCt / kTile)) + 8u * 16u + pad16_64(uint64_t(kD) * kMaxCt);
   uint64_t raw = pad16_64(uint64_t(s.s_end + (s.T - s.r_start)) * kD * 2u);
-  uint64_t b = (mid > raw ? mid : raw) + 2ull * kD * kMaxCt + 64u;
+  uint64_t b = (mid > raw ? mid : raw) + kWordsArea + kCodesArea;
   return (b + 255u) & ~uint64_t(255);
 }
 
