@@ -98,7 +98,6 @@ constexpr uint32_t kTabPool = 512;     // sum over widths 1..8 of 2^b, rounded u
 constexpr uint32_t kHistOffset = kCodesRow * kD;      // counts follow the codes in the slot
 constexpr uint32_t kCodesArea = kHistOffset + 4u * kTabPool;
 constexpr uint32_t kWordsArea = 2u * kD * kMaxCt + 64u;  // rANS word scratch: a word per symbol
-constexpr uint32_t kYStride = kD + 1u;                 // y[t][c] row stride in floats (odd: conflict-free)
 
 __device__ inline uint32_t tab_base(uint32_t b) { return (1u << b) - 2u; }  // 2 + 4 + ... + 2^(b-1)
 
@@ -106,7 +105,8 @@ struct __align__(16) ProjSmem {
   double Qd[kD * kD];                          // Q[k][c], coded components c < n_coded, fp64
   double x[kD * kProjTokens];                  // x[k][t]; then y[c][t] as fp32 in the same space
   uint32_t hist[kTabPool];                     // symbol counts of the record per width stream
-  float2 mm[2][kD];                            // per coded component: the two half-blocks' min and max
+  float2 part[kThreads / 32][kD];              // per warp and coded component: (min, max) of its tokens
+  float4 qp[kD];                               // per coded component: z, s, 1/s, levels | exact << 16
   uint32_t ccnt[8][kD];                        // counts of symbols 0..7 per coded component
   CompInfo ci;
   uint32_t cidx[kD];                           // coded component c -> channel-space index j
@@ -184,39 +184,124 @@ struct XFetch {
   }
 };
 
-// y[t][c] = sum_k Q[k][c] x[k][t] for this thread's tokens 4tg .. 4tg+3 and
-// components cg + 16jb (jb < NJB), fused multiply-adds with k ascending; then,
-// after a barrier (y overwrites x), the fp32 results of components c < nc.
+// One 64-token tile, which is quantiser block blk (bl valid tokens). y[t][c] =
+// sum_k Q[k][c] x[k][t] for this thread's tokens 4tg .. 4tg+3 and components
+// cc = cg + 16jb (jb < NJB): fused multiply-adds in fp64 with k ascending,
+// rounded to fp32. The block's minimum and maximum per component are then
+// combined in token order, the earlier of two equal values winning (the
+// sequential scan's result, -0 and +0 included): over the thread's tokens,
+// with the other half of the warp, and over the warps in order. Each thread
+// quantises its own values and writes a component's four codes with one
+// store; counts of symbols 0..7 per component gather in cnt, a byte each.
 template <uint32_t NJB>
-__device__ __forceinline__ void project_tile(const double* x, const double* Qd, float* y, uint32_t tg,
-                                             uint32_t cg, uint32_t nc) {
+__device__ __forceinline__ void project_quantize_tile(ProjSmem& S, uint32_t tg, uint32_t cg, uint32_t nc,
+                                                      uint32_t bl, uint32_t tb, uint32_t nb, uint8_t* rec,
+                                                      uint8_t* codes, uint32_t (&cnt)[8][2]) {
+  const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
   double acc[4][NJB];
 #pragma unroll
   for (uint32_t i = 0; i < 4; ++i)
 #pragma unroll
     for (uint32_t jb = 0; jb < NJB; ++jb) acc[i][jb] = 0.0;
+  // operands of row k + 1 are loaded before the multiply-adds of row k
+  const double* xb = &S.x[4u * tg];
+  const double* qb = &S.Qd[cg];
+  double2 x0 = reinterpret_cast<const double2*>(xb)[0], x1 = reinterpret_cast<const double2*>(xb)[1];
+  double qv[NJB];
+#pragma unroll
+  for (uint32_t jb = 0; jb < NJB; ++jb) qv[jb] = qb[16u * jb];
 #pragma unroll 2
   for (uint32_t k = 0; k < kD; ++k) {
-    const double2* xp = reinterpret_cast<const double2*>(&x[k * kProjTokens + 4u * tg]);
-    const double2 x0 = xp[0], x1 = xp[1];
-    const double xv[4] = {x0.x, x0.y, x1.x, x1.y};
-    const double* qrow = &Qd[k * kD + cg];
-    double qv[NJB];
+    const uint32_t kn = k + 1u < kD ? k + 1u : k;
+    const double2 n0 = reinterpret_cast<const double2*>(xb + kn * kProjTokens)[0];
+    const double2 n1 = reinterpret_cast<const double2*>(xb + kn * kProjTokens)[1];
+    double nq[NJB];
 #pragma unroll
-    for (uint32_t jb = 0; jb < NJB; ++jb) qv[jb] = qrow[16u * jb];
+    for (uint32_t jb = 0; jb < NJB; ++jb) nq[jb] = qb[kn * kD + 16u * jb];
+    const double xv[4] = {x0.x, x0.y, x1.x, x1.y};
 #pragma unroll
     for (uint32_t i = 0; i < 4; ++i)
 #pragma unroll
       for (uint32_t jb = 0; jb < NJB; ++jb) acc[i][jb] = fma(qv[jb], xv[i], acc[i][jb]);
+    x0 = n0;
+    x1 = n1;
+#pragma unroll
+    for (uint32_t jb = 0; jb < NJB; ++jb) qv[jb] = nq[jb];
+  }
+  float yv[4][NJB];
+#pragma unroll
+  for (uint32_t i = 0; i < 4; ++i)
+#pragma unroll
+    for (uint32_t jb = 0; jb < NJB; ++jb) yv[i][jb] = __double2float_rn(acc[i][jb]);
+  const uint32_t nv = bl > 4u * tg ? min(4u, bl - 4u * tg) : 0u;  // this thread's valid tokens
+#pragma unroll
+  for (uint32_t jb = 0; jb < NJB; ++jb) {
+    float mn = __int_as_float(0x7f800000), mx = __int_as_float(0xff800000);
+#pragma unroll
+    for (uint32_t i = 0; i < 4; ++i) {
+      if (i < nv) {
+        const float v = yv[i][jb];
+        if (v < mn) mn = v;
+        if (v > mx) mx = v;
+      }
+    }
+    // lanes 0-15 hold tokens 8w .. 8w+3, lanes 16-31 the next four
+    const float pmn = __shfl_xor_sync(0xffffffffu, mn, 16), pmx = __shfl_xor_sync(0xffffffffu, mx, 16);
+    if (lane < 16u) {
+      if (pmn < mn) mn = pmn;
+      if (pmx > mx) mx = pmx;
+    } else {
+      mn = mn < pmn ? mn : pmn;
+      mx = mx > pmx ? mx : pmx;
+    }
+    const uint32_t cc = cg + 16u * jb;
+    if (lane < 16u && cc < nc) S.part[warp][cc] = make_float2(mn, mx);
+  }
+  __syncthreads();
+  // thread cc < nc: the block's minimum, maximum and scale of component cc
+  if (threadIdx.x < nc) {
+    const uint32_t cc = threadIdx.x;
+    float mn = __int_as_float(0x7f800000), mx = __int_as_float(0xff800000);
+#pragma unroll
+    for (uint32_t w = 0; w < kThreads / 32u; ++w) {
+      const float2 p = S.part[w][cc];
+      if (p.x < mn) mn = p.x;
+      if (p.y > mx) mx = p.y;
+    }
+    const uint32_t levels = (1u << S.ci.width[S.cidx[cc]]) - 1u;
+    const float s = (mx == mn) ? 0.0f : __fdiv_rn(__fsub_rn(mx, mn), float(levels));
+    const float rs = s == 0.0f ? 0.0f : __frcp_rn(s);
+    const uint32_t exact = !(rs < 0x1p126f) ? 1u : 0u;
+    uint32_t* zp = reinterpret_cast<uint32_t*>(rec + 8u * (cc * nb + tb / kTile));
+    zp[0] = __float_as_uint(mn);
+    zp[1] = __float_as_uint(s);
+    S.qp[cc] = make_float4(mn, s, rs, __uint_as_float(levels | (exact << 16)));
   }
   __syncthreads();
 #pragma unroll
   for (uint32_t jb = 0; jb < NJB; ++jb) {
     const uint32_t cc = cg + 16u * jb;
-    if (cc < nc) {
+    if (cc >= nc) continue;
+    const float4 qp = S.qp[cc];
+    const float mn = qp.x, s = qp.y, rs = qp.z;
+    const uint32_t levels = __float_as_uint(qp.w) & 0xffffu;
+    const bool exact = (__float_as_uint(qp.w) >> 16) != 0u;
+    const uint32_t j = S.cidx[cc];
+    uint32_t word = 0;
 #pragma unroll
-      for (uint32_t i = 0; i < 4; ++i) y[(4u * tg + i) * kYStride + cc] = __double2float_rn(acc[i][jb]);
+    for (uint32_t i = 0; i < 4; ++i) {
+      if (i < nv) {
+        bool nd;
+        uint32_t q = quantize_fast(yv[i][jb], mn, rs, levels, exact, nd);
+        if (nd) q = quantize(yv[i][jb], mn, s, levels);  // near a half-integer: the IEEE division decides
+        word |= q << (8u * i);
+        const uint32_t inc = 1u << (8u * (q & 3u));
+        if (q < 4u) cnt[jb][0] += inc;
+        else if (q < 8u) cnt[jb][1] += inc;
+        else atomicAdd(&S.hist[levels - 1u + q], 1u);  // tab_base(b) = 2^b - 2 = levels - 1
+      }
     }
+    *reinterpret_cast<uint32_t*>(codes + uint64_t(j) * kCodesRow + tb + 4u * tg) = word;
   }
 }
 
@@ -276,111 +361,44 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
   if (tid < pad16(side) - side) rec[side + tid] = 0;
   __syncthreads();
 
-  float* y = reinterpret_cast<float*>(S.x);    // y[t][c] (row stride kYStride), after the projection
   // thread: tokens 4tg .. 4tg+3 and components cg + 16jb, jb < ceil(nc / 16)
   const uint32_t tg = tid >> 4, cg = tid & 15u;
   const uint32_t njb = (nc + 15u) >> 4;
+  uint32_t cnt[8][2];  // per jb: counts of symbols 0..3 and 4..7 of this thread's codes, a byte each
+#pragma unroll
+  for (uint32_t jb = 0; jb < 8; ++jb) cnt[jb][0] = cnt[jb][1] = 0;
   XFetch xf;
   xf.load(xs, pl.rope, is_key, t0, 0, min(kProjTokens, tcc));
   for (uint32_t tb = 0; tb < tcc; tb += kProjTokens) {
     const uint32_t bl = min(kProjTokens, tcc - tb);
     xf.stage(S.x, is_key);
     __syncthreads();
-    switch (njb) {
-      case 1: project_tile<1>(S.x, S.Qd, y, tg, cg, nc); break;
-      case 2: project_tile<2>(S.x, S.Qd, y, tg, cg, nc); break;
-      case 3: project_tile<3>(S.x, S.Qd, y, tg, cg, nc); break;
-      case 4: project_tile<4>(S.x, S.Qd, y, tg, cg, nc); break;
-      case 5: project_tile<5>(S.x, S.Qd, y, tg, cg, nc); break;
-      case 6: project_tile<6>(S.x, S.Qd, y, tg, cg, nc); break;
-      case 7: project_tile<7>(S.x, S.Qd, y, tg, cg, nc); break;
-      default: project_tile<8>(S.x, S.Qd, y, tg, cg, nc); break;
-    }
-    __syncthreads();
-    // quantiser: thread (component cc, half h) owns tokens 32h .. 32h+31 of the
-    // block. The halves' minima and maxima, each a sequential scan, combine with
-    // the first half winning ties, which is the sequential scan of the block.
-    const uint32_t blk = tb / kTile;
-    const bool qthr = tid < 2u * nc;
-    const uint32_t h = tid >= nc ? 1u : 0u, cc = tid - h * nc;
-    const uint32_t lo = 32u * h, n = bl > lo ? min(32u, bl - lo) : 0u;
-    if (qthr) {
-      const float* yc = y + lo * kYStride + cc;
-      float mn = __int_as_float(0x7f800000), mx = __int_as_float(0xff800000);
-      if (n) {
-        mn = mx = yc[0];
-#pragma unroll 8
-        for (uint32_t tt = 1; tt < n; ++tt) {
-          const float v = yc[tt * kYStride];
-          if (v < mn) mn = v;
-          if (v > mx) mx = v;
-        }
-      }
-      S.mm[h][cc] = make_float2(mn, mx);
-    }
-    __syncthreads();
-    // the next tile's rows are fetched now and land while this one is quantised
+    // the next tile's rows are fetched now and land during this one's projection
     if (tb + kProjTokens < tcc) xf.load(xs, pl.rope, is_key, t0, tb + kProjTokens, min(kProjTokens, tcc - tb - kProjTokens));
-    if (qthr) {
-      const float2 m0 = S.mm[0][cc], m1 = S.mm[1][cc];
-      const float mn = m1.x < m0.x ? m1.x : m0.x, mx = m1.y > m0.y ? m1.y : m0.y;
-      const uint32_t j = S.cidx[cc], w = S.ci.width[j];
-      const uint32_t levels = (1u << w) - 1u;
-      const float s = (mx == mn) ? 0.0f : __fdiv_rn(__fsub_rn(mx, mn), float(levels));
-      const float rs = s == 0.0f ? 0.0f : __frcp_rn(s);
-      const bool exact = !(rs < 0x1p126f);
-      if (h == 0) {
-        uint32_t* zp = reinterpret_cast<uint32_t*>(rec + 8u * (cc * nb + blk));
-        zp[0] = __float_as_uint(mn);
-        zp[1] = __float_as_uint(s);
-      }
-      uint32_t cnt_lo = 0, cnt_hi = 0;  // counts of symbols 0..3 and 4..7, a byte each
-      for (uint32_t t8 = 0; t8 < n; t8 += 8u) {
-        float v[8];
-        uint32_t qv[8], need = 0;
+    switch (njb) {
+      case 1: project_quantize_tile<1>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
+      case 2: project_quantize_tile<2>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
+      case 3: project_quantize_tile<3>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
+      case 4: project_quantize_tile<4>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
+      case 5: project_quantize_tile<5>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
+      case 6: project_quantize_tile<6>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
+      case 7: project_quantize_tile<7>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
+      default: project_quantize_tile<8>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
+    }
+    __syncthreads();  // x and the warp partials are rewritten by the next tile
+  }
 #pragma unroll
-        for (uint32_t i = 0; i < 8; ++i) v[i] = t8 + i < n ? y[(lo + t8 + i) * kYStride + cc] : mn;
-#pragma unroll
-        for (uint32_t i = 0; i < 8; ++i) {
-          bool nd;
-          qv[i] = quantize_fast(v[i], mn, rs, levels, exact, nd);
-          need |= uint32_t(nd) << i;
-        }
-        while (need) {  // quotients near a half-integer: the IEEE division decides
-          const uint32_t i = __ffs(need) - 1u;
-          need &= need - 1u;
-          float vi = v[0];
-#pragma unroll
-          for (uint32_t u = 1; u < 8; ++u) vi = u == i ? v[u] : vi;
-          const uint32_t qi = quantize(vi, mn, s, levels);
-#pragma unroll
-          for (uint32_t u = 0; u < 8; ++u) qv[u] = u == i ? qi : qv[u];
-        }
-        // the 8 codes (past n: zeros) go to the component's row in one store
-        *reinterpret_cast<uint2*>(codes + uint64_t(j) * kCodesRow + tb + lo + t8) =
-            make_uint2(qv[0] | (qv[1] << 8) | (qv[2] << 16) | (qv[3] << 24),
-                       qv[4] | (qv[5] << 8) | (qv[6] << 16) | (qv[7] << 24));
-#pragma unroll
-        for (uint32_t i = 0; i < 8; ++i) {
-          if (t8 + i < n) {
-            const uint32_t q = qv[i];
-            if (q < 8u) {
-              const uint32_t inc = 1u << (8u * (q & 3u));
-              if (q < 4u) cnt_lo += inc; else cnt_hi += inc;
-            } else {
-              atomicAdd(&S.hist[tab_base(w) + q], 1u);
-            }
-          }
-        }
-      }
+  for (uint32_t jb = 0; jb < 8; ++jb) {
+    const uint32_t cc = cg + 16u * jb;
+    if (jb < njb && cc < nc) {
 #pragma unroll
       for (uint32_t q = 0; q < 8; ++q) {
-        const uint32_t c = ((q < 4u ? cnt_lo : cnt_hi) >> (8u * (q & 3u))) & 0xffu;
+        const uint32_t c = (cnt[jb][q >> 2] >> (8u * (q & 3u))) & 0xffu;
         if (c) atomicAdd(&S.ccnt[q][cc], c);
       }
     }
-    __syncthreads();
   }
+  __syncthreads();
   // counts of symbols 0..7 summed over the components of each width
   if (tid < 64u) {
     const uint32_t bw = (tid >> 3) + 1u, q = tid & 7u;
