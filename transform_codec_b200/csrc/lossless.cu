@@ -772,63 +772,54 @@ __device__ __forceinline__ uint32_t merge_planes(uint32_t j, uint32_t a, uint32_
 // which leave a zero register unchanged; comp complements the record's first
 // four bytes, the standard CRC's initial value) or left-aligned (trailing zero
 // units, processed: the result is then multiplied by x^(8 * (2048q - len))).
-// The units are spread over the 16 tiles and loaded one tile ahead.
+// It runs before the tiles, four loads ahead, so that none of its state is
+// live during the decode loop.
 struct PreRun {
   const uint8_t* p;
-  uint32_t len, q, upt;  // upt: units per tile, ceil(q / 16) <= 3
+  uint32_t len, q;
   int32_t run0;
   bool left, comp;
   uint32_t c;
-  uint4 nxt[3];
-  __device__ __forceinline__ void init(const uint8_t* base, uint32_t n, bool left_aligned, bool comp_first) {
+  __device__ __forceinline__ void run(const uint8_t* base, uint32_t n, bool left_aligned, bool comp_first,
+                                      const uint32_t* t) {
     p = base;
     len = n;
     q = (n + 2047u) >> 11;
-    upt = (q + 15u) >> 4;
     left = left_aligned;
     comp = comp_first;
     run0 = int32_t(threadIdx.x * 16u * q) - (left ? 0 : int32_t(128u * 16u * q - n));
     c = 0;
-    fetch(0);
-  }
-  __device__ __forceinline__ void fetch(uint32_t k) {
+    for (uint32_t u0 = 0; u0 < q; u0 += 4u) {
+      uint4 v[4];
 #pragma unroll
-    for (uint32_t i = 0; i < 3; ++i) {
-      const uint32_t u = k * upt + i;
-      const int32_t off = run0 + int32_t(16u * u);
-      const bool in = i < upt && u < q && off >= 0 && uint32_t(off) < len;
-      nxt[i] = in ? __ldcg(reinterpret_cast<const uint4*>(p + off)) : make_uint4(0, 0, 0, 0);
-    }
-  }
-  // fold in tile k's units (loaded by the previous fetch) and load tile k + 1's
-  __device__ __forceinline__ void tile(const uint32_t* t, uint32_t k) {
-    uint4 cur[3] = {nxt[0], nxt[1], nxt[2]};
-    if (k + 1 < 16) fetch(k + 1);
+      for (uint32_t i = 0; i < 4; ++i) {
+        const int32_t off = run0 + int32_t(16u * (u0 + i));
+        const bool in = u0 + i < q && off >= 0 && uint32_t(off) < len;
+        v[i] = in ? __ldcg(reinterpret_cast<const uint4*>(p + off)) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-    for (uint32_t i = 0; i < 3; ++i) {
-      const uint32_t u = k * upt + i;
-      const int32_t off = run0 + int32_t(16u * u);
-      if (i < upt && u < q && (left || off >= 0)) {
-        if (comp && off == 0) cur[i].x = ~cur[i].x;
-        c = crc_word(t, c, cur[i].x);
-        c = crc_word(t, c, cur[i].y);
-        c = crc_word(t, c, cur[i].z);
-        c = crc_word(t, c, cur[i].w);
+      for (uint32_t i = 0; i < 4; ++i) {
+        const int32_t off = run0 + int32_t(16u * (u0 + i));
+        if (u0 + i < q && (left || off >= 0)) {
+          if (comp && off == 0) v[i].x = ~v[i].x;
+          c = crc_word(t, c, v[i].x);
+          c = crc_word(t, c, v[i].y);
+          c = crc_word(t, c, v[i].z);
+          c = crc_word(t, c, v[i].w);
+        }
       }
     }
   }
 };
 
 // Decode the 16 tiles of 32 steps of one record. crc0 / crc1 return the CRC
-// register of this lane's 512 bytes of plane 0 / 1 when that plane is RAW; pre
-// folds in this thread's run of the pre-pass region.
+// register of this lane's 512 bytes of plane 0 / 1 when that plane is RAW.
 template <uint32_t M0, uint32_t M1, uint32_t D>
 __device__ inline bool fast_tiles(FastSmem& S, const uint8_t* const recp[2], uint16_t* out,
-                                  PreRun& pre, uint32_t& crc0, uint32_t& crc1) {
+                                  uint32_t& crc0, uint32_t& crc1) {
   constexpr uint32_t LPC = 128u / D;  // lanes per channel
   constexpr bool kRaw0 = M0 == kModeRaw, kRaw1 = M1 == kModeRaw;
   constexpr bool kRans = (M0 == kModeRans || M1 == kModeRans);
-  constexpr bool kPre = !(kRaw0 && kRaw1);
   constexpr uint32_t RP = (M0 == kModeRans) ? 0u : 1u;  // the rANS plane, if any
   const uint32_t l = threadIdx.x, lane = l & 31u, g = l >> 5;
   const uint32_t lt = lanemask_lt();
@@ -885,7 +876,6 @@ __device__ inline bool fast_tiles(FastSmem& S, const uint8_t* const recp[2], uin
         n1b = __ldcg(reinterpret_cast<const uint4*>(raw1 + 32u * (k + 1) + 16u));
       }
     }
-    if (kPre) pre.tile(S.crc_t, k);
     uint32_t* o = o32 + (k * 32u) * (D / 2u);
     // four stages of 8 steps; each consumes raw words 0 and 1, then the words shift down
 #pragma unroll 1
@@ -934,15 +924,15 @@ __device__ inline bool fast_tiles(FastSmem& S, const uint8_t* const recp[2], uin
 
 template <uint32_t D>
 __device__ inline bool fast_dispatch(FastSmem& S, const uint8_t* const recp[2], uint16_t* out,
-                                     uint32_t m0, uint32_t m1, PreRun& pre, uint32_t& crc0, uint32_t& crc1) {
-  if (m0 == kModeRaw && m1 == kModeRans) return fast_tiles<kModeRaw, kModeRans, D>(S, recp, out, pre, crc0, crc1);
-  if (m0 == kModeRaw && m1 == kModeRaw) return fast_tiles<kModeRaw, kModeRaw, D>(S, recp, out, pre, crc0, crc1);
-  if (m0 == kModeRaw && m1 == kModeConst) return fast_tiles<kModeRaw, kModeConst, D>(S, recp, out, pre, crc0, crc1);
-  if (m0 == kModeRans && m1 == kModeRaw) return fast_tiles<kModeRans, kModeRaw, D>(S, recp, out, pre, crc0, crc1);
-  if (m0 == kModeRans && m1 == kModeConst) return fast_tiles<kModeRans, kModeConst, D>(S, recp, out, pre, crc0, crc1);
-  if (m0 == kModeConst && m1 == kModeRans) return fast_tiles<kModeConst, kModeRans, D>(S, recp, out, pre, crc0, crc1);
-  if (m0 == kModeConst && m1 == kModeRaw) return fast_tiles<kModeConst, kModeRaw, D>(S, recp, out, pre, crc0, crc1);
-  return fast_tiles<kModeConst, kModeConst, D>(S, recp, out, pre, crc0, crc1);
+                                     uint32_t m0, uint32_t m1, uint32_t& crc0, uint32_t& crc1) {
+  if (m0 == kModeRaw && m1 == kModeRans) return fast_tiles<kModeRaw, kModeRans, D>(S, recp, out, crc0, crc1);
+  if (m0 == kModeRaw && m1 == kModeRaw) return fast_tiles<kModeRaw, kModeRaw, D>(S, recp, out, crc0, crc1);
+  if (m0 == kModeRaw && m1 == kModeConst) return fast_tiles<kModeRaw, kModeConst, D>(S, recp, out, crc0, crc1);
+  if (m0 == kModeRans && m1 == kModeRaw) return fast_tiles<kModeRans, kModeRaw, D>(S, recp, out, crc0, crc1);
+  if (m0 == kModeRans && m1 == kModeConst) return fast_tiles<kModeRans, kModeConst, D>(S, recp, out, crc0, crc1);
+  if (m0 == kModeConst && m1 == kModeRans) return fast_tiles<kModeConst, kModeRans, D>(S, recp, out, crc0, crc1);
+  if (m0 == kModeConst && m1 == kModeRaw) return fast_tiles<kModeConst, kModeRaw, D>(S, recp, out, crc0, crc1);
+  return fast_tiles<kModeConst, kModeConst, D>(S, recp, out, crc0, crc1);
 }
 
 // CRC register of a 16-byte stream header; comp complements its first four
@@ -956,7 +946,7 @@ __device__ inline uint32_t crc_header16(const uint32_t* t, const uint8_t* h, boo
   return crc_word(t, c, v.w);
 }
 
-__global__ void __launch_bounds__(kFastThreads, 6)
+__global__ void __launch_bounds__(kFastThreads, 5)
 k_lossless_decode_fast(LosslessShape sh, FrameBatch b, uint8_t* ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   FastSmem& S = *reinterpret_cast<FastSmem*>(smem_raw);
@@ -1025,17 +1015,17 @@ k_lossless_decode_fast(LosslessShape sh, FrameBatch b, uint8_t* ws) {
     // neither plane is RAW, else the other stream record (left-aligned when it
     // follows the RAW stream, so that no shift by its runtime length is needed)
     PreRun pre;
-    if (!raw0 && !raw1) pre.init(rec, len, false, true);
-    else if (raw0 && !raw1) pre.init(rec + b0, b1, true, false);
-    else if (!raw0 && raw1) pre.init(rec, b0, false, true);
-    else pre.init(rec, 0, false, false);
+    if (!raw0 && !raw1) pre.run(rec, len, false, true, S.crc_t);
+    else if (raw0 && !raw1) pre.run(rec + b0, b1, true, false, S.crc_t);
+    else if (!raw0 && raw1) pre.run(rec, b0, false, true, S.crc_t);
+    else pre.run(rec, 0, false, false, S.crc_t);
     if (m0 == kModeRans) block_dec_lut(S.freq[0], S.cum, S.lut, S.tmp);
     else if (m1 == kModeRans) block_dec_lut(S.freq[1], S.cum, S.lut, S.tmp);
     const uint8_t* recp[2] = {rec, rec + b0};
     uint16_t* out = dst + (uint64_t(slice) * sh.T + t0) * D;
     uint32_t cr0 = 0, cr1 = 0;
-    bool ok = D == 128u ? fast_dispatch<128>(S, recp, out, m0, m1, pre, cr0, cr1)
-                        : fast_dispatch<64>(S, recp, out, m0, m1, pre, cr0, cr1);
+    bool ok = D == 128u ? fast_dispatch<128>(S, recp, out, m0, m1, cr0, cr1)
+                        : fast_dispatch<64>(S, recp, out, m0, m1, cr0, cr1);
     const uint32_t prc = !(raw0 && raw1) ? crc_join_lanes(pre.c, pre.q, S.red) : 0u;
     const uint32_t p0 = raw0 ? crc_join_lanes(cr0, 32u, S.red) : 0u;  // 512-byte lane runs
     const uint32_t p1 = raw1 ? crc_join_lanes(cr1, 32u, S.red) : 0u;
