@@ -33,17 +33,19 @@ WORKLOAD_L = "lossless-64x8x32768x128-bf16"
 WORKLOAD_T = "transform-64x8x32768x128-bf16"
 METRIC = "KV codec encode/decode GB/s (raw bytes) vs HBM roofline; compression ratio"
 
-# algorithmic work per step of each kernel, given the step's raw bytes R, its
-# container bytes C and its middle (transform-coded) values V
-# Algorithmic work per step of each kernel with a roofline: bytes for the
-# lossless kernels (raw + container), and for the transform contraction 2 * 128
-# flops per middle value (one contraction; the projection kernel runs it in
-# fp64 on the CUDA cores, the decoder in bf16 pieces on the tensor cores).
-# R = raw bytes, C = container bytes, V = middle values of the step.
+# Algorithmic work per step of each kernel with a roofline, given the step's
+# raw bytes R, its container bytes C and its middle (transform-coded) values V:
+# bytes for the lossless kernels (raw + container) and for the transform
+# entropy stages (a code byte per middle value + the records), and 2 * 128
+# flops per middle value for the transform contraction (one contraction; the
+# projection kernel runs it in fp64 on the CUDA cores, the decoder in bf16
+# pieces on the tensor cores).
 KERNEL_WORK = {
     "lossless_encode": ("hbm", lambda R, C, V: R + C),
     "lossless_decode": ("hbm", lambda R, C, V: R + C),
     "transform_project": ("alu", lambda R, C, V: 2 * 128 * V),
+    "transform_entropy": ("hbm", lambda R, C, V: V + C),          # codes in, records out
+    "transform_decode_codes": ("hbm", lambda R, C, V: C + V),     # records in, codes out
     "transform_decode": ("tensor", lambda R, C, V: 2 * 128 * V),
 }
 
@@ -366,8 +368,8 @@ def run_kvc(args):
     hbm_peak, bf16_peak, sm_max, peak_kind = measured_peaks()
     fp64_peak = 148 * 64 * 2 * sm_max * 1e6 / 1e12  # TFLOP/s, 64 fp64 FMA/clk/SM
     launches = sum(n for n, _ in kernels.values())
-    step_cont = {"lossless_encode": cont_l, "lossless_decode": cont_l,
-                 "transform_project": cont_t, "transform_decode": cont_t}
+    step_cont = {"lossless_encode": cont_l, "lossless_decode": cont_l, "transform_project": cont_t,
+                 "transform_entropy": cont_t, "transform_decode_codes": cont_t, "transform_decode": cont_t}
     kern_out = {}
     total_kern_ms = sum(t for _, t in kernels.values()) or 1.0
     for name, (n, t) in kernels.items():
