@@ -196,3 +196,42 @@ def test_transform_full_size_sampled():
         st_o, y_o = oracle.decode_transform(oplan, one, n_slices_cap=1)
         assert st_o == oracle.OK
         assert rel_rms(y_o[0], y_g[s]) <= REL_RMS
+
+
+@pytest.mark.parametrize("T", [1024, 644])
+def test_transform_container_equals_oracle_bytes(T):
+    """The encoder's projection reproduces the oracle's fp64 y bit for bit (the
+    same fused multiply-adds in the same order), so the whole container, side
+    information included, is the oracle's byte for byte."""
+    w = _w(n_tokens=T)
+    bases, _, widths = _small_inputs(w)
+    plan, oplan = _plans(w, bases, widths)
+    x = kvgen.slices(w)
+    st, got = encode(plan, kvc.TRANSFORM, x)
+    assert st == kvc.OK
+    want = oracle.encode_transform(oplan, x)
+    assert len(got) == len(want)
+    assert got == want
+
+
+def test_transform_container_equals_oracle_bytes_extremes():
+    """Tokens of very different scales (2^-60, 2^40), all-zero tokens and
+    repeated tokens (tied block extremes, signed zeros) keep the bytes exact."""
+    w = _w(n_tokens=644)
+    bases, _, widths = _small_inputs(w)
+    plan, oplan = _plans(w, bases, widths)
+    x = kvgen.slices(w).copy()
+    rng = np.random.default_rng(11)
+    mid = np.arange(w.n_sink, w.n_tokens - w.n_recent)
+    zero = rng.choice(mid, 40, replace=False)
+    x[:, zero, :] = 0
+    small = rng.choice(np.setdiff1d(mid, zero), 40, replace=False)
+    f = (x[:, small, :].astype(np.uint32) << 16).view(np.float32) * np.float32(2.0 ** -60)
+    x[:, small, :] = (f.view(np.uint32) >> 16).astype(np.uint16)
+    big = rng.choice(np.setdiff1d(mid, np.union1d(zero, small)), 40, replace=False)
+    f = (x[:, big, :].astype(np.uint32) << 16).view(np.float32) * np.float32(2.0 ** 40)
+    x[:, big, :] = (f.view(np.uint32) >> 16).astype(np.uint16)
+    x[:, mid[100:110], :] = x[:, mid[99:100], :]  # repeated tokens: tied extremes
+    st, got = encode(plan, kvc.TRANSFORM, x)
+    assert st == kvc.OK
+    assert got == oracle.encode_transform(oplan, x)
