@@ -1024,32 +1024,38 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
     uint32_t wmask = 0;
 #pragma unroll
     for (uint32_t i = 0; i < 8; ++i) wmask |= S.ci.width[j0 + i] ? (1u << i) : 0u;
-    if (tid < kD && S.ci.width[tid]) {
-      const uint32_t* p32 = reinterpret_cast<const uint32_t*>(rec + 8u * S.ci.coded_idx[tid] * nb);
-      for (uint32_t blk = 0; blk < nb; ++blk) {
-        S.zsT[tid & 7u][blk][tid >> 3] =
-            make_float2(__uint_as_float(__ldg(&p32[2 * blk])), __uint_as_float(__ldg(&p32[2 * blk + 1])));
-      }
+    if (tid < kD && S.ci.width[tid]) {  // all of the component's (z, s) pairs are loaded before any is stored
+      const uint2* p64 = reinterpret_cast<const uint2*>(rec + 8u * S.ci.coded_idx[tid] * nb);
+      uint2 zs[kMaxCt / kTile];
+#pragma unroll
+      for (uint32_t blk = 0; blk < kMaxCt / kTile; ++blk) zs[blk] = blk < nb ? __ldg(p64 + blk) : make_uint2(0, 0);
+#pragma unroll
+      for (uint32_t blk = 0; blk < kMaxCt / kTile; ++blk)
+        if (blk < nb) S.zsT[tid & 7u][blk][tid >> 3] = make_float2(__uint_as_float(zs[blk].x), __uint_as_float(zs[blk].y));
     }
     // inverse projection on the tensor cores, 128 tokens at a time:
     // x^[t][k] = sum_j y^[t][j] Q[k][j] with y^ and Q split into bf16 hi + lo
-    // pieces (hi*hi + hi*lo + lo*hi, fp32 accumulation in tensor memory)
-    for (uint32_t t_base = 0; t_base < tcc; t_base += kTcRows) {
-      const uint32_t bl = min(kTcRows, tcc - t_base);
-      __syncthreads();
-      // item k of this thread: token tt = tid / 16 + 16 k, components j0 .. j0 + 7
-      // (the same for all its items) -> one 16-byte chunk of each piece. The
-      // codes are loaded first, so their latencies overlap; the scales and zero
-      // points of the tile's two blocks come from shared memory once.
-      constexpr uint32_t kItems = kTcRows * (kD / 8u) / kThreads;
-      static_assert(kItems == 8 && kTcRows == 2 * kTile, "item k lies in the tile's block k / 4");
-      uint2 cw8[kItems];
+    // pieces (hi*hi + hi*lo + lo*hi, fp32 accumulation in tensor memory).
+    // Item k of this thread: token tt = tid / 16 + 16 k, components j0 .. j0 + 7
+    // (the same for all its items) -> one 16-byte chunk of each piece. A tile's
+    // codes are loaded while the previous tile's products run (the first tile's
+    // here), so that their latency overlaps the tensor cores and the epilogue.
+    constexpr uint32_t kItems = kTcRows * (kD / 8u) / kThreads;
+    static_assert(kItems == 8 && kTcRows == 2 * kTile, "item k lies in the tile's block k / 4");
+    uint2 cw8[kItems];
+    auto load_codes = [&](uint32_t tb) {
+      const uint32_t n = min(kTcRows, tcc - tb);
 #pragma unroll
       for (uint32_t k = 0; k < kItems; ++k) {
         const uint32_t tt = (tid >> 4) + 16u * k;
-        cw8[k] = tt < bl ? __ldcg(reinterpret_cast<const uint2*>(codes + (t_base + tt) * kCodeRow + j0))
-                         : make_uint2(0, 0);
+        cw8[k] = tt < n ? __ldcg(reinterpret_cast<const uint2*>(codes + (tb + tt) * kCodeRow + j0)) : make_uint2(0, 0);
       }
+    };
+    load_codes(0);
+    for (uint32_t t_base = 0; t_base < tcc; t_base += kTcRows) {
+      const uint32_t bl = min(kTcRows, tcc - t_base);
+      __syncthreads();
+      // the scales and zero points of the tile's two blocks come from shared memory once
       float2 zr[2][8];
 #pragma unroll
       for (uint32_t b2 = 0; b2 < 2; ++b2)
@@ -1098,14 +1104,18 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
         }
         tc::mma_commit(&S.bar);
       }
-      if (is_key) {  // this thread's RoPE pairs for the epilogue, fetched while the MMAs run
+      // while the MMAs run: this thread's RoPE pairs for the epilogue (warp w:
+      // token rows 32 (w % 4) .., channel pairs 32 (w / 4) .. + 32) and the next
+      // tile's codes
+      float4 rp[16];
+      {
         const uint32_t ptt = (warp & 3u) * 32u + lane;
-        if (ptt < bl) {
-          const float* cs = pl.rope + (uint64_t(t0 + t_base + ptt) * (kD / 2) + (warp >> 2) * 32u) * 2u;
-          asm volatile("prefetch.global.L1 [%0];" ::"l"(cs));
-          asm volatile("prefetch.global.L1 [%0];" ::"l"(cs + 32));
-        }
+        const float4* cs4 = reinterpret_cast<const float4*>(pl.rope + (uint64_t(t0 + t_base + ptt) * (kD / 2) + (warp >> 2) * 32u) * 2u);
+        const bool rl = is_key && ptt < bl;
+#pragma unroll
+        for (uint32_t i = 0; i < 16; ++i) rp[i] = rl ? __ldg(cs4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
+      if (t_base + kTcRows < tcc) load_codes(t_base + kTcRows);
       const bool done = tc::mbar_wait(&S.bar, phase, 1u << 22);
       phase ^= 1u;
       if (!__syncthreads_and(done)) {
@@ -1130,14 +1140,13 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
         tc::tmem_wait_ld();
         if (tt < bl) {
           const uint32_t t = t0 + t_base + tt;
-          const float2* cs = reinterpret_cast<const float2*>(pl.rope) + uint64_t(t) * (kD / 2) + c0;
           uint32_t pa[16], pb[16];
 #pragma unroll
           for (uint32_t i = 0; i < 32; i += 2) {
             float a0 = __uint_as_float(va[i]), b0 = __uint_as_float(vb[i]);
             float a1 = __uint_as_float(va[i + 1]), b1 = __uint_as_float(vb[i + 1]);
             if (is_key) {
-              const float4 kk = __ldg(reinterpret_cast<const float4*>(cs) + (i >> 1));  // pairs i, i + 1
+              const float4 kk = rp[i >> 1];  // (cos, sin) of pairs i, i + 1
               const float2 k0 = make_float2(kk.x, kk.y), k1 = make_float2(kk.z, kk.w);
               const float na0 = __fsub_rn(__fmul_rn(a0, k0.x), __fmul_rn(b0, k0.y));
               const float nb0 = __fadd_rn(__fmul_rn(a0, k0.y), __fmul_rn(b0, k0.x));
