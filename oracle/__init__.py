@@ -83,6 +83,8 @@ def _load():
         "kvco_container_codes": ([P(Desc), vp, sz, u32, vp, vp, P(u32)], i32),
         "kvco_pca": ([vp, u32, u32, u32, i32, dbl, vp, vp], i32),
         "kvco_jacobi_eigen": ([vp, u32, vp, vp], i32),
+        "kvco_fixed_basis": ([u32, u32, vp], i32),
+        "kvco_basis_variances": ([vp, u32, u32, u32, i32, dbl, vp, vp], i32),
         "kvco_bf16_to_f32": ([ctypes.c_uint16], ctypes.c_float),
         "kvco_f32_to_bf16": ([ctypes.c_float], ctypes.c_uint16),
     }
@@ -342,6 +344,28 @@ def pca(calib: np.ndarray, is_key: bool, theta: float):
     if st != OK:
         raise ValueError("oracle PCA refused its arguments")
     return Q, lam
+
+
+HADAMARD, DCT = 1, 2
+
+
+def fixed_basis(kind: int, D: int) -> np.ndarray:
+    """Calibration-free basis [D][D] fp32 (element [k][j]: channel k of component j)."""
+    Q = np.zeros((D, D), dtype=np.float32)
+    if _load().kvco_fixed_basis(kind, D, _ptr(Q)) != OK:
+        raise ValueError("oracle refused the basis kind or size")
+    return Q
+
+
+def basis_variances(calib: np.ndarray, is_key: bool, theta: float, Q: np.ndarray) -> np.ndarray:
+    """Second moment of each component of basis Q over the calibration tokens."""
+    c = np.ascontiguousarray(calib, dtype=np.uint16)
+    q = np.ascontiguousarray(Q, dtype=np.float32)
+    n_tok, D = c.shape
+    lam = np.zeros(D, dtype=np.float64)
+    if _load().kvco_basis_variances(_ptr(c), n_tok, D, BF16, int(is_key), theta, _ptr(q), _ptr(lam)) != OK:
+        raise ValueError("oracle refused its arguments")
+    return lam
 
 
 def jacobi_eigen(A: np.ndarray):

@@ -1325,9 +1325,9 @@ int kvco_jacobi_eigen(const double* A, uint32_t n, double* V, double* w) {
   return KVCO_OK;
 }
 
-int kvco_pca(const uint16_t* calib, uint32_t n_tok, uint32_t D, uint32_t dtype, int is_key,
-             double theta, float* Q, double* lambda) {
-  if (dtype != KVCO_BF16 || n_tok == 0 || D == 0 || (D & 1u)) return KVCO_INVALID;
+/* Uncentered second moments C = (1/n) sum_t x_t x_t^T of the calibration
+ * tokens (keys de-rotated), accumulated in fp64 over t ascending. */
+static double* second_moments(const uint16_t* calib, uint32_t n_tok, uint32_t D, int is_key, double theta) {
   uint32_t half = D / 2;
   float* cs = (float*)malloc(sizeof(float) * (size_t)n_tok * half * 2);
   kvco_rope_table(n_tok, D, theta, cs);
@@ -1340,6 +1340,15 @@ int kvco_pca(const uint16_t* calib, uint32_t n_tok, uint32_t D, uint32_t dtype, 
       for (uint32_t b = 0; b < D; b++) C[(size_t)a * D + b] += (double)x[a] * (double)x[b];
   }
   for (size_t i = 0; i < (size_t)D * D; i++) C[i] /= (double)n_tok;
+  free(cs);
+  free(x);
+  return C;
+}
+
+int kvco_pca(const uint16_t* calib, uint32_t n_tok, uint32_t D, uint32_t dtype, int is_key,
+             double theta, float* Q, double* lambda) {
+  if (dtype != KVCO_BF16 || n_tok == 0 || D == 0 || (D & 1u)) return KVCO_INVALID;
+  double* C = second_moments(calib, n_tok, D, is_key, theta);
   double* V = (double*)malloc(sizeof(double) * D * D);
   double* w = (double*)malloc(sizeof(double) * D);
   kvco_jacobi_eigen(C, D, V, w);
@@ -1363,6 +1372,63 @@ int kvco_pca(const uint16_t* calib, uint32_t n_tok, uint32_t D, uint32_t dtype, 
     for (uint32_t k = 0; k < D; k++) Q[(size_t)k * D + j] = (float)(sign * V[(size_t)k * D + c]);
     lambda[j] = w[c];
   }
-  free(cs); free(C); free(x); free(V); free(w); free(order); free(used);
+  free(C); free(V); free(w); free(order); free(used);
+  return KVCO_OK;
+}
+
+/* ---------------------------------------------------------------------------
+ * Calibration-free bases ([Codec-Gauge] "Compression Conditions": a coordinate
+ * control run with Hadamard and DCT coordinates beside PCA/KLT; "Coordinate
+ * Controls"). Reading: the orthonormal forms with columns as components, the
+ * Hadamard matrix in Sylvester (natural) order, H[k][j] = (-1)^popcount(k & j)
+ * / sqrt(D) for D a power of two, and the DCT-II, Q[k][j] = c_j cos(pi (2k + 1)
+ * j / (2D)) with c_0 = sqrt(1/D), c_j = sqrt(2/D); both in fp64, rounded to
+ * fp32. The bit allocation ranks components by variance; in a fixed basis that
+ * is the calibration second moment of each coordinate, q_j^T C q_j.
+ * ------------------------------------------------------------------------- */
+int kvco_fixed_basis(uint32_t kind, uint32_t D, float* Q) {
+  if (D == 0) return KVCO_INVALID;
+  if (kind == KVCO_BASIS_HADAMARD) {
+    if (D & (D - 1u)) return KVCO_INVALID;
+    double inv = 1.0 / sqrt((double)D);
+    for (uint32_t k = 0; k < D; k++)
+      for (uint32_t j = 0; j < D; j++) {
+        uint32_t v = k & j, odd = 0;
+        while (v) {  /* parity of the common bits */
+          odd ^= 1u;
+          v &= v - 1u;
+        }
+        Q[(size_t)k * D + j] = (float)(odd ? -inv : inv);
+      }
+    return KVCO_OK;
+  }
+  if (kind == KVCO_BASIS_DCT) {
+    for (uint32_t j = 0; j < D; j++) {
+      double c = j == 0 ? sqrt(1.0 / (double)D) : sqrt(2.0 / (double)D);
+      for (uint32_t k = 0; k < D; k++) {
+        double ang = 3.141592653589793 * (double)((2u * k + 1u) * j) / (double)(2u * D);
+        Q[(size_t)k * D + j] = (float)(c * cos(ang));
+      }
+    }
+    return KVCO_OK;
+  }
+  return KVCO_INVALID;
+}
+
+/* lambda_j = sum_a Q[a][j] (sum_b C[a][b] Q[b][j]), a and b ascending, in fp64. */
+int kvco_basis_variances(const uint16_t* calib, uint32_t n_tok, uint32_t D, uint32_t dtype, int is_key,
+                         double theta, const float* Q, double* lambda) {
+  if (dtype != KVCO_BF16 || n_tok == 0 || D == 0 || (D & 1u)) return KVCO_INVALID;
+  double* C = second_moments(calib, n_tok, D, is_key, theta);
+  for (uint32_t j = 0; j < D; j++) {
+    double lam = 0.0;
+    for (uint32_t a = 0; a < D; a++) {
+      double s = 0.0;
+      for (uint32_t b = 0; b < D; b++) s += C[(size_t)a * D + b] * (double)Q[(size_t)b * D + j];
+      lam += (double)Q[(size_t)a * D + j] * s;
+    }
+    lambda[j] = lam;
+  }
+  free(C);
   return KVCO_OK;
 }

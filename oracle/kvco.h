@@ -101,6 +101,12 @@ int kvco_pca(const uint16_t* calib, uint32_t n_tok, uint32_t D, uint32_t dtype, 
              double theta, float* Q, double* lambda);
 int kvco_jacobi_eigen(const double* A, uint32_t n, double* V, double* w);
 
+/* Calibration-free bases and the component second moments in a given basis. */
+enum { KVCO_BASIS_HADAMARD = 1, KVCO_BASIS_DCT = 2 };
+int kvco_fixed_basis(uint32_t kind, uint32_t D, float* Q);
+int kvco_basis_variances(const uint16_t* calib, uint32_t n_tok, uint32_t D, uint32_t dtype, int is_key,
+                         double theta, const float* Q, double* lambda);
+
 float kvco_bf16_to_f32(uint16_t h);
 uint16_t kvco_f32_to_bf16(float f);
 

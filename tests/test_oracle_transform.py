@@ -324,3 +324,67 @@ def test_transform_refuses_tamper_truncation_and_plan_mismatch():
     other_w[0, 0] ^= 1
     other = oracle.Plan.from_workload(w, bases=plan.bases, widths=other_w)
     assert oracle.decode_transform(other, bytes(c))[0] == oracle.PLAN_MISMATCH
+
+
+# ------------------------------------------------- calibration-free bases (f4)
+@pytest.mark.parametrize("D", [2, 8, 64, 128])
+def test_hadamard_basis_is_sylvester_hadamard(D):
+    """Sylvester Hadamard matrix / sqrt(D), against scipy's construction; its
+    columns multiply elementwise as the XOR of their indices (Walsh functions)."""
+    import scipy.linalg
+    Q = oracle.fixed_basis(oracle.HADAMARD, D)
+    want = (scipy.linalg.hadamard(D).astype(np.float64) / np.sqrt(D)).astype(np.float32)
+    assert np.array_equal(Q, want)
+    if D == 2:
+        h = np.float32(1.0 / np.sqrt(2.0))
+        assert np.array_equal(Q, np.array([[h, h], [h, -h]], np.float32))
+    s = np.sign(Q).astype(np.int64)
+    j, l = 3 % D, (D - 1)
+    assert np.array_equal(s[:, j] * s[:, l], s[:, j ^ l])
+    assert np.abs(Q.astype(np.float64).T @ Q.astype(np.float64) - np.eye(D)).max() < 1e-6
+
+
+@pytest.mark.parametrize("D", [2, 8, 64, 128])
+def test_dct_basis_is_orthonormal_dct2(D):
+    """Q^T x is the orthonormal DCT-II of x (scipy.fft.dct, norm='ortho'); the
+    first component is the mean direction; a cosine of frequency m has all its
+    energy in component m."""
+    import scipy.fft
+    Q = oracle.fixed_basis(oracle.DCT, D).astype(np.float64)
+    M = scipy.fft.dct(np.eye(D), type=2, norm="ortho", axis=0)  # y = M x
+    assert np.abs(Q.T - M).max() < 1e-7
+    assert np.abs(Q[:, 0] - 1.0 / np.sqrt(D)).max() < 1e-7  # fp32 rounding of 1/sqrt(D)
+    m = D // 2 - 1 if D > 2 else 1
+    x = np.cos(np.pi * (2 * np.arange(D) + 1) * m / (2 * D))
+    y = Q.T @ x
+    assert abs(y[m] - np.sqrt(D / 2.0)) < 1e-5
+    assert np.abs(np.delete(y, m)).max() < 1e-5
+    assert np.abs(Q.T @ Q - np.eye(D)).max() < 1e-6
+
+
+def test_fixed_basis_refusals():
+    with pytest.raises(ValueError):
+        oracle.fixed_basis(oracle.HADAMARD, 96)  # not a power of two
+    with pytest.raises(ValueError):
+        oracle.fixed_basis(7, 8)
+
+
+@pytest.mark.parametrize("kind", [oracle.HADAMARD, oracle.DCT])
+@pytest.mark.parametrize("is_key", [True, False])
+def test_basis_variances_are_coordinate_second_moments(kind, is_key):
+    """lambda_j equals the mean of y_j^2 over the calibration tokens (y = Q^T x
+    per token, keys de-rotated) and the variances sum to the trace of C."""
+    w = dataclasses.replace(kvgen.WORKLOADS["transform-32x8x8192x128-bf16"], n_layers=1,
+                            n_heads=1)
+    cal = kvgen.calibration(w)[0 if is_key else 1][:256]
+    D = 128
+    Q = oracle.fixed_basis(kind, D)
+    lam = oracle.basis_variances(cal, is_key, w.theta, Q)
+    cs = oracle.rope_table(cal.shape[0], D, w.theta)
+    xs = np.stack([oracle.rope_inverse(cs[t], _f32(cal[t])) if is_key else _f32(cal[t])
+                   for t in range(cal.shape[0])]).astype(np.float64)
+    y = xs @ Q.astype(np.float64)
+    ref = (y ** 2).mean(axis=0)
+    assert np.allclose(lam, ref, rtol=1e-10, atol=1e-12 * ref.max())
+    trace = (xs ** 2).sum(axis=1).mean()
+    assert abs(lam.sum() - trace) < 1e-5 * trace  # fp32 basis: orthonormal to ~1e-7
