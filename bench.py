@@ -49,6 +49,19 @@ KERNEL_WORK = {
     "transform_decode": ("tensor", lambda R, C, V: 2 * 128 * V),
 }
 
+# DRAM bytes (read + write) per frame of 64 MiB, from the ncu capture summarised
+# in profiles/kernels_qwen3-32b-32k_4frames.md (one launch over 4 frames, larger
+# than L2; the traffic of these kernels grows with the frames a launch covers).
+# A kernel that changed after that capture has no entry.
+DRAM_BYTES_PER_FRAME = {
+    "transform_project": (303.8e6 + 104.0e6) / 4,
+    "lossless_encode": (759.9e6 + 353.7e6) / 4,
+    "transform_decode_codes": (82.2e6 + 94.5e6) / 4,
+    "transform_entropy": (128.5e6 + 27.9e6) / 4,
+    "lossless_decode": (198.8e6 + 220.9e6) / 4,
+    "transform_decode": (199.5e6 + 221.8e6) / 4,
+}
+
 
 def measured_peaks():
     """(HBM GB/s, sustained bf16 TFLOP/s, max SM MHz, source): the driver's
@@ -151,8 +164,11 @@ def barrier(world):
 
 
 # ------------------------------------------------------------------ the codec
+BASES = {"pca": 0, "hadamard": 1, "dct": 2}  # transform basis: calibrated PCA, or a fixed one
+
+
 class Job:
-    def __init__(self, w_l, w_t, n_frames=None):
+    def __init__(self, w_l, w_t, n_frames=None, basis="pca"):
         import torch
 
         import kvgen
@@ -172,7 +188,7 @@ class Job:
         self.x = self.host.cuda()
         t0 = time.time()
         shape_t = kvc.Shape.from_workload(w_t)
-        bases, lam = kvc.calibrate_pca(shape_t, kvgen.calibration(w_t))
+        bases, lam = kvc.calibrate_basis(shape_t, BASES[basis], kvgen.calibration(w_t))
         self.plan_t = kvc.Plan(shape_t, bases=bases, eigvals=lam)
         self.plan_l = kvc.Plan(kvc.Shape.from_workload(w_l))
         self.bases = bases
@@ -333,7 +349,7 @@ def run_kvc(args):
     world, rank, local = dist_setup()
     torch.cuda.set_device(local)
     w_l, w_t = kvgen.WORKLOADS[WORKLOAD_L], kvgen.WORKLOADS[WORKLOAD_T]
-    job = Job(w_l, w_t, n_frames=args.frames)
+    job = Job(w_l, w_t, n_frames=args.frames, basis=args.basis)
     ok = job.check()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
     for _ in range(args.warmup):
@@ -389,13 +405,15 @@ def run_kvc(args):
                 entry.update(bound=bound, achieved=round(ach, 3), peak=round(peak, 2),
                              unit="TFLOP/s", frac=round(ach / peak, 4),
                              algorithmic_flops_per_launch=int(work / n))
+        if name in DRAM_BYTES_PER_FRAME and n:
+            entry["traffic"] = int(DRAM_BYTES_PER_FRAME[name] * job.frames * args.steps / n)
         kern_out[name] = entry
     dominant = max(kern_out, key=lambda k: kern_out[k]["total_ms"]) if kern_out else None
     roof = None
     if dominant and "bound" in kern_out[dominant]:
         d = kern_out[dominant]
         roof = {"kernel": dominant, "bound": d["bound"], "achieved": d["achieved"],
-                "peak": d["peak"], "unit": d["unit"], "frac": d["frac"], "traffic": None,
+                "peak": d["peak"], "unit": d["unit"], "frac": d["frac"], "traffic": d.get("traffic"),
                 "peak_source": {"hbm": peak_kind + " copy bandwidth",
                                 "tensor": peak_kind + " sustained cuBLAS bf16",
                                 "alu": "derived: 148 SMs x 64 fp64 FMA/clk x 2 x max SM clock"}[d["bound"]]}
@@ -422,7 +440,7 @@ def run_kvc(args):
             "data": "synthetic (seeded per-channel AR(1) KV, RoPE'd keys)",
             "config": {"workload": "qwen3-32b-shaped cache 64x8x32768x128 bf16 K+V, "
                                    "128 frames of 64 MiB, lossless + transform at 1.6 bits",
-                       "raw_bytes": raw, "frames": job.frames, "frame_bytes": job.frame_bytes,
+                       "basis": args.basis, "raw_bytes": raw, "frames": job.frames, "frame_bytes": job.frame_bytes,
                        "l2": "inputs larger than L2 (8.59 GB per step)",
                        "value_definition": "4 x raw bytes per step / step time, all ranks"},
             "ops": {"lossless_encode_gbs": gbs(phase[0]), "transform_encode_gbs": gbs(phase[1]),
@@ -454,7 +472,7 @@ def run_reference(args):
     import transform_codec_b200 as kvc  # plan-time host calibration for the bases only
     w_l, w_t = kvgen.WORKLOADS[WORKLOAD_L], kvgen.WORKLOADS[WORKLOAD_T]
     shape = kvc.Shape.from_workload(w_t)
-    bases, lam = kvc.calibrate_pca(shape, kvgen.calibration(w_t))
+    bases, lam = kvc.calibrate_basis(shape, BASES[args.basis], kvgen.calibration(w_t))
     widths = kvc.allocate_bits(lam, w_t.avg_bits, w_t.max_bits).reshape(lam.shape)
     x = kvgen.slices(w_l, 0, 1)
     pl = oracle.Plan.from_workload(w_l)
@@ -500,6 +518,8 @@ def main():
     ap.add_argument("--cpu-slices", type=int, default=3)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--basis", choices=sorted(BASES), default="pca",
+                    help="transform basis: calibrated PCA (default) or a fixed Hadamard / DCT-II")
     args = ap.parse_args()
     if args.warmup < 3 and args.frames is None:
         args.warmup = 3

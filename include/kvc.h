@@ -215,6 +215,25 @@ const char* kvc_status_string(int status);
 int kvc_calibrate_pca(const kvc_plan_desc* desc, const uint16_t* h_calib, uint32_t n_calib,
                       float* h_bases, double* h_eigvals, int n_threads);
 
+/* Calibration-free bases (Codec-Gauge page, "Compression Conditions" and
+ * "Coordinate Controls": Hadamard and DCT coordinates beside PCA/KLT), fp64
+ * values rounded to fp32, element [k*D + j] = channel k of component j:
+ *   KVC_BASIS_HADAMARD  Sylvester order, (-1)^popcount(k & j) / sqrt(D);
+ *                       D must be a power of two
+ *   KVC_BASIS_DCT       orthonormal DCT-II, c_j cos(pi (2k + 1) j / (2D)),
+ *                       c_0 = sqrt(1/D), c_j = sqrt(2/D)
+ * kvc_fixed_basis writes one [D][D] basis to h_basis (host). Returns
+ * KVC_ERR_INVALID for another kind, a NULL pointer or D = 0. */
+enum { KVC_BASIS_PCA = 0, KVC_BASIS_HADAMARD = 1, KVC_BASIS_DCT = 2 };
+int kvc_fixed_basis(int kind, uint32_t D, float* h_basis);
+/* kvc_calibrate_pca for kind KVC_BASIS_PCA; otherwise the fixed basis of that
+ * kind for every slice (h_bases [L*2*H][D][D]) and, as h_eigvals, each
+ * component's second moment over the slice's calibration tokens (keys
+ * de-rotated): q_j^T C q_j with C = (1/n_calib) sum_t x_t x_t^T, fp64, sums over
+ * tokens and then channels in ascending order. Host, multithreaded over slices. */
+int kvc_calibrate_basis(const kvc_plan_desc* desc, int kind, const uint16_t* h_calib, uint32_t n_calib,
+                        float* h_bases, double* h_eigvals, int n_threads);
+
 /* Greedy bit allocation on its own (host): the widths kvc_plan_create would
  * assign. h_eigvals [n_units] (negative values count as 0), h_widths out
  * [n_units]; the budget is floor(avg_bits * n_units + 0.5) bits, each unit at

@@ -235,3 +235,31 @@ def test_transform_container_equals_oracle_bytes_extremes():
     st, got = encode(plan, kvc.TRANSFORM, x)
     assert st == kvc.OK
     assert got == oracle.encode_transform(oplan, x)
+
+
+@pytest.mark.parametrize("kind", [kvc.BASIS_HADAMARD, kvc.BASIS_DCT])
+def test_fixed_basis_container_equals_oracle_bytes(kind):
+    """Calibration-free bases: the library's bases, variances and widths feed
+    the GPU encoder; the oracle builds its own from the same calibration tokens;
+    the containers agree byte for byte and decode within the reconstruction bar
+    of the same plan on the oracle."""
+    w = _w(n_tokens=1024)
+    shape = kvc.Shape.from_workload(w)
+    cal = kvgen.calibration(w)
+    bases, lam = kvc.calibrate_basis(shape, kind, cal)
+    plan = kvc.Plan(shape, bases=bases, eigvals=lam)
+    obases = np.stack([oracle.fixed_basis(kind, w.head_dim)] * w.n_slices)
+    olam = np.stack([oracle.basis_variances(cal[s], (s // w.n_heads) % 2 == 0, w.theta, obases[s])
+                     for s in range(w.n_slices)])
+    owidths = oracle.allocate(olam, w.avg_bits, w.max_bits).reshape(olam.shape)
+    assert np.array_equal(plan.widths().reshape(owidths.shape), owidths)
+    oplan = oracle.Plan.from_workload(w, bases=obases, widths=owidths)
+    x = kvgen.slices(w)
+    st, got = encode(plan, kvc.TRANSFORM, x)
+    assert st == kvc.OK
+    assert got == oracle.encode_transform(oplan, x)
+    st, y = decode(plan, kvc.TRANSFORM, got, w.n_slices)
+    assert st == kvc.OK
+    ost, oy = oracle.decode_transform(oplan, got)
+    assert ost == oracle.OK
+    assert rel_rms(y, oy) < REL_RMS

@@ -108,3 +108,31 @@ def test_calibration_matches_oracle_pca(heads):
         sep = gap > 1e-3
         # same sign convention, so separated components agree column by column
         assert np.abs(bases[s][:, sep] - Qo[:, sep]).max() < 1e-4
+
+
+@pytest.mark.parametrize("kind", [kvc.BASIS_HADAMARD, kvc.BASIS_DCT])
+def test_fixed_basis_calibration_matches_oracle_bit_for_bit(kind):
+    """The library's calibration-free bases and component variances equal the
+    oracle's exactly (same closed forms, same fp64 sums in the same order)."""
+    for D in (8, 128):
+        a = kvc.fixed_basis(kind, D)
+        b = oracle.fixed_basis(kind, D)
+        assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+    w = dataclasses.replace(kvgen.WORKLOADS["transform-32x8x8192x128-bf16"], n_layers=1, n_heads=2)
+    shape = kvc.Shape.from_workload(w)
+    cal = kvgen.calibration(w)
+    bases, lam = kvc.calibrate_basis(shape, kind, cal)
+    for s in range(w.n_slices):
+        assert np.array_equal(bases[s], oracle.fixed_basis(kind, w.head_dim))
+        lo = oracle.basis_variances(cal[s], (s // w.n_heads) % 2 == 0, w.theta, bases[s])
+        assert np.array_equal(lam[s].view(np.uint64), lo.view(np.uint64))
+    widths = kvc.allocate_bits(lam, w.avg_bits, w.max_bits)
+    owidths = oracle.allocate(lam, w.avg_bits, w.max_bits).reshape(lam.shape)
+    assert np.array_equal(widths.reshape(lam.shape), owidths)
+
+
+def test_fixed_basis_refusals():
+    with pytest.raises(kvc.KvcError):
+        kvc.fixed_basis(kvc.BASIS_HADAMARD, 96)
+    with pytest.raises(kvc.KvcError):
+        kvc.fixed_basis(9, 8)

@@ -26,6 +26,7 @@ EXPORTS = [
     "kvc_max_encoded_bytes", "kvc_workspace_bytes",
     "kvc_encode_lossless", "kvc_decode_lossless", "kvc_encode_transform", "kvc_decode_transform",
     "kvc_status_string", "kvc_calibrate_pca", "kvc_allocate_bits",
+    "kvc_fixed_basis", "kvc_calibrate_basis",
     "kvc_stage_crc32", "kvc_stage_stream_encode", "kvc_stage_stream_decode",
     "kvc_stage_stream_encode_noalloc",
     "kvc_profile_begin", "kvc_profile_end",
@@ -84,6 +85,8 @@ def _load():
         "kvc_status_string": ([i32], ctypes.c_char_p),
         "kvc_calibrate_pca": ([ctypes.POINTER(PlanDesc), vp, u32, vp, vp, i32], i32),
         "kvc_allocate_bits": ([vp, ctypes.c_uint64, ctypes.c_double, u32, vp], i32),
+        "kvc_fixed_basis": ([i32, u32, vp], i32),
+        "kvc_calibrate_basis": ([ctypes.POINTER(PlanDesc), i32, vp, u32, vp, vp, i32], i32),
         "kvc_batch_workspace_bytes": ([vp, i32, i32, u32, u32], sz),
         "kvc_encode_batch": ([vp, i32, ctypes.POINTER(Frame), u32, vp, sz, vp], i32),
         "kvc_decode_batch": ([vp, i32, ctypes.POINTER(Frame), u32, u32, vp, sz, vp], i32),
@@ -290,6 +293,28 @@ def calibrate_pca(shape: Shape, calib: np.ndarray, n_threads: int = 0):
     desc = shape.desc()
     _check(_lib.kvc_calibrate_pca(ctypes.byref(desc), c.ctypes.data, n_calib, bases.ctypes.data,
                                   lam.ctypes.data, n_threads), "kvc_calibrate_pca")
+    return bases, lam
+
+
+BASIS_PCA, BASIS_HADAMARD, BASIS_DCT = 0, 1, 2
+
+
+def fixed_basis(kind: int, D: int) -> np.ndarray:
+    """Calibration-free basis [D][D] fp32 (Hadamard or DCT-II)."""
+    q = np.zeros((D, D), np.float32)
+    _check(_lib.kvc_fixed_basis(kind, D, q.ctypes.data), "kvc_fixed_basis")
+    return q
+
+
+def calibrate_basis(shape: Shape, kind: int, calib: np.ndarray, n_threads: int = 0):
+    """Bases [S][D][D] and component variances [S][D] for a basis kind."""
+    c = np.ascontiguousarray(calib, dtype=np.uint16)
+    S, n_calib, D = c.shape
+    bases = np.zeros((S, D, D), np.float32)
+    lam = np.zeros((S, D), np.float64)
+    desc = shape.desc()
+    _check(_lib.kvc_calibrate_basis(ctypes.byref(desc), kind, c.ctypes.data, n_calib, bases.ctypes.data,
+                                    lam.ctypes.data, n_threads), "kvc_calibrate_basis")
     return bases, lam
 
 

@@ -861,47 +861,61 @@ void sym_eigen(std::vector<double>& a, int n, std::vector<double>& w) {
 
 }  // namespace
 
+namespace {
+// Uncentered second moments C = (1/n) sum_t x_t x_t^T of slice s's calibration
+// tokens (keys de-rotated with the fp32 table cs), fp64, t ascending.
+void calib_moments(const kvc_plan_desc& d, uint32_t s, const uint16_t* h_calib, uint32_t n_calib,
+                   const std::vector<float>& cs, std::vector<double>& C) {
+  const uint32_t D = d.head_dim, half = D / 2;
+  const bool key = ((s / d.n_heads) & 1u) == 0;
+  C.assign(size_t(D) * D, 0.0);
+  std::vector<float> x(D);
+  const uint16_t* xs = h_calib + size_t(s) * n_calib * D;
+  for (uint32_t t = 0; t < n_calib; ++t) {
+    for (uint32_t k = 0; k < D; ++k) {
+      uint32_t bits = uint32_t(xs[size_t(t) * D + k]) << 16;
+      std::memcpy(&x[k], &bits, 4);
+    }
+    if (key) {
+      const float* row = cs.data() + size_t(t) * half * 2;
+      for (uint32_t i = 0; i < half; ++i) {
+        volatile float a = x[i], b = x[i + half], c = row[2 * i], sn = row[2 * i + 1];
+        volatile float ac = a * c, bs = b * sn, bc = b * c, as = a * sn;
+        x[i] = ac + bs;
+        x[i + half] = bc - as;
+      }
+    }
+    for (uint32_t a = 0; a < D; ++a) {
+      const double xa = x[a];
+      double* Ca = C.data() + size_t(a) * D;
+      for (uint32_t b = 0; b <= a; ++b) Ca[b] += xa * double(x[b]);
+    }
+  }
+  for (uint32_t a = 0; a < D; ++a)
+    for (uint32_t b = 0; b <= a; ++b) {
+      double v = C[size_t(a) * D + b] / double(n_calib);
+      C[size_t(a) * D + b] = v;
+      C[size_t(b) * D + a] = v;
+    }
+}
+
+bool calib_desc_ok(const kvc_plan_desc& d) {
+  return d.dtype == KVC_DTYPE_BF16 && d.head_dim && !(d.head_dim & 1u) && d.rope_theta > 0.0 && d.n_layers &&
+         d.n_heads;
+}
+}  // namespace
+
 extern "C" int kvc_calibrate_pca(const kvc_plan_desc* desc, const uint16_t* h_calib, uint32_t n_calib,
                                  float* h_bases, double* h_eigvals, int n_threads) {
   if (!desc || !h_calib || !h_bases || !h_eigvals || !n_calib) return KVC_ERR_INVALID;
   const kvc_plan_desc& d = *desc;
-  if (d.dtype != KVC_DTYPE_BF16 || !d.head_dim || (d.head_dim & 1u) || !(d.rope_theta > 0.0) ||
-      !d.n_layers || !d.n_heads)
-    return KVC_ERR_INVALID;
-  const uint32_t D = d.head_dim, S = d.n_layers * 2u * d.n_heads, half = D / 2;
+  if (!calib_desc_ok(d)) return KVC_ERR_INVALID;
+  const uint32_t D = d.head_dim, S = d.n_layers * 2u * d.n_heads;
   std::vector<float> cs;
   rope_table(n_calib, D, d.rope_theta, cs);
   parallel_for(S, n_workers(n_threads), [&](uint32_t s) {
-    const bool key = ((s / d.n_heads) & 1u) == 0;
-    std::vector<double> C(size_t(D) * D, 0.0);
-    std::vector<float> x(D);
-    const uint16_t* xs = h_calib + size_t(s) * n_calib * D;
-    for (uint32_t t = 0; t < n_calib; ++t) {
-      for (uint32_t k = 0; k < D; ++k) {
-        uint32_t bits = uint32_t(xs[size_t(t) * D + k]) << 16;
-        std::memcpy(&x[k], &bits, 4);
-      }
-      if (key) {
-        const float* row = cs.data() + size_t(t) * half * 2;
-        for (uint32_t i = 0; i < half; ++i) {
-          volatile float a = x[i], b = x[i + half], c = row[2 * i], sn = row[2 * i + 1];
-          volatile float ac = a * c, bs = b * sn, bc = b * c, as = a * sn;
-          x[i] = ac + bs;
-          x[i + half] = bc - as;
-        }
-      }
-      for (uint32_t a = 0; a < D; ++a) {
-        const double xa = x[a];
-        double* Ca = C.data() + size_t(a) * D;
-        for (uint32_t b = 0; b <= a; ++b) Ca[b] += xa * double(x[b]);
-      }
-    }
-    for (uint32_t a = 0; a < D; ++a)
-      for (uint32_t b = 0; b <= a; ++b) {
-        double v = C[size_t(a) * D + b] / double(n_calib);
-        C[size_t(a) * D + b] = v;
-        C[size_t(b) * D + a] = v;
-      }
+    std::vector<double> C;
+    calib_moments(d, s, h_calib, n_calib, cs, C);
     std::vector<double> w;
     sym_eigen(C, int(D), w);
     std::vector<uint32_t> order(D);
@@ -916,6 +930,59 @@ extern "C" int kvc_calibrate_pca(const kvc_plan_desc* desc, const uint16_t* h_ca
       const double sign = C[size_t(arg) * D + c] < 0.0 ? -1.0 : 1.0;
       for (uint32_t k = 0; k < D; ++k) Q[size_t(k) * D + j] = float(sign * C[size_t(k) * D + c]);
       h_eigvals[size_t(s) * D + j] = w[c];
+    }
+  });
+  return KVC_OK;
+}
+
+extern "C" int kvc_fixed_basis(int kind, uint32_t D, float* h_basis) {
+  if (!h_basis || !D) return KVC_ERR_INVALID;
+  if (kind == KVC_BASIS_HADAMARD) {
+    if (D & (D - 1u)) return KVC_ERR_INVALID;
+    const double inv = 1.0 / std::sqrt(double(D));
+    for (uint32_t k = 0; k < D; ++k)
+      for (uint32_t j = 0; j < D; ++j)
+        h_basis[size_t(k) * D + j] = float((__builtin_popcount(k & j) & 1) ? -inv : inv);
+    return KVC_OK;
+  }
+  if (kind == KVC_BASIS_DCT) {
+    const double pi = 3.141592653589793;
+    for (uint32_t j = 0; j < D; ++j) {
+      const double c = j == 0 ? std::sqrt(1.0 / double(D)) : std::sqrt(2.0 / double(D));
+      for (uint32_t k = 0; k < D; ++k) {
+        const double ang = pi * double((2u * k + 1u) * j) / double(2u * D);
+        h_basis[size_t(k) * D + j] = float(c * std::cos(ang));
+      }
+    }
+    return KVC_OK;
+  }
+  return KVC_ERR_INVALID;
+}
+
+extern "C" int kvc_calibrate_basis(const kvc_plan_desc* desc, int kind, const uint16_t* h_calib,
+                                   uint32_t n_calib, float* h_bases, double* h_eigvals, int n_threads) {
+  if (kind == KVC_BASIS_PCA) return kvc_calibrate_pca(desc, h_calib, n_calib, h_bases, h_eigvals, n_threads);
+  if (!desc || !h_calib || !h_bases || !h_eigvals || !n_calib) return KVC_ERR_INVALID;
+  const kvc_plan_desc& d = *desc;
+  if (!calib_desc_ok(d)) return KVC_ERR_INVALID;
+  const uint32_t D = d.head_dim, S = d.n_layers * 2u * d.n_heads;
+  std::vector<float> Q(size_t(D) * D);
+  const int st = kvc_fixed_basis(kind, D, Q.data());
+  if (st != KVC_OK) return st;
+  std::vector<float> cs;
+  rope_table(n_calib, D, d.rope_theta, cs);
+  parallel_for(S, n_workers(n_threads), [&](uint32_t s) {
+    std::vector<double> C;
+    calib_moments(d, s, h_calib, n_calib, cs, C);
+    std::memcpy(h_bases + size_t(s) * D * D, Q.data(), sizeof(float) * D * D);
+    for (uint32_t j = 0; j < D; ++j) {  // q_j^T C q_j, a and b ascending
+      double lam = 0.0;
+      for (uint32_t a = 0; a < D; ++a) {
+        double acc = 0.0;
+        for (uint32_t b = 0; b < D; ++b) acc += C[size_t(a) * D + b] * double(Q[size_t(b) * D + j]);
+        lam += double(Q[size_t(a) * D + j]) * acc;
+      }
+      h_eigvals[size_t(s) * D + j] = lam;
     }
   });
   return KVC_OK;
