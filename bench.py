@@ -54,7 +54,6 @@ KERNEL_WORK = {
 # than L2; the traffic of these kernels grows with the frames a launch covers).
 # A kernel that changed after that capture has no entry.
 DRAM_BYTES_PER_FRAME = {
-    "transform_project": (303.8e6 + 104.0e6) / 4,
     "lossless_encode": (759.9e6 + 353.7e6) / 4,
     "transform_decode_codes": (82.2e6 + 94.5e6) / 4,
     "transform_entropy": (128.5e6 + 27.9e6) / 4,

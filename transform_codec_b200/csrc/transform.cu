@@ -325,6 +325,9 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
   uint8_t* rec = ws.slots + uint64_t(r) * ws.slot_bytes;
   uint8_t* codes = slot_codes(rec, ws.slot_bytes);
 
+  // the first tile's rows are requested first, so they land while the basis loads
+  XFetch xf;
+  xf.load(xs, pl.rope, is_key, t0, 0, min(kProjTokens, tcc));
   load_comp_info(pl.comp + sidx, S.ci);
   if (tid < kD && S.ci.width[tid]) S.cidx[S.ci.coded_idx[tid]] = tid;
   for (uint32_t i = tid; i < kTabPool; i += nthr) S.hist[i] = 0;
@@ -338,23 +341,23 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
     uint32_t col[4];
 #pragma unroll
     for (uint32_t u = 0; u < 4; ++u) col[u] = lane + 32u * u < nc ? S.cidx[lane + 32u * u] : 0u;
-    for (uint32_t k0 = warp; k0 < kD; k0 += 4u * (nthr >> 5)) {
-      float v[4][4];
+    // all of this thread's rows are requested before any is stored (one latency)
+    constexpr uint32_t kRows = kD / (kThreads / 32u);
+    float v[kRows][4];
 #pragma unroll
-      for (uint32_t kk = 0; kk < 4; ++kk)
+    for (uint32_t kk = 0; kk < kRows; ++kk)
 #pragma unroll
-        for (uint32_t u = 0; u < 4; ++u) {
-          const uint32_t k = k0 + kk * (nthr >> 5);
-          v[kk][u] = (k < kD && lane + 32u * u < nc) ? __ldg(q + k * kD + col[u]) : 0.0f;
-        }
+      for (uint32_t u = 0; u < 4; ++u) {
+        const uint32_t k = warp + kk * (kThreads / 32u);
+        v[kk][u] = lane + 32u * u < nc ? __ldg(q + k * kD + col[u]) : 0.0f;
+      }
 #pragma unroll
-      for (uint32_t kk = 0; kk < 4; ++kk)
+    for (uint32_t kk = 0; kk < kRows; ++kk)
 #pragma unroll
-        for (uint32_t u = 0; u < 4; ++u) {
-          const uint32_t k = k0 + kk * (nthr >> 5);
-          if (k < kD && lane + 32u * u < nc) S.Qd[k * kD + lane + 32u * u] = double(v[kk][u]);
-        }
-    }
+      for (uint32_t u = 0; u < 4; ++u) {
+        const uint32_t k = warp + kk * (kThreads / 32u);
+        if (lane + 32u * u < nc) S.Qd[k * kD + lane + 32u * u] = double(v[kk][u]);
+      }
   }
   // side-information padding of the record (its values are written below)
   const uint32_t side = 8u * nc * nb;
@@ -367,8 +370,6 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
   uint32_t cnt[8][2];  // per jb: counts of symbols 0..3 and 4..7 of this thread's codes, a byte each
 #pragma unroll
   for (uint32_t jb = 0; jb < 8; ++jb) cnt[jb][0] = cnt[jb][1] = 0;
-  XFetch xf;
-  xf.load(xs, pl.rope, is_key, t0, 0, min(kProjTokens, tcc));
   for (uint32_t tb = 0; tb < tcc; tb += kProjTokens) {
     const uint32_t bl = min(kProjTokens, tcc - tb);
     xf.stage(S.x, is_key);
