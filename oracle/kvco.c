@@ -839,10 +839,13 @@ uint32_t kvco_plan_crc(const kvco_desc* d) {
  *     the chunk start, last may be shorter): z = min y, s = fl(max - min) /
  *     (2^b - 1) in fp32 (0 if max == min);
  *     code = clamp(rint_even(fl(fl(y - z) / s)), 0, 2^b - 1), 0 if s == 0;
- *   record: side info (for j ascending with b_j > 0, for each block: z, s as
- *     fp32) zero padded to 16, then for b = 1..8 with m_b > 0 components one
- *     stream of m_b * tc codes (components ascending, each component's tokens in
- *     order) in the stream record format above.
+ *   record: the side information as four stream records, then for b = 1..8
+ *     with m_b > 0 components one stream of m_b * tc codes (components
+ *     ascending, each component's tokens in order) in the stream record format
+ *     above. The side information is the sequence V of 2 * coded * nb fp32
+ *     values: every z (for j ascending with b_j > 0, for each block), then
+ *     every s in the same order; stream p (p = 0..3) holds byte p of each value
+ *     of V and may take the lane delta (no side streams when nothing is coded).
  *   decode: y^ = fmaf(code, s, z) (0 for b_j = 0); x^_k = (float) sum_j
  *     (double) Q[k][j] * (double) y^_j in fp64; keys: forward rotation;
  *     bf16 round-to-nearest-even.
@@ -883,12 +886,20 @@ static uint32_t count_width(const uint8_t* w, uint32_t D, uint32_t b) {
 static size_t mid_record_bound(const kvco_desc* d, const uint8_t* w, uint32_t tcc) {
   uint32_t nb = (tcc + d->block_tokens - 1) / d->block_tokens;
   uint32_t coded = d->head_dim - count_width(w, d->head_dim, 0);
-  size_t bytes = pad16((size_t)8 * coded * nb);
+  size_t bytes = coded ? 4u * (16u + pad16((size_t)2 * coded * nb)) : 0u;  /* side streams at most RAW */
   for (uint32_t b = 1; b <= 8; b++) {
     uint32_t m = count_width(w, d->head_dim, b);
     if (m) bytes += 16u + pad16((size_t)m * tcc);
   }
   return bytes;
+}
+
+/* Bytes of the parser's scratch: a stream of codes (ct * D) or the four side
+ * planes (8 * D * ct / B). */
+static size_t parse_buf_bytes(const kvco_desc* d) {
+  size_t a = (size_t)d->chunk_tokens * d->head_dim;
+  size_t b = (size_t)8 * d->head_dim * (d->chunk_tokens / d->block_tokens);
+  return a > b ? a : b;
 }
 
 size_t kvco_transform_bound(const kvco_desc* d, uint32_t n_slices) {
@@ -1008,8 +1019,9 @@ size_t kvco_encode_transform(const kvco_desc* d, uint32_t first_slice, uint32_t 
   kvco_rope_table(T, D, d->rope_theta, cs);
   float* y = (float*)malloc(sizeof(float) * (size_t)ct * D);
   uint8_t* codes = (uint8_t*)malloc((size_t)ct * D);
-  uint8_t* syms = (uint8_t*)malloc((size_t)ct * D);
+  uint8_t* syms = (uint8_t*)malloc(parse_buf_bytes(d));
   float* zs = (float*)malloc(sizeof(float) * (size_t)D * nbmax * 2);
+  uint8_t* side = (uint8_t*)malloc((size_t)4 * 2 * D * nbmax);  /* four byte planes of V */
   size_t p = HDR_BYTES + (size_t)IDX_ENTRY * nr;
   uint32_t r = 0;
   for (uint32_t s = 0; s < n_slices; s++) {
@@ -1036,18 +1048,19 @@ size_t kvco_encode_transform(const kvco_desc* d, uint32_t first_slice, uint32_t 
       uint32_t nb = (tcc + B - 1) / B;
       mid_chunk_quantize(d, sidx, xs, cs, t0, tcc, y, codes, NULL, zs);
       start = p;
-      for (uint32_t j = 0; j < D; j++) {
-        if (!w[j]) continue;
-        for (uint32_t blk = 0; blk < nb; blk++) {
-          uint32_t zb, sb;
-          memcpy(&zb, &zs[((size_t)j * nbmax + blk) * 2], 4);
-          memcpy(&sb, &zs[((size_t)j * nbmax + blk) * 2 + 1], 4);
-          put32(dst + p, zb);
-          put32(dst + p + 4, sb);
-          p += 8;
+      /* side information: V = every z, then every s, split into byte planes */
+      uint32_t coded = D - count_width(w, D, 0), nv = 2u * coded * nb, i = 0;
+      for (uint32_t half_v = 0; half_v < 2; half_v++)
+        for (uint32_t j = 0; j < D; j++) {
+          if (!w[j]) continue;
+          for (uint32_t blk = 0; blk < nb; blk++, i++) {
+            uint32_t v;
+            memcpy(&v, &zs[((size_t)j * nbmax + blk) * 2 + half_v], 4);
+            for (uint32_t q = 0; q < 4; q++) side[(size_t)q * nv + i] = (uint8_t)(v >> (8u * q));
+          }
         }
-      }
-      while (p & 15u) dst[p++] = 0;
+      if (nv)
+        for (uint32_t q = 0; q < 4; q++) p += kvco_stream_encode_delta(side + (size_t)q * nv, nv, dst + p);
       for (uint32_t b = 1; b <= 8; b++) {
         uint32_t m = 0;
         for (uint32_t j = 0; j < D; j++) {
@@ -1063,7 +1076,7 @@ size_t kvco_encode_transform(const kvco_desc* d, uint32_t first_slice, uint32_t 
       put32(e + 12, kvco_crc32(dst + start, p - start));
     }
   }
-  free(cs); free(y); free(codes); free(syms); free(zs);
+  free(cs); free(y); free(codes); free(syms); free(zs); free(side);
   write_header(dst, KVCO_TRANSFORM, d, first_slice, n_slices, ct, nr, p, kvco_plan_crc(d));
   put32(dst + 60, header_crc(dst, nr));
   return p;
@@ -1075,23 +1088,30 @@ static int mid_chunk_parse(const kvco_desc* d, uint32_t sidx, const uint8_t* rec
   uint32_t D = d->head_dim, ct = d->chunk_tokens, B = d->block_tokens, nbmax = ct / B;
   const uint8_t* w = d->widths + (size_t)sidx * D;
   uint32_t nb = (tcc + B - 1) / B;
-  uint32_t coded = D - count_width(w, D, 0);
-  size_t side = pad16((size_t)8 * coded * nb);
-  if (side > len) return KVCO_CORRUPT;
+  uint32_t coded = D - count_width(w, D, 0), nv = 2u * coded * nb;
   size_t p = 0;
+  /* side streams: byte q of every value of V (the syms buffer holds ct * D >= 4 nv bytes) */
+  for (uint32_t q = 0; q < 4 && nv; q++) {
+    size_t used = 0;
+    int st = stream_decode(rec + p, len - p, nv, syms + (size_t)q * nv, &used, 1);
+    if (st) return st;
+    p += used;
+  }
+  uint32_t i = 0;
   for (uint32_t j = 0; j < D; j++) {
     for (uint32_t blk = 0; blk < nbmax; blk++)
       zs[((size_t)j * nbmax + blk) * 2] = zs[((size_t)j * nbmax + blk) * 2 + 1] = 0.0f;
     memset(codes + (size_t)j * ct, 0, ct);
-    if (!w[j]) continue;
-    for (uint32_t blk = 0; blk < nb; blk++) {
-      uint32_t zb = get32(rec + p), sb = get32(rec + p + 4);
-      memcpy(&zs[((size_t)j * nbmax + blk) * 2], &zb, 4);
-      memcpy(&zs[((size_t)j * nbmax + blk) * 2 + 1], &sb, 4);
-      p += 8;
-    }
   }
-  p = side;
+  for (uint32_t half_v = 0; half_v < 2; half_v++)
+    for (uint32_t j = 0; j < D; j++) {
+      if (!w[j]) continue;
+      for (uint32_t blk = 0; blk < nb; blk++, i++) {
+        uint32_t v = 0;
+        for (uint32_t q = 0; q < 4; q++) v |= (uint32_t)syms[(size_t)q * nv + i] << (8u * q);
+        memcpy(&zs[((size_t)j * nbmax + blk) * 2 + half_v], &v, 4);
+      }
+    }
   for (uint32_t b = 1; b <= 8; b++) {
     uint32_t m = count_width(w, D, b);
     if (!m) continue;
@@ -1132,7 +1152,7 @@ int kvco_decode_transform(const kvco_desc* d, const uint8_t* src, size_t n, uint
   float* cs = (float*)malloc(sizeof(float) * (size_t)T * half * 2);
   kvco_rope_table(T, D, d->rope_theta, cs);
   uint8_t* codes = (uint8_t*)malloc((size_t)ct * D);
-  uint8_t* syms = (uint8_t*)malloc((size_t)ct * D);
+  uint8_t* syms = (uint8_t*)malloc(parse_buf_bytes(d));
   float* zs = (float*)malloc(sizeof(float) * (size_t)D * nbmax * 2);
   float* yh = (float*)malloc(sizeof(float) * D);
   float* xh = (float*)malloc(sizeof(float) * D);
@@ -1223,7 +1243,7 @@ int kvco_record_codes(const kvco_desc* d, uint32_t sidx, const uint8_t* rec, uin
     return KVCO_INVALID;
   uint32_t D = d->head_dim, ct = d->chunk_tokens;
   uint8_t* cc = (uint8_t*)malloc((size_t)ct * D);
-  uint8_t* syms = (uint8_t*)malloc((size_t)ct * D);
+  uint8_t* syms = (uint8_t*)malloc(parse_buf_bytes(d));
   int st = mid_chunk_parse(d, sidx, rec, len, tcc, cc, zs, syms);
   for (uint32_t t = 0; t < tcc && !st; t++)
     for (uint32_t j = 0; j < D; j++) codes[(size_t)t * D + j] = cc[(size_t)j * ct + t];
@@ -1248,7 +1268,7 @@ int kvco_container_codes(const kvco_desc* d, const uint8_t* src, size_t n, uint3
   regions(d, &s_end, &r_start);
   uint32_t nm = n_mid_chunks(d);
   uint8_t* cc = (uint8_t*)malloc((size_t)ct * D);
-  uint8_t* syms = (uint8_t*)malloc((size_t)ct * D);
+  uint8_t* syms = (uint8_t*)malloc(parse_buf_bytes(d));
   memset(codes, 0, (size_t)ns * T * D);
   uint32_t r = 0;
   for (uint32_t s = 0; s < ns && !st; s++) {

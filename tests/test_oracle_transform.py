@@ -388,3 +388,26 @@ def test_basis_variances_are_coordinate_second_moments(kind, is_key):
     assert np.allclose(lam, ref, rtol=1e-10, atol=1e-12 * ref.max())
     trace = (xs ** 2).sum(axis=1).mean()
     assert abs(lam.sum() - trace) < 1e-5 * trace  # fp32 basis: orthonormal to ~1e-7
+
+
+def test_side_information_streams_layout():
+    """A middle record opens with four stream records: byte plane q (low to high)
+    of V = every z, then every s (coded components ascending, blocks in order),
+    each coded with the lane-delta candidate; the code streams follow. Also: the
+    side streams of the AR(1) workload are smaller than the raw fp32 values."""
+    w = _workload(n_tokens=1024)
+    plan = _pca_plan(w)
+    x = kvgen.slices(w)
+    c = oracle.encode_transform(plan, x)
+    _, _, zs = oracle.transform_slice_codes(plan, 0, x[0])
+    coded = np.flatnonzero(plan.widths.reshape(w.n_slices, 128)[0])
+    entries = np.frombuffer(c, dtype=np.uint8)[64:64 + 16 * 3].reshape(3, 16)
+    off = int(entries[1, :8].view(np.uint64)[0])
+    length = int(entries[1, 8:12].view(np.uint32)[0])
+    nb = 8  # first middle chunk: 512 tokens
+    V = np.concatenate([zs[0][coded, :nb, 0].reshape(-1), zs[0][coded, :nb, 1].reshape(-1)]).astype(np.float32)
+    planes = V.view(np.uint32)
+    want = b"".join(oracle.stream_encode_delta(((planes >> (8 * q)) & 0xFF).astype(np.uint8))
+                    for q in range(4))
+    assert c[off:off + len(want)] == want
+    assert len(want) < 4 * (16 + V.size) and len(want) < length

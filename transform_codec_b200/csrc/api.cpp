@@ -120,7 +120,8 @@ uint64_t mid_record_bound(const uint8_t* w, uint32_t D, uint32_t tcc, uint32_t b
     coded += w[j] > 0;
     m[w[j]]++;
   }
-  uint64_t b = pad16u(8ull * coded * nb);
+  // side information: four byte-plane streams of 2 * coded * nb values, each at most RAW
+  uint64_t b = coded ? 4ull * (16 + pad16u(2ull * coded * nb)) : 0ull;
   for (uint32_t k = 1; k <= 8; ++k)
     if (m[k]) b += 16 + pad16u(uint64_t(m[k]) * tcc);
   return b;

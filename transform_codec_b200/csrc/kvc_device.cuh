@@ -39,6 +39,13 @@ __host__ __device__ inline void lane_range(uint32_t n, uint32_t N, uint32_t l, u
   len = base + (l < extra ? 1u : 0u);
   start = l * base + (l < extra ? l : extra);
 }
+// Whether stream index i starts a rANS lane (lanes of a stream of n symbols on N lanes).
+__device__ inline bool lane_start(uint32_t i, uint32_t n, uint32_t N) {
+  const uint32_t base = n / N, extra = n - base * N;
+  const uint32_t big = extra * (base + 1u);
+  return i < big ? (i % (base + 1u)) == 0u : ((i - big) % base) == 0u;
+}
+
 __host__ __device__ inline uint32_t rans_groups(uint32_t N) {
   return (N + kGroupLanes - 1) / kGroupLanes;
 }

@@ -52,13 +52,6 @@ struct ChanMajor {
   }
 };
 
-// Whether stream index i starts a rANS lane (lanes of a stream of n symbols on N lanes).
-__device__ inline bool lane_start(uint32_t i, uint32_t n, uint32_t N) {
-  const uint32_t base = n / N, extra = n - base * N;
-  const uint32_t big = extra * (base + 1u);
-  return i < big ? (i % (base + 1u)) == 0u : ((i - big) % base) == 0u;
-}
-
 __global__ void __launch_bounds__(kEncThreads)
 k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws, uint32_t tail_only) {
   extern __shared__ __align__(16) uint8_t smem_raw[];

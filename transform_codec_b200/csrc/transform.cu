@@ -416,6 +416,174 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
 }
 
 // ---------------------------------------------------------------------------
+// Transform encode, part 1b (k_transform_side): one CTA per middle record. The
+// projection leaves the record's side information raw at the start of the
+// slot's record area: (z, s) of coded component cc and block blk at 8 (cc nb +
+// blk). It becomes the sequence V = every z, then every s (components and
+// blocks in order), and V's four byte planes become four stream records with
+// the lane-delta candidate (the lossless rule: CONST for one symbol; the lane
+// deltas' RANS record if strictly smaller than both the plain RANS record and
+// RAW; else plain RANS if smaller than RAW; else RAW). They replace the raw
+// values, and their total length goes to rec_len, where the entropy kernel
+// finds the offset of its code streams.
+constexpr uint32_t kSideMax = 2u * kD * (kMaxCt / kTile);  // values of V at most
+
+struct __align__(16) SideSmem {
+  uint8_t sym[4][kSideMax];                // byte plane q of V
+  uint32_t hist[8][256], freq[8][256], rem[8][256];  // variant 2q: plane q; 2q + 1: its lane deltas
+  uint2 tab[8][256];
+  uint32_t states[8][4];                   // at most 4 lanes (one group)
+  uint32_t W[8][4], wbeg[8][4], sub_len[8][4], k[8];
+  uint32_t mode[4], bytes[4], var[4], off[5];
+  uint32_t tmp[32];
+  CompInfo ci;
+};
+
+// One rANS group (lanes l < N <= 32) of a stream of n symbols sym(i), with the
+// encode table tab[s] = {f | cum << 16, floor((2^32 - 1) / f)}; words go
+// backwards into words[0, cap); returns their count (the steps and the word
+// placement of rans_encode_group).
+template <class SymFn>
+__device__ inline uint32_t side_encode_group(SymFn sym, uint32_t n, uint32_t N, const uint2* tab, uint16_t* words,
+                                             uint32_t cap, uint32_t* x_out) {
+  const uint32_t lane = threadIdx.x & 31u;
+  const bool live = lane < N;
+  uint32_t start = 0, len = 0, start0, maxlen;
+  if (live) lane_range(n, N, lane, start, len);
+  lane_range(n, N, 0u, start0, maxlen);
+  uint32_t x = kRansLow, pos = cap;
+  const uint32_t lt = lanemask_lt();
+  for (uint32_t tau = maxlen; tau-- > 0;) {
+    const bool act = live && tau < len;
+    const uint2 e = tab[act ? sym(start + tau) : 0u];
+    const uint32_t f = e.x & 0xffffu, cum = e.x >> 16;
+    const bool emit = act && x >= (f << 20);
+    const uint32_t mask = __ballot_sync(0xffffffffu, emit);
+    pos -= __popc(mask);
+    if (emit) words[pos + __popc(mask & lt)] = uint16_t(x & 0xffffu);
+    const uint32_t xe = emit ? (x >> 16) : x;
+    uint32_t q = __umulhi(xe, e.y);
+    uint32_t r = xe - q * f;
+    const bool over = r >= f;
+    q += over ? 1u : 0u;
+    r -= over ? f : 0u;
+    x = act ? (q << kProbBits) + r + cum : x;
+  }
+  *x_out = x;
+  return cap - pos;
+}
+
+__global__ void __launch_bounds__(kThreads)
+k_transform_side(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLayout ws) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  SideSmem& S = *reinterpret_cast<SideSmem*>(smem_raw);
+  const uint32_t tid = threadIdx.x, nthr = blockDim.x;
+  const uint32_t warp = tid >> 5, lane = tid & 31u;
+  const uint32_t rps = 1u + sh.n_mid;
+  const uint32_t gs = blockIdx.x / sh.n_mid, c = blockIdx.x % sh.n_mid;
+  const uint32_t r = gs * rps + 1u + c;
+  const uint32_t fr = frame_of(b.rec_base, b.n, r);
+  const uint32_t ls = (r - b.rec_base[fr]) / rps;
+  const uint32_t sidx = b.f[fr].first_slice + ls;
+  const uint32_t t0 = sh.s_end + c * sh.ct, tcc = min(sh.ct, sh.r_start - t0);
+  const uint32_t nb = (tcc + kTile - 1) / kTile;
+  uint8_t* rec = ws.slots + uint64_t(r) * ws.slot_bytes;
+  uint16_t* scratch = slot_words(rec, ws.slot_bytes);  // variant v's words at v * kSideMax
+  load_comp_info(pl.comp + sidx, S.ci);
+  const uint32_t half = S.ci.n_coded * nb, n = 2u * half;
+  if (n == 0) {  // nothing coded: no side streams
+    if (tid == 0) ws.rec_len[r] = 0;
+    return;
+  }
+  for (uint32_t i = tid; i < 8u * 256u; i += nthr) (&S.hist[0][0])[i] = 0;
+  for (uint32_t i = tid; i < half; i += nthr) {
+    const uint2 v = *reinterpret_cast<const uint2*>(rec + 8u * i);  // (z, s) of pair i
+#pragma unroll
+    for (uint32_t q = 0; q < 4; ++q) {
+      S.sym[q][i] = uint8_t(v.x >> (8u * q));
+      S.sym[q][half + i] = uint8_t(v.y >> (8u * q));
+    }
+  }
+  __syncthreads();  // the raw values are in shared memory; the records may overwrite them
+  const uint32_t N = rans_lanes(n);  // at most 4 lanes: one group
+  for (uint32_t i = tid; i < n; i += nthr) {
+    const bool first = lane_start(i, n, N);
+#pragma unroll
+    for (uint32_t q = 0; q < 4; ++q) {
+      const uint32_t v = S.sym[q][i];
+      atomicAdd(&S.hist[2 * q][v], 1u);
+      atomicAdd(&S.hist[2 * q + 1][first ? v : v ^ S.sym[q][i - 1]], 1u);
+    }
+  }
+  __syncthreads();
+  // warp v: the table of variant v and, when it can be chosen, its words
+  {
+    const uint32_t v = warp, q = v >> 1;
+    const uint32_t kv = warp_normalize(S.hist[v], 256u, n, S.freq[v], S.rem[v], S.tab[v]);
+    const uint32_t kp = __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane] ? 1u : 0u) +
+                        __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane + 32u] ? 1u : 0u) +
+                        __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane + 64u] ? 1u : 0u) +
+                        __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane + 96u] ? 1u : 0u) +
+                        __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane + 128u] ? 1u : 0u) +
+                        __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane + 160u] ? 1u : 0u) +
+                        __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane + 192u] ? 1u : 0u) +
+                        __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane + 224u] ? 1u : 0u);
+    if (lane == 0) S.k[v] = kv;
+    if (kp >= 2 && kv >= 2) {  // the lane deltas only compete with a plain RANS record
+      const uint8_t* sy = S.sym[q];
+      uint32_t x, Wg;
+      if ((v & 1u) == 0)
+        Wg = side_encode_group([sy](uint32_t i) -> uint32_t { return sy[i]; }, n, N, S.tab[v],
+                               scratch + v * kSideMax, n, &x);
+      else
+        Wg = side_encode_group(
+            [sy, n, N](uint32_t i) -> uint32_t {
+              return lane_start(i, n, N) ? uint32_t(sy[i]) : uint32_t(sy[i] ^ sy[i - 1]);
+            },
+            n, N, S.tab[v], scratch + v * kSideMax, n, &x);
+      if (lane < N) S.states[v][lane] = x;
+      if (lane == 0) {
+        S.W[v][0] = Wg;
+        S.wbeg[v][0] = v * kSideMax + n - Wg;
+      }
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {  // per plane: CONST; lane-delta RANS if strictly smaller than plain RANS and RAW; RANS; RAW
+    const uint32_t raw_b = 16u + pad16(n);
+    uint32_t off = 0;
+    for (uint32_t q = 0; q < 4; ++q) {
+      const uint32_t kp = S.k[2 * q], kd = S.k[2 * q + 1];
+      uint32_t mode = kModeRaw, bytes = raw_b, var = 2 * q;
+      if (kp == 1) {
+        mode = kModeConst;
+        bytes = 16;
+      } else if (kp >= 2) {
+        const uint32_t rb = rans_layout(n, kp, S.W[2 * q], S.sub_len[2 * q]);
+        const uint32_t rd = kd >= 2 ? rans_layout(n, kd, S.W[2 * q + 1], S.sub_len[2 * q + 1]) : 0xffffffffu;
+        if (rd < rb && rd < raw_b) {
+          mode = kModeRans; bytes = rd; var = 2 * q + 1;
+        } else if (rb < raw_b) {
+          mode = kModeRans; bytes = rb;
+        }
+      }
+      S.mode[q] = mode; S.bytes[q] = bytes; S.var[q] = var; S.off[q] = off;
+      off += bytes;
+    }
+    S.off[4] = off;
+  }
+  __syncthreads();
+  for (uint32_t q = 0; q < 4; ++q) {
+    const uint32_t v = S.var[q];
+    const uint8_t* sy = S.sym[q];
+    block_write_stream(rec + S.off[q], S.mode[q], n, S.bytes[q], uint32_t(sy[0]), S.k[v], S.freq[v], S.states[v],
+                       scratch, S.wbeg[v], S.W[v], S.sub_len[v], [sy](uint32_t i) -> uint32_t { return sy[i]; },
+                       S.tmp, v & 1u);
+  }
+  if (tid == 0) ws.rec_len[r] = S.off[4];
+}
+
+// ---------------------------------------------------------------------------
 // Transform encode, part 2 (k_transform_entropy): one CTA per middle record,
 // several per SM (no codes in shared memory). Warp w owns the stream of width
 // b = w + 1: it normalises the stream's counts and builds its coding tables.
@@ -488,11 +656,11 @@ k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
   const uint32_t ls = (r - b.rec_base[fr]) / rps;
   const uint32_t sidx = b.f[fr].first_slice + ls;
   const uint32_t t0 = sh.s_end + c * sh.ct, tcc = min(sh.ct, sh.r_start - t0);
-  const uint32_t nb = (tcc + kTile - 1) / kTile;
   uint8_t* rec = ws.slots + uint64_t(r) * ws.slot_bytes;
   const uint8_t* codes_g = slot_codes(rec, ws.slot_bytes);
   uint16_t* scratch = slot_words(rec, ws.slot_bytes);
 
+  const uint32_t side_len = __ldcg(&ws.rec_len[r]);  // written by k_transform_side
   crc_tables_init(S.crc_t);
   load_comp_info(pl.comp + sidx, S.ci);
   for (uint32_t i = tid; i < kTabPool; i += nthr)
@@ -545,9 +713,8 @@ k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
   }
   __syncthreads();
   // ---- layout: modes and record offsets
-  const uint32_t side = 8u * S.ci.n_coded * nb;
   if (tid == 0) {
-    uint32_t off = pad16(side);
+    uint32_t off = side_len;  // the side streams come first
     for (uint32_t bw = 1; bw <= 8; ++bw) {
       S.off[bw - 1] = off;
       const uint32_t m = S.ci.bcount[bw];
@@ -641,18 +808,20 @@ constexpr uint32_t kCodeRow = kD;  // bytes of a code block's token row
 struct CodeBlocks {
   uint32_t* status;  // per record of the batch: kOk when the code block is complete
   uint8_t* codes;    // per record of the batch: ct token rows of kCodeRow bytes
+  float2* zs;        // per record of the batch: (z, s) of coded component cc, block blk at cc * (ct / kTile) + blk
 };
-__device__ inline CodeBlocks code_blocks(uint8_t* ws, uint32_t max_records) {
+__device__ inline CodeBlocks code_blocks(uint8_t* ws, uint32_t max_records, uint32_t ct) {
   uint8_t* p = ws + kDecodeWsFixed + ((8ull * max_records + 255u) & ~255ull);
   CodeBlocks c;
   c.status = reinterpret_cast<uint32_t*>(p);
   c.codes = p + ((4ull * max_records + 255u) & ~255ull);
+  c.zs = reinterpret_cast<float2*>(c.codes + uint64_t(max_records) * ct * kCodeRow);
   return c;
 }
 
 struct __align__(16) DecEntSmem {
   uint8_t lut[8][kProbScale];          // per width stream: symbol of each slot
-  uint16_t ring[kThreads / 32][1024];  // one refill window per warp
+  alignas(16) uint16_t ring[kThreads / 32][1024];  // one refill window per warp (cp.async targets)
   uint32_t crc_t[1024];
   uint32_t freq[8][256];               // per width stream; f << 16 | cum after the table build
   uint32_t tmp[32], red[32];
@@ -661,6 +830,8 @@ struct __align__(16) DecEntSmem {
   CompInfo ci;
   uint32_t base[kBatchMax + 1];
   uint32_t crc_ok, bad, walk_ok;
+  uint8_t side[4][kSideMax];           // the side streams' byte planes of V
+  uint32_t side_off[5];                // the side stream records' offsets in the record
 };
 
 // Decode table of one rANS stream built by one warp: freq[256] (validated, sum
@@ -795,7 +966,48 @@ __device__ inline bool decode_codes_group(const uint8_t* sub, uint32_t sl, uint3
   return __all_sync(0xffffffffu, ok);
 }
 
+// rANS decode of a side stream's single group by one warp (lanes l < N <= 4)
+// from the sub-stream copied to shared memory (sl bytes at sub, 4-byte
+// aligned): byte table lut, f << 16 | cum per symbol in fc; dm = 0xff undoes
+// lane deltas. Returns false (on every lane) when a lane reads past the
+// words or the final states and word count do not match.
+__device__ inline bool side_decode_group(const uint8_t* sub, uint32_t sl, uint32_t n, const uint8_t* lut,
+                                         const uint32_t* fc, uint32_t dm, uint8_t* out) {
+  const uint32_t lane = threadIdx.x & 31u, N = rans_lanes(n);
+  if (sl < 4u * N || ((sl - 4u * N) & 1u)) return false;
+  const uint32_t W = (sl - 4u * N) >> 1;
+  const bool live = lane < N;
+  uint32_t start = 0, len = 0, start0, maxlen;
+  if (live) lane_range(n, N, lane, start, len);
+  lane_range(n, N, 0u, start0, maxlen);
+  const uint16_t* words = reinterpret_cast<const uint16_t*>(sub + 4u * N);
+  uint32_t x = live ? reinterpret_cast<const uint32_t*>(sub)[lane] : kRansLow;
+  uint32_t pos = 0, prev = 0, over = 0;
+  const uint32_t lt = lanemask_lt();
+  for (uint32_t tau = 0; tau < maxlen; ++tau) {
+    const bool act = live && tau < len;
+    if (act) {
+      const uint32_t slot = x & (kProbScale - 1u), sym = lut[slot], e = fc[sym];
+      x = (e >> 16) * (x >> kProbBits) + slot - (e & 0xffffu);
+      prev = sym ^ (prev & dm);
+      out[start + tau] = uint8_t(prev);
+    }
+    const bool need = act && x < kRansLow;
+    const uint32_t mask = __ballot_sync(0xffffffffu, need);
+    const uint32_t idx = pos + __popc(mask & lt);
+    if (need) {
+      over |= idx >= W ? 1u : 0u;
+      x = (x << 16) | words[idx < W ? idx : 0u];
+    }
+    pos += __popc(mask);
+  }
+  const bool ok = !over && pos == W && (!live || x == kRansLow);
+  return __all_sync(0xffffffffu, ok);
+}
+
 static_assert(sizeof(DecEntSmem) <= 232448 / 3, "entropy stage should fit three blocks per SM");
+static_assert(offsetof(DecEntSmem, ring) % 16 == 0 && offsetof(DecEntSmem, lut) % 4 == 0,
+              "refill rings take 16-byte copies; the side streams' table reads 4-byte words");
 
 __global__ void __launch_bounds__(kThreads, 3)
 k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t* ws,
@@ -816,7 +1028,7 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
   __syncthreads();
   const uint32_t nrec = S.base[b.n];
   if (blockIdx.x >= nrec) return;
-  const CodeBlocks cb = code_blocks(ws, max_records);
+  const CodeBlocks cb = code_blocks(ws, max_records, sh.ct);
   crc_tables_init(S.crc_t);
   const uint32_t rps = 1u + sh.n_mid;
   for (uint32_t g = blockIdx.x; g < nrec; g += gridDim.x) {
@@ -855,11 +1067,58 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
     const uint32_t t0 = sh.s_end + c * sh.ct, tcc = min(sh.ct, sh.r_start - t0);
     const uint32_t nb = (tcc + kTile - 1) / kTile;
     load_comp_info(pl.comp + sidx, S.ci);
-    const uint32_t side = 8u * S.ci.n_coded * nb;
-    if (st == kOk && pad16(side) > len) st = kErrCorrupt;
-    // stream records: walk the headers for their offsets, then parse each one
+    // side information: four byte-plane streams of V = every z, then every s.
+    // Their headers are checked one by one (the tables go to the width streams'
+    // table slots, which are built only later); their bytes are copied to shared
+    // memory (the refill rings, idle until the code streams), and warp q decodes
+    // plane q from there.
+    const uint32_t half = S.ci.n_coded * nb, nv = 2u * half;
+    if (tid == 0) S.side_off[0] = 0;
+    for (uint32_t q = 0; q < 4u && nv && st == kOk; ++q) {
+      const uint32_t o = S.side_off[q];
+      st = block_parse_stream(rec + o, len - o, nv, &S.si[q], S.freq[q], S.tmp, true);
+      if (tid == 0) S.side_off[q + 1] = o + S.si[q].bytes;
+      __syncthreads();
+    }
+    if (st == kOk && nv) {
+      const uint32_t side_bytes = S.side_off[4];  // at most 4 (16 + pad16(kSideMax)) <= sizeof(ring)
+      uint4* stage = reinterpret_cast<uint4*>(&S.ring[0][0]);
+      for (uint32_t i = tid; i < side_bytes / 16u; i += nthr) stage[i] = __ldg(reinterpret_cast<const uint4*>(rec) + i);
+      if (warp < 4 && S.si[warp].mode == kModeRans) warp_dec_lut8(S.freq[warp], S.lut[warp]);
+      __syncthreads();
+      bool okw = true;
+      if (warp < 4) {
+        const StreamInfo& si = S.si[warp];
+        uint8_t* plane = S.side[warp];
+        const uint8_t* base = reinterpret_cast<const uint8_t*>(stage) + S.side_off[warp];
+        if (si.mode == kModeRaw) {
+          for (uint32_t i = lane; i < nv; i += 32u) plane[i] = base[16u + i];
+        } else if (si.mode == kModeConst) {
+          for (uint32_t i = lane; i < nv; i += 32u) plane[i] = uint8_t(si.sym);
+        } else {
+          okw = side_decode_group(base + si.sub_off[0], si.sub_len[0], nv, S.lut[warp], S.freq[warp],
+                                  si.delta ? 0xffu : 0u, plane);
+        }
+      }
+      if (!__syncthreads_and(okw)) st = kErrCorrupt;
+    }
+    const uint32_t o_side = nv && st == kOk ? S.side_off[4] : 0u;
+    if (st == kOk && nv) {
+      float2* zs = cb.zs + uint64_t(g) * kD * (sh.ct / kTile);
+      for (uint32_t i = tid; i < half; i += nthr) {
+        uint32_t z = 0, sc = 0;
+#pragma unroll
+        for (uint32_t q = 0; q < 4; ++q) {
+          z |= uint32_t(S.side[q][i]) << (8u * q);
+          sc |= uint32_t(S.side[q][half + i]) << (8u * q);
+        }
+        const uint32_t cc = i / nb, blk = i - cc * nb;
+        zs[cc * (sh.ct / kTile) + blk] = make_float2(__uint_as_float(z), __uint_as_float(sc));
+      }
+    }
+    // code stream records: walk the headers for their offsets, then parse each one
     if (tid == 0) {
-      uint32_t o = pad16(side), ok = st == kOk ? 1u : 0u;
+      uint32_t o = o_side, ok = st == kOk ? 1u : 0u;
       for (uint32_t bw = 1; bw <= 8 && ok; ++bw) {
         if (!S.ci.bcount[bw]) continue;
         S.str_off[bw - 1] = o;
@@ -980,7 +1239,7 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
   const uint32_t per = (nrec + gridDim.x - 1) / gridDim.x;
   const uint32_t rbeg = blockIdx.x * per, rend = min(nrec, rbeg + per);
   if (rbeg >= rend) return;
-  const CodeBlocks cb = code_blocks(ws, max_records);
+  const CodeBlocks cb = code_blocks(ws, max_records, sh.ct);
   if (warp == 0) {
     tc::tmem_alloc(&S.tmem_base, kTcCols);
     tc::tmem_relinquish();
@@ -1026,13 +1285,14 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
 #pragma unroll
     for (uint32_t i = 0; i < 8; ++i) wmask |= S.ci.width[j0 + i] ? (1u << i) : 0u;
     if (tid < kD && S.ci.width[tid]) {  // all of the component's (z, s) pairs are loaded before any is stored
-      const uint2* p64 = reinterpret_cast<const uint2*>(rec + 8u * S.ci.coded_idx[tid] * nb);
-      uint2 zs[kMaxCt / kTile];
+      // decoded from the record's side streams by the entropy stage
+      const float2* p64 = cb.zs + (uint64_t(g) * kD + S.ci.coded_idx[tid]) * (sh.ct / kTile);
+      float2 zs[kMaxCt / kTile];
 #pragma unroll
-      for (uint32_t blk = 0; blk < kMaxCt / kTile; ++blk) zs[blk] = blk < nb ? __ldg(p64 + blk) : make_uint2(0, 0);
+      for (uint32_t blk = 0; blk < kMaxCt / kTile; ++blk) zs[blk] = blk < nb ? __ldg(p64 + blk) : make_float2(0.f, 0.f);
 #pragma unroll
       for (uint32_t blk = 0; blk < kMaxCt / kTile; ++blk)
-        if (blk < nb) S.zsT[tid & 7u][blk][tid >> 3] = make_float2(__uint_as_float(zs[blk].x), __uint_as_float(zs[blk].y));
+        if (blk < nb) S.zsT[tid & 7u][blk][tid >> 3] = zs[blk];
     }
     // inverse projection on the tensor cores, 128 tokens at a time:
     // x^[t][k] = sum_j y^[t][j] Q[k][j] with y^ and Q split into bf16 hi + lo
@@ -1193,7 +1453,7 @@ int num_sms() {
 
 uint64_t transform_slot_bytes(const TransformShape& s) {
   // largest record: side info + up to 8 streams of the codes, or the raw rows
-  uint64_t mid = pad16_64(8ull * kD * (kMaxCt / kTile)) + 8u * 16u + pad16_64(uint64_t(kD) * kMaxCt);
+  uint64_t mid = 4u * (16u + pad16_64(kSideMax)) + 8u * 16u + pad16_64(uint64_t(kD) * kMaxCt);
   uint64_t raw = pad16_64(uint64_t(s.s_end + (s.T - s.r_start)) * kD * 2u);
   uint64_t b = (mid > raw ? mid : raw) + kWordsArea + kCodesArea;
   return (b + 255u) & ~uint64_t(255);
@@ -1216,9 +1476,17 @@ cudaError_t launch_transform_encode(const TransformShape& s, const TransformPlan
   e = cudaFuncSetAttribute(k_transform_entropy, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            int(sizeof(EntSmem)));
   if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(k_transform_side, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(SideSmem)));
+  if (e != cudaSuccess) return e;
   {
     ProfRange pr_("transform_project", st);
     k_transform_project<<<grid, kThreads, sizeof(ProjSmem), st>>>(s, p, b, ws);
+  }
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  {
+    ProfRange pr_("transform_side", st);
+    k_transform_side<<<grid, kThreads, sizeof(SideSmem), st>>>(s, p, b, ws);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -1261,7 +1529,8 @@ cudaError_t launch_transform_decode(const TransformShape& s, const TransformPlan
 }
 
 uint64_t transform_decode_ws_extra(const TransformShape& s, uint64_t records) {
-  return ((4u * records + 255u) & ~uint64_t(255)) + records * uint64_t(s.ct) * kCodeRow;
+  return ((4u * records + 255u) & ~uint64_t(255)) + records * uint64_t(s.ct) * kCodeRow +
+         records * uint64_t(kD) * (s.ct / kTile) * sizeof(float2);
 }
 
 }  // namespace kvc
