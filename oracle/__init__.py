@@ -61,6 +61,8 @@ def _load():
         "kvco_stream_bound": ([u32], sz),
         "kvco_stream_encode": ([vp, u32, vp], sz),
         "kvco_stream_encode_delta": ([vp, u32, vp], sz),
+        "kvco_side_stream_encode": ([vp, u32, vp], sz),
+        "kvco_side_stream_decode": ([vp, sz, u32, vp, P(sz)], i32),
         "kvco_lane_delta": ([vp, u32, vp], None),
         "kvco_lane_undelta": ([vp, u32], None),
         "kvco_stream_decode": ([vp, sz, u32, vp, P(sz)], i32),
@@ -156,6 +158,26 @@ def stream_encode_delta(sym: np.ndarray) -> bytes:
     out = np.zeros(lib.kvco_stream_bound(s.size), dtype=np.uint8)
     n = lib.kvco_stream_encode_delta(_ptr(s) if s.size else None, s.size, _ptr(out))
     return out[:n].tobytes()
+
+
+def side_stream_encode(sym: np.ndarray) -> bytes:
+    """Side stream record (a byte plane of a middle record's zero points and
+    scales): the lane-delta choice on min(32, max(1, n // 64)) lanes."""
+    s = np.ascontiguousarray(sym, dtype=np.uint8)
+    lib = _load()
+    out = np.zeros(lib.kvco_stream_bound(s.size), dtype=np.uint8)
+    n = lib.kvco_side_stream_encode(_ptr(s) if s.size else None, s.size, _ptr(out))
+    return out[:n].tobytes()
+
+
+def side_stream_decode(rec: bytes, n: int):
+    """(status, symbols, bytes used) of a side stream record of n symbols."""
+    buf = np.frombuffer(bytes(rec), dtype=np.uint8).copy()
+    out = np.zeros(max(n, 1), dtype=np.uint8)
+    used = ctypes.c_size_t(0)
+    st = _load().kvco_side_stream_decode(_ptr(buf) if buf.size else None, buf.size, n, _ptr(out),
+                                         ctypes.byref(used))
+    return st, out[:n], used.value
 
 
 def lane_delta(sym: np.ndarray) -> np.ndarray:

@@ -147,6 +147,17 @@ static uint32_t lanes_for(uint32_t n) {
   return N;
 }
 
+/* Side streams (the byte planes of a middle record's zero points and scales,
+ * at most 2 * D * ct / B symbols) take one lane per 64 symbols, at most one
+ * group: N = min(32, max(1, floor(n / 64))). This codec's reading: it keeps a
+ * lane's serial chain at most 127 steps, a quarter of a code stream's. */
+static uint32_t side_lanes_for(uint32_t n) {
+  uint32_t N = n / 64u;
+  if (N < 1) N = 1;
+  if (N > LANES_PER_GROUP) N = LANES_PER_GROUP;
+  return N;
+}
+
 static void lane_range(uint32_t n, uint32_t N, uint32_t l, uint32_t* start, uint32_t* len) {
   uint32_t base = n / N, extra = n % N;
   *len = base + (l < extra ? 1u : 0u);
@@ -278,11 +289,10 @@ static size_t stream_raw(const uint8_t* sym, uint32_t n, uint8_t* out) {
 }
 
 /* Build the RANS record into out (capacity 2n + 4096); returns its size. */
-static size_t stream_rans(const uint8_t* sym, uint32_t n, const uint16_t freq[256],
+static size_t stream_rans(const uint8_t* sym, uint32_t n, uint32_t N, const uint16_t freq[256],
                           uint32_t k, uint32_t flags, uint8_t* out, size_t* payload) {
   uint32_t cum[256];
   cum_from_freq(freq, cum);
-  uint32_t N = lanes_for(n);
   uint32_t G = (N + LANES_PER_GROUP - 1) / LANES_PER_GROUP;
   size_t p = 16;
   memset(out, 0, 16 + 32);
@@ -327,9 +337,7 @@ static int stream_table(const uint8_t* sym, uint32_t n, uint16_t freq[256]) {
  * order). Reading: within each rANS lane's contiguous range of the stream, a
  * symbol is replaced by its XOR with the previous symbol of the same lane; the
  * lane's first symbol is kept. Undone lane by lane in order. */
-void kvco_lane_delta(const uint8_t* sym, uint32_t n, uint8_t* out) {
-  if (!n) return;
-  uint32_t N = lanes_for(n);
+static void lane_delta_n(const uint8_t* sym, uint32_t n, uint32_t N, uint8_t* out) {
   for (uint32_t l = 0; l < N; l++) {
     uint32_t start, len;
     lane_range(n, N, l, &start, &len);
@@ -338,9 +346,7 @@ void kvco_lane_delta(const uint8_t* sym, uint32_t n, uint8_t* out) {
   }
 }
 
-void kvco_lane_undelta(uint8_t* sym, uint32_t n) {
-  if (!n) return;
-  uint32_t N = lanes_for(n);
+static void lane_undelta_n(uint8_t* sym, uint32_t n, uint32_t N) {
   for (uint32_t l = 0; l < N; l++) {
     uint32_t start, len;
     lane_range(n, N, l, &start, &len);
@@ -348,22 +354,43 @@ void kvco_lane_undelta(uint8_t* sym, uint32_t n) {
   }
 }
 
-/* Stream with the lane-delta candidate: the plain choice of
- * kvco_stream_encode, unless a RANS record of the lane-delta symbols (flag
- * byte 1) is strictly smaller than both the plain RANS record and RAW. */
-size_t kvco_stream_encode_delta(const uint8_t* sym, uint32_t n, uint8_t* out) {
+void kvco_lane_delta(const uint8_t* sym, uint32_t n, uint8_t* out) {
+  if (n) lane_delta_n(sym, n, lanes_for(n), out);
+}
+
+void kvco_lane_undelta(uint8_t* sym, uint32_t n) {
+  if (n) lane_undelta_n(sym, n, lanes_for(n));
+}
+
+/* One stream record of n symbols on N rANS lanes: CONST for a single symbol;
+ * with allow_delta, a RANS record of the lane-delta symbols (flag byte 1) when
+ * strictly smaller than both the plain RANS record and RAW; else plain RANS if
+ * strictly smaller than RAW; else RAW. */
+static size_t stream_encode_lanes(const uint8_t* sym, uint32_t n, uint32_t N, int allow_delta, uint8_t* out) {
   uint16_t freq[256], dfreq[256];
   int k = stream_table(sym, n, freq);
-  if (k < 2) return kvco_stream_encode(sym, n, out);
-  uint8_t* dsym = (uint8_t*)malloc(n);
-  kvco_lane_delta(sym, n, dsym);
-  int kd = stream_table(dsym, n, dfreq);
+  if (k == 0) return stream_raw(sym, n, out);
+  if (k == 1) {
+    memset(out, 0, 16);
+    out[0] = MODE_CONST;
+    out[1] = sym[0];
+    put32(out + 4, 16);
+    put32(out + 8, n);
+    put32(out + 12, 1);
+    return 16;
+  }
   size_t raw_bytes = 16u + pad16(n);
   uint8_t* tmp = (uint8_t*)malloc(2u * (size_t)n + 4096u);
   uint8_t* dtmp = (uint8_t*)malloc(2u * (size_t)n + 4096u);
+  uint8_t* dsym = (uint8_t*)malloc(n);
   size_t payload;
-  size_t rb = stream_rans(sym, n, freq, (uint32_t)k, 0, tmp, &payload);
-  size_t rd = kd >= 2 ? stream_rans(dsym, n, dfreq, (uint32_t)kd, 1, dtmp, &payload) : (size_t)-1;
+  size_t rb = stream_rans(sym, n, N, freq, (uint32_t)k, 0, tmp, &payload);
+  size_t rd = (size_t)-1;
+  if (allow_delta) {
+    lane_delta_n(sym, n, N, dsym);
+    int kd = stream_table(dsym, n, dfreq);
+    if (kd >= 2) rd = stream_rans(dsym, n, N, dfreq, (uint32_t)kd, 1, dtmp, &payload);
+  }
   size_t out_bytes;
   if (rd < rb && rd < raw_bytes) {
     memcpy(out, dtmp, rd);
@@ -381,31 +408,17 @@ size_t kvco_stream_encode_delta(const uint8_t* sym, uint32_t n, uint8_t* out) {
 }
 
 size_t kvco_stream_encode(const uint8_t* sym, uint32_t n, uint8_t* out) {
-  uint16_t freq[256];
-  int k = stream_table(sym, n, freq);
-  if (k == 0) return stream_raw(sym, n, out);
-  if (k == 1) {
-    memset(out, 0, 16);
-    out[0] = MODE_CONST;
-    out[1] = sym[0];
-    put32(out + 4, 16);
-    put32(out + 8, n);
-    put32(out + 12, 1);
-    return 16;
-  }
-  size_t raw_bytes = 16u + pad16(n);
-  uint8_t* tmp = (uint8_t*)malloc(2u * (size_t)n + 4096u);
-  size_t payload;
-  size_t rb = stream_rans(sym, n, freq, (uint32_t)k, 0, tmp, &payload);
-  size_t out_bytes;
-  if (rb < raw_bytes) {
-    memcpy(out, tmp, rb);
-    out_bytes = rb;
-  } else {
-    out_bytes = stream_raw(sym, n, out);
-  }
-  free(tmp);
-  return out_bytes;
+  return stream_encode_lanes(sym, n, lanes_for(n), 0, out);
+}
+
+/* Stream with the lane-delta candidate (the high byte plane of lossless chunks). */
+size_t kvco_stream_encode_delta(const uint8_t* sym, uint32_t n, uint8_t* out) {
+  return stream_encode_lanes(sym, n, lanes_for(n), 1, out);
+}
+
+/* Side stream: the lane-delta choice on the side lane rule. */
+size_t kvco_side_stream_encode(const uint8_t* sym, uint32_t n, uint8_t* out) {
+  return stream_encode_lanes(sym, n, side_lanes_for(n), 1, out);
 }
 
 /* rANS payload (states + words, no header, table or padding) for n symbols,
@@ -416,13 +429,13 @@ size_t kvco_rans_payload_bytes(const uint8_t* sym, uint32_t n) {
   if (k < 2) return 0;
   uint8_t* tmp = (uint8_t*)malloc(2u * (size_t)n + 4096u);
   size_t payload;
-  stream_rans(sym, n, freq, (uint32_t)k, 0, tmp, &payload);
+  stream_rans(sym, n, lanes_for(n), freq, (uint32_t)k, 0, tmp, &payload);
   free(tmp);
   return payload;
 }
 
 static int stream_decode(const uint8_t* rec, size_t avail, uint32_t n, uint8_t* sym, size_t* used,
-                         int allow_delta) {
+                         int allow_delta, int side) {
   if (avail < 16) return KVCO_CORRUPT;
   uint32_t mode = rec[0], csym = rec[1], G = rec[2], flags = rec[3];
   uint32_t bytes = get32(rec + 4), rn = get32(rec + 8), k = get32(rec + 12);
@@ -441,7 +454,7 @@ static int stream_decode(const uint8_t* rec, size_t avail, uint32_t n, uint8_t* 
     return KVCO_OK;
   }
   if (mode != MODE_RANS || csym != 0 || n == 0) return KVCO_CORRUPT;
-  uint32_t N = lanes_for(n);
+  uint32_t N = side ? side_lanes_for(n) : lanes_for(n);
   if (G != (N + LANES_PER_GROUP - 1) / LANES_PER_GROUP) return KVCO_CORRUPT;
   if (k < 2 || k > 256) return KVCO_CORRUPT;
   size_t p = 16;
@@ -477,13 +490,17 @@ static int stream_decode(const uint8_t* rec, size_t avail, uint32_t n, uint8_t* 
     p += pad16(sub);
   }
   if (p != bytes) return KVCO_CORRUPT;
-  if (flags) kvco_lane_undelta(sym, n);
+  if (flags) lane_undelta_n(sym, n, N);
   return KVCO_OK;
 }
 
 int kvco_stream_decode(const uint8_t* rec, size_t avail, uint32_t n, uint8_t* sym,
                        size_t* used) {
-  return stream_decode(rec, avail, n, sym, used, 1);
+  return stream_decode(rec, avail, n, sym, used, 1, 0);
+}
+
+int kvco_side_stream_decode(const uint8_t* rec, size_t avail, uint32_t n, uint8_t* sym, size_t* used) {
+  return stream_decode(rec, avail, n, sym, used, 1, 1);
 }
 
 /* ---------------------------------------------------------------------------
@@ -845,7 +862,8 @@ uint32_t kvco_plan_crc(const kvco_desc* d) {
  *     above. The side information is the sequence V of 2 * coded * nb fp32
  *     values: every z (for j ascending with b_j > 0, for each block), then
  *     every s in the same order; stream p (p = 0..3) holds byte p of each value
- *     of V and may take the lane delta (no side streams when nothing is coded).
+ *     of V, on the side lane rule, and may take the lane delta (no side streams
+ *     when nothing is coded).
  *   decode: y^ = fmaf(code, s, z) (0 for b_j = 0); x^_k = (float) sum_j
  *     (double) Q[k][j] * (double) y^_j in fp64; keys: forward rotation;
  *     bf16 round-to-nearest-even.
@@ -1060,7 +1078,7 @@ size_t kvco_encode_transform(const kvco_desc* d, uint32_t first_slice, uint32_t 
           }
         }
       if (nv)
-        for (uint32_t q = 0; q < 4; q++) p += kvco_stream_encode_delta(side + (size_t)q * nv, nv, dst + p);
+        for (uint32_t q = 0; q < 4; q++) p += kvco_side_stream_encode(side + (size_t)q * nv, nv, dst + p);
       for (uint32_t b = 1; b <= 8; b++) {
         uint32_t m = 0;
         for (uint32_t j = 0; j < D; j++) {
@@ -1093,7 +1111,7 @@ static int mid_chunk_parse(const kvco_desc* d, uint32_t sidx, const uint8_t* rec
   /* side streams: byte q of every value of V (the syms buffer holds ct * D >= 4 nv bytes) */
   for (uint32_t q = 0; q < 4 && nv; q++) {
     size_t used = 0;
-    int st = stream_decode(rec + p, len - p, nv, syms + (size_t)q * nv, &used, 1);
+    int st = stream_decode(rec + p, len - p, nv, syms + (size_t)q * nv, &used, 1, 1);
     if (st) return st;
     p += used;
   }
@@ -1116,7 +1134,7 @@ static int mid_chunk_parse(const kvco_desc* d, uint32_t sidx, const uint8_t* rec
     uint32_t m = count_width(w, D, b);
     if (!m) continue;
     size_t used = 0;
-    int st = stream_decode(rec + p, len - p, m * tcc, syms, &used, 0);  /* no lane delta here */
+    int st = stream_decode(rec + p, len - p, m * tcc, syms, &used, 0, 0);  /* no lane delta here */
     if (st) return st;
     p += used;
     uint32_t mm = 0;

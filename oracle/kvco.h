@@ -67,6 +67,10 @@ size_t kvco_stream_encode_delta(const uint8_t* sym, uint32_t n, uint8_t* out);
 void kvco_lane_delta(const uint8_t* sym, uint32_t n, uint8_t* out);
 void kvco_lane_undelta(uint8_t* sym, uint32_t n);
 size_t kvco_rans_payload_bytes(const uint8_t* sym, uint32_t n);
+/* Side streams of a middle record (the byte planes of its zero points and
+ * scales): the lane-delta choice on N = min(32, max(1, floor(n / 64))) lanes. */
+size_t kvco_side_stream_encode(const uint8_t* sym, uint32_t n, uint8_t* out);
+int kvco_side_stream_decode(const uint8_t* rec, size_t avail, uint32_t n, uint8_t* sym, size_t* used);
 
 size_t kvco_lossless_bound(const kvco_desc* d, uint32_t n_slices);
 size_t kvco_encode_lossless(const kvco_desc* d, uint32_t first_slice, uint32_t n_slices,

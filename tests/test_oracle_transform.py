@@ -393,7 +393,8 @@ def test_basis_variances_are_coordinate_second_moments(kind, is_key):
 def test_side_information_streams_layout():
     """A middle record opens with four stream records: byte plane q (low to high)
     of V = every z, then every s (coded components ascending, blocks in order),
-    each coded with the lane-delta candidate; the code streams follow. Also: the
+    each coded with the lane-delta candidate on the side lane rule; the code
+    streams follow. Also: the
     side streams of the AR(1) workload are smaller than the raw fp32 values."""
     w = _workload(n_tokens=1024)
     plan = _pca_plan(w)
@@ -407,7 +408,60 @@ def test_side_information_streams_layout():
     nb = 8  # first middle chunk: 512 tokens
     V = np.concatenate([zs[0][coded, :nb, 0].reshape(-1), zs[0][coded, :nb, 1].reshape(-1)]).astype(np.float32)
     planes = V.view(np.uint32)
-    want = b"".join(oracle.stream_encode_delta(((planes >> (8 * q)) & 0xFF).astype(np.uint8))
+    want = b"".join(oracle.side_stream_encode(((planes >> (8 * q)) & 0xFF).astype(np.uint8))
                     for q in range(4))
     assert c[off:off + len(want)] == want
     assert len(want) < 4 * (16 + V.size) and len(want) < length
+
+
+def _side_lanes(n):
+    N = min(32, max(1, n // 64))
+    base, extra = divmod(n, N)
+    return [base + (l < extra) for l in range(N)]
+
+
+@pytest.mark.parametrize("n", [64, 127, 128, 200, 1000, 1600, 2047, 2048])
+@pytest.mark.parametrize("kbits", [1, 3])
+def test_side_stream_lane_rule_by_bit_packing(n, kbits):
+    """Side streams take min(32, max(1, n // 64)) lanes in one group. With a
+    uniform alphabet of 2^k symbols (f = 2^(12-k)) every symbol inserts exactly
+    k bits, so the group's sub-stream is sum over lanes of 4 + 2 floor(k len / 16)
+    bytes: the closed form fixes the lane count and the lane ranges."""
+    reps = -(-n // (1 << kbits))
+    sym = np.tile(np.arange(1 << kbits, dtype=np.uint8), reps)[:n]
+    if n % (1 << kbits):
+        return  # the closed form needs every symbol equally often
+    rng = np.random.default_rng(n * 10 + kbits)
+    rng.shuffle(sym)
+    rec = oracle.side_stream_encode(sym)
+    k = 1 << kbits
+    sub_pred = sum(4 + 2 * ((kbits * ln) // 16) for ln in _side_lanes(n))
+    rans_pred = (48 + 2 * k + 15) // 16 * 16 + 16 + (sub_pred + 15) // 16 * 16
+    raw = 16 + (n + 15) // 16 * 16
+    if rec[0] == 2 and rec[3] == 0:  # plain RANS: one group whose sub-stream has the closed-form length
+        assert rec[2] == 1 and rans_pred < raw
+        lens_at = (48 + 2 * k + 15) // 16 * 16
+        assert int.from_bytes(rec[lens_at:lens_at + 4], "little") == sub_pred
+    elif rec[0] == 0:
+        assert rans_pred >= raw
+    else:  # lane deltas, taken only when strictly smaller than both
+        assert rec[0] == 2 and rec[2] == 1 and len(rec) < min(rans_pred, raw)
+    st, out, used = oracle.side_stream_decode(rec, n)
+    assert st == 0 and used == len(rec) and np.array_equal(out, sym)
+
+
+@pytest.mark.parametrize("n", [1, 63, 64, 500, 2048])
+def test_side_stream_roundtrip_and_refusals(n):
+    """Round trip of smooth side planes (the lane delta is taken where it is
+    strictly smaller); a side record read on the code streams' lane rule, or
+    with one byte changed in its header, is refused."""
+    rng = np.random.default_rng(n)
+    x = (np.cumsum(rng.integers(-2, 3, n)) % 256).astype(np.uint8)
+    rec = oracle.side_stream_encode(x)
+    st, out, used = oracle.side_stream_decode(rec, n)
+    assert st == 0 and used == len(rec) and np.array_equal(out, x)
+    if rec[0] == 2 and n // 64 > 1:
+        assert oracle.stream_decode(rec, n)[0] != 0  # other lane count: refused or wrong end state
+    bad = bytearray(rec)
+    bad[8] ^= 1  # symbol count
+    assert oracle.side_stream_decode(bytes(bad), n)[0] != 0

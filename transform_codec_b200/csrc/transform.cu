@@ -420,42 +420,66 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
 // projection leaves the record's side information raw at the start of the
 // slot's record area: (z, s) of coded component cc and block blk at 8 (cc nb +
 // blk). It becomes the sequence V = every z, then every s (components and
-// blocks in order), and V's four byte planes become four stream records with
-// the lane-delta candidate (the lossless rule: CONST for one symbol; the lane
-// deltas' RANS record if strictly smaller than both the plain RANS record and
-// RAW; else plain RANS if smaller than RAW; else RAW). They replace the raw
-// values, and their total length goes to rec_len, where the entropy kernel
-// finds the offset of its code streams.
+// blocks in order), and V's four byte planes become four stream records, the
+// lane-delta candidate included (the rule of the lossless high plane: CONST
+// for one symbol; the lane deltas' RANS record if strictly smaller than both
+// the plain RANS record and RAW; else plain RANS if smaller than RAW; else
+// RAW). Side streams take one lane per 64 symbols, at most 32 (one group), so
+// a lane's chain is at most 127 steps. Warp v owns variant v (plane v / 2,
+// its lane deltas when v is odd): histogram, then a bound on its RANS record
+// from the empirical entropy; only a variant that could beat RAW is
+// normalised and coded. The streams replace the raw values, and their total
+// length goes to rec_len, where the entropy kernel finds the offset of its
+// code streams.
 constexpr uint32_t kSideMax = 2u * kD * (kMaxCt / kTile);  // values of V at most
 
-struct __align__(16) SideSmem {
-  uint8_t sym[4][kSideMax];                // byte plane q of V
-  uint32_t hist[8][256], freq[8][256], rem[8][256];  // variant 2q: plane q; 2q + 1: its lane deltas
-  uint2 tab[8][256];
-  uint32_t states[8][4];                   // at most 4 lanes (one group)
-  uint32_t W[8][4], wbeg[8][4], sub_len[8][4], k[8];
-  uint32_t mode[4], bytes[4], var[4], off[5];
-  uint32_t tmp[32];
-  CompInfo ci;
-};
+__host__ __device__ inline uint32_t side_lanes(uint32_t n) {
+  const uint32_t N = n / 64u;
+  return N < 1u ? 1u : (N > kGroupLanes ? kGroupLanes : N);
+}
+// Bytes of a side stream's RANS record: header, bitmap, k frequencies, one
+// group length, the N states and W words.
+__host__ __device__ inline uint32_t side_rans_bytes(uint32_t k, uint32_t N, uint32_t W) {
+  return 48u + pad16(2u * k) + 16u + pad16(4u * N + 2u * W);
+}
 
-// One rANS group (lanes l < N <= 32) of a stream of n symbols sym(i), with the
-// encode table tab[s] = {f | cum << 16, floor((2^32 - 1) / f)}; words go
-// backwards into words[0, cap); returns their count (the steps and the word
-// placement of rans_encode_group).
-template <class SymFn>
-__device__ inline uint32_t side_encode_group(SymFn sym, uint32_t n, uint32_t N, const uint2* tab, uint16_t* words,
-                                             uint32_t cap, uint32_t* x_out) {
+struct __align__(16) SideSmem {
+  uint8_t sym[4][kSideMax];   // byte plane q of V
+  uint32_t hist[8][256];      // counts of variant v; its frequencies once normalised
+  uint32_t rem[8][256];       // normalisation scratch
+  uint2 tab[8][256];          // coding table of variant v: {f | cum << 16, floor((2^32 - 1) / f)}
+  uint32_t states[8][kGroupLanes];
+  uint32_t W[8], k[8], ran[8];
+  uint32_t mode[4], bytes[4], var[4], off[5];
+};
+static_assert(sizeof(SideSmem) <= 232448 / 5, "side kernel should fit five blocks per SM");
+
+// rANS chain of one side-stream variant by one warp (lanes l < N <= 32): lane
+// l codes its range of plane sy (the lane deltas when delta), last symbol
+// first, with the symbol and table entry of the next two steps fetched ahead.
+// Words go backwards into words[0, cap); returns their count.
+__device__ inline uint32_t side_chain(const uint8_t* sy, bool delta, uint32_t n, uint32_t N, const uint2* tab,
+                                      uint16_t* words, uint32_t cap, uint32_t* x_out) {
   const uint32_t lane = threadIdx.x & 31u;
   const bool live = lane < N;
   uint32_t start = 0, len = 0, start0, maxlen;
   if (live) lane_range(n, N, lane, start, len);
   lane_range(n, N, 0u, start0, maxlen);
+  auto sym_at = [&](int t) -> uint32_t {  // symbol of step t, 0 where the lane has none
+    if (!live || t < 0 || uint32_t(t) >= len) return 0u;
+    const uint32_t a = sy[start + t];
+    return (delta && t > 0) ? (a ^ sy[start + t - 1]) : a;
+  };
   uint32_t x = kRansLow, pos = cap;
   const uint32_t lt = lanemask_lt();
-  for (uint32_t tau = maxlen; tau-- > 0;) {
-    const bool act = live && tau < len;
-    const uint2 e = tab[act ? sym(start + tau) : 0u];
+  uint2 e_next = tab[sym_at(int(maxlen) - 1)];
+  uint32_t s_next = sym_at(int(maxlen) - 2);
+#pragma unroll 1
+  for (int tau = int(maxlen) - 1; tau >= 0; --tau) {
+    const bool act = live && uint32_t(tau) < len;
+    const uint2 e = e_next;
+    e_next = tab[s_next];
+    s_next = sym_at(tau - 2);
     const uint32_t f = e.x & 0xffffu, cum = e.x >> 16;
     const bool emit = act && x >= (f << 20);
     const uint32_t mask = __ballot_sync(0xffffffffu, emit);
@@ -473,6 +497,53 @@ __device__ inline uint32_t side_encode_group(SymFn sym, uint32_t n, uint32_t N, 
   return cap - pos;
 }
 
+// One side stream record at dst (global, 16-byte aligned), written by one warp
+// with every padding byte zero: RAW (the plane), CONST (its one symbol) or RANS
+// (frequencies freq[256], one group: N states, then W words).
+__device__ inline void warp_write_side(uint8_t* dst, uint32_t mode, uint32_t bytes, uint32_t n, uint32_t k,
+                                       const uint8_t* sy, const uint32_t* freq, const uint32_t* states,
+                                       const uint16_t* words, uint32_t W, uint32_t N, uint32_t delta) {
+  const uint32_t lane = threadIdx.x & 31u;
+  for (uint32_t i = lane; i < bytes / 16u; i += 32u) reinterpret_cast<uint4*>(dst)[i] = make_uint4(0, 0, 0, 0);
+  __syncwarp();
+  if (mode == kModeConst) {
+    if (lane == 0) *reinterpret_cast<uint4*>(dst) = make_uint4(kModeConst | (uint32_t(sy[0]) << 8), 16u, n, 1u);
+    return;
+  }
+  if (mode == kModeRaw) {
+    if (lane == 0) *reinterpret_cast<uint4*>(dst) = make_uint4(kModeRaw, bytes, n, 0u);
+    for (uint32_t i = lane; i < n; i += 32u) dst[16u + i] = sy[i];
+    return;
+  }
+  if (lane == 0) *reinterpret_cast<uint4*>(dst) = make_uint4(kModeRans | (1u << 16) | (delta << 24), bytes, n, k);
+#pragma unroll
+  for (uint32_t w = 0; w < 8; ++w) {
+    const uint32_t bits = __ballot_sync(0xffffffffu, freq[32u * w + lane] != 0u);
+    if (lane == 0) reinterpret_cast<uint32_t*>(dst + 16)[w] = bits;
+  }
+  uint32_t f[8], cnt = 0;
+#pragma unroll
+  for (uint32_t i = 0; i < 8; ++i) {
+    f[i] = freq[8u * lane + i];
+    cnt += f[i] ? 1u : 0u;
+  }
+  uint32_t incl = cnt;
+#pragma unroll
+  for (uint32_t o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  uint32_t idx = incl - cnt;
+#pragma unroll
+  for (uint32_t i = 0; i < 8; ++i)
+    if (f[i]) st_u16(dst + 48u + 2u * idx++, f[i]);
+  const uint32_t lens_at = pad16(48u + 2u * k), sub = lens_at + 16u;
+  if (lane == 0) *reinterpret_cast<uint32_t*>(dst + lens_at) = 4u * N + 2u * W;
+  if (lane < N) reinterpret_cast<uint32_t*>(dst + sub)[lane] = states[lane];
+  uint16_t* w16 = reinterpret_cast<uint16_t*>(dst + sub + 4u * N);
+  for (uint32_t i = lane; i < W; i += 32u) w16[i] = words[i];
+}
+
 __global__ void __launch_bounds__(kThreads)
 k_transform_side(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLayout ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -488,9 +559,8 @@ k_transform_side(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLay
   const uint32_t t0 = sh.s_end + c * sh.ct, tcc = min(sh.ct, sh.r_start - t0);
   const uint32_t nb = (tcc + kTile - 1) / kTile;
   uint8_t* rec = ws.slots + uint64_t(r) * ws.slot_bytes;
-  uint16_t* scratch = slot_words(rec, ws.slot_bytes);  // variant v's words at v * kSideMax
-  load_comp_info(pl.comp + sidx, S.ci);
-  const uint32_t half = S.ci.n_coded * nb, n = 2u * half;
+  uint16_t* scratch = slot_words(rec, ws.slot_bytes);  // variant v's words end at (v + 1) * kSideMax
+  const uint32_t half = __ldg(&pl.comp[sidx].n_coded) * nb, n = 2u * half;
   if (n == 0) {  // nothing coded: no side streams
     if (tid == 0) ws.rec_len[r] = 0;
     return;
@@ -505,64 +575,76 @@ k_transform_side(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLay
     }
   }
   __syncthreads();  // the raw values are in shared memory; the records may overwrite them
-  const uint32_t N = rans_lanes(n);  // at most 4 lanes: one group
-  for (uint32_t i = tid; i < n; i += nthr) {
-    const bool first = lane_start(i, n, N);
-#pragma unroll
-    for (uint32_t q = 0; q < 4; ++q) {
-      const uint32_t v = S.sym[q][i];
-      atomicAdd(&S.hist[2 * q][v], 1u);
-      atomicAdd(&S.hist[2 * q + 1][first ? v : v ^ S.sym[q][i - 1]], 1u);
-    }
-  }
-  __syncthreads();
-  // warp v: the table of variant v and, when it can be chosen, its words
+  const uint32_t N = side_lanes(n), raw_b = 16u + pad16(n);
   {
     const uint32_t v = warp, q = v >> 1;
-    const uint32_t kv = warp_normalize(S.hist[v], 256u, n, S.freq[v], S.rem[v], S.tab[v]);
-    const uint32_t kp = __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane] ? 1u : 0u) +
-                        __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane + 32u] ? 1u : 0u) +
-                        __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane + 64u] ? 1u : 0u) +
-                        __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane + 96u] ? 1u : 0u) +
-                        __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane + 128u] ? 1u : 0u) +
-                        __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane + 160u] ? 1u : 0u) +
-                        __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane + 192u] ? 1u : 0u) +
-                        __reduce_add_sync(0xffffffffu, S.hist[2 * q][lane + 224u] ? 1u : 0u);
-    if (lane == 0) S.k[v] = kv;
-    if (kp >= 2 && kv >= 2) {  // the lane deltas only compete with a plain RANS record
-      const uint8_t* sy = S.sym[q];
-      uint32_t x, Wg;
-      if ((v & 1u) == 0)
-        Wg = side_encode_group([sy](uint32_t i) -> uint32_t { return sy[i]; }, n, N, S.tab[v],
-                               scratch + v * kSideMax, n, &x);
-      else
-        Wg = side_encode_group(
-            [sy, n, N](uint32_t i) -> uint32_t {
-              return lane_start(i, n, N) ? uint32_t(sy[i]) : uint32_t(sy[i] ^ sy[i - 1]);
-            },
-            n, N, S.tab[v], scratch + v * kSideMax, n, &x);
-      if (lane < N) S.states[v][lane] = x;
-      if (lane == 0) {
-        S.W[v][0] = Wg;
-        S.wbeg[v][0] = v * kSideMax + n - Wg;
+    const bool delta = (v & 1u) != 0;
+    const uint8_t* sy = S.sym[q];
+    uint32_t* h = S.hist[v];
+    // histogram: lanes holding the same symbol add once
+    const uint32_t base = n / N, extra = n - base * N, big = extra * (base + 1u);
+    for (uint32_t i0 = 0; i0 < n; i0 += 32u) {
+      const uint32_t i = i0 + lane;
+      uint32_t s = 256u + lane;  // past the end: a key no other lane holds
+      if (i < n) {
+        s = sy[i];
+        if (delta) {
+          const bool first = i < big ? (i % (base + 1u)) == 0u : ((i - big) % base) == 0u;
+          if (!first) s ^= sy[i - 1];
+        }
       }
+      const uint32_t same = __match_any_sync(0xffffffffu, s);
+      if (s < 256u && lane == uint32_t(__ffs(same) - 1)) atomicAdd(&h[s], uint32_t(__popc(same)));
+    }
+    __syncwarp();
+    // Could its RANS record be smaller than RAW? Every coding step adds at least
+    // log2(M / f_s) - log2(16/15) bits to the state and every word at most
+    // 16 + log2(16/15), the final states hold at most 32 - 16 bits each beyond
+    // their start, and sum_s c_s log2(M / f_s) >= n H for the empirical entropy
+    // H (Gibbs), so W >= (n H - n log2(16/15) - 16 N) / (16 + log2(16/15)).
+    uint32_t present = 0;
+    float bits = 0.0f;
+    const float lgn = log2f(float(n));
+    for (uint32_t s = lane; s < 256u; s += 32u) {
+      const uint32_t cs = h[s];
+      if (cs) {
+        ++present;
+        bits += float(cs) * (lgn - log2f(float(cs)));
+      }
+    }
+    const uint32_t k = __reduce_add_sync(0xffffffffu, present);
+#pragma unroll
+    for (uint32_t o = 16; o; o >>= 1) bits += __shfl_xor_sync(0xffffffffu, bits, o);
+    const float slack = 0.0932f;  // > log2(16/15)
+    const float w_lb = (bits * 0.9999f - 2.0f - slack * float(n) - 16.0f * float(N)) / (16.0f + slack);
+    const float rec_lb = float(48u + pad16(2u * k) + 16u + 4u * N) + 2.0f * fmaxf(w_lb, 0.0f);
+    const bool run = k >= 2 && rec_lb < float(raw_b);
+    if (lane == 0) {
+      S.k[v] = k;
+      S.ran[v] = run ? 1u : 0u;
+    }
+    if (run) {
+      warp_normalize(h, 256u, n, h, S.rem[v], S.tab[v]);  // frequencies replace the counts
+      uint32_t x;
+      const uint32_t Wv = side_chain(sy, delta, n, N, S.tab[v], scratch + v * kSideMax, kSideMax, &x);
+      if (lane < N) S.states[v][lane] = x;
+      if (lane == 0) S.W[v] = Wv;
     }
   }
   __syncthreads();
   if (tid == 0) {  // per plane: CONST; lane-delta RANS if strictly smaller than plain RANS and RAW; RANS; RAW
-    const uint32_t raw_b = 16u + pad16(n);
     uint32_t off = 0;
     for (uint32_t q = 0; q < 4; ++q) {
-      const uint32_t kp = S.k[2 * q], kd = S.k[2 * q + 1];
-      uint32_t mode = kModeRaw, bytes = raw_b, var = 2 * q;
-      if (kp == 1) {
+      const uint32_t vp = 2u * q, vd = vp + 1u;
+      uint32_t mode = kModeRaw, bytes = raw_b, var = vp;
+      if (S.k[vp] == 1) {
         mode = kModeConst;
         bytes = 16;
-      } else if (kp >= 2) {
-        const uint32_t rb = rans_layout(n, kp, S.W[2 * q], S.sub_len[2 * q]);
-        const uint32_t rd = kd >= 2 ? rans_layout(n, kd, S.W[2 * q + 1], S.sub_len[2 * q + 1]) : 0xffffffffu;
+      } else {
+        const uint32_t rb = S.ran[vp] ? side_rans_bytes(S.k[vp], N, S.W[vp]) : 0xffffffffu;
+        const uint32_t rd = S.ran[vd] ? side_rans_bytes(S.k[vd], N, S.W[vd]) : 0xffffffffu;
         if (rd < rb && rd < raw_b) {
-          mode = kModeRans; bytes = rd; var = 2 * q + 1;
+          mode = kModeRans; bytes = rd; var = vd;
         } else if (rb < raw_b) {
           mode = kModeRans; bytes = rb;
         }
@@ -573,12 +655,11 @@ k_transform_side(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLay
     S.off[4] = off;
   }
   __syncthreads();
-  for (uint32_t q = 0; q < 4; ++q) {
-    const uint32_t v = S.var[q];
-    const uint8_t* sy = S.sym[q];
-    block_write_stream(rec + S.off[q], S.mode[q], n, S.bytes[q], uint32_t(sy[0]), S.k[v], S.freq[v], S.states[v],
-                       scratch, S.wbeg[v], S.W[v], S.sub_len[v], [sy](uint32_t i) -> uint32_t { return sy[i]; },
-                       S.tmp, v & 1u);
+  if (warp < 4) {
+    const uint32_t q = warp, v = S.var[q];
+    const uint32_t Wv = S.mode[q] == kModeRans ? S.W[v] : 0u;
+    warp_write_side(rec + S.off[q], S.mode[q], S.bytes[q], n, S.k[v], S.sym[q], S.hist[v], S.states[v],
+                    scratch + (v + 1u) * kSideMax - Wv, Wv, N, v & 1u);
   }
   if (tid == 0) ws.rec_len[r] = S.off[4];
 }
@@ -829,7 +910,7 @@ struct __align__(16) DecEntSmem {
   uint32_t str_off[8];                 // stream record offsets within the record, by width - 1
   CompInfo ci;
   uint32_t base[kBatchMax + 1];
-  uint32_t crc_ok, bad, walk_ok;
+  uint32_t crc_ok, bad, walk_ok, side_ok;
   uint8_t side[4][kSideMax];           // the side streams' byte planes of V
   uint32_t side_off[5];                // the side stream records' offsets in the record
 };
@@ -966,14 +1047,81 @@ __device__ inline bool decode_codes_group(const uint8_t* sub, uint32_t sl, uint3
   return __all_sync(0xffffffffu, ok);
 }
 
-// rANS decode of a side stream's single group by one warp (lanes l < N <= 4)
-// from the sub-stream copied to shared memory (sl bytes at sub, 4-byte
-// aligned): byte table lut, f << 16 | cum per symbol in fc; dm = 0xff undoes
-// lane deltas. Returns false (on every lane) when a lane reads past the
-// words or the final states and word count do not match.
+// Check the side stream record at rec (16-byte aligned, avail bytes: exactly
+// its own length from the header walk) for n symbols on N lanes (one group)
+// and, for RANS, load its frequencies into freq[256]. Warp-cooperative; lane
+// 0 fills si; returns the status on every lane.
+__device__ inline int warp_parse_side(const uint8_t* rec, uint32_t avail, uint32_t n, uint32_t N, StreamInfo& si,
+                                      uint32_t* freq) {
+  const uint32_t lane = threadIdx.x & 31u;
+  if (avail < 16u) return kErrCorrupt;
+  const uint4 hv = __ldg(reinterpret_cast<const uint4*>(rec));
+  const uint32_t mode = hv.x & 0xffu, csym = (hv.x >> 8) & 0xffu, G = (hv.x >> 16) & 0xffu, b3 = hv.x >> 24;
+  const uint32_t bytes = hv.y, rn = hv.z, k = hv.w;
+  bool bad = b3 > (mode == kModeRans ? 1u : 0u) || rn != n || (bytes & 15u) || bytes < 16u || bytes != avail;
+  uint32_t sub_off = 0, sub_len = 0;
+  if (!bad) {
+    if (mode == kModeRaw) bad = csym || G || k || bytes != 16u + pad16(n);
+    else if (mode == kModeConst) bad = G || k != 1u || bytes != 16u;
+    else if (mode == kModeRans) {
+      bad = csym || n == 0 || G != 1u || k < 2u || k > 256u;
+      if (!bad) {
+        const uint32_t lens_at = pad16(48u + 2u * k);
+        sub_off = lens_at + 16u;
+        bad = sub_off > bytes;
+        if (!bad) {
+          sub_len = ld_u32(rec + lens_at);
+          bad = sub_len > bytes || sub_off + pad16(sub_len) != bytes;
+        }
+      }
+    } else {
+      bad = true;
+    }
+  }
+  if (lane == 0) {
+    si.mode = mode; si.sym = csym; si.groups = G; si.bytes = bytes; si.k = k; si.delta = b3;
+    si.sub_off[0] = sub_off; si.sub_len[0] = sub_len;
+  }
+  if (bad || mode != kModeRans) {
+    __syncwarp();
+    return bad ? kErrCorrupt : kOk;
+  }
+  // presence bitmap byte `lane` covers symbols 8 lane .. 8 lane + 7
+  const uint32_t bm = rec[16u + lane];
+  const uint32_t cnt = __popc(bm);
+  uint32_t incl = cnt;
+#pragma unroll
+  for (uint32_t o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+  uint32_t idx = incl - cnt, fs = 0;
+  bool zero = false;
+#pragma unroll
+  for (uint32_t i = 0; i < 8; ++i) {
+    uint32_t f = 0;
+    if (total == k && ((bm >> i) & 1u)) {
+      f = ld_u16(rec + 48u + 2u * idx++);
+      zero |= f == 0;
+    }
+    freq[8u * lane + i] = f;
+    fs += f;
+  }
+  fs = __reduce_add_sync(0xffffffffu, fs);
+  bad = total != k || __any_sync(0xffffffffu, zero) || fs != kProbScale;
+  __syncwarp();
+  return bad ? kErrCorrupt : kOk;
+}
+
+// rANS decode of a side stream's single group by one warp (lanes l < N <= 32,
+// the side lane rule) from the sub-stream copied to shared memory (sl bytes at
+// sub, 4-byte aligned): byte table lut, f << 16 | cum per symbol in fc; dm =
+// 0xff undoes lane deltas. Returns false (on every lane) when a lane reads
+// past the words or the final states and word count do not match.
 __device__ inline bool side_decode_group(const uint8_t* sub, uint32_t sl, uint32_t n, const uint8_t* lut,
                                          const uint32_t* fc, uint32_t dm, uint8_t* out) {
-  const uint32_t lane = threadIdx.x & 31u, N = rans_lanes(n);
+  const uint32_t lane = threadIdx.x & 31u, N = side_lanes(n);
   if (sl < 4u * N || ((sl - 4u * N) & 1u)) return false;
   const uint32_t W = (sl - 4u * N) >> 1;
   const bool live = lane < N;
@@ -1068,41 +1216,51 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
     const uint32_t nb = (tcc + kTile - 1) / kTile;
     load_comp_info(pl.comp + sidx, S.ci);
     // side information: four byte-plane streams of V = every z, then every s.
-    // Their headers are checked one by one (the tables go to the width streams'
-    // table slots, which are built only later); their bytes are copied to shared
-    // memory (the refill rings, idle until the code streams), and warp q decodes
-    // plane q from there.
+    // One thread walks their headers for the offsets; warp q then checks stream
+    // q, loads its table (into the width streams' table slots, rebuilt only
+    // later), copies its bytes to its part of the refill rings (idle until the
+    // code streams) and decodes plane q from there.
     const uint32_t half = S.ci.n_coded * nb, nv = 2u * half;
-    if (tid == 0) S.side_off[0] = 0;
-    for (uint32_t q = 0; q < 4u && nv && st == kOk; ++q) {
-      const uint32_t o = S.side_off[q];
-      st = block_parse_stream(rec + o, len - o, nv, &S.si[q], S.freq[q], S.tmp, true);
-      if (tid == 0) S.side_off[q + 1] = o + S.si[q].bytes;
-      __syncthreads();
+    if (tid == 0) {
+      uint32_t o = 0, ok = st == kOk ? 1u : 0u;
+      for (uint32_t q = 0; q < 4u && nv && ok; ++q) {
+        S.side_off[q] = o;
+        if (o + 16u > len) { ok = 0; break; }
+        const uint32_t bytes = ld_u32(rec + o + 4);
+        if (bytes < 16u || (bytes & 15u) || bytes > len - o || bytes > 16u + pad16(nv)) { ok = 0; break; }
+        o += bytes;
+      }
+      S.side_off[4] = nv ? o : 0u;
+      S.side_ok = ok;
     }
+    __syncthreads();
+    if (st == kOk && !S.side_ok) st = kErrCorrupt;
     if (st == kOk && nv) {
-      const uint32_t side_bytes = S.side_off[4];  // at most 4 (16 + pad16(kSideMax)) <= sizeof(ring)
-      uint4* stage = reinterpret_cast<uint4*>(&S.ring[0][0]);
-      for (uint32_t i = tid; i < side_bytes / 16u; i += nthr) stage[i] = __ldg(reinterpret_cast<const uint4*>(rec) + i);
-      if (warp < 4 && S.si[warp].mode == kModeRans) warp_dec_lut8(S.freq[warp], S.lut[warp]);
-      __syncthreads();
       bool okw = true;
       if (warp < 4) {
-        const StreamInfo& si = S.si[warp];
-        uint8_t* plane = S.side[warp];
-        const uint8_t* base = reinterpret_cast<const uint8_t*>(stage) + S.side_off[warp];
-        if (si.mode == kModeRaw) {
-          for (uint32_t i = lane; i < nv; i += 32u) plane[i] = base[16u + i];
-        } else if (si.mode == kModeConst) {
-          for (uint32_t i = lane; i < nv; i += 32u) plane[i] = uint8_t(si.sym);
-        } else {
-          okw = side_decode_group(base + si.sub_off[0], si.sub_len[0], nv, S.lut[warp], S.freq[warp],
-                                  si.delta ? 0xffu : 0u, plane);
+        const uint32_t q = warp, o = S.side_off[q];
+        StreamInfo& si = S.si[q];
+        okw = warp_parse_side(rec + o, S.side_off[q + 1] - o, nv, side_lanes(nv), si, S.freq[q]) == kOk;
+        if (okw) {
+          uint8_t* stage = reinterpret_cast<uint8_t*>(&S.ring[2u * q][0]);  // 4 KiB >= 16 + pad16(kSideMax)
+          uint8_t* plane = S.side[q];
+          if (si.mode == kModeRaw) {
+            for (uint32_t i = lane; i < nv; i += 32u) plane[i] = __ldg(rec + o + 16u + i);
+          } else if (si.mode == kModeConst) {
+            for (uint32_t i = lane; i < nv; i += 32u) plane[i] = uint8_t(si.sym);
+          } else {
+            for (uint32_t i = lane; i < si.bytes / 16u; i += 32u)
+              reinterpret_cast<uint4*>(stage)[i] = __ldg(reinterpret_cast<const uint4*>(rec + o) + i);
+            warp_dec_lut8(S.freq[q], S.lut[q]);
+            __syncwarp();
+            okw = side_decode_group(stage + si.sub_off[0], si.sub_len[0], nv, S.lut[q], S.freq[q],
+                                    si.delta ? 0xffu : 0u, plane);
+          }
         }
       }
       if (!__syncthreads_and(okw)) st = kErrCorrupt;
     }
-    const uint32_t o_side = nv && st == kOk ? S.side_off[4] : 0u;
+    const uint32_t o_side = st == kOk ? S.side_off[4] : 0u;
     if (st == kOk && nv) {
       float2* zs = cb.zs + uint64_t(g) * kD * (sh.ct / kTile);
       for (uint32_t i = tid; i < half; i += nthr) {
