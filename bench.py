@@ -55,7 +55,6 @@ KERNEL_WORK = {
 # A kernel that changed after that capture has no entry.
 DRAM_BYTES_PER_FRAME = {
     "lossless_encode": (759.9e6 + 353.7e6) / 4,
-    "transform_decode_codes": (82.2e6 + 94.5e6) / 4,
     "transform_entropy": (128.5e6 + 27.9e6) / 4,
     "lossless_decode": (198.8e6 + 220.9e6) / 4,
     "transform_decode": (199.5e6 + 221.8e6) / 4,

@@ -443,6 +443,9 @@ static int stream_decode(const uint8_t* rec, size_t avail, uint32_t n, uint8_t* 
       bytes < 16 || bytes > avail)
     return KVCO_CORRUPT;
   *used = bytes;
+  /* a side stream is never longer than RAW (the never-worse choice); a longer
+   * one cannot come from the encoder and is refused */
+  if (side && bytes > 16u + pad16(n)) return KVCO_CORRUPT;
   if (mode == MODE_RAW) {
     if (csym != 0 || G != 0 || k != 0 || bytes != 16u + pad16(n)) return KVCO_CORRUPT;
     if (n) memcpy(sym, rec + 16, n);
