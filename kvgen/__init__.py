@@ -20,7 +20,7 @@ _SRC = os.path.join(_HERE, "kvgen.c")
 _LIB = os.path.join(_HERE, "libkvgen.so")
 _lib = None
 
-BF16, FP16 = 1, 2
+BF16, FP16, F32 = 1, 2, 3
 
 
 def compile_command() -> list[str]:
@@ -54,7 +54,7 @@ def _load():
 class Workload:
     name: str
     path: str            # "lossless" or "transform"
-    dtype: int           # BF16 or FP16
+    dtype: int           # BF16, FP16 or F32
     n_layers: int
     n_heads: int
     n_tokens: int
@@ -77,8 +77,12 @@ class Workload:
         return self.n_layers * 2 * self.n_heads
 
     @property
+    def elem_bytes(self) -> int:
+        return 4 if self.dtype == F32 else 2
+
+    @property
     def raw_bytes(self) -> int:
-        return self.n_slices * self.n_tokens * self.head_dim * 2
+        return self.n_slices * self.n_tokens * self.head_dim * self.elem_bytes
 
 
 WORKLOADS = {
@@ -90,6 +94,9 @@ WORKLOADS = {
     "lossless-12x12x1024x64-fp16": Workload(
         "lossless-12x12x1024x64-fp16", "lossless", FP16, 12, 12, 1024, 64, 0.8, 1e4,
         control_bytes=4 << 20),
+    # the GPT-2-small shape at fp32 (QATQ and AT-1 code f32 tensors too)
+    "lossless-12x12x1024x64-f32": Workload(
+        "lossless-12x12x1024x64-f32", "lossless", F32, 12, 12, 1024, 64, 0.8, 1e4),
     # live-migration block of 50,331,648 bytes: 8 layers x 8 heads x 1536 x 128
     "lossless-8x8x1536x128-bf16": Workload(
         "lossless-8x8x1536x128-bf16", "lossless", BF16, 8, 8, 1536, 128, 0.95, 1e4),
@@ -111,13 +118,14 @@ WORKLOADS = {
 
 
 def slices(w: Workload, first: int = 0, n: int | None = None, out=None, n_threads: int = 0):
-    """Slices [first, first+n) as uint16 [n][T][D]; out may be a preallocated
-    (e.g. pinned) uint16 buffer with at least n*T*D elements (numpy or ctypes address)."""
+    """Slices [first, first+n) as [n][T][D] value bits (uint16, or uint32 for F32);
+    out may be a preallocated (e.g. pinned) buffer with room for n*T*D values
+    (numpy or ctypes address)."""
     lib = _load()
     n = w.n_slices - first if n is None else n
     count = n * w.n_tokens * w.head_dim
     if out is None:
-        arr = np.empty(count, dtype=np.uint16)
+        arr = np.empty(count, dtype=np.uint32 if w.dtype == F32 else np.uint16)
         ptr = arr.ctypes.data
     elif isinstance(out, int):
         arr, ptr = None, out

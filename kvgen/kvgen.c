@@ -31,6 +31,7 @@
 
 #define KVGEN_BF16 1
 #define KVGEN_FP16 2
+#define KVGEN_F32 3   /* 4-byte IEEE single: the fp64 value rounded to nearest */
 
 static uint64_t mix64(uint64_t z) {
   z += 0x9e3779b97f4a7c15ULL;
@@ -107,7 +108,7 @@ typedef struct {
   double rho, theta;
   uint32_t first_slice, n_slices;
   uint64_t noise_stream; /* 1 = data, 2 = calibration */
-  uint16_t* out;         /* [n_slices][T][D] */
+  void* out;             /* [n_slices][T][D] 16-bit values, or 32-bit for F32 */
   const double* cs;      /* [T][D/2][2] cos, sin (keys) */
   uint32_t next;         /* work counter */
   pthread_mutex_t mu;
@@ -133,7 +134,8 @@ static void gen_slice(gen_job* J, uint32_t local) {
     sg[d] = exp(0.5 * n1);
     nkey[d] = channel_key(J->seed, J->noise_stream, l, kv, h, d);
   }
-  uint16_t* out = J->out + (size_t)local * T * D;
+  uint16_t* out = J->dtype == KVGEN_F32 ? NULL : (uint16_t*)J->out + (size_t)local * T * D;
+  uint32_t* out32 = J->dtype == KVGEN_F32 ? (uint32_t*)J->out + (size_t)local * T * D : NULL;
   for (uint32_t t = 0; t < T; t++) {
     for (uint32_t d = 0; d < D; d++) {
       double e;
@@ -155,7 +157,14 @@ static void gen_slice(gen_job* J, uint32_t local) {
         row[i + half] = x0 * si + x1 * co;
       }
     }
-    for (uint32_t d = 0; d < D; d++) out[(size_t)t * D + d] = to_dtype(row[d], J->dtype);
+    if (out32) {
+      for (uint32_t d = 0; d < D; d++) {
+        float f = (float)row[d];
+        memcpy(&out32[(size_t)t * D + d], &f, 4);
+      }
+    } else {
+      for (uint32_t d = 0; d < D; d++) out[(size_t)t * D + d] = to_dtype(row[d], J->dtype);
+    }
   }
   free(mu); free(sg); free(z); free(nz); free(nkey); free(row);
 }
@@ -200,7 +209,7 @@ static int run_gen(gen_job* J, int n_threads) {
 /* Slices [first_slice, first_slice + n_slices) of the [L][2][H][T][D] cache. */
 int kvgen_slices(uint64_t seed, uint32_t L, uint32_t H, uint32_t T, uint32_t D, int dtype,
                  double rho, double theta, uint32_t first_slice, uint32_t n_slices,
-                 int n_threads, uint16_t* out) {
+                 int n_threads, void* out) {
   if (D == 0 || (D & 1u) || first_slice + n_slices > L * 2 * H) return -1;
   gen_job J;
   memset(&J, 0, sizeof J);
@@ -213,7 +222,7 @@ int kvgen_slices(uint64_t seed, uint32_t L, uint32_t H, uint32_t T, uint32_t D, 
 /* Calibration draw: same channel parameters, separate noise stream, n_calib
  * tokens at positions 0..n_calib-1, every slice. Output [L*2*H][n_calib][D]. */
 int kvgen_calibration(uint64_t seed, uint32_t L, uint32_t H, uint32_t n_calib, uint32_t D,
-                      int dtype, double rho, double theta, int n_threads, uint16_t* out) {
+                      int dtype, double rho, double theta, int n_threads, void* out) {
   if (D == 0 || (D & 1u)) return -1;
   gen_job J;
   memset(&J, 0, sizeof J);

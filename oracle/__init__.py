@@ -18,7 +18,7 @@ _HDR = os.path.join(_HERE, "kvco.h")
 _LIB = os.path.join(_HERE, "libkvco.so")
 _lib = None
 
-BF16, FP16 = 1, 2
+BF16, FP16, F32 = 1, 2, 3
 OK, INVALID, CAPACITY, CORRUPT, TRUNCATED, PLAN_MISMATCH = 0, 1, 2, 3, 4, 5
 
 
@@ -213,8 +213,13 @@ def lossless_bound(plan: Plan, n_slices: int) -> int:
     return _load().kvco_lossless_bound(ctypes.byref(plan.desc), n_slices)
 
 
+def _vtype(plan: Plan):
+    """numpy type of one value's bits: uint32 for f32, else uint16."""
+    return np.uint32 if plan.desc.dtype == F32 else np.uint16
+
+
 def encode_lossless(plan: Plan, src: np.ndarray, first_slice: int = 0) -> bytes:
-    s = np.ascontiguousarray(src, dtype=np.uint16)
+    s = np.ascontiguousarray(src, dtype=_vtype(plan))
     n_slices = s.size // (plan.desc.n_tokens * plan.desc.head_dim)
     lib = _load()
     cap = lib.kvco_lossless_bound(ctypes.byref(plan.desc), n_slices)
@@ -229,11 +234,11 @@ def encode_lossless(plan: Plan, src: np.ndarray, first_slice: int = 0) -> bytes:
 def _decode(fn, plan, buf, n_slices_cap):
     b = _buf(buf)
     D, T = plan.desc.head_dim, plan.desc.n_tokens
-    out = np.zeros(max(n_slices_cap * T * D, 1), dtype=np.uint16)
+    out = np.zeros(max(n_slices_cap * T * D, 1), dtype=_vtype(plan))
     written = ctypes.c_uint64(0)
     st = fn(ctypes.byref(plan.desc), _ptr(b) if b.size else None, b.size, _ptr(out),
             out.nbytes if n_slices_cap else 0, ctypes.byref(written))
-    ns = written.value // (T * D * 2)
+    ns = written.value // (T * D * out.itemsize)
     return st, out[: ns * T * D].reshape(ns, T, D)
 
 

@@ -521,7 +521,7 @@ int kvco_side_stream_decode(const uint8_t* rec, size_t avail, uint32_t n, uint8_
 
 static int desc_ok(const kvco_desc* d) {
   if (!d) return 0;
-  if (d->dtype != KVCO_BF16 && d->dtype != KVCO_FP16) return 0;
+  if (d->dtype != KVCO_BF16 && d->dtype != KVCO_FP16 && d->dtype != KVCO_F32) return 0;
   if (!d->n_layers || !d->n_heads || !d->n_tokens || !d->head_dim) return 0;
   return 1;
 }
@@ -621,6 +621,10 @@ static int check_container(const kvco_desc* d, int path, const uint8_t* src, siz
  * ------------------------------------------------------------------------- */
 static uint32_t lossless_tc(const kvco_desc* d) { return d->values_per_chunk / d->head_dim; }
 
+/* Bytes per value, and so byte planes per chunk: 2 for bf16 / fp16, 4 for f32
+ * ([QATQ] "f32, f16, and bf16"; [AT-1] "Works on fp32/fp16/bf16"). */
+static uint32_t elem_bytes(const kvco_desc* d) { return d->dtype == KVCO_F32 ? 4u : 2u; }
+
 static int lossless_ok(const kvco_desc* d) {
   return desc_ok(d) && d->values_per_chunk <= 65536u && d->values_per_chunk >= d->head_dim;
 }
@@ -632,39 +636,41 @@ static uint64_t lossless_records(const kvco_desc* d, uint32_t n_slices) {
 
 size_t kvco_lossless_bound(const kvco_desc* d, uint32_t n_slices) {
   if (!lossless_ok(d)) return 0;
-  uint32_t tc = lossless_tc(d), T = d->n_tokens, D = d->head_dim;
+  uint32_t tc = lossless_tc(d), T = d->n_tokens, D = d->head_dim, E = elem_bytes(d);
   size_t per_slice = 0;
   for (uint32_t t0 = 0; t0 < T; t0 += tc) {
     uint32_t tcc = T - t0 < tc ? T - t0 : tc;
-    per_slice += 2u * (16u + pad16((size_t)tcc * D)) + IDX_ENTRY;
+    per_slice += E * (16u + pad16((size_t)tcc * D)) + IDX_ENTRY;
   }
   return HDR_BYTES + per_slice * n_slices;
 }
 
+/* Chunk record: for p = 0 .. E-1, the stream record of plane p (byte p of
+ * every little-endian value, channel-major order inside the chunk). The upper
+ * half of the planes, which hold the sign and exponent bits (plane 1 of a
+ * 16-bit value; planes 2 and 3 of an f32), take the lane-delta candidate. */
 size_t kvco_encode_lossless(const kvco_desc* d, uint32_t first_slice, uint32_t n_slices,
-                            const uint16_t* src, uint8_t* dst, size_t cap) {
+                            const void* src, uint8_t* dst, size_t cap) {
   if (!lossless_ok(d) || (uint64_t)first_slice + n_slices > n_slices_total(d)) return 0;
   size_t bound = kvco_lossless_bound(d, n_slices);
   if (cap < bound) return 0;
-  uint32_t tc = lossless_tc(d), T = d->n_tokens, D = d->head_dim;
+  uint32_t tc = lossless_tc(d), T = d->n_tokens, D = d->head_dim, E = elem_bytes(d);
+  const uint8_t* in = (const uint8_t*)src;
   uint32_t nr = (uint32_t)lossless_records(d, n_slices);
-  uint8_t* p0 = (uint8_t*)malloc((size_t)tc * D);
-  uint8_t* p1 = (uint8_t*)malloc((size_t)tc * D);
+  uint8_t* pl = (uint8_t*)malloc((size_t)tc * D);
   size_t p = HDR_BYTES + (size_t)IDX_ENTRY * nr;
   uint32_t r = 0;
   for (uint32_t s = 0; s < n_slices; s++) {
     for (uint32_t t0 = 0; t0 < T; t0 += tc) {
       uint32_t tcc = T - t0 < tc ? T - t0 : tc;
       uint32_t n = tcc * D;
-      for (uint32_t dd = 0; dd < D; dd++)
-        for (uint32_t t = 0; t < tcc; t++) {
-          uint16_t v = src[((size_t)s * T + t0 + t) * D + dd];
-          p0[(size_t)dd * tcc + t] = (uint8_t)(v & 0xffu);
-          p1[(size_t)dd * tcc + t] = (uint8_t)(v >> 8);
-        }
       size_t start = p;
-      p += kvco_stream_encode(p0, n, dst + p);
-      p += kvco_stream_encode_delta(p1, n, dst + p);
+      for (uint32_t b = 0; b < E; b++) {
+        for (uint32_t dd = 0; dd < D; dd++)
+          for (uint32_t t = 0; t < tcc; t++)
+            pl[(size_t)dd * tcc + t] = in[(((size_t)s * T + t0 + t) * D + dd) * E + b];
+        p += 2u * b < E ? kvco_stream_encode(pl, n, dst + p) : kvco_stream_encode_delta(pl, n, dst + p);
+      }
       uint8_t* e = dst + HDR_BYTES + (size_t)IDX_ENTRY * r;
       put64(e, start);
       put32(e + 8, (uint32_t)(p - start));
@@ -672,25 +678,24 @@ size_t kvco_encode_lossless(const kvco_desc* d, uint32_t first_slice, uint32_t n
       r++;
     }
   }
-  free(p0);
-  free(p1);
+  free(pl);
   write_header(dst, KVCO_LOSSLESS, d, first_slice, n_slices, tc, nr, p, 0);
   put32(dst + 60, header_crc(dst, nr));
   return p;
 }
 
-int kvco_decode_lossless(const kvco_desc* d, const uint8_t* src, size_t n, uint16_t* dst,
+int kvco_decode_lossless(const kvco_desc* d, const uint8_t* src, size_t n, void* dst,
                          size_t cap, uint64_t* written) {
   if (!lossless_ok(d)) return KVCO_INVALID;
   uint32_t first, ns, nr;
   int st = check_container(d, KVCO_LOSSLESS, src, n, lossless_records, lossless_tc(d), 0,
                            &first, &ns, &nr);
   if (st) return st;
-  uint32_t tc = lossless_tc(d), T = d->n_tokens, D = d->head_dim;
-  uint64_t out_bytes = (uint64_t)ns * T * D * 2u;
+  uint32_t tc = lossless_tc(d), T = d->n_tokens, D = d->head_dim, E = elem_bytes(d);
+  uint64_t out_bytes = (uint64_t)ns * T * D * E;
   if (out_bytes > cap) return KVCO_CAPACITY;
-  uint8_t* p0 = (uint8_t*)malloc((size_t)tc * D);
-  uint8_t* p1 = (uint8_t*)malloc((size_t)tc * D);
+  uint8_t* out = (uint8_t*)dst;
+  uint8_t* pl = (uint8_t*)malloc((size_t)tc * D);
   uint32_t r = 0;
   st = KVCO_OK;
   for (uint32_t s = 0; s < ns && !st; s++) {
@@ -701,19 +706,20 @@ int kvco_decode_lossless(const kvco_desc* d, const uint8_t* src, size_t n, uint1
       const uint8_t* rec = src + get64(e);
       uint32_t len = get32(e + 8);
       if (kvco_crc32(rec, len) != get32(e + 12)) { st = KVCO_CORRUPT; break; }
-      size_t u0 = 0, u1 = 0;
-      st = kvco_stream_decode(rec, len, nv, p0, &u0);
-      if (!st) st = kvco_stream_decode(rec + u0, len - u0, nv, p1, &u1);
-      if (!st && u0 + u1 != len) st = KVCO_CORRUPT;
-      if (st) break;
-      for (uint32_t dd = 0; dd < D; dd++)
-        for (uint32_t t = 0; t < tcc; t++)
-          dst[((size_t)s * T + t0 + t) * D + dd] =
-              (uint16_t)(p0[(size_t)dd * tcc + t] | ((uint16_t)p1[(size_t)dd * tcc + t] << 8));
+      size_t off = 0;
+      for (uint32_t b = 0; b < E && !st; b++) {
+        size_t used = 0;
+        st = kvco_stream_decode(rec + off, len - off, nv, pl, &used);
+        if (st) break;
+        off += used;
+        for (uint32_t dd = 0; dd < D; dd++)
+          for (uint32_t t = 0; t < tcc; t++)
+            out[(((size_t)s * T + t0 + t) * D + dd) * E + b] = pl[(size_t)dd * tcc + t];
+      }
+      if (!st && off != len) st = KVCO_CORRUPT;
     }
   }
-  free(p0);
-  free(p1);
+  free(pl);
   if (!st && written) *written = out_bytes;
   return st;
 }

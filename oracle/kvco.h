@@ -34,7 +34,7 @@
 extern "C" {
 #endif
 
-enum { KVCO_BF16 = 1, KVCO_FP16 = 2 };
+enum { KVCO_BF16 = 1, KVCO_FP16 = 2, KVCO_F32 = 3 };
 enum { KVCO_LOSSLESS = 0, KVCO_TRANSFORM = 1 };
 enum {
   KVCO_OK = 0, KVCO_INVALID = 1, KVCO_CAPACITY = 2, KVCO_CORRUPT = 3,
@@ -42,7 +42,7 @@ enum {
 };
 
 typedef struct {
-  uint32_t dtype;            /* KVCO_BF16 or KVCO_FP16 */
+  uint32_t dtype;            /* KVCO_BF16, KVCO_FP16 or (lossless only) KVCO_F32 */
   uint32_t n_layers, n_heads, n_tokens, head_dim;
   uint32_t values_per_chunk; /* lossless chunk bound, 65536 */
   /* transform coding only */
@@ -73,9 +73,11 @@ size_t kvco_side_stream_encode(const uint8_t* sym, uint32_t n, uint8_t* out);
 int kvco_side_stream_decode(const uint8_t* rec, size_t avail, uint32_t n, uint8_t* sym, size_t* used);
 
 size_t kvco_lossless_bound(const kvco_desc* d, uint32_t n_slices);
+/* src / dst: [n_slices][T][D] little-endian values of 2 bytes (bf16, fp16)
+ * or 4 bytes (f32); cap in bytes. */
 size_t kvco_encode_lossless(const kvco_desc* d, uint32_t first_slice, uint32_t n_slices,
-                            const uint16_t* src, uint8_t* dst, size_t cap);
-int kvco_decode_lossless(const kvco_desc* d, const uint8_t* src, size_t n, uint16_t* dst,
+                            const void* src, uint8_t* dst, size_t cap);
+int kvco_decode_lossless(const kvco_desc* d, const uint8_t* src, size_t n, void* dst,
                          size_t cap, uint64_t* written);
 
 void kvco_rope_table(uint32_t T, uint32_t D, double theta, float* cs);

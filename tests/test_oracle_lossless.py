@@ -158,3 +158,89 @@ def test_plan_mismatch_and_capacity():
     other = oracle.Plan(oracle.BF16, 1, 1, 97, 128)
     assert oracle.decode_lossless(other, c)[0] == oracle.PLAN_MISMATCH
     assert oracle.decode_lossless(plan, c, n_slices_cap=0)[0] == oracle.CAPACITY
+
+
+def test_hand_worked_container_f32_2x2():
+    """f32 (QATQ and AT-1 code f32 tensors too): one slice of 2 tokens x 2
+    channels, chunks of 4 values. Values (t, d) = (0,0) 0x04030201, (0,1)
+    0x14131211, (1,0) 0x24232221, (1,1) 0x34333231; channel-major order (d, t)
+    is (0,0), (1,0), (0,1), (1,1), so plane p holds byte p of 0x..01, 0x..21,
+    0x..11, 0x..31 in that order: four RAW records, plane 0 first."""
+    plan = oracle.Plan(oracle.F32, 1, 1, 2, 2, values_per_chunk=4)
+    src = np.array([[[0x04030201, 0x14131211], [0x24232221, 0x34333231]]], np.uint32)
+    got = oracle.encode_lossless(plan, src)
+
+    def raw_stream(b):
+        return bytes([0, 0, 0, 0]) + struct.pack("<III", 32, 4, 0) + bytes(b) + bytes(12)
+
+    # byte p of value (t, d) is 0x01 + p + 0x10 * (2t + d); in channel-major order (0,0) (1,0) (0,1) (1,1)
+    record = b"".join(raw_stream([0x01 + p + 0x10 * k for k in (0, 2, 1, 3)]) for p in range(4))
+    n_rec, total = 1, 64 + 16 + len(record)
+    head = b"KVC1" + struct.pack("<HBB", 1, 0, 3) + struct.pack(
+        "<IIIIIIII", 1, 1, 2, 2, 0, 1, 2, n_rec) + struct.pack("<Q", total) + struct.pack(
+        "<IHHHH", 0, 0, 0, 0, 0)
+    index = struct.pack("<QII", 80, len(record), zlib.crc32(record))
+    head += struct.pack("<I", zlib.crc32(head + index))
+    assert got == head + index + record
+    st, back = oracle.decode_lossless(plan, got)
+    assert st == oracle.OK and np.array_equal(back, src)
+
+
+F32_CASES = [
+    _small("lossless-12x12x1024x64-f32", n_layers=1, n_heads=2),
+    _small("lossless-12x12x1024x64-f32", n_layers=1, n_heads=1, n_tokens=1500),  # ragged last chunk
+    _small("lossless-12x12x1024x64-f32", n_layers=1, n_heads=1, n_tokens=700, head_dim=128),
+    _small("lossless-12x12x1024x64-f32", n_layers=1, n_heads=1, n_tokens=5, head_dim=6, values_per_chunk=12),
+]
+
+
+@pytest.mark.parametrize("w", F32_CASES, ids=lambda w: f"{w.n_tokens}x{w.head_dim}")
+def test_f32_roundtrip_never_worse_and_planes(w):
+    """Round trip; size within raw + container overhead; every record is four
+    stream records whose lengths add up to the record; the sign/exponent plane
+    of the AR(1) fixture takes a RANS record (it carries the structure) and the
+    low mantissa plane is RAW."""
+    plan = oracle.Plan.from_workload(w)
+    x = kvgen.slices(w)
+    assert x.dtype == np.uint32
+    c = oracle.encode_lossless(plan, x)
+    assert len(c) <= oracle.lossless_bound(plan, w.n_slices)
+    st, y = oracle.decode_lossless(plan, c)
+    assert st == oracle.OK and np.array_equal(x, y)
+    n_rec = struct.unpack_from("<I", c, 36)[0]
+    modes = []
+    for i in range(n_rec):
+        off, ln, _ = struct.unpack_from("<QII", c, 64 + 16 * i)
+        o, m = 0, []
+        for _ in range(4):
+            m.append(c[off + o])
+            o += struct.unpack_from("<I", c, off + o + 4)[0]
+        assert o == ln
+        modes.append(m)
+    if w.n_tokens * w.head_dim >= 4096:
+        assert modes[0][0] == 0 and modes[0][3] == 2
+
+
+def test_f32_random_block_takes_raw_exactly():
+    """Uniform random bytes viewed as f32: four RAW streams per chunk, so the
+    size equals raw + 64 + (16 + 4 * 16) per chunk."""
+    w = _small("lossless-12x12x1024x64-f32", n_layers=1, n_heads=1)
+    plan = oracle.Plan.from_workload(w)
+    x = kvgen.random_bytes(w.raw_bytes, seed=5).view(np.uint32).reshape(w.n_slices, w.n_tokens, w.head_dim)
+    c = oracle.encode_lossless(plan, x)
+    n_chunks = w.n_slices * (w.n_tokens // (65536 // w.head_dim))
+    assert len(c) == w.raw_bytes + 64 + n_chunks * (16 + 4 * 16)
+    st, y = oracle.decode_lossless(plan, c)
+    assert st == oracle.OK and np.array_equal(x, y)
+
+
+def test_f32_tamper_refused():
+    w = _small("lossless-12x12x1024x64-f32", n_layers=1, n_heads=1, n_tokens=256)
+    plan = oracle.Plan.from_workload(w)
+    c = bytearray(oracle.encode_lossless(plan, kvgen.slices(w)))
+    rng = np.random.default_rng(3)
+    for pos in rng.integers(0, len(c), 60):
+        old = c[int(pos)]
+        c[int(pos)] = old ^ int(rng.integers(1, 256))
+        assert oracle.decode_lossless(plan, bytes(c))[0] != oracle.OK
+        c[int(pos)] = old
