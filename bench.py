@@ -49,12 +49,14 @@ KERNEL_WORK = {
     "transform_decode": ("tensor", lambda R, C, V: 2 * 128 * V),
 }
 
-# DRAM bytes (read + write) per frame of 64 MiB, from the ncu capture summarised
+# DRAM bytes (read + write) per frame of 64 MiB, from the ncu captures summarised
 # in profiles/kernels_qwen3-32b-32k_4frames.md (one launch over 4 frames, larger
 # than L2; the traffic of these kernels grows with the frames a launch covers).
 # A kernel that changed after that capture has no entry.
 DRAM_BYTES_PER_FRAME = {
     "lossless_encode": (759.9e6 + 353.7e6) / 4,
+    "transform_project": (304.5e6 + 100.5e6) / 4,
+    "transform_side": (14.0e6 + 0.001e6) / 4,
     "transform_entropy": (128.5e6 + 27.9e6) / 4,
     "lossless_decode": (198.8e6 + 220.9e6) / 4,
     "transform_decode": (199.5e6 + 221.8e6) / 4,

@@ -62,7 +62,10 @@ enum {
   KVC_ERR_UNSUPPORTED = 8    /* valid request this build does not handle */
 };
 
-enum { KVC_DTYPE_BF16 = 1, KVC_DTYPE_FP16 = 2 };
+/* Value types: 16-bit bf16 / fp16 (two byte planes) and, lossless only, f32
+ * (four byte planes; QATQ "qatq encode" and AT-1 "KV & tensor mode" code f32
+ * tensors too). */
+enum { KVC_DTYPE_BF16 = 1, KVC_DTYPE_FP16 = 2, KVC_DTYPE_F32 = 3 };
 enum { KVC_PATH_LOSSLESS = 0, KVC_PATH_TRANSFORM = 1 };
 
 /* Written by the device at the end of an encode or decode: status, and the
@@ -77,7 +80,8 @@ typedef struct kvc_plan_s kvc_plan_t;
 
 /* Plan description (host memory; copied by kvc_plan_create).
  *   abi_version       KVC_ABI_VERSION
- *   dtype             KVC_DTYPE_BF16 or KVC_DTYPE_FP16 (transform: bf16 only)
+ *   dtype             KVC_DTYPE_BF16, KVC_DTYPE_FP16 or KVC_DTYPE_F32 (f32:
+ *                     lossless only; transform: bf16 only)
  *   n_layers, n_heads, n_tokens, head_dim   cache shape L, H, T, D
  *   values_per_chunk  lossless chunk bound (65536): chunks hold
  *                     floor(values_per_chunk / D) tokens, at most 65536 values

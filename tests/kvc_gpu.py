@@ -7,7 +7,9 @@ import transform_codec_b200 as kvc
 
 
 def dev_u16(x: np.ndarray) -> torch.Tensor:
-    return torch.from_numpy(np.ascontiguousarray(x).view(np.int16).ravel()).cuda()
+    """Value bits on the device: int16 elements, or int32 for 4-byte values."""
+    x = np.ascontiguousarray(x)
+    return torch.from_numpy(x.view(np.int32 if x.itemsize == 4 else np.int16).ravel()).cuda()
 
 
 def encode(plan, path, x, first_slice=0):
@@ -22,19 +24,21 @@ def encode(plan, path, x, first_slice=0):
 
 
 def decode(plan, path, container: bytes, n_slices_cap: int):
-    """Status and decoded [n][T][D] uint16 of the GPU decode of a container."""
+    """Status and decoded [n][T][D] value bits (uint16, or uint32 for f32) of the
+    GPU decode of a container."""
     s = plan.shape
+    wide = s.dtype == kvc.F32
     codec = kvc.Codec(plan, path, max(n_slices_cap, 1))
     buf = torch.zeros(max(len(container), 16), dtype=torch.uint8, device="cuda")
     if container:
         buf[: len(container)] = torch.frombuffer(bytearray(container), dtype=torch.uint8).cuda()
-    out = torch.zeros(max(n_slices_cap * s.n_tokens * s.head_dim, 8), dtype=torch.int16,
-                      device="cuda")
+    out = torch.zeros(max(n_slices_cap * s.n_tokens * s.head_dim, 8),
+                      dtype=torch.int32 if wide else torch.int16, device="cuda")
     res = codec.decode(buf, len(container), out=out[: n_slices_cap * s.n_tokens * s.head_dim]
                        if n_slices_cap else out[:0])
     st, nbytes = kvc.read_result(res)
-    n = nbytes // (2 * s.n_tokens * s.head_dim)
-    y = out[: n * s.n_tokens * s.head_dim].cpu().numpy().view(np.uint16)
+    n = nbytes // ((4 if wide else 2) * s.n_tokens * s.head_dim)
+    y = out[: n * s.n_tokens * s.head_dim].cpu().numpy().view(np.uint32 if wide else np.uint16)
     return st, y.reshape(n, s.n_tokens, s.head_dim)
 
 

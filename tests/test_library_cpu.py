@@ -43,6 +43,8 @@ SHAPES = [
     kvc.Shape(kvc.FP16, 12, 12, 1024, 64),
     kvc.Shape(kvc.BF16, 1, 8, 3, 10, values_per_chunk=16),
     kvc.Shape(kvc.BF16, 64, 8, 32768, 128),
+    kvc.Shape(kvc.F32, 12, 12, 1024, 64),
+    kvc.Shape(kvc.F32, 1, 2, 700, 128),
 ]
 
 
@@ -62,7 +64,11 @@ def test_plan_validation():
         kvc.Plan(kvc.Shape(kvc.BF16, 0, 8, 512, 128))
     assert e.value.status == kvc.ERR_INVALID
     with pytest.raises(kvc.KvcError):
-        kvc.Plan(kvc.Shape(3, 1, 8, 512, 128))
+        kvc.Plan(kvc.Shape(4, 1, 8, 512, 128))  # no such value type
+    q = np.eye(128, dtype=np.float32)[None].repeat(16, 0)
+    with pytest.raises(kvc.KvcError) as e:  # f32 is lossless only
+        kvc.Plan(kvc.Shape(kvc.F32, 1, 8, 512, 128), bases=q, widths=np.ones((16, 128), np.uint8))
+    assert e.value.status == kvc.ERR_INVALID
     with pytest.raises(kvc.KvcError):
         kvc.Plan(kvc.Shape(kvc.BF16, 1, 8, 512, 128, values_per_chunk=100000))
 

@@ -17,7 +17,8 @@ LIB_PATH = os.path.join(_HERE, "libkvc.so")
 
 OK, ERR_INVALID, ERR_CAPACITY, ERR_CORRUPT, ERR_TRUNCATED, ERR_PLAN_MISMATCH = 0, 1, 2, 3, 4, 5
 ERR_TIMEOUT, ERR_CUDA, ERR_UNSUPPORTED = 6, 7, 8
-BF16, FP16 = 1, 2
+BF16, FP16, F32 = 1, 2, 3  # value types (f32: lossless only)
+DTYPE_F32 = F32
 LOSSLESS, TRANSFORM = 0, 1
 ABI_VERSION = 1
 
@@ -218,13 +219,14 @@ class Codec:
         s = plan.shape
         self.cap = plan.max_encoded_bytes(path, n_slices)
         self.out_elems = n_slices * s.n_tokens * s.head_dim
+        vt = torch.int32 if s.dtype == DTYPE_F32 else torch.int16  # one element per value
         self.container = torch.empty(max(self.cap, 16), dtype=torch.uint8, device=dev)
         self.ws_enc = torch.empty(max(plan.workspace_bytes(path, False, n_slices), 256),
                                   dtype=torch.uint8, device=dev)
         self.ws_dec = torch.empty(max(plan.workspace_bytes(path, True, n_slices), 256),
                                   dtype=torch.uint8, device=dev)
         self.res = torch.zeros(4, dtype=torch.int64, device=dev)  # kvc_result (16 bytes) x 2
-        self.decoded = torch.empty(max(self.out_elems, 8), dtype=torch.int16, device=dev)
+        self.decoded = torch.empty(max(self.out_elems, 8), dtype=vt, device=dev)
 
     def encode(self, src, first_slice: int = 0, stream=None, res=None):
         fn = _lib.kvc_encode_lossless if self.path == LOSSLESS else _lib.kvc_encode_transform

@@ -256,7 +256,7 @@ extern "C" int kvc_plan_create(const kvc_plan_desc* desc, kvc_plan_t** out) {
   *out = nullptr;
   const kvc_plan_desc& d = *desc;
   if (d.abi_version != KVC_ABI_VERSION) return KVC_ERR_INVALID;
-  if (d.dtype != KVC_DTYPE_BF16 && d.dtype != KVC_DTYPE_FP16) return KVC_ERR_INVALID;
+  if (d.dtype != KVC_DTYPE_BF16 && d.dtype != KVC_DTYPE_FP16 && d.dtype != KVC_DTYPE_F32) return KVC_ERR_INVALID;
   if (!d.n_layers || !d.n_heads || !d.n_tokens || !d.head_dim) return KVC_ERR_INVALID;
   if (uint64_t(d.n_layers) * 2u * d.n_heads > 0x7fffffffu) return KVC_ERR_INVALID;
   if (d.values_per_chunk < d.head_dim || d.values_per_chunk > kMaxChunkValues) return KVC_ERR_INVALID;
@@ -271,6 +271,7 @@ extern "C" int kvc_plan_create(const kvc_plan_desc* desc, kvc_plan_t** out) {
   p->ls.D = d.head_dim;
   p->ls.tc = d.values_per_chunk / d.head_dim;
   p->ls.cps = (d.n_tokens + p->ls.tc - 1) / p->ls.tc;
+  p->ls.E = d.dtype == KVC_DTYPE_F32 ? 4u : 2u;
   if (d.bases) {
     int st = KVC_OK;
     if (d.dtype != KVC_DTYPE_BF16 || (d.head_dim & 1u) || d.max_bits > 8 || !(d.rope_theta > 0.0) ||
@@ -494,6 +495,7 @@ int decode_frames(const kvc_plan_s* plan, int path, const kvc_frame* fr, uint32_
   ex.L = plan->d.n_layers; ex.H = plan->d.n_heads; ex.T = plan->d.n_tokens; ex.D = plan->d.head_dim;
   ex.recs_per_slice = records_per_slice(plan, path);
   ex.max_slices = max_slices;
+  ex.E = path == KVC_PATH_LOSSLESS ? plan->ls.E : 2u;
   if (path == KVC_PATH_LOSSLESS) {
     ex.chunk_tokens = plan->ls.tc;
   } else {
@@ -567,7 +569,7 @@ extern "C" size_t kvc_max_encoded_bytes(const kvc_plan_t* plan, int path, uint32
     uint64_t per = 0;
     for (uint32_t t0 = 0; t0 < s.T; t0 += s.tc) {
       uint32_t tcc = std::min(s.tc, s.T - t0);
-      per += kIndexEntry + 2u * (16u + pad16u(uint64_t(tcc) * s.D));
+      per += kIndexEntry + s.E * (16u + pad16u(uint64_t(tcc) * s.D));
     }
     return size_t(kHeaderBytes + per * n_slices);
   }

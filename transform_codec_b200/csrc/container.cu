@@ -208,7 +208,7 @@ k_check_container(FrameBatch b, ContainerExpect e, uint8_t* ws) {
       bad = __syncthreads_or(bad);
       if (tid == 0) {
         int st = bad ? kErrCorrupt : kOk;
-        if (st == kOk && (uint64_t(ns_s) * e.T * e.D * 2u > b.f[f].dst_cap || ns_s > e.max_slices))
+        if (st == kOk && (uint64_t(ns_s) * e.T * e.D * e.E > b.f[f].dst_cap || ns_s > e.max_slices))
           st = kErrCapacity;
         st_s = st;
       }
@@ -222,7 +222,7 @@ k_check_container(FrameBatch b, ContainerExpect e, uint8_t* ws) {
     ds->n_slices = st == kOk ? ns_s : 0;
     ds->n_records = st == kOk ? nr_s : 0;
     ds->err_key = ~0ull;
-    ds->out_bytes = st == kOk ? uint64_t(ns_s) * e.T * e.D * 2u : 0;
+    ds->out_bytes = st == kOk ? uint64_t(ns_s) * e.T * e.D * e.E : 0;
     if (f == 0) batch_state(ws)->n_deferred = 0;
     res->status = st;
     res->bytes = 0;

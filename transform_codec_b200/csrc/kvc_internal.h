@@ -85,6 +85,7 @@ struct EncodeLayout {
 // What a valid container header must carry for this plan.
 struct ContainerExpect {
   uint32_t path, dtype, L, H, T, D, chunk_tokens;
+  uint32_t E;                  // bytes per value of the decoded output
   uint32_t n_sink, n_recent, block_tokens, plan_crc;
   uint32_t recs_per_slice;     // records per slice
   uint32_t max_slices;         // slices a container may hold in this call
@@ -117,6 +118,7 @@ __device__ inline uint32_t frame_of(const uint32_t* base, uint32_t n, uint32_t g
 // lossless
 struct LosslessShape {
   uint32_t T, D, tc, cps;      // tokens, head_dim, chunk tokens, chunks per slice
+  uint32_t E;                  // bytes per value (byte planes per chunk): 2, or 4 for f32
 };
 uint64_t lossless_slot_bytes(const LosslessShape& s);
 cudaError_t launch_lossless_encode(const LosslessShape& s, const FrameBatch& b,

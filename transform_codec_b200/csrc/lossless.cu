@@ -1046,6 +1046,213 @@ k_lossless_decode_fast(LosslessShape sh, FrameBatch b, uint8_t* ws) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Wide values (f32: four byte planes; QATQ and AT-1 code f32 tensors too).
+// Encode: one CTA per chunk, 512 threads. The planes are coded one after
+// another through one shared plane buffer of the chunk's size: plane p is
+// gathered channel-major from the chunk (which stays in L2 across the
+// planes), counted (and, for the upper planes, which hold the sign and
+// exponent bits, its lane deltas too), its tables built, coded by one warp per
+// (variant, rANS group), and its stream record written at the record's
+// running offset by the never-worse rule. The record's CRC follows.
+struct __align__(16) WideEncSmem {
+  uint32_t crc_t[1024];
+  uint32_t hist[2][256], freq[2][256], rem[256], fc[2][256], rcp[2][256];
+  uint32_t states[2][kMaxLanes];
+  uint32_t tmp[32], red[32];
+  uint32_t k[2], W[2][4], wbeg[2][4], sub_len[2][4];
+  uint32_t mode, bytes, var, off;
+};
+
+template <uint32_t E>
+__global__ void __launch_bounds__(kEncThreads)
+k_lossless_encode_wide(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  WideEncSmem& S = *reinterpret_cast<WideEncSmem*>(smem_raw);
+  uint8_t* pl = smem_raw + sizeof(WideEncSmem);  // one plane of the chunk, channel-major
+  const uint32_t tid = threadIdx.x, nthr = blockDim.x, warp = tid >> 5, lane = tid & 31u;
+  const uint32_t gr = blockIdx.x;
+  const uint32_t fr = frame_of(b.rec_base, b.n, gr), r = gr - b.rec_base[fr];
+  const uint32_t slice = r / sh.cps, c = r % sh.cps;
+  const uint32_t t0 = c * sh.tc, tcc = min(sh.tc, sh.T - t0), D = sh.D, n = tcc * D;
+  const uint32_t n_max = sh.tc * D;
+  const uint8_t* g = b.f[fr].src + (uint64_t(slice) * sh.T + t0) * D * E;
+  uint8_t* rec = ws.slots + uint64_t(gr) * ws.slot_bytes;
+  uint16_t* scratch0 = reinterpret_cast<uint16_t*>(rec + E * (16u + pad16(n_max)));
+  const uint32_t N = rans_lanes(n), G = rans_groups(N), raw_b = 16u + pad16(n);
+  crc_tables_init(S.crc_t);
+  if (tid == 0) S.off = 0;
+  for (uint32_t p = 0; p < E; ++p) {
+    const bool upper = 2u * p >= E;
+    const uint32_t nvar = upper ? 2u : 1u;
+    for (uint32_t i = tid; i < 2u * 256u; i += nthr) (&S.hist[0][0])[i] = 0;
+    for (uint32_t q = tid; q < n; q += nthr) {
+      const uint32_t t = q / D, d = q - t * D;
+      pl[d * tcc + t] = g[uint64_t(q) * E + p];
+    }
+    __syncthreads();
+    for (uint32_t i = tid; i < n; i += nthr) {
+      const uint32_t v = pl[i];
+      atomicAdd(&S.hist[0][v], 1u);
+      if (upper) atomicAdd(&S.hist[1][lane_start(i, n, N) ? v : (v ^ pl[i - 1])], 1u);
+    }
+    __syncthreads();
+    for (uint32_t v = 0; v < nvar; ++v) {
+      const uint32_t k = block_normalize(S.hist[v], n, S.freq[v], S.rem, S.tmp);
+      if (tid == 0) S.k[v] = k;
+      block_enc_tables(S.freq[v], S.fc[v], S.rcp[v], S.tmp);
+    }
+    __syncthreads();
+    {
+      const uint32_t v = warp >> 2, gg = warp & 3u;
+      if (v < nvar && S.k[v] >= 2 && gg < G) {
+        uint32_t b0, len0, b1 = n, len1;
+        lane_range(n, N, gg * kGroupLanes, b0, len0);
+        if (gg + 1 < G) lane_range(n, N, (gg + 1) * kGroupLanes, b1, len1);
+        uint16_t* scratch = scratch0 + uint64_t(v) * (n_max + 32u);
+        uint32_t x, Wg;
+        if (v == 0)
+          Wg = rans_encode_group([pl](uint32_t i) -> uint32_t { return pl[i]; }, n, N, gg, S.fc[0], S.rcp[0],
+                                 scratch + b0, b1 - b0, &x);
+        else
+          Wg = rans_encode_group(
+              [pl, n, N](uint32_t i) -> uint32_t {
+                return lane_start(i, n, N) ? uint32_t(pl[i]) : uint32_t(pl[i] ^ pl[i - 1]);
+              },
+              n, N, gg, S.fc[1], S.rcp[1], scratch + b0, b1 - b0, &x);
+        const uint32_t l = gg * kGroupLanes + lane;
+        if (l < N) S.states[v][l] = x;
+        if (lane == 0) {
+          S.W[v][gg] = Wg;
+          S.wbeg[v][gg] = b0 + (b1 - b0) - Wg;
+        }
+      }
+    }
+    __syncthreads();
+    if (tid == 0) {  // CONST; lane-delta RANS if strictly smaller than plain RANS and RAW; RANS; RAW
+      const uint32_t k = S.k[0];
+      uint32_t mode = kModeRaw, bytes = raw_b, var = 0;
+      if (k == 1) {
+        mode = kModeConst;
+        bytes = 16;
+      } else if (k >= 2) {
+        const uint32_t rb = rans_layout(n, k, S.W[0], S.sub_len[0]);
+        const uint32_t rd = upper && S.k[1] >= 2 ? rans_layout(n, S.k[1], S.W[1], S.sub_len[1]) : 0xffffffffu;
+        if (rd < rb && rd < raw_b) {
+          mode = kModeRans; bytes = rd; var = 1;
+        } else if (rb < raw_b) {
+          mode = kModeRans; bytes = rb;
+        }
+      }
+      S.mode = mode; S.bytes = bytes; S.var = var;
+    }
+    __syncthreads();
+    const uint32_t v = S.var;
+    block_write_stream(rec + S.off, S.mode, n, S.bytes, uint32_t(pl[0]), S.k[v], S.freq[v], S.states[v],
+                       scratch0 + uint64_t(v) * (n_max + 32u), S.wbeg[v], S.W[v], S.sub_len[v],
+                       [pl](uint32_t i) -> uint32_t { return pl[i]; }, S.tmp, v);
+    __syncthreads();
+    if (tid == 0) S.off += S.bytes;
+    __syncthreads();
+  }
+  const uint32_t len = S.off;
+  const uint32_t crc = crc32_block_aligned(rec, len, S.crc_t, S.red);
+  if (tid == 0) {
+    ws.rec_len[gr] = len;
+    ws.rec_crc[gr] = crc;
+  }
+}
+
+// Decode of wide values: persistent CTAs of 256 threads over the batch's
+// records. Per record the CRC, then per plane: its stream record checked, a
+// RANS table built, the plane decoded into shared memory (one warp per rANS
+// group, lane deltas undone per lane) and written as byte p of every value of
+// the chunk; the stream records must fill the record exactly.
+struct __align__(16) WideDecSmem {
+  uint32_t crc_t[1024];
+  uint32_t freq[256], cum[260], lut[kProbScale];
+  uint32_t tmp[32], red[32];
+  StreamInfo si;
+  uint32_t crc_ok;
+  uint32_t base[kBatchMax + 1];
+};
+
+template <uint32_t E>
+__global__ void __launch_bounds__(kThreads)
+k_lossless_decode_wide(LosslessShape sh, FrameBatch b, uint8_t* ws) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  WideDecSmem& S = *reinterpret_cast<WideDecSmem*>(smem_raw);
+  uint8_t* pl = smem_raw + sizeof(WideDecSmem);
+  const uint32_t tid = threadIdx.x, nthr = blockDim.x, warp = tid >> 5;
+  if (tid == 0) {  // records of the batch: prefix over frames that passed the header check
+    uint32_t acc = 0;
+    for (uint32_t f = 0; f < b.n; ++f) {
+      S.base[f] = acc;
+      const DecodeState* d = decode_state(ws, f);
+      acc += d->status == kOk ? d->n_records : 0u;
+    }
+    S.base[b.n] = acc;
+  }
+  __syncthreads();
+  const uint32_t nrec = S.base[b.n], D = sh.D;
+  if (blockIdx.x >= nrec) return;
+  crc_tables_init(S.crc_t);
+  for (uint32_t g = blockIdx.x; g < nrec; g += gridDim.x) {
+    __syncthreads();
+    const uint32_t fr = frame_of(S.base, b.n, g), r = g - S.base[fr];
+    const uint8_t* src = b.f[fr].src;
+    DecodeState* ds = decode_state(ws, fr);
+    const uint8_t* e = src + kHeaderBytes + uint64_t(kIndexEntry) * r;
+    const uint64_t roff = ld_u64(e);
+    const uint32_t len = ld_u32(e + 8), want = ld_u32(e + 12);
+    const uint8_t* rec = src + roff;
+    const uint32_t slice = r / sh.cps, c = r % sh.cps;
+    const uint32_t t0 = c * sh.tc, tcc = min(sh.tc, sh.T - t0), n = tcc * D;
+    uint8_t* out = b.f[fr].dst + (uint64_t(slice) * sh.T + t0) * D * E;
+    const uint32_t got = crc32_block_aligned(rec, len, S.crc_t, S.red);
+    if (tid == 0) S.crc_ok = (got == want);
+    __syncthreads();
+    int st = S.crc_ok ? kOk : kErrCorrupt;
+    const uint32_t N = rans_lanes(n), G = rans_groups(N);
+    uint32_t off = 0;
+    for (uint32_t p = 0; p < E && st == kOk; ++p) {
+      st = block_parse_stream(rec + off, len - off, n, &S.si, S.freq, S.tmp);
+      if (st != kOk) break;
+      const StreamInfo si = S.si;
+      if (si.mode == kModeRans) {
+        block_dec_lut(S.freq, S.cum, S.lut, S.tmp);
+      } else if (si.mode == kModeRaw) {
+        for (uint32_t i = tid; i < n; i += nthr) pl[i] = rec[off + 16u + i];
+      } else {
+        for (uint32_t i = tid; i < n; i += nthr) pl[i] = uint8_t(si.sym);
+      }
+      __syncthreads();
+      bool ok = true;
+      if (si.mode == kModeRans && warp < G) {
+        const uint32_t dm = si.delta ? 0xffu : 0u;
+        uint32_t prev = 0;
+        ok = rans_decode_group(rec + off + si.sub_off[warp], si.sub_len[warp], n, N, warp, S.lut,
+                               [&](uint32_t i, uint32_t s) {
+                                 prev = s ^ (prev & dm);
+                                 pl[i] = uint8_t(prev);
+                               });
+      }
+      if (!__syncthreads_and(ok)) {
+        st = kErrCorrupt;
+        break;
+      }
+      for (uint32_t q = tid; q < n; q += nthr) {
+        const uint32_t t = q / D, d = q - t * D;
+        out[uint64_t(q) * E + p] = pl[d * tcc + t];
+      }
+      off += si.bytes;
+      __syncthreads();  // the plane buffer and the stream info are reused
+    }
+    if (st == kOk && off != len) st = kErrCorrupt;
+    if (st != kOk && tid == 0) atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(st));
+  }
+}
+
 int g_num_sms = 0;
 int num_sms() {
   if (!g_num_sms) {
@@ -1061,7 +1268,11 @@ int num_sms() {
 
 uint64_t lossless_slot_bytes(const LosslessShape& s) {
   const uint64_t n_max = uint64_t(s.tc) * s.D;
-  uint64_t b = 2u * (16u + pad16_64(n_max)) + 3u * (2u * n_max + 64u);  // records + 3 word scratch areas
+  // the record (a stream per byte plane, each at most RAW), then the word
+  // scratch of the variants coded side by side: three for 16-bit values
+  // (plane 0, plane 1 and its lane deltas), two for wide values (one plane at
+  // a time and its lane deltas)
+  uint64_t b = s.E * (16u + pad16_64(n_max)) + (s.E == 4u ? 2u : 3u) * (2u * n_max + 64u);
   return (b + 255u) & ~uint64_t(255);
 }
 
@@ -1069,6 +1280,15 @@ cudaError_t launch_lossless_encode(const LosslessShape& s, const FrameBatch& b,
                                    const EncodeLayout& ws, cudaStream_t st) {
   const uint32_t nrec = b.rec_base[b.n];
   if (nrec == 0) return cudaSuccess;
+  if (s.E == 4u) {  // f32: the plane-at-a-time encoder for every chunk
+    const size_t smem = sizeof(WideEncSmem) + pad16(s.tc * s.D);
+    cudaError_t e = cudaFuncSetAttribute(k_lossless_encode_wide<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(smem));
+    if (e != cudaSuccess) return e;
+    ProfRange pr_("lossless_encode_wide", st);
+    k_lossless_encode_wide<4><<<nrec, kEncThreads, smem, st>>>(s, b, ws);
+    return cudaGetLastError();
+  }
   // full chunks of 65536 values with D = 128 or 64 and 16-byte aligned input go
   // to the fast encoder; the general one takes the rest (with the fast one, only
   // the ragged last chunk of each slice)
@@ -1101,6 +1321,16 @@ cudaError_t launch_lossless_encode(const LosslessShape& s, const FrameBatch& b,
 cudaError_t launch_lossless_decode(const LosslessShape& s, const FrameBatch& b, uint8_t* ws,
                                    uint32_t max_records, cudaStream_t st) {
   if (max_records == 0 || b.n == 0) return cudaSuccess;
+  if (s.E == 4u) {  // f32: the plane-at-a-time decoder for every record
+    const size_t smem = sizeof(WideDecSmem) + pad16(s.tc * s.D);
+    cudaError_t e = cudaFuncSetAttribute(k_lossless_decode_wide<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         int(smem));
+    if (e != cudaSuccess) return e;
+    ProfRange pr_("lossless_decode_wide", st);
+    const uint32_t grid = min(max_records, uint32_t(num_sms() * 2));
+    k_lossless_decode_wide<4><<<grid, kThreads, smem, st>>>(s, b, ws);
+    return cudaGetLastError();
+  }
   static int fast_blocks_per_sm = 0;
   const size_t fsmem = sizeof(FastSmem);
   cudaError_t e = cudaFuncSetAttribute(k_lossless_decode_fast,
