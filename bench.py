@@ -57,7 +57,6 @@ DRAM_BYTES_PER_FRAME = {
     "lossless_encode": (759.9e6 + 353.7e6) / 4,
     "transform_project": (304.5e6 + 100.5e6) / 4,
     "transform_side": (14.0e6 + 0.001e6) / 4,
-    "transform_entropy": (128.5e6 + 27.9e6) / 4,
     "lossless_decode": (198.8e6 + 220.9e6) / 4,
     "transform_decode": (199.5e6 + 221.8e6) / 4,
 }
@@ -278,48 +277,83 @@ class Job:
 def run_e2e(job, steps, warmup):
     """Host-to-host through the public API: per frame, pinned H2D of the raw
     frame, both encodes, D2H of both containers, both decodes and D2H of both
-    decoded frames; one CUDA stream, device-timed with events."""
+    decoded frames. Three CUDA streams overlap the copies with the codec: the
+    H2D of frame f + 1 and the D2H of frame f - 1 run while frame f is coded
+    (two-deep device rings; events order the reuse of each buffer). The host
+    reads each frame's container sizes once its encodes are done, since the
+    decoders and the container copies take exact byte counts. Device-timed
+    with events around the whole step."""
     torch, kvc = job.torch, job.kvc
-    stage_in = torch.empty(job.frame_vals, dtype=torch.int16, device="cuda")
-    dev_out = torch.empty(job.frame_vals, dtype=torch.int16, device="cuda")
+    F = job.frames
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    stage = [torch.empty(job.frame_vals, dtype=torch.int16, device="cuda") for _ in range(2)]
+    dec_l = [torch.empty(job.frame_vals, dtype=torch.int16, device="cuda") for _ in range(2)]
+    dec_t = [torch.empty(job.frame_vals, dtype=torch.int16, device="cuda") for _ in range(2)]
     h_cont_l = torch.empty(job.cap_l, dtype=torch.uint8).pin_memory()
     h_cont_t = torch.empty(job.cap_t, dtype=torch.uint8).pin_memory()
     h_out = torch.empty(2 * job.frame_vals, dtype=torch.int16).pin_memory()
-    res = torch.zeros(4, 2, dtype=torch.int64, device="cuda")
-    h_res = torch.zeros(4, 2, dtype=torch.int64).pin_memory()
+    res = torch.zeros(F, 4, 2, dtype=torch.int64, device="cuda")
+    h_res = torch.zeros(F, 2, 2, dtype=torch.int64).pin_memory()
     cl, ct = job.codec_l, job.codec_t
+    ev = lambda: torch.cuda.Event()  # noqa: E731
     d2h = 0
 
     def one_step():
         nonlocal d2h
         d2h = 0
-        for f in range(job.frames):
-            stage_in.copy_(job.host[f * job.frame_vals:(f + 1) * job.frame_vals], non_blocking=True)
-            cl.container = job.cont_l[: job.cap_l]
-            ct.container = job.cont_t[: job.cap_t]
-            cl.encode(stage_in, f * job.spf, res=res[0])
-            ct.encode(stage_in, f * job.spf, res=res[1])
-            h_res[:2].copy_(res[:2], non_blocking=True)
-            torch.cuda.current_stream().synchronize()
-            nl, nt = int(h_res[0, 1]), int(h_res[1, 1])
-            h_cont_l[:nl].copy_(cl.container[:nl], non_blocking=True)
-            h_cont_t[:nt].copy_(ct.container[:nt], non_blocking=True)
-            cl.decode(cl.container, nl, out=dev_out, res=res[2])
-            h_out[: job.frame_vals].copy_(dev_out, non_blocking=True)
-            ct.decode(ct.container, nt, out=dev_out, res=res[3])
-            h_out[job.frame_vals:].copy_(dev_out, non_blocking=True)
+        ev_in, ev_enc, ev_cmp, ev_out = [ev() for _ in range(F)], [ev() for _ in range(F)], \
+            [ev() for _ in range(F)], [ev() for _ in range(F)]
+
+        def h2d(f):
+            if f >= 2:
+                s_in.wait_event(ev_cmp[f - 2])  # stage[f % 2] read by frame f - 2's encodes
+            with torch.cuda.stream(s_in):
+                stage[f % 2].copy_(job.host[f * job.frame_vals:(f + 1) * job.frame_vals], non_blocking=True)
+            ev_in[f].record(s_in)
+
+        h2d(0)
+        for f in range(F):
+            if f + 1 < F:
+                h2d(f + 1)
+            cl.container = job.cont_l[f * job.cap_l:(f + 1) * job.cap_l]
+            ct.container = job.cont_t[f * job.cap_t:(f + 1) * job.cap_t]
+            s_cmp.wait_event(ev_in[f])
+            cl.encode(stage[f % 2], f * job.spf, stream=s_cmp, res=res[f, 0])
+            ct.encode(stage[f % 2], f * job.spf, stream=s_cmp, res=res[f, 1])
+            with torch.cuda.stream(s_cmp):
+                h_res[f].copy_(res[f, :2], non_blocking=True)
+            ev_enc[f].record(s_cmp)
+            ev_enc[f].synchronize()
+            nl, nt = int(h_res[f, 0, 1]), int(h_res[f, 1, 1])
+            if f >= 2:
+                s_cmp.wait_event(ev_out[f - 2])  # dec_*[f % 2] copied out for frame f - 2
+            cl.decode(cl.container, nl, out=dec_l[f % 2], stream=s_cmp, res=res[f, 2])
+            ct.decode(ct.container, nt, out=dec_t[f % 2], stream=s_cmp, res=res[f, 3])
+            ev_cmp[f].record(s_cmp)
+            s_out.wait_event(ev_cmp[f])
+            with torch.cuda.stream(s_out):
+                h_cont_l[:nl].copy_(cl.container[:nl], non_blocking=True)
+                h_cont_t[:nt].copy_(ct.container[:nt], non_blocking=True)
+                h_out[: job.frame_vals].copy_(dec_l[f % 2], non_blocking=True)
+                h_out[job.frame_vals:].copy_(dec_t[f % 2], non_blocking=True)
+            ev_out[f].record(s_out)
             d2h += nl + nt + 2 * job.frame_bytes
+        s_in.wait_event(ev_out[F - 1])
+        s_in.wait_event(ev_cmp[F - 1])
 
     for _ in range(warmup):
         one_step()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
+    e0.record(s_in)
     for _ in range(steps):
         one_step()
-    e1.record()
+    e1.record(s_in)
     torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / steps
+    st = res[:, :, 0].cpu().numpy() & 0xFFFFFFFF
+    if st.any():
+        raise RuntimeError(f"end-to-end step: codec status {set(st.ravel().tolist())}")
     return ms, job.raw_bytes, d2h
 
 

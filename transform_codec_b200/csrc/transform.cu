@@ -724,7 +724,7 @@ __device__ inline uint32_t rans_encode_rows(const uint8_t* row, bool live, const
   return cap - pos;
 }
 
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, 5)
 k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLayout ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   EntSmem& S = *reinterpret_cast<EntSmem*>(smem_raw);
@@ -1373,7 +1373,7 @@ struct __align__(1024) DecSmem {
 
 static_assert(sizeof(DecSmem) + 1024 <= 232448, "decoder shared memory exceeds the per-block limit");
 static_assert(sizeof(ProjSmem) <= 232448, "projection shared memory exceeds the per-block limit");
-static_assert(sizeof(EntSmem) <= 232448 / 4, "entropy kernel should fit four blocks per SM");
+static_assert(sizeof(EntSmem) + 1024 <= 233472 / 5, "entropy kernel should fit five blocks per SM");
 
 __global__ void __launch_bounds__(kThreads, 1)
 k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t* ws, uint32_t max_records) {
