@@ -17,6 +17,8 @@
  *                with a scale and zero point per 64-token block (KVTC page, "How
  *                the Pipeline Works", "Why RoPE Has to Be Reversed First", "Bit
  *                Budget Is Not Fair"; Codec-Gauge page, "Compression Conditions").
+ *                The fp32 zero points and scales of a record are themselves
+ *                entropy coded: four byte-plane streams of all z, then all s.
  *   back-end   — chunked, 128-lane interleaved rANS with per-stream frequency
  *                tables (KVTC page, "rANS Makes the Last Mile Smaller").
  *   container  — 64-byte header, chunk-offset index with a CRC-32 per record,
