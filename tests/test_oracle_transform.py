@@ -125,6 +125,39 @@ def test_allocation_matches_brute_force():
             assert _distortion(lam, w) <= best * (1 + 1e-12)
 
 
+def _dp_min_distortion(lam, budget, max_bits=8):
+    """Dynamic programming over units (KVTC "Bit Budget Is Not Fair": the
+    reference path allocates by dynamic programming): best[c] is the least
+    distortion of the units so far with exactly c bits spent."""
+    best = np.full(budget + 1, np.inf)
+    best[0] = 0.0
+    for l in lam:
+        nxt = np.full(budget + 1, np.inf)
+        for b in range(max_bits + 1):
+            if b > budget:
+                break
+            cand = best[: budget + 1 - b] + l * 4.0 ** (-b)
+            nxt[b:] = np.minimum(nxt[b:], cand)
+        best = nxt
+    return best[budget]
+
+
+@pytest.mark.parametrize("k", [16, 64, 200])
+def test_allocation_equals_dynamic_programming(k):
+    """The greedy allocation reaches the dynamic-programming optimum of
+    sum lam * 4^-b at every budget (the marginal gains lam * 3/4 * 4^-b fall
+    with b, so taking the largest gain first is exact)."""
+    rng = np.random.default_rng(k)
+    lam = np.exp(rng.standard_normal(k) * 3)
+    lam[rng.integers(0, k, k // 8)] = lam[0]  # ties
+    for avg in (0.25, 1.0, 1.6, 2.0, 4.5, 7.9):
+        w = oracle.allocate(lam, avg, 8)
+        budget = int(np.floor(avg * k + 0.5))
+        assert int(w.sum()) == budget
+        opt = _dp_min_distortion(lam, budget)
+        assert abs(_distortion(lam, w) - opt) <= 1e-12 * max(opt, 1e-300) + 1e-300
+
+
 def test_allocation_ties_go_to_lower_index_and_cap():
     w = oracle.allocate(np.ones(3), 4 / 3, 8)
     assert list(w) == [2, 1, 1]
