@@ -545,106 +545,55 @@ def run_reference(args):
 def run_migration(args):
     """Host-streamed migration of the 50,331,648-byte live-migration block
     (QATQ "Measured evidence": raw streamed blocks against the codec's
-    transferred bytes), lossless, through the public API. Send: per frame of
-    `--migration-slices` slices, the pinned H2D copy of the raw frame, the
-    encode and the D2H copy of its container; receive: the H2D copy of each
-    container, the decode and the D2H copy of the restored frame. Three CUDA
-    streams overlap the copies with the codec (three-deep device rings); the
-    host reads each container's size two frames after its encode was issued,
-    so the copy engines never wait on it. Device-timed with events; the
-    restored bytes are checked against the input."""
+    transferred bytes), lossless, through the library's host-streamed calls:
+    send = kvc_stream_encode_host (pinned H2D of each frame of
+    `--migration-slices` slices, encode, D2H of its container), receive =
+    kvc_stream_decode_host (H2D of each container, decode, D2H of the restored
+    frame); each call overlaps the copies with the codec on three streams.
+    Device-timed with events around each blocking call; the restored bytes are
+    checked against the input."""
     import torch
 
     import kvgen
     import transform_codec_b200 as kvc
     w = kvgen.WORKLOADS["lossless-8x8x1536x128-bf16"]
     spf = args.migration_slices
-    F = w.n_slices // spf
-    fv = spf * w.n_tokens * w.head_dim
-    host = torch.empty(F * fv, dtype=torch.int16).pin_memory()
-    kvgen.slices(w, 0, F * spf, out=host.data_ptr())
+    n = w.n_slices
+    F = -(-n // spf)
+    host = torch.empty(n * w.n_tokens * w.head_dim, dtype=torch.int16).pin_memory()
+    kvgen.slices(w, 0, n, out=host.data_ptr())
     plan = kvc.Plan(kvc.Shape.from_workload(w))
-    R = 3  # ring depth of the device buffers
-    codecs = [kvc.Codec(plan, kvc.LOSSLESS, spf) for _ in range(R)]
-    cap = codecs[0].cap
-    h_cont = torch.empty(F * cap, dtype=torch.uint8).pin_memory()
-    h_back = torch.empty(F * fv, dtype=torch.int16).pin_memory()
-    stage = [torch.empty(fv, dtype=torch.int16, device="cuda") for _ in range(R)]
-    cbuf = [torch.empty(cap, dtype=torch.uint8, device="cuda") for _ in range(R)]
-    outb = [torch.empty(fv, dtype=torch.int16, device="cuda") for _ in range(R)]
-    res = torch.zeros(F, 2, 2, dtype=torch.int64, device="cuda")
-    h_res = torch.zeros(F, 2, dtype=torch.int64).pin_memory()
-    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    sizes = [0] * F
+    cap = sum(plan.max_encoded_bytes(kvc.LOSSLESS, min(spf, n - f * spf)) for f in range(F))
+    h_cont = torch.empty(cap, dtype=torch.uint8).pin_memory()
+    h_back = torch.empty_like(host).pin_memory()
+    fb = torch.zeros(F, dtype=torch.int64)
+    res = torch.zeros(F, 2, dtype=torch.int64).pin_memory()
+    buf = torch.empty(kvc.stream_buffer_bytes(plan, kvc.LOSSLESS, spf), dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.Stream()
 
     def send():
-        ev_in, ev_enc, ev_out = ([torch.cuda.Event() for _ in range(F)] for _ in range(3))
-
-        def d2h(g):  # frame g's container, once its encode has reported the size
-            ev_enc[g].synchronize()
-            sizes[g] = n = int(h_res[g, 1])
-            s_out.wait_event(ev_enc[g])
-            with torch.cuda.stream(s_out):
-                h_cont[g * cap:g * cap + n].copy_(codecs[g % R].container[:n], non_blocking=True)
-            ev_out[g].record(s_out)
-
-        for f in range(F):
-            if f >= R:
-                s_in.wait_event(ev_enc[f - R])  # stage[f % R] read by frame f - R's encode
-            with torch.cuda.stream(s_in):
-                stage[f % R].copy_(host[f * fv:(f + 1) * fv], non_blocking=True)
-            ev_in[f].record(s_in)
-            if f >= R - 1:
-                d2h(f - (R - 1))  # two frames back: its encode is normally done by now
-            s_cmp.wait_event(ev_in[f])
-            if f >= R:
-                s_cmp.wait_event(ev_out[f - R])  # codec f % R's container copied out
-            codecs[f % R].encode(stage[f % R], f * spf, stream=s_cmp, res=res[f, 0])
-            with torch.cuda.stream(s_cmp):
-                h_res[f].copy_(res[f, 0], non_blocking=True)
-            ev_enc[f].record(s_cmp)
-        for g in range(max(0, F - (R - 1)), F):
-            d2h(g)
-        s_in.wait_event(ev_out[F - 1])
+        kvc.stream_encode_host(plan, kvc.LOSSLESS, 0, n, spf, host, h_cont, fb, res, buf, stream=stream)
 
     def receive():
-        ev_in, ev_dec, ev_out = ([torch.cuda.Event() for _ in range(F)] for _ in range(3))
-        for f in range(F):
-            n = sizes[f]
-            if f >= R:
-                s_in.wait_event(ev_dec[f - R])  # cbuf[f % R] read by frame f - R's decode
-            with torch.cuda.stream(s_in):
-                cbuf[f % R][:n].copy_(h_cont[f * cap:f * cap + n], non_blocking=True)
-            ev_in[f].record(s_in)
-            s_cmp.wait_event(ev_in[f])
-            if f >= R:
-                s_cmp.wait_event(ev_out[f - R])  # outb[f % R] copied out for frame f - R
-            codecs[f % R].decode(cbuf[f % R], n, out=outb[f % R], stream=s_cmp, res=res[f, 1])
-            ev_dec[f].record(s_cmp)
-            s_out.wait_event(ev_dec[f])
-            with torch.cuda.stream(s_out):
-                h_back[f * fv:(f + 1) * fv].copy_(outb[f % R], non_blocking=True)
-            ev_out[f].record(s_out)
-        s_in.wait_event(ev_out[F - 1])
+        kvc.stream_decode_host(plan, kvc.LOSSLESS, n, spf, h_cont, fb, h_back, res, buf, stream=stream)
 
     def timed(fn, steps, warmup):
         for _ in range(warmup):
             fn()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(s_in)
+        e0.record(stream)
         for _ in range(steps):
             fn()
-        e1.record(s_in)
+        e1.record(stream)
         torch.cuda.synchronize()
         return e0.elapsed_time(e1) / steps
 
     ms_send = timed(send, args.steps, args.warmup)
+    sent = int(fb.sum())
     ms_recv = timed(receive, args.steps, args.warmup)
-    st = res[:, :, 0].cpu().numpy() & 0xFFFFFFFF
-    exact = bool(torch.equal(h_back, host)) and not st.any()
-    raw = F * fv * 2
-    sent = sum(sizes)
+    exact = bool(torch.equal(h_back, host)) and not bool((res[:, 0] & 0xFFFFFFFF).any())
+    raw = n * w.n_tokens * w.head_dim * 2
     print(json.dumps({
         "metric": "host-streamed migration, lossless: GB/s of raw bytes from and to pinned host memory",
         "workload": f"live-migration block {w.n_layers}x{w.n_heads}x{w.n_tokens}x{w.head_dim} bf16 K+V "
@@ -667,7 +616,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--migration", action="store_true",
                     help="instead of the bench step: the host-streamed migration workload")
-    ap.add_argument("--migration-slices", type=int, default=16, help="slices per streamed frame")
+    ap.add_argument("--migration-slices", type=int, default=32, help="slices per streamed frame")
     ap.add_argument("--basis", choices=sorted(BASES), default="pca",
                     help="transform basis: calibrated PCA (default) or a fixed Hadamard / DCT-II")
     args = ap.parse_args()

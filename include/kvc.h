@@ -206,6 +206,41 @@ int kvc_encode_batch(const kvc_plan_t* plan, int path, const kvc_frame* h_frames
 int kvc_decode_batch(const kvc_plan_t* plan, int path, const kvc_frame* h_frames, uint32_t n_frames,
                      uint32_t max_slices_per_frame, void* d_ws, size_t ws_bytes, cudaStream_t stream);
 
+/* Host-streamed coding (QATQ page, "Measured evidence": raw blocks streamed
+ * through the codec in a live migration). A range of slices in host memory
+ * is coded frame by frame, each frame of frame_slices slices (the last may be
+ * shorter) an independent container; the H2D copies, the codec and the D2H
+ * copies of consecutive frames overlap on three streams (the caller's stream
+ * runs the codec; two copy streams and the ring's events are made by the
+ * first such call on a plan and kept until kvc_plan_destroy) through a ring
+ * of device slots in d_buf. The calls are blocking: they return when every
+ * copy has landed. Host-streamed calls on one plan must not run at the same
+ * time from several host threads (they share the plan's copy streams).
+ * h_src, h_dst and h_results should be pinned (cudaHostAlloc or registered)
+ * memory, else the copies do not overlap.
+ *   kvc_stream_buffer_bytes: size of d_buf (device, 256-byte aligned) for
+ *     frames of frame_slices slices.
+ *   kvc_stream_encode_host: slices [first_slice, first_slice + n_slices) of
+ *     h_src ([n_slices][T][D] values) into h_dst, containers back to back in
+ *     frame order; h_frame_bytes[i] gets frame i's container size and
+ *     h_results[i] its device result (n_frames = ceil(n_slices / frame_slices)
+ *     entries each). KVC_ERR_CAPACITY if the containers outgrow dst_cap (the
+ *     frames coded so far are in place).
+ *   kvc_stream_decode_host: the n_frames containers back to back in h_src
+ *     (sizes h_frame_bytes), as written by kvc_stream_encode_host for
+ *     n_slices slices in frames of frame_slices, into h_dst ([n_slices][T][D]
+ *     values, dst_cap bytes); h_results[i] gets frame i's status (a corrupt
+ *     frame leaves its part of h_dst unspecified and the others decoded).
+ * Return values report host-visible errors, as for the other calls. */
+size_t kvc_stream_buffer_bytes(const kvc_plan_t* plan, int path, uint32_t frame_slices);
+int kvc_stream_encode_host(const kvc_plan_t* plan, int path, uint32_t first_slice, uint32_t n_slices,
+                           uint32_t frame_slices, const void* h_src, void* h_dst, size_t dst_cap,
+                           uint64_t* h_frame_bytes, kvc_result* h_results, void* d_buf, size_t buf_bytes,
+                           cudaStream_t stream);
+int kvc_stream_decode_host(const kvc_plan_t* plan, int path, uint32_t n_slices, uint32_t frame_slices,
+                           const void* h_src, const uint64_t* h_frame_bytes, void* h_dst, size_t dst_cap,
+                           kvc_result* h_results, void* d_buf, size_t buf_bytes, cudaStream_t stream);
+
 /* Human-readable name of a status code (static string). */
 const char* kvc_status_string(int status);
 

@@ -57,6 +57,8 @@ def test_lossless_bound_matches_oracle(s):
     assert plan.workspace_bytes(kvc.LOSSLESS, False, 2) > 0
     assert plan.workspace_bytes(kvc.LOSSLESS, True, 0) >= 32
     assert plan.max_encoded_bytes(kvc.TRANSFORM, 1) == 0  # no bases: lossless-only plan
+    assert kvc.stream_buffer_bytes(plan, kvc.LOSSLESS, 1) > 3 * plan.max_encoded_bytes(kvc.LOSSLESS, 1)
+    assert kvc.stream_buffer_bytes(plan, kvc.LOSSLESS, 0) == 0
 
 
 def test_plan_validation():

@@ -32,6 +32,7 @@ EXPORTS = [
     "kvc_stage_stream_encode_noalloc",
     "kvc_profile_begin", "kvc_profile_end",
     "kvc_batch_workspace_bytes", "kvc_encode_batch", "kvc_decode_batch",
+    "kvc_stream_buffer_bytes", "kvc_stream_encode_host", "kvc_stream_decode_host",
 ]
 
 
@@ -91,6 +92,9 @@ def _load():
         "kvc_batch_workspace_bytes": ([vp, i32, i32, u32, u32], sz),
         "kvc_encode_batch": ([vp, i32, ctypes.POINTER(Frame), u32, vp, sz, vp], i32),
         "kvc_decode_batch": ([vp, i32, ctypes.POINTER(Frame), u32, u32, vp, sz, vp], i32),
+        "kvc_stream_buffer_bytes": ([vp, i32, u32], sz),
+        "kvc_stream_encode_host": ([vp, i32, u32, u32, u32, vp, vp, sz, vp, vp, vp, sz, vp], i32),
+        "kvc_stream_decode_host": ([vp, i32, u32, u32, vp, vp, vp, sz, vp, vp, sz, vp], i32),
         "kvc_profile_begin": ([], i32),
         "kvc_profile_end": ([ctypes.POINTER(KernelTime), i32, ctypes.POINTER(i32)], i32),
         "kvc_stage_crc32": ([vp, sz, vp, vp], i32),
@@ -278,6 +282,32 @@ def decode_batch(plan: Plan, path: int, frames, ws, max_slices_per_frame: int = 
     _check(_lib.kvc_decode_batch(plan.handle, path, _frames(items), len(items),
                                  max_slices_per_frame, _dptr(ws), ws.numel() * ws.element_size(),
                                  _stream(stream)), "kvc_decode_batch")
+
+
+def stream_buffer_bytes(plan: Plan, path: int, frame_slices: int) -> int:
+    return _lib.kvc_stream_buffer_bytes(plan.handle, path, frame_slices)
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
+def stream_encode_host(plan: Plan, path: int, first_slice: int, n_slices: int, frame_slices: int,
+                       h_src, h_dst, h_frame_bytes, h_results, d_buf, stream=None):
+    """kvc_stream_encode_host (blocking): h_src / h_dst host tensors (pinned for
+    overlap), h_frame_bytes host int64 [n_frames], h_results host int64
+    [n_frames, 2] (kvc_result), d_buf device uint8 of stream_buffer_bytes."""
+    _check(_lib.kvc_stream_encode_host(plan.handle, path, first_slice, n_slices, frame_slices, _dptr(h_src),
+                                       _dptr(h_dst), _nbytes(h_dst), _dptr(h_frame_bytes), _dptr(h_results),
+                                       _dptr(d_buf), _nbytes(d_buf), _stream(stream)), "kvc_stream_encode_host")
+
+
+def stream_decode_host(plan: Plan, path: int, n_slices: int, frame_slices: int, h_src, h_frame_bytes, h_dst,
+                       h_results, d_buf, stream=None):
+    """kvc_stream_decode_host (blocking); arguments as for stream_encode_host."""
+    _check(_lib.kvc_stream_decode_host(plan.handle, path, n_slices, frame_slices, _dptr(h_src),
+                                       _dptr(h_frame_bytes), _dptr(h_dst), _nbytes(h_dst), _dptr(h_results),
+                                       _dptr(d_buf), _nbytes(d_buf), _stream(stream)), "kvc_stream_decode_host")
 
 
 def read_result(res) -> tuple[int, int]:

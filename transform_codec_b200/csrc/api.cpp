@@ -76,6 +76,10 @@ struct kvc_plan_s {
   float* d_rope = nullptr;
   uint8_t* d_qsplit = nullptr;
   CompInfo* d_comp = nullptr;
+  // host-streamed calls: two copy streams and the ring's events, made by the
+  // first such call and kept until the plan is destroyed
+  cudaStream_t copy_in = nullptr, copy_out = nullptr;
+  cudaEvent_t ring_ev[3][3] = {};   // [in, coded, out][slot]
 };
 
 namespace {
@@ -246,6 +250,13 @@ void free_plan(kvc_plan_s* p) {
   if (p->d_rope) cudaFree(p->d_rope);
   if (p->d_qsplit) cudaFree(p->d_qsplit);
   if (p->d_comp) cudaFree(p->d_comp);
+  if (p->copy_in) cudaStreamSynchronize(p->copy_in);
+  if (p->copy_out) cudaStreamSynchronize(p->copy_out);
+  for (auto& row : p->ring_ev)
+    for (cudaEvent_t e : row)
+      if (e) cudaEventDestroy(e);
+  if (p->copy_in) cudaStreamDestroy(p->copy_in);
+  if (p->copy_out) cudaStreamDestroy(p->copy_out);
   delete p;
 }
 
@@ -727,6 +738,187 @@ extern "C" int kvc_profile_end(kvc_kernel_time* out, int max_kernels, int* n_ker
   for (int i = 0; i < n; ++i) out[i] = agg[i];
   if (n_kernels) *n_kernels = n;
   return st;
+}
+
+// ------------------------------------------------------------------ host-streamed coding
+namespace {
+
+constexpr uint32_t kStreamSlots = 3;  // depth of the device ring
+
+uint32_t value_bytes(const kvc_plan_s* p, int path) { return path == KVC_PATH_LOSSLESS ? p->ls.E : 2u; }
+
+struct StreamRing {
+  uint64_t raw_bytes = 0, cont_bytes = 0, slot_bytes = 0, ws_bytes = 0;
+};
+
+// Per slot: a raw frame, a container of frame_slices slices and a result;
+// then one workspace shared by the frames (they are coded one after another).
+StreamRing stream_ring(const kvc_plan_s* p, int path, uint32_t fs) {
+  StreamRing r;
+  r.raw_bytes = pad256u(uint64_t(fs) * p->d.n_tokens * p->d.head_dim * value_bytes(p, path));
+  r.cont_bytes = pad256u(kvc_max_encoded_bytes(p, path, fs));
+  r.slot_bytes = r.raw_bytes + r.cont_bytes + 256u;
+  r.ws_bytes = pad256u(std::max(encode_ws_for(p, path, uint64_t(fs) * records_per_slice(p, path)),
+                                decode_ws_for(p, path, 1, fs)));
+  return r;
+}
+
+// The plan's two copy streams and the ring's events, made on first use.
+struct StreamCall {
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t *ev_in = nullptr, *ev_coded = nullptr, *ev_out = nullptr;
+  bool ok = true;
+  explicit StreamCall(kvc_plan_s* p) {
+    if (!p->copy_in) ok = cudaStreamCreateWithFlags(&p->copy_in, cudaStreamNonBlocking) == cudaSuccess;
+    if (ok && !p->copy_out) ok = cudaStreamCreateWithFlags(&p->copy_out, cudaStreamNonBlocking) == cudaSuccess;
+    for (auto& row : p->ring_ev)
+      for (cudaEvent_t& e : row)
+        if (ok && !e) ok = cudaEventCreateWithFlags(&e, cudaEventDisableTiming) == cudaSuccess;
+    in = p->copy_in;
+    out = p->copy_out;
+    ev_in = p->ring_ev[0];
+    ev_coded = p->ring_ev[1];
+    ev_out = p->ring_ev[2];
+  }
+};
+
+}  // namespace
+
+extern "C" size_t kvc_stream_buffer_bytes(const kvc_plan_t* plan, int path, uint32_t frame_slices) {
+  if (!path_ok(plan, path) || frame_slices == 0 || frame_slices > plan->S) return 0;
+  const StreamRing r = stream_ring(plan, path, frame_slices);
+  return size_t(kStreamSlots * r.slot_bytes + r.ws_bytes);
+}
+
+extern "C" int kvc_stream_encode_host(const kvc_plan_t* plan, int path, uint32_t first_slice, uint32_t n_slices,
+                                      uint32_t frame_slices, const void* h_src, void* h_dst, size_t dst_cap,
+                                      uint64_t* h_frame_bytes, kvc_result* h_results, void* d_buf,
+                                      size_t buf_bytes, cudaStream_t stream) {
+  if (!path_ok(plan, path)) return plan ? KVC_ERR_UNSUPPORTED : KVC_ERR_INVALID;
+  if (frame_slices == 0 || frame_slices > plan->S || uint64_t(first_slice) + n_slices > plan->S || !d_buf ||
+      (reinterpret_cast<uintptr_t>(d_buf) & 255u) ||
+      (n_slices && (!h_src || !h_dst || !h_frame_bytes || !h_results)))
+    return KVC_ERR_INVALID;
+  int st = check_plan_device(plan);
+  if (st) return st;
+  const StreamRing R = stream_ring(plan, path, frame_slices);
+  if (buf_bytes < kStreamSlots * R.slot_bytes + R.ws_bytes) return KVC_ERR_CAPACITY;
+  if (n_slices == 0) return KVC_OK;
+  StreamCall sc(const_cast<kvc_plan_s*>(plan));
+  if (!sc.ok) return KVC_ERR_CUDA;
+  uint8_t* base = static_cast<uint8_t*>(d_buf);
+  auto raw = [&](uint32_t k) { return base + k * R.slot_bytes; };
+  auto cont = [&](uint32_t k) { return raw(k) + R.raw_bytes; };
+  auto res = [&](uint32_t k) { return reinterpret_cast<kvc_result*>(cont(k) + R.cont_bytes); };
+  uint8_t* ws = base + kStreamSlots * R.slot_bytes;
+  const uint64_t slice_bytes = uint64_t(plan->d.n_tokens) * plan->d.head_dim * value_bytes(plan, path);
+  const uint32_t nf = (n_slices + frame_slices - 1) / frame_slices;
+  const uint8_t* src = static_cast<const uint8_t*>(h_src);
+  uint8_t* dst = static_cast<uint8_t*>(h_dst);
+  uint64_t dst_off = 0;
+  int ret = KVC_OK;
+  auto ck = [&](cudaError_t e) {
+    if (e != cudaSuccess && ret == KVC_OK) ret = KVC_ERR_CUDA;
+  };
+  // Frame g's container goes out once its encode has reported the size; the
+  // host asks two frames after issuing it, so the copy engines never idle on it.
+  auto drain = [&](uint32_t g) {
+    const uint32_t k = g % kStreamSlots;
+    ck(cudaEventSynchronize(sc.ev_coded[k]));
+    uint64_t n = ret == KVC_OK && h_results[g].status == KVC_OK ? h_results[g].bytes : 0u;
+    if (n > R.cont_bytes && ret == KVC_OK) ret = KVC_ERR_CUDA;  // a size no encode can report
+    if (n > R.cont_bytes || dst_off + n > dst_cap) {
+      if (ret == KVC_OK) ret = KVC_ERR_CAPACITY;
+      n = 0;
+    }
+    h_frame_bytes[g] = n;
+    ck(cudaStreamWaitEvent(sc.out, sc.ev_coded[k], 0));
+    if (n) ck(cudaMemcpyAsync(dst + dst_off, cont(k), n, cudaMemcpyDeviceToHost, sc.out));
+    ck(cudaEventRecord(sc.ev_out[k], sc.out));
+    dst_off += n;
+  };
+  for (uint32_t f = 0; f < nf && ret == KVC_OK; ++f) {
+    const uint32_t k = f % kStreamSlots, s0 = f * frame_slices, ns = std::min(frame_slices, n_slices - s0);
+    if (f >= kStreamSlots) ck(cudaStreamWaitEvent(sc.in, sc.ev_coded[k], 0));  // frame f - 3 read the slot
+    ck(cudaMemcpyAsync(raw(k), src + s0 * slice_bytes, ns * slice_bytes, cudaMemcpyHostToDevice, sc.in));
+    ck(cudaEventRecord(sc.ev_in[k], sc.in));
+    if (f + 1 >= kStreamSlots) drain(f + 1 - kStreamSlots);
+    ck(cudaStreamWaitEvent(stream, sc.ev_in[k], 0));
+    if (f >= kStreamSlots) ck(cudaStreamWaitEvent(stream, sc.ev_out[k], 0));  // its container is out
+    if (ret != KVC_OK) break;
+    const kvc_frame fr{first_slice + s0, ns, raw(k), 0, cont(k), size_t(R.cont_bytes), res(k)};
+    const int e = encode_frames(plan, path, &fr, 1, ws, size_t(R.ws_bytes), stream);
+    if (e != KVC_OK) ret = e;
+    ck(cudaMemcpyAsync(&h_results[f], res(k), sizeof(kvc_result), cudaMemcpyDeviceToHost, stream));
+    ck(cudaEventRecord(sc.ev_coded[k], stream));
+  }
+  for (uint32_t g = nf + 1 > kStreamSlots ? nf + 1 - kStreamSlots : 0u; g < nf && ret == KVC_OK; ++g) drain(g);
+  ck(cudaStreamSynchronize(sc.in));
+  ck(cudaStreamSynchronize(stream));
+  ck(cudaStreamSynchronize(sc.out));
+  return ret;
+}
+
+extern "C" int kvc_stream_decode_host(const kvc_plan_t* plan, int path, uint32_t n_slices, uint32_t frame_slices,
+                                      const void* h_src, const uint64_t* h_frame_bytes, void* h_dst,
+                                      size_t dst_cap, kvc_result* h_results, void* d_buf, size_t buf_bytes,
+                                      cudaStream_t stream) {
+  if (!path_ok(plan, path)) return plan ? KVC_ERR_UNSUPPORTED : KVC_ERR_INVALID;
+  if (frame_slices == 0 || frame_slices > plan->S || n_slices > plan->S || !d_buf ||
+      (reinterpret_cast<uintptr_t>(d_buf) & 255u) ||
+      (n_slices && (!h_src || !h_dst || !h_frame_bytes || !h_results)))
+    return KVC_ERR_INVALID;
+  int st = check_plan_device(plan);
+  if (st) return st;
+  const StreamRing R = stream_ring(plan, path, frame_slices);
+  if (buf_bytes < kStreamSlots * R.slot_bytes + R.ws_bytes) return KVC_ERR_CAPACITY;
+  const uint64_t slice_bytes = uint64_t(plan->d.n_tokens) * plan->d.head_dim * value_bytes(plan, path);
+  if (dst_cap < n_slices * slice_bytes) return KVC_ERR_CAPACITY;
+  if (n_slices == 0) return KVC_OK;
+  StreamCall sc(const_cast<kvc_plan_s*>(plan));
+  if (!sc.ok) return KVC_ERR_CUDA;
+  uint8_t* base = static_cast<uint8_t*>(d_buf);
+  auto raw = [&](uint32_t k) { return base + k * R.slot_bytes; };
+  auto cont = [&](uint32_t k) { return raw(k) + R.raw_bytes; };
+  auto res = [&](uint32_t k) { return reinterpret_cast<kvc_result*>(cont(k) + R.cont_bytes); };
+  uint8_t* ws = base + kStreamSlots * R.slot_bytes;
+  const uint32_t nf = (n_slices + frame_slices - 1) / frame_slices;
+  const uint8_t* src = static_cast<const uint8_t*>(h_src);
+  uint8_t* dst = static_cast<uint8_t*>(h_dst);
+  uint64_t src_off = 0;
+  int ret = KVC_OK;
+  auto ck = [&](cudaError_t e) {
+    if (e != cudaSuccess && ret == KVC_OK) ret = KVC_ERR_CUDA;
+  };
+  for (uint32_t f = 0; f < nf && ret == KVC_OK; ++f) {
+    const uint32_t k = f % kStreamSlots, s0 = f * frame_slices, ns = std::min(frame_slices, n_slices - s0);
+    const uint64_t nb = h_frame_bytes[f];
+    if (nb > R.cont_bytes) {  // longer than any container of frame_slices slices
+      h_results[f].status = KVC_ERR_CORRUPT;
+      h_results[f].bytes = 0;
+      src_off += nb;
+      continue;
+    }
+    if (f >= kStreamSlots) ck(cudaStreamWaitEvent(sc.in, sc.ev_coded[k], 0));  // frame f - 3 read the slot
+    if (nb) ck(cudaMemcpyAsync(cont(k), src + src_off, nb, cudaMemcpyHostToDevice, sc.in));
+    ck(cudaEventRecord(sc.ev_in[k], sc.in));
+    ck(cudaStreamWaitEvent(stream, sc.ev_in[k], 0));
+    if (f >= kStreamSlots) ck(cudaStreamWaitEvent(stream, sc.ev_out[k], 0));  // its values are out
+    if (ret != KVC_OK) break;
+    const kvc_frame fr{0, 0, cont(k), size_t(nb), raw(k), size_t(ns * slice_bytes), res(k)};
+    const int e = decode_frames(plan, path, &fr, 1, frame_slices, ws, size_t(R.ws_bytes), stream);
+    if (e != KVC_OK) ret = e;
+    ck(cudaMemcpyAsync(&h_results[f], res(k), sizeof(kvc_result), cudaMemcpyDeviceToHost, stream));
+    ck(cudaEventRecord(sc.ev_coded[k], stream));
+    ck(cudaStreamWaitEvent(sc.out, sc.ev_coded[k], 0));
+    ck(cudaMemcpyAsync(dst + s0 * slice_bytes, raw(k), ns * slice_bytes, cudaMemcpyDeviceToHost, sc.out));
+    ck(cudaEventRecord(sc.ev_out[k], sc.out));
+    src_off += nb;
+  }
+  ck(cudaStreamSynchronize(sc.in));
+  ck(cudaStreamSynchronize(stream));
+  ck(cudaStreamSynchronize(sc.out));
+  return ret;
 }
 
 extern "C" const char* kvc_status_string(int status) {
