@@ -144,3 +144,35 @@ def test_fixed_basis_refusals():
         kvc.fixed_basis(kvc.BASIS_HADAMARD, 96)
     with pytest.raises(kvc.KvcError):
         kvc.fixed_basis(9, 8)
+
+
+def test_stream_host_argument_checks():
+    """The host-streamed calls refuse bad arguments before touching a device:
+    no frame size, a misaligned or too small device ring, too many slices."""
+    import types
+
+    import torch
+    null = types.SimpleNamespace(cuda_stream=0)  # the legacy default stream; no CUDA context needed here
+    plan = kvc.Plan(kvc.Shape(kvc.BF16, 1, 8, 512, 128))
+    n = plan.shape.n_slices
+    src = torch.zeros(n * 512 * 128, dtype=torch.int16)
+    dst = torch.zeros(plan.max_encoded_bytes(kvc.LOSSLESS, n), dtype=torch.uint8)
+    fb = torch.zeros(n, dtype=torch.int64)
+    res = torch.zeros(n, 2, dtype=torch.int64)
+    need = kvc.stream_buffer_bytes(plan, kvc.LOSSLESS, 4)
+    assert need > 0 and kvc.stream_buffer_bytes(plan, kvc.LOSSLESS, n + 1) == 0
+    assert kvc.stream_buffer_bytes(plan, kvc.TRANSFORM, 4) == 0  # no bases: lossless-only plan
+    raw = torch.zeros(1024 + 256, dtype=torch.uint8)
+    small = raw[(-raw.data_ptr()) % 256:][:1024]  # 256-byte aligned, far too small
+    cases = [
+        (lambda: kvc.stream_encode_host(plan, kvc.LOSSLESS, 0, n, 0, src, dst, fb, res, small, null), kvc.ERR_INVALID),
+        (lambda: kvc.stream_encode_host(plan, kvc.LOSSLESS, 1, n, 4, src, dst, fb, res, small, null), kvc.ERR_INVALID),
+        (lambda: kvc.stream_encode_host(plan, kvc.LOSSLESS, 0, n, 4, src, dst, fb, res, small, null), kvc.ERR_CAPACITY),
+        (lambda: kvc.stream_decode_host(plan, kvc.LOSSLESS, n, 0, dst, fb, src, res, small, null), kvc.ERR_INVALID),
+        (lambda: kvc.stream_decode_host(plan, kvc.LOSSLESS, n, 4, dst, fb, src, res, small, null), kvc.ERR_CAPACITY),
+        (lambda: kvc.stream_encode_host(plan, kvc.TRANSFORM, 0, n, 4, src, dst, fb, res, small, null), kvc.ERR_UNSUPPORTED),
+    ]
+    for call, want in cases:
+        with pytest.raises(kvc.KvcError) as e:
+            call()
+        assert e.value.status == want
