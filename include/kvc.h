@@ -224,8 +224,9 @@ int kvc_decode_batch(const kvc_plan_t* plan, int path, const kvc_frame* h_frames
  *     h_src ([n_slices][T][D] values) into h_dst, containers back to back in
  *     frame order; h_frame_bytes[i] gets frame i's container size and
  *     h_results[i] its device result (n_frames = ceil(n_slices / frame_slices)
- *     entries each). KVC_ERR_CAPACITY if the containers outgrow dst_cap (the
- *     frames coded so far are in place).
+ *     entries each). KVC_ERR_CAPACITY if the containers outgrow dst_cap: the
+ *     frames whose sizes were written are in place, the later entries of
+ *     h_frame_bytes are not written.
  *   kvc_stream_decode_host: the n_frames containers back to back in h_src
  *     (sizes h_frame_bytes), as written by kvc_stream_encode_host for
  *     n_slices slices in frames of frame_slices, into h_dst ([n_slices][T][D]
