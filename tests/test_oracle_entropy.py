@@ -208,3 +208,39 @@ def test_stream_decoder_refuses_bad_records():
         st, out, _ = oracle.stream_decode(bytes(bad), 5000)
         refused += (st != oracle.OK) or (not np.array_equal(out, sym))
     assert refused > 150
+
+
+def test_rans_words_lower_bound():
+    """A lower bound on the words of an rANS record, used by the GPU side
+    encoder to skip a variant that cannot beat RAW. Before each coding step the
+    state x is at least 16 f (after renormalisation), so a step multiplies x by
+    more than (M / f)(15/16); an emitted word removes at most 16 + log2(16/15)
+    bits; the N final states hold at most 16 bits each beyond their start; and
+    sum_s c_s log2(M / f_s) >= n H (Gibbs) for the empirical entropy H. Hence
+    W >= (n H - n log2(16/15) - 16 N) / (16 + log2(16/15)). Checked on skewed,
+    uniform, heavy-tailed and sorted streams, with the kernel's margins too."""
+    rng = np.random.default_rng(17)
+    d = math.log2(16 / 15)
+    for trial in range(250):
+        n = int(rng.integers(2, 70000))
+        kind = trial % 5
+        if kind == 0:
+            s = rng.integers(0, int(rng.integers(2, 257)), n)
+        elif kind == 1:
+            s = np.minimum(rng.geometric(float(rng.uniform(0.05, 0.9)), n) - 1, 255)
+        elif kind == 2:
+            s = np.minimum(rng.zipf(1.5, n) - 1, 255)
+        elif kind == 3:
+            s = np.where(rng.random(n) < 0.99, 0, rng.integers(1, 256, n))
+        else:
+            s = np.sort(rng.integers(0, 256, n))
+        s = s.astype(np.uint8)
+        payload = oracle.rans_payload_bytes(s)
+        if payload == 0:
+            continue
+        N = min(128, max(1, n // 512))
+        W = (payload - 4 * N) / 2
+        _, c = np.unique(s, return_counts=True)
+        H = float((c * np.log2(n / c)).sum())
+        assert W >= (H - d * n - 16 * N) / (16 + d) - 1e-9, (trial, n, kind)
+        assert W >= (H * 0.9999 - 2.0 - 0.0932 * n - 16.0 * N) / (16.0 + 0.0932)  # the kernel's form
