@@ -417,17 +417,23 @@ __device__ inline void block_enc_tables(const uint32_t* freq, uint32_t* fc, uint
 
 // Largest-remainder normalisation by one warp (the rule of block_normalize) of
 // hist[0 .. A), A <= 256, n symbols: writes freq[0 .. 256) and the coding table
-// tab[0 .. A) = {f | cum << 16, floor((2^32-1)/f)}; rem[0 .. A) is scratch.
-// Returns k. The d symbols that get one more are found by a radix select over
-// the keys 1 << 24 | r << 8 | (255 - s) of the present symbols (absent: 0).
+// tab[0 .. A) = {f | cum << 16, floor((2^32-1)/f)}; rem is not used (kept for
+// the callers' layouts). Returns k. The d symbols that get one more are found
+// by a radix select over the keys 1 << 24 | r << 8 | (255 - s) of the present
+// symbols (absent: 0), held in registers: lane l keeps the keys of symbols
+// l + 32 j. freq may alias hist: each lane reads a symbol's count before it
+// writes that symbol's frequency.
 __device__ inline uint32_t warp_normalize(const uint32_t* hist, uint32_t A, uint32_t n, uint32_t* freq,
                                           uint32_t* rem, uint2* tab) {
+  (void)rem;
   const uint32_t lane = threadIdx.x & 31u;
   uint32_t present = 0;
   for (uint32_t s = lane; s < A; s += 32u) present += hist[s] ? 1u : 0u;
   const uint32_t k = __reduce_add_sync(0xffffffffu, present);
-  uint32_t fsum = 0;
-  for (uint32_t s = lane; s < 256u; s += 32u) {
+  uint32_t fsum = 0, key[8];
+#pragma unroll
+  for (uint32_t j = 0; j < 8; ++j) {
+    const uint32_t s = lane + 32u * j;
     const uint32_t c = s < A ? hist[s] : 0u;
     uint32_t f = 0, r = 0;
     if (k >= 2 && c) {
@@ -437,7 +443,7 @@ __device__ inline uint32_t warp_normalize(const uint32_t* hist, uint32_t A, uint
     } else if (k == 1 && c) {
       f = kProbScale;
     }
-    if (s < A) rem[s] = c ? (1u << 24) | (r << 8) | (255u - s) : 0u;
+    key[j] = c ? (1u << 24) | (r << 8) | (255u - s) : 0u;
     freq[s] = f;
     fsum += f;
   }
@@ -448,19 +454,18 @@ __device__ inline uint32_t warp_normalize(const uint32_t* hist, uint32_t A, uint
     uint32_t P = 1, need = kProbScale - sum;
     for (int bit = 23; bit >= 0; --bit) {
       uint32_t cnt = 0;
-      for (uint32_t s0 = 0; s0 < A; s0 += 32u) {
-        const uint32_t s = s0 + lane;
-        const bool hit = s < A && (rem[s] >> bit) == ((P << 1) | 1u);
-        cnt += __popc(__ballot_sync(0xffffffffu, hit));
-      }
+#pragma unroll
+      for (uint32_t j = 0; j < 8; ++j)
+        if (32u * j < A) cnt += __popc(__ballot_sync(0xffffffffu, (key[j] >> bit) == ((P << 1) | 1u)));
       if (cnt >= need) P = (P << 1) | 1u;
       else {
         need -= cnt;
         P <<= 1;
       }
     }
-    for (uint32_t s = lane; s < A; s += 32u)
-      if (rem[s] >= P) freq[s] += 1u;
+#pragma unroll
+    for (uint32_t j = 0; j < 8; ++j)
+      if (key[j] >= P) freq[lane + 32u * j] += 1u;
   }
   __syncwarp();
   uint32_t carry = 0;
