@@ -54,10 +54,7 @@ KERNEL_WORK = {
 # than L2; the traffic of these kernels grows with the frames a launch covers).
 # A kernel that changed after that capture has no entry.
 DRAM_BYTES_PER_FRAME = {
-    "lossless_encode": (759.9e6 + 353.7e6) / 4,
     "transform_project": (304.5e6 + 100.5e6) / 4,
-    "transform_side": (14.0e6 + 0.001e6) / 4,
-    "transform_entropy": (126.1e6 + 27.1e6) / 4,
     "transform_decode_codes": (80.0e6 + 109.4e6) / 4,
     "lossless_decode": (198.8e6 + 220.9e6) / 4,
     "transform_decode": (199.5e6 + 221.8e6) / 4,
