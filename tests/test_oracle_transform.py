@@ -498,3 +498,49 @@ def test_side_stream_roundtrip_and_refusals(n):
     bad = bytearray(rec)
     bad[8] ^= 1  # symbol count
     assert oracle.side_stream_decode(bytes(bad), n)[0] != 0
+
+
+def _rans_record_one_lane(sym):
+    """A RANS stream record of one lane (one group), written here from the
+    format (header, presence bitmap, frequencies, one sub-stream length, the
+    final state and the words) with a plain single-lane rANS encoder (J. Duda,
+    arXiv:1311.2540; 32-bit state, L = 2^16, 16-bit words, M = 2^12), whatever
+    its size against RAW."""
+    n = sym.size
+    counts = np.bincount(sym, minlength=256).astype(np.uint32)
+    freq, k = oracle.normalize(counts)
+    freq = freq.astype(np.int64)
+    cum = np.concatenate([[0], np.cumsum(freq)[:-1]])
+    x, words = 1 << 16, []
+    for s in sym[::-1].tolist():
+        f = int(freq[s])
+        if x >= f << 20:
+            words.append(x & 0xFFFF)
+            x >>= 16
+        x = ((x // f) << 12) + (x % f) + int(cum[s])
+    words = words[::-1]  # the decoder reads the last emitted word first
+    pad = lambda b: b + bytes(-len(b) % 16)  # noqa: E731
+    bitmap = bytearray(32)
+    for s in np.flatnonzero(freq):
+        bitmap[s >> 3] |= 1 << (s & 7)
+    table = pad(bytes(bitmap) + b"".join(struct.pack("<H", int(freq[s])) for s in np.flatnonzero(freq)))
+    sub = struct.pack("<I", x) + b"".join(struct.pack("<H", w) for w in words)
+    body = table + pad(struct.pack("<I", len(sub))) + pad(sub)
+    return bytes([2, 0, 1, 0]) + struct.pack("<III", 16 + len(body), n, int(k)) + body
+
+
+def test_side_stream_longer_than_raw_refused():
+    """A RANS record longer than RAW is valid as a code stream (the general
+    decoder restores it) but never comes from the side-stream encoder, whose
+    never-worse choice would have written RAW; the side decoder refuses it."""
+    rng = np.random.default_rng(5)
+    sym = rng.integers(0, 64, 100).astype(np.uint8)  # one lane under both lane rules
+    rec = _rans_record_one_lane(sym)
+    assert len(rec) > 16 + 112  # longer than the RAW record of 100 symbols
+    st, out, used = oracle.stream_decode(rec, sym.size)
+    assert st == oracle.OK and used == len(rec) and np.array_equal(out, sym)
+    assert oracle.side_stream_decode(rec, sym.size)[0] == oracle.CORRUPT
+    small = rng.choice(np.array([3, 3, 3, 3, 9], np.uint8), 100)  # compressible: RANS below RAW
+    rec2 = _rans_record_one_lane(small)
+    assert len(rec2) < 16 + 112
+    assert oracle.side_stream_decode(rec2, small.size)[0] == oracle.OK
