@@ -544,3 +544,18 @@ def test_side_stream_longer_than_raw_refused():
     rec2 = _rans_record_one_lane(small)
     assert len(rec2) < 16 + 112
     assert oracle.side_stream_decode(rec2, small.size)[0] == oracle.OK
+
+
+@pytest.mark.parametrize("n", [100, 300, 511, 1023])
+def test_oracle_rans_records_equal_independent_encoder(n):
+    """Where the oracle writes a one-lane RANS record (n < 1024, compressible
+    symbols), its bytes equal those of the independent single-lane encoder
+    above: the state update, the renormalisation, the word order and the
+    record layout are pinned byte for byte."""
+    rng = np.random.default_rng(n)
+    sym = np.minimum(rng.geometric(0.35 if n > 400 else 0.8, n) - 1, 255).astype(np.uint8)
+    if np.unique(sym).size < 2:
+        sym[0] = sym[0] ^ 1
+    rec = oracle.stream_encode(sym)
+    assert rec[0] == 2  # RANS is the smaller record for these symbols
+    assert rec == _rans_record_one_lane(sym)
