@@ -500,31 +500,43 @@ def test_side_stream_roundtrip_and_refusals(n):
     assert oracle.side_stream_decode(bytes(bad), n)[0] != 0
 
 
-def _rans_record_one_lane(sym):
-    """A RANS stream record of one lane (one group), written here from the
-    format (header, presence bitmap, frequencies, one sub-stream length, the
-    final state and the words) with a plain single-lane rANS encoder (J. Duda,
-    arXiv:1311.2540; 32-bit state, L = 2^16, 16-bit words, M = 2^12), whatever
-    its size against RAW."""
+def _rans_record_one_lane(sym, N=1):
+    """A RANS stream record of N <= 32 interleaved lanes (one group), written
+    here from the format (header, presence bitmap, frequencies, one sub-stream
+    length, the lanes' final states and the words) with a plain rANS encoder
+    (J. Duda, arXiv:1311.2540; 32-bit state, L = 2^16, 16-bit words,
+    M = 2^12; lane l codes the contiguous range [start_l, start_l + len_l),
+    len_l = n // N + (l < n % N)), whatever its size against RAW. The decoder
+    reads, step by step, the lanes in ascending order, so the encoder runs
+    the steps backwards with the lanes in descending order and prepends its
+    words."""
     n = sym.size
     counts = np.bincount(sym, minlength=256).astype(np.uint32)
     freq, k = oracle.normalize(counts)
     freq = freq.astype(np.int64)
     cum = np.concatenate([[0], np.cumsum(freq)[:-1]])
-    x, words = 1 << 16, []
-    for s in sym[::-1].tolist():
-        f = int(freq[s])
-        if x >= f << 20:
-            words.append(x & 0xFFFF)
-            x >>= 16
-        x = ((x // f) << 12) + (x % f) + int(cum[s])
+    base, extra = divmod(n, N)
+    lens = [base + (1 if l < extra else 0) for l in range(N)]
+    starts = np.concatenate([[0], np.cumsum(lens)[:-1]]).astype(int)
+    x, words = [1 << 16] * N, []
+    syms = sym.tolist()
+    for tau in range(lens[0] - 1, -1, -1):
+        for l in range(N - 1, -1, -1):
+            if tau >= lens[l]:
+                continue
+            s = syms[starts[l] + tau]
+            f = int(freq[s])
+            if x[l] >= f << 20:
+                words.append(x[l] & 0xFFFF)
+                x[l] >>= 16
+            x[l] = ((x[l] // f) << 12) + (x[l] % f) + int(cum[s])
     words = words[::-1]  # the decoder reads the last emitted word first
     pad = lambda b: b + bytes(-len(b) % 16)  # noqa: E731
     bitmap = bytearray(32)
     for s in np.flatnonzero(freq):
         bitmap[s >> 3] |= 1 << (s & 7)
     table = pad(bytes(bitmap) + b"".join(struct.pack("<H", int(freq[s])) for s in np.flatnonzero(freq)))
-    sub = struct.pack("<I", x) + b"".join(struct.pack("<H", w) for w in words)
+    sub = b"".join(struct.pack("<I", v) for v in x) + b"".join(struct.pack("<H", w) for w in words)
     body = table + pad(struct.pack("<I", len(sub))) + pad(sub)
     return bytes([2, 0, 1, 0]) + struct.pack("<III", 16 + len(body), n, int(k)) + body
 
@@ -559,3 +571,25 @@ def test_oracle_rans_records_equal_independent_encoder(n):
     rec = oracle.stream_encode(sym)
     assert rec[0] == 2  # RANS is the smaller record for these symbols
     assert rec == _rans_record_one_lane(sym)
+
+
+@pytest.mark.parametrize("n", [1100, 5000, 16000])
+def test_oracle_interleaved_rans_equals_independent_encoder(n):
+    """Code streams of 2 to 31 lanes (n // 512, one group) and side streams of
+    3 to 32 lanes (n // 64): the oracle's RANS records equal the independent
+    interleaved encoder's byte for byte."""
+    rng = np.random.default_rng(n)
+    sym = np.minimum(rng.geometric(0.3, n) - 1, 255).astype(np.uint8)
+    rec = oracle.stream_encode(sym)
+    assert rec[0] == 2 and rec[2] == 1
+    assert rec == _rans_record_one_lane(sym, min(128, max(1, n // 512)))
+    m = min(n // 4, 2048)
+    side = sym[:m].copy()
+    srec = oracle.side_stream_encode(side)
+    plain = _rans_record_one_lane(side, min(32, max(1, m // 64)))
+    if srec[0] == 2 and srec[3] == 0:  # plain RANS: the same bytes
+        assert srec == plain
+    elif srec[0] == 0:  # RAW: the plain RANS record is not smaller
+        assert len(plain) >= len(srec)
+    else:  # lane deltas: strictly smaller than the plain record
+        assert srec[0] == 2 and len(srec) < len(plain) and oracle.side_stream_decode(srec, m)[0] == oracle.OK
