@@ -501,9 +501,9 @@ def test_side_stream_roundtrip_and_refusals(n):
 
 
 def _rans_record_one_lane(sym, N=1):
-    """A RANS stream record of N <= 32 interleaved lanes (one group), written
+    """A RANS stream record of N interleaved lanes (groups of 32), written
     here from the format (header, presence bitmap, frequencies, one sub-stream
-    length, the lanes' final states and the words) with a plain rANS encoder
+    lengths, each group's final states and words) with a plain rANS encoder
     (J. Duda, arXiv:1311.2540; 32-bit state, L = 2^16, 16-bit words,
     M = 2^12; lane l codes the contiguous range [start_l, start_l + len_l),
     len_l = n // N + (l < n % N)), whatever its size against RAW. The decoder
@@ -518,27 +518,30 @@ def _rans_record_one_lane(sym, N=1):
     base, extra = divmod(n, N)
     lens = [base + (1 if l < extra else 0) for l in range(N)]
     starts = np.concatenate([[0], np.cumsum(lens)[:-1]]).astype(int)
-    x, words = [1 << 16] * N, []
     syms = sym.tolist()
-    for tau in range(lens[0] - 1, -1, -1):
-        for l in range(N - 1, -1, -1):
-            if tau >= lens[l]:
-                continue
-            s = syms[starts[l] + tau]
-            f = int(freq[s])
-            if x[l] >= f << 20:
-                words.append(x[l] & 0xFFFF)
-                x[l] >>= 16
-            x[l] = ((x[l] // f) << 12) + (x[l] % f) + int(cum[s])
-    words = words[::-1]  # the decoder reads the last emitted word first
     pad = lambda b: b + bytes(-len(b) % 16)  # noqa: E731
+    subs = []
+    for g0 in range(0, N, 32):  # one sub-stream per group of 32 lanes
+        lanes = range(g0, min(N, g0 + 32))
+        x, words = {l: 1 << 16 for l in lanes}, []
+        for tau in range(lens[g0] - 1, -1, -1):
+            for l in reversed(lanes):
+                if tau >= lens[l]:
+                    continue
+                s = syms[starts[l] + tau]
+                f = int(freq[s])
+                if x[l] >= f << 20:
+                    words.append(x[l] & 0xFFFF)
+                    x[l] >>= 16
+                x[l] = ((x[l] // f) << 12) + (x[l] % f) + int(cum[s])
+        words = words[::-1]  # the decoder reads the last emitted word first
+        subs.append(b"".join(struct.pack("<I", x[l]) for l in lanes) + b"".join(struct.pack("<H", w) for w in words))
     bitmap = bytearray(32)
     for s in np.flatnonzero(freq):
         bitmap[s >> 3] |= 1 << (s & 7)
     table = pad(bytes(bitmap) + b"".join(struct.pack("<H", int(freq[s])) for s in np.flatnonzero(freq)))
-    sub = b"".join(struct.pack("<I", v) for v in x) + b"".join(struct.pack("<H", w) for w in words)
-    body = table + pad(struct.pack("<I", len(sub))) + pad(sub)
-    return bytes([2, 0, 1, 0]) + struct.pack("<III", 16 + len(body), n, int(k)) + body
+    body = table + pad(b"".join(struct.pack("<I", len(b)) for b in subs)) + b"".join(pad(b) for b in subs)
+    return bytes([2, 0, len(subs), 0]) + struct.pack("<III", 16 + len(body), n, int(k)) + body
 
 
 def test_side_stream_longer_than_raw_refused():
@@ -593,3 +596,13 @@ def test_oracle_interleaved_rans_equals_independent_encoder(n):
         assert len(plain) >= len(srec)
     else:  # lane deltas: strictly smaller than the plain record
         assert srec[0] == 2 and len(srec) < len(plain) and oracle.side_stream_decode(srec, m)[0] == oracle.OK
+
+
+def test_oracle_lossless_plane_equals_independent_encoder():
+    """A full 65,536-symbol lossless plane: 128 lanes in four groups; the
+    oracle's RANS record equals the independent encoder's byte for byte."""
+    rng = np.random.default_rng(65536)
+    sym = np.minimum(rng.geometric(0.25, 65536) - 1, 255).astype(np.uint8)
+    rec = oracle.stream_encode(sym)
+    assert rec[0] == 2 and rec[2] == 4
+    assert rec == _rans_record_one_lane(sym, 128)
