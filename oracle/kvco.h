@@ -20,10 +20,11 @@
  *            First", "Bit Budget Is Not Fair", "rANS Makes the Last Mile Smaller".
  *
  * Parity status: every function here is pinned by tests against closed forms,
- * invariants, library routines or brute force, except the frequency
- * normalisation rule, which is a definition of this codec (parity unpinned
- * beyond its invariants), and the cyclic Jacobi PCA, which is pinned only
- * through closed forms and invariants.
+ * invariants, library routines or brute force. The frequency normalisation
+ * rule, a definition of this codec, is pinned to hand-worked tables, to the
+ * defining property of largest-remainder apportionment and to a restatement of
+ * Hamilton's method in exact rationals; the cyclic Jacobi PCA to closed forms
+ * and to numpy's symmetric eigensolver.
  */
 #ifndef KVCO_H
 #define KVCO_H

@@ -83,6 +83,95 @@ def test_normalize_hand_cases():
         assert np.all(f[: 1 << kbits] == 4096 >> kbits) and np.all(f[1 << kbits:] == 0)
 
 
+def test_normalize_remainder_not_on_largest_count():
+    """Hand-worked tables where the slots left over go to the largest
+    remainders, not to the largest counts (a rule that hands them to the
+    largest counts fails both)."""
+    c = np.zeros(256, np.uint32)
+    c[[0, 1, 2]] = [10, 3, 2]
+    # n = 15, k = 3, M - k = 4093: c (M - k) = 40930, 12279, 8186
+    # floor / 15 = 2728, 818, 545 -> f = 2729, 819, 546 (sum 4094, d = 2)
+    # remainders mod 15 = 10, 9, 11 -> symbols 2 and 0 take one more each
+    f, k = oracle.normalize(c)
+    assert k == 3 and (f[0], f[1], f[2]) == (2730, 819, 547)
+    c = np.zeros(256, np.uint32)
+    c[[0, 1, 2]] = [1, 2, 10]
+    # n = 13: c (M - k) = 4093, 8186, 40930; floor / 13 = 314, 629, 3148
+    # -> f = 315, 630, 3149 (sum 4094, d = 2 = k - 1); remainders 11, 9, 6:
+    # the two smaller counts round up, the largest count stays
+    f, k = oracle.normalize(c)
+    assert k == 3 and (f[0], f[1], f[2]) == (316, 631, 3149)
+    c = np.zeros(256, np.uint32)
+    c[[40, 41, 200, 201]] = [7, 5, 5, 1]
+    # n = 18, k = 4, M - k = 4092: c (M - k) = 28644, 20460, 20460, 4092
+    # floor / 18 = 1591, 1136, 1136, 227 -> f = 1592, 1137, 1137, 228
+    # (sum 4094, d = 2); remainders 6, 12, 12, 6: the tie at 12 takes both
+    f, k = oracle.normalize(c)
+    assert k == 4 and (f[40], f[41], f[200], f[201]) == (1592, 1138, 1138, 228)
+    c = np.zeros(256, np.uint32)
+    c[[3, 9, 250]] = [4, 4, 4]
+    # equal counts, n = 12: 16372 / 12 = 1364 r 4 -> 1365 each (sum 4095),
+    # d = 1, equal remainders: the smallest symbol takes it
+    f, k = oracle.normalize(c)
+    assert (f[3], f[9], f[250]) == (1366, 1365, 1365)
+
+
+def test_normalize_quota_property():
+    """Every present symbol gets 1 + floor(q) or 1 + ceil(q) of its quota
+    q = c (M - k) / n; exactly M - sum(1 + floor(q)) symbols round up, and no
+    symbol left at its floor has a larger remainder than one that rounded up
+    (nor an equal remainder and a smaller symbol): the defining property of
+    largest-remainder apportionment, checked with exact rationals."""
+    from fractions import Fraction
+    rng = np.random.default_rng(11)
+    for trial in range(300):
+        k = int(rng.integers(2, 257))
+        counts = np.zeros(256, np.uint32)
+        syms = rng.choice(256, k, replace=False)
+        counts[syms] = rng.integers(1, int(rng.choice([3, 50, 5000])), k)
+        n = int(counts.sum())
+        f, kk = oracle.normalize(counts)
+        assert kk == k
+        q = {s: Fraction(int(counts[s]) * (4096 - k), n) for s in map(int, syms)}
+        fl = {s: q[s].numerator // q[s].denominator for s in q}
+        up = {s for s in q if int(f[s]) == 2 + fl[s]}
+        assert all(int(f[s]) in (1 + fl[s], 2 + fl[s]) for s in q)
+        assert len(up) == 4096 - sum(1 + fl[s] for s in q)
+        down = set(q) - up
+        for u in up:
+            ru = q[u] - fl[u]
+            for s in down:
+                rs = q[s] - fl[s]
+                assert rs < ru or (rs == ru and s > u)
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_normalize_equals_textbook_apportionment(seed):
+    """The oracle's table equals Hamilton's largest-remainder method restated
+    with exact rationals in tests/apportion.py, on skewed, flat, tiny and
+    one-dominant count vectors."""
+    from apportion import largest_remainder
+    rng = np.random.default_rng(100 + seed)
+    for trial in range(150):
+        counts = np.zeros(256, np.uint32)
+        k = int(rng.integers(1, 257))
+        syms = rng.choice(256, k, replace=False)
+        kind = trial % 4
+        if kind == 0:
+            counts[syms] = np.minimum(rng.geometric(0.05, k), 65536)
+        elif kind == 1:
+            counts[syms] = rng.integers(1, 4, k)
+        elif kind == 2:
+            counts[syms] = 1
+            counts[syms[0]] = int(rng.integers(1, 65536))
+        else:
+            counts[syms] = rng.integers(1, 65536 // k + 2, k)
+        f, kk = oracle.normalize(counts)
+        want, wk = largest_remainder(counts)
+        assert kk == wk
+        assert f.astype(int).tolist() == want
+
+
 def _roundtrip(sym):
     rec = oracle.stream_encode(sym)
     assert len(rec) % 16 == 0 and len(rec) <= 16 + (len(sym) + 15) // 16 * 16
