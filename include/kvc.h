@@ -80,7 +80,7 @@ typedef struct {
 
 typedef struct kvc_plan_s kvc_plan_t;
 
-/* Plan description (host memory; copied by kvc_plan_create).
+/* Plan description (host memory; copied by kvc_plan).
  *   abi_version       KVC_ABI_VERSION
  *   dtype             KVC_DTYPE_BF16, KVC_DTYPE_FP16 or KVC_DTYPE_F32 (f32:
  *                     lossless only; transform: bf16 only)
@@ -118,10 +118,20 @@ typedef struct {
   const uint8_t* widths;
 } kvc_plan_desc;
 
-/* Validate the description, allocate bit widths, build the fp32 cos/sin table
- * (fp64-computed) and upload the plan to the current device. Checks each basis
- * for orthonormality (max |Q^T Q - I| <= 1e-3). Returns KVC_OK and *out, or an
- * error (nothing allocated). Blocking; call outside stream capture. */
+/* kvc_plan — the plan of a cache shape (KVTC page, "How the Pipeline Works":
+ * the per-component bit widths, scales and zero points that reconstruction
+ * needs; "Bit Budget Is Not Fair": widths spent unevenly; "Why RoPE Has to Be
+ * Reversed First": the rotation undone before the basis).
+ * Validates the description, allocates bit widths, builds the fp32 cos/sin
+ * table (fp64-computed) and uploads the plan to the current device. Checks
+ * each basis for orthonormality (max |Q^T Q - I| <= 1e-3).
+ *   desc  host plan description (read only; copied)
+ *   out   host out: the new library-owned plan, released by kvc_plan_destroy
+ * Returns KVC_OK and *out, or KVC_ERR_INVALID (bad description), KVC_ERR_CUDA
+ * (device allocation or copy failed) with *out = NULL and nothing allocated.
+ * Blocking; call outside stream capture. kvc_plan_create is the same call
+ * under its earlier name. */
+int kvc_plan(const kvc_plan_desc* desc, kvc_plan_t** out);
 int kvc_plan_create(const kvc_plan_desc* desc, kvc_plan_t** out);
 /* Free the plan (device memory included). NULL is ignored. */
 void kvc_plan_destroy(kvc_plan_t* plan);
@@ -139,8 +149,12 @@ size_t kvc_max_encoded_bytes(const kvc_plan_t* plan, int path, uint32_t n_slices
  * KVC_ERR_CAPACITY in its result. */
 size_t kvc_workspace_bytes(const kvc_plan_t* plan, int path, int decode, uint32_t n_slices);
 
-/* Encode slices [first_slice, first_slice + n_slices) of the cache.
- *   d_src     device [n_slices][T][D] 16-bit values (the selected slices only)
+/* kvc_encode_lossless — lossless coding of slices [first_slice, first_slice +
+ * n_slices) of the cache (AT-1 Memory page, "KV & tensor mode": token-major
+ * values reordered channel-major, split into byte planes, the smaller of coded
+ * and plain kept; QATQ page, "qatq encode": chunks of at most 65536 values).
+ *   d_src     device [n_slices][T][D] values (the selected slices only;
+ *             16-bit, or 32-bit for an f32 plan), read only
  *   d_dst     device output, dst_cap bytes (>= kvc_max_encoded_bytes)
  *   d_ws      device workspace, ws_bytes (>= kvc_workspace_bytes(..., 0, n_slices))
  *   d_res     device kvc_result: status and container bytes
@@ -150,7 +164,10 @@ int kvc_encode_lossless(const kvc_plan_t* plan, uint32_t first_slice, uint32_t n
                         const void* d_src, void* d_dst, size_t dst_cap, void* d_ws,
                         size_t ws_bytes, kvc_result* d_res, cudaStream_t stream);
 
-/* Decode a lossless container.
+/* kvc_decode_lossless — restore the exact value bytes of a lossless container
+ * (QATQ page, "QATC v2 checksum validated": corrupt or truncated payloads are
+ * refused; AT-1 Memory page, "What's proven": byte-exact round trip, tamper
+ * refusal).
  *   d_src/src_bytes  device container and its exact length in bytes
  *   d_dst/dst_cap    device output [n_slices][T][D] 16-bit values
  *   d_ws/ws_bytes    device workspace (>= kvc_workspace_bytes(..., 1, 0))
@@ -163,12 +180,22 @@ int kvc_decode_lossless(const kvc_plan_t* plan, const void* d_src, size_t src_by
                         size_t dst_cap, void* d_ws, size_t ws_bytes, kvc_result* d_res,
                         cudaStream_t stream);
 
-/* Transform coding of slices [first_slice, first_slice + n_slices); arguments
- * as kvc_encode_lossless. Needs a plan with bases; D = 128, bf16. */
+/* kvc_encode_transform — transform coding of slices [first_slice, first_slice
+ * + n_slices) (KVTC page, "How the Pipeline Works": sinks and recent window
+ * kept, RoPE undone, PCA projection, bit allocation, quantisation, entropy
+ * coding; Codec-Gauge page, "Problem Statement and Overview": Z = G X with an
+ * orthogonal G). Arguments, ownership and error channels as
+ * kvc_encode_lossless. Needs a plan with bases; D = 128, bf16, 64-token
+ * blocks, at most 512-token records (else KVC_ERR_UNSUPPORTED). */
 int kvc_encode_transform(const kvc_plan_t* plan, uint32_t first_slice, uint32_t n_slices,
                          const void* d_src, void* d_dst, size_t dst_cap, void* d_ws,
                          size_t ws_bytes, kvc_result* d_res, cudaStream_t stream);
-/* Decode a transform container; arguments as kvc_decode_lossless. */
+/* kvc_decode_transform — reconstruct a transform container (KVTC page, "How
+ * the Pipeline Works": dequantise with the stored scales and zero points, and
+ * reverse the process; Codec-Gauge page, "Problem Statement and Overview":
+ * X^ = G^-1 Z^ with G^-1 = G^T): codes dequantised, projected back, keys
+ * rotated forward, rounded to bf16. Arguments, ownership and error channels
+ * as kvc_decode_lossless; the raw sink and recent rows come back bit-exact. */
 int kvc_decode_transform(const kvc_plan_t* plan, const void* d_src, size_t src_bytes, void* d_dst,
                          size_t dst_cap, void* d_ws, size_t ws_bytes, kvc_result* d_res,
                          cudaStream_t stream);
@@ -318,8 +345,11 @@ int kvc_stage_stream_decode(const uint8_t* d_rec, uint32_t rec_bytes, uint32_t n
  * a fixed 128 KiB array inside the library, one per device, so n is limited to
  * 65536 symbols; larger n returns KVC_ERR_CAPACITY. The output bytes and
  * d_res are those of kvc_stage_stream_encode for the same symbols.
- * The first call on a device looks the array up (set-up on the host); make
- * that first call before starting any stream capture. Calls that overlap on
+ * Every call looks up the array's device address on the current device
+ * (cudaGetSymbolAddress, host side). The first call on a device, and the first
+ * after a cudaDeviceReset, also loads the library's device code there, which
+ * is when the array is reserved: make that first call before starting any
+ * stream capture. Calls that overlap on
  * the device (on different streams, or from different host threads without
  * ordering) share the one array and race: order them. The container format
  * has no counterpart of this call; it only changes where the scratch lives. */

@@ -13,7 +13,12 @@ from dataclasses import dataclass
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libkvc.so")
+# KVC_BUILD_VARIANT=<name> loads the in-tree test build libkvc_<name>.so (see
+# build.VARIANTS) instead of libkvc.so; a missing library fails the import.
+_VARIANT = os.environ.get("KVC_BUILD_VARIANT", "")
+if _VARIANT and not _VARIANT.isidentifier():
+    raise ImportError(f"bad KVC_BUILD_VARIANT {_VARIANT!r}")
+LIB_PATH = os.path.join(_HERE, f"libkvc_{_VARIANT}.so" if _VARIANT else "libkvc.so")
 
 OK, ERR_INVALID, ERR_CAPACITY, ERR_CORRUPT, ERR_TRUNCATED, ERR_PLAN_MISMATCH = 0, 1, 2, 3, 4, 5
 ERR_TIMEOUT, ERR_CUDA, ERR_UNSUPPORTED = 6, 7, 8
@@ -23,7 +28,7 @@ LOSSLESS, TRANSFORM = 0, 1
 ABI_VERSION = 1
 
 EXPORTS = [
-    "kvc_plan_create", "kvc_plan_destroy", "kvc_plan_widths", "kvc_plan_crc",
+    "kvc_plan", "kvc_plan_create", "kvc_plan_destroy", "kvc_plan_widths", "kvc_plan_crc",
     "kvc_max_encoded_bytes", "kvc_workspace_bytes",
     "kvc_encode_lossless", "kvc_decode_lossless", "kvc_encode_transform", "kvc_decode_transform",
     "kvc_status_string", "kvc_calibrate_pca", "kvc_allocate_bits",
@@ -74,6 +79,7 @@ def _load():
     lib = ctypes.CDLL(LIB_PATH)
     vp, sz, u32, i32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_uint32, ctypes.c_int
     sig = {
+        "kvc_plan": ([ctypes.POINTER(PlanDesc), ctypes.POINTER(vp)], i32),
         "kvc_plan_create": ([ctypes.POINTER(PlanDesc), ctypes.POINTER(vp)], i32),
         "kvc_plan_destroy": ([vp], None),
         "kvc_plan_widths": ([vp, vp, sz], i32),
@@ -182,7 +188,7 @@ class Plan:
         w = None if widths is None else np.ascontiguousarray(widths, dtype=np.uint8)
         desc = shape.desc(b, e, w)
         h = ctypes.c_void_p()
-        _check(_lib.kvc_plan_create(ctypes.byref(desc), ctypes.byref(h)), "kvc_plan_create")
+        _check(_lib.kvc_plan(ctypes.byref(desc), ctypes.byref(h)), "kvc_plan")
         self._h = h
         self.has_transform = b is not None
 

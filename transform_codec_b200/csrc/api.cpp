@@ -262,7 +262,7 @@ void free_plan(kvc_plan_s* p) {
 
 }  // namespace
 
-extern "C" int kvc_plan_create(const kvc_plan_desc* desc, kvc_plan_t** out) {
+extern "C" int kvc_plan(const kvc_plan_desc* desc, kvc_plan_t** out) {
   if (!desc || !out) return KVC_ERR_INVALID;
   *out = nullptr;
   const kvc_plan_desc& d = *desc;
@@ -352,6 +352,8 @@ extern "C" int kvc_plan_create(const kvc_plan_desc* desc, kvc_plan_t** out) {
   *out = p;
   return KVC_OK;
 }
+
+extern "C" int kvc_plan_create(const kvc_plan_desc* desc, kvc_plan_t** out) { return kvc_plan(desc, out); }
 
 extern "C" void kvc_plan_destroy(kvc_plan_t* plan) { free_plan(plan); }
 
