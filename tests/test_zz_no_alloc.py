@@ -40,13 +40,20 @@ def test_noalloc_matches_scratch_entry_point_twice(name, sym):
     d_sym = torch.from_numpy(sym.copy()).cuda()
     st_ref, want = _encode_with_scratch(d_sym, n)
     assert st_ref == kvc.OK
-    for _ in range(2):
-        out = torch.full((16 + (n + 15) // 16 * 16,), 0xA5, dtype=torch.uint8, device="cuda")
-        res = torch.zeros(2, dtype=torch.int64, device="cuda")
-        kvc.stage_stream_encode_noalloc(d_sym, n, out, res)
-        st, nbytes = kvc.read_result(res)
+    outs = [torch.full((16 + (n + 15) // 16 * 16,), 0xA5, dtype=torch.uint8, device="cuda")
+            for _ in range(2)]
+    ress = [torch.zeros(2, dtype=torch.int64, device="cuda") for _ in range(2)]
+    for i in range(2):
+        if i == 1:  # after the first call's set-up, a call takes no device memory
+            torch.cuda.synchronize()
+            free_before = torch.cuda.mem_get_info()[0]
+        kvc.stage_stream_encode_noalloc(d_sym, n, outs[i], ress[i])
+        if i == 1:
+            torch.cuda.synchronize()
+            assert torch.cuda.mem_get_info()[0] == free_before
+        st, nbytes = kvc.read_result(ress[i])
         assert st == kvc.OK
-        assert out[:nbytes].cpu().numpy().tobytes() == want
+        assert outs[i][:nbytes].cpu().numpy().tobytes() == want
 
 
 def test_noalloc_refuses_sizes_past_its_scratch():

@@ -4,7 +4,6 @@
 // aggregate checksum; "QATC v2 checksum validated": corrupt or truncated
 // payloads are refused before restore). Also the stage kernels used to check
 // the CRC and rANS stages on their own.
-#include <mutex>
 
 #include "kvc.h"
 #include "kvc_device.cuh"
@@ -405,29 +404,18 @@ cudaError_t launch_stage_stream_decode(const uint8_t* rec, uint32_t rec_bytes, u
 static __device__ __align__(256) uint16_t g_noalloc_scratch[kvc::kMaxChunkValues];
 
 namespace {
-constexpr int kNoAllocMaxDevices = 64;
-std::mutex g_noalloc_mu;
-uint16_t* g_noalloc_ptr[kNoAllocMaxDevices] = {};
-
-// Device address of the scratch array on the current device, looked up once
-// per device (the first call on a device does this set-up).
+// Device address of the scratch array in the current context. It is looked up
+// on every call: the lookup is host-side and allocates nothing once the
+// library's device code is loaded, and a cached address would go stale after
+// a cudaDeviceReset or under another context made current on the same device.
 uint16_t* noalloc_scratch(int* status) {
-  int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
     *status = KVC_ERR_CUDA;
     return nullptr;
   }
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
-      *status = KVC_ERR_CUDA;
-      return nullptr;
-    }
-    g_noalloc_ptr[dev] = static_cast<uint16_t*>(p);
-  }
   *status = KVC_OK;
-  return g_noalloc_ptr[dev];
+  return static_cast<uint16_t*>(p);
 }
 }  // namespace
 
