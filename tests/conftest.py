@@ -15,7 +15,7 @@ def _build_library():
     spec = importlib.util.spec_from_file_location("_kvc_build", path)
     mod = importlib.util.module_from_spec(spec)
     spec.loader.exec_module(mod)
-    mod.build()
+    mod.build_all()
 
 
 _build_library()

@@ -24,6 +24,14 @@ constexpr uint32_t kTile = 64;      // tokens per tile = quantiser block
 constexpr uint32_t kMaxCt = 512;    // max tokens per middle chunk
 constexpr uint32_t kTcRows = 128;   // tokens per tensor-core tile (MMA M)
 constexpr uint32_t kTcCols = 128;   // tensor-memory columns: one fp32 128 x 128 accumulator
+// Polls of the tensor stage's wait for its own MMAs before the record is
+// reported as KVC_ERR_TIMEOUT. A build with -DKVC_MMA_WAIT_POLLS=0
+// makes that wait give up on purpose, so tests can check the timeout status;
+// the drain wait that follows keeps its own long bound in every build.
+#ifndef KVC_MMA_WAIT_POLLS
+#define KVC_MMA_WAIT_POLLS (1u << 22)
+#endif
+constexpr uint32_t kMmaDrainPolls = 1u << 22;
 
 __device__ inline float bf16_to_f32(uint32_t h) { return __uint_as_float(h << 16); }
 
@@ -1408,7 +1416,7 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
   tc::fence_after_sync();
   const uint32_t tmem = S.tmem_base;
   uint32_t phase = 0;
-  bool alive = true;
+  bool alive = true, drained = true;
   const uint32_t rps = 1u + sh.n_mid;
   constexpr uint32_t idesc = tc::idesc_bf16_f32(kTcRows, kD);
   uint32_t cur_sidx = 0xffffffffu;  // slice whose component order and Q pieces are loaded
@@ -1535,11 +1543,13 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
         for (uint32_t i = 0; i < 16; ++i) rp[i] = rl ? __ldg(cs4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
       if (t_base + kTcRows < tcc) load_codes(t_base + kTcRows);
-      const bool done = tc::mbar_wait(&S.bar, phase, 1u << 22);
+      const bool done = tc::mbar_wait(&S.bar, phase, KVC_MMA_WAIT_POLLS);
       phase ^= 1u;
       if (!__syncthreads_and(done)) {
         if (tid == 0) atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(kErrTimeout));
-        tc::mbar_wait(&S.bar, phase ^ 1u, 1u << 22);
+        // drain: the same completion again, with the long bound, so that the
+        // accumulator is no longer written when the block frees it
+        drained = __syncthreads_and(tc::mbar_wait(&S.bar, phase ^ 1u, kMmaDrainPolls));
         alive = false;
         break;
       }
@@ -1590,7 +1600,10 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
   }
   tc::fence_before_sync();
   __syncthreads();
-  if (warp == 0) {
+  // MMAs still pending after the drain's bound would write tensor memory
+  // after it is freed (and handed to another block): the block then keeps its
+  // allocation, and the record already carries the timeout status
+  if (warp == 0 && drained) {
     tc::fence_after_sync();
     tc::tmem_dealloc(tmem, kTcCols);
   }
