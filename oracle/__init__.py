@@ -43,6 +43,7 @@ class Desc(ctypes.Structure):
         ("block_tokens", ctypes.c_uint32), ("chunk_tokens", ctypes.c_uint32),
         ("max_bits", ctypes.c_uint32), ("rope_theta", ctypes.c_double),
         ("bases", ctypes.c_void_p), ("widths", ctypes.c_void_p),
+        ("plan_crc", ctypes.c_uint32), ("plan_crc_set", ctypes.c_uint32),
     ]
 
 
@@ -119,6 +120,11 @@ class Plan:
                          n_sink, n_recent, block_tokens, chunk_tokens, max_bits, rope_theta,
                          None if self.bases is None else _ptr(self.bases),
                          None if self.widths is None else _ptr(self.widths))
+        self._bound = {}
+        if self.bases is not None and self.widths is not None:
+            # the plan CRC every transform container carries, computed once here
+            self.desc.plan_crc = _load().kvco_plan_crc(ctypes.byref(self.desc))
+            self.desc.plan_crc_set = 1
 
     @property
     def n_slices(self):
@@ -304,7 +310,9 @@ def encode_transform(plan: Plan, src: np.ndarray, first_slice: int = 0) -> bytes
     s = np.ascontiguousarray(src, dtype=np.uint16)
     n_slices = s.size // (plan.desc.n_tokens * plan.desc.head_dim)
     lib = _load()
-    cap = lib.kvco_transform_bound(ctypes.byref(plan.desc), n_slices)
+    if n_slices not in plan._bound:
+        plan._bound[n_slices] = lib.kvco_transform_bound(ctypes.byref(plan.desc), n_slices)
+    cap = plan._bound[n_slices]
     out = np.zeros(max(cap, 1), dtype=np.uint8)
     n = lib.kvco_encode_transform(ctypes.byref(plan.desc), first_slice, n_slices,
                                   _ptr(s) if s.size else None, _ptr(out), cap)

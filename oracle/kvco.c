@@ -849,6 +849,11 @@ uint32_t kvco_plan_crc(const kvco_desc* d) {
   return crc;
 }
 
+/* The plan CRC a container carries: the caller's precomputed value when set. */
+static uint32_t plan_crc_of(const kvco_desc* d) {
+  return d->plan_crc_set ? d->plan_crc : kvco_plan_crc(d);
+}
+
 /* ---------------------------------------------------------------------------
  * Transform coding ([KVTC] "How the Pipeline Works": sink tokens and a recent
  * window kept at full fidelity, the middle RoPE-undone, projected on a PCA basis,
@@ -929,23 +934,35 @@ static size_t parse_buf_bytes(const kvco_desc* d) {
   return a > b ? a : b;
 }
 
-size_t kvco_transform_bound(const kvco_desc* d, uint32_t n_slices) {
-  if (!transform_ok(d)) return 0;
+/* Largest record bytes of one slice (raw record + middle records at most RAW). */
+static size_t slice_bound(const kvco_desc* d, uint32_t sl) {
   uint32_t s_end, r_start, T = d->n_tokens, D = d->head_dim;
   regions(d, &s_end, &r_start);
   uint32_t nm = n_mid_chunks(d);
-  size_t raw = pad16((size_t)(s_end + T - r_start) * D * 2u);
+  size_t b = pad16((size_t)(s_end + T - r_start) * D * 2u);
+  for (uint32_t c = 0; c < nm; c++) {
+    uint32_t t0 = s_end + c * d->chunk_tokens;
+    uint32_t tcc = r_start - t0 < d->chunk_tokens ? r_start - t0 : d->chunk_tokens;
+    b += mid_record_bound(d, d->widths + (size_t)sl * D, tcc);
+  }
+  return b;
+}
+
+size_t kvco_transform_bound(const kvco_desc* d, uint32_t n_slices) {
+  if (!transform_ok(d)) return 0;
   size_t max_slice = 0;
   for (uint32_t sl = 0; sl < n_slices_total(d); sl++) {
-    size_t b = raw;
-    for (uint32_t c = 0; c < nm; c++) {
-      uint32_t t0 = s_end + c * d->chunk_tokens;
-      uint32_t tcc = r_start - t0 < d->chunk_tokens ? r_start - t0 : d->chunk_tokens;
-      b += mid_record_bound(d, d->widths + (size_t)sl * D, tcc);
-    }
+    size_t b = slice_bound(d, sl);
     if (b > max_slice) max_slice = b;
   }
-  return HDR_BYTES + (size_t)n_slices * ((size_t)IDX_ENTRY * (1u + nm) + max_slice);
+  return HDR_BYTES + (size_t)n_slices * ((size_t)IDX_ENTRY * (1u + n_mid_chunks(d)) + max_slice);
+}
+
+/* The most bytes slices [first, first + n) can take (at most the bound above). */
+static size_t transform_range_bound(const kvco_desc* d, uint32_t first, uint32_t n) {
+  size_t b = HDR_BYTES + (size_t)n * IDX_ENTRY * (1u + n_mid_chunks(d));
+  for (uint32_t sl = first; sl < first + n; sl++) b += slice_bound(d, sl);
+  return b;
 }
 
 /* y_j = (float) sum_k (double) Q[k][j] * (double) x_k, k ascending, fp64 sum
@@ -1035,7 +1052,7 @@ static void mid_chunk_quantize(const kvco_desc* d, uint32_t sidx, const uint16_t
 size_t kvco_encode_transform(const kvco_desc* d, uint32_t first_slice, uint32_t n_slices,
                              const uint16_t* src, uint8_t* dst, size_t cap) {
   if (!transform_ok(d) || (uint64_t)first_slice + n_slices > n_slices_total(d)) return 0;
-  if (cap < kvco_transform_bound(d, n_slices)) return 0;
+  if (cap < transform_range_bound(d, first_slice, n_slices)) return 0;
   uint32_t T = d->n_tokens, D = d->head_dim, half = D / 2, ct = d->chunk_tokens;
   uint32_t B = d->block_tokens, nbmax = ct / B;
   uint32_t s_end, r_start;
@@ -1104,7 +1121,7 @@ size_t kvco_encode_transform(const kvco_desc* d, uint32_t first_slice, uint32_t 
     }
   }
   free(cs); free(y); free(codes); free(syms); free(zs); free(side);
-  write_header(dst, KVCO_TRANSFORM, d, first_slice, n_slices, ct, nr, p, kvco_plan_crc(d));
+  write_header(dst, KVCO_TRANSFORM, d, first_slice, n_slices, ct, nr, p, plan_crc_of(d));
   put32(dst + 60, header_crc(dst, nr));
   return p;
 }
@@ -1166,7 +1183,7 @@ int kvco_decode_transform(const kvco_desc* d, const uint8_t* src, size_t n, uint
   if (!transform_ok(d)) return KVCO_INVALID;
   uint32_t first, ns, nr;
   int st = check_container(d, KVCO_TRANSFORM, src, n, transform_records, d->chunk_tokens,
-                           kvco_plan_crc(d), &first, &ns, &nr);
+                           plan_crc_of(d), &first, &ns, &nr);
   if (st) return st;
   uint32_t T = d->n_tokens, D = d->head_dim, half = D / 2, ct = d->chunk_tokens;
   uint32_t H = d->n_heads, B = d->block_tokens, nbmax = ct / B;
@@ -1287,7 +1304,7 @@ int kvco_container_codes(const kvco_desc* d, const uint8_t* src, size_t n, uint3
   if (!transform_ok(d)) return KVCO_INVALID;
   uint32_t first, ns, nr;
   int st = check_container(d, KVCO_TRANSFORM, src, n, transform_records, d->chunk_tokens,
-                           kvco_plan_crc(d), &first, &ns, &nr);
+                           plan_crc_of(d), &first, &ns, &nr);
   if (st) return st;
   uint32_t T = d->n_tokens, D = d->head_dim, ct = d->chunk_tokens;
   uint32_t nbmax = ct / d->block_tokens;

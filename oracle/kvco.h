@@ -51,6 +51,10 @@ typedef struct {
   double rope_theta;
   const float* bases;        /* [L*2*H][D][D], Q[k*D + j], column j = component j */
   const uint8_t* widths;     /* [L*2*H][D] bits per component */
+  /* optional: kvco_plan_crc(d) computed once by the caller (plan_crc_set = 1),
+   * so that each transform call does not recompute it over all the bases;
+   * 0 and 0 make every call compute it */
+  uint32_t plan_crc, plan_crc_set;
 } kvco_desc;
 
 uint32_t kvco_crc32(const void* p, size_t n);

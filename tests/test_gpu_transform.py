@@ -198,6 +198,85 @@ def test_transform_full_size_sampled():
         assert rel_rms(y_o[0], y_g[s]) <= REL_RMS
 
 
+def test_transform_full_size_32k_sampled():
+    """Qwen3-32B-shaped cache at 32k (64 x 8 x 32768 x 128 bf16, 8.59 GB,
+    theta 5e5, 1.6 bits per value), coded as the benchmark codes it: 128 frames
+    of 8 slices (64 MiB), encoded 16 frames per batch call and decoded in one
+    batch call. Every frame must report OK; sampled K and V slices in four
+    frames are checked against the oracle under the parity rule (codes) and the
+    reconstruction bar. 1.6 bits reach other coded-component counts per slice
+    than the 2.0-bit workloads."""
+    import torch
+    w = kvgen.WORKLOADS["transform-64x8x32768x128-bf16"]
+    shape = kvc.Shape.from_workload(w)
+    spf = w.slices_per_frame
+    F = w.n_slices // spf
+    sampled = [0, 13, 518, 1023]
+    pcs, cal = _oracle_pca(w, sampled)
+    bases, lam = kvc.calibrate_pca(shape, cal)
+    for s in sampled:
+        bases[s], lam[s] = pcs[s]
+    widths = oracle.allocate(lam, w.avg_bits, w.max_bits).reshape(lam.shape)
+    plan, oplan = _plans(w, bases, widths)
+    assert plan.crc == oracle.plan_crc(oplan)
+    vals = spf * w.n_tokens * w.head_dim
+    host = torch.empty(F * vals, dtype=torch.int16).pin_memory()
+    kvgen.slices(w, 0, w.n_slices, out=host.data_ptr())
+    x = host.cuda()
+    cap = plan.max_encoded_bytes(kvc.TRANSFORM, spf)
+    cont = torch.empty(F * cap, dtype=torch.uint8, device="cuda")
+    out = torch.zeros(F * vals, dtype=torch.int16, device="cuda")
+    res = torch.zeros(2 * F, 2, dtype=torch.int64, device="cuda")
+    grp = 16
+    ws = torch.empty(kvc.batch_workspace_bytes(plan, kvc.TRANSFORM, False, grp, spf), dtype=torch.uint8,
+                     device="cuda")
+    for g in range(0, F, grp):
+        kvc.encode_batch(plan, kvc.TRANSFORM,
+                         [(f * spf, spf, x[f * vals:(f + 1) * vals], cont[f * cap:(f + 1) * cap], res[f])
+                          for f in range(g, min(F, g + grp))], ws)
+    r = res[:F].cpu().numpy()
+    assert np.all((r[:, 0] & 0xFFFFFFFF) == 0)
+    sizes = r[:, 1].tolist()
+    wsd = torch.empty(kvc.batch_workspace_bytes(plan, kvc.TRANSFORM, True, F, spf), dtype=torch.uint8,
+                      device="cuda")
+    kvc.decode_batch(plan, kvc.TRANSFORM,
+                     [(cont[f * cap:(f + 1) * cap], sizes[f], out[f * vals:(f + 1) * vals], res[F + f])
+                      for f in range(F)], wsd, spf)
+    r = res[F:].cpu().numpy()
+    assert np.all((r[:, 0] & 0xFFFFFFFF) == 0)
+    assert r[:, 1].tolist() == [2 * vals] * F
+    s_end, r_start = _regions(w)
+    rps = 1 + (r_start - s_end + w.chunk_tokens - 1) // w.chunk_tokens
+    xs = host.numpy().view(np.uint16).reshape(w.n_slices, w.n_tokens, w.head_dim)
+    ys = out.cpu().numpy().view(np.uint16).reshape(w.n_slices, w.n_tokens, w.head_dim)
+    total = mism = 0
+    for s in sampled:
+        f = s // spf
+        got = cont[f * cap:f * cap + sizes[f]].cpu().numpy().tobytes()
+        recs = _records(got)
+        assert len(recs) == spf * rps
+        i0 = (s - f * spf) * rps
+        raw = np.concatenate([xs[s, :s_end], xs[s, r_start:]]).tobytes()
+        assert recs[i0] == raw + bytes((-len(raw)) % 16)
+        oc, qp, _ = oracle.transform_slice_codes(oplan, s, xs[s])
+        codes = np.zeros_like(oc)
+        for c in range(rps - 1):
+            t0 = s_end + c * w.chunk_tokens
+            tcc = min(w.chunk_tokens, r_start - t0)
+            st, cc, _ = oracle.record_codes(oplan, s, recs[i0 + 1 + c], tcc)
+            assert st == oracle.OK
+            codes[t0:t0 + tcc] = cc
+        n, m = _check_codes(codes, oc, qp, widths[s], slice(s_end, r_start))
+        total, mism = total + n, mism + m
+        one = oracle.encode_transform(oplan, xs[s:s + 1], first_slice=s)
+        st_o, y_o = oracle.decode_transform(oplan, one, n_slices_cap=1)
+        assert st_o == oracle.OK
+        assert rel_rms(y_o[0], ys[s]) <= REL_RMS
+        assert np.array_equal(ys[s, :s_end], xs[s, :s_end])
+        assert np.array_equal(ys[s, r_start:], xs[s, r_start:])
+    assert mism <= (1 - CODE_MATCH) * total
+
+
 @pytest.mark.parametrize("T", [1024, 644])
 def test_transform_container_equals_oracle_bytes(T):
     """The encoder's projection reproduces the oracle's fp64 y bit for bit (the
