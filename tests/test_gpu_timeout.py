@@ -1,9 +1,10 @@
-"""The transform decoder's one device wait (its tensor-core MMAs' completion)
-is bounded: when it gives up, the record reports KVC_ERR_TIMEOUT in the
-device result instead of spinning, and the context stays usable.
+"""The codec's device waits (the transform encoder's and decoder's waits for
+their own tensor-core MMAs) are bounded: when one gives up, the frame reports
+KVC_ERR_TIMEOUT in its device result instead of spinning, and the context
+stays usable.
 
-The wait is made to run out on purpose with the library's "wait0" test build
-(the first completion wait gives up without polling; the drain wait that
+The waits are made to run out on purpose with the library's "wait0" test
+build (the first completion wait gives up without polling; the drain wait that
 follows keeps its long bound, so the MMAs have finished before the block frees
 their tensor memory). Nothing faults: the kernel only takes its error path.
 The build runs in a child process, since a process loads one libkvc."""
@@ -35,11 +36,13 @@ bases = np.stack([p[0] for p in pcs])
 widths = oracle.allocate(np.stack([p[1] for p in pcs]), w.avg_bits, w.max_bits).reshape(w.n_slices, 128)
 x = kvgen.slices(w)
 plan = kvc.Plan(kvc.Shape.from_workload(w), bases=bases, widths=widths)
-st, c = encode(plan, kvc.TRANSFORM, x)
-assert st == kvc.OK, st
-# the container is the oracle's (the encoder has no bounded wait to trip)
+# the encoder's projection waits for its MMAs too: the frame reports the timeout
+for _ in range(2):
+    st, _ = encode(plan, kvc.TRANSFORM, x)
+    assert st == kvc.ERR_TIMEOUT, kvc.status_string(st)
+# the decoder's tensor stage, on the oracle's container
 oplan = oracle.Plan.from_workload(w, bases=bases, widths=widths)
-assert oracle.decode_transform(oplan, c)[0] == oracle.OK
+c = oracle.encode_transform(oplan, x)
 for _ in range(2):
     st, _ = decode(plan, kvc.TRANSFORM, c, w.n_slices)
     assert st == kvc.ERR_TIMEOUT, kvc.status_string(st)

@@ -76,6 +76,9 @@ struct kvc_plan_s {
   float* d_rope = nullptr;
   uint8_t* d_qsplit = nullptr;
   CompInfo* d_comp = nullptr;
+  uint8_t* d_qdig = nullptr;
+  QColInfo* d_qcol = nullptr;
+  float* d_qt = nullptr;
   // host-streamed calls: two copy streams and the ring's events, made by the
   // first such call and kept until the plan is destroyed
   cudaStream_t copy_in = nullptr, copy_out = nullptr;
@@ -243,6 +246,52 @@ void split_bases(const float* bases, uint32_t S, std::vector<uint8_t>& out) {
   }
 }
 
+// Per slice, the coded columns of Q as the B operand of the encoder's exact
+// tensor-core projection (see QColInfo): integer J = rint(Q 2^(29 - f)) as four
+// byte planes (byte 0 the signed top byte), row cc, K index k; and Q
+// transposed (fp32) for the fp64 chains that settle open decisions.
+void digit_bases(const float* bases, const uint8_t* widths, uint32_t S, std::vector<uint8_t>& dig,
+                 std::vector<QColInfo>& col, std::vector<float>& qt) {
+  const uint32_t D = 128;
+  dig.assign(size_t(S) * kQDigBytes, 0);
+  col.assign(S, QColInfo{});
+  qt.assign(size_t(S) * D * D, 0.0f);
+  for (uint32_t s = 0; s < S; ++s) {
+    const float* Q = bases + size_t(s) * D * D;
+    uint8_t* planes = dig.data() + size_t(s) * kQDigBytes;
+    for (uint32_t j = 0; j < D; ++j)
+      for (uint32_t k = 0; k < D; ++k) qt[(size_t(s) * D + j) * D + k] = Q[size_t(k) * D + j];
+    uint32_t cc = 0;
+    for (uint32_t j = 0; j < D; ++j) {
+      if (!widths[size_t(s) * D + j]) continue;
+      double m = 0.0, l1 = 0.0;
+      for (uint32_t k = 0; k < D; ++k) {
+        const double q = std::fabs(double(Q[size_t(k) * D + j]));
+        m = std::max(m, q);
+        l1 += q;
+      }
+      // l1 is within 128 * 2^-53 relative of the exact sum; the margin makes
+      // the stored value an upper bound
+      float q1 = float(l1 * (1.0 + 0x1p-40));
+      if (double(q1) < l1 * (1.0 + 0x1p-40)) q1 = std::nextafter(q1, INFINITY);
+      col[s].q1[cc] = q1;
+      if (m == 0.0) {
+        col[s].f[cc] = kQColZero;
+      } else {
+        const int f = std::ilogb(m);
+        col[s].f[cc] = f;
+        for (uint32_t k = 0; k < D; ++k) {
+          const int64_t J = int64_t(std::nearbyint(std::ldexp(double(Q[size_t(k) * D + j]), 29 - f)));
+          const uint32_t u = uint32_t(int32_t(J));
+          for (uint32_t p = 0; p < 4; ++p)
+            planes[p * kQDigPlane + sw128_offset_host(cc, k, D)] = uint8_t(u >> (24 - 8 * p));
+        }
+      }
+      ++cc;
+    }
+  }
+}
+
 void free_plan(kvc_plan_s* p) {
   if (!p) return;
   if (p->d_bases) cudaFree(p->d_bases);
@@ -250,6 +299,9 @@ void free_plan(kvc_plan_s* p) {
   if (p->d_rope) cudaFree(p->d_rope);
   if (p->d_qsplit) cudaFree(p->d_qsplit);
   if (p->d_comp) cudaFree(p->d_comp);
+  if (p->d_qdig) cudaFree(p->d_qdig);
+  if (p->d_qcol) cudaFree(p->d_qcol);
+  if (p->d_qt) cudaFree(p->d_qt);
   if (p->copy_in) cudaStreamSynchronize(p->copy_in);
   if (p->copy_out) cudaStreamSynchronize(p->copy_out);
   for (auto& row : p->ring_ev)
@@ -330,6 +382,10 @@ extern "C" int kvc_plan(const kvc_plan_desc* desc, kvc_plan_t** out) {
     split_bases(d.bases, p->S, qs);
     std::vector<CompInfo> ci(p->S);
     for (uint32_t s = 0; s < p->S; ++s) comp_info(p->widths.data() + size_t(s) * 128u, ci[s]);
+    std::vector<uint8_t> qd;
+    std::vector<QColInfo> qc;
+    std::vector<float> qt;
+    digit_bases(d.bases, p->widths.data(), p->S, qd, qc, qt);
     const size_t nb = size_t(p->S) * d.head_dim * d.head_dim * sizeof(float);
     bool ok = cudaMalloc(&p->d_bases, nb) == cudaSuccess &&
               cudaMalloc(&p->d_widths, p->widths.size()) == cudaSuccess &&
@@ -343,7 +399,14 @@ extern "C" int kvc_plan(const kvc_plan_desc* desc, kvc_plan_t** out) {
               cudaMemcpy(p->d_qsplit, qs.data(), qs.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
               cudaMalloc(&p->d_comp, ci.size() * sizeof(CompInfo)) == cudaSuccess &&
               cudaMemcpy(p->d_comp, ci.data(), ci.size() * sizeof(CompInfo), cudaMemcpyHostToDevice) ==
-                  cudaSuccess;
+                  cudaSuccess &&
+              cudaMalloc(&p->d_qdig, qd.size()) == cudaSuccess &&
+              cudaMemcpy(p->d_qdig, qd.data(), qd.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMalloc(&p->d_qcol, qc.size() * sizeof(QColInfo)) == cudaSuccess &&
+              cudaMemcpy(p->d_qcol, qc.data(), qc.size() * sizeof(QColInfo), cudaMemcpyHostToDevice) ==
+                  cudaSuccess &&
+              cudaMalloc(&p->d_qt, qt.size() * sizeof(float)) == cudaSuccess &&
+              cudaMemcpy(p->d_qt, qt.data(), qt.size() * sizeof(float), cudaMemcpyHostToDevice) == cudaSuccess;
     if (!ok) {
       free_plan(p);
       return KVC_ERR_CUDA;
@@ -478,7 +541,8 @@ int encode_frames(const kvc_plan_s* plan, int path, const kvc_frame* fr, uint32_
     if (path == KVC_PATH_LOSSLESS) {
       e = launch_lossless_encode(plan->ls, b, L, stream);
     } else {
-      TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope, plan->d_qsplit, plan->d_comp};
+      TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope, plan->d_qsplit, plan->d_comp,
+                          plan->d_qdig, plan->d_qcol, plan->d_qt};
       e = launch_transform_encode(plan->ts, pd, b, L, stream);
     }
     if (e != cudaSuccess) return KVC_ERR_CUDA;
@@ -537,7 +601,8 @@ int decode_frames(const kvc_plan_s* plan, int path, const kvc_frame* fr, uint32_
     if (path == KVC_PATH_LOSSLESS) {
       e = launch_lossless_decode(plan->ls, b, ws, max_rec, stream);
     } else {
-      TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope, plan->d_qsplit, plan->d_comp};
+      TransformPlanDev pd{plan->d_bases, plan->d_widths, plan->d_rope, plan->d_qsplit, plan->d_comp,
+                          plan->d_qdig, plan->d_qcol, plan->d_qt};
       e = launch_transform_decode(plan->ts, pd, b, ws, max_rec, stream);
     }
     if (e != cudaSuccess) return KVC_ERR_CUDA;

@@ -63,11 +63,27 @@ k_finalize(HeaderFields h, FrameBatch b, EncodeLayout ws) {
   uint8_t* dst = fd.dst;
   Result* res = static_cast<Result*>(fd.res);
   EncodeState* es = ws.state + f;
+  __shared__ int kerr;
+  if (tid == 0) kerr = 0;
   crc_tables_init(crc_t);
   const uint32_t per = (nr + nthr - 1) / nthr;
   const uint32_t beg = min(nr, tid * per), end = min(nr, beg + per);
   uint64_t mine = 0;
-  for (uint32_t i = beg; i < end; ++i) mine += ws.rec_len[g0 + i];
+  for (uint32_t i = beg; i < end; ++i) {
+    const uint32_t len = ws.rec_len[g0 + i];
+    if (len >= kRecLenError) atomicMax(&kerr, int(len & 0xffu));
+    mine += len;
+  }
+  __syncthreads();
+  if (kerr) {  // a record its encoder could not produce: the frame reports its status
+    if (tid == 0) {
+      es->status = kerr;
+      es->total_bytes = 0;
+      res->status = kerr;
+      res->bytes = 0;
+    }
+    return;
+  }
   uint64_t sum_all;
   uint64_t pre = block_exclusive_scan64(mine, tmp64, &sum_all);
   const uint64_t first = uint64_t(kHeaderBytes) + uint64_t(kIndexEntry) * nr;

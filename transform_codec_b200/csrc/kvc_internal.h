@@ -142,14 +142,32 @@ struct alignas(16) CompInfo {
   uint32_t bstart[10], bcount[10];
   uint32_t n_coded;
 };
+// Per slice, the coded columns of Q (coded components in index order, "cc")
+// for the encoder's tensor-core projection: J[k][cc] = rint(Q[k][j] 2^r), r =
+// 29 - f, f = ilogb(max_k |Q[k][j]|), so |J| <= 2^30; the four bytes of J (two's
+// complement, byte 0 the top one) are the planes of qdig, each 128 rows (cc) x
+// 128 K bytes in the B-operand layout, zero past the coded columns.
+struct alignas(16) QColInfo {
+  int32_t f[128];   // ilogb(max_k |Q[k][j]|); kQColZero for an all-zero column
+  float q1[128];    // an upper bound of sum_k |Q[k][j]|
+};
+constexpr int32_t kQColZero = -100000;
+constexpr uint32_t kQDigPlane = 128u * 128u;         // bytes of one digit plane
+constexpr uint32_t kQDigBytes = 4u * kQDigPlane;     // per slice
 struct TransformPlanDev {
   const float* bases;      // [S][D][D], Q[k*D + j]
   const uint8_t* widths;   // [S][D]
   const float* rope;       // [T][D/2][2] cos, sin
   const uint8_t* qsplit;   // [S][hi, lo][128 x 256 B] Q as bf16 pieces, B-operand layout
   const CompInfo* comp;    // [S]
+  const uint8_t* qdig;     // [S][4 planes][128 x 128 B] Q's digits (QColInfo)
+  const QColInfo* qcol;    // [S]
+  const float* qt;         // [S][D][D] Q transposed: qt[j*D + k] = Q[k][j]
 };
 constexpr uint32_t kQSplitBytes = 2u * 128u * 256u;  // per slice
+// A record length at or above kRecLenError marks a record its encoder could not
+// produce; its low byte is the status the frame reports.
+constexpr uint32_t kRecLenError = 0xffffff00u;
 uint64_t transform_slot_bytes(const TransformShape& s);
 cudaError_t launch_transform_encode(const TransformShape& s, const TransformPlanDev& p,
                                     const FrameBatch& b, const EncodeLayout& ws, cudaStream_t st);

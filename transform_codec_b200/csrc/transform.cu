@@ -87,38 +87,62 @@ struct Split {  // i -> (component slot, token) for i = slot * tcc + t
 };
 
 // ---------------------------------------------------------------------------
-// Transform encode, part 1 (k_transform_project): one CTA per middle record,
-// 64-token tiles (one quantiser block each). The keys are de-rotated in fp32
-// and x is kept as fp64 in x[k][t]; every thread accumulates a 4-token x
-// 8-component tile of y_c = sum_k Q[k][c] x_k with fused multiply-adds, k
-// ascending, over the coded components (Q's coded columns converted to fp64
-// once per record), and y is rounded to fp32. Two threads per coded
-// component, one per half-block, find the block's minimum and maximum as a
-// sequential scan does, set the scale and quantise their tokens. Zero point
-// and scale go straight to the record's side information in the slot.
-// The codes are staged in padded token rows and
-// copied to a token-major [t][128] byte array in the slot's scratch area, and
-// the symbol counts of every width stream are gathered behind them for the
-// entropy kernel.
-constexpr uint32_t kProjTokens = 64;   // tokens per projection tile = quantiser block
+// Transform encode, part 1 (k_transform_project): the projection on the
+// tensor cores, reproducing the oracle's y to the bit.
+//
+// The quantiser must see y[t][j] = fl32(acc), acc the fp64 sum over k
+// ascending of Q[k][j] x_k (each product exact in fp64, one rounding per
+// addition; x is the token after the keys' RoPE undo, in fp32). Per 128-token
+// tile the kernel computes an estimate of acc with a rigorous bound, from exact
+// integer products on the tensor cores:
+//   X[t][k] = rint(x_k 2^s), s = 29 - e_t, e_t = ilogb(max_k |x_k|)   |X| <= 2^30
+//   J[k][j] = rint(Q[k][j] 2^r), r = 29 - f_j (plan time, QColInfo)   |J| <= 2^30
+// both as four bytes (two's complement; byte 0, the top one, signed, the others
+// unsigned). tcgen05.mma kind::i8 sums the products of byte a of X and byte b
+// of J over k exactly in s32; the ten pairs with a + b <= 3 add into four
+// accumulators (level w = a + b: four times the coded components' columns of
+// tensor memory), and
+//   V = ((P0 2^8 + P1) 2^8 + P2) 2^8 + P3,   S~ = V 2^(24 - s - r)
+// are exact in fp64. The six dropped pairs (a + b >= 4: unsigned bytes, 128
+// terms of at most 255^2) add at most 128 255^2 (3 2^16 + 2 2^8 + 1) units of
+// 2^(-s-r); rounding x and Q to X, J adds at most x1 2^(-r-1) + q1 2^(-s-1) +
+// 96 2^(-s-r) (x1 >= sum_k |x_k|, q1 >= sum_k |Q[k][j]|); and the oracle's fp64
+// chain is within 127 2^-53 sum_k |Q[k][j] x_k| <= 2^-46 x1 2^(f+1) of the exact
+// sum. So |acc - S~| <= E, and |y - fl32(S~)| <= R = E + one fp32 ulp of the
+// largest magnitude involved, with E taken per 64-token block and component at
+// the block's largest e_t and x1.
+//
+// Where R leaves a decision open, the fp64 chain itself is run (exact_y):
+//   - every token whose estimate lies within 2R of the block's smallest or
+//     largest estimate: the true minimum and maximum are among them, and every
+//     other token is strictly inside, so the sequential scan over the block
+//     (exact values for these tokens, estimates for the rest) gives the
+//     oracle's zero point and scale, -0 / +0 and ties included;
+//   - every code whose interval [y~ - R, y~ + R] maps to two different codes
+//     (the quantiser is monotone in y).
+// Tokens whose x is all zero are exact (+0) without a chain.
+//
+// Layout: one CTA per SM (persistent, contiguous runs of middle records, so a
+// slice's Q digits stay in shared memory across its records), 512 threads.
+// Per tile: digits (thread: token t = tid / 4, channels 16g .. 16g+15 and
+// their RoPE partners, g = tid % 4) -> 40 MMAs issued by one thread (four
+// K-steps of 32 bytes x ten pairs) -> epilogue (warp w: tensor-memory lanes
+// 32 (w % 4) .., column chunks w / 4 + 4i) writes y~ to y[cc][t] -> per-word
+// phase (thread: block tid / 256, coded component (tid / 2) % 128, half tid % 2
+// of the block = 32 tokens): bound, candidates, chains, zero point and scale,
+// codes, counts. The side information (z, s per coded component and block)
+// goes to the record area of the slot, the codes component-major to the code
+// array, the symbol counts per width stream behind them.
 constexpr uint32_t kCodesRow = kMaxCt;  // bytes per component row of the code array in the slot
 constexpr uint32_t kTabPool = 512;     // sum over widths 1..8 of 2^b, rounded up
 constexpr uint32_t kHistOffset = kCodesRow * kD;      // counts follow the codes in the slot
 constexpr uint32_t kCodesArea = kHistOffset + 4u * kTabPool;
 constexpr uint32_t kWordsArea = 2u * kD * kMaxCt + 64u;  // rANS word scratch: a word per symbol
+// last count of a record whose projection gave up waiting for its MMAs (the
+// entropy kernel then marks the record as failed)
+constexpr uint32_t kHistTimeout = 0xffffffffu;
 
 __device__ inline uint32_t tab_base(uint32_t b) { return (1u << b) - 2u; }  // 2 + 4 + ... + 2^(b-1)
-
-struct __align__(16) ProjSmem {
-  double Qd[kD * kD];                          // Q[k][c], coded components c < n_coded, fp64
-  double x[kD * kProjTokens];                  // x[k][t]; then y[c][t] as fp32 in the same space
-  uint32_t hist[kTabPool];                     // symbol counts of the record per width stream
-  float2 part[kThreads / 32][kD];              // per warp and coded component: (min, max) of its tokens
-  float4 qp[kD];                               // per coded component: z, s, 1/s, levels | exact << 16
-  uint32_t ccnt[8][kD];                        // counts of symbols 0..7 per coded component
-  CompInfo ci;
-  uint32_t cidx[kD];                           // coded component c -> channel-space index j
-};
 
 // The tail of a middle record's slot: the rANS word scratch, then the code
 // array (component-major: codes[j * kCodesRow + t] for component j, token t)
@@ -128,299 +152,530 @@ __device__ inline uint16_t* slot_words(uint8_t* slot, uint64_t slot_bytes) {
   return reinterpret_cast<uint16_t*>(slot + slot_bytes - kCodesArea - kWordsArea);
 }
 
-// One thread's share of a tile's inputs: items (token tt, 8-channel group q)
-// for idx = tid + 256u, u < 2: bf16 channels 8q .. 8q+7 and their RoPE partners
-// 8q+64 .. 8q+71 and, for keys, the cos/sin pairs. load() issues the global
-// reads; stage() de-rotates in fp32 and writes x[k][t] as fp64.
-struct XFetch {
-  uint4 va[2], vb[2];
-  float4 cs[2][4];
-  uint32_t bl;
-  __device__ __forceinline__ void load(const uint16_t* xs, const float* rope, bool is_key, uint32_t t0,
-                                       uint32_t tb, uint32_t n) {
-    bl = n;
-#pragma unroll
-    for (uint32_t u = 0; u < 2; ++u) {
-      const uint32_t idx = threadIdx.x + u * kThreads, tt = idx % kProjTokens, q = idx / kProjTokens;
-      if (tt < bl) {
-        const uint4* row = reinterpret_cast<const uint4*>(xs + uint64_t(t0 + tb + tt) * kD);
-        va[u] = __ldg(row + q);
-        vb[u] = __ldg(row + q + 8u);
-        if (is_key) {
-          const float4* c4 = reinterpret_cast<const float4*>(rope + (uint64_t(t0 + tb + tt) * (kD / 2) + 8u * q) * 2u);
-#pragma unroll
-          for (uint32_t i = 0; i < 4; ++i) cs[u][i] = __ldg(c4 + i);  // (cos, sin) of channels 8q+2i, 8q+2i+1
-        }
-      }
-    }
-  }
-  __device__ __forceinline__ void stage(double* x, bool is_key) const {
-#pragma unroll
-    for (uint32_t u = 0; u < 2; ++u) {
-      const uint32_t idx = threadIdx.x + u * kThreads, tt = idx % kProjTokens, q = idx / kProjTokens;
-      float a[8], bb[8];
-      if (tt < bl) {
-        const uint32_t wa[4] = {va[u].x, va[u].y, va[u].z, va[u].w}, wb[4] = {vb[u].x, vb[u].y, vb[u].z, vb[u].w};
-#pragma unroll
-        for (uint32_t i = 0; i < 4; ++i) {
-          a[2 * i] = bf16_to_f32(wa[i] & 0xffffu);
-          a[2 * i + 1] = bf16_to_f32(wa[i] >> 16);
-          bb[2 * i] = bf16_to_f32(wb[i] & 0xffffu);
-          bb[2 * i + 1] = bf16_to_f32(wb[i] >> 16);
-        }
-        if (is_key) {
-#pragma unroll
-          for (uint32_t i = 0; i < 4; ++i) {
-            const float c0 = cs[u][i].x, s0 = cs[u][i].y, c1 = cs[u][i].z, s1 = cs[u][i].w;
-            const float na0 = __fadd_rn(__fmul_rn(a[2 * i], c0), __fmul_rn(bb[2 * i], s0));
-            const float nb0 = __fsub_rn(__fmul_rn(bb[2 * i], c0), __fmul_rn(a[2 * i], s0));
-            const float na1 = __fadd_rn(__fmul_rn(a[2 * i + 1], c1), __fmul_rn(bb[2 * i + 1], s1));
-            const float nb1 = __fsub_rn(__fmul_rn(bb[2 * i + 1], c1), __fmul_rn(a[2 * i + 1], s1));
-            a[2 * i] = na0; bb[2 * i] = nb0; a[2 * i + 1] = na1; bb[2 * i + 1] = nb1;
-          }
-        }
-      } else {
-#pragma unroll
-        for (uint32_t i = 0; i < 8; ++i) a[i] = bb[i] = 0.0f;
-      }
-#pragma unroll
-      for (uint32_t i = 0; i < 8; ++i) {
-        x[(8u * q + i) * kProjTokens + tt] = double(a[i]);
-        x[(8u * q + i + 64u) * kProjTokens + tt] = double(bb[i]);
-      }
-    }
-  }
-};
+constexpr uint32_t kPThreads = 512;
+constexpr uint32_t kPTok = 128;                  // tokens per tile (MMA M)
+constexpr uint32_t kYStride = kPTok + 1u;        // y rows, one per coded component (odd stride)
+constexpr int32_t kZeroTok = INT32_MIN;          // exponent of an all-zero token
+constexpr uint32_t kChainList = 2048;            // chains per tile run by all threads; the rest by their word
+constexpr double kDropUnits = 128.0 * 255.0 * 255.0 * (3.0 * 65536.0 + 2.0 * 256.0 + 1.0) + 96.0;
 
-// One 64-token tile, which is quantiser block blk (bl valid tokens). y[t][c] =
-// sum_k Q[k][c] x[k][t] for this thread's tokens 4tg .. 4tg+3 and components
-// cc = cg + 16jb (jb < NJB): fused multiply-adds in fp64 with k ascending,
-// rounded to fp32. The block's minimum and maximum per component are then
-// combined in token order, the earlier of two equal values winning (the
-// sequential scan's result, -0 and +0 included): over the thread's tokens,
-// with the other half of the warp, and over the warps in order. Each thread
-// quantises its own values and writes a component's four codes with one
-// store; counts of symbols 0..7 per component gather in cnt, a byte each.
-template <uint32_t NJB>
-__device__ __forceinline__ void project_quantize_tile(ProjSmem& S, uint32_t tg, uint32_t cg, uint32_t nc,
-                                                      uint32_t bl, uint32_t tb, uint32_t nb, uint8_t* rec,
-                                                      uint8_t* codes, uint32_t (&cnt)[8][2]) {
-  const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
-  double acc[4][NJB];
-#pragma unroll
-  for (uint32_t i = 0; i < 4; ++i)
-#pragma unroll
-    for (uint32_t jb = 0; jb < NJB; ++jb) acc[i][jb] = 0.0;
-  // operands of row k + 1 are loaded before the multiply-adds of row k
-  const double* xb = &S.x[4u * tg];
-  const double* qb = &S.Qd[cg];
-  double2 x0 = reinterpret_cast<const double2*>(xb)[0], x1 = reinterpret_cast<const double2*>(xb)[1];
-  double qv[NJB];
-#pragma unroll
-  for (uint32_t jb = 0; jb < NJB; ++jb) qv[jb] = qb[16u * jb];
-#pragma unroll 2
-  for (uint32_t k = 0; k < kD; ++k) {
-    const uint32_t kn = k + 1u < kD ? k + 1u : k;
-    const double2 n0 = reinterpret_cast<const double2*>(xb + kn * kProjTokens)[0];
-    const double2 n1 = reinterpret_cast<const double2*>(xb + kn * kProjTokens)[1];
-    double nq[NJB];
-#pragma unroll
-    for (uint32_t jb = 0; jb < NJB; ++jb) nq[jb] = qb[kn * kD + 16u * jb];
-    const double xv[4] = {x0.x, x0.y, x1.x, x1.y};
-#pragma unroll
-    for (uint32_t i = 0; i < 4; ++i)
-#pragma unroll
-      for (uint32_t jb = 0; jb < NJB; ++jb) acc[i][jb] = fma(qv[jb], xv[i], acc[i][jb]);
-    x0 = n0;
-    x1 = n1;
-#pragma unroll
-    for (uint32_t jb = 0; jb < NJB; ++jb) qv[jb] = nq[jb];
-  }
-  float yv[4][NJB];
-#pragma unroll
-  for (uint32_t i = 0; i < 4; ++i)
-#pragma unroll
-    for (uint32_t jb = 0; jb < NJB; ++jb) yv[i][jb] = __double2float_rn(acc[i][jb]);
-  const uint32_t nv = bl > 4u * tg ? min(4u, bl - 4u * tg) : 0u;  // this thread's valid tokens
-#pragma unroll
-  for (uint32_t jb = 0; jb < NJB; ++jb) {
-    float mn = __int_as_float(0x7f800000), mx = __int_as_float(0xff800000);
-#pragma unroll
-    for (uint32_t i = 0; i < 4; ++i) {
-      if (i < nv) {
-        const float v = yv[i][jb];
-        if (v < mn) mn = v;
-        if (v > mx) mx = v;
-      }
-    }
-    // lanes 0-15 hold tokens 8w .. 8w+3, lanes 16-31 the next four
-    const float pmn = __shfl_xor_sync(0xffffffffu, mn, 16), pmx = __shfl_xor_sync(0xffffffffu, mx, 16);
-    if (lane < 16u) {
-      if (pmn < mn) mn = pmn;
-      if (pmx > mx) mx = pmx;
-    } else {
-      mn = mn < pmn ? mn : pmn;
-      mx = mx > pmx ? mx : pmx;
-    }
-    const uint32_t cc = cg + 16u * jb;
-    if (lane < 16u && cc < nc) S.part[warp][cc] = make_float2(mn, mx);
-  }
-  __syncthreads();
-  // thread cc < nc: the block's minimum, maximum and scale of component cc
-  if (threadIdx.x < nc) {
-    const uint32_t cc = threadIdx.x;
-    float mn = __int_as_float(0x7f800000), mx = __int_as_float(0xff800000);
-#pragma unroll
-    for (uint32_t w = 0; w < kThreads / 32u; ++w) {
-      const float2 p = S.part[w][cc];
-      if (p.x < mn) mn = p.x;
-      if (p.y > mx) mx = p.y;
-    }
-    const uint32_t levels = (1u << S.ci.width[S.cidx[cc]]) - 1u;
-    const float s = (mx == mn) ? 0.0f : __fdiv_rn(__fsub_rn(mx, mn), float(levels));
-    const float rs = s == 0.0f ? 0.0f : __frcp_rn(s);
-    const uint32_t exact = !(rs < 0x1p126f) ? 1u : 0u;
-    uint32_t* zp = reinterpret_cast<uint32_t*>(rec + 8u * (cc * nb + tb / kTile));
-    zp[0] = __float_as_uint(mn);
-    zp[1] = __float_as_uint(s);
-    S.qp[cc] = make_float4(mn, s, rs, __uint_as_float(levels | (exact << 16)));
-  }
-  __syncthreads();
-#pragma unroll
-  for (uint32_t jb = 0; jb < NJB; ++jb) {
-    const uint32_t cc = cg + 16u * jb;
-    if (cc >= nc) continue;
-    const float4 qp = S.qp[cc];
-    const float mn = qp.x, s = qp.y, rs = qp.z;
-    const uint32_t levels = __float_as_uint(qp.w) & 0xffffu;
-    const bool exact = (__float_as_uint(qp.w) >> 16) != 0u;
-    const uint32_t j = S.cidx[cc];
-    uint32_t word = 0;
-#pragma unroll
-    for (uint32_t i = 0; i < 4; ++i) {
-      if (i < nv) {
-        bool nd;
-        uint32_t q = quantize_fast(yv[i][jb], mn, rs, levels, exact, nd);
-        if (nd) q = quantize(yv[i][jb], mn, s, levels);  // near a half-integer: the IEEE division decides
-        word |= q << (8u * i);
-        const uint32_t inc = 1u << (8u * (q & 3u));
-        if (q < 4u) cnt[jb][0] += inc;
-        else if (q < 8u) cnt[jb][1] += inc;
-        else atomicAdd(&S.hist[levels - 1u + q], 1u);  // tab_base(b) = 2^b - 2 = levels - 1
-      }
-    }
-    *reinterpret_cast<uint32_t*>(codes + uint64_t(j) * kCodesRow + tb + 4u * tg) = word;
-  }
+struct __align__(1024) PtSmem {
+  uint8_t a[4][kQDigPlane];    // x digits of the tile (A operand): byte p of X, p = 0 the top byte
+  uint8_t b[4][kQDigPlane];    // Q digits of the slice's coded columns (B operand)
+  float y[kD * kYStride];      // y[cc][t]: fl32(S~), the exact y where a chain ran
+  int32_t tok_e[kPTok];        // e_t, or kZeroTok
+  int32_t blk_e[2][2];         // per tile parity and block: largest e_t (kZeroTok: all tokens zero)
+  uint32_t blk_x1[2][2];       // largest x1 (bits of a non-negative float)
+  uint32_t zero_tok[2][4];     // per 32-token word: tokens whose x is all zero
+  uint32_t clist[kChainList];  // chains of the tile: token | coded component << 8
+  uint32_t n_chain;
+  uint32_t hist[kTabPool];     // symbol counts of the record per width stream
+  uint32_t ccnt[8][kD];        // counts of symbols 0..7 per coded component
+  uint32_t cidx[kD];           // coded component cc -> component j
+  int32_t col_f[kD];
+  float col_q1[kD];
+  CompInfo ci;
+  uint64_t bar;
+  uint32_t tmem_base;
+};
+static_assert(sizeof(PtSmem) + 1024 <= 232448, "projection shared memory exceeds the per-block limit");
+
+__device__ __forceinline__ double pow2d(int e) {  // 2^e, e clamped to the normal range
+  e = max(-1022, min(1023, e));
+  return __longlong_as_double(static_cast<long long>(1023 + e) << 52);
 }
 
-__global__ void __launch_bounds__(kThreads)
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }  // -126 <= e <= 127
+
+// The oracle's y of one token and component: xr the token's de-rotated x and
+// qr = Q[0..127][j] (a row of the transposed basis), both fp32 in shared memory
+// as 32 float4 chunks, chunk c stored at c ^ xs and c ^ qs: fp64 fused
+// multiply-adds over k ascending (each fp32 x fp32 product is exact in fp64, so
+// each step is the oracle's rounded addition), rounded to fp32 once.
+__device__ __forceinline__ float exact_y_inl(const float4* xr, uint32_t xs, const float4* qr, uint32_t qs) {
+  double acc = 0.0;
+  float4 xn = xr[xs], qn = qr[qs];
+#pragma unroll 4
+  for (uint32_t c = 0; c < 32; ++c) {
+    const float4 xv = xn, qv = qn;
+    if (c + 1u < 32u) {
+      xn = xr[(c + 1u) ^ xs];
+      qn = qr[(c + 1u) ^ qs];
+    }
+    acc = fma(double(qv.x), double(xv.x), acc);
+    acc = fma(double(qv.y), double(xv.y), acc);
+    acc = fma(double(qv.z), double(xv.z), acc);
+    acc = fma(double(qv.w), double(xv.w), acc);
+  }
+  return __double2float_rn(acc);
+}
+// the same as a call, for the rare paths
+__device__ __noinline__ float exact_y(const float4* xr, uint32_t xs, const float4* qr, uint32_t qs) {
+  return exact_y_inl(xr, xs, qr, qs);
+}
+
+// quantise with the reciprocal where it decides, else the IEEE division
+__device__ __forceinline__ uint32_t quantize_any(float y, float z, float s, float rs, uint32_t levels,
+                                                 bool exact_rs) {
+  bool nd;
+  const uint32_t q = quantize_fast(y, z, rs, levels, exact_rs, nd);
+  return nd ? quantize(y, z, s, levels) : q;
+}
+
+__global__ void __launch_bounds__(kPThreads, 1)
 k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLayout ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
-  ProjSmem& S = *reinterpret_cast<ProjSmem*>(smem_raw);
-  const uint32_t tid = threadIdx.x, nthr = blockDim.x;
-  const uint32_t warp = tid >> 5, lane = tid & 31u;
+  // the swizzled operand tiles need 1024-byte-aligned shared addresses
+  const uint32_t pad = (1024u - (tc::smem_addr(smem_raw) & 1023u)) & 1023u;
+  PtSmem& S = *reinterpret_cast<PtSmem*>(smem_raw + pad);
+  const uint32_t tid = threadIdx.x, warp = tid >> 5, lane = tid & 31u;
   const uint32_t rps = 1u + sh.n_mid;
-  const uint32_t gs = blockIdx.x / sh.n_mid, c = blockIdx.x % sh.n_mid;  // slice of the batch
-  const uint32_t r = gs * rps + 1u + c;                                   // record of the batch
-  const uint32_t fr = frame_of(b.rec_base, b.n, r);
-  const uint32_t ls = (r - b.rec_base[fr]) / rps;
-  const uint16_t* src = reinterpret_cast<const uint16_t*>(b.f[fr].src);
-  const uint32_t sidx = b.f[fr].first_slice + ls;
-  const bool is_key = ((sidx / sh.H) & 1u) == 0;
-  const uint32_t t0 = sh.s_end + c * sh.ct, tcc = min(sh.ct, sh.r_start - t0);
-  const uint32_t nb = (tcc + kTile - 1) / kTile;
-  const uint16_t* xs = src + uint64_t(ls) * sh.T * kD;
-  uint8_t* rec = ws.slots + uint64_t(r) * ws.slot_bytes;
-  uint8_t* codes = slot_codes(rec, ws.slot_bytes);
-
-  // the first tile's rows are requested first, so they land while the basis loads
-  XFetch xf;
-  xf.load(xs, pl.rope, is_key, t0, 0, min(kProjTokens, tcc));
-  load_comp_info(pl.comp + sidx, S.ci);
-  if (tid < kD && S.ci.width[tid]) S.cidx[S.ci.coded_idx[tid]] = tid;
-  for (uint32_t i = tid; i < kTabPool; i += nthr) S.hist[i] = 0;
-  for (uint32_t i = tid; i < 8u * kD; i += nthr) (&S.ccnt[0][0])[i] = 0;
-  __syncthreads();
-  const uint32_t nc = S.ci.n_coded;
-  {
-    const float* q = pl.bases + uint64_t(sidx) * kD * kD;
-    // warp per row k, lanes along the coded columns; a lane's four column
-    // indices are read once and four rows' loads are issued together
-    uint32_t col[4];
-#pragma unroll
-    for (uint32_t u = 0; u < 4; ++u) col[u] = lane + 32u * u < nc ? S.cidx[lane + 32u * u] : 0u;
-    // all of this thread's rows are requested before any is stored (one latency)
-    constexpr uint32_t kRows = kD / (kThreads / 32u);
-    float v[kRows][4];
-#pragma unroll
-    for (uint32_t kk = 0; kk < kRows; ++kk)
-#pragma unroll
-      for (uint32_t u = 0; u < 4; ++u) {
-        const uint32_t k = warp + kk * (kThreads / 32u);
-        v[kk][u] = lane + 32u * u < nc ? __ldg(q + k * kD + col[u]) : 0.0f;
-      }
-#pragma unroll
-    for (uint32_t kk = 0; kk < kRows; ++kk)
-#pragma unroll
-      for (uint32_t u = 0; u < 4; ++u) {
-        const uint32_t k = warp + kk * (kThreads / 32u);
-        if (lane + 32u * u < nc) S.Qd[k * kD + lane + 32u * u] = double(v[kk][u]);
-      }
+  const uint32_t n_mid_total = (b.rec_base[b.n] / rps) * sh.n_mid;
+  const uint32_t mbeg = uint32_t(uint64_t(blockIdx.x) * n_mid_total / gridDim.x);
+  const uint32_t mend = uint32_t(uint64_t(blockIdx.x + 1u) * n_mid_total / gridDim.x);
+  if (mbeg >= mend) return;
+  if (warp == 0) {
+    tc::tmem_alloc(&S.tmem_base, 512u);
+    tc::tmem_relinquish();
   }
-  // side-information padding of the record (its values are written below)
-  const uint32_t side = 8u * nc * nb;
-  if (tid < pad16(side) - side) rec[side + tid] = 0;
+  if (tid == 0) tc::mbar_init(&S.bar, 1);
+  tc::fence_before_sync();
   __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tmem = S.tmem_base;
+  uint32_t phase = 0;
+  bool alive = true, drained = true;
+  int32_t cur_slice = -1;
+  // per-word roles: block blk2 of the tile, coded component wc, half hf
+  const uint32_t blk2 = tid >> 8, wc = (tid >> 1) & 127u, hf = tid & 1u;
+  // digit roles: token dt, channel quarter dg
+  const uint32_t dt = tid >> 2, dg = tid & 3u;
 
-  // thread: tokens 4tg .. 4tg+3 and components cg + 16jb, jb < ceil(nc / 16)
-  const uint32_t tg = tid >> 4, cg = tid & 15u;
-  const uint32_t njb = (nc + 15u) >> 4;
-  uint32_t cnt[8][2];  // per jb: counts of symbols 0..3 and 4..7 of this thread's codes, a byte each
-#pragma unroll
-  for (uint32_t jb = 0; jb < 8; ++jb) cnt[jb][0] = cnt[jb][1] = 0;
-  for (uint32_t tb = 0; tb < tcc; tb += kProjTokens) {
-    const uint32_t bl = min(kProjTokens, tcc - tb);
-    xf.stage(S.x, is_key);
-    __syncthreads();
-    // the next tile's rows are fetched now and land during this one's projection
-    if (tb + kProjTokens < tcc) xf.load(xs, pl.rope, is_key, t0, tb + kProjTokens, min(kProjTokens, tcc - tb - kProjTokens));
-    switch (njb) {
-      case 1: project_quantize_tile<1>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
-      case 2: project_quantize_tile<2>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
-      case 3: project_quantize_tile<3>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
-      case 4: project_quantize_tile<4>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
-      case 5: project_quantize_tile<5>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
-      case 6: project_quantize_tile<6>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
-      case 7: project_quantize_tile<7>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
-      default: project_quantize_tile<8>(S, tg, cg, nc, bl, tb, nb, rec, codes, cnt); break;
+  for (uint32_t m = mbeg; m < mend && alive; ++m) {
+    const uint32_t gs = m / sh.n_mid, c = m % sh.n_mid;
+    const uint32_t r = gs * rps + 1u + c;
+    const uint32_t fr = frame_of(b.rec_base, b.n, r);
+    const uint32_t ls = (r - b.rec_base[fr]) / rps;
+    const uint16_t* src = reinterpret_cast<const uint16_t*>(b.f[fr].src);
+    const uint32_t sidx = b.f[fr].first_slice + ls;
+    const bool is_key = ((sidx / sh.H) & 1u) == 0;
+    const uint32_t t0 = sh.s_end + c * sh.ct, tcc = min(sh.ct, sh.r_start - t0);
+    const uint32_t nb = (tcc + kTile - 1) / kTile;
+    const uint16_t* xs = src + uint64_t(ls) * sh.T * kD;
+    uint8_t* rec = ws.slots + uint64_t(r) * ws.slot_bytes;
+    uint8_t* codes = slot_codes(rec, ws.slot_bytes);
+
+    if (int32_t(sidx) != cur_slice) {  // the slice's component order and Q digits
+      cur_slice = int32_t(sidx);
+      load_comp_info(pl.comp + sidx, S.ci);
+      if (tid < kD) {
+        if (S.ci.width[tid]) S.cidx[S.ci.coded_idx[tid]] = tid;
+        S.col_f[tid] = pl.qcol[sidx].f[tid];
+        S.col_q1[tid] = pl.qcol[sidx].q1[tid];
+      }
     }
-    __syncthreads();  // x and the warp partials are rewritten by the next tile
-  }
+    for (uint32_t i = tid; i < kTabPool; i += kPThreads) S.hist[i] = 0;
+    for (uint32_t i = tid; i < 8u * kD; i += kPThreads) (&S.ccnt[0][0])[i] = 0;
+    if (tid < 4u) {
+      S.blk_e[tid >> 1][tid & 1u] = kZeroTok;
+      S.blk_x1[tid >> 1][tid & 1u] = 0u;
+    }
+    if (tid < 8u) S.zero_tok[tid >> 2][tid & 3u] = 0u;
+    if (tid == 0) S.n_chain = 0;
+    const uint32_t nc = S.ci.n_coded;
+    const uint32_t N = max(16u, (nc + 15u) & ~15u);
+    {  // side-information padding of the record (its values are written below)
+      const uint32_t side = 8u * nc * nb;
+      if (tid < pad16(side) - side) rec[side + tid] = 0;
+    }
+    __syncthreads();
+    const bool wlive = wc < nc;
+    const uint32_t wj = wlive ? S.cidx[wc] : 0u;
+    const uint32_t levels = (1u << S.ci.width[wj]) - 1u;
+    uint32_t cnt[2] = {0u, 0u};  // counts of symbols 0..3 and 4..7 of this thread's codes, a byte each
+
+    for (uint32_t tb = 0; tb < tcc && alive; tb += kPTok) {
+      const uint32_t bl = min(kPTok, tcc - tb);
+      const uint32_t par = (tb / kPTok) & 1u;
+      if (tid < 2u) {  // the next tile's block statistics start empty
+        S.blk_e[par ^ 1u][tid] = kZeroTok;
+        S.blk_x1[par ^ 1u][tid] = 0u;
+      } else if (tid < 6u) {
+        S.zero_tok[par ^ 1u][tid - 2u] = 0u;
+      }
+      {  // the slice's Q digits (their space holds Q itself during the previous tile's chains)
+        const char* g = reinterpret_cast<const char*>(pl.qdig + uint64_t(sidx) * kQDigBytes);
+        const uint32_t d0 = tc::smem_addr(&S.b[0][0]);
 #pragma unroll
-  for (uint32_t jb = 0; jb < 8; ++jb) {
-    const uint32_t cc = cg + 16u * jb;
-    if (jb < njb && cc < nc) {
+        for (uint32_t u = 0; u < kQDigBytes / 16u / kPThreads; ++u) {
+          const uint32_t i = tid + u * kPThreads;
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d0 + 16u * i), "l"(g + 16u * i) : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+      }
+      // ---- digits of token dt, channels 16 dg .. + 15 and their partners
+      float xa[16], xb[16];  // de-rotated x, kept for the chains (stored once the MMAs are done)
+      {
+        if (dt < bl) {
+          const uint4* row = reinterpret_cast<const uint4*>(xs + uint64_t(t0 + tb + dt) * kD);
+          const uint4 v[4] = {__ldg(row + 2u * dg), __ldg(row + 2u * dg + 1u), __ldg(row + 8u + 2u * dg),
+                              __ldg(row + 8u + 2u * dg + 1u)};
+#pragma unroll
+          for (uint32_t h = 0; h < 2; ++h) {
+            const uint32_t w[4] = {v[h].x, v[h].y, v[h].z, v[h].w}, u[4] = {v[2 + h].x, v[2 + h].y, v[2 + h].z, v[2 + h].w};
+#pragma unroll
+            for (uint32_t i = 0; i < 4; ++i) {
+              xa[8 * h + 2 * i] = bf16_to_f32(w[i] & 0xffffu);
+              xa[8 * h + 2 * i + 1] = bf16_to_f32(w[i] >> 16);
+              xb[8 * h + 2 * i] = bf16_to_f32(u[i] & 0xffffu);
+              xb[8 * h + 2 * i + 1] = bf16_to_f32(u[i] >> 16);
+            }
+          }
+          if (is_key) {
+            const float4* c4 = reinterpret_cast<const float4*>(pl.rope + (uint64_t(t0 + tb + dt) * (kD / 2) + 16u * dg) * 2u);
+#pragma unroll
+            for (uint32_t i = 0; i < 8; ++i) {
+              const float4 k = __ldg(c4 + i);  // (cos, sin) of pairs 16 dg + 2i, + 2i + 1
+              const float a0 = xa[2 * i], a1 = xa[2 * i + 1], b0 = xb[2 * i], b1 = xb[2 * i + 1];
+              xa[2 * i] = __fadd_rn(__fmul_rn(a0, k.x), __fmul_rn(b0, k.y));
+              xb[2 * i] = __fsub_rn(__fmul_rn(b0, k.x), __fmul_rn(a0, k.y));
+              xa[2 * i + 1] = __fadd_rn(__fmul_rn(a1, k.z), __fmul_rn(b1, k.w));
+              xb[2 * i + 1] = __fsub_rn(__fmul_rn(b1, k.z), __fmul_rn(a1, k.w));
+            }
+          }
+        } else {
+#pragma unroll
+          for (uint32_t i = 0; i < 16; ++i) xa[i] = xb[i] = 0.0f;
+        }
+        float mx = 0.0f, x1 = 0.0f;
+#pragma unroll
+        for (uint32_t i = 0; i < 16; ++i) {
+          mx = fmaxf(mx, fmaxf(fabsf(xa[i]), fabsf(xb[i])));
+          x1 = __fadd_ru(x1, __fadd_ru(fabsf(xa[i]), fabsf(xb[i])));
+        }
+#pragma unroll
+        for (uint32_t o = 1; o < 4; o <<= 1) {
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+          x1 = __fadd_ru(x1, __shfl_xor_sync(0xffffffffu, x1, o));
+        }
+        const int32_t e = mx > 0.0f ? ilogbf(mx) : kZeroTok;
+        int32_t X[32];
+        if (e == kZeroTok || e >= -98) {  // 2^(29 - e) is an fp32 number: x * 2^(29 - e) is exact
+          const float sc = e == kZeroTok ? 0.0f : pow2f(29 - e);
+#pragma unroll
+          for (uint32_t i = 0; i < 16; ++i) {
+            X[i] = __float2int_rn(__fmul_rn(xa[i], sc));
+            X[16 + i] = __float2int_rn(__fmul_rn(xb[i], sc));
+          }
+        } else {  // tiny tokens
+          const double sc = pow2d(29 - e);
+#pragma unroll
+          for (uint32_t i = 0; i < 16; ++i) {
+            X[i] = __double2int_rn(double(xa[i]) * sc);
+            X[16 + i] = __double2int_rn(double(xb[i]) * sc);
+          }
+        }
+#pragma unroll
+        for (uint32_t p = 0; p < 4; ++p) {
+          const uint32_t sel = (3u - p) | ((7u - p) << 4);  // byte 3 - p of two words
+#pragma unroll
+          for (uint32_t h = 0; h < 2; ++h) {
+            uint32_t wv[4];
+#pragma unroll
+            for (uint32_t q = 0; q < 4; ++q) {
+              const int32_t* x4 = X + 16 * h + 4 * q;
+              wv[q] = __byte_perm(__byte_perm(x4[0], x4[1], sel), __byte_perm(x4[2], x4[3], sel), 0x5410);
+            }
+            *reinterpret_cast<uint4*>(&S.a[p][0] + tc::sw128_offset(dt, 16u * (dg + 4u * h), kPTok)) =
+                make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          }
+        }
+        if (dg == 0) {
+          S.tok_e[dt] = e;
+          if (dt < bl) {
+            if (e == kZeroTok) atomicOr(&S.zero_tok[par][dt >> 5], 1u << (dt & 31u));
+            else {
+              atomicMax(&S.blk_e[par][dt >> 6], e);
+              atomicMax(&S.blk_x1[par][dt >> 6], __float_as_uint(x1));
+            }
+          }
+        }
+      }
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      tc::fence_async_smem();
+      tc::fence_before_sync();
+      __syncthreads();
+      // ---- ten digit pairs x four K-steps on the tensor cores
+      if (tid == 0) {
+        tc::fence_after_sync();
+        const uint32_t a0 = tc::smem_addr(&S.a[0][0]), b0 = tc::smem_addr(&S.b[0][0]);
+#pragma unroll 1
+        for (uint32_t ks = 0; ks < 4; ++ks) {
+#pragma unroll
+          for (uint32_t w = 0; w < 4; ++w) {
+#pragma unroll
+            for (uint32_t pa = 0; pa <= w; ++pa) {
+              const uint32_t pb = w - pa;
+              const uint64_t da = tc::desc_sw128(a0 + pa * kQDigPlane + ks * 32u);
+              const uint64_t db = tc::desc_sw128(b0 + pb * kQDigPlane + ks * 32u);
+              tc::mma_i8(tmem + w * N, da, db, tc::idesc_i8_s32(kPTok, N, pa == 0, pb == 0),
+                         (ks > 0 || pa > 0) ? 1u : 0u);
+            }
+          }
+        }
+        tc::mma_commit(&S.bar);
+      }
+      {  // while the MMAs run: the next 128 tokens' rows (and keys' cos/sin) toward L2
+        const uint32_t tn = t0 + tb + kPTok + dt;
+        if (tn < sh.r_start) {
+          const char* pr = dg < 2u ? reinterpret_cast<const char*>(xs + uint64_t(tn) * kD) + 128u * dg
+                                   : reinterpret_cast<const char*>(pl.rope + uint64_t(tn) * kD) + 256u * (dg - 2u);
+          if (dg < 2u || is_key) {
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(pr));
+            if (dg >= 2u) asm volatile("prefetch.global.L2 [%0];" ::"l"(pr + 128));
+          }
+        }
+      }
+      const bool done = tc::mbar_wait(&S.bar, phase, KVC_MMA_WAIT_POLLS);
+      phase ^= 1u;
+      if (!__syncthreads_and(done)) {
+        // drain: the same completion again, with the long bound, so that the
+        // accumulator is no longer written when the block frees it
+        drained = __syncthreads_and(tc::mbar_wait(&S.bar, phase ^ 1u, kMmaDrainPolls));
+        alive = false;
+        break;
+      }
+      tc::fence_after_sync();
+      {  // the Q digits are consumed: their space holds the coded rows of Q^T for the chains
+        const char* g = reinterpret_cast<const char*>(pl.qt + uint64_t(sidx) * kD * kD);
+        const uint32_t d0 = tc::smem_addr(&S.b[0][0]);
+        for (uint32_t i = tid; i < nc * 32u; i += kPThreads) {
+          const uint32_t cc = i >> 5, ch = i & 31u;
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d0 + 512u * cc + 16u * (ch ^ (cc & 7u))),
+                       "l"(g + 512u * S.cidx[cc] + 16u * ch) : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+      }
+      {  // the x digits are consumed: their space holds x as fp32 rows for the chains
+        float4* xp = reinterpret_cast<float4*>(&S.a[0][0]) + dt * 32u;
+        const uint32_t sw = dt & 7u;
+#pragma unroll
+        for (uint32_t i = 0; i < 4; ++i) {
+          xp[(4u * dg + i) ^ sw] = make_float4(xa[4 * i], xa[4 * i + 1], xa[4 * i + 2], xa[4 * i + 3]);
+          xp[(16u + 4u * dg + i) ^ sw] = make_float4(xb[4 * i], xb[4 * i + 1], xb[4 * i + 2], xb[4 * i + 3]);
+        }
+      }
+      // ---- epilogue: the estimates y~ = fl32(S~)
+      {
+        const uint32_t g4 = warp & 3u, tt = 32u * g4 + lane;
+        const int32_t et = S.tok_e[tt];
+        const bool tv = tt < bl;
+        for (uint32_t cch = warp >> 2; cch < N / 16u; cch += 4u) {
+          uint32_t p[4][16];
+#pragma unroll
+          for (uint32_t w = 0; w < 4; ++w) tc::tmem_ld16(tmem + ((32u * g4) << 16) + w * N + 16u * cch, p[w]);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (uint32_t i = 0; i < 16; ++i) {
+            const uint32_t cc = 16u * cch + i;
+            if (tv && cc < nc) {
+              // the levels in fp32 (exact below 2^24: |P0| <= 2^19, |P1| < 2^22, |P2|
+              // < 2^24; |P3| < 2^25 rounds by at most 1), combined with fused
+              // multiply-adds: within 2^-22 |V~| + 2^11 of V
+              const float f0 = __int2float_rn(int32_t(p[0][i])), f1 = __int2float_rn(int32_t(p[1][i]));
+              const float f2 = __int2float_rn(int32_t(p[2][i])), f3 = __int2float_rn(int32_t(p[3][i]));
+              const float v = __fmaf_rn(__fmaf_rn(__fmaf_rn(f0, 256.0f, f1), 256.0f, f2), 256.0f, f3);
+              float yv = 0.0f;
+              if (et != kZeroTok) {
+                const int k = et + S.col_f[cc] - 34;
+                yv = k >= -126 ? __fmul_rn(v, pow2f(min(k, 127))) : __fmul_rn(__fmul_rn(v, pow2f(k + 64)), 0x1p-64f);
+              }
+              S.y[cc * kYStride + tt] = yv;
+            }
+          }
+        }
+      }
+      tc::fence_before_sync();
+      __syncthreads();
+      // ---- per word: bound, candidates, chains, zero point and scale, codes
+      {
+        const uint32_t w0 = blk2 * 64u + hf * 32u;  // first token of the word in the tile
+        const uint32_t nv = bl > w0 ? min(32u, bl - w0) : 0u;
+        const bool live = wlive && blk2 * 64u < bl;
+        float* yr = S.y + wc * kYStride + w0;
+        const int32_t em = S.blk_e[par][blk2];
+        const float xm = __uint_as_float(S.blk_x1[par][blk2]);
+        const uint32_t zmask = S.zero_tok[par][blk2 * 2u + hf];
+        float mn = __int_as_float(0x7f800000), mx = __int_as_float(0xff800000);
+        for (uint32_t i = 0; i < nv; ++i) {
+          const float v = yr[i];
+          mn = fminf(mn, v);
+          mx = fmaxf(mx, v);
+        }
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        const int32_t f = S.col_f[wc];
+        const bool all_exact = em == kZeroTok || f == kQColZero;
+        float R = 0.0f;
+        uint32_t exact = zmask, cand = 0;
+        const uint32_t vmask = nv == 32u ? 0xffffffffu : (1u << nv) - 1u;
+        if (live) {
+          if (all_exact) {
+            exact = vmask;
+          } else {
+            double E = pow2d(em + f - 58) * kDropUnits + double(xm) * (pow2d(f - 30) + pow2d(f - 45)) +
+                       double(S.col_q1[wc]) * pow2d(em - 30);
+            // the estimates are within dl of S~ (fp32 combination of the levels)
+            const double Ma = double(fmaxf(fabsf(mn), fabsf(mx)));
+            const double dl = Ma * 0x1p-21 + pow2d(em + f - 22) + 0x1p-148;
+            E *= 1.0 + 0x1p-40;
+            const double M = Ma * (1.0 + 0x1p-21) + E + dl;
+            const int lm = M > 0.0 ? ilogb(M) : -1000;
+            R = __double2float_ru((E + dl + pow2d(max(lm - 23, -149))) * (1.0 + 0x1p-40));
+            const float two = __fmul_ru(R, 2.0f);
+            const float lo_thr = __fadd_ru(mn, two), hi_thr = __fsub_rd(mx, two);
+            for (uint32_t i = 0; i < nv; ++i) {
+              const float v = yr[i];
+              if (v <= lo_thr || v >= hi_thr) cand |= 1u << i;
+            }
+            cand &= ~zmask;
+          }
+        }
+        const float4* xp = reinterpret_cast<const float4*>(&S.a[0][0]) + w0 * 32u;
+        const float4* qr = reinterpret_cast<const float4*>(&S.b[0][0]) + wc * 32u;
+        {  // the candidates go to the tile's list; what does not fit stays with the word.
+           // Every slot below min(n_chain, kChainList) is written by the thread that
+           // reserved it, so the list holds no stale entry.
+          const uint32_t n = __popc(cand);
+          if (n) {
+            const uint32_t base = atomicAdd(&S.n_chain, n);
+            const uint32_t fit = base < kChainList ? min(n, kChainList - base) : 0u;
+            for (uint32_t u = 0; u < fit; ++u) {
+              const uint32_t i = __ffs(cand) - 1u;
+              cand &= cand - 1u;
+              S.clist[base + u] = (w0 + i) | (wc << 8);
+              exact |= 1u << i;
+            }
+          }
+        }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");  // Q^T rows landed
+        __syncthreads();
+        {  // the listed chains, spread over all threads
+          const uint32_t nl = min(S.n_chain, kChainList);
+          for (uint32_t u = tid; u < nl; u += kPThreads) {
+            const uint32_t e = S.clist[u], t = e & 0xffu, cc = e >> 8;
+            S.y[cc * kYStride + t] = exact_y_inl(reinterpret_cast<const float4*>(&S.a[0][0]) + t * 32u, t & 7u,
+                                                 reinterpret_cast<const float4*>(&S.b[0][0]) + cc * 32u, cc & 7u);
+          }
+        }
+        __syncthreads();
+        if (tid == 0) S.n_chain = 0;  // for the next tile (read again only after two barriers)
+        while (cand) {  // chains that did not fit the list
+          const uint32_t i = __ffs(cand) - 1u;
+          cand &= cand - 1u;
+          yr[i] = exact_y(xp + i * 32u, (w0 + i) & 7u, qr, wc & 7u);
+          exact |= 1u << i;
+        }
+        // the oracle's scan over the block: exact values where they decide
+        float z = __int_as_float(0x7f800000), zx = __int_as_float(0xff800000);
+        for (uint32_t i = 0; i < nv; ++i) {
+          const float v = yr[i];
+          if (v < z) z = v;
+          if (v > zx) zx = v;
+        }
+        {  // lower half first: the upper half's value wins only when strictly beyond
+          const float pz = __shfl_xor_sync(0xffffffffu, z, 1), pzx = __shfl_xor_sync(0xffffffffu, zx, 1);
+          if (hf == 0) {
+            if (pz < z) z = pz;
+            if (pzx > zx) zx = pzx;
+          } else {
+            z = z < pz ? z : pz;
+            zx = zx > pzx ? zx : pzx;
+          }
+        }
+        if (live) {
+          const float s = (zx == z) ? 0.0f : __fdiv_rn(__fsub_rn(zx, z), float(levels));
+          const float rs = s == 0.0f ? 0.0f : __frcp_rn(s);
+          const bool exact_rs = !(rs < 0x1p126f);
+          if (hf == 0) {
+            uint32_t* zp = reinterpret_cast<uint32_t*>(rec + 8u * (wc * nb + tb / kTile + blk2));
+            zp[0] = __float_as_uint(z);
+            zp[1] = __float_as_uint(s);
+          }
+          // With qa = RN(RN(y~ - z) * RN(1/s)), the oracle's quotient for any y in
+          // [y~ - R, y~ + R] is within R/s (1 + 2^-21) + |qa| 2^-21 of qa; decisions
+          // change only at half-integers, so a larger distance settles the code.
+          const float mR = exact_rs ? __int_as_float(0x7f800000) : __fmul_ru(__fmul_ru(R, rs), 1.0f + 0x1p-19f);
+          uint32_t word[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+          for (uint32_t i = 0; i < nv; ++i) {
+            const float v = yr[i];
+            uint32_t q;
+            if ((exact >> i) & 1u) {
+              q = quantize_any(v, z, s, rs, levels, exact_rs);
+            } else {
+              const float qa = __fmul_rn(__fsub_rn(v, z), rs);
+              // rint by the magic constant (|qa| is small here): iq the integer, rq as fp32
+              const float mg = __fadd_rn(qa, 12582912.0f);
+              const int32_t iq = __float_as_int(mg) - 0x4b400000;
+              const float d = __fsub_rn(0.5f, fabsf(__fsub_rn(qa, __fsub_rn(mg, 12582912.0f))));  // to the nearest half-integer
+              if (d > __fadd_ru(mR, __fmul_ru(fabsf(qa), 0x1p-19f))) {
+                q = uint32_t(min(max(iq, 0), int32_t(levels)));
+              } else {
+                const uint32_t q1 = quantize_any(__fsub_rd(v, R), z, s, rs, levels, exact_rs);
+                const uint32_t q2 = quantize_any(__fadd_ru(v, R), z, s, rs, levels, exact_rs);
+                q = q1 == q2 ? q1 : quantize_any(exact_y(xp + i * 32u, (w0 + i) & 7u, qr, wc & 7u), z, s, rs, levels, exact_rs);
+              }
+            }
+            word[i >> 2] |= q << (8u * (i & 3u));
+            if (q < 8u) cnt[q >> 2] += 1u << (8u * (q & 3u));
+            else atomicAdd(&S.hist[levels - 1u + q], 1u);  // tab_base(b) = 2^b - 2 = levels - 1
+          }
+          uint4* cd = reinterpret_cast<uint4*>(codes + uint64_t(wj) * kCodesRow + tb + w0);
+          cd[0] = make_uint4(word[0], word[1], word[2], word[3]);
+          cd[1] = make_uint4(word[4], word[5], word[6], word[7]);
+        }
+      }
+      __syncthreads();  // y and the token arrays are rewritten by the next tile
+    }
+    if (!alive) break;
+    if (wlive) {
 #pragma unroll
       for (uint32_t q = 0; q < 8; ++q) {
-        const uint32_t c = (cnt[jb][q >> 2] >> (8u * (q & 3u))) & 0xffu;
-        if (c) atomicAdd(&S.ccnt[q][cc], c);
+        const uint32_t n = (cnt[q >> 2] >> (8u * (q & 3u))) & 0xffu;
+        if (n) atomicAdd(&S.ccnt[q][wc], n);
       }
     }
+    __syncthreads();
+    // counts of symbols 0..7 summed over the components of each width
+    if (tid < 64u) {
+      const uint32_t bw = (tid >> 3) + 1u, q = tid & 7u;
+      if (q < (1u << bw)) {
+        uint32_t sum = 0;
+        for (uint32_t cc = 0; cc < nc; ++cc)
+          if (S.ci.width[S.cidx[cc]] == bw) sum += S.ccnt[q][cc];
+        S.hist[tab_base(bw) + q] += sum;
+      }
+    }
+    __syncthreads();
+    for (uint32_t i = tid; i < kTabPool; i += kPThreads)
+      reinterpret_cast<uint32_t*>(codes + kHistOffset)[i] = S.hist[i];
   }
-  __syncthreads();
-  // counts of symbols 0..7 summed over the components of each width
-  if (tid < 64u) {
-    const uint32_t bw = (tid >> 3) + 1u, q = tid & 7u;
-    if (q < (1u << bw)) {
-      uint32_t sum = 0;
-      for (uint32_t cc = 0; cc < nc; ++cc)
-        if (S.ci.width[S.cidx[cc]] == bw) sum += S.ccnt[q][cc];
-      S.hist[tab_base(bw) + q] += sum;
+  if (!alive) {  // this block's records from the one that timed out on are marked failed
+    for (uint32_t m = mbeg; m < mend; ++m) {
+      const uint32_t r = (m / sh.n_mid) * rps + 1u + m % sh.n_mid;
+      uint8_t* codes = slot_codes(ws.slots + uint64_t(r) * ws.slot_bytes, ws.slot_bytes);
+      if (tid == 0) reinterpret_cast<uint32_t*>(codes + kHistOffset)[kTabPool - 1u] = kHistTimeout;
     }
   }
+  tc::fence_before_sync();
   __syncthreads();
-  for (uint32_t i = tid; i < kTabPool; i += nthr)
-    reinterpret_cast<uint32_t*>(codes + kHistOffset)[i] = S.hist[i];
+  // MMAs still pending after the drain's bound would write tensor memory
+  // after it is freed (and handed to another block): the block then keeps its
+  // allocation, and its records already carry the timeout status
+  if (warp == 0 && drained) {
+    tc::fence_after_sync();
+    tc::tmem_dealloc(tmem, 512u);
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -755,6 +1010,13 @@ k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
   for (uint32_t i = tid; i < kTabPool; i += nthr)
     S.hist[i] = __ldcg(reinterpret_cast<const uint32_t*>(codes_g + kHistOffset) + i);
   __syncthreads();
+  if (S.hist[kTabPool - 1u] == kHistTimeout) {  // the projection gave up on this record
+    if (tid == 0) {
+      ws.rec_len[r] = kRecLenError | uint32_t(kErrTimeout);
+      ws.rec_crc[r] = 0;
+    }
+    return;
+  }
 
   const Split split(tcc);
   // ---- per-stream tables from the counts: warp w takes width b = w + 1
@@ -1380,7 +1642,6 @@ struct __align__(1024) DecSmem {
 };
 
 static_assert(sizeof(DecSmem) + 1024 <= 232448, "decoder shared memory exceeds the per-block limit");
-static_assert(sizeof(ProjSmem) <= 232448, "projection shared memory exceeds the per-block limit");
 static_assert(sizeof(EntSmem) + 1024 <= 233472 / 5, "entropy kernel should fit five blocks per SM");
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -1641,8 +1902,8 @@ cudaError_t launch_transform_encode(const TransformShape& s, const TransformPlan
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || s.n_mid == 0) return e;
   const uint32_t grid = n_slices * s.n_mid;
-  e = cudaFuncSetAttribute(k_transform_project, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           int(sizeof(ProjSmem)));
+  const size_t psmem = sizeof(PtSmem) + 1024;
+  e = cudaFuncSetAttribute(k_transform_project, cudaFuncAttributeMaxDynamicSharedMemorySize, int(psmem));
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(k_transform_entropy, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            int(sizeof(EntSmem)));
@@ -1651,7 +1912,7 @@ cudaError_t launch_transform_encode(const TransformShape& s, const TransformPlan
   if (e != cudaSuccess) return e;
   {
     ProfRange pr_("transform_project", st);
-    k_transform_project<<<grid, kThreads, sizeof(ProjSmem), st>>>(s, p, b, ws);
+    k_transform_project<<<min(grid, uint32_t(num_sms())), kPThreads, psmem, st>>>(s, p, b, ws);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
