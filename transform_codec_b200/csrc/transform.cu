@@ -51,23 +51,6 @@ __device__ inline uint32_t quantize(float y, float z, float s, uint32_t levels) 
   return uint32_t(r);
 }
 
-// quantize() without the division where it cannot matter. With r = RN(1/s),
-// qa = RN((y - z) * r) is within 2^-22 * qa of the correctly rounded quotient
-// RN((y - z) / s) (two roundings of relative size 2^-24 against one). Every
-// decision quantize() takes on the quotient (rounding to an integer, the
-// clamps at 0 and at levels) changes only at half-integers, so when qa is
-// farther than qa * 2^-19 from the nearest half-integer both give the same
-// code. `need` flags the values inside that window, and every value of a
-// block whose reciprocal is not finite: for those the caller uses quantize().
-// A zero scale has r = 0 and gives code 0, as quantize() does.
-__device__ inline uint32_t quantize_fast(float y, float z, float r, uint32_t levels, bool exact, bool& need) {
-  const float q = __fmul_rn(__fsub_rn(y, z), r);
-  const float fl = floorf(q);
-  const float d = fabsf(__fsub_rn(__fsub_rn(q, fl), 0.5f));  // distance to floor(q) + 0.5
-  need = exact || d <= __fmul_rn(q, 0x1p-19f);
-  return min(__float2uint_rz(rintf(q)), levels);  // negative values convert to 0
-}
-
 // The plan's per-slice component order, copied into shared memory.
 __device__ inline void load_comp_info(const CompInfo* src, CompInfo& dst) {
   const uint4* s4 = reinterpret_cast<const uint4*>(src);
@@ -214,14 +197,6 @@ __device__ __noinline__ float exact_y(const float4* xr, uint32_t xs, const float
   return exact_y_inl(xr, xs, qr, qs);
 }
 
-// quantise with the reciprocal where it decides, else the IEEE division
-__device__ __forceinline__ uint32_t quantize_any(float y, float z, float s, float rs, uint32_t levels,
-                                                 bool exact_rs) {
-  bool nd;
-  const uint32_t q = quantize_fast(y, z, rs, levels, exact_rs, nd);
-  return nd ? quantize(y, z, s, levels) : q;
-}
-
 __global__ void __launch_bounds__(kPThreads, 1)
 k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLayout ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -292,7 +267,7 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
     const bool wlive = wc < nc;
     const uint32_t wj = wlive ? S.cidx[wc] : 0u;
     const uint32_t levels = (1u << S.ci.width[wj]) - 1u;
-    uint32_t cnt[2] = {0u, 0u};  // counts of symbols 0..3 and 4..7 of this thread's codes, a byte each
+    uint32_t cnt0 = 0u, cnt1 = 0u;  // counts of symbols 0..3 and 4..7 of this thread's codes, a byte each
 
     for (uint32_t tb = 0; tb < tcc && alive; tb += kPTok) {
       const uint32_t bl = min(kPTok, tcc - tb);
@@ -479,11 +454,14 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
           for (uint32_t i = 0; i < 16; ++i) {
             const uint32_t cc = 16u * cch + i;
             if (tv && cc < nc) {
-              // the levels in fp32 (exact below 2^24: |P0| <= 2^19, |P1| < 2^22, |P2|
-              // < 2^24; |P3| < 2^25 rounds by at most 1), combined with fused
-              // multiply-adds: within 2^-22 |V~| + 2^11 of V
-              const float f0 = __int2float_rn(int32_t(p[0][i])), f1 = __int2float_rn(int32_t(p[1][i]));
-              const float f2 = __int2float_rn(int32_t(p[2][i])), f3 = __int2float_rn(int32_t(p[3][i]));
+              // integers to fp32 by the magic constant 1.5 * 2^23 (exact below 2^22 in
+              // magnitude: |P0| <= 2^19, |P1| < 2^22); P2 and P3 (below 2^24 and 2^25)
+              // rounded down to multiples of 4 and 8 first; the levels combined with
+              // fused multiply-adds: within 2^-22 |V~| + 2^11 of V
+              const float f0 = __int_as_float(0x4b400000 + int32_t(p[0][i])) - 12582912.0f;
+              const float f1 = __int_as_float(0x4b400000 + int32_t(p[1][i])) - 12582912.0f;
+              const float f2 = (__int_as_float(0x4b400000 + (int32_t(p[2][i]) >> 2)) - 12582912.0f) * 4.0f;
+              const float f3 = (__int_as_float(0x4b400000 + (int32_t(p[3][i]) >> 3)) - 12582912.0f) * 8.0f;
               const float v = __fmaf_rn(__fmaf_rn(__fmaf_rn(f0, 256.0f, f1), 256.0f, f2), 256.0f, f3);
               float yv = 0.0f;
               if (et != kZeroTok) {
@@ -602,33 +580,64 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
             zp[0] = __float_as_uint(z);
             zp[1] = __float_as_uint(s);
           }
-          // With qa = RN(RN(y~ - z) * RN(1/s)), the oracle's quotient for any y in
-          // [y~ - R, y~ + R] is within R/s (1 + 2^-21) + |qa| 2^-21 of qa; decisions
-          // change only at half-integers, so a larger distance settles the code.
-          const float mR = exact_rs ? __int_as_float(0x7f800000) : __fmul_ru(__fmul_ru(R, rs), 1.0f + 0x1p-19f);
+          // Codes. With qa = RN(RN(y~ - z) * RN(1/s)), the oracle's quotient for any y
+          // in [y~ - R, y~ + R] is within R/s (1 + 2^-21) + |qa| 2^-21 of qa (R = 0
+          // where y~ is exact); decisions change only at half-integers, so a larger
+          // distance to the nearest one settles the code (rint by the magic
+          // constant 1.5 * 2^23: |qa| is small). The rest is settled after the pass.
+          const float mR = __fmul_ru(__fmul_ru(R, rs), 1.0f + 0x1p-19f);
+          // symbols 0..7 in the packed counters, the rest (widths >= 4) by atomics
+          auto count_code = [&](uint32_t q, int32_t sign = 1) {
+            const uint32_t inc = uint32_t(sign) << (8u * (q & 3u));
+            if (q < 4u) cnt0 += inc;
+            else if (q < 8u) cnt1 += inc;
+            else atomicAdd(&S.hist[levels - 1u + q], uint32_t(sign));  // tab_base(b) = 2^b - 2 = levels - 1
+          };
           uint32_t word[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-          for (uint32_t i = 0; i < nv; ++i) {
+          uint32_t unc = 0;
+#pragma unroll
+          for (uint32_t i = 0; i < 32; ++i) {
+            const float v = yr[i];
+            const float qa = __fmul_rn(__fsub_rn(v, z), rs);
+            const float mg = __fadd_rn(qa, 12582912.0f);
+            const int32_t iq = __float_as_int(mg) - 0x4b400000;
+            const float d = __fsub_rn(0.5f, fabsf(__fsub_rn(qa, __fsub_rn(mg, 12582912.0f))));
+            const float m = __fadd_ru(((exact >> i) & 1u) ? 0.0f : mR, __fmul_ru(fabsf(qa), 0x1p-19f));
+            const uint32_t q = uint32_t(min(max(iq, 0), int32_t(levels)));
+            word[i >> 2] |= q << (8u * (i & 3u));
+            if (!(d > m)) unc |= 1u << i;
+            if (i < nv) count_code(q);
+          }
+          unc = exact_rs ? vmask : (unc & vmask);
+          while (unc) {  // the IEEE quotient at both ends, else the chain decides
+            const uint32_t i = __ffs(unc) - 1u;
+            unc &= unc - 1u;
             const float v = yr[i];
             uint32_t q;
             if ((exact >> i) & 1u) {
-              q = quantize_any(v, z, s, rs, levels, exact_rs);
+              q = quantize(v, z, s, levels);
             } else {
-              const float qa = __fmul_rn(__fsub_rn(v, z), rs);
-              // rint by the magic constant (|qa| is small here): iq the integer, rq as fp32
-              const float mg = __fadd_rn(qa, 12582912.0f);
-              const int32_t iq = __float_as_int(mg) - 0x4b400000;
-              const float d = __fsub_rn(0.5f, fabsf(__fsub_rn(qa, __fsub_rn(mg, 12582912.0f))));  // to the nearest half-integer
-              if (d > __fadd_ru(mR, __fmul_ru(fabsf(qa), 0x1p-19f))) {
-                q = uint32_t(min(max(iq, 0), int32_t(levels)));
-              } else {
-                const uint32_t q1 = quantize_any(__fsub_rd(v, R), z, s, rs, levels, exact_rs);
-                const uint32_t q2 = quantize_any(__fadd_ru(v, R), z, s, rs, levels, exact_rs);
-                q = q1 == q2 ? q1 : quantize_any(exact_y(xp + i * 32u, (w0 + i) & 7u, qr, wc & 7u), z, s, rs, levels, exact_rs);
+              const uint32_t q1 = quantize(__fsub_rd(v, R), z, s, levels);
+              const uint32_t q2 = quantize(__fadd_ru(v, R), z, s, levels);
+              q = q1 == q2 ? q1 : quantize(exact_y(xp + i * 32u, (w0 + i) & 7u, qr, wc & 7u), z, s, levels);
+            }
+            const uint32_t sh = 8u * (i & 3u);
+#pragma unroll
+            for (uint32_t j = 0; j < 8; ++j) {
+              if (j == (i >> 2)) {
+                const uint32_t old = (word[j] >> sh) & 0xffu;
+                if (old != q) {
+                  count_code(old, -1);
+                  count_code(q);
+                }
+                word[j] = (word[j] & ~(0xffu << sh)) | (q << sh);
               }
             }
-            word[i >> 2] |= q << (8u * (i & 3u));
-            if (q < 8u) cnt[q >> 2] += 1u << (8u * (q & 3u));
-            else atomicAdd(&S.hist[levels - 1u + q], 1u);  // tab_base(b) = 2^b - 2 = levels - 1
+          }
+#pragma unroll
+          for (uint32_t j = 0; j < 8; ++j) {  // tokens past the tile's end code as 0
+            const uint32_t vb = nv > 4u * j ? min(4u, nv - 4u * j) : 0u;
+            if (vb < 4u) word[j] &= (1u << (8u * vb)) - 1u;
           }
           uint4* cd = reinterpret_cast<uint4*>(codes + uint64_t(wj) * kCodesRow + tb + w0);
           cd[0] = make_uint4(word[0], word[1], word[2], word[3]);
@@ -641,7 +650,7 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
     if (wlive) {
 #pragma unroll
       for (uint32_t q = 0; q < 8; ++q) {
-        const uint32_t n = (cnt[q >> 2] >> (8u * (q & 3u))) & 0xffu;
+        const uint32_t n = ((q < 4u ? cnt0 : cnt1) >> (8u * (q & 3u))) & 0xffu;
         if (n) atomicAdd(&S.ccnt[q][wc], n);
       }
     }
