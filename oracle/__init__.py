@@ -158,7 +158,7 @@ def stream_encode(sym: np.ndarray) -> bytes:
 
 
 def stream_encode_delta(sym: np.ndarray) -> bytes:
-    """Stream record with the lane-delta candidate (the high byte plane's coder)."""
+    """Stream record with the lane-delta candidate (the lossless planes' coder)."""
     s = np.ascontiguousarray(sym, dtype=np.uint8)
     lib = _load()
     out = np.zeros(lib.kvco_stream_bound(s.size), dtype=np.uint8)

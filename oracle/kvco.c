@@ -411,9 +411,33 @@ size_t kvco_stream_encode(const uint8_t* sym, uint32_t n, uint8_t* out) {
   return stream_encode_lanes(sym, n, lanes_for(n), 0, out);
 }
 
-/* Stream with the lane-delta candidate (the high byte plane of lossless chunks). */
+/* Sum of the squared symbol counts (the number of ordered pairs of equal symbols). */
+static uint64_t sq_counts(const uint8_t* sym, uint32_t n) {
+  uint64_t c[256] = {0}, q = 0;
+  for (uint32_t i = 0; i < n; i++) c[sym[i]]++;
+  for (int s = 0; s < 256; s++) q += c[s] * c[s];
+  return q;
+}
+
+/* Stream of a lossless chunk's byte plane with the lane-delta candidate. The
+ * candidate is coded only when the lane deltas' counts are more concentrated
+ * than the plane's own (sum of squared counts strictly larger) and their
+ * collision entropy -log2(sum (c/n)^2) is below log2(181), about 7.5 bits
+ * (181 sum c^2 > n^2): deltas of noise-like bytes cannot beat RAW by enough to
+ * pay for coding them. Exact integer tests on the two histograms, so any
+ * encoder takes the same decision before coding; the candidate is then kept
+ * only where strictly the smallest record. */
 size_t kvco_stream_encode_delta(const uint8_t* sym, uint32_t n, uint8_t* out) {
-  return stream_encode_lanes(sym, n, lanes_for(n), 1, out);
+  uint32_t N = lanes_for(n);
+  int allow = 0;
+  if (n) {
+    uint8_t* dsym = (uint8_t*)malloc(n);
+    lane_delta_n(sym, n, N, dsym);
+    uint64_t qd = sq_counts(dsym, n);
+    allow = qd > sq_counts(sym, n) && 181u * qd > (uint64_t)n * n;
+    free(dsym);
+  }
+  return stream_encode_lanes(sym, n, N, allow, out);
 }
 
 /* Side stream: the lane-delta choice on the side lane rule. */
@@ -646,9 +670,15 @@ size_t kvco_lossless_bound(const kvco_desc* d, uint32_t n_slices) {
 }
 
 /* Chunk record: for p = 0 .. E-1, the stream record of plane p (byte p of
- * every little-endian value, channel-major order inside the chunk). The upper
- * half of the planes, which hold the sign and exponent bits (plane 1 of a
- * 16-bit value; planes 2 and 3 of an f32), take the lane-delta candidate. */
+ * every little-endian value, channel-major order inside the chunk). Every
+ * plane takes the lane-delta candidate ([QATQ] "How it works", lossless
+ * candidates: delta-XOR, native 16-bit adjacent-XOR, shape-aware strided-XOR).
+ * In the channel-major chunk a value's stream predecessor is the previous
+ * token of its channel, which is also the value one row (the row width, the
+ * shape-aware stride) back in the token-major input; XOR is bytewise, so the
+ * 16-bit XOR with that predecessor is the lane delta of each byte plane; a
+ * plane codes it where its counts are concentrated enough (the gate of
+ * kvco_stream_encode_delta) and keeps it where it is strictly the smallest. */
 size_t kvco_encode_lossless(const kvco_desc* d, uint32_t first_slice, uint32_t n_slices,
                             const void* src, uint8_t* dst, size_t cap) {
   if (!lossless_ok(d) || (uint64_t)first_slice + n_slices > n_slices_total(d)) return 0;
@@ -669,7 +699,7 @@ size_t kvco_encode_lossless(const kvco_desc* d, uint32_t first_slice, uint32_t n
         for (uint32_t dd = 0; dd < D; dd++)
           for (uint32_t t = 0; t < tcc; t++)
             pl[(size_t)dd * tcc + t] = in[(((size_t)s * T + t0 + t) * D + dd) * E + b];
-        p += 2u * b < E ? kvco_stream_encode(pl, n, dst + p) : kvco_stream_encode_delta(pl, n, dst + p);
+        p += kvco_stream_encode_delta(pl, n, dst + p);
       }
       uint8_t* e = dst + HDR_BYTES + (size_t)IDX_ENTRY * r;
       put64(e, start);

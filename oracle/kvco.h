@@ -64,10 +64,13 @@ int kvco_normalize(const uint32_t count[256], uint16_t freq[256]);
 size_t kvco_stream_bound(uint32_t n);
 size_t kvco_stream_encode(const uint8_t* sym, uint32_t n, uint8_t* out);
 int kvco_stream_decode(const uint8_t* rec, size_t avail, uint32_t n, uint8_t* sym, size_t* used);
-/* Lane-delta candidate (used for the high byte plane of lossless chunks): the
- * plain choice unless RANS of the lane-delta symbols is strictly smaller than
- * both the plain RANS record and RAW. kvco_lane_delta / _undelta apply and
- * undo the transform (XOR with the previous symbol of the same rANS lane). */
+/* Lane-delta candidate (used for every byte plane of lossless chunks): coded
+ * when the lane deltas' counts are more concentrated than the plane's (sum of
+ * squared counts strictly larger) and their collision entropy is below
+ * log2(181) bits (181 sum c^2 > n^2), then taken only if its RANS record is
+ * strictly smaller than both the plain RANS record and RAW; the plain choice
+ * otherwise. kvco_lane_delta / _undelta apply and undo the transform (XOR with
+ * the previous symbol of the same rANS lane). */
 size_t kvco_stream_encode_delta(const uint8_t* sym, uint32_t n, uint8_t* out);
 void kvco_lane_delta(const uint8_t* sym, uint32_t n, uint8_t* out);
 void kvco_lane_undelta(uint8_t* sym, uint32_t n);

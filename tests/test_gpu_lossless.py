@@ -198,3 +198,50 @@ def test_full_chunk_mode_pairs_and_damage(D):
             got, _ = decode(plan, kvc.LOSSLESS, bytes(c), len(pairs))
             assert want != oracle.OK and got == want, (pos - off, got, want)
             c[pos] = orig
+
+
+def _ramp(w, scale=3, dtype=np.uint16):
+    t = np.arange(w.n_tokens)[None, :, None]
+    ch = np.arange(w.head_dim)[None, None, :]
+    s = np.arange(w.n_slices)[:, None, None]
+    x = (scale * t + 17 * ch + 29 * s + 4096)
+    return (x & (0xFFFF if dtype == np.uint16 else 0xFFFFFFFF)).astype(dtype)
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("lossless-1x8x512x128-bf16", dict(n_heads=2)),                    # full chunks of 128 channels
+    ("lossless-12x12x1024x64-fp16", dict(n_layers=1, n_heads=2)),      # full chunks of 64 channels
+    ("lossless-1x8x512x128-bf16", dict(n_heads=1, n_tokens=700)),      # a full and a ragged chunk
+])
+def test_low_plane_lane_deltas_equal_oracle_bytes(name, kw):
+    """Values that change by a few steps per token (a ramp along tokens) make
+    the low byte plane's lane deltas the smallest record: the low plane takes
+    the 16-bit XOR with the previous token of the channel too. The fast
+    encoder hands such chunks to the general encoder; the container is the
+    oracle's byte for byte and the GPU decoder restores it."""
+    w = _w(name, **kw)
+    plan, oplan = _plans(w)
+    x = _ramp(w)
+    want = oracle.encode_lossless(oplan, x)
+    st, got = encode(plan, kvc.LOSSLESS, x)
+    assert st == kvc.OK
+    assert got == want
+    n_rec = int.from_bytes(want[36:40], "little")
+    off0 = int.from_bytes(want[64:72], "little")
+    assert want[off0] == 2 and want[off0 + 3] == 1  # the first chunk's low plane: RANS of lane deltas
+    st, y = decode(plan, kvc.LOSSLESS, got, w.n_slices)
+    assert st == kvc.OK and np.array_equal(y, x)
+    assert n_rec >= 1
+
+
+def test_f32_low_planes_lane_deltas_equal_oracle_bytes():
+    """f32: every byte plane may take the lane deltas (a ramp in the low bits)."""
+    w = _w("lossless-1x8x512x128-bf16", dtype=kvgen.F32, n_heads=1, n_tokens=512, head_dim=64,
+           values_per_chunk=8192)
+    plan, oplan = _plans(w)
+    x = _ramp(w, scale=5, dtype=np.uint32)
+    want = oracle.encode_lossless(oplan, x)
+    st, got = encode(plan, kvc.LOSSLESS, x)
+    assert st == kvc.OK and got == want
+    st, y = decode(plan, kvc.LOSSLESS, got, w.n_slices)
+    assert st == kvc.OK and np.array_equal(y, x)

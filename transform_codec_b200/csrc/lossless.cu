@@ -12,23 +12,50 @@ namespace {
 
 constexpr uint32_t kThreads = 256;  // 8 warps: plane p = warp / 4, group = warp % 4
 
-// Encode: one CTA per chunk, 16 warps. Warps 0-11 code the variants v = warp / 4:
-// plane 0 (v = 0), plane 1 (v = 1) and plane 1's lane deltas (v = 2), warp % 4
-// being the rANS group; all 16 share the histograms, the writes and the CRC.
+// Encode: persistent CTAs of 16 warps, a chunk at a time. Warp w codes variant
+// v = w / 4: plane 0 (v = 0), plane 1 (v = 1), plane 1's lane deltas (v = 2)
+// and plane 0's lane deltas (v = 3), warp % 4 being the rANS group; all 16
+// share the histograms, the writes and the CRC.
 constexpr uint32_t kEncThreads = 512;
+constexpr uint32_t kEncVars = 4;
+// rec_len of a full chunk the fast encoder leaves to the general one
+constexpr uint32_t kRecLenDefer = kRecLenError | 0xfeu;
+__host__ __device__ constexpr uint32_t var_plane(uint32_t v) { return (v == 1u || v == 2u) ? 1u : 0u; }
+
+// Sum of the squared counts of a 256-bin histogram, by one warp (all lanes get
+// it). A plane's lane-delta candidate is coded only when its deltas' sum qd is
+// strictly larger than the plane's own and 181 qd > n^2 (delta_gate): their
+// counts are more concentrated, with a collision entropy under log2(181) bits.
+__device__ inline unsigned long long warp_sq_counts(const uint32_t* h) {
+  const uint32_t lane = threadIdx.x & 31u;
+  unsigned long long q = 0;
+#pragma unroll
+  for (uint32_t i = 0; i < 8; ++i) {
+    const unsigned long long c = h[lane + 32u * i];
+    q += c * c;
+  }
+#pragma unroll
+  for (uint32_t o = 16; o; o >>= 1) q += __shfl_xor_sync(0xffffffffu, q, o);
+  return q;
+}
+__device__ inline bool delta_gate(unsigned long long qd, unsigned long long qp, uint32_t n) {
+  return qd > qp && 181ull * qd > uint64_t(n) * n;
+}
 
 struct __align__(16) EncSmem {
   uint32_t crc_t[1024];
-  uint32_t hist[3][256];
-  uint32_t freq[3][256];
+  uint32_t hist[kEncVars][256];
+  uint32_t freq[kEncVars][256];
   uint32_t rem[256];
-  uint32_t fc[3][256];
-  uint32_t rcp[3][256];
-  uint2 tab[3][256];             // {f | cum << 16, 1/f} per variant
-  uint32_t states[3][kMaxLanes];
+  uint32_t fc[kEncVars][256];
+  uint32_t rcp[kEncVars][256];
+  uint2 tab[kEncVars][256];      // {f | cum << 16, 1/f} per variant
+  uint32_t states[kEncVars][kMaxLanes];
   uint32_t tmp[32], red[32];
-  uint32_t k[3], mode[2], bytes[2], csym[2], var[2];
-  uint32_t W[3][4], wbeg[3][4], sub_len[3][4];
+  uint32_t k[kEncVars], mode[2], bytes[2], csym[2], var[2];
+  uint32_t W[kEncVars][4], wbeg[kEncVars][4], sub_len[kEncVars][4];
+  unsigned long long sq[kEncVars];
+  uint32_t take;
 };
 
 struct __align__(16) DecSmem {
@@ -52,15 +79,24 @@ struct ChanMajor {
   }
 };
 
+// sel = 0: every record; sel = 1: the ragged last chunk of each slice and the
+// full chunks the fast encoder deferred (rec_len kRecLenDefer).
 __global__ void __launch_bounds__(kEncThreads)
-k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws, uint32_t tail_only) {
+k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws, uint32_t sel) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   EncSmem& S = *reinterpret_cast<EncSmem*>(smem_raw);
   uint16_t* vals = reinterpret_cast<uint16_t*>(smem_raw + sizeof(EncSmem));
   const uint32_t tid = threadIdx.x, nthr = blockDim.x;
-  // record of the batch: every record, or the last chunk of every slice (frames
-  // hold whole slices, so those are records cps - 1, 2 cps - 1, ...)
-  const uint32_t gr = tail_only ? (blockIdx.x + 1u) * sh.cps - 1u : blockIdx.x;
+  const uint32_t nrec = b.rec_base[b.n];
+  const bool ragged_tail = sh.T % sh.tc != 0;
+  crc_tables_init(S.crc_t);
+  for (uint32_t gr = blockIdx.x; gr < nrec; gr += gridDim.x) {
+  __syncthreads();
+  if (tid == 0)
+    S.take = sel == 0u || (ragged_tail && (gr - b.rec_base[frame_of(b.rec_base, b.n, gr)]) % sh.cps == sh.cps - 1u) ||
+             ws.rec_len[gr] == kRecLenDefer;
+  __syncthreads();
+  if (!S.take) continue;
   const uint32_t fr = frame_of(b.rec_base, b.n, gr);
   const uint32_t r = gr - b.rec_base[fr];
   const uint16_t* src = reinterpret_cast<const uint16_t*>(b.f[fr].src);
@@ -69,8 +105,7 @@ k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws, uint32_t tail
   const uint32_t n_max = sh.tc * D;
   const uint16_t* g = src + (uint64_t(slice) * sh.T + t0) * D;
 
-  crc_tables_init(S.crc_t);
-  for (uint32_t i = tid; i < 3u * 256u; i += nthr) (&S.hist[0][0])[i] = 0;
+  for (uint32_t i = tid; i < kEncVars * 256u; i += nthr) (&S.hist[0][0])[i] = 0;
   if ((reinterpret_cast<uintptr_t>(g) & 15u) == 0 && (n & 7u) == 0) {
     const uint4* g4 = reinterpret_cast<const uint4*>(g);
     uint4* v4 = reinterpret_cast<uint4*>(vals);
@@ -88,16 +123,21 @@ k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws, uint32_t tail
       atomicAdd(&S.hist[0][v & 0xffu], 1u);
       atomicAdd(&S.hist[1][v >> 8], 1u);
       const uint32_t t = i / D, d = i - t * D, si = d * tcc + t;
-      uint32_t dv = v >> 8;
-      if (!lane_start(si, n, N)) {
-        const uint32_t pv = t ? vals[i - D] : vals[(tcc - 1u) * D + d - 1u];
-        dv ^= pv >> 8;
-      }
-      atomicAdd(&S.hist[2][dv], 1u);
+      uint32_t dv = v;  // the 16-bit XOR with the predecessor: both planes' lane deltas
+      if (!lane_start(si, n, N)) dv ^= t ? vals[i - D] : vals[(tcc - 1u) * D + d - 1u];
+      atomicAdd(&S.hist[2][dv >> 8], 1u);
+      atomicAdd(&S.hist[3][dv & 0xffu], 1u);
     }
   }
   __syncthreads();
-  for (uint32_t v = 0; v < 3; ++v) {
+  {
+    const uint32_t warp = tid >> 5;
+    if (warp < kEncVars) {
+      const unsigned long long q = warp_sq_counts(S.hist[warp]);
+      if ((tid & 31u) == 0) S.sq[warp] = q;
+    }
+  }
+  for (uint32_t v = 0; v < kEncVars; ++v) {
     uint32_t k = block_normalize(S.hist[v], n, S.freq[v], S.rem, S.tmp);
     if (tid == 0) S.k[v] = k;
     block_enc_tables(S.freq[v], S.fc[v], S.rcp[v], S.tmp);
@@ -112,12 +152,14 @@ k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws, uint32_t tail
   {
     const uint32_t warp = tid >> 5, lane = tid & 31u;
     const uint32_t v = warp >> 2, gg = warp & 3u;
-    if (v < 3 && S.k[v] >= 2 && gg < G) {
+    // variant 2 (3): plane 1's (0's) lane deltas, coded where their counts are more concentrated
+    const bool gated = v < 2u || delta_gate(S.sq[v], S.sq[var_plane(v)], n);
+    if (v < kEncVars && S.k[v] >= 2 && gg < G && gated) {
       uint32_t b0, len0, b1 = n, len1;
       lane_range(n, N, gg * kGroupLanes, b0, len0);
       if (gg + 1 < G) lane_range(n, N, (gg + 1) * kGroupLanes, b1, len1);
       // symbol i of plane p: byte p of the value of channel d = i / tcc, token t = i % tcc
-      const uint8_t* v8 = reinterpret_cast<const uint8_t*>(vals) + (v ? 1u : 0u);
+      const uint8_t* v8 = reinterpret_cast<const uint8_t*>(vals) + var_plane(v);
       uint16_t* scratch = scratch0 + uint64_t(v) * (n_max + 32u);
       uint32_t x, Wg;
       if (v < 2)
@@ -137,10 +179,10 @@ k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws, uint32_t tail
   __syncthreads();
   if (tid == 0) {
     // per plane: CONST for one symbol; else the smallest of RANS (plain), RANS of
-    // the lane deltas (plane 1, only if strictly smaller than both others) and RAW
+    // the plane's lane deltas (only if strictly smaller than both others) and RAW
     const uint32_t raw_b = 16u + pad16(n);
     for (uint32_t p = 0; p < 2; ++p) {
-      const uint32_t k = S.k[p];
+      const uint32_t k = S.k[p], vd = p ? 2u : 3u;
       const uint32_t v0 = vals[0];
       S.csym[p] = p ? (v0 >> 8) : (v0 & 0xffu);
       S.var[p] = p;
@@ -148,8 +190,8 @@ k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws, uint32_t tail
       if (k < 2) { S.mode[p] = kModeRaw; S.bytes[p] = raw_b; continue; }
       const uint32_t rb = rans_layout(n, k, S.W[p], S.sub_len[p]);
       uint32_t rd = 0xffffffffu;
-      if (p == 1 && S.k[2] >= 2) rd = rans_layout(n, S.k[2], S.W[2], S.sub_len[2]);
-      if (rd < rb && rd < raw_b) { S.mode[p] = kModeRans; S.bytes[p] = rd; S.var[p] = 2; }
+      if (S.k[vd] >= 2 && delta_gate(S.sq[vd], S.sq[p], n)) rd = rans_layout(n, S.k[vd], S.W[vd], S.sub_len[vd]);
+      if (rd < rb && rd < raw_b) { S.mode[p] = kModeRans; S.bytes[p] = rd; S.var[p] = vd; }
       else if (rb < raw_b) { S.mode[p] = kModeRans; S.bytes[p] = rb; }
       else { S.mode[p] = kModeRaw; S.bytes[p] = raw_b; }
     }
@@ -179,7 +221,7 @@ k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws, uint32_t tail
     } else {
       block_write_stream(rec + off, S.mode[p], n, S.bytes[p], S.csym[p], S.k[v], S.freq[v], S.states[v],
                          scratch0 + uint64_t(v) * (n_max + 32u), S.wbeg[v], S.W[v], S.sub_len[v], raw, S.tmp,
-                         v == 2 ? 1u : 0u);
+                         v >= 2u ? 1u : 0u);
     }
     off += S.bytes[p];
   }
@@ -188,6 +230,7 @@ k_lossless_encode(LosslessShape sh, FrameBatch b, EncodeLayout ws, uint32_t tail
   if (tid == 0) {
     ws.rec_len[gr] = off;
     ws.rec_crc[gr] = crc;
+  }
   }
 }
 
@@ -327,7 +370,7 @@ struct __align__(16) FencSmem {
   uint32_t states[3][kMaxLanes];
   union {
     struct {
-      uint32_t hist[3][256];
+      uint32_t hist[4][256];                            // plane 0, plane 1, their lane deltas (1, 0)
       uint32_t rem[3][256];
     } h;                                                // phases 1-2
     uint8_t ring[kFencThreads / 32][kFencSlots][kFencSlotBytes];  // phase 3
@@ -340,6 +383,7 @@ struct __align__(16) FencSmem {
   uint32_t tmp[32], red[32];
   uint32_t k[3], W[3][4], sub_len[2][4], subst[2][5];
   uint32_t mode[2], bytes[2], var[2], csym[2], pbytes[2], crc[2];
+  uint32_t gate[2];  // the lane deltas of plane p are more concentrated than the plane
 };
 
 __device__ __forceinline__ uint32_t crc_unit(const uint32_t* t, uint32_t c, uint4 v) {
@@ -389,23 +433,27 @@ k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
   const uint16_t* g = reinterpret_cast<const uint16_t*>(b.f[fr].src) + (uint64_t(slice) * sh.T + t0) * D;
   const uint4* g4 = reinterpret_cast<const uint4*>(g);
 
-  for (uint32_t i = tid; i < 3u * 256u; i += kFencThreads) (&S.u.h.hist[0][0])[i] = 0;
+  for (uint32_t i = tid; i < 4u * 256u; i += kFencThreads) (&S.u.h.hist[0][0])[i] = 0;
   __syncthreads();
   {
-    // thread: column block cb (8 channels), tokens [tb, tb + SEGLEN); cur[j] is
-    // the previous token's high byte (0 before a lane's first token, which
-    // makes its delta the byte itself), run[j] the count of equal bytes so far
+    // thread: column block cb (8 channels), tokens [tb, tb + SEGLEN); cur[j] and
+    // lo[j] are the previous token's high and low bytes (0 before a lane's first
+    // token, which makes its delta the byte itself), run[j] the count of equal
+    // high bytes so far
     const uint32_t cb = tid % CB, tb = (tid / CB) * SEGLEN;
     const uint4* col = g4 + cb;
-    uint32_t cur[8], run[8], zeros = 0;
+    uint32_t cur[8], lo[8], run[8], zeros = 0, zlo = 0;
     if (tb % 512u == 0) {
 #pragma unroll
-      for (uint32_t j = 0; j < 8; ++j) cur[j] = 0;
+      for (uint32_t j = 0; j < 8; ++j) cur[j] = lo[j] = 0;
     } else {
       const uint4 w = __ldg(col + uint64_t(tb - 1u) * CB);
       const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (uint32_t j = 0; j < 8; ++j) cur[j] = (wv[j >> 1] >> (16u * (j & 1u) + 8u)) & 0xffu;
+      for (uint32_t j = 0; j < 8; ++j) {
+        cur[j] = (wv[j >> 1] >> (16u * (j & 1u) + 8u)) & 0xffu;
+        lo[j] = (wv[j >> 1] >> (16u * (j & 1u))) & 0xffu;
+      }
     }
 #pragma unroll
     for (uint32_t j = 0; j < 8; ++j) run[j] = 0;
@@ -420,7 +468,11 @@ k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
 #pragma unroll
         for (uint32_t j = 0; j < 8; ++j) {
           const uint32_t v = wv[j >> 1] >> (16u * (j & 1u));
-          atomicAdd(&S.u.h.hist[0][v & 0xffu], 1u);
+          const uint32_t lb = v & 0xffu, dl = lb ^ lo[j];
+          atomicAdd(&S.u.h.hist[0][lb], 1u);
+          if (dl) atomicAdd(&S.u.h.hist[3][dl], 1u);
+          else ++zlo;
+          lo[j] = lb;
           const uint32_t hb = (v >> 8) & 0xffu;
           if (hb == cur[j]) {
             ++run[j];
@@ -438,14 +490,26 @@ k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
     for (uint32_t j = 0; j < 8; ++j)
       if (run[j]) atomicAdd(&S.u.h.hist[1][cur[j]], run[j]);
     if (zeros) atomicAdd(&S.u.h.hist[2][0], zeros);
+    if (zlo) atomicAdd(&S.u.h.hist[3][0], zlo);
   }
   __syncthreads();
   if (warp < 3) {  // warp v: the table of variant v
     const uint32_t k = warp_normalize(S.u.h.hist[warp], 256u, n, S.freq[warp], S.u.h.rem[warp], S.tab[warp]);
     if (lane == 0) S.k[warp] = k;
+  } else {  // warp 3: the lane-delta gates of both planes
+    const unsigned long long q0 = warp_sq_counts(S.u.h.hist[0]), q1 = warp_sq_counts(S.u.h.hist[1]);
+    const unsigned long long q2 = warp_sq_counts(S.u.h.hist[2]), q3 = warp_sq_counts(S.u.h.hist[3]);
+    if (lane == 0) {
+      S.gate[0] = delta_gate(q3, q0, n) ? 1u : 0u;
+      S.gate[1] = delta_gate(q2, q1, n) ? 1u : 0u;
+    }
   }
   __syncthreads();
-  const bool en0 = S.k[0] >= 2, en1 = S.k[1] >= 2, en2 = en1 && S.k[2] >= 2;
+  if (S.gate[0] && S.k[0] >= 2u) {  // plane 0 codes its lane deltas too: the general encoder's chunk
+    if (tid == 0) ws.rec_len[gr] = kRecLenDefer;
+    return;
+  }
+  const bool en0 = S.k[0] >= 2, en1 = S.k[1] >= 2, en2 = en1 && S.k[2] >= 2 && S.gate[1];
   uint8_t* slot = ws.slots + uint64_t(gr) * ws.slot_bytes;
   uint16_t* scratch0 = reinterpret_cast<uint16_t*>(slot + kRecArea);
   {
@@ -525,7 +589,7 @@ k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
       }
       const uint32_t rb = rans_layout(n, k, S.W[p], S.sub_len[p]);
       uint32_t rd = 0xffffffffu, dl[4];
-      if (p == 1 && S.k[2] >= 2) rd = rans_layout(n, S.k[2], S.W[2], dl);
+      if (p == 1 && S.k[2] >= 2 && S.gate[1]) rd = rans_layout(n, S.k[2], S.W[2], dl);
       if (rd < rb && rd < raw_b) {
         S.mode[p] = kModeRans;
         S.bytes[p] = rd;
@@ -1051,8 +1115,7 @@ k_lossless_decode_fast(LosslessShape sh, FrameBatch b, uint8_t* ws) {
 // Encode: one CTA per chunk, 512 threads. The planes are coded one after
 // another through one shared plane buffer of the chunk's size: plane p is
 // gathered channel-major from the chunk (which stays in L2 across the
-// planes), counted (and, for the upper planes, which hold the sign and
-// exponent bits, its lane deltas too), its tables built, coded by one warp per
+// planes), counted with its lane deltas, its tables built, coded by one warp per
 // (variant, rANS group), and its stream record written at the record's
 // running offset by the never-worse rule. The record's CRC follows.
 struct __align__(16) WideEncSmem {
@@ -1061,7 +1124,7 @@ struct __align__(16) WideEncSmem {
   uint32_t states[2][kMaxLanes];
   uint32_t tmp[32], red[32];
   uint32_t k[2], W[2][4], wbeg[2][4], sub_len[2][4];
-  uint32_t mode, bytes, var, off;
+  uint32_t mode, bytes, var, off, gate;
 };
 
 template <uint32_t E>
@@ -1083,8 +1146,7 @@ k_lossless_encode_wide(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
   crc_tables_init(S.crc_t);
   if (tid == 0) S.off = 0;
   for (uint32_t p = 0; p < E; ++p) {
-    const bool upper = 2u * p >= E;
-    const uint32_t nvar = upper ? 2u : 1u;
+    uint32_t nvar = 2u;  // the plane and its lane deltas
     for (uint32_t i = tid; i < 2u * 256u; i += nthr) (&S.hist[0][0])[i] = 0;
     for (uint32_t q = tid; q < n; q += nthr) {
       const uint32_t t = q / D, d = q - t * D;
@@ -1094,9 +1156,15 @@ k_lossless_encode_wide(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
     for (uint32_t i = tid; i < n; i += nthr) {
       const uint32_t v = pl[i];
       atomicAdd(&S.hist[0][v], 1u);
-      if (upper) atomicAdd(&S.hist[1][lane_start(i, n, N) ? v : (v ^ pl[i - 1])], 1u);
+      atomicAdd(&S.hist[1][lane_start(i, n, N) ? v : (v ^ pl[i - 1])], 1u);
     }
     __syncthreads();
+    if (warp == 0) {  // the lane deltas are coded where their counts are more concentrated
+      const unsigned long long q0 = warp_sq_counts(S.hist[0]), q1 = warp_sq_counts(S.hist[1]);
+      if (lane == 0) S.gate = delta_gate(q1, q0, n) ? 1u : 0u;
+    }
+    __syncthreads();
+    nvar = S.gate ? 2u : 1u;
     for (uint32_t v = 0; v < nvar; ++v) {
       const uint32_t k = block_normalize(S.hist[v], n, S.freq[v], S.rem, S.tmp);
       if (tid == 0) S.k[v] = k;
@@ -1137,7 +1205,7 @@ k_lossless_encode_wide(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
         bytes = 16;
       } else if (k >= 2) {
         const uint32_t rb = rans_layout(n, k, S.W[0], S.sub_len[0]);
-        const uint32_t rd = upper && S.k[1] >= 2 ? rans_layout(n, S.k[1], S.W[1], S.sub_len[1]) : 0xffffffffu;
+        const uint32_t rd = nvar == 2u && S.k[1] >= 2 ? rans_layout(n, S.k[1], S.W[1], S.sub_len[1]) : 0xffffffffu;
         if (rd < rb && rd < raw_b) {
           mode = kModeRans; bytes = rd; var = 1;
         } else if (rb < raw_b) {
@@ -1269,10 +1337,10 @@ int num_sms() {
 uint64_t lossless_slot_bytes(const LosslessShape& s) {
   const uint64_t n_max = uint64_t(s.tc) * s.D;
   // the record (a stream per byte plane, each at most RAW), then the word
-  // scratch of the variants coded side by side: three for 16-bit values
-  // (plane 0, plane 1 and its lane deltas), two for wide values (one plane at
-  // a time and its lane deltas)
-  uint64_t b = s.E * (16u + pad16_64(n_max)) + (s.E == 4u ? 2u : 3u) * (2u * n_max + 64u);
+  // scratch of the variants coded side by side: four for 16-bit values (each
+  // plane and its lane deltas), two for wide values (one plane at a time and
+  // its lane deltas)
+  uint64_t b = s.E * (16u + pad16_64(n_max)) + (s.E == 4u ? 2u : kEncVars) * (2u * n_max + 64u);
   return (b + 255u) & ~uint64_t(255);
 }
 
@@ -1306,14 +1374,16 @@ cudaError_t launch_lossless_encode(const LosslessShape& s, const FrameBatch& b,
       kern<<<nrec, kFencThreads, fsmem, st>>>(s, b, ws);
     }
     e = cudaGetLastError();
-    if (e != cudaSuccess || s.T % s.tc == 0) return e;
+    if (e != cudaSuccess) return e;
   }
+  // the general encoder: every record, or (after the fast one) the ragged last
+  // chunks and the chunks it deferred
   size_t smem = sizeof(EncSmem) + pad16(s.tc * s.D * 2u);
   e = cudaFuncSetAttribute(k_lossless_encode, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   {
     ProfRange pr_(fast ? "lossless_encode_tail" : "lossless_encode", st);
-    k_lossless_encode<<<fast ? nrec / s.cps : nrec, kEncThreads, smem, st>>>(s, b, ws, fast ? 1u : 0u);
+    k_lossless_encode<<<min(nrec, uint32_t(num_sms())), kEncThreads, smem, st>>>(s, b, ws, fast ? 1u : 0u);
   }
   return cudaGetLastError();
 }
