@@ -49,7 +49,7 @@
 extern "C" {
 #endif
 
-#define KVC_ABI_VERSION 1u
+#define KVC_ABI_VERSION 2u
 
 /* status codes (return values and kvc_result.status) */
 enum {
@@ -104,6 +104,14 @@ typedef struct kvc_plan_s kvc_plan_t;
  *                     widths is NULL; negative values count as 0)
  *   widths            transform: optional host [L*2*H][D] bit widths that
  *                     replace the greedy allocation
+ *   range_mode        transform: KVC_RANGES_BLOCK (0: a zero point and scale per
+ *                     component and block of block_tokens tokens, keys and
+ *                     values) or KVC_RANGES_KIVI (Codec-Gauge page, "Compression
+ *                     Conditions": per-channel key ranges, per-token value
+ *                     ranges: keys as BLOCK; each value token one zero point z
+ *                     and range r over its coded components, a component of
+ *                     width b quantised in steps r / (2^b - 1); needs D >=
+ *                     block_tokens). Part of the plan CRC when not BLOCK.
  * For a lossless-only plan set bases, eigvals and widths to NULL. */
 typedef struct {
   uint32_t abi_version;
@@ -116,7 +124,10 @@ typedef struct {
   const float* bases;
   const double* eigvals;
   const uint8_t* widths;
+  uint32_t range_mode;
+  uint32_t reserved;
 } kvc_plan_desc;
+enum { KVC_RANGES_BLOCK = 0, KVC_RANGES_KIVI = 1 };
 
 /* kvc_plan — the plan of a cache shape (KVTC page, "How the Pipeline Works":
  * the per-component bit widths, scales and zero points that reconstruction

@@ -44,7 +44,11 @@ class Desc(ctypes.Structure):
         ("max_bits", ctypes.c_uint32), ("rope_theta", ctypes.c_double),
         ("bases", ctypes.c_void_p), ("widths", ctypes.c_void_p),
         ("plan_crc", ctypes.c_uint32), ("plan_crc_set", ctypes.c_uint32),
+        ("ranges", ctypes.c_uint32),
     ]
+
+
+RANGES_BLOCK, RANGES_KIVI = 0, 1
 
 
 def _load():
@@ -113,7 +117,7 @@ class Plan:
 
     def __init__(self, dtype, n_layers, n_heads, n_tokens, head_dim, values_per_chunk=65536,
                  n_sink=4, n_recent=128, block_tokens=64, chunk_tokens=512, max_bits=8,
-                 rope_theta=1e4, bases=None, widths=None):
+                 rope_theta=1e4, bases=None, widths=None, ranges=RANGES_BLOCK):
         self.bases = None if bases is None else np.ascontiguousarray(bases, dtype=np.float32)
         self.widths = None if widths is None else np.ascontiguousarray(widths, dtype=np.uint8)
         self.desc = Desc(dtype, n_layers, n_heads, n_tokens, head_dim, values_per_chunk,
@@ -121,6 +125,7 @@ class Plan:
                          None if self.bases is None else _ptr(self.bases),
                          None if self.widths is None else _ptr(self.widths))
         self._bound = {}
+        self.desc.ranges = ranges
         if self.bases is not None and self.widths is not None:
             # the plan CRC every transform container carries, computed once here
             self.desc.plan_crc = _load().kvco_plan_crc(ctypes.byref(self.desc))
@@ -131,10 +136,10 @@ class Plan:
         return self.desc.n_layers * 2 * self.desc.n_heads
 
     @classmethod
-    def from_workload(cls, w, bases=None, widths=None):
+    def from_workload(cls, w, bases=None, widths=None, ranges=RANGES_BLOCK):
         return cls(w.dtype, w.n_layers, w.n_heads, w.n_tokens, w.head_dim, w.values_per_chunk,
                    w.n_sink, w.n_recent, w.block_tokens, w.chunk_tokens, w.max_bits, w.theta,
-                   bases, widths)
+                   bases, widths, ranges)
 
 
 def crc32(data) -> int:

@@ -857,10 +857,11 @@ int kvco_allocate(const double* lambda, uint64_t n_units, double avg_bits, uint3
 
 /* CRC32 over the plan parameters that the bytes depend on: u32 dtype, L, H, T, D,
  * n_sink, n_recent, block_tokens, chunk_tokens, max_bits; u64 bits of theta;
- * the U widths; the bases as little-endian fp32. */
+ * the U widths; the bases as little-endian fp32; then, for a range mode other
+ * than BLOCK, u32 ranges. */
 uint32_t kvco_plan_crc(const kvco_desc* d) {
   uint64_t U = (uint64_t)n_slices_total(d) * d->head_dim;
-  size_t len = 48 + U + U * d->head_dim * 4u;
+  size_t len = 48 + U + U * d->head_dim * 4u + (d->ranges ? 4u : 0u);
   uint8_t* b = (uint8_t*)malloc(len);
   uint32_t v[10] = {d->dtype, d->n_layers, d->n_heads, d->n_tokens, d->head_dim,
                     d->n_sink, d->n_recent, d->block_tokens, d->chunk_tokens, d->max_bits};
@@ -874,6 +875,7 @@ uint32_t kvco_plan_crc(const kvco_desc* d) {
     memcpy(&fb, &d->bases[i], 4);
     put32(b + 48 + U + 4 * i, fb);
   }
+  if (d->ranges) put32(b + len - 4, d->ranges);  /* only a non-default range mode */
   uint32_t crc = kvco_crc32(b, len);
   free(b);
   return crc;
@@ -919,7 +921,25 @@ static int transform_ok(const kvco_desc* d) {
   if ((uint64_t)d->chunk_tokens * d->head_dim > 65536u) return 0;
   if (d->n_sink > 65535u || d->n_recent > 65535u || d->block_tokens > 65535u) return 0;
   if (!(d->rope_theta > 0.0)) return 0;
+  if (d->ranges > KVCO_RANGES_KIVI) return 0;
+  /* a KIVI-style chunk's (z, range) pairs, one per token, use the side buffers
+   * of its D x (ct / B) (z, s) pairs */
+  if (d->ranges == KVCO_RANGES_KIVI && d->head_dim < d->block_tokens) return 0;
   return 1;
+}
+
+/* Values of a KIVI-style plan take one range per token ([GAUGE] "Compression
+ * Conditions": per-channel key ranges, per-token value ranges); keys keep the
+ * per-component block ranges, which are per-channel ranges in the basis. */
+static int kivi_values(const kvco_desc* d, uint32_t sidx) {
+  return d->ranges == KVCO_RANGES_KIVI && ((sidx / d->n_heads) % 2u) == 1u;
+}
+
+/* Values of V, the side information of a middle record of tcc tokens: every
+ * zero point, then every scale or range. */
+static uint32_t side_values(const kvco_desc* d, uint32_t sidx, uint32_t coded, uint32_t tcc) {
+  if (!coded) return 0;
+  return kivi_values(d, sidx) ? 2u * tcc : 2u * coded * ((tcc + d->block_tokens - 1) / d->block_tokens);
 }
 
 static void regions(const kvco_desc* d, uint32_t* s_end, uint32_t* r_start) {
@@ -945,10 +965,11 @@ static uint32_t count_width(const uint8_t* w, uint32_t D, uint32_t b) {
   return m;
 }
 
-static size_t mid_record_bound(const kvco_desc* d, const uint8_t* w, uint32_t tcc) {
-  uint32_t nb = (tcc + d->block_tokens - 1) / d->block_tokens;
+static size_t mid_record_bound(const kvco_desc* d, uint32_t sidx, uint32_t tcc) {
+  const uint8_t* w = d->widths + (size_t)sidx * d->head_dim;
   uint32_t coded = d->head_dim - count_width(w, d->head_dim, 0);
-  size_t bytes = coded ? 4u * (16u + pad16((size_t)2 * coded * nb)) : 0u;  /* side streams at most RAW */
+  uint32_t nv = side_values(d, sidx, coded, tcc);
+  size_t bytes = nv ? 4u * (16u + pad16((size_t)nv)) : 0u;  /* side streams at most RAW */
   for (uint32_t b = 1; b <= 8; b++) {
     uint32_t m = count_width(w, d->head_dim, b);
     if (m) bytes += 16u + pad16((size_t)m * tcc);
@@ -973,7 +994,7 @@ static size_t slice_bound(const kvco_desc* d, uint32_t sl) {
   for (uint32_t c = 0; c < nm; c++) {
     uint32_t t0 = s_end + c * d->chunk_tokens;
     uint32_t tcc = r_start - t0 < d->chunk_tokens ? r_start - t0 : d->chunk_tokens;
-    b += mid_record_bound(d, d->widths + (size_t)sl * D, tcc);
+    b += mid_record_bound(d, sl, tcc);
   }
   return b;
 }
@@ -1029,7 +1050,8 @@ static uint32_t quantize(float y, float z, float s, uint32_t levels, float* qpre
 }
 
 /* Project and quantise one middle chunk. codes[j * ct + t]; qpre[t * D + j]
- * (optional); zs[(j * nbmax + blk) * 2 + {0: z, 1: s}]. */
+ * (optional); zs[(j * nbmax + blk) * 2 + {0: z, 1: s}], or for the values of a
+ * KIVI-style plan zs[t * 2 + {0: z, 1: range}]. */
 static void mid_chunk_quantize(const kvco_desc* d, uint32_t sidx, const uint16_t* xs,
                                const float* cs, uint32_t t0, uint32_t tcc, float* y,
                                uint8_t* codes, float* qpre, float* zs) {
@@ -1046,6 +1068,39 @@ static void mid_chunk_quantize(const kvco_desc* d, uint32_t sidx, const uint16_t
     kvco_project(Q, D, x, y + (size_t)t * D);
   }
   free(x);
+  if (kivi_values(d, sidx)) {
+    /* per token: z = min over the coded components (ascending), range =
+     * fl(max - min); a component of width b uses s = fl(range / (2^b - 1)) */
+    for (uint32_t t = 0; t < tcc; t++) {
+      float mn = 0.0f, mx = 0.0f;
+      int first = 1;
+      for (uint32_t j = 0; j < D; j++) {
+        if (!w[j]) continue;
+        float v = y[(size_t)t * D + j];
+        if (first) { mn = mx = v; first = 0; continue; }
+        if (v < mn) mn = v;
+        if (v > mx) mx = v;
+      }
+      float rng = mx - mn;
+      for (uint32_t j = 0; j < D; j++) {
+        uint32_t b = w[j];
+        if (!b) {
+          codes[(size_t)j * ct + t] = 0;
+          if (qpre) qpre[(size_t)t * D + j] = 0.0f;
+          continue;
+        }
+        uint32_t levels = (1u << b) - 1u;
+        float sc = (mx == mn) ? 0.0f : rng / (float)levels;
+        codes[(size_t)j * ct + t] =
+            (uint8_t)quantize(y[(size_t)t * D + j], mn, sc, levels, qpre ? &qpre[(size_t)t * D + j] : NULL);
+      }
+      if (zs) {
+        zs[(size_t)t * 2] = mn;
+        zs[(size_t)t * 2 + 1] = first ? 0.0f : rng;
+      }
+    }
+    return;
+  }
   uint32_t nb = (tcc + B - 1) / B;
   for (uint32_t j = 0; j < D; j++) {
     uint32_t b = w[j];
@@ -1122,9 +1177,18 @@ size_t kvco_encode_transform(const kvco_desc* d, uint32_t first_slice, uint32_t 
       uint32_t nb = (tcc + B - 1) / B;
       mid_chunk_quantize(d, sidx, xs, cs, t0, tcc, y, codes, NULL, zs);
       start = p;
-      /* side information: V = every z, then every s, split into byte planes */
-      uint32_t coded = D - count_width(w, D, 0), nv = 2u * coded * nb, i = 0;
-      for (uint32_t half_v = 0; half_v < 2; half_v++)
+      /* side information: V = every z, then every s (KIVI-style values: every
+       * token's z, then every token's range), split into byte planes */
+      uint32_t coded = D - count_width(w, D, 0), nv = side_values(d, sidx, coded, tcc), i = 0;
+      for (uint32_t half_v = 0; half_v < 2 && nv; half_v++) {
+        if (kivi_values(d, sidx)) {
+          for (uint32_t t = 0; t < tcc; t++, i++) {
+            uint32_t v;
+            memcpy(&v, &zs[(size_t)t * 2 + half_v], 4);
+            for (uint32_t q = 0; q < 4; q++) side[(size_t)q * nv + i] = (uint8_t)(v >> (8u * q));
+          }
+          continue;
+        }
         for (uint32_t j = 0; j < D; j++) {
           if (!w[j]) continue;
           for (uint32_t blk = 0; blk < nb; blk++, i++) {
@@ -1133,6 +1197,7 @@ size_t kvco_encode_transform(const kvco_desc* d, uint32_t first_slice, uint32_t 
             for (uint32_t q = 0; q < 4; q++) side[(size_t)q * nv + i] = (uint8_t)(v >> (8u * q));
           }
         }
+      }
       if (nv)
         for (uint32_t q = 0; q < 4; q++) p += kvco_side_stream_encode(side + (size_t)q * nv, nv, dst + p);
       for (uint32_t b = 1; b <= 8; b++) {
@@ -1162,7 +1227,7 @@ static int mid_chunk_parse(const kvco_desc* d, uint32_t sidx, const uint8_t* rec
   uint32_t D = d->head_dim, ct = d->chunk_tokens, B = d->block_tokens, nbmax = ct / B;
   const uint8_t* w = d->widths + (size_t)sidx * D;
   uint32_t nb = (tcc + B - 1) / B;
-  uint32_t coded = D - count_width(w, D, 0), nv = 2u * coded * nb;
+  uint32_t coded = D - count_width(w, D, 0), nv = side_values(d, sidx, coded, tcc);
   size_t p = 0;
   /* side streams: byte q of every value of V (the syms buffer holds ct * D >= 4 nv bytes) */
   for (uint32_t q = 0; q < 4 && nv; q++) {
@@ -1177,7 +1242,15 @@ static int mid_chunk_parse(const kvco_desc* d, uint32_t sidx, const uint8_t* rec
       zs[((size_t)j * nbmax + blk) * 2] = zs[((size_t)j * nbmax + blk) * 2 + 1] = 0.0f;
     memset(codes + (size_t)j * ct, 0, ct);
   }
-  for (uint32_t half_v = 0; half_v < 2; half_v++)
+  for (uint32_t half_v = 0; half_v < 2 && nv; half_v++) {
+    if (kivi_values(d, sidx)) {
+      for (uint32_t t = 0; t < tcc; t++, i++) {
+        uint32_t v = 0;
+        for (uint32_t q = 0; q < 4; q++) v |= (uint32_t)syms[(size_t)q * nv + i] << (8u * q);
+        memcpy(&zs[(size_t)t * 2 + half_v], &v, 4);
+      }
+      continue;
+    }
     for (uint32_t j = 0; j < D; j++) {
       if (!w[j]) continue;
       for (uint32_t blk = 0; blk < nb; blk++, i++) {
@@ -1186,6 +1259,7 @@ static int mid_chunk_parse(const kvco_desc* d, uint32_t sidx, const uint8_t* rec
         memcpy(&zs[((size_t)j * nbmax + blk) * 2 + half_v], &v, 4);
       }
     }
+  }
   for (uint32_t b = 1; b <= 8; b++) {
     uint32_t m = count_width(w, D, b);
     if (!m) continue;
@@ -1258,11 +1332,20 @@ int kvco_decode_transform(const kvco_desc* d, const uint8_t* src, size_t n, uint
       if (kvco_crc32(rec, len) != get32(e + 12)) { st = KVCO_CORRUPT; break; }
       st = mid_chunk_parse(d, sidx, rec, len, tcc, codes, zs, syms);
       if (st) break;
+      const int kv = kivi_values(d, sidx);
       for (uint32_t t = 0; t < tcc; t++) {
         uint32_t blk = t / B;
         for (uint32_t j = 0; j < D; j++) {
           if (!w[j]) { yh[j] = 0.0f; continue; }
-          float z = zs[((size_t)j * nbmax + blk) * 2], sc = zs[((size_t)j * nbmax + blk) * 2 + 1];
+          float z, sc;
+          if (kv) {  /* the token's zero point; its range in 2^b - 1 steps */
+            float rng = zs[(size_t)t * 2 + 1];
+            z = zs[(size_t)t * 2];
+            sc = rng == 0.0f ? 0.0f : rng / (float)((1u << w[j]) - 1u);
+          } else {
+            z = zs[((size_t)j * nbmax + blk) * 2];
+            sc = zs[((size_t)j * nbmax + blk) * 2 + 1];
+          }
           yh[j] = fmaf((float)codes[(size_t)j * ct + t], sc, z);
         }
         kvco_unproject(Q, D, yh, xh);

@@ -55,7 +55,12 @@ typedef struct {
    * so that each transform call does not recompute it over all the bases;
    * 0 and 0 make every call compute it */
   uint32_t plan_crc, plan_crc_set;
+  /* transform value ranges: KVCO_RANGES_BLOCK (per component and block of
+   * tokens, keys and values) or KVCO_RANGES_KIVI (keys as BLOCK; values one
+   * range per token over its coded components) */
+  uint32_t ranges;
 } kvco_desc;
+enum { KVCO_RANGES_BLOCK = 0, KVCO_RANGES_KIVI = 1 };
 
 uint32_t kvco_crc32(const void* p, size_t n);
 

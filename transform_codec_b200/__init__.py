@@ -25,7 +25,8 @@ ERR_TIMEOUT, ERR_CUDA, ERR_UNSUPPORTED = 6, 7, 8
 BF16, FP16, F32 = 1, 2, 3  # value types (f32: lossless only)
 DTYPE_F32 = F32
 LOSSLESS, TRANSFORM = 0, 1
-ABI_VERSION = 1
+ABI_VERSION = 2
+RANGES_BLOCK, RANGES_KIVI = 0, 1  # transform value ranges: per block, or KIVI-style per-token values
 
 EXPORTS = [
     "kvc_plan", "kvc_plan_create", "kvc_plan_destroy", "kvc_plan_widths", "kvc_plan_crc",
@@ -58,6 +59,7 @@ class PlanDesc(ctypes.Structure):
         ("max_bits", ctypes.c_uint32),
         ("rope_theta", ctypes.c_double), ("avg_bits", ctypes.c_double),
         ("bases", ctypes.c_void_p), ("eigvals", ctypes.c_void_p), ("widths", ctypes.c_void_p),
+        ("range_mode", ctypes.c_uint32), ("reserved", ctypes.c_uint32),
     ]
 
 
@@ -160,6 +162,7 @@ class Shape:
     max_bits: int = 8
     rope_theta: float = 1e4
     avg_bits: float = 2.0
+    range_mode: int = 0  # RANGES_BLOCK or RANGES_KIVI
 
     @property
     def n_slices(self) -> int:
@@ -175,7 +178,7 @@ class Shape:
         return PlanDesc(ABI_VERSION, self.dtype, self.n_layers, self.n_heads, self.n_tokens,
                         self.head_dim, self.values_per_chunk, self.n_sink, self.n_recent,
                         self.block_tokens, self.chunk_tokens, self.max_bits, self.rope_theta,
-                        self.avg_bits, _np_ptr(bases), _np_ptr(eigvals), _np_ptr(widths))
+                        self.avg_bits, _np_ptr(bases), _np_ptr(eigvals), _np_ptr(widths), self.range_mode, 0)
 
 
 class Plan:

@@ -121,14 +121,16 @@ void regions(const kvc_plan_desc& d, uint32_t& s_end, uint32_t& r_start) {
   r_start = std::max(rs, s_end);
 }
 
-uint64_t mid_record_bound(const uint8_t* w, uint32_t D, uint32_t tcc, uint32_t block) {
+uint64_t mid_record_bound(const uint8_t* w, uint32_t D, uint32_t tcc, uint32_t block, bool kivi_values) {
   uint32_t nb = (tcc + block - 1) / block, coded = 0, m[9] = {0};
   for (uint32_t j = 0; j < D; ++j) {
     coded += w[j] > 0;
     m[w[j]]++;
   }
-  // side information: four byte-plane streams of 2 * coded * nb values, each at most RAW
-  uint64_t b = coded ? 4ull * (16 + pad16u(2ull * coded * nb)) : 0ull;
+  // side information: four byte-plane streams of 2 * coded * nb values (per-token
+  // value ranges: 2 * tcc), each at most RAW
+  const uint64_t nv = kivi_values ? 2ull * tcc : 2ull * coded * nb;
+  uint64_t b = coded ? 4ull * (16 + pad16u(nv)) : 0ull;
   for (uint32_t k = 1; k <= 8; ++k)
     if (m[k]) b += 16 + pad16u(uint64_t(m[k]) * tcc);
   return b;
@@ -167,6 +169,11 @@ uint32_t compute_plan_crc(const kvc_plan_desc& d, const std::vector<uint8_t>& wi
     for (int b = 0; b < 4; ++b) le[4 * i + b] = uint8_t(x >> (8 * b));
   }
   crc = h.update(crc, le.data(), le.size());
+  if (d.range_mode) {  // only a non-default range mode
+    uint8_t rm[4];
+    for (int b = 0; b < 4; ++b) rm[b] = uint8_t(d.range_mode >> (8 * b));
+    crc = h.update(crc, rm, 4);
+  }
   return crc ^ 0xffffffffu;
 }
 
@@ -323,6 +330,7 @@ extern "C" int kvc_plan(const kvc_plan_desc* desc, kvc_plan_t** out) {
   if (!d.n_layers || !d.n_heads || !d.n_tokens || !d.head_dim) return KVC_ERR_INVALID;
   if (uint64_t(d.n_layers) * 2u * d.n_heads > 0x7fffffffu) return KVC_ERR_INVALID;
   if (d.values_per_chunk < d.head_dim || d.values_per_chunk > kMaxChunkValues) return KVC_ERR_INVALID;
+  if (d.range_mode > KVC_RANGES_KIVI || d.reserved) return KVC_ERR_INVALID;
   auto* p = new kvc_plan_s();
   p->d = d;
   p->d.bases = nullptr;
@@ -340,7 +348,7 @@ extern "C" int kvc_plan(const kvc_plan_desc* desc, kvc_plan_t** out) {
     if (d.dtype != KVC_DTYPE_BF16 || (d.head_dim & 1u) || d.max_bits > 8 || !(d.rope_theta > 0.0) ||
         !d.block_tokens || !d.chunk_tokens || d.chunk_tokens % d.block_tokens ||
         d.n_sink > 65535u || d.n_recent > 65535u || d.block_tokens > 65535u ||
-        (!d.eigvals && !d.widths))
+        (!d.eigvals && !d.widths) || (d.range_mode == KVC_RANGES_KIVI && d.head_dim < d.block_tokens))
       st = KVC_ERR_INVALID;
     else if (d.head_dim != 128 || d.block_tokens != 64 || d.chunk_tokens > 512)
       st = KVC_ERR_UNSUPPORTED;
@@ -364,6 +372,7 @@ extern "C" int kvc_plan(const kvc_plan_desc* desc, kvc_plan_t** out) {
     TransformShape& ts = p->ts;
     ts.L = d.n_layers; ts.H = d.n_heads; ts.T = d.n_tokens; ts.D = d.head_dim;
     ts.ct = d.chunk_tokens; ts.block = d.block_tokens; ts.n_sink = d.n_sink; ts.n_recent = d.n_recent;
+    ts.kivi = d.range_mode == KVC_RANGES_KIVI ? 1u : 0u;
     regions(d, ts.s_end, ts.r_start);
     ts.n_mid = (ts.r_start - ts.s_end + ts.ct - 1) / ts.ct;
     const uint64_t raw = pad16u(uint64_t(ts.s_end + ts.T - ts.r_start) * ts.D * 2u);
@@ -371,7 +380,8 @@ extern "C" int kvc_plan(const kvc_plan_desc* desc, kvc_plan_t** out) {
       uint64_t b = raw;
       for (uint32_t c = 0; c < ts.n_mid; ++c) {
         uint32_t t0 = ts.s_end + c * ts.ct, tcc = std::min(ts.ct, ts.r_start - t0);
-        b += mid_record_bound(p->widths.data() + size_t(s) * ts.D, ts.D, tcc, ts.block);
+        b += mid_record_bound(p->widths.data() + size_t(s) * ts.D, ts.D, tcc, ts.block,
+                              ts.kivi && ((s / ts.H) & 1u) == 1u);
       }
       p->max_slice_bytes = std::max(p->max_slice_bytes, b);
     }

@@ -130,6 +130,7 @@ cudaError_t launch_lossless_decode(const LosslessShape& s, const FrameBatch& b, 
 struct TransformShape {
   uint32_t L, H, T, D, ct, block, n_sink, n_recent;
   uint32_t s_end, r_start, n_mid;   // regions and middle chunks per slice
+  uint32_t kivi;                    // values take per-token ranges (KVC_RANGES_KIVI)
 };
 // Per-slice component order of the transform path (head_dim 128), computed on
 // the host when the plan is made: the coded components (width >= 1) grouped by

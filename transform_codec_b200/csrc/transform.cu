@@ -147,6 +147,9 @@ struct __align__(1024) PtSmem {
   uint8_t b[4][kQDigPlane];    // Q digits of the slice's coded columns (B operand)
   float y[kD * kYStride];      // y[cc][t]: fl32(S~), the exact y where a chain ran
   int32_t tok_e[kPTok];        // e_t, or kZeroTok
+  float tok_x1[kPTok];         // x1 of the token (per-token ranges)
+  int32_t kq_fmax;             // per-token ranges: the slice's largest coded column exponent
+  float kq_q1max;              // and 1-norm bound
   int32_t blk_e[2][2];         // per tile parity and block: largest e_t (kZeroTok: all tokens zero)
   uint32_t blk_x1[2][2];       // largest x1 (bits of a non-negative float)
   uint32_t zero_tok[2][4];     // per 32-token word: tokens whose x is all zero
@@ -234,6 +237,7 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
     const uint16_t* src = reinterpret_cast<const uint16_t*>(b.f[fr].src);
     const uint32_t sidx = b.f[fr].first_slice + ls;
     const bool is_key = ((sidx / sh.H) & 1u) == 0;
+    const bool kiv = sh.kivi && !is_key;  // values with per-token ranges
     const uint32_t t0 = sh.s_end + c * sh.ct, tcc = min(sh.ct, sh.r_start - t0);
     const uint32_t nb = (tcc + kTile - 1) / kTile;
     const uint16_t* xs = src + uint64_t(ls) * sh.T * kD;
@@ -248,6 +252,24 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
         S.col_f[tid] = pl.qcol[sidx].f[tid];
         S.col_q1[tid] = pl.qcol[sidx].q1[tid];
       }
+      __syncthreads();
+      if (tid < 32u) {  // the largest column exponent and 1-norm bound of the coded columns
+        int32_t fm = kQColZero;
+        float qm = 0.0f;
+        for (uint32_t cc = tid; cc < S.ci.n_coded; cc += 32u) {
+          fm = max(fm, S.col_f[cc]);
+          qm = fmaxf(qm, S.col_q1[cc]);
+        }
+#pragma unroll
+        for (uint32_t o = 16; o; o >>= 1) {
+          fm = max(fm, __shfl_xor_sync(0xffffffffu, fm, o));
+          qm = fmaxf(qm, __shfl_xor_sync(0xffffffffu, qm, o));
+        }
+        if (tid == 0) {
+          S.kq_fmax = fm;
+          S.kq_q1max = qm;
+        }
+      }
     }
     for (uint32_t i = tid; i < kTabPool; i += kPThreads) S.hist[i] = 0;
     for (uint32_t i = tid; i < 8u * kD; i += kPThreads) (&S.ccnt[0][0])[i] = 0;
@@ -260,7 +282,7 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
     const uint32_t nc = S.ci.n_coded;
     const uint32_t N = max(16u, (nc + 15u) & ~15u);
     {  // side-information padding of the record (its values are written below)
-      const uint32_t side = 8u * nc * nb;
+      const uint32_t side = nc ? 8u * (kiv ? tcc : nc * nb) : 0u;
       if (tid < pad16(side) - side) rec[side + tid] = 0;
     }
     __syncthreads();
@@ -367,6 +389,7 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
         }
         if (dg == 0) {
           S.tok_e[dt] = e;
+          S.tok_x1[dt] = x1;
           if (dt < bl) {
             if (e == kZeroTok) atomicOr(&S.zero_tok[par][dt >> 5], 1u << (dt & 31u));
             else {
@@ -475,6 +498,7 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
       }
       tc::fence_before_sync();
       __syncthreads();
+      if (!kiv) {
       // ---- per word: bound, candidates, chains, zero point and scale, codes
       {
         const uint32_t w0 = blk2 * 64u + hf * 32u;  // first token of the word in the tile
@@ -643,6 +667,147 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
           cd[0] = make_uint4(word[0], word[1], word[2], word[3]);
           cd[1] = make_uint4(word[4], word[5], word[6], word[7]);
         }
+      }
+      } else {
+      // ---- values with per-token ranges (KIVI-style): thread t = tid / 4 takes
+      // quarter q = tid % 4 of the coded components of token t; the four
+      // quarters of a token are neighbouring lanes
+      {
+        const uint32_t t = tid >> 2, q = tid & 3u, nq = (nc + 3u) >> 2;
+        const uint32_t c0 = min(nc, q * nq), c1 = min(nc, c0 + nq);
+        const bool tv = t < bl;
+        const int32_t et = S.tok_e[t];
+        float mn = __int_as_float(0x7f800000), mx = __int_as_float(0xff800000);
+        for (uint32_t cc = c0; cc < c1; ++cc) {
+          const float v = S.y[cc * kYStride + t];
+          mn = fminf(mn, v);
+          mx = fmaxf(mx, v);
+        }
+#pragma unroll
+        for (uint32_t o = 1; o < 4; o <<= 1) {
+          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+        }
+        const uint32_t qmask = (c1 - c0) == 32u ? 0xffffffffu : (1u << (c1 - c0)) - 1u;
+        uint32_t exact = 0, cand = 0;
+        float R = 0.0f;
+        if (tv && nc) {
+          if (et == kZeroTok || S.kq_fmax == kQColZero) {
+            exact = qmask;  // an all-zero token (or basis): every y is +0
+          } else {
+            // the bound at the slice's largest column exponent and 1-norm bound
+            const int32_t f = S.kq_fmax;
+            double E = pow2d(et + f - 58) * kDropUnits + double(S.tok_x1[t]) * (pow2d(f - 30) + pow2d(f - 45)) +
+                       double(S.kq_q1max) * pow2d(et - 30);
+            const double Ma = double(fmaxf(fabsf(mn), fabsf(mx)));
+            const double dl = Ma * 0x1p-21 + pow2d(et + f - 22) + 0x1p-148;
+            E *= 1.0 + 0x1p-40;
+            const double M = Ma * (1.0 + 0x1p-21) + E + dl;
+            const int lm = M > 0.0 ? ilogb(M) : -1000;
+            R = __double2float_ru((E + dl + pow2d(max(lm - 23, -149))) * (1.0 + 0x1p-40));
+            const float two = __fmul_ru(R, 2.0f);
+            const float lo_thr = __fadd_ru(mn, two), hi_thr = __fsub_rd(mx, two);
+            for (uint32_t cc = c0; cc < c1; ++cc) {
+              const float v = S.y[cc * kYStride + t];
+              if (v <= lo_thr || v >= hi_thr) cand |= 1u << (cc - c0);
+            }
+          }
+        }
+        {  // the candidates go to the tile's list (see the block path)
+          const uint32_t n = __popc(cand);
+          if (n) {
+            const uint32_t base = atomicAdd(&S.n_chain, n);
+            const uint32_t fit = base < kChainList ? min(n, kChainList - base) : 0u;
+            for (uint32_t u = 0; u < fit; ++u) {
+              const uint32_t i = __ffs(cand) - 1u;
+              cand &= cand - 1u;
+              S.clist[base + u] = t | ((c0 + i) << 8);
+              exact |= 1u << i;
+            }
+          }
+        }
+        asm volatile("cp.async.wait_group 0;" ::: "memory");  // Q^T rows landed
+        __syncthreads();
+        {  // the listed chains, spread over all threads
+          const uint32_t nl = min(S.n_chain, kChainList);
+          for (uint32_t u = tid; u < nl; u += kPThreads) {
+            const uint32_t e = S.clist[u], tt = e & 0xffu, cc = e >> 8;
+            S.y[cc * kYStride + tt] = exact_y_inl(reinterpret_cast<const float4*>(&S.a[0][0]) + tt * 32u, tt & 7u,
+                                                  reinterpret_cast<const float4*>(&S.b[0][0]) + cc * 32u, cc & 7u);
+          }
+        }
+        __syncthreads();
+        if (tid == 0) S.n_chain = 0;  // for the next tile (read again only after two barriers)
+        const float4* xp = reinterpret_cast<const float4*>(&S.a[0][0]) + t * 32u;
+        while (cand) {  // chains that did not fit the list
+          const uint32_t i = __ffs(cand) - 1u;
+          cand &= cand - 1u;
+          const uint32_t cc = c0 + i;
+          S.y[cc * kYStride + t] =
+              exact_y(xp, t & 7u, reinterpret_cast<const float4*>(&S.b[0][0]) + cc * 32u, cc & 7u);
+          exact |= 1u << i;
+        }
+        // the oracle's scan over the token's coded components, ascending
+        float z = __int_as_float(0x7f800000), zx = __int_as_float(0xff800000);
+        for (uint32_t cc = c0; cc < c1; ++cc) {
+          const float v = S.y[cc * kYStride + t];
+          if (v < z) z = v;
+          if (v > zx) zx = v;
+        }
+#pragma unroll
+        for (uint32_t o = 1; o < 4; o <<= 1) {  // lower quarters first
+          const float pz = __shfl_xor_sync(0xffffffffu, z, o), pzx = __shfl_xor_sync(0xffffffffu, zx, o);
+          if ((q & o) == 0) {
+            if (pz < z) z = pz;
+            if (pzx > zx) zx = pzx;
+          } else {
+            z = z < pz ? z : pz;
+            zx = zx > pzx ? zx : pzx;
+          }
+        }
+        if (tv && nc) {
+          const float rng = __fsub_rn(zx, z);
+          if (q == 0) {
+            uint32_t* zp = reinterpret_cast<uint32_t*>(rec + 8u * (tb + t));
+            zp[0] = __float_as_uint(z);
+            zp[1] = __float_as_uint(zx == z ? 0.0f : rng);
+          }
+          for (uint32_t cc = c0; cc < c1; ++cc) {
+            const uint32_t i = cc - c0, j = S.cidx[cc], bw = S.ci.width[j], levels = (1u << bw) - 1u;
+            const float s = (zx == z) ? 0.0f : __fdiv_rn(rng, float(levels));
+            const float rs = s == 0.0f ? 0.0f : __frcp_rn(s);
+            const bool exact_rs = !(rs < 0x1p126f);
+            const float v = S.y[cc * kYStride + t];
+            uint32_t qv;
+            bool done = false;
+            if (!exact_rs) {  // the distance test of the block path, at this token's bound
+              const float qa = __fmul_rn(__fsub_rn(v, z), rs);
+              const float mg = __fadd_rn(qa, 12582912.0f);
+              const int32_t iq = __float_as_int(mg) - 0x4b400000;
+              const float d = __fsub_rn(0.5f, fabsf(__fsub_rn(qa, __fsub_rn(mg, 12582912.0f))));
+              const float mR = ((exact >> i) & 1u) ? 0.0f : __fmul_ru(__fmul_ru(R, rs), 1.0f + 0x1p-19f);
+              if (d > __fadd_ru(mR, __fmul_ru(fabsf(qa), 0x1p-19f))) {
+                qv = uint32_t(min(max(iq, 0), int32_t(levels)));
+                done = true;
+              }
+            }
+            if (!done) {
+              if ((exact >> i) & 1u) {
+                qv = quantize(v, z, s, levels);
+              } else {
+                const uint32_t q1 = quantize(__fsub_rd(v, R), z, s, levels);
+                const uint32_t q2 = quantize(__fadd_ru(v, R), z, s, levels);
+                qv = q1 == q2 ? q1
+                              : quantize(exact_y(xp, t & 7u, reinterpret_cast<const float4*>(&S.b[0][0]) + cc * 32u,
+                                                 cc & 7u),
+                                         z, s, levels);
+              }
+            }
+            codes[uint64_t(j) * kCodesRow + tb + t] = uint8_t(qv);
+            atomicAdd(&S.hist[levels - 1u + qv], 1u);  // tab_base(b) = 2^b - 2 = levels - 1
+          }
+        }
+      }
       }
       __syncthreads();  // y and the token arrays are rewritten by the next tile
     }
@@ -832,7 +997,11 @@ k_transform_side(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLay
   const uint32_t nb = (tcc + kTile - 1) / kTile;
   uint8_t* rec = ws.slots + uint64_t(r) * ws.slot_bytes;
   uint16_t* scratch = slot_words(rec, ws.slot_bytes);  // variant v's words end at (v + 1) * kSideMax
-  const uint32_t half = __ldg(&pl.comp[sidx].n_coded) * nb, n = 2u * half;
+  // pairs of the record: one per coded component and block, or one per token
+  // for values with per-token ranges
+  const uint32_t n_coded = __ldg(&pl.comp[sidx].n_coded);
+  const bool kiv = sh.kivi && ((sidx / sh.H) & 1u) == 1u;
+  const uint32_t half = n_coded ? (kiv ? tcc : n_coded * nb) : 0u, n = 2u * half;
   if (n == 0) {  // nothing coded: no side streams
     if (tid == 0) ws.rec_len[r] = 0;
     return;
@@ -1499,7 +1668,8 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
     // q, loads its table (into the width streams' table slots, rebuilt only
     // later), copies its bytes to its part of the refill rings (idle until the
     // code streams) and decodes plane q from there.
-    const uint32_t half = S.ci.n_coded * nb, nv = 2u * half;
+    const bool kiv = sh.kivi && ((sidx / sh.H) & 1u) == 1u;  // values with per-token ranges
+    const uint32_t half = S.ci.n_coded ? (kiv ? tcc : S.ci.n_coded * nb) : 0u, nv = 2u * half;
     if (tid == 0) {
       uint32_t o = 0, ok = st == kOk ? 1u : 0u;
       for (uint32_t q = 0; q < 4u && nv && ok; ++q) {
@@ -1549,8 +1719,12 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
           z |= uint32_t(S.side[q][i]) << (8u * q);
           sc |= uint32_t(S.side[q][half + i]) << (8u * q);
         }
-        const uint32_t cc = i / nb, blk = i - cc * nb;
-        zs[cc * (sh.ct / kTile) + blk] = make_float2(__uint_as_float(z), __uint_as_float(sc));
+        if (kiv) {  // (z, range) of token i
+          zs[i] = make_float2(__uint_as_float(z), __uint_as_float(sc));
+        } else {
+          const uint32_t cc = i / nb, blk = i - cc * nb;
+          zs[cc * (sh.ct / kTile) + blk] = make_float2(__uint_as_float(z), __uint_as_float(sc));
+        }
       }
     }
     // code stream records: walk the headers for their offsets, then parse each one
@@ -1644,6 +1818,10 @@ struct __align__(1024) DecSmem {
   // scale and zero point (s, z) of component j in block blk at zsT[j % 8][blk][j / 8]:
   // the 16 threads that share a token read 16 consecutive entries
   float2 zsT[8][kMaxCt / kTile][kD / 8];
+  // values with per-token ranges: each token's zero point, and its range in
+  // 2^b - 1 steps for each width b
+  float kz[kMaxCt];
+  float ks[kMaxCt][8];
   CompInfo ci;
   uint64_t bar;
   uint32_t base[kBatchMax + 1];
@@ -1717,10 +1895,24 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
     }
     // this thread's A-operand components j0 .. j0 + 7 and which of them are coded
     const uint32_t j0 = 8u * (tid & 15u);
-    uint32_t wmask = 0;
+    const bool kiv = sh.kivi && !is_key;  // values with per-token ranges
+    uint32_t wmask = 0, wpack = 0;  // coded components; their widths - 1, 4 bits each
 #pragma unroll
-    for (uint32_t i = 0; i < 8; ++i) wmask |= S.ci.width[j0 + i] ? (1u << i) : 0u;
-    if (tid < kD && S.ci.width[tid]) {  // all of the component's (z, s) pairs are loaded before any is stored
+    for (uint32_t i = 0; i < 8; ++i) {
+      const uint32_t bw = S.ci.width[j0 + i];
+      wmask |= bw ? (1u << i) : 0u;
+      wpack |= (bw ? bw - 1u : 0u) << (4u * i);
+    }
+    if (kiv) {  // each token's zero point and range, decoded from the side streams by the entropy stage
+      const float2* p64 = cb.zs + uint64_t(g) * kD * (sh.ct / kTile);
+      for (uint32_t t = tid; t < tcc; t += nthr) {
+        const float2 zr = __ldg(p64 + t);
+        S.kz[t] = zr.x;
+#pragma unroll
+        for (uint32_t bw = 1; bw <= 8; ++bw)
+          if (S.ci.bcount[bw]) S.ks[t][bw - 1] = zr.y == 0.0f ? 0.0f : __fdiv_rn(zr.y, float((1u << bw) - 1u));
+      }
+    } else if (tid < kD && S.ci.width[tid]) {  // all of the component's (z, s) pairs are loaded before any is stored
       // decoded from the record's side streams by the entropy stage
       const float2* p64 = cb.zs + (uint64_t(g) * kD + S.ci.coded_idx[tid]) * (sh.ct / kTile);
       float2 zs[kMaxCt / kTile];
@@ -1768,7 +1960,8 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
           const uint32_t c4[2] = {cw8[k].x, cw8[k].y};
 #pragma unroll
           for (uint32_t i = 0; i < 8; ++i) {
-            const float2 zs = zr[k >> 2][i];
+            float2 zs = zr[k >> 2][i];
+            if (kiv) zs = make_float2(S.kz[t_base + tt], S.ks[t_base + tt][(wpack >> (4u * i)) & 15u]);
             const float y = __fmaf_rn(float((c4[i >> 2] >> (8u * (i & 3u))) & 0xffu), zs.y, zs.x);
             v[i] = (wmask >> i) & 1u ? y : 0.0f;
           }
