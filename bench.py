@@ -37,27 +37,35 @@ METRIC = "KV codec encode/decode GB/s (raw bytes) vs HBM roofline; compression r
 # raw bytes R, its container bytes C and its middle (transform-coded) values V:
 # bytes for the lossless kernels (raw + container) and for the transform
 # entropy stages (a code byte per middle value + the records), and 2 * 128
-# flops per middle value for the transform contraction (one contraction; the
-# projection kernel runs it in fp64 on the CUDA cores, the decoder in bf16
-# pieces on the tensor cores).
+# flops per middle value for the transform contraction, counted once although
+# the kernels split it into several tensor-core products (ten int8 byte-pair
+# products in the encoder's projection, three bf16 hi/lo products in the
+# decoder). The third field is the dtype whose tensor peak bounds the kernel.
 KERNEL_WORK = {
-    "lossless_encode": ("hbm", lambda R, C, V: R + C),
-    "lossless_decode": ("hbm", lambda R, C, V: R + C),
-    "transform_project": ("alu", lambda R, C, V: 2 * 128 * V),
-    "transform_entropy": ("hbm", lambda R, C, V: V + C),          # codes in, records out
-    "transform_decode_codes": ("hbm", lambda R, C, V: C + V),     # records in, codes out
-    "transform_decode": ("tensor", lambda R, C, V: 2 * 128 * V),
+    "lossless_encode": ("hbm", lambda R, C, V: R + C, None),
+    "lossless_decode": ("hbm", lambda R, C, V: R + C, None),
+    "transform_project": ("tensor", lambda R, C, V: 2 * 128 * V, "i8"),
+    "transform_entropy": ("hbm", lambda R, C, V: V + C, None),          # codes in, records out
+    "transform_decode_codes": ("hbm", lambda R, C, V: C + V, None),     # records in, codes out
+    "transform_decode": ("tensor", lambda R, C, V: 2 * 128 * V, "bf16"),
 }
 
-# DRAM bytes (read + write) per frame of 64 MiB, from an ncu capture of one
-# launch over 4 frames (larger than L2; the traffic of these kernels grows with
-# the frames a launch covers), kept with the profiles of this repository. A
-# kernel that changed after its capture has no entry.
+# Dense tensor peak of a dtype as a multiple of the measured bf16 figure
+# (nominal B200 ratios: int8 and fp8 run at twice the bf16 rate).
+TENSOR_RATIO = {"bf16": 1.0, "i8": 2.0}
+
+# DRAM bytes (read + write) per frame of 64 MiB, from one ncu capture of each
+# kernel over 4 frames (larger than L2; the traffic of these kernels grows
+# with the frames a launch covers). A kernel changed after its capture has no
+# entry.
 DRAM_BYTES_PER_FRAME = {
-    "transform_project": (304.5e6 + 100.5e6) / 4,
-    "transform_decode_codes": (80.0e6 + 109.4e6) / 4,
-    "lossless_decode": (198.8e6 + 220.9e6) / 4,
-    "transform_decode": (199.5e6 + 221.8e6) / 4,
+    "lossless_encode": (756.4e6 + 353.1e6) / 4,
+    "transform_project": (328.3e6 + 106.1e6) / 4,
+    "transform_side": (14.0e6 + 0.0e6) / 4,
+    "transform_entropy": (126.4e6 + 23.1e6) / 4,
+    "lossless_decode": (199.0e6 + 217.0e6) / 4,
+    "transform_decode_codes": (80.2e6 + 103.7e6) / 4,
+    "transform_decode": (199.8e6 + 216.6e6) / 4,
 }
 
 
@@ -493,7 +501,6 @@ def run_kvc(args):
     cont_l, cont_t = sum(job.sizes_l), sum(job.sizes_t)
     value = world * 4 * raw / (ms_step * 1e-3) / 1e9
     hbm_peak, bf16_peak, sm_max, peak_kind = measured_peaks()
-    fp64_peak = 148 * 64 * 2 * sm_max * 1e6 / 1e12  # TFLOP/s, 64 fp64 FMA/clk/SM
     launches = sum(n for n, _ in kernels.values())
     step_cont = {"lossless_encode": cont_l, "lossless_decode": cont_l, "transform_project": cont_t,
                  "transform_entropy": cont_t, "transform_decode_codes": cont_t, "transform_decode": cont_t}
@@ -502,7 +509,7 @@ def run_kvc(args):
     for name, (n, t) in kernels.items():
         entry = {"launches": n, "total_ms": round(t, 3), "share": round(t / total_kern_ms, 4)}
         if name in KERNEL_WORK and n:
-            bound, fn = KERNEL_WORK[name]
+            bound, fn, dt = KERNEL_WORK[name]
             work = fn(raw, step_cont[name], job.mid_vals * job.frames) * args.steps
             secs = t * 1e-3
             if bound == "hbm":
@@ -512,9 +519,9 @@ def run_kvc(args):
                              algorithmic_bytes_per_launch=int(work / n))
             else:
                 ach = work / secs / 1e12
-                peak = fp64_peak if bound == "alu" else bf16_peak
+                peak = bf16_peak * TENSOR_RATIO[dt]
                 entry.update(bound=bound, achieved=round(ach, 3), peak=round(peak, 2),
-                             unit="TFLOP/s", frac=round(ach / peak, 4),
+                             unit="TFLOP/s", frac=round(ach / peak, 4), dtype=dt,
                              algorithmic_flops_per_launch=int(work / n))
         if name in DRAM_BYTES_PER_FRAME and n:
             entry["traffic"] = int(DRAM_BYTES_PER_FRAME[name] * job.frames * args.steps / n)
@@ -525,9 +532,9 @@ def run_kvc(args):
         d = kern_out[dominant]
         roof = {"kernel": dominant, "bound": d["bound"], "achieved": d["achieved"],
                 "peak": d["peak"], "unit": d["unit"], "frac": d["frac"], "traffic": d.get("traffic"),
-                "peak_source": {"hbm": peak_kind + " copy bandwidth",
-                                "tensor": peak_kind + " sustained cuBLAS bf16",
-                                "alu": "derived: 148 SMs x 64 fp64 FMA/clk x 2 x max SM clock"}[d["bound"]]}
+                "peak_source": (peak_kind + " copy bandwidth" if d["bound"] == "hbm" else
+                                peak_kind + " sustained cuBLAS bf16"
+                                + (" x 2 (nominal int8/bf16 ratio)" if d.get("dtype") == "i8" else ""))}
     e2e = None
     if not args.no_e2e:
         e_ms, h2d, d2h = run_e2e(job, max(1, min(args.steps, 3)), 1)
