@@ -171,7 +171,11 @@ __device__ inline int ilog2_u32(uint32_t v) { return 31 - __clz(v); }
 // the whole block; result valid in thread 0. The message is padded in front
 // with zero bytes to whole rounds (a zero-initialised CRC ignores leading
 // zeros); the standard initial value is applied by complementing the first
-// four message bytes, and the final xor at the end.
+// four message bytes, and the final xor at the end. A thread's run is loaded
+// four 16-byte units at a time, so that its loads overlap. kReadOnly: the
+// bytes are not written while the kernel runs, so the loads may allocate in L1
+// (where the caller's later reads of the same record then find them).
+template <bool kReadOnly = false>
 __device__ inline uint32_t crc32_block_aligned(const uint8_t* p, uint32_t len, const uint32_t* t,
                                                uint32_t* red) {
   const uint32_t nthr = blockDim.x;
@@ -182,17 +186,28 @@ __device__ inline uint32_t crc32_block_aligned(const uint8_t* p, uint32_t len, c
   uint32_t acc = 0;
   for (uint32_t r = 0; r < rounds; ++r) {
     acc = gf2_mul(acc, step);
-    int64_t run0 = int64_t(r) * round_bytes + int64_t(threadIdx.x) * kCrcRun - int64_t(pad);
+    const int64_t run0 = int64_t(r) * round_bytes + int64_t(threadIdx.x) * kCrcRun - int64_t(pad);
     uint32_t c = 0;
-    for (uint32_t k = 0; k < kCrcRun; k += 16) {
-      int64_t off = run0 + k;
-      if (off < 0) continue;
-      uint4 v = __ldcg(reinterpret_cast<const uint4*>(p + off));
-      if (off == 0) v.x = ~v.x;
-      c = crc_word(t, c, v.x);
-      c = crc_word(t, c, v.y);
-      c = crc_word(t, c, v.z);
-      c = crc_word(t, c, v.w);
+    if (run0 + int64_t(kCrcRun) > 0) {  // runs wholly inside the padding leave c = 0
+      for (uint32_t k = 0; k < kCrcRun; k += 64) {
+        uint4 v[4];
+#pragma unroll
+        for (uint32_t i = 0; i < 4; ++i) {
+          const int64_t off = run0 + k + 16u * i;
+          const uint4* q = reinterpret_cast<const uint4*>(p + off);
+          v[i] = off < 0 ? make_uint4(0, 0, 0, 0) : kReadOnly ? __ldg(q) : __ldcg(q);
+        }
+#pragma unroll
+        for (uint32_t i = 0; i < 4; ++i) {
+          const int64_t off = run0 + k + 16u * i;
+          if (off < 0) continue;
+          if (off == 0) v[i].x = ~v[i].x;
+          c = crc_word(t, c, v[i].x);
+          c = crc_word(t, c, v[i].y);
+          c = crc_word(t, c, v[i].z);
+          c = crc_word(t, c, v[i].w);
+        }
+      }
     }
     acc ^= c;
   }

@@ -259,7 +259,7 @@ k_lossless_decode(LosslessShape sh, FrameBatch b, uint8_t* ws) {
     const uint8_t* rec = src + off;
     const uint32_t slice = r / sh.cps, c = r % sh.cps;
     const uint32_t t0 = c * sh.tc, tcc = min(sh.tc, sh.T - t0), n = tcc * D;
-    uint32_t got = crc32_block_aligned(rec, len, S.crc_t, S.red);
+    uint32_t got = crc32_block_aligned<true>(rec, len, S.crc_t, S.red);
     if (tid == 0) S.crc_ok = (got == want);
     __syncthreads();
     int st = S.crc_ok ? kOk : kErrCorrupt;
@@ -880,12 +880,11 @@ __device__ inline bool fast_tiles(FastSmem& S, const uint8_t* const recp[2], uin
   constexpr uint32_t RP = (M0 == kModeRans) ? 0u : 1u;  // the rANS plane, if any
   const uint32_t l = threadIdx.x, lane = l & 31u, g = l >> 5;
   const uint32_t lt = lanemask_lt();
-  // Lanes l and l ^ LPC hold neighbouring channels (ch, ch ^ 1) of the same
-  // tokens. Of each pair of steps (j, j + 1) the even channel stores token j
-  // and the odd channel token j + 1, both channels in one 32-bit word.
-  const uint32_t ch = l / LPC, role = ch & 1u;
-  const uint32_t pair_sel = role ? 0x1054u : 0x5410u;
-  uint32_t* o32 = reinterpret_cast<uint32_t*>(out + (uint64_t(l % LPC) * 512u + role) * D + (ch & ~1u));
+  // Lane l decodes channel ch = l / LPC of tokens (l % LPC) * 512 + j and
+  // stores each value as it comes: the warp's 32 lanes write 64 contiguous
+  // bytes of a token row (two rows for D = 64), whole 32-byte sectors.
+  const uint32_t ch = l / LPC;
+  uint16_t* o16 = out + uint64_t(l % LPC) * 512u * D + ch;
   LaneRans rs{kRansLow, 0, 0, S.ring[g]};
   RefillWindow win{nullptr, 0, 0, tc::smem_addr(S.ring[g])};
   const uint8_t* raw0 = recp[0] + 16 + l * 512u;
@@ -933,44 +932,29 @@ __device__ inline bool fast_tiles(FastSmem& S, const uint8_t* const recp[2], uin
         n1b = __ldcg(reinterpret_cast<const uint4*>(raw1 + 32u * (k + 1) + 16u));
       }
     }
-    uint32_t* o = o32 + (k * 32u) * (D / 2u);
-    // four stages of 8 steps; each consumes raw words 0 and 1, then the words shift down
-#pragma unroll 1
+    uint16_t* o = o16 + (k * 32u) * D;
+    // four stages of 8 steps, unrolled so that raw word indices and output
+    // offsets are constants; stage st consumes raw words 2 st and 2 st + 1
+#pragma unroll
     for (uint32_t st = 0; st < 4; ++st) {
       if (kRans) {
         win.settle();
         win.request(rs.pos, lane);
       }
 #pragma unroll
-      for (uint32_t j = 0; j < 8; j += 2) {
-        uint32_t v[2];
-#pragma unroll
-        for (uint32_t h = 0; h < 2; ++h) {
-          const uint32_t jj = j + h;
-          uint32_t e = 0u;
-          if (kRans) {
-            e = rs.step(S.lut, lt) ^ (prev & dm);
-            prev = e;
-          }
-          const uint32_t a = kRaw0 ? r0[jj >> 2] : (M0 == kModeRans ? e : c0);
-          const uint32_t b = kRaw1 ? r1[jj >> 2] : (M1 == kModeRans ? e : c1);
-          v[h] = merge_planes<M0, M1>(jj, a, b);
+      for (uint32_t j = 0; j < 8; ++j) {
+        const uint32_t jj = 8u * st + j;
+        uint32_t e = 0u;
+        if (kRans) {
+          e = rs.step(S.lut, lt) ^ (prev & dm);
+          prev = e;
         }
-        const uint32_t send = role ? v[0] : v[1];
-        const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, LPC);
-        o[j * (D / 2u)] = __byte_perm(role ? v[1] : v[0], recv, pair_sel);
+        const uint32_t a = kRaw0 ? r0[jj >> 2] : (M0 == kModeRans ? e : c0);
+        const uint32_t b = kRaw1 ? r1[jj >> 2] : (M1 == kModeRans ? e : c1);
+        o[jj * D] = uint16_t(merge_planes<M0, M1>(jj, a, b));
       }
-      if (kRaw0) {
-        k0 = crc_word(S.crc_t, crc_word(S.crc_t, k0, r0[0]), r0[1]);
-#pragma unroll
-        for (uint32_t i = 0; i < 6; ++i) r0[i] = r0[i + 2];
-      }
-      if (kRaw1) {
-        k1 = crc_word(S.crc_t, crc_word(S.crc_t, k1, r1[0]), r1[1]);
-#pragma unroll
-        for (uint32_t i = 0; i < 6; ++i) r1[i] = r1[i + 2];
-      }
-      o += 8u * (D / 2u);
+      if (kRaw0) k0 = crc_word(S.crc_t, crc_word(S.crc_t, k0, r0[2 * st]), r0[2 * st + 1]);
+      if (kRaw1) k1 = crc_word(S.crc_t, crc_word(S.crc_t, k1, r1[2 * st]), r1[2 * st + 1]);
     }
   }
   crc0 = k0;
@@ -1277,7 +1261,7 @@ k_lossless_decode_wide(LosslessShape sh, FrameBatch b, uint8_t* ws) {
     const uint32_t slice = r / sh.cps, c = r % sh.cps;
     const uint32_t t0 = c * sh.tc, tcc = min(sh.tc, sh.T - t0), n = tcc * D;
     uint8_t* out = b.f[fr].dst + (uint64_t(slice) * sh.T + t0) * D * E;
-    const uint32_t got = crc32_block_aligned(rec, len, S.crc_t, S.red);
+    const uint32_t got = crc32_block_aligned<true>(rec, len, S.crc_t, S.red);
     if (tid == 0) S.crc_ok = (got == want);
     __syncthreads();
     int st = S.crc_ok ? kOk : kErrCorrupt;

@@ -423,6 +423,9 @@ k_transform_project(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
         }
         tc::mma_commit(&S.bar);
       }
+      // the issuing warp reconverges before it polls the barrier: a suspended poll
+      // of its other lanes would otherwise hold back the issue
+      __syncwarp();
       {  // while the MMAs run: the next 128 tokens' rows (and keys' cos/sin) toward L2
         const uint32_t tn = t0 + tb + kPTok + dt;
         if (tn < sh.r_start) {
@@ -1639,7 +1642,7 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
     const uint8_t* rec = src + off0;
     const uint32_t ls = r / rps, kind = r % rps;
     const uint32_t sidx = ds->first_slice + ls;
-    uint32_t got = crc32_block_aligned(rec, len, S.crc_t, S.red);
+    uint32_t got = crc32_block_aligned<true>(rec, len, S.crc_t, S.red);
     if (tid == 0) S.crc_ok = (got == want);
     __syncthreads();
     int st = S.crc_ok ? kOk : kErrCorrupt;
@@ -1994,6 +1997,7 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
         }
         tc::mma_commit(&S.bar);
       }
+      __syncwarp();  // the issuing warp reconverges before its lanes poll the barrier
       // while the MMAs run: this thread's RoPE pairs for the epilogue (warp w:
       // token rows 32 (w % 4) .., channel pairs 32 (w / 4) .. + 32) and the next
       // tile's codes
