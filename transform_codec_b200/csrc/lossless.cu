@@ -759,9 +759,11 @@ constexpr uint32_t kRawStream = 16u + kMaxChunkValues;  // bytes of a full-chunk
 struct __align__(16) FastSmem {
   uint32_t crc_t[1024];
   uint32_t lut[kProbScale];
-  uint16_t ring[kFastThreads / 32][1024];  // per-group window of rANS refill words
+  union {
+    uint16_t ring[kFastThreads / 32][1024];  // per-group window of rANS refill words
+    uint32_t cum[260];                       // table build scratch; the build ends before any refill
+  };
   uint32_t freq[2][256];
-  uint32_t cum[260];
   uint32_t tmp[32], red[32];
   StreamInfo si[2];
   uint32_t base[kBatchMax + 1];
@@ -987,7 +989,7 @@ __device__ inline uint32_t crc_header16(const uint32_t* t, const uint8_t* h, boo
   return crc_word(t, c, v.w);
 }
 
-__global__ void __launch_bounds__(kFastThreads, 5)
+__global__ void __launch_bounds__(kFastThreads, 6)
 k_lossless_decode_fast(LosslessShape sh, FrameBatch b, uint8_t* ws) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   FastSmem& S = *reinterpret_cast<FastSmem*>(smem_raw);
