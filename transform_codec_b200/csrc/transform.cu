@@ -1351,9 +1351,14 @@ __device__ inline CodeBlocks code_blocks(uint8_t* ws, uint32_t max_records, uint
   return c;
 }
 
+constexpr uint32_t kRingWords = 512;              // refill ring of one warp
+constexpr uint32_t kRingUnits = kRingWords / 8u;  // its 16-byte units
+
 struct __align__(16) DecEntSmem {
-  uint8_t lut[8][kProbScale];          // per width stream: symbol of each slot
-  alignas(16) uint16_t ring[kThreads / 32][1024];  // one refill window per warp (cp.async targets)
+  // per width stream: symbol of each slot. While the side streams are decoded,
+  // slots 0-3 hold their tables and slots 4-5 the four decoded byte planes.
+  uint8_t lut[8][kProbScale];
+  alignas(16) uint16_t ring[kThreads / 32][kRingWords];  // one refill window per warp (cp.async targets)
   uint32_t crc_t[1024];
   uint32_t freq[8][256];               // per width stream; f << 16 | cum after the table build
   uint32_t tmp[32], red[32];
@@ -1362,9 +1367,11 @@ struct __align__(16) DecEntSmem {
   CompInfo ci;
   uint32_t base[kBatchMax + 1];
   uint32_t crc_ok, bad, walk_ok, side_ok;
-  uint8_t side[4][kSideMax];           // the side streams' byte planes of V
   uint32_t side_off[5];                // the side stream records' offsets in the record
 };
+// byte plane q of the side values V (kSideMax bytes each), in table slots 4-5
+__device__ inline uint8_t* side_plane(DecEntSmem& S, uint32_t q) { return &S.lut[4][0] + q * kSideMax; }
+static_assert(4u * kSideMax <= 2u * kProbScale, "the side planes fit two table slots");
 
 // Decode table of one rANS stream built by one warp: freq[256] (validated, sum
 // 4096) becomes freq[s] = f_s << 16 | cum_s, and lut[slot] the symbol whose
@@ -1423,15 +1430,14 @@ __device__ inline void warp_dec_lut8(uint32_t* freq, uint8_t* lut) {
 // components, codes in global memory). The sub-stream (sl bytes at sub,
 // 16-byte aligned) holds the lanes' states, then the refill words. Its 16-byte
 // units, from the one holding the first word on, are copied by cp.async into
-// a 1024-entry ring of 16-bit positions counted from the sub-stream's start
-// (the words begin at position 2 * lanes_g), so no more than the ring's 128
-// units are requested at once: at every stage of 8 steps (at most 256 words
-// consumed) the warp waits for all but the newest copy group and requests
-// units up to 1024 positions past the unit holding the next word, so no unit
-// is overwritten before it is consumed and the coming stage's words were
-// requested a stage earlier. Returns false (on every lane) when a symbol
-// exceeds levels, a lane reads past its sub-stream or the final states and
-// word count do not match.
+// the warp's ring of kRingWords 16-bit positions counted from the sub-stream's
+// start (the words begin at position 2 * lanes_g): at every stage of 8 steps
+// (at most 256 words consumed) the warp waits for all its copies, then
+// requests units up to kRingWords positions past the unit holding the next
+// word. The words of a stage were thus requested a stage earlier, and a unit's
+// ring slot is reused only once every word in it has been consumed. Returns
+// false (on every lane) when a symbol exceeds levels, a lane reads past its
+// sub-stream or the final states and word count do not match.
 __device__ inline bool decode_codes_group(const uint8_t* sub, uint32_t sl, uint32_t n, uint32_t N, uint32_t g,
                                           const uint8_t* lut, const uint32_t* fc, uint16_t* ring, uint8_t* codes,
                                           const uint32_t* comp, uint32_t m, uint32_t tcc, uint32_t levels) {
@@ -1451,20 +1457,19 @@ __device__ inline bool decode_codes_group(const uint8_t* sub, uint32_t sl, uint3
   uint32_t left = tcc - t;                          // steps until the lane moves to the next component
   uint32_t rp = w0, orv = 0;                        // ring position of the next word; OR of the symbols
   const uint32_t n_units = (sl + 15u) >> 4, ring_saddr = static_cast<uint32_t>(__cvta_generic_to_shared(ring));
-  uint32_t loaded = w0 >> 3;  // units wholly inside the states are never needed (and would alias live slots)
+  uint32_t loaded = w0 >> 3;  // units wholly inside the states are never needed
   auto request = [&]() {
-    const uint32_t target = min(n_units, (rp >> 3) + 128u);
+    const uint32_t target = min(n_units, (rp >> 3) + kRingUnits);
     for (uint32_t u = loaded + lane; u < target; u += 32u)
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ring_saddr + ((u & 127u) << 4)),
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ring_saddr + ((u & (kRingUnits - 1u)) << 4)),
                    "l"(sub + (uint64_t(u) << 4))
                    : "memory");
     asm volatile("cp.async.commit_group;" ::: "memory");
     loaded = max(loaded, target);
   };
   request();
-  asm volatile("cp.async.commit_group;" ::: "memory");  // empty group: the first wait covers the window
   for (uint32_t tau0 = 0; tau0 < maxlen; tau0 += 8u) {
-    asm volatile("cp.async.wait_group 1;" ::: "memory");
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncwarp();
     request();
 #pragma unroll
@@ -1486,7 +1491,7 @@ __device__ inline bool decode_codes_group(const uint8_t* sub, uint32_t sl, uint3
       }
       const bool need = act && x < kRansLow;
       const uint32_t mask = __ballot_sync(0xffffffffu, need);
-      const uint32_t w = ring[(rp + __popc(mask & lt)) & 1023u];
+      const uint32_t w = ring[(rp + __popc(mask & lt)) & (kRingWords - 1u)];
       if (need) x = (x << 16) | w;
       rp += __popc(mask);
     }
@@ -1604,11 +1609,11 @@ __device__ inline bool side_decode_group(const uint8_t* sub, uint32_t sl, uint32
   return __all_sync(0xffffffffu, ok);
 }
 
-static_assert(sizeof(DecEntSmem) <= 232448 / 3, "entropy stage should fit three blocks per SM");
+static_assert(sizeof(DecEntSmem) + 1024 <= 233472 / 4, "entropy stage should fit four blocks per SM");
 static_assert(offsetof(DecEntSmem, ring) % 16 == 0 && offsetof(DecEntSmem, lut) % 4 == 0,
               "refill rings take 16-byte copies; the side streams' table reads 4-byte words");
 
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, 4)
 k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t* ws,
                          uint32_t max_records) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
@@ -1694,19 +1699,22 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
         StreamInfo& si = S.si[q];
         okw = warp_parse_side(rec + o, S.side_off[q + 1] - o, nv, side_lanes(nv), si, S.freq[q]) == kOk;
         if (okw) {
-          uint8_t* stage = reinterpret_cast<uint8_t*>(&S.ring[2u * q][0]);  // 4 KiB >= 16 + pad16(kSideMax)
-          uint8_t* plane = S.side[q];
+          // the sub-stream is staged in the rings of warps 2q and 2q + 1: it
+          // starts past the header and table (at least 80 bytes) of a record of at
+          // most 16 + pad16(kSideMax) bytes, so it fits their 2 KiB
+          uint8_t* stage = reinterpret_cast<uint8_t*>(&S.ring[2u * q][0]);
+          uint8_t* plane = side_plane(S, q);
           if (si.mode == kModeRaw) {
             for (uint32_t i = lane; i < nv; i += 32u) plane[i] = __ldg(rec + o + 16u + i);
           } else if (si.mode == kModeConst) {
             for (uint32_t i = lane; i < nv; i += 32u) plane[i] = uint8_t(si.sym);
           } else {
-            for (uint32_t i = lane; i < si.bytes / 16u; i += 32u)
-              reinterpret_cast<uint4*>(stage)[i] = __ldg(reinterpret_cast<const uint4*>(rec + o) + i);
+            const uint4* sub4 = reinterpret_cast<const uint4*>(rec + o + si.sub_off[0]);
+            for (uint32_t i = lane; i < pad16(si.sub_len[0]) / 16u; i += 32u)
+              reinterpret_cast<uint4*>(stage)[i] = __ldg(sub4 + i);
             warp_dec_lut8(S.freq[q], S.lut[q]);
             __syncwarp();
-            okw = side_decode_group(stage + si.sub_off[0], si.sub_len[0], nv, S.lut[q], S.freq[q],
-                                    si.delta ? 0xffu : 0u, plane);
+            okw = side_decode_group(stage, si.sub_len[0], nv, S.lut[q], S.freq[q], si.delta ? 0xffu : 0u, plane);
           }
         }
       }
@@ -1719,8 +1727,8 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
         uint32_t z = 0, sc = 0;
 #pragma unroll
         for (uint32_t q = 0; q < 4; ++q) {
-          z |= uint32_t(S.side[q][i]) << (8u * q);
-          sc |= uint32_t(S.side[q][half + i]) << (8u * q);
+          z |= uint32_t(side_plane(S, q)[i]) << (8u * q);
+          sc |= uint32_t(side_plane(S, q)[half + i]) << (8u * q);
         }
         if (kiv) {  // (z, range) of token i
           zs[i] = make_float2(__uint_as_float(z), __uint_as_float(sc));
