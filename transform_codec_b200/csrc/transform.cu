@@ -1570,6 +1570,94 @@ __device__ inline int warp_parse_side(const uint8_t* rec, uint32_t avail, uint32
   return bad ? kErrCorrupt : kOk;
 }
 
+// Check the width stream record at rec (16-byte aligned, avail bytes from its
+// offset to the end of the record) for n symbols under the code streams' lane
+// rule, with the checks of block_parse_stream (no lane-delta flag), and for
+// RANS load its frequencies into freq[256]. Warp-cooperative; lane 0 fills si;
+// returns the status on every lane.
+__device__ inline int warp_parse_stream(const uint8_t* rec, uint32_t avail, uint32_t n, StreamInfo& si,
+                                        uint32_t* freq) {
+  const uint32_t lane = threadIdx.x & 31u;
+  if (avail < 16u) {
+    if (lane == 0) si.status = kErrCorrupt;
+    __syncwarp();
+    return kErrCorrupt;
+  }
+  const uint4 hv = __ldg(reinterpret_cast<const uint4*>(rec));
+  const uint32_t mode = hv.x & 0xffu, csym = (hv.x >> 8) & 0xffu, G = (hv.x >> 16) & 0xffu, b3 = hv.x >> 24;
+  const uint32_t bytes = hv.y, rn = hv.z, k = hv.w;
+  bool bad = b3 != 0u || rn != n || (bytes & 15u) || bytes < 16u || bytes > avail;
+  uint32_t offs[4] = {0, 0, 0, 0}, lens[4] = {0, 0, 0, 0};
+  if (!bad) {
+    if (mode == kModeRaw) {
+      bad = csym || G || k || bytes != 16u + pad16(n);
+    } else if (mode == kModeConst) {
+      bad = G || k != 1u || bytes != 16u;
+    } else if (mode == kModeRans) {
+      bad = csym || n == 0 || G != rans_groups(rans_lanes(n)) || k < 2u || k > 256u;
+      if (!bad) {
+        const uint32_t lens_at = pad16(48u + 2u * k);
+        uint32_t p = pad16(lens_at + 4u * G);
+        bad = p > bytes;
+        if (!bad) {  // G <= 4 lengths in one aligned 16-byte load
+          const uint4 lv = __ldg(reinterpret_cast<const uint4*>(rec + lens_at));
+          lens[0] = lv.x; lens[1] = lv.y; lens[2] = lv.z; lens[3] = lv.w;
+#pragma unroll
+          for (uint32_t g = 0; g < 4; ++g) {
+            if (g >= G || bad) continue;
+            if (lens[g] > bytes || p + pad16(lens[g]) > bytes) {
+              bad = true;
+            } else {
+              offs[g] = p;
+              p += pad16(lens[g]);
+            }
+          }
+          bad = bad || p != bytes;
+        }
+      }
+    } else {
+      bad = true;
+    }
+  }
+  if (lane == 0) {
+    si.mode = mode; si.sym = csym; si.groups = G; si.bytes = bytes; si.k = k; si.delta = 0;
+#pragma unroll
+    for (uint32_t g = 0; g < 4; ++g) {
+      si.sub_off[g] = offs[g];
+      si.sub_len[g] = g < G ? lens[g] : 0u;
+    }
+  }
+  if (!bad && mode == kModeRans) {
+    // presence bitmap byte `lane` covers symbols 8 lane .. 8 lane + 7
+    const uint32_t bm = rec[16u + lane];
+    const uint32_t cnt = __popc(bm);
+    uint32_t incl = cnt;
+#pragma unroll
+    for (uint32_t o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t total = __shfl_sync(0xffffffffu, incl, 31);
+    uint32_t idx = incl - cnt, fs = 0;
+    bool zero = false;
+#pragma unroll
+    for (uint32_t i = 0; i < 8; ++i) {
+      uint32_t f = 0;
+      if (total == k && ((bm >> i) & 1u)) {
+        f = ld_u16(rec + 48u + 2u * idx++);
+        zero |= f == 0;
+      }
+      freq[8u * lane + i] = f;
+      fs += f;
+    }
+    fs = __reduce_add_sync(0xffffffffu, fs);
+    bad = total != k || __any_sync(0xffffffffu, zero) || fs != kProbScale;
+  }
+  if (lane == 0) si.status = bad ? kErrCorrupt : kOk;
+  __syncwarp();
+  return bad ? kErrCorrupt : kOk;
+}
+
 // rANS decode of a side stream's single group by one warp (lanes l < N <= 32,
 // the side lane rule) from the sub-stream copied to shared memory (sl bytes at
 // sub, 4-byte aligned): byte table lut, f << 16 | cum per symbol in fc; dm =
@@ -1671,11 +1759,14 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
     const uint32_t t0 = sh.s_end + c * sh.ct, tcc = min(sh.ct, sh.r_start - t0);
     const uint32_t nb = (tcc + kTile - 1) / kTile;
     load_comp_info(pl.comp + sidx, S.ci);
-    // side information: four byte-plane streams of V = every z, then every s.
-    // One thread walks their headers for the offsets; warp q then checks stream
-    // q, loads its table (into the width streams' table slots, rebuilt only
-    // later), copies its bytes to its part of the refill rings (idle until the
-    // code streams) and decodes plane q from there.
+    // Stream headers. One thread walks the side streams' headers (side
+    // information: four byte-plane streams of V = every z, then every s) and
+    // then the width streams' for their offsets. Warp q < 4 then checks side
+    // stream q, loads its table (into width-stream table slot q, rebuilt only
+    // later), copies its sub-stream to the rings of warps 2q and 2q + 1 (idle
+    // until the width streams) and decodes plane q from there, while warps 4-7
+    // check the headers and frequencies of width streams 5-8; warps 0-3 then
+    // check width streams 1-4 while the block assembles the (z, s) pairs.
     const bool kiv = sh.kivi && ((sidx / sh.H) & 1u) == 1u;  // values with per-token ranges
     const uint32_t half = S.ci.n_coded ? (kiv ? tcc : S.ci.n_coded * nb) : 0u, nv = 2u * half;
     if (tid == 0) {
@@ -1688,13 +1779,22 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
         o += bytes;
       }
       S.side_off[4] = nv ? o : 0u;
-      S.side_ok = ok;
+      for (uint32_t bw = 1; bw <= 8 && ok; ++bw) {
+        if (!S.ci.bcount[bw]) continue;
+        S.str_off[bw - 1] = o;
+        if (o + 16u > len) { ok = 0; break; }
+        const uint32_t bytes = ld_u32(rec + o + 4);
+        if (bytes < 16u || (bytes & 15u) || bytes > len - o) { ok = 0; break; }
+        o += bytes;
+      }
+      S.walk_ok = ok && o == len;
+      S.bad = 0;
     }
     __syncthreads();
-    if (st == kOk && !S.side_ok) st = kErrCorrupt;
-    if (st == kOk && nv) {
+    if (st == kOk && !S.walk_ok) st = kErrCorrupt;
+    if (st == kOk) {
       bool okw = true;
-      if (warp < 4) {
+      if (warp < 4 && nv) {
         const uint32_t q = warp, o = S.side_off[q];
         StreamInfo& si = S.si[q];
         okw = warp_parse_side(rec + o, S.side_off[q + 1] - o, nv, side_lanes(nv), si, S.freq[q]) == kOk;
@@ -1717,48 +1817,36 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
             okw = side_decode_group(stage, si.sub_len[0], nv, S.lut[q], S.freq[q], si.delta ? 0xffu : 0u, plane);
           }
         }
+      } else if (warp >= 4 && S.ci.bcount[warp + 1]) {
+        const uint32_t o = S.str_off[warp];
+        okw = warp_parse_stream(rec + o, len - o, S.ci.bcount[warp + 1] * tcc, S.si[warp], S.freq[warp]) == kOk;
       }
       if (!__syncthreads_and(okw)) st = kErrCorrupt;
     }
-    const uint32_t o_side = st == kOk ? S.side_off[4] : 0u;
-    if (st == kOk && nv) {
-      float2* zs = cb.zs + uint64_t(g) * kD * (sh.ct / kTile);
-      for (uint32_t i = tid; i < half; i += nthr) {
-        uint32_t z = 0, sc = 0;
+    if (st == kOk) {
+      bool okw = true;
+      if (warp < 4 && S.ci.bcount[warp + 1]) {
+        const uint32_t o = S.str_off[warp];
+        okw = warp_parse_stream(rec + o, len - o, S.ci.bcount[warp + 1] * tcc, S.si[warp], S.freq[warp]) == kOk;
+      }
+      if (nv) {
+        float2* zs = cb.zs + uint64_t(g) * kD * (sh.ct / kTile);
+        for (uint32_t i = tid; i < half; i += nthr) {
+          uint32_t z = 0, sc = 0;
 #pragma unroll
-        for (uint32_t q = 0; q < 4; ++q) {
-          z |= uint32_t(side_plane(S, q)[i]) << (8u * q);
-          sc |= uint32_t(side_plane(S, q)[half + i]) << (8u * q);
-        }
-        if (kiv) {  // (z, range) of token i
-          zs[i] = make_float2(__uint_as_float(z), __uint_as_float(sc));
-        } else {
-          const uint32_t cc = i / nb, blk = i - cc * nb;
-          zs[cc * (sh.ct / kTile) + blk] = make_float2(__uint_as_float(z), __uint_as_float(sc));
+          for (uint32_t q = 0; q < 4; ++q) {
+            z |= uint32_t(side_plane(S, q)[i]) << (8u * q);
+            sc |= uint32_t(side_plane(S, q)[half + i]) << (8u * q);
+          }
+          if (kiv) {  // (z, range) of token i
+            zs[i] = make_float2(__uint_as_float(z), __uint_as_float(sc));
+          } else {
+            const uint32_t cc = i / nb, blk = i - cc * nb;
+            zs[cc * (sh.ct / kTile) + blk] = make_float2(__uint_as_float(z), __uint_as_float(sc));
+          }
         }
       }
-    }
-    // code stream records: walk the headers for their offsets, then parse each one
-    if (tid == 0) {
-      uint32_t o = o_side, ok = st == kOk ? 1u : 0u;
-      for (uint32_t bw = 1; bw <= 8 && ok; ++bw) {
-        if (!S.ci.bcount[bw]) continue;
-        S.str_off[bw - 1] = o;
-        if (o + 16u > len) { ok = 0; break; }
-        const uint32_t bytes = ld_u32(rec + o + 4);
-        if (bytes < 16u || (bytes & 15u) || bytes > len - o) { ok = 0; break; }
-        o += bytes;
-      }
-      S.walk_ok = ok && o == len;
-      S.bad = 0;
-    }
-    __syncthreads();
-    if (st == kOk && !S.walk_ok) st = kErrCorrupt;
-    for (uint32_t bw = 1; bw <= 8 && st == kOk; ++bw) {
-      const uint32_t m = S.ci.bcount[bw];
-      if (!m) continue;
-      const uint32_t o = S.str_off[bw - 1];
-      st = block_parse_stream(rec + o, len - o, m * tcc, &S.si[bw - 1], S.freq[bw - 1], S.tmp, false);
+      if (!__syncthreads_and(okw)) st = kErrCorrupt;
     }
     if (st != kOk) {
       if (tid == 0) {
