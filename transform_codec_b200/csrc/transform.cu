@@ -1354,6 +1354,16 @@ __device__ inline CodeBlocks code_blocks(uint8_t* ws, uint32_t max_records, uint
 constexpr uint32_t kRingWords = 512;              // refill ring of one warp
 constexpr uint32_t kRingUnits = kRingWords / 8u;  // its 16-byte units
 
+// A rANS group of a record's width stream, placed in a warp: lanes base ..
+// base + lanes - 1 of the warp decode it, through ring_words refill words at
+// ring_off of the block's ring area.
+struct PackEntry {
+  uint16_t sw, gg, base, lanes, ring_off, ring_words;
+};
+// At most 11 groups: sum over widths of ceil(lanes / 32) with at most 128
+// lanes in all is at most 128 / 32 + 8 * 31 / 32 < 12.
+constexpr uint32_t kMaxGroupsRec = 12;
+
 struct __align__(16) DecEntSmem {
   // per width stream: symbol of each slot. While the side streams are decoded,
   // slots 0-3 hold their tables and slots 4-5 the four decoded byte planes.
@@ -1368,6 +1378,8 @@ struct __align__(16) DecEntSmem {
   uint32_t base[kBatchMax + 1];
   uint32_t crc_ok, bad, walk_ok, side_ok;
   uint32_t side_off[5];                // the side stream records' offsets in the record
+  PackEntry pk[kMaxGroupsRec];         // the record's rANS groups, by warp (first pk_first[w])
+  uint32_t pk_first[9];
 };
 // byte plane q of the side values V (kSideMax bytes each), in table slots 4-5
 __device__ inline uint8_t* side_plane(DecEntSmem& S, uint32_t q) { return &S.lut[4][0] + q * kSideMax; }
@@ -1425,50 +1437,82 @@ __device__ inline void warp_dec_lut8(uint32_t* freq, uint8_t* lut) {
   __syncwarp();
 }
 
-// rANS decode of group g of one width stream by one warp: n symbols on N
-// lanes; symbol i = a * tcc + t is written to codes[t * 128 + comp[a]] (m
-// components, codes in global memory). The sub-stream (sl bytes at sub,
-// 16-byte aligned) holds the lanes' states, then the refill words. Its 16-byte
-// units, from the one holding the first word on, are copied by cp.async into
-// the warp's ring of kRingWords 16-bit positions counted from the sub-stream's
-// start (the words begin at position 2 * lanes_g): at every stage of 8 steps
-// (at most 256 words consumed) the warp waits for all its copies, then
-// requests units up to kRingWords positions past the unit holding the next
-// word. The words of a stage were thus requested a stage earlier, and a unit's
-// ring slot is reused only once every word in it has been consumed. Returns
-// false (on every lane) when a symbol exceeds levels, a lane reads past its
-// sub-stream or the final states and word count do not match.
-__device__ inline bool decode_codes_group(const uint8_t* sub, uint32_t sl, uint32_t n, uint32_t N, uint32_t g,
-                                          const uint8_t* lut, const uint32_t* fc, uint16_t* ring, uint8_t* codes,
-                                          const uint32_t* comp, uint32_t m, uint32_t tcc, uint32_t levels) {
+// rANS decode of the groups packed into one warp (entries pe[0 .. ne - 1]).
+// Group g of width stream sw holds lanes g * 32 .. of the stream's N lanes (n
+// symbols); symbol i = a * tcc + t of the stream is written to codes[t * 128 +
+// comp[a]] (codes in global memory). Each lane decodes its group's lane; the
+// group's lanes of the ballot (mask gm) order its refill words. A group's
+// sub-stream (sl bytes, 16-byte aligned) holds its lanes' states, then the
+// refill words; its 16-byte units, from the one holding the first word on, are
+// copied by cp.async into the group's ring of ring_words 16-bit positions
+// counted from the sub-stream's start (the words begin at position 2 * lanes):
+// at every stage of 8 steps (at most 8 words per lane consumed, half the ring)
+// the warp waits for all its copies, then requests units up to ring_words
+// positions past the unit holding the group's next word. The words of a stage
+// were thus requested a stage earlier, and a unit's ring slot is reused only
+// once every word in it has been consumed. Lanes outside every group idle.
+// Returns false (on every lane) when a group's sub-stream cannot hold its
+// states, a symbol exceeds its width's levels, a lane reads past its
+// sub-stream, or the final states and word counts do not match.
+template <class Smem>
+__device__ inline bool decode_codes_packed(Smem& S, const PackEntry* pe, uint32_t ne, const uint8_t* rec,
+                                           uint8_t* codes, uint32_t tcc) {
   const uint32_t lane = threadIdx.x & 31u;
-  const uint32_t lanes_g = min(kGroupLanes, N - g * kGroupLanes);
-  if (sl < 4u * lanes_g || ((sl - 4u * lanes_g) & 1u)) return false;
-  const uint32_t W = (sl - 4u * lanes_g) >> 1, w0 = 2u * lanes_g;
-  const bool live = lane < lanes_g;
-  uint32_t start = 0, len = 0, start0, maxlen;
-  if (live) lane_range(n, N, g * kGroupLanes + lane, start, len);
-  lane_range(n, N, g * kGroupLanes, start0, maxlen);
   const uint32_t lt = lanemask_lt();
-  uint32_t x = live ? reinterpret_cast<const uint32_t*>(sub)[lane] : kRansLow;
+  int me = -1;
+  for (uint32_t i = 0; i < ne; ++i)
+    if (lane >= pe[i].base && lane < pe[i].base + pe[i].lanes) me = int(i);
+  bool live = me >= 0, ok = true;
+  uint32_t sw = 1, gg = 0, li = 0, lanes_g = 1, rw = 16, roff = 0;
+  if (live) {
+    sw = pe[me].sw;
+    gg = pe[me].gg;
+    li = lane - pe[me].base;
+    lanes_g = pe[me].lanes;
+    rw = pe[me].ring_words;
+    roff = pe[me].ring_off;
+  }
+  const uint32_t m = live ? S.ci.bcount[sw] : 1u, n = m * tcc, N = rans_lanes(n), levels = (1u << sw) - 1u;
+  const uint32_t sl = live ? S.si[sw - 1].sub_len[gg] : 0u;
+  const uint8_t* sub = live ? rec + S.str_off[sw - 1] + S.si[sw - 1].sub_off[gg] : rec;
+  if (live && (sl < 4u * lanes_g || ((sl - 4u * lanes_g) & 1u))) {
+    ok = false;
+    live = false;
+  }
+  const uint32_t W = live ? (sl - 4u * lanes_g) >> 1 : 0u, w0 = 2u * lanes_g;
+  uint32_t start = 0, len = 0, start0 = 0, gmax = 0;
+  if (live) {
+    lane_range(n, N, gg * kGroupLanes + li, start, len);
+    lane_range(n, N, gg * kGroupLanes, start0, gmax);
+  }
+  const uint32_t wmax = __reduce_max_sync(0xffffffffu, live ? gmax : 0u);
+  const uint32_t gm = live ? (lanes_g == 32u ? 0xffffffffu : ((1u << lanes_g) - 1u) << pe[me].base) : 0u;
+  const uint8_t* lut = &S.lut[live ? sw - 1 : 0][0];
+  const uint32_t* fc = &S.freq[live ? sw - 1 : 0][0];
+  const uint16_t* ring = &S.ring[0][0] + roff;
+  const uint32_t ring_saddr = static_cast<uint32_t>(__cvta_generic_to_shared(ring)), runits = rw >> 3;
+  uint32_t x = live ? reinterpret_cast<const uint32_t*>(sub)[li] : kRansLow;
   uint32_t a = start / tcc, t = start - a * tcc;
+  const uint32_t* comp = S.ci.comp + S.ci.bstart[sw];
   uint32_t j = (live && len && a < m) ? comp[a] : 0u;
   uint8_t* cp = codes + uint64_t(t) * kCodeRow + j;  // this lane's next code
   uint32_t left = tcc - t;                          // steps until the lane moves to the next component
-  uint32_t rp = w0, orv = 0;                        // ring position of the next word; OR of the symbols
-  const uint32_t n_units = (sl + 15u) >> 4, ring_saddr = static_cast<uint32_t>(__cvta_generic_to_shared(ring));
+  uint32_t rp = w0, orv = 0;                        // ring position of the group's next word; OR of the symbols
+  const uint32_t n_units = (sl + 15u) >> 4;
   uint32_t loaded = w0 >> 3;  // units wholly inside the states are never needed
   auto request = [&]() {
-    const uint32_t target = min(n_units, (rp >> 3) + kRingUnits);
-    for (uint32_t u = loaded + lane; u < target; u += 32u)
-      asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ring_saddr + ((u & (kRingUnits - 1u)) << 4)),
-                   "l"(sub + (uint64_t(u) << 4))
-                   : "memory");
+    if (live) {
+      const uint32_t target = min(n_units, (rp >> 3) + runits);
+      for (uint32_t u = loaded + li; u < target; u += lanes_g)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ring_saddr + ((u & (runits - 1u)) << 4)),
+                     "l"(sub + (uint64_t(u) << 4))
+                     : "memory");
+      loaded = max(loaded, target);
+    }
     asm volatile("cp.async.commit_group;" ::: "memory");
-    loaded = max(loaded, target);
   };
   request();
-  for (uint32_t tau0 = 0; tau0 < maxlen; tau0 += 8u) {
+  for (uint32_t tau0 = 0; tau0 < wmax; tau0 += 8u) {
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     __syncwarp();
     request();
@@ -1490,16 +1534,15 @@ __device__ inline bool decode_codes_group(const uint8_t* sub, uint32_t sl, uint3
         }
       }
       const bool need = act && x < kRansLow;
-      const uint32_t mask = __ballot_sync(0xffffffffu, need);
-      const uint32_t w = ring[(rp + __popc(mask & lt)) & (kRingWords - 1u)];
+      const uint32_t mask = __ballot_sync(0xffffffffu, need) & gm;
+      const uint32_t w = ring[(rp + __popc(mask & lt)) & (rw - 1u)];
       if (need) x = (x << 16) | w;
       rp += __popc(mask);
     }
   }
-  const uint32_t pos = rp - w0, bad = (orv & ~levels) != 0u;
   asm volatile("cp.async.wait_group 0;" ::: "memory");
   __syncwarp();
-  const bool ok = !bad && pos == W && x == kRansLow;
+  ok = ok && (!live || ((orv & ~levels) == 0u && rp - w0 == W && x == kRansLow));
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -1877,26 +1920,58 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
         if (bad) S.bad = 1;
       }
     }
-    // rANS streams: warp w builds the table of width w + 1, then one warp per
-    // (stream, group) decodes
+    // rANS streams: warp w builds the table of width w + 1 while one thread
+    // packs the record's groups into warps (first fit, larger groups first:
+    // with at most 128 lanes in groups of at most 32 this never needs more
+    // than eight warps) and gives each group a ring of 16 words per lane
+    // (rounded up to a power of two; 4096 words at most); then each warp
+    // decodes its groups side by side
     if (S.ci.bcount[warp + 1] && S.si[warp].mode == kModeRans) warp_dec_lut8(S.freq[warp], S.lut[warp]);
-    __syncthreads();
-    {
-      uint32_t pair = 0;
+    if (tid == 0) {
+      PackEntry gl[kMaxGroupsRec];
+      uint32_t ng = 0;
       for (uint32_t sw = 1; sw <= 8; ++sw) {
         const uint32_t m = S.ci.bcount[sw];
         if (!m || S.si[sw - 1].mode != kModeRans) continue;
-        const uint32_t n = m * tcc, N = rans_lanes(n), G = rans_groups(N);
-        const StreamInfo& si = S.si[sw - 1];
-        for (uint32_t gg = 0; gg < G; ++gg, ++pair) {
-          if (pair % (nthr >> 5) != warp) continue;
-          const bool ok = decode_codes_group(rec + S.str_off[sw - 1] + si.sub_off[gg], si.sub_len[gg], n, N, gg,
-                                             S.lut[sw - 1], S.freq[sw - 1], S.ring[warp], codes,
-                                             S.ci.comp + S.ci.bstart[sw], m, tcc, (1u << sw) - 1u);
-          if (!ok && lane == 0) S.bad = 1;
+        const uint32_t N = rans_lanes(m * tcc), G = rans_groups(N);
+        for (uint32_t gg = 0; gg < G && ng < kMaxGroupsRec; ++gg) {
+          const uint32_t ln = min(kGroupLanes, N - gg * kGroupLanes);
+          uint32_t i = ng++;  // insertion by lanes, descending
+          while (i > 0 && gl[i - 1].lanes < ln) {
+            gl[i] = gl[i - 1];
+            --i;
+          }
+          gl[i].sw = uint16_t(sw);
+          gl[i].gg = uint16_t(gg);
+          gl[i].lanes = uint16_t(ln);
         }
       }
+      uint32_t fill[8] = {0, 0, 0, 0, 0, 0, 0, 0}, bin[kMaxGroupsRec], roff = 0;
+      for (uint32_t i = 0; i < ng; ++i) {
+        uint32_t bsel = 0;
+        while (bsel < 7u && fill[bsel] + gl[i].lanes > kGroupLanes) ++bsel;
+        bin[i] = bsel;
+        gl[i].base = uint16_t(fill[bsel]);
+        fill[bsel] += gl[i].lanes;
+        uint32_t rw = 16u;
+        while (rw < 16u * gl[i].lanes) rw <<= 1;
+        gl[i].ring_words = uint16_t(rw);
+        gl[i].ring_off = uint16_t(roff);
+        roff += rw;
+      }
+      uint32_t k = 0;
+      for (uint32_t w = 0; w < 8; ++w) {
+        S.pk_first[w] = k;
+        for (uint32_t i = 0; i < ng; ++i)
+          if (bin[i] == w) S.pk[k++] = gl[i];
+      }
+      S.pk_first[8] = k;
     }
+    __syncthreads();
+    if (S.pk_first[warp + 1] > S.pk_first[warp] &&
+        !decode_codes_packed(S, S.pk + S.pk_first[warp], S.pk_first[warp + 1] - S.pk_first[warp], rec, codes, tcc) &&
+        lane == 0)
+      S.bad = 1;
     __syncthreads();
     if (tid == 0) {
       if (S.bad) atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(kErrCorrupt));
