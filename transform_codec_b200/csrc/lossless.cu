@@ -3,6 +3,7 @@
 // stream record that keeps the smallest of CONST / RANS / RAW (AT-1 Memory
 // page, "KV & tensor mode": channel-major reorder, byte planes, keep whichever
 // is smaller; QATQ page, "qatq encode": bounded chunks, known row width).
+#include <type_traits>
 #include "kvc_device.cuh"
 #include "tcgen05.cuh"
 #include "kvc_internal.h"
@@ -417,7 +418,7 @@ __device__ __forceinline__ uint32_t lds_u16(const uint8_t* p) {
 }
 
 template <uint32_t D>
-__global__ void __launch_bounds__(kFencThreads, 8)
+__global__ void __launch_bounds__(kFencThreads, 9)
 k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
   constexpr uint32_t TCC = kMaxChunkValues / D, LPC = 128u / D;
   constexpr uint32_t CB = D / 8u;                       // 16-byte column blocks of a token row
@@ -540,28 +541,45 @@ k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
     constexpr uint32_t kStages = 512u / kFencStage;
     issue(kStages - 1);
     issue(kStages - 2);
-    uint32_t vcur = 0;
+    // the chains a chunk codes are fixed before the loop: one instance of the
+    // loop per combination, so that no step branches on them
+    auto chains = [&](auto E0, auto E1, auto E2) {
+      constexpr bool e0 = decltype(E0)::value, e1 = decltype(E1)::value, e2 = decltype(E2)::value;
+      uint32_t vcur = 0;
 #pragma unroll 1
-    for (int s = int(kStages) - 1; s >= 0; --s) {
-      __syncwarp();  // every lane is done with the slot the next copy overwrites
-      if (s >= 2) issue(uint32_t(s) - 2u);
-      else asm volatile("cp.async.commit_group;" ::: "memory");
-      asm volatile("cp.async.wait_group 1;" ::: "memory");  // stages s and s - 1 landed
-      __syncwarp();
-      const uint8_t* cur = ring + (uint32_t(s) % kFencSlots) * kFencSlotBytes + loff;
-      const uint8_t* prv = ring + ((uint32_t(s) + kFencSlots - 1u) % kFencSlots) * kFencSlotBytes + loff;
-      if (s == int(kStages) - 1) vcur = lds_u16(cur + (kFencStage - 1u) * kFencRowBytes);
+      for (int s = int(kStages) - 1; s >= 0; --s) {
+        __syncwarp();  // every lane is done with the slot the next copy overwrites
+        if (s >= 2) issue(uint32_t(s) - 2u);
+        else asm volatile("cp.async.commit_group;" ::: "memory");
+        asm volatile("cp.async.wait_group 1;" ::: "memory");  // stages s and s - 1 landed
+        __syncwarp();
+        const uint8_t* cur = ring + (uint32_t(s) % kFencSlots) * kFencSlotBytes + loff;
+        const uint8_t* prv = ring + ((uint32_t(s) + kFencSlots - 1u) % kFencSlots) * kFencSlotBytes + loff;
+        if (s == int(kStages) - 1) vcur = lds_u16(cur + (kFencStage - 1u) * kFencRowBytes);
 #pragma unroll
-      for (int j = int(kFencStage) - 1; j >= 0; --j) {
-        // the value one step earlier in the lane (0 before the lane's first)
-        const uint32_t vprev = j ? lds_u16(cur + uint32_t(j - 1) * kFencRowBytes)
-                                 : (s ? lds_u16(prv + (kFencStage - 1u) * kFencRowBytes) : 0u);
-        const uint32_t hb = vcur >> 8;
-        if (en0) fenc_step(S.tab[0], vcur & 0xffu, x0, p0, sc0, lt);
-        if (en1) fenc_step(S.tab[1], hb, x1, p1, sc1, lt);
-        if (en2) fenc_step(S.tab[2], hb ^ (vprev >> 8), x2, p2, sc2, lt);
-        vcur = vprev;
+        for (int j = int(kFencStage) - 1; j >= 0; --j) {
+          // the value one step earlier in the lane (0 before the lane's first)
+          const uint32_t vprev = j ? lds_u16(cur + uint32_t(j - 1) * kFencRowBytes)
+                                   : (s ? lds_u16(prv + (kFencStage - 1u) * kFencRowBytes) : 0u);
+          const uint32_t hb = vcur >> 8;
+          if constexpr (e0) fenc_step(S.tab[0], vcur & 0xffu, x0, p0, sc0, lt);
+          if constexpr (e1) fenc_step(S.tab[1], hb, x1, p1, sc1, lt);
+          if constexpr (e2) fenc_step(S.tab[2], hb ^ (vprev >> 8), x2, p2, sc2, lt);
+          vcur = vprev;
+        }
       }
+    };
+    using T1 = std::true_type;
+    using F0 = std::false_type;
+    if (en2) {  // en2 implies en1
+      if (en0) chains(T1{}, T1{}, T1{});
+      else chains(F0{}, T1{}, T1{});
+    } else if (en1) {
+      if (en0) chains(T1{}, T1{}, F0{});
+      else chains(F0{}, T1{}, F0{});
+    } else {
+      if (en0) chains(T1{}, F0{}, F0{});
+      else chains(F0{}, F0{}, F0{});
     }
     asm volatile("cp.async.wait_group 0;" ::: "memory");
     S.states[0][tid] = x0;
