@@ -1118,6 +1118,66 @@ k_transform_side(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLay
 // otherwise symbol by symbol. The record is then laid out and written stream
 // by stream.
 
+// A rANS group of a record's width stream, placed in a warp: lanes base ..
+// base + lanes - 1 of the warp code it (the decoder gives it ring_words refill
+// words at ring_off of the block's ring area).
+struct PackEntry {
+  uint16_t sw, gg, base, lanes, ring_off, ring_words;
+};
+// At most 11 groups: sum over widths of ceil(lanes / 32) with at most 128
+// lanes in all is at most 128 / 32 + 8 * 31 / 32 < 12.
+constexpr uint32_t kMaxGroupsRec = 12;
+
+// Packing of a record's rANS groups into warps, by one thread: the groups of
+// every width stream sw with bit sw - 1 of rans set (one per 32 of its lanes),
+// first fit into warps of 32 lanes, larger groups first. With at most 128
+// lanes in groups of at most 32 this never needs more than eight warps: a
+// group of at most 16 lanes opens a new warp only when every open warp holds
+// more than 16, and groups of more than 16 lanes number at most 7. Each group
+// gets a ring of 16 words per lane rounded up to a power of two (4096 words at
+// most in all). Entries are listed by warp: warp w's are pk[first[w] ..
+// first[w + 1]).
+__device__ inline void pack_groups(const CompInfo& ci, uint32_t rans, uint32_t tcc, PackEntry* pk, uint32_t* first) {
+  PackEntry gl[kMaxGroupsRec];
+  uint32_t ng = 0;
+  for (uint32_t sw = 1; sw <= 8; ++sw) {
+    const uint32_t m = ci.bcount[sw];
+    if (!m || !((rans >> (sw - 1)) & 1u)) continue;
+    const uint32_t N = rans_lanes(m * tcc), G = rans_groups(N);
+    for (uint32_t gg = 0; gg < G && ng < kMaxGroupsRec; ++gg) {
+      const uint32_t ln = min(kGroupLanes, N - gg * kGroupLanes);
+      uint32_t i = ng++;  // insertion by lanes, descending
+      while (i > 0 && gl[i - 1].lanes < ln) {
+        gl[i] = gl[i - 1];
+        --i;
+      }
+      gl[i].sw = uint16_t(sw);
+      gl[i].gg = uint16_t(gg);
+      gl[i].lanes = uint16_t(ln);
+    }
+  }
+  uint32_t fill[8] = {0, 0, 0, 0, 0, 0, 0, 0}, bin[kMaxGroupsRec], roff = 0;
+  for (uint32_t i = 0; i < ng; ++i) {
+    uint32_t bsel = 0;
+    while (bsel < 7u && fill[bsel] + gl[i].lanes > kGroupLanes) ++bsel;
+    bin[i] = bsel;
+    gl[i].base = uint16_t(fill[bsel]);
+    fill[bsel] += gl[i].lanes;
+    uint32_t rw = 16u;
+    while (rw < 16u * gl[i].lanes) rw <<= 1;
+    gl[i].ring_words = uint16_t(rw);
+    gl[i].ring_off = uint16_t(roff);
+    roff += rw;
+  }
+  uint32_t k = 0;
+  for (uint32_t w = 0; w < 8; ++w) {
+    first[w] = k;
+    for (uint32_t i = 0; i < ng; ++i)
+      if (bin[i] == w) pk[k++] = gl[i];
+  }
+  first[8] = k;
+}
+
 struct __align__(16) EntSmem {
   uint32_t freq[8][256];                 // per width stream, zero past its alphabet
   uint2 tab[kTabPool];                   // per symbol of each width stream: {f | cum << 16, 1/f}
@@ -1128,6 +1188,8 @@ struct __align__(16) EntSmem {
   uint32_t crc_t[1024];
   uint32_t tmp[32], red[32];
   CompInfo ci;
+  PackEntry pk[kMaxGroupsRec];           // the record's rANS groups, by warp (first pk_first[w])
+  uint32_t pk_first[9];
 };
 
 // rANS encode of one group (warp-synchronous) of a stream in which lane l
@@ -1151,6 +1213,42 @@ __device__ inline uint32_t rans_encode_rows(const uint8_t* row, bool live, const
       const uint32_t f = e.x & 0xffffu, cum = e.x >> 16;
       const bool emit = live && x >= (f << 20);
       const uint32_t mask = __ballot_sync(0xffffffffu, emit);
+      pos -= __popc(mask);
+      if (emit) words[pos + __popc(mask & lt)] = uint16_t(x & 0xffffu);
+      const uint32_t xe = emit ? (x >> 16) : x;
+      uint32_t q = __umulhi(xe, e.y);
+      uint32_t r = xe - q * f;
+      const bool over = r >= f;
+      q += over ? 1u : 0u;
+      r -= over ? f : 0u;
+      x = live ? (q << kProbBits) + r + cum : x;
+    }
+    cur = nxt;
+    nxt = nn;
+  }
+  *x_out = x;
+  return cap - pos;
+}
+
+// The same for the groups packed into one warp: the lanes of a group (mask gm)
+// order its words and share its position; returns the group's word count.
+__device__ inline uint32_t rans_encode_rows_packed(const uint8_t* row, bool live, const uint2* tab, uint16_t* words,
+                                                   uint32_t cap, uint32_t gm, uint32_t* x_out) {
+  const uint32_t lt = lanemask_lt();
+  const uint4* r4 = reinterpret_cast<const uint4*>(row);
+  const uint4 z4 = make_uint4(0, 0, 0, 0);
+  uint4 cur = live ? __ldcg(r4 + 31) : z4, nxt = live ? __ldcg(r4 + 30) : z4;
+  uint32_t x = kRansLow, pos = cap;
+#pragma unroll 1
+  for (int c = 31; c >= 0; --c) {
+    const uint4 nn = (live && c >= 2) ? __ldcg(r4 + (c - 2)) : z4;
+    const uint32_t w[4] = {cur.x, cur.y, cur.z, cur.w};
+#pragma unroll
+    for (int i = 15; i >= 0; --i) {
+      const uint2 e = tab[(w[i >> 2] >> (8 * (i & 3))) & 0xffu];
+      const uint32_t f = e.x & 0xffffu, cum = e.x >> 16;
+      const bool emit = live && x >= (f << 20);
+      const uint32_t mask = __ballot_sync(0xffffffffu, emit) & gm;
       pos -= __popc(mask);
       if (emit) words[pos + __popc(mask & lt)] = uint16_t(x & 0xffffu);
       const uint32_t xe = emit ? (x >> 16) : x;
@@ -1210,6 +1308,42 @@ k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
     }
   }
   __syncthreads();
+  if (tcc == kMaxCt) {
+    // ---- full chunk (lane l of a stream: component l, all 512 tokens): the
+    // rANS groups packed into warps
+    if (tid == 0) {
+      uint32_t rans = 0;
+      for (uint32_t bw = 1; bw <= 8; ++bw)
+        if (S.ci.bcount[bw] && S.k[bw - 1] >= 2) rans |= 1u << (bw - 1);
+      pack_groups(S.ci, rans, tcc, S.pk, S.pk_first);
+    }
+    __syncthreads();
+    const uint32_t e0 = S.pk_first[warp], e1 = S.pk_first[warp + 1];
+    if (e1 > e0) {
+      int me = -1;
+      for (uint32_t i = e0; i < e1; ++i)
+        if (lane >= S.pk[i].base && lane < S.pk[i].base + S.pk[i].lanes) me = int(i);
+      const bool live = me >= 0;
+      const PackEntry pe = S.pk[live ? me : e0];
+      const uint32_t bw = pe.sw, g = pe.gg, li = lane - pe.base;
+      const uint32_t m = S.ci.bcount[bw], n = m * tcc, base = S.ci.bstart[bw];
+      const uint32_t N = rans_lanes(n), G = rans_groups(N);
+      uint32_t b0, len0, b1 = n, len1;
+      lane_range(n, N, g * kGroupLanes, b0, len0);
+      if (g + 1 < G) lane_range(n, N, (g + 1) * kGroupLanes, b1, len1);
+      const uint32_t wbase = base * tcc;  // word scratch of this stream: one word per symbol
+      const uint32_t l = g * kGroupLanes + li;
+      const uint32_t gm = live ? (pe.lanes == 32u ? 0xffffffffu : ((1u << pe.lanes) - 1u) << pe.base) : 0u;
+      uint32_t x;
+      const uint32_t Wg = rans_encode_rows_packed(codes_g + uint64_t(live ? S.ci.comp[base + l] : 0u) * kCodesRow, live,
+                                                  S.tab + tab_base(bw), scratch + wbase + b0, b1 - b0, gm, &x);
+      if (live) S.states[bw - 1][l] = x;
+      if (live && li == 0) {
+        S.W[bw - 1][g] = Wg;
+        S.wbeg[bw - 1][g] = wbase + b1 - Wg;
+      }
+    }
+  } else {
   // ---- rANS groups of every stream, one warp per (stream, group)
   {
     uint32_t pair = 0;
@@ -1242,6 +1376,7 @@ k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
         }
       }
     }
+  }
   }
   __syncthreads();
   // ---- layout: modes and record offsets
@@ -1353,16 +1488,6 @@ __device__ inline CodeBlocks code_blocks(uint8_t* ws, uint32_t max_records, uint
 
 constexpr uint32_t kRingWords = 512;              // refill ring of one warp
 constexpr uint32_t kRingUnits = kRingWords / 8u;  // its 16-byte units
-
-// A rANS group of a record's width stream, placed in a warp: lanes base ..
-// base + lanes - 1 of the warp decode it, through ring_words refill words at
-// ring_off of the block's ring area.
-struct PackEntry {
-  uint16_t sw, gg, base, lanes, ring_off, ring_words;
-};
-// At most 11 groups: sum over widths of ceil(lanes / 32) with at most 128
-// lanes in all is at most 128 / 32 + 8 * 31 / 32 < 12.
-constexpr uint32_t kMaxGroupsRec = 12;
 
 struct __align__(16) DecEntSmem {
   // per width stream: symbol of each slot. While the side streams are decoded,
@@ -1921,51 +2046,14 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
       }
     }
     // rANS streams: warp w builds the table of width w + 1 while one thread
-    // packs the record's groups into warps (first fit, larger groups first:
-    // with at most 128 lanes in groups of at most 32 this never needs more
-    // than eight warps) and gives each group a ring of 16 words per lane
-    // (rounded up to a power of two; 4096 words at most); then each warp
-    // decodes its groups side by side
+    // packs the record's groups into warps (pack_groups), each with its own
+    // refill ring; then each warp decodes its groups side by side
     if (S.ci.bcount[warp + 1] && S.si[warp].mode == kModeRans) warp_dec_lut8(S.freq[warp], S.lut[warp]);
     if (tid == 0) {
-      PackEntry gl[kMaxGroupsRec];
-      uint32_t ng = 0;
-      for (uint32_t sw = 1; sw <= 8; ++sw) {
-        const uint32_t m = S.ci.bcount[sw];
-        if (!m || S.si[sw - 1].mode != kModeRans) continue;
-        const uint32_t N = rans_lanes(m * tcc), G = rans_groups(N);
-        for (uint32_t gg = 0; gg < G && ng < kMaxGroupsRec; ++gg) {
-          const uint32_t ln = min(kGroupLanes, N - gg * kGroupLanes);
-          uint32_t i = ng++;  // insertion by lanes, descending
-          while (i > 0 && gl[i - 1].lanes < ln) {
-            gl[i] = gl[i - 1];
-            --i;
-          }
-          gl[i].sw = uint16_t(sw);
-          gl[i].gg = uint16_t(gg);
-          gl[i].lanes = uint16_t(ln);
-        }
-      }
-      uint32_t fill[8] = {0, 0, 0, 0, 0, 0, 0, 0}, bin[kMaxGroupsRec], roff = 0;
-      for (uint32_t i = 0; i < ng; ++i) {
-        uint32_t bsel = 0;
-        while (bsel < 7u && fill[bsel] + gl[i].lanes > kGroupLanes) ++bsel;
-        bin[i] = bsel;
-        gl[i].base = uint16_t(fill[bsel]);
-        fill[bsel] += gl[i].lanes;
-        uint32_t rw = 16u;
-        while (rw < 16u * gl[i].lanes) rw <<= 1;
-        gl[i].ring_words = uint16_t(rw);
-        gl[i].ring_off = uint16_t(roff);
-        roff += rw;
-      }
-      uint32_t k = 0;
-      for (uint32_t w = 0; w < 8; ++w) {
-        S.pk_first[w] = k;
-        for (uint32_t i = 0; i < ng; ++i)
-          if (bin[i] == w) S.pk[k++] = gl[i];
-      }
-      S.pk_first[8] = k;
+      uint32_t rans = 0;
+      for (uint32_t sw = 1; sw <= 8; ++sw)
+        if (S.ci.bcount[sw] && S.si[sw - 1].mode == kModeRans) rans |= 1u << (sw - 1);
+      pack_groups(S.ci, rans, tcc, S.pk, S.pk_first);
     }
     __syncthreads();
     if (S.pk_first[warp + 1] > S.pk_first[warp] &&
