@@ -2093,7 +2093,9 @@ struct __align__(1024) DecSmem {
 static_assert(sizeof(DecSmem) + 1024 <= 232448, "decoder shared memory exceeds the per-block limit");
 static_assert(sizeof(EntSmem) + 1024 <= 233472 / 5, "entropy kernel should fit five blocks per SM");
 
-__global__ void __launch_bounds__(kThreads, 1)
+constexpr uint32_t kTThreads = 512;  // tensor stage: 16 warps, four per tensor-memory lane quarter
+
+__global__ void __launch_bounds__(kTThreads, 1)
 k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t* ws, uint32_t max_records) {
   extern __shared__ __align__(16) uint8_t smem_raw[];
   // the swizzled operand tiles need 1024-byte-aligned shared addresses
@@ -2187,18 +2189,18 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
     // inverse projection on the tensor cores, 128 tokens at a time:
     // x^[t][k] = sum_j y^[t][j] Q[k][j] with y^ and Q split into bf16 hi + lo
     // pieces (hi*hi + hi*lo + lo*hi, fp32 accumulation in tensor memory).
-    // Item k of this thread: token tt = tid / 16 + 16 k, components j0 .. j0 + 7
+    // Item k of this thread: token tt = tid / 16 + 32 k, components j0 .. j0 + 7
     // (the same for all its items) -> one 16-byte chunk of each piece. A tile's
     // codes are loaded while the previous tile's products run (the first tile's
     // here), so that their latency overlaps the tensor cores and the epilogue.
-    constexpr uint32_t kItems = kTcRows * (kD / 8u) / kThreads;
-    static_assert(kItems == 8 && kTcRows == 2 * kTile, "item k lies in the tile's block k / 4");
+    constexpr uint32_t kItems = kTcRows * (kD / 8u) / kTThreads;
+    static_assert(kItems == 4 && kTcRows == 2 * kTile, "item k lies in the tile's block k / 2");
     uint2 cw8[kItems];
     auto load_codes = [&](uint32_t tb) {
       const uint32_t n = min(kTcRows, tcc - tb);
 #pragma unroll
       for (uint32_t k = 0; k < kItems; ++k) {
-        const uint32_t tt = (tid >> 4) + 16u * k;
+        const uint32_t tt = (tid >> 4) + 32u * k;
         cw8[k] = tt < n ? __ldcg(reinterpret_cast<const uint2*>(codes + (tb + tt) * kCodeRow + j0)) : make_uint2(0, 0);
       }
     };
@@ -2214,7 +2216,7 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
         for (uint32_t i = 0; i < 8; ++i) zr[b2][i] = S.zsT[i][t_base / kTile + b2][tid & 15u];
 #pragma unroll
       for (uint32_t k = 0; k < kItems; ++k) {
-        const uint32_t tt = (tid >> 4) + 16u * k;
+        const uint32_t tt = (tid >> 4) + 32u * k;
         float v[8];
 #pragma unroll
         for (uint32_t i = 0; i < 8; ++i) v[i] = 0.0f;
@@ -2222,7 +2224,7 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
           const uint32_t c4[2] = {cw8[k].x, cw8[k].y};
 #pragma unroll
           for (uint32_t i = 0; i < 8; ++i) {
-            float2 zs = zr[k >> 2][i];
+            float2 zs = zr[k >> 1][i];
             if (kiv) zs = make_float2(S.kz[t_base + tt], S.ks[t_base + tt][(wpack >> (4u * i)) & 15u]);
             const float y = __fmaf_rn(float((c4[i >> 2] >> (8u * (i & 3u))) & 0xffu), zs.y, zs.x);
             v[i] = (wmask >> i) & 1u ? y : 0.0f;
@@ -2258,15 +2260,15 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
       }
       __syncwarp();  // the issuing warp reconverges before its lanes poll the barrier
       // while the MMAs run: this thread's RoPE pairs for the epilogue (warp w:
-      // token rows 32 (w % 4) .., channel pairs 32 (w / 4) .. + 32) and the next
+      // token rows 32 (w % 4) .., channel pairs 16 (w / 4) .. + 16) and the next
       // tile's codes
-      float4 rp[16];
+      float4 rp[8];
       {
         const uint32_t ptt = (warp & 3u) * 32u + lane;
-        const float4* cs4 = reinterpret_cast<const float4*>(pl.rope + (uint64_t(t0 + t_base + ptt) * (kD / 2) + (warp >> 2) * 32u) * 2u);
+        const float4* cs4 = reinterpret_cast<const float4*>(pl.rope + (uint64_t(t0 + t_base + ptt) * (kD / 2) + (warp >> 2) * 16u) * 2u);
         const bool rl = is_key && ptt < bl;
 #pragma unroll
-        for (uint32_t i = 0; i < 16; ++i) rp[i] = rl ? __ldg(cs4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (uint32_t i = 0; i < 8; ++i) rp[i] = rl ? __ldg(cs4 + i) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
       if (t_base + kTcRows < tcc) load_codes(t_base + kTcRows);
       const bool done = tc::mbar_wait(&S.bar, phase, KVC_MMA_WAIT_POLLS);
@@ -2280,24 +2282,22 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
         break;
       }
       tc::fence_after_sync();
-      // epilogue: warp w reads token rows 32 (w % 4) .., channel quarter (w / 4):
-      // channels [32q, 32q + 32) and their RoPE partners [32q + 64, 32q + 96)
+      // epilogue: warp w reads token rows 32 (w % 4) .., channel sixteenth w / 4:
+      // channels [16q, 16q + 16) and their RoPE partners [16q + 64, 16q + 80)
       {
         const uint32_t sub = warp & 3u, q = warp >> 2;
         const uint32_t tt = sub * 32u + lane;
-        const uint32_t c0 = q * 32u;
-        uint32_t va[32], vb[32];
+        const uint32_t c0 = q * 16u;
+        uint32_t va[16], vb[16];
         const uint32_t ta = tmem + ((sub * 32u) << 16);
         tc::tmem_ld16(ta + c0, va);
-        tc::tmem_ld16(ta + c0 + 16u, va + 16);
         tc::tmem_ld16(ta + c0 + 64u, vb);
-        tc::tmem_ld16(ta + c0 + 80u, vb + 16);
         tc::tmem_wait_ld();
         if (tt < bl) {
           const uint32_t t = t0 + t_base + tt;
-          uint32_t pa[16], pb[16];
+          uint32_t pa[8], pb[8];
 #pragma unroll
-          for (uint32_t i = 0; i < 32; i += 2) {
+          for (uint32_t i = 0; i < 16; i += 2) {
             float a0 = __uint_as_float(va[i]), b0 = __uint_as_float(vb[i]);
             float a1 = __uint_as_float(va[i + 1]), b1 = __uint_as_float(vb[i + 1]);
             if (is_key) {
@@ -2314,11 +2314,10 @@ k_transform_decode(TransformShape sh, TransformPlanDev pl, FrameBatch b, uint8_t
           }
           uint4* ra = reinterpret_cast<uint4*>(xs + uint64_t(t) * kD + c0);
           uint4* rb = reinterpret_cast<uint4*>(xs + uint64_t(t) * kD + c0 + 64u);
-#pragma unroll
-          for (uint32_t v = 0; v < 4; ++v) {
-            ra[v] = make_uint4(pa[4 * v], pa[4 * v + 1], pa[4 * v + 2], pa[4 * v + 3]);
-            rb[v] = make_uint4(pb[4 * v], pb[4 * v + 1], pb[4 * v + 2], pb[4 * v + 3]);
-          }
+          ra[0] = make_uint4(pa[0], pa[1], pa[2], pa[3]);
+          ra[1] = make_uint4(pa[4], pa[5], pa[6], pa[7]);
+          rb[0] = make_uint4(pb[0], pb[1], pb[2], pb[3]);
+          rb[1] = make_uint4(pb[4], pb[5], pb[6], pb[7]);
         }
       }
       tc::fence_before_sync();
@@ -2420,7 +2419,7 @@ cudaError_t launch_transform_decode(const TransformShape& s, const TransformPlan
   {
     ProfRange pr_("transform_decode", st);
     const uint32_t grid = min(max_records, uint32_t(num_sms()));
-    k_transform_decode<<<grid, kThreads, smem, st>>>(s, p, b, ws, max_records);
+    k_transform_decode<<<grid, kTThreads, smem, st>>>(s, p, b, ws, max_records);
   }
   return cudaGetLastError();
 }
