@@ -342,3 +342,45 @@ def test_fixed_basis_container_equals_oracle_bytes(kind):
     ost, oy = oracle.decode_transform(oplan, got)
     assert ost == oracle.OK
     assert rel_rms(y, oy) < REL_RMS
+
+
+def _width_mix(counts, seed):
+    """A width per component with counts[b] components of width b (b = 1..8,
+    the rest 0), assigned in a seeded random order."""
+    ws = np.concatenate([np.full(c, b, np.int32) for b, c in counts.items()])
+    ws = np.concatenate([ws, np.zeros(128 - ws.size, np.int32)])
+    return np.random.default_rng(seed).permutation(ws)
+
+
+# Width mixes that drive the packing of a record's rANS groups into warps to
+# its extremes: eleven groups (the most 128 components can make), seven groups
+# of 17 lanes (one warp each, the largest ring space), four full groups of one
+# width, and a scatter of small groups.
+WIDTH_MIXES = {
+    "eleven-groups": {1: 33, 2: 33, 3: 33, 4: 1, 5: 1, 6: 1, 7: 1, 8: 25},
+    "groups-of-17": {1: 17, 2: 17, 3: 17, 4: 17, 5: 17, 6: 17, 7: 17, 8: 9},
+    "one-width": {3: 128},
+    "small-groups": {1: 3, 2: 5, 4: 2, 6: 1, 8: 1},
+}
+
+
+@pytest.mark.parametrize("mix", sorted(WIDTH_MIXES))
+def test_packed_rans_groups_extreme_width_mixes(mix):
+    """Full chunks (512 tokens) and a ragged one (380): the containers equal the
+    oracle's byte for byte, and the GPU decoder restores the oracle's values
+    within the reconstruction bar."""
+    w = _w(n_tokens=1024)
+    bases, _, _ = _small_inputs(w)
+    widths = np.stack([_width_mix(WIDTH_MIXES[mix], 100 + s) for s in range(w.n_slices)]).astype(np.uint8)
+    plan, oplan = _plans(w, bases, widths)
+    x = kvgen.slices(w)
+    st, got = encode(plan, kvc.TRANSFORM, x)
+    assert st == kvc.OK
+    want = oracle.encode_transform(oplan, x)
+    assert got == want
+    st, y = decode(plan, kvc.TRANSFORM, want, w.n_slices)
+    assert st == kvc.OK
+    ost, oy = oracle.decode_transform(oplan, want)
+    assert ost == oracle.OK
+    for s in range(w.n_slices):
+        assert rel_rms(y[s], oy[s]) <= REL_RMS
