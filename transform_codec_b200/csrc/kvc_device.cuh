@@ -141,28 +141,41 @@ __device__ inline uint32_t crc_byte(const uint32_t* t, uint32_t crc, uint32_t b)
   return (crc >> 8) ^ t[(crc ^ b) & 0xffu];
 }
 
-// Join per-thread raw CRCs (thread order = message order) into thread 0's
-// value. red must hold blockDim.x / 32 words. blockDim.x is a power of two.
+// x^(8 kCrcRun d) mod P for d < 1024: the factor that carries the register of
+// a run of kCrcRun bytes past d further runs.
+struct CrcRunPow {
+  uint32_t v[1024];
+};
+constexpr CrcRunPow make_crc_run_pow() {
+  CrcRunPow t{};
+  const uint32_t step = gf2_xpow8(kCrcRun);
+  uint32_t p = 0x80000000u;
+  for (int d = 0; d < 1024; ++d) {
+    t.v[d] = p;
+    p = gf2_mul(p, step);
+  }
+  return t;
+}
+__device__ const CrcRunPow kCrcRunPow = make_crc_run_pow();
+
+// Join per-thread raw CRCs (thread order = message order, one run of kCrcRun
+// bytes per thread) into thread 0's value: crc(A B) = crc(A) x^(8|B|) + crc(B),
+// so each register is carried past the runs after it by one multiplication
+// (in parallel; zero registers need none) and the products are summed by
+// exclusive or. red must hold blockDim.x / 32 words.
 __device__ inline uint32_t crc_block_join(uint32_t c, uint32_t* red) {
   const uint32_t lane = threadIdx.x & 31u, warp = threadIdx.x >> 5;
   const uint32_t nwarps = blockDim.x >> 5;
-#pragma unroll
-  for (int l = 0; l < 5; ++l) {
-    uint32_t other = __shfl_down_sync(0xffffffffu, c, 1u << l);
-    if ((lane & ((2u << l) - 1u)) == 0) c = gf2_mul(c, kCrcShift.v[l]) ^ other;
-  }
+  if (c) c = gf2_mul(c, __ldg(&kCrcRunPow.v[blockDim.x - 1u - threadIdx.x]));
+  c = __reduce_xor_sync(0xffffffffu, c);
   __syncthreads();
   if (lane == 0) red[warp] = c;
   __syncthreads();
-  if (warp == 0) {
-    c = lane < nwarps ? red[lane] : 0u;
-    for (int l = 0; (1u << l) < nwarps; ++l) {
-      uint32_t other = __shfl_down_sync(0xffffffffu, c, 1u << l);
-      if ((lane & ((2u << l) - 1u)) == 0) c = gf2_mul(c, kCrcShift.v[5 + l]) ^ other;
-    }
-  }
+  uint32_t total = 0;
+  if (threadIdx.x == 0)
+    for (uint32_t w = 0; w < nwarps; ++w) total ^= red[w];
   __syncthreads();
-  return c;  // valid in thread 0
+  return total;  // valid in thread 0
 }
 
 __device__ inline int ilog2_u32(uint32_t v) { return 31 - __clz(v); }
@@ -185,7 +198,7 @@ __device__ inline uint32_t crc32_block_aligned(const uint8_t* p, uint32_t len, c
   const uint32_t step = kCrcShift.v[ilog2_u32(nthr)];
   uint32_t acc = 0;
   for (uint32_t r = 0; r < rounds; ++r) {
-    acc = gf2_mul(acc, step);
+    if (acc) acc = gf2_mul(acc, step);
     const int64_t run0 = int64_t(r) * round_bytes + int64_t(threadIdx.x) * kCrcRun - int64_t(pad);
     uint32_t c = 0;
     if (run0 + int64_t(kCrcRun) > 0) {  // runs wholly inside the padding leave c = 0
@@ -229,7 +242,7 @@ __device__ inline uint32_t crc32_block_bytes(Fetch fetch, uint64_t len, const ui
   const uint32_t step = kCrcShift.v[ilog2_u32(nthr)];
   uint32_t acc = 0;
   for (uint64_t r = 0; r < rounds; ++r) {
-    acc = gf2_mul(acc, step);
+    if (acc) acc = gf2_mul(acc, step);
     int64_t run0 = int64_t(r * round_bytes) + int64_t(threadIdx.x) * kCrcRun - int64_t(pad);
     uint32_t c = 0;
     for (uint32_t k = 0; k < kCrcRun; ++k) {

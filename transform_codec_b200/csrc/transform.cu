@@ -1487,7 +1487,6 @@ __device__ inline CodeBlocks code_blocks(uint8_t* ws, uint32_t max_records, uint
 }
 
 constexpr uint32_t kRingWords = 512;              // refill ring of one warp
-constexpr uint32_t kRingUnits = kRingWords / 8u;  // its 16-byte units
 
 struct __align__(16) DecEntSmem {
   // per width stream: symbol of each slot. While the side streams are decoded,
@@ -1579,7 +1578,7 @@ __device__ inline void warp_dec_lut8(uint32_t* freq, uint8_t* lut) {
 // Returns false (on every lane) when a group's sub-stream cannot hold its
 // states, a symbol exceeds its width's levels, a lane reads past its
 // sub-stream, or the final states and word counts do not match.
-template <class Smem>
+template <bool kFull, class Smem>
 __device__ inline bool decode_codes_packed(Smem& S, const PackEntry* pe, uint32_t ne, const uint8_t* rec,
                                            uint8_t* codes, uint32_t tcc) {
   const uint32_t lane = threadIdx.x & 31u;
@@ -1652,10 +1651,12 @@ __device__ inline bool decode_codes_packed(Smem& S, const PackEntry* pe, uint32_
         orv |= sym;
         *cp = uint8_t(sym);
         cp += kCodeRow;
-        if (--left == 0u) {
-          ++a;
-          cp = codes + (a < m ? comp[a] : 0u);
-          left = tcc;
+        if constexpr (!kFull) {  // a full chunk's lane is one component: it never moves on
+          if (--left == 0u) {
+            ++a;
+            cp = codes + (a < m ? comp[a] : 0u);
+            left = tcc;
+          }
         }
       }
       const bool need = act && x < kRansLow;
@@ -2048,18 +2049,22 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
     // rANS streams: warp w builds the table of width w + 1 while one thread
     // packs the record's groups into warps (pack_groups), each with its own
     // refill ring; then each warp decodes its groups side by side
-    if (S.ci.bcount[warp + 1] && S.si[warp].mode == kModeRans) warp_dec_lut8(S.freq[warp], S.lut[warp]);
-    if (tid == 0) {
-      uint32_t rans = 0;
-      for (uint32_t sw = 1; sw <= 8; ++sw)
-        if (S.ci.bcount[sw] && S.si[sw - 1].mode == kModeRans) rans |= 1u << (sw - 1);
-      pack_groups(S.ci, rans, tcc, S.pk, S.pk_first);
-    }
+    uint32_t rans = 0;  // width streams with rANS groups
+    for (uint32_t sw = 1; sw <= 8; ++sw)
+      if (S.ci.bcount[sw] && S.si[sw - 1].mode == kModeRans) rans |= 1u << (sw - 1);
+    if ((rans >> warp) & 1u) warp_dec_lut8(S.freq[warp], S.lut[warp]);
+    // the packing runs in a warp that builds no table (the highest such warp;
+    // warp 0 after its table when every width has one)
+    const uint32_t pw = rans == 0xffu ? 0u : 31u - __clz(~rans & 0xffu);
+    if (warp == pw && lane == 0) pack_groups(S.ci, rans, tcc, S.pk, S.pk_first);
     __syncthreads();
-    if (S.pk_first[warp + 1] > S.pk_first[warp] &&
-        !decode_codes_packed(S, S.pk + S.pk_first[warp], S.pk_first[warp + 1] - S.pk_first[warp], rec, codes, tcc) &&
-        lane == 0)
-      S.bad = 1;
+    if (S.pk_first[warp + 1] > S.pk_first[warp]) {
+      const PackEntry* pe = S.pk + S.pk_first[warp];
+      const uint32_t ne = S.pk_first[warp + 1] - S.pk_first[warp];
+      const bool ok = tcc == kMaxCt ? decode_codes_packed<true>(S, pe, ne, rec, codes, tcc)
+                                    : decode_codes_packed<false>(S, pe, ne, rec, codes, tcc);
+      if (!ok && lane == 0) S.bad = 1;
+    }
     __syncthreads();
     if (tid == 0) {
       if (S.bad) atomicMin(&ds->err_key, (static_cast<unsigned long long>(r) << 8) | unsigned(kErrCorrupt));
