@@ -556,7 +556,7 @@ k_lossless_encode_fast(LosslessShape sh, FrameBatch b, EncodeLayout ws) {
         const uint8_t* cur = ring + (uint32_t(s) % kFencSlots) * kFencSlotBytes + loff;
         const uint8_t* prv = ring + ((uint32_t(s) + kFencSlots - 1u) % kFencSlots) * kFencSlotBytes + loff;
         if (s == int(kStages) - 1) vcur = lds_u16(cur + (kFencStage - 1u) * kFencRowBytes);
-#pragma unroll 8
+#pragma unroll 4
         for (int j = int(kFencStage) - 1; j >= 0; --j) {
           // the value one step earlier in the lane (0 before the lane's first)
           const uint32_t vprev = j ? lds_u16(cur + uint32_t(j - 1) * kFencRowBytes)
