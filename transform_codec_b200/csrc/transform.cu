@@ -1128,54 +1128,85 @@ struct PackEntry {
 // lanes in all is at most 128 / 32 + 8 * 31 / 32 < 12.
 constexpr uint32_t kMaxGroupsRec = 12;
 
-// Packing of a record's rANS groups into warps, by one thread: the groups of
+// Packing of a record's rANS groups into warps, by one warp: the groups of
 // every width stream sw with bit sw - 1 of rans set (one per 32 of its lanes),
-// first fit into warps of 32 lanes, larger groups first. With at most 128
-// lanes in groups of at most 32 this never needs more than eight warps: a
-// group of at most 16 lanes opens a new warp only when every open warp holds
-// more than 16, and groups of more than 16 lanes number at most 7. Each group
-// gets a ring of 16 words per lane rounded up to a power of two (4096 words at
-// most in all). Entries are listed by warp: warp w's are pk[first[w] ..
-// first[w + 1]).
-__device__ inline void pack_groups(const CompInfo& ci, uint32_t rans, uint32_t tcc, PackEntry* pk, uint32_t* first) {
-  PackEntry gl[kMaxGroupsRec];
-  uint32_t ng = 0;
-  for (uint32_t sw = 1; sw <= 8; ++sw) {
-    const uint32_t m = ci.bcount[sw];
-    if (!m || !((rans >> (sw - 1)) & 1u)) continue;
+// first fit into warps of 32 lanes, larger groups first (ties in stream
+// order). With at most 128 lanes in groups of at most 32 this never needs more
+// than eight warps: a group of at most 16 lanes opens a new warp only when
+// every open warp holds more than 16, and groups of more than 16 lanes number
+// at most 7. Each group gets a ring of 16 words per lane rounded up to a power
+// of two (4096 words at most in all). Entries are listed by warp: warp w's are
+// pk[first[w] .. first[w + 1]). Lane i handles group i; the eight fills live
+// in every lane's registers.
+__device__ inline void warp_pack_groups(const CompInfo& ci, uint32_t rans, uint32_t tcc, PackEntry* pk,
+                                        uint32_t* first) {
+  const uint32_t lane = threadIdx.x & 31u;
+  uint32_t sw = 0, gg = 0, L = 0, ng = 0;
+  for (uint32_t b = 1; b <= 8; ++b) {
+    const uint32_t m = ci.bcount[b];
+    if (!m || !((rans >> (b - 1)) & 1u)) continue;
     const uint32_t N = rans_lanes(m * tcc), G = rans_groups(N);
-    for (uint32_t gg = 0; gg < G && ng < kMaxGroupsRec; ++gg) {
-      const uint32_t ln = min(kGroupLanes, N - gg * kGroupLanes);
-      uint32_t i = ng++;  // insertion by lanes, descending
-      while (i > 0 && gl[i - 1].lanes < ln) {
-        gl[i] = gl[i - 1];
-        --i;
-      }
-      gl[i].sw = uint16_t(sw);
-      gl[i].gg = uint16_t(gg);
-      gl[i].lanes = uint16_t(ln);
+    if (lane >= ng && lane < ng + G) {
+      sw = b;
+      gg = lane - ng;
+      L = min(kGroupLanes, N - gg * kGroupLanes);
     }
+    ng += G;
   }
-  uint32_t fill[8] = {0, 0, 0, 0, 0, 0, 0, 0}, bin[kMaxGroupsRec], roff = 0;
-  for (uint32_t i = 0; i < ng; ++i) {
-    uint32_t bsel = 0;
-    while (bsel < 7u && fill[bsel] + gl[i].lanes > kGroupLanes) ++bsel;
-    bin[i] = bsel;
-    gl[i].base = uint16_t(fill[bsel]);
-    fill[bsel] += gl[i].lanes;
-    uint32_t rw = 16u;
-    while (rw < 16u * gl[i].lanes) rw <<= 1;
-    gl[i].ring_words = uint16_t(rw);
-    gl[i].ring_off = uint16_t(roff);
+  const bool item = lane < ng;
+  uint32_t rank = 0;  // position in the order: larger groups first, ties in stream order
+  for (uint32_t j = 0; j < ng; ++j) {
+    const uint32_t Lj = __shfl_sync(0xffffffffu, L, j);
+    rank += (Lj > L || (Lj == L && j < lane)) ? 1u : 0u;
+  }
+  uint32_t fill[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  uint32_t bin = 0, base = 0, my_roff = 0, my_rw = 0, roff = 0;
+  for (uint32_t r = 0; r < ng; ++r) {
+    const uint32_t src = __ffs(__ballot_sync(0xffffffffu, item && rank == r)) - 1u;
+    const uint32_t Lr = __shfl_sync(0xffffffffu, L, src);
+    uint32_t bb = 7u;
+#pragma unroll
+    for (int q = 6; q >= 0; --q)
+      if (fill[q] + Lr <= kGroupLanes) bb = uint32_t(q);
+    uint32_t at = 0;
+#pragma unroll
+    for (uint32_t q = 0; q < 8; ++q) {
+      if (q == bb) {
+        at = fill[q];
+        fill[q] += Lr;
+      }
+    }
+    const uint32_t rw = Lr > 1u ? 16u << (32 - __clz(Lr - 1u)) : 16u;
+    if (lane == src) {
+      bin = bb;
+      base = at;
+      my_roff = roff;
+      my_rw = rw;
+    }
     roff += rw;
   }
-  uint32_t k = 0;
-  for (uint32_t w = 0; w < 8; ++w) {
-    first[w] = k;
-    for (uint32_t i = 0; i < ng; ++i)
-      if (bin[i] == w) pk[k++] = gl[i];
+  uint32_t f[9];  // first entry of each warp
+#pragma unroll
+  for (uint32_t w = 0; w < 9; ++w) f[w] = __popc(__ballot_sync(0xffffffffu, item && bin < w));
+  const uint32_t same = __match_any_sync(0xffffffffu, item ? bin : 0xffu);
+  uint32_t fb = 0;
+#pragma unroll
+  for (uint32_t w = 0; w < 8; ++w)
+    if (w == bin) fb = f[w];
+  if (item) {
+    PackEntry e;
+    e.sw = uint16_t(sw);
+    e.gg = uint16_t(gg);
+    e.base = uint16_t(base);
+    e.lanes = uint16_t(L);
+    e.ring_off = uint16_t(my_roff);
+    e.ring_words = uint16_t(my_rw);
+    pk[fb + __popc(same & lanemask_lt())] = e;
   }
-  first[8] = k;
+#pragma unroll
+  for (uint32_t w = 0; w < 9; ++w)
+    if (lane == w) first[w] = f[w];
+  __syncwarp();
 }
 
 struct __align__(16) EntSmem {
@@ -1228,6 +1259,76 @@ __device__ inline uint32_t rans_encode_rows(const uint8_t* row, bool live, const
   }
   *x_out = x;
   return cap - pos;
+}
+
+// A width stream's record (RAW, CONST or RANS; the layout of
+// block_write_stream) written by one warp, so that the streams of a record are
+// written side by side. raw(i) gives symbol i for RAW.
+template <class RawFn>
+__device__ inline void warp_write_stream(uint8_t* rec, uint32_t mode, uint32_t n, uint32_t bytes, uint32_t csym,
+                                         uint32_t k, const uint32_t* freq, const uint32_t* states,
+                                         const uint16_t* words, const uint32_t* wbeg, const uint32_t* W,
+                                         const uint32_t* sub_len, RawFn raw) {
+  const uint32_t lane = threadIdx.x & 31u;
+  if (mode == kModeRaw || mode == kModeConst) {
+    if (lane == 0)
+      *reinterpret_cast<uint4*>(rec) =
+          make_uint4(mode | (mode == kModeConst ? (csym << 8) : 0u), bytes, n, mode == kModeConst ? 1u : 0u);
+    if (mode == kModeRaw) {
+      for (uint32_t q = lane; q < pad16(n) / 16u; q += 32u) {
+        uint32_t w[4] = {0, 0, 0, 0};
+        for (uint32_t b = 0; b < 16; ++b) {
+          const uint32_t i = q * 16u + b;
+          w[b >> 2] |= (i < n ? raw(i) : 0u) << (8 * (b & 3u));
+        }
+        *reinterpret_cast<uint4*>(rec + 16 + q * 16u) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    }
+    __syncwarp();
+    return;
+  }
+  const uint32_t N = rans_lanes(n), G = rans_groups(N);
+  if (lane == 0) *reinterpret_cast<uint4*>(rec) = make_uint4(kModeRans | (G << 16), bytes, n, k);
+#pragma unroll
+  for (uint32_t w = 0; w < 8; ++w) {  // presence bitmap, 32 symbols per word
+    const uint32_t bits = __ballot_sync(0xffffffffu, freq[32 * w + lane] != 0u);
+    if (lane == 0) reinterpret_cast<uint32_t*>(rec + 16)[w] = bits;
+  }
+  uint32_t cnt = 0;  // lane covers symbols 8 lane .. 8 lane + 7
+#pragma unroll
+  for (uint32_t i = 0; i < 8; ++i) cnt += freq[8 * lane + i] != 0u ? 1u : 0u;
+  uint32_t incl = cnt;
+#pragma unroll
+  for (uint32_t o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  uint32_t idx = incl - cnt;
+#pragma unroll
+  for (uint32_t i = 0; i < 8; ++i) {
+    const uint32_t f = freq[8 * lane + i];
+    if (f) st_u16(rec + 48 + 2u * idx++, f);
+  }
+  const uint32_t ftab_end = 48u + 2u * k, lens_at = pad16(ftab_end);
+  if (lane < lens_at - ftab_end) rec[ftab_end + lane] = 0;
+  const uint32_t lens_end = lens_at + 4u * G, sub0 = pad16(lens_end);
+  if (lane < G) reinterpret_cast<uint32_t*>(rec + lens_at)[lane] = sub_len[lane];
+  if (lane < sub0 - lens_end) rec[lens_end + lane] = 0;
+  uint32_t off = sub0;
+  for (uint32_t g = 0; g < G; ++g) {
+    const uint32_t lanes_g = min(kGroupLanes, N - g * kGroupLanes);
+    uint8_t* sub = rec + off;
+    if (lane < lanes_g) reinterpret_cast<uint32_t*>(sub)[lane] = states[g * kGroupLanes + lane];
+    uint16_t* w16 = reinterpret_cast<uint16_t*>(sub + 4u * lanes_g);
+    const uint16_t* src = words + wbeg[g];
+    const uint32_t Wg = W[g];
+#pragma unroll 4
+    for (uint32_t i = lane; i < Wg; i += 32u) w16[i] = src[i];
+    const uint32_t end = off + sub_len[g], padded = off + pad16(sub_len[g]);
+    if (lane < padded - end) rec[end + lane] = 0;
+    off = padded;
+  }
+  __syncwarp();
 }
 
 // The same for the groups packed into one warp: the lanes of a group (mask gm)
@@ -1298,7 +1399,10 @@ k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
   }
 
   const Split split(tcc);
-  // ---- per-stream tables from the counts: warp w takes width b = w + 1
+  // ---- per-stream tables from the counts: warp w takes width b = w + 1. In
+  // a full chunk the record's rANS groups are packed into warps meanwhile, by
+  // a warp with no table to build (warp 0 after its table when every width has
+  // one), from the counts: a stream is rANS coded when it holds two symbols
   {
     const uint32_t bw = warp + 1u, m = S.ci.bcount[bw];
     if (m) {
@@ -1306,18 +1410,24 @@ k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
                                         S.rem + tab_base(bw), S.tab + tab_base(bw));
       if (lane == 0) S.k[warp] = k;
     }
+    uint32_t present = 0;
+    for (uint32_t b = 1; b <= 8; ++b) present |= S.ci.bcount[b] ? 1u << (b - 1) : 0u;
+    const uint32_t pw = present == 0xffu ? 0u : 31u - __clz(~present & 0xffu);
+    if (tcc == kMaxCt && warp == pw) {
+      uint32_t rans = 0;
+      for (uint32_t b = 1; b <= 8; ++b) {
+        if (!S.ci.bcount[b]) continue;
+        uint32_t c = 0;
+        for (uint32_t i = lane; i < (1u << b); i += 32u) c += S.hist[tab_base(b) + i] != 0u ? 1u : 0u;
+        if (__reduce_add_sync(0xffffffffu, c) >= 2u) rans |= 1u << (b - 1);
+      }
+      warp_pack_groups(S.ci, rans, tcc, S.pk, S.pk_first);
+    }
   }
   __syncthreads();
   if (tcc == kMaxCt) {
     // ---- full chunk (lane l of a stream: component l, all 512 tokens): the
     // rANS groups packed into warps
-    if (tid == 0) {
-      uint32_t rans = 0;
-      for (uint32_t bw = 1; bw <= 8; ++bw)
-        if (S.ci.bcount[bw] && S.k[bw - 1] >= 2) rans |= 1u << (bw - 1);
-      pack_groups(S.ci, rans, tcc, S.pk, S.pk_first);
-    }
-    __syncthreads();
     const uint32_t e0 = S.pk_first[warp], e1 = S.pk_first[warp + 1];
     if (e1 > e0) {
       int me = -1;
@@ -1401,20 +1511,21 @@ k_transform_entropy(TransformShape sh, TransformPlanDev pl, FrameBatch b, Encode
     S.off[8] = off;
   }
   __syncthreads();
-  for (uint32_t bw = 1; bw <= 8; ++bw) {
-    const uint32_t m = S.ci.bcount[bw];
-    if (!m) continue;
-    const uint32_t n = m * tcc, base = S.ci.bstart[bw];
-    auto sym = [&](uint32_t i) -> uint32_t {
-      uint32_t a, t;
-      split(i, a, t);
-      return uint32_t(codes_g[uint64_t(S.ci.comp[base + a]) * kCodesRow + t]);
-    };
-    block_write_stream(rec + S.off[bw - 1], S.mode[bw - 1], n, S.bytes[bw - 1], sym(0), S.k[bw - 1],
-                       S.freq[bw - 1], S.states[bw - 1], scratch, S.wbeg[bw - 1], S.W[bw - 1],
-                       S.sub_len[bw - 1], sym, S.tmp);
-    __syncthreads();
+  {  // warp w writes the stream of width w + 1, all streams side by side
+    const uint32_t bw = warp + 1u, m = S.ci.bcount[bw];
+    if (m) {
+      const uint32_t n = m * tcc, base = S.ci.bstart[bw];
+      auto sym = [&](uint32_t i) -> uint32_t {
+        uint32_t a, t;
+        split(i, a, t);
+        return uint32_t(codes_g[uint64_t(S.ci.comp[base + a]) * kCodesRow + t]);
+      };
+      warp_write_stream(rec + S.off[bw - 1], S.mode[bw - 1], n, S.bytes[bw - 1], sym(0), S.k[bw - 1],
+                        S.freq[bw - 1], S.states[bw - 1], scratch, S.wbeg[bw - 1], S.W[bw - 1], S.sub_len[bw - 1],
+                        sym);
+    }
   }
+  __syncthreads();
   const uint32_t len = S.off[8];
   const uint32_t crc = crc32_block_aligned(rec, len, S.crc_t, S.red);
   if (tid == 0) {
@@ -2046,9 +2157,9 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
         if (bad) S.bad = 1;
       }
     }
-    // rANS streams: warp w builds the table of width w + 1 while one thread
-    // packs the record's groups into warps (pack_groups), each with its own
-    // refill ring; then each warp decodes its groups side by side
+    // rANS streams: warp w builds the table of width w + 1 while another warp
+    // packs the record's groups into warps (warp_pack_groups), each with its
+    // own refill ring; then each warp decodes its groups side by side
     uint32_t rans = 0;  // width streams with rANS groups
     for (uint32_t sw = 1; sw <= 8; ++sw)
       if (S.ci.bcount[sw] && S.si[sw - 1].mode == kModeRans) rans |= 1u << (sw - 1);
@@ -2056,7 +2167,7 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
     // the packing runs in a warp that builds no table (the highest such warp;
     // warp 0 after its table when every width has one)
     const uint32_t pw = rans == 0xffu ? 0u : 31u - __clz(~rans & 0xffu);
-    if (warp == pw && lane == 0) pack_groups(S.ci, rans, tcc, S.pk, S.pk_first);
+    if (warp == pw) warp_pack_groups(S.ci, rans, tcc, S.pk, S.pk_first);
     __syncthreads();
     if (S.pk_first[warp + 1] > S.pk_first[warp]) {
       const PackEntry* pe = S.pk + S.pk_first[warp];
