@@ -59,13 +59,13 @@ TENSOR_RATIO = {"bf16": 1.0, "i8": 2.0}
 # with the frames a launch covers). A kernel changed after its capture has no
 # entry.
 DRAM_BYTES_PER_FRAME = {
-    "lossless_encode": (731.1e6 + 345.8e6) / 4,
-    "transform_project": (331.9e6 + 106.8e6) / 4,
+    "lossless_encode": (717.4e6 + 345.0e6) / 4,
+    "transform_project": (328.1e6 + 106.2e6) / 4,
     "transform_side": (14.0e6 + 0.0e6) / 4,
-    "transform_entropy": (129.7e6 + 24.8e6) / 4,
-    "lossless_decode": (200.6e6 + 217.7e6) / 4,
-    "transform_decode_codes": (86.6e6 + 108.2e6) / 4,
-    "transform_decode": (200.6e6 + 217.0e6) / 4,
+    "transform_entropy": (126.2e6 + 21.8e6) / 4,
+    "lossless_decode": (200.7e6 + 217.5e6) / 4,
+    "transform_decode_codes": (84.5e6 + 105.6e6) / 4,
+    "transform_decode": (200.7e6 + 217.0e6) / 4,
 }
 
 
