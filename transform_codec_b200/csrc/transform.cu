@@ -1112,11 +1112,11 @@ k_transform_side(TransformShape sh, TransformPlanDev pl, FrameBatch b, EncodeLay
 // Transform encode, part 2 (k_transform_entropy): one CTA per middle record,
 // several per SM (no codes in shared memory). Warp w owns the stream of width
 // b = w + 1: it normalises the stream's counts and builds its coding tables.
-// The rANS groups of all streams then run side by side, one warp per (stream,
-// group), reading the codes from the slot: in a full chunk every lane is one
-// component, whose 512 codes are one row, read 16 at a time into registers;
-// otherwise symbol by symbol. The record is then laid out and written stream
-// by stream.
+// The rANS groups of all streams then run side by side, reading the codes from
+// the slot: in a full chunk every lane is one component, whose 512 codes are
+// one row, read 16 at a time into registers, and the groups are packed into
+// warps (warp_pack_groups); otherwise one warp per (stream, group), symbol by
+// symbol. The record is then laid out and its streams written one warp each.
 
 // A rANS group of a record's width stream, placed in a warp: lanes base ..
 // base + lanes - 1 of the warp code it (the decoder gives it ring_words refill
@@ -1568,15 +1568,16 @@ k_transform_encode_raw(TransformShape sh, FrameBatch b, EncodeLayout ws) {
 // ---------------------------------------------------------------------------
 // Transform decoder, in two stages.
 //
-// Entropy stage (k_transform_decode_codes): one block of 8 warps per record,
-// three blocks per SM. A raw record is copied to its rows. A middle record is
-// checked (CRC, stream walk, stream headers, side information length) and its
-// codes are decoded into the record's code block in the workspace,
+// Entropy stage (k_transform_decode_codes): blocks of 8 warps, four per SM,
+// each taking records in turn. A raw record is copied to its rows. A middle
+// record is checked (CRC, stream walk, stream headers, side information) and
+// its codes are decoded into the record's code block in the workspace,
 // codes[t * 128 + j] for token t of the chunk and component j; the record's
 // status word tells the tensor stage whether to use the block. A width
 // stream's decode table is one byte per slot (its symbol) and f << 16 | cum
 // per symbol: 5 KiB instead of a word per slot, so the tables of all eight
-// streams of a record and the warps' refill rings fit a third of an SM.
+// streams of a record and the refill rings fit a quarter of an SM. The
+// record's rANS groups are packed into warps (warp_pack_groups).
 //
 // Tensor stage (k_transform_decode): dequantisation, the inverse projection
 // on the tensor cores and the RoPE epilogue of every middle record whose
