@@ -1,6 +1,7 @@
 // Host/device interface between the C-ABI layer and the kernels of the KV codec
 // library. GPU-library only.
 #pragma once
+#include <atomic>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -15,6 +16,27 @@ constexpr uint32_t kMaxChunkValues = 65536;  // values per lossless chunk at mos
 // CUDA events before and after it on the launch stream.
 bool prof_enabled();
 void prof_record(const char* name, cudaStream_t st, bool end);
+// A kernel's dynamic shared-memory limit, raised only when a launch needs
+// more than the device already allows it (track: one per launch site, the
+// largest size set on each of the first 8 devices). cudaFuncSetAttribute on
+// every launch made concurrent calls from other host threads serialise.
+struct SmemAttr {
+  std::atomic<int> set[8];
+};
+inline cudaError_t smem_attr(SmemAttr& track, const void* kern, size_t bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+  const int need = int(bytes);
+  if (dev >= 0 && dev < 8 && track.set[dev].load(std::memory_order_relaxed) >= need) return cudaSuccess;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, need);
+  if (e == cudaSuccess && dev >= 0 && dev < 8) {
+    int cur = track.set[dev].load(std::memory_order_relaxed);
+    while (cur < need && !track.set[dev].compare_exchange_weak(cur, need, std::memory_order_relaxed)) {
+    }
+  }
+  return e;
+}
+
 struct ProfRange {
   const char* name;
   cudaStream_t st;

@@ -1354,8 +1354,8 @@ cudaError_t launch_lossless_encode(const LosslessShape& s, const FrameBatch& b,
   if (nrec == 0) return cudaSuccess;
   if (s.E == 4u) {  // f32: the plane-at-a-time encoder for every chunk
     const size_t smem = sizeof(WideEncSmem) + pad16(s.tc * s.D);
-    cudaError_t e = cudaFuncSetAttribute(k_lossless_encode_wide<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(smem));
+    static SmemAttr attr;
+    cudaError_t e = smem_attr(attr, reinterpret_cast<const void*>(k_lossless_encode_wide<4>), smem);
     if (e != cudaSuccess) return e;
     ProfRange pr_("lossless_encode_wide", st);
     k_lossless_encode_wide<4><<<nrec, kEncThreads, smem, st>>>(s, b, ws);
@@ -1371,7 +1371,8 @@ cudaError_t launch_lossless_encode(const LosslessShape& s, const FrameBatch& b,
   if (fast) {
     const size_t fsmem = sizeof(FencSmem);
     auto kern = s.D == 128u ? k_lossless_encode_fast<128> : k_lossless_encode_fast<64>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(fsmem));
+    static SmemAttr attr128, attr64;
+    e = smem_attr(s.D == 128u ? attr128 : attr64, reinterpret_cast<const void*>(kern), fsmem);
     if (e != cudaSuccess) return e;
     {
       ProfRange pr_("lossless_encode", st);
@@ -1383,7 +1384,8 @@ cudaError_t launch_lossless_encode(const LosslessShape& s, const FrameBatch& b,
   // the general encoder: every record, or (after the fast one) the ragged last
   // chunks and the chunks it deferred
   size_t smem = sizeof(EncSmem) + pad16(s.tc * s.D * 2u);
-  e = cudaFuncSetAttribute(k_lossless_encode, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  static SmemAttr attr_gen;
+  e = smem_attr(attr_gen, reinterpret_cast<const void*>(k_lossless_encode), smem);
   if (e != cudaSuccess) return e;
   {
     ProfRange pr_(fast ? "lossless_encode_tail" : "lossless_encode", st);
@@ -1397,8 +1399,8 @@ cudaError_t launch_lossless_decode(const LosslessShape& s, const FrameBatch& b, 
   if (max_records == 0 || b.n == 0) return cudaSuccess;
   if (s.E == 4u) {  // f32: the plane-at-a-time decoder for every record
     const size_t smem = sizeof(WideDecSmem) + pad16(s.tc * s.D);
-    cudaError_t e = cudaFuncSetAttribute(k_lossless_decode_wide<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         int(smem));
+    static SmemAttr attr;
+    cudaError_t e = smem_attr(attr, reinterpret_cast<const void*>(k_lossless_decode_wide<4>), smem);
     if (e != cudaSuccess) return e;
     ProfRange pr_("lossless_decode_wide", st);
     const uint32_t grid = min(max_records, uint32_t(num_sms() * 2));
@@ -1407,8 +1409,8 @@ cudaError_t launch_lossless_decode(const LosslessShape& s, const FrameBatch& b, 
   }
   static int fast_blocks_per_sm = 0;
   const size_t fsmem = sizeof(FastSmem);
-  cudaError_t e = cudaFuncSetAttribute(k_lossless_decode_fast,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, int(fsmem));
+  static SmemAttr attr_fast;
+  cudaError_t e = smem_attr(attr_fast, reinterpret_cast<const void*>(k_lossless_decode_fast), fsmem);
   if (e != cudaSuccess) return e;
   if (!fast_blocks_per_sm) {
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&fast_blocks_per_sm, k_lossless_decode_fast,
@@ -1423,7 +1425,8 @@ cudaError_t launch_lossless_decode(const LosslessShape& s, const FrameBatch& b, 
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t smem = sizeof(DecSmem) + 2u * pad16(s.tc * s.D);
-  e = cudaFuncSetAttribute(k_lossless_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  static SmemAttr attr_gen;
+  e = smem_attr(attr_gen, reinterpret_cast<const void*>(k_lossless_decode), smem);
   if (e != cudaSuccess) return e;
   {
     ProfRange pr_("lossless_decode_general", st);

@@ -2484,12 +2484,12 @@ cudaError_t launch_transform_encode(const TransformShape& s, const TransformPlan
   if (e != cudaSuccess || s.n_mid == 0) return e;
   const uint32_t grid = n_slices * s.n_mid;
   const size_t psmem = sizeof(PtSmem) + 1024;
-  e = cudaFuncSetAttribute(k_transform_project, cudaFuncAttributeMaxDynamicSharedMemorySize, int(psmem));
+  static SmemAttr attr_p, attr_e, attr_s;
+  e = smem_attr(attr_p, reinterpret_cast<const void*>(k_transform_project), psmem);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_transform_entropy, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           int(sizeof(EntSmem)));
+  e = smem_attr(attr_e, reinterpret_cast<const void*>(k_transform_entropy), sizeof(EntSmem));
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(k_transform_side, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sizeof(SideSmem)));
+  e = smem_attr(attr_s, reinterpret_cast<const void*>(k_transform_side), sizeof(SideSmem));
   if (e != cudaSuccess) return e;
   {
     ProfRange pr_("transform_project", st);
@@ -2516,8 +2516,8 @@ cudaError_t launch_transform_decode(const TransformShape& s, const TransformPlan
   if (max_records == 0 || b.n == 0) return cudaSuccess;
   static int ent_blocks_per_sm = 0;
   const size_t esmem = sizeof(DecEntSmem);
-  cudaError_t e = cudaFuncSetAttribute(k_transform_decode_codes, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       int(esmem));
+  static SmemAttr attr_c, attr_t;
+  cudaError_t e = smem_attr(attr_c, reinterpret_cast<const void*>(k_transform_decode_codes), esmem);
   if (e != cudaSuccess) return e;
   if (!ent_blocks_per_sm) {
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ent_blocks_per_sm, k_transform_decode_codes, kThreads, esmem);
@@ -2531,7 +2531,7 @@ cudaError_t launch_transform_decode(const TransformShape& s, const TransformPlan
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   size_t smem = sizeof(DecSmem) + 1024;
-  e = cudaFuncSetAttribute(k_transform_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  e = smem_attr(attr_t, reinterpret_cast<const void*>(k_transform_decode), smem);
   if (e != cudaSuccess) return e;
   {
     ProfRange pr_("transform_decode", st);
