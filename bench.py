@@ -64,7 +64,6 @@ DRAM_BYTES_PER_FRAME = {
     "transform_side": (14.0e6 + 0.0e6) / 4,
     "transform_entropy": (126.2e6 + 21.8e6) / 4,
     "lossless_decode": (200.7e6 + 217.5e6) / 4,
-    "transform_decode_codes": (84.5e6 + 105.6e6) / 4,
     "transform_decode": (200.7e6 + 217.0e6) / 4,
 }
 

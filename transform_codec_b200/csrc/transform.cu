@@ -1614,12 +1614,11 @@ struct __align__(16) DecEntSmem {
   uint32_t base[kBatchMax + 1];
   uint32_t crc_ok, bad, walk_ok, side_ok;
   uint32_t side_off[5];                // the side stream records' offsets in the record
+  StreamInfo side_si[4];               // the side streams (their f << 16 | cum tables overlay crc_t)
   PackEntry pk[kMaxGroupsRec];         // the record's rANS groups, by warp (first pk_first[w])
   uint32_t pk_first[9];
 };
-// byte plane q of the side values V (kSideMax bytes each), in table slots 4-5
-__device__ inline uint8_t* side_plane(DecEntSmem& S, uint32_t q) { return &S.lut[4][0] + q * kSideMax; }
-static_assert(4u * kSideMax <= 2u * kProbScale, "the side planes fit two table slots");
+static_assert(sizeof(DecEntSmem{}.crc_t) == 4u * 256u * sizeof(uint32_t), "four side tables overlay the CRC table");
 
 // Decode table of one rANS stream built by one warp: freq[256] (validated, sum
 // 4096) becomes freq[s] = f_s << 16 | cum_s, and lut[slot] the symbol whose
@@ -1940,12 +1939,16 @@ __device__ inline int warp_parse_stream(const uint8_t* rec, uint32_t avail, uint
 }
 
 // rANS decode of a side stream's single group by one warp (lanes l < N <= 32,
-// the side lane rule) from the sub-stream copied to shared memory (sl bytes at
-// sub, 4-byte aligned): byte table lut, f << 16 | cum per symbol in fc; dm =
-// 0xff undoes lane deltas. Returns false (on every lane) when a lane reads
-// past the words or the final states and word count do not match.
-__device__ inline bool side_decode_group(const uint8_t* sub, uint32_t sl, uint32_t n, const uint8_t* lut,
-                                         const uint32_t* fc, uint32_t dm, uint8_t* out) {
+// the side lane rule) straight from the record (sl bytes at sub, 4-byte
+// aligned), with no per-slot table: the symbol of a slot is the largest s with
+// cum_s <= slot in fc[256] = f << 16 | cum (absent symbols carry the next
+// present symbol's cum, so the search lands on the present one), found in
+// eight steps. dm = 0xff undoes lane deltas; out(i, byte) takes value i's byte.
+// Returns false (on every lane) when a lane reads past the words or the final
+// states and word count do not match.
+template <class Out>
+__device__ inline bool side_decode_search(const uint8_t* sub, uint32_t sl, uint32_t n, const uint32_t* fc,
+                                          uint32_t dm, Out out) {
   const uint32_t lane = threadIdx.x & 31u, N = side_lanes(n);
   if (sl < 4u * N || ((sl - 4u * N) & 1u)) return false;
   const uint32_t W = (sl - 4u * N) >> 1;
@@ -1954,28 +1957,58 @@ __device__ inline bool side_decode_group(const uint8_t* sub, uint32_t sl, uint32
   if (live) lane_range(n, N, lane, start, len);
   lane_range(n, N, 0u, start0, maxlen);
   const uint16_t* words = reinterpret_cast<const uint16_t*>(sub + 4u * N);
-  uint32_t x = live ? reinterpret_cast<const uint32_t*>(sub)[lane] : kRansLow;
+  uint32_t x = live ? __ldg(reinterpret_cast<const uint32_t*>(sub) + lane) : kRansLow;
   uint32_t pos = 0, prev = 0, over = 0;
   const uint32_t lt = lanemask_lt();
   for (uint32_t tau = 0; tau < maxlen; ++tau) {
     const bool act = live && tau < len;
     if (act) {
-      const uint32_t slot = x & (kProbScale - 1u), sym = lut[slot], e = fc[sym];
+      const uint32_t slot = x & (kProbScale - 1u);
+      uint32_t sym = 0;
+#pragma unroll
+      for (uint32_t step = 128u; step; step >>= 1)
+        if ((fc[sym + step] & 0xffffu) <= slot) sym += step;
+      const uint32_t e = fc[sym];
       x = (e >> 16) * (x >> kProbBits) + slot - (e & 0xffffu);
       prev = sym ^ (prev & dm);
-      out[start + tau] = uint8_t(prev);
+      out(start + tau, prev);
     }
     const bool need = act && x < kRansLow;
     const uint32_t mask = __ballot_sync(0xffffffffu, need);
     const uint32_t idx = pos + __popc(mask & lt);
     if (need) {
       over |= idx >= W ? 1u : 0u;
-      x = (x << 16) | words[idx < W ? idx : 0u];
+      x = (x << 16) | (idx < W ? uint32_t(__ldg(words + idx)) : 0u);  // never past the sub-stream
     }
     pos += __popc(mask);
   }
   const bool ok = !over && pos == W && (!live || x == kRansLow);
   return __all_sync(0xffffffffu, ok);
+}
+
+// A stream's frequencies freq[256] (validated, sum 4096) become f << 16 | cum
+// in place, by one warp.
+__device__ inline void warp_fc_table(uint32_t* freq) {
+  const uint32_t lane = threadIdx.x & 31u;
+  uint32_t f[8], mine = 0;
+#pragma unroll
+  for (uint32_t i = 0; i < 8; ++i) {
+    f[i] = freq[8u * lane + i];
+    mine += f[i];
+  }
+  uint32_t incl = mine;
+#pragma unroll
+  for (uint32_t o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  uint32_t cum = incl - mine;
+#pragma unroll
+  for (uint32_t i = 0; i < 8; ++i) {
+    freq[8u * lane + i] = (f[i] << 16) | cum;
+    cum += f[i];
+  }
+  __syncwarp();
 }
 
 static_assert(sizeof(DecEntSmem) + 1024 <= 233472 / 4, "entropy stage should fit four blocks per SM");
@@ -2016,6 +2049,7 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
     const uint8_t* rec = src + off0;
     const uint32_t ls = r / rps, kind = r % rps;
     const uint32_t sidx = ds->first_slice + ls;
+    if (g != blockIdx.x) crc_tables_init(S.crc_t);  // the previous record's side tables overlaid it
     uint32_t got = crc32_block_aligned<true>(rec, len, S.crc_t, S.red);
     if (tid == 0) S.crc_ok = (got == want);
     __syncthreads();
@@ -2043,11 +2077,10 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
     // Stream headers. One thread walks the side streams' headers (side
     // information: four byte-plane streams of V = every z, then every s) and
     // then the width streams' for their offsets. Warp q < 4 then checks side
-    // stream q, loads its table (into width-stream table slot q, rebuilt only
-    // later), copies its sub-stream to the rings of warps 2q and 2q + 1 (idle
-    // until the width streams) and decodes plane q from there, while warps 4-7
-    // check the headers and frequencies of width streams 5-8; warps 0-3 then
-    // check width streams 1-4 while the block assembles the (z, s) pairs.
+    // stream q and turns its frequencies into a f << 16 | cum table over the
+    // CRC table (rebuilt for the next record), while warps 4-7 check width
+    // streams 5-8; warps 0-3 then check width streams 1-4. The side streams are
+    // decoded later, beside the width streams, by warps without a rANS group.
     const bool kiv = sh.kivi && ((sidx / sh.H) & 1u) == 1u;  // values with per-token ranges
     const uint32_t half = S.ci.n_coded ? (kiv ? tcc : S.ci.n_coded * nb) : 0u, nv = 2u * half;
     if (tid == 0) {
@@ -2077,27 +2110,9 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
       bool okw = true;
       if (warp < 4 && nv) {
         const uint32_t q = warp, o = S.side_off[q];
-        StreamInfo& si = S.si[q];
-        okw = warp_parse_side(rec + o, S.side_off[q + 1] - o, nv, side_lanes(nv), si, S.freq[q]) == kOk;
-        if (okw) {
-          // the sub-stream is staged in the rings of warps 2q and 2q + 1: it
-          // starts past the header and table (at least 80 bytes) of a record of at
-          // most 16 + pad16(kSideMax) bytes, so it fits their 2 KiB
-          uint8_t* stage = reinterpret_cast<uint8_t*>(&S.ring[2u * q][0]);
-          uint8_t* plane = side_plane(S, q);
-          if (si.mode == kModeRaw) {
-            for (uint32_t i = lane; i < nv; i += 32u) plane[i] = __ldg(rec + o + 16u + i);
-          } else if (si.mode == kModeConst) {
-            for (uint32_t i = lane; i < nv; i += 32u) plane[i] = uint8_t(si.sym);
-          } else {
-            const uint4* sub4 = reinterpret_cast<const uint4*>(rec + o + si.sub_off[0]);
-            for (uint32_t i = lane; i < pad16(si.sub_len[0]) / 16u; i += 32u)
-              reinterpret_cast<uint4*>(stage)[i] = __ldg(sub4 + i);
-            warp_dec_lut8(S.freq[q], S.lut[q]);
-            __syncwarp();
-            okw = side_decode_group(stage, si.sub_len[0], nv, S.lut[q], S.freq[q], si.delta ? 0xffu : 0u, plane);
-          }
-        }
+        uint32_t* fcq = S.crc_t + 256u * q;
+        okw = warp_parse_side(rec + o, S.side_off[q + 1] - o, nv, side_lanes(nv), S.side_si[q], fcq) == kOk;
+        if (okw && S.side_si[q].mode == kModeRans) warp_fc_table(fcq);
       } else if (warp >= 4 && S.ci.bcount[warp + 1]) {
         const uint32_t o = S.str_off[warp];
         okw = warp_parse_stream(rec + o, len - o, S.ci.bcount[warp + 1] * tcc, S.si[warp], S.freq[warp]) == kOk;
@@ -2109,23 +2124,6 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
       if (warp < 4 && S.ci.bcount[warp + 1]) {
         const uint32_t o = S.str_off[warp];
         okw = warp_parse_stream(rec + o, len - o, S.ci.bcount[warp + 1] * tcc, S.si[warp], S.freq[warp]) == kOk;
-      }
-      if (nv) {
-        float2* zs = cb.zs + uint64_t(g) * kD * (sh.ct / kTile);
-        for (uint32_t i = tid; i < half; i += nthr) {
-          uint32_t z = 0, sc = 0;
-#pragma unroll
-          for (uint32_t q = 0; q < 4; ++q) {
-            z |= uint32_t(side_plane(S, q)[i]) << (8u * q);
-            sc |= uint32_t(side_plane(S, q)[half + i]) << (8u * q);
-          }
-          if (kiv) {  // (z, range) of token i
-            zs[i] = make_float2(__uint_as_float(z), __uint_as_float(sc));
-          } else {
-            const uint32_t cc = i / nb, blk = i - cc * nb;
-            zs[cc * (sh.ct / kTile) + blk] = make_float2(__uint_as_float(z), __uint_as_float(sc));
-          }
-        }
       }
       if (!__syncthreads_and(okw)) st = kErrCorrupt;
     }
@@ -2175,6 +2173,31 @@ k_transform_decode_codes(TransformShape sh, TransformPlanDev pl, FrameBatch b, u
       const uint32_t ne = S.pk_first[warp + 1] - S.pk_first[warp];
       const bool ok = tcc == kMaxCt ? decode_codes_packed<true>(S, pe, ne, rec, codes, tcc)
                                     : decode_codes_packed<false>(S, pe, ne, rec, codes, tcc);
+      if (!ok && lane == 0) S.bad = 1;
+    }
+    if (nv && warp >= 4) {
+      // side stream q = 7 - warp (warps that hold no rANS group unless a record
+      // fills more than four): byte q of each value of V goes straight into the
+      // record's (z, s) pairs; value i < half is a zero point, the rest scales
+      // (ranges), in the order of V
+      const uint32_t q = 7u - warp, o = S.side_off[q];
+      const StreamInfo& si = S.side_si[q];
+      uint8_t* zb = reinterpret_cast<uint8_t*>(cb.zs + uint64_t(g) * kD * (sh.ct / kTile));
+      const uint32_t bstride = sh.ct / kTile;
+      auto out = [&](uint32_t i, uint32_t v) {
+        const uint32_t hi = i >= half ? 1u : 0u, j = i - hi * half;
+        const uint32_t pair = kiv ? j : (j / nb) * bstride + (j % nb);
+        zb[8u * pair + 4u * hi + q] = uint8_t(v);
+      };
+      bool ok = true;
+      if (si.mode == kModeRaw) {
+        for (uint32_t i = lane; i < nv; i += 32u) out(i, __ldg(rec + o + 16u + i));
+      } else if (si.mode == kModeConst) {
+        for (uint32_t i = lane; i < nv; i += 32u) out(i, si.sym);
+      } else {
+        ok = side_decode_search(rec + o + si.sub_off[0], si.sub_len[0], nv, S.crc_t + 256u * q,
+                                si.delta ? 0xffu : 0u, out);
+      }
       if (!ok && lane == 0) S.bad = 1;
     }
     __syncthreads();
