@@ -1601,11 +1601,9 @@ __device__ inline CodeBlocks code_blocks(uint8_t* ws, uint32_t max_records, uint
 constexpr uint32_t kRingWords = 512;              // refill ring of one warp
 
 struct __align__(16) DecEntSmem {
-  // per width stream: symbol of each slot. While the side streams are decoded,
-  // slots 0-3 hold their tables and slots 4-5 the four decoded byte planes.
-  uint8_t lut[8][kProbScale];
-  alignas(16) uint16_t ring[kThreads / 32][kRingWords];  // one refill window per warp (cp.async targets)
-  uint32_t crc_t[1024];
+  uint8_t lut[8][kProbScale];  // per width stream: symbol of each slot
+  alignas(16) uint16_t ring[kThreads / 32][kRingWords];  // refill rings of the packed rANS groups (cp.async targets)
+  uint32_t crc_t[1024];        // CRC tables; after the record's CRC, the side streams' f << 16 | cum tables
   uint32_t freq[8][256];               // per width stream; f << 16 | cum after the table build
   uint32_t tmp[32], red[32];
   StreamInfo si[8];
