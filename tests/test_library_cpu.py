@@ -176,3 +176,21 @@ def test_stream_host_argument_checks():
         with pytest.raises(kvc.KvcError) as e:
             call()
         assert e.value.status == want
+
+
+def test_plan_held_until_interpreter_exit_is_released_quietly():
+    # A plan still referenced by a module global is collected after the
+    # binding's own globals are cleared; its destructor must not need them.
+    import subprocess
+    import sys
+    # Importing torch first is what puts the binding's module teardown ahead
+    # of the plan's collection.
+    code = ("import torch\n"
+            "import transform_codec_b200 as kvc\n"
+            "p = kvc.Plan(kvc.Shape(kvc.BF16, 2, 2, 1024, 128))\n"
+            "print(p.max_encoded_bytes(kvc.LOSSLESS, 4))\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True,
+                       text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert int(r.stdout.split()[-1]) > 0
+    assert "Exception ignored" not in r.stderr, r.stderr

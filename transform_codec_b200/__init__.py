@@ -193,12 +193,16 @@ class Plan:
         h = ctypes.c_void_p()
         _check(_lib.kvc_plan(ctypes.byref(desc), ctypes.byref(h)), "kvc_plan")
         self._h = h
+        # Held by the object: at interpreter exit the module's globals may be
+        # cleared before the last plan is collected.
+        self._destroy = _lib.kvc_plan_destroy
         self.has_transform = b is not None
 
     def __del__(self):
         h = getattr(self, "_h", None)
-        if h is not None and h.value:
-            _lib.kvc_plan_destroy(h)
+        destroy = getattr(self, "_destroy", None)
+        if h is not None and h.value and destroy is not None:
+            destroy(h)
             self._h = None
 
     @property
