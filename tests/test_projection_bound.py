@@ -19,6 +19,14 @@ scaled, adversarial and PCA-of-cache inputs, for R per 64-token block and
 column (block ranges) and per token over its coded columns (per-token ranges,
 Codec-Gauge "Compression Conditions"), and that every level stays inside the
 range its fp32 conversion is exact in.
+
+The second half checks the rule by which a code is taken from the estimate
+without the chain: with qa = RN(RN(y~ - z) RN(1/s)), a code is settled when the
+distance from qa to the nearest half-integer exceeds RU(R RN(1/s) (1 + 2^-19))
++ |qa| 2^-19. The oracle's quantiser (q = rint(RN(RN(y - z) / s)), clamped to
+[0, 2^b - 1]) is monotone in y, so a settled code is right for every fp32 y in
+[y~ - R, y~ + R] exactly when the oracle's codes at the two ends of that set
+equal rint(qa); that is checked on quotients placed next to half-integers.
 """
 import dataclasses
 import math
@@ -271,3 +279,108 @@ def test_a_planted_mistake_in_the_bound_is_caught():
             _check_block_ranges(Q, x)
     finally:
         DROP_UNITS = saved
+
+
+# ------------------------------------------------------------ settling codes
+F32 = np.float32
+MAGIC = F32(12582912.0)  # 1.5 * 2^23: adding it rounds |q| < 2^22 to an integer
+
+
+def _round_dir(a: np.ndarray, b: np.ndarray, up: bool) -> np.ndarray:
+    """a + b (fp32 arrays) rounded to fp32 toward +inf (up) or -inf, from the
+    exact sum as an unevaluated pair of fp64 numbers (two-sum)."""
+    a64, b64 = a.astype(np.float64), b.astype(np.float64)
+    s = a64 + b64
+    bb = s - a64
+    err = (a64 - (s - bb)) + (b64 - bb)
+    r = s.astype(np.float32)
+    r64 = r.astype(np.float64)
+    if up:
+        low = (r64 < s) | ((r64 == s) & (err > 0))
+        return np.where(low, np.nextafter(r, F32(np.inf)), r)
+    high = (r64 > s) | ((r64 == s) & (err < 0))
+    return np.where(high, np.nextafter(r, F32(-np.inf)), r)
+
+
+def _mul_up(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """a b (fp32) rounded toward +inf: the fp64 product of two fp32 numbers is exact."""
+    p = a.astype(np.float64) * b.astype(np.float64)
+    r = p.astype(np.float32)
+    return np.where(r.astype(np.float64) < p, np.nextafter(r, F32(np.inf)), r)
+
+
+def _oracle_code(y, z, s, levels):
+    """The block-uniform quantiser of the oracle (Codec-Gauge, "Compression
+    Conditions"): rint(RN(RN(y - z) / s)) clamped to [0, levels]."""
+    q = np.rint((y - z) / s)
+    return np.clip(q, 0, levels).astype(np.int64)
+
+
+def _settle(v, z, s, R, exact, interval=True, quotient=True):
+    """The encoder's decision from the estimate v: (settled, code). The two
+    flags leave out the margin's interval term or its quotient term."""
+    rs = F32(1.0) / s
+    qa = (v - z) * rs
+    mg = qa + MAGIC
+    iq = mg.view(np.int32).astype(np.int64) - 0x4B400000
+    d = F32(0.5) - np.abs(qa - (mg - MAGIC))
+    mR = _mul_up(_mul_up(R, rs), np.full_like(R, F32(1.0 + 2.0 ** -19)))
+    mR = mR if interval else np.zeros_like(R)
+    mq = _mul_up(np.abs(qa), np.full_like(qa, F32(2.0 ** -19)))
+    mq = mq if quotient else np.zeros_like(qa)
+    m = _round_dir(np.where(exact, F32(0.0), mR), mq, up=True)
+    return d > m, iq
+
+
+def _settling_cases(rng, n):
+    """Block ranges of random widths and offsets, quotients next to
+    half-integers (offsets from 2^-30 to 1/2 of a code on either side, below
+    0 and above the top code too), error bounds from 10^-9 to 10^-1 of a
+    code, and exact estimates (R = 0)."""
+    bits = rng.integers(1, 9, n)
+    levels = (1 << bits) - 1
+    z = (rng.standard_normal(n) * 10.0 ** rng.uniform(-4, 3, n)).astype(np.float32)
+    span = (10.0 ** rng.uniform(-4, 3, n)).astype(np.float32)
+    zx = (z + span).astype(np.float32)
+    s = ((zx - z) / levels.astype(np.float32)).astype(np.float32)
+    k = rng.integers(-1, levels + 1)
+    off = np.where(rng.random(n) < 0.5, -1.0, 1.0) * 2.0 ** rng.uniform(-30, -1, n)
+    v = (z.astype(np.float64) + (k + 0.5 + off) * s.astype(np.float64)).astype(np.float32)
+    R = (s.astype(np.float64) * 10.0 ** rng.uniform(-9, -1, n)).astype(np.float32)
+    exact = rng.random(n) < 0.2
+    R = np.where(exact, F32(0.0), R)
+    ok = (s > 0) & (F32(1.0) / s < F32(2.0 ** 126))
+    return v[ok], z[ok], s[ok], R[ok], exact[ok], levels[ok]
+
+
+def _settling_errors(v, z, s, R, exact, levels, **kw):
+    settled, iq = _settle(v, z, s, R, exact, **kw)
+    lo = _round_dir(v, -R, up=True)   # the fp32 numbers in [v - R, v + R] run
+    hi = _round_dir(v, R, up=False)   # from RU(v - R) to RD(v + R)
+    want = np.clip(iq, 0, levels)
+    bad = settled & ((_oracle_code(lo, z, s, levels) != want) | (_oracle_code(hi, z, s, levels) != want))
+    return settled, bad
+
+
+def test_settled_codes_equal_the_oracles_on_the_whole_interval():
+    rng = np.random.default_rng(21)
+    v, z, s, R, exact, levels = _settling_cases(rng, 400_000)
+    settled, bad = _settling_errors(v, z, s, R, exact, levels)
+    assert not bad.any(), np.flatnonzero(bad)[:5]
+    # both outcomes occur, and settled codes close to their margin are among them
+    assert 0.2 < settled.mean() < 0.95
+    rs = F32(1.0) / s
+    qa = (v - z) * rs
+    d = F32(0.5) - np.abs(qa - np.rint(qa))
+    assert np.count_nonzero(settled & (d < 2 * (R * rs + np.abs(qa) * 2.0 ** -19))) > 1000
+
+
+@pytest.mark.parametrize("interval,quotient", [(False, True), (True, False)])
+def test_settling_without_a_margin_term_is_caught(interval, quotient):
+    """Without the estimate's interval term (R / s), or without the term for
+    the quotient's own rounding (|qa| 2^-19), some settled codes differ from
+    the oracle's: the check sees either term go missing."""
+    rng = np.random.default_rng(21)
+    cases = _settling_cases(rng, 400_000)
+    _, bad = _settling_errors(*cases, interval=interval, quotient=quotient)
+    assert bad.any()
