@@ -44,6 +44,7 @@ BLOCK = 64
 # plus 96 units for rounding x and Q to integers
 DROP_UNITS = 128 * 255 ** 2 * (3 * 2 ** 16 + 2 * 2 ** 8 + 1) + 96
 SLACK = 1.0 + 2.0 ** -40
+F32 = np.float32
 
 
 def _ilogb(a):
@@ -135,11 +136,38 @@ def _r(e, f, x1, q1, Ma):
     return float(_f32_up((E + dl + math.ldexp(1.0, max(lm - 23, -149))) * SLACK))
 
 
+def _scan_bits(vals: np.ndarray):
+    """The oracle's sequential scan for the smallest and largest value (a
+    later value replaces the current one only when strictly beyond it), as
+    fp32 bit patterns, so that -0 and +0 are told apart."""
+    lo, hi = F32(np.inf), F32(-np.inf)
+    for v in vals.astype(np.float32):
+        if v < lo:
+            lo = v
+        if v > hi:
+            hi = v
+    return int(np.float32(lo).view(np.uint32)), int(np.float32(hi).view(np.uint32))
+
+
+def _extremes_agree(y_f32, v_f32, exact, R, reach=2.0):
+    """Candidates: estimates within reach R (2R in the encoder) of the
+    smallest or largest estimate (thresholds rounded outward in fp32). The scan
+    over exact values for candidates and exact entries, estimates elsewhere,
+    must give the oracle's smallest and largest value bit for bit."""
+    mn, mx = F32(v_f32.min()), F32(v_f32.max())
+    two = F32(reach) * F32(R)
+    lo_thr = _round_dir(np.array([mn]), np.array([two]), up=True)[0]
+    hi_thr = _round_dir(np.array([mx]), np.array([-two]), up=False)[0]
+    cand = (v_f32 <= lo_thr) | (v_f32 >= hi_thr)
+    used = np.where(cand | exact, y_f32, v_f32)
+    return _scan_bits(used) == _scan_bits(y_f32), int(cand.sum())
+
+
 def _oracle_y(Q, x):
     return np.stack([oracle.project(Q, x[t]) for t in range(x.shape[0])])
 
 
-def _check_block_ranges(Q, x):
+def _check_block_ranges(Q, x, reach=2.0):
     """Block ranges: R per 64-token block and column, from the block's largest
     token exponent and 1-norm bound. Returns the largest |y - y~| / R."""
     y = _oracle_y(Q, x).astype(np.float64)
@@ -162,6 +190,9 @@ def _check_block_ranges(Q, x):
             err = np.abs(yb - vb).max()
             assert err <= R, (b0, j, err, R)
             worst = max(worst, err / R)
+            agree, _ = _extremes_agree(y[b0:b0 + BLOCK, j].astype(np.float32), yv[b0:b0 + BLOCK, j],
+                                       zt[b0:b0 + BLOCK], R, reach)
+            assert agree, (b0, j)
     return worst
 
 
@@ -183,6 +214,8 @@ def _check_token_ranges(Q, x, coded):
         err = np.abs(y[t, live_cols] - yv[t, live_cols].astype(np.float64)).max()
         assert err <= R, (t, err, R)
         worst = max(worst, err / R)
+        agree, _ = _extremes_agree(y[t, cols].astype(np.float32), yv[t, cols], zj[cols], R)
+        assert agree, t
     return worst
 
 
@@ -239,6 +272,33 @@ def test_block_ranges_bound_tiny_tokens():
     assert _check_block_ranges(Q, x) <= 1.0
 
 
+def _near_ties(rng):
+    """Two blocks of one token with a few entries moved by one ulp each, and a
+    block of one token repeated: the block extremes lie within R of many
+    other tokens, and the repeated block ties everywhere."""
+    base = (rng.standard_normal(D) * 3).astype(np.float32)
+    x = np.repeat(base[None], 3 * BLOCK, 0)
+    for t in range(2 * BLOCK):
+        idx = rng.integers(0, D, 4)
+        way = np.where(rng.random(4) < 0.5, np.inf, -np.inf).astype(np.float32)
+        x[t, idx] = np.nextafter(x[t, idx], way)
+    x[2 * BLOCK:] = x[2 * BLOCK]
+    return x
+
+
+def test_block_extremes_among_near_ties():
+    rng = np.random.default_rng(31)
+    assert _check_block_ranges(_orthonormal(rng), _near_ties(rng)) <= 1.0
+
+
+def test_extremes_without_candidates_are_caught():
+    """With no reach (only the smallest and largest estimate run the chain),
+    the scan misses true extremes among near ties: the check sees it."""
+    rng = np.random.default_rng(31)
+    with pytest.raises(AssertionError):
+        _check_block_ranges(_orthonormal(rng), _near_ties(rng), reach=0.0)
+
+
 @pytest.mark.parametrize("is_key", [True, False])
 def test_block_and_token_ranges_bound_on_pca_of_the_cache(is_key):
     """The cache workload's own inputs: a slice of the 8k-token cache (keys
@@ -282,7 +342,6 @@ def test_a_planted_mistake_in_the_bound_is_caught():
 
 
 # ------------------------------------------------------------ settling codes
-F32 = np.float32
 MAGIC = F32(12582912.0)  # 1.5 * 2^23: adding it rounds |q| < 2^22 to an integer
 
 
