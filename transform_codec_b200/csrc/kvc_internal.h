@@ -1,7 +1,9 @@
 // Host/device interface between the C-ABI layer and the kernels of the KV codec
 // library. GPU-library only.
 #pragma once
+#include <algorithm>
 #include <atomic>
+#include <mutex>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -17,23 +19,30 @@ constexpr uint32_t kMaxChunkValues = 65536;  // values per lossless chunk at mos
 bool prof_enabled();
 void prof_record(const char* name, cudaStream_t st, bool end);
 // A kernel's dynamic shared-memory limit, raised only when a launch needs
-// more than the device already allows it (track: one per launch site, the
-// largest size set on each of the first 8 devices). cudaFuncSetAttribute on
-// every launch made concurrent calls from other host threads serialise.
+// more than the device already allows it (track: one per kernel, the largest
+// size set on each of the first 64 devices). cudaFuncSetAttribute on every
+// launch made concurrent calls from other host threads serialise. The limit
+// only grows, under one process-wide lock, so first launches of one kernel
+// with different sizes on several threads cannot leave it below a recorded
+// size.
+constexpr int kSmemAttrDevices = 64;
 struct SmemAttr {
-  std::atomic<int> set[8];
+  std::atomic<int> set[kSmemAttrDevices];
 };
+inline std::mutex& smem_attr_lock() {
+  static std::mutex m;
+  return m;
+}
 inline cudaError_t smem_attr(SmemAttr& track, const void* kern, size_t bytes) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
   const int need = int(bytes);
-  if (dev >= 0 && dev < 8 && track.set[dev].load(std::memory_order_relaxed) >= need) return cudaSuccess;
-  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, need);
-  if (e == cudaSuccess && dev >= 0 && dev < 8) {
-    int cur = track.set[dev].load(std::memory_order_relaxed);
-    while (cur < need && !track.set[dev].compare_exchange_weak(cur, need, std::memory_order_relaxed)) {
-    }
-  }
+  const bool tracked = dev >= 0 && dev < kSmemAttrDevices;
+  if (tracked && track.set[dev].load(std::memory_order_acquire) >= need) return cudaSuccess;
+  std::lock_guard<std::mutex> lock(smem_attr_lock());
+  const int target = tracked ? std::max(need, track.set[dev].load(std::memory_order_relaxed)) : need;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, target);
+  if (e == cudaSuccess && tracked) track.set[dev].store(target, std::memory_order_release);
   return e;
 }
 
